@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Benchmark of the HGA segment training step on B200.
+
+One step is one pass of the whole hot path over one segment: the summaries
+of the segment's 2048 new keys (history summaries persist from earlier
+segments), block queries + chunk routing, group routing, the routed
+attention forward and its backward.  The metric is segment tokens per second
+(B * T_seg per step), measured on the device with CUDA events; inputs are
+resident in HBM and L2 is flushed (a 256 MiB write) between timed steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU oracle, same metric
+
+Under torchrun each rank runs its own independent problem (weak scaling;
+the hot path has no exchange step) and rank 0 prints one JSON line with the
+whole-job value: all ranks' tokens over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hierarchical_routed_sparse_b200 import workloads as W  # noqa: E402
+
+METRIC = "HGA routed-attention fwd+bwd tokens/s at 16K ctx; % of roofline (TFLOP/s or HBM GB/s)"
+DEFAULT_WORKLOAD = W.QWEN3_CTX16K_TRAIN.name
+L2_FLUSH_BYTES = 256 << 20
+# Kernels of this library launched per step: summaries, chunk router, group
+# router, attention forward, backward row-dot, attention backward.
+LAUNCHES_PER_STEP = 6
+
+
+def peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        return dict(hbm_gbs=m["hbm_gbs"], bf16_tflops=m["bf16_tflops"],
+                    bf16_tflops_sustained=m["bf16_tflops_sustained"], source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                source="fallback")
+
+
+# ---- algorithmic work (bytes and FLOPs a perfect kernel must move / do) -----
+def routed_groups(w, qb: int) -> int:
+    """Groups routed for query block qb: min(k_g, 8 * min(k_c, eligible))."""
+    c0 = w.T_hist // 64 + qb
+    nc = c0 if w.k_c <= 0 else min(w.k_c, c0)
+    return 8 * nc if w.k_g <= 0 else min(w.k_g, 8 * nc)
+
+
+def algorithmic(w) -> dict:
+    """Per-launch algorithmic bytes and FLOPs of each stage of one step."""
+    el = 2 if w.dtype == "bf16" else 4
+    B, Hq, Hkv, d, Ts, G = w.B, w.Hq, w.Hkv, w.d, w.T_seg, w.G
+    nQB = Ts // 64
+    ng = [routed_groups(w, qb) for qb in range(nQB)]
+    # Keys per (q-head, query): 8*n_g routed + (i+1) own-chunk keys.
+    key_pairs = sum(64 * 8 * n + 64 * 65 // 2 for n in ng)            # per q-head
+    kv_tokens = sum(8 * n + 64 for n in ng)                            # per kv-head
+    wc = w.k_c if w.k_c > 0 else w.T // 64
+    wg = w.k_g if w.k_g > 0 else 8 * wc
+    q_bytes = B * Hq * Ts * d * el
+    kv_gather = B * Hkv * kv_tokens * d * el * 2
+    o_bytes = B * Hq * Ts * d * 4
+    lse_bytes = B * Hq * Ts * 4
+    gidx_bytes = B * Hkv * nQB * wg * 4
+    fwd_bytes = q_bytes + kv_gather + o_bytes + lse_bytes + gidx_bytes
+    bwd_bytes = (q_bytes + kv_gather + q_bytes            # Q, K/V gathered, dO
+                 + o_bytes + lse_bytes + 2 * lse_bytes     # O, LSE, D written + read
+                 + o_bytes                                 # dQ
+                 + 2 * B * Hkv * Ts * d * 4                # dK_seg, dV_seg
+                 + gidx_bytes)
+    seg_keys = B * Hkv * Ts * d * el
+    summ_bytes = seg_keys + B * Hkv * (Ts // 64 + Ts // 8) * d * 4
+    csum_read = B * Hkv * nQB * (w.T_hist // 64 + nQB / 2) * d * 4    # eligible chunks
+    rc_bytes = q_bytes + csum_read + B * Hkv * nQB * (d * 4 + wc * 4)
+    rg_bytes = B * Hkv * nQB * (d * 4 + wc * 4 + 8 * wc * d * 4 + wg * 4)
+    return dict(
+        attn_fwd=dict(bytes=fwd_bytes, flops=4.0 * d * B * Hq * key_pairs),
+        attn_bwd=dict(bytes=bwd_bytes, flops=10.0 * d * B * Hq * key_pairs),
+        summaries=dict(bytes=summ_bytes, flops=0.0),
+        route_chunks=dict(bytes=rc_bytes, flops=0.0),
+        route_groups=dict(bytes=rg_bytes, flops=0.0),
+    )
+
+
+# Source files of each timed kernel: a recorded ncu traffic figure is used
+# only while these files are unchanged since the capture.
+KERNEL_SOURCES = {
+    "attn_fwd": ["attn_simt.cu"],
+    "attn_bwd": ["attn_simt.cu"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "hierarchical_routed_sparse_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, w) -> float | None:
+    """DRAM bytes per launch from profiles/traffic.json, if still current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or rec.get("workload") != w.name or rec.get("source_sha256") != kernel_source_hash(kernel):
+        return None
+    return float(rec["dram_bytes_per_launch"])
+
+
+# ---- clocks sampled during the timed region -----------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, out_path: str | None = None):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out_path = out_path
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            if self.out_path:
+                with open(self.out_path, "w") as f:
+                    f.write("\n".join(self.lines) + "\n")
+
+    def summary(self) -> dict | None:
+        if not getattr(self, "lines", None):
+            return None
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            try:
+                sm.append(float(f[1]))
+                smax = max(smax, float(f[2]))
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * max(sm)]
+        return dict(sm_mhz=statistics.median(loaded), sm_max_mhz=smax, reasons=sorted(reasons),
+                    samples=len(sm))
+
+
+# ---- the CPU oracle, timed on this host ------------------------------------------------------
+def oracle_step_rate(w, min_seconds: float = 10.0, max_reps: int = 50) -> dict:
+    """Time the oracle's segment step (same stages as the GPU step) on the host.
+
+    The sample is the whole workload, repeated until min_seconds of CPU work.
+    """
+    import oracle
+    oracle.build()
+    x = {k: v.astype(np.float64) for k, v in w.full().items()}
+    dims = oracle.Dims(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T_hist=w.T_hist, T_seg=w.T_seg,
+                       k_c=w.k_c, k_g=w.k_g)
+    csum, gsum = oracle.build_summaries(dims, x["K"], 0, w.T_hist)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        c, g = oracle.build_summaries(dims, x["K"], w.T_hist, w.T, csum, gsum)
+        qbar = oracle.block_query(dims, x["Q"])
+        cidx, _ = oracle.route_chunks(dims, qbar, c)
+        gidx, _ = oracle.route_groups(dims, qbar, g, cidx)
+        oracle.attn_fwd(dims, x["Q"], x["K"], x["V"], gidx)
+        if w.backward:
+            oracle.attn_bwd(dims, x["Q"], x["K"], x["V"], x["dO"], gidx)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= max_reps:
+            break
+    return dict(value=reps * w.B * w.T_seg / el, unit="tokens/s", cores=oracle.num_threads(),
+                kind="oracle", seconds=el,
+                sample=f"whole {w.name} step (all {w.B * w.Hkv} (batch, kv-head) units) "
+                       f"x {reps} repetitions, float64, OpenMP",
+                cpu=_cpu_model())
+
+
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ---- main ------------------------------------------------------------------------------------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def config_of(w) -> dict:
+    return dict(workload=w.name, B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T_hist=w.T_hist,
+                T_seg=w.T_seg, T=w.T, k_c=w.k_c, k_g=w.k_g, keys=w.keys,
+                l2="flushed between timed steps (256 MiB write)")
+
+
+def run_reference(args, w) -> None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    cb = oracle_step_rate(w, min_seconds=args.ref_seconds)
+    steps = args.steps
+    line = dict(metric=METRIC, value=cb["value"], unit="tokens/s", n_gpus=args.gpus, steps=steps,
+                warmup=args.warmup, ms_per_step=1e3 * w.B * w.T_seg / cb["value"],
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                data="synthetic", impl="reference", config=config_of(w), cpu_baseline=cb,
+                e2e=dict(value=cb["value"], unit="tokens/s", h2d_bytes_per_step=0,
+                         d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args, w) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import hierarchical_routed_sparse_b200 as hga
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    wr = w.with_(seed=w.seed + rank)                 # independent problem per rank
+    x = wr.full()
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    Q = torch.from_numpy(x["Q"]).to(dev, tdt)
+    K = torch.from_numpy(x["K"]).to(dev, tdt)
+    V = torch.from_numpy(x["V"]).to(dev, tdt)
+    dO = torch.from_numpy(x["dO"]).to(dev, tdt) if w.backward else None
+    p = hga.Params.from_workload(w)
+    buf = hga.Buffers(p, device=dev)
+    buf.summaries(K, 0, w.T_hist)                    # history summaries persist
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    stages = ["summaries", "route", "attn_fwd", "attn_bwd"]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        buf.summaries(K, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        buf.route(Q, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        buf.forward(Q, K, V, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        if dO is not None:
+            buf.backward(Q, K, V, dO, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks_path = os.path.join(ROOT, "gpurun_out", "clocks.csv") if os.path.isdir(
+        os.path.join(ROOT, "gpurun_out")) else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local, clocks_path) as clk:
+        for i in range(args.steps):
+            flush.zero_()                            # outside the timed events
+            step(events[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    per_stage = {s: [] for s in stages}
+    totals = []
+    for ev in events:
+        for j, s in enumerate(stages):
+            per_stage[s].append(ev[j].elapsed_time(ev[j + 1]))
+        totals.append(ev[0].elapsed_time(ev[4]))
+    total_ms = sum(totals)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    tokens = world * args.steps * w.B * w.T_seg
+    value = tokens / (total_ms * 1e-3)
+
+    # ---- end to end through the public API with host buffers ----------------------
+    Qh = torch.from_numpy(x["Q"]).to(tdt).pin_memory()
+    Kh = torch.from_numpy(np.ascontiguousarray(x["K"][:, :, w.T_hist:])).to(tdt).pin_memory()
+    Vh = torch.from_numpy(np.ascontiguousarray(x["V"][:, :, w.T_hist:])).to(tdt).pin_memory()
+    dOh = torch.from_numpy(x["dO"]).to(tdt).pin_memory() if w.backward else None
+    outs_dev = [buf.dQ, buf.dK, buf.dV] if w.backward else [buf.O, buf.lse]
+    outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs_dev]
+    h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh, dOh) if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+
+    def e2e_step():
+        Q.copy_(Qh, non_blocking=True)
+        K[:, :, w.T_hist:].copy_(Kh, non_blocking=True)
+        V[:, :, w.T_hist:].copy_(Vh, non_blocking=True)
+        if dOh is not None:
+            dO.copy_(dOh, non_blocking=True)
+        step()
+        for hst, dv in zip(outs_h, outs_dev):
+            hst.copy_(dv, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = tokens / (float(t.item()) * 1e-3)
+
+    if rank == 0:
+        alg = algorithmic(w)
+        pk = peaks()
+        fwd_ms = statistics.mean(per_stage["attn_fwd"])
+        bwd_ms = statistics.mean(per_stage["attn_bwd"]) if w.backward else 0.0
+        dom = "attn_bwd" if bwd_ms >= fwd_ms else "attn_fwd"
+        dom_ms = bwd_ms if dom == "attn_bwd" else fwd_ms
+        a = alg[dom]
+        ai = a["flops"] / a["bytes"]
+        ridge = pk["bf16_tflops_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+        if ai < ridge:
+            achieved = a["bytes"] / (dom_ms * 1e-3) / 1e9
+            roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s")
+        else:
+            achieved = a["flops"] / (dom_ms * 1e-3) / 1e12
+            roof = dict(bound="tensor", achieved=achieved, peak=pk["bf16_tflops_sustained"],
+                        unit="TFLOP/s")
+        roof.update(frac=roof["achieved"] / roof["peak"],
+                    traffic=args.traffic if args.traffic is not None else recorded_traffic(dom, w),
+                    kernel=dom, launch_ms=dom_ms, algorithmic_bytes=a["bytes"],
+                    algorithmic_flops=a["flops"], peak_source=pk["source"])
+        stage_ms = {s: statistics.mean(v) for s, v in per_stage.items()}
+        line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
+                    warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
+                    scaling="weak", vs_baseline=None, dtype=w.dtype, data="synthetic",
+                    config=config_of(w), stage_ms=stage_ms, roofline=roof,
+                    gpu_launches=(LAUNCHES_PER_STEP if w.backward else 4) * args.steps,
+                    e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d,
+                             d2h_bytes_per_step=d2h),
+                    clocks=clk.summary())
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_step_rate(w, min_seconds=args.ref_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["hga", "reference"], default="hga")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.BY_NAME))
+    ap.add_argument("--ref-seconds", type=float, default=10.0,
+                    help="seconds of oracle work in the CPU baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu DRAM bytes per launch of the dominant kernel, if captured")
+    args = ap.parse_args()
+    w = W.BY_NAME[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

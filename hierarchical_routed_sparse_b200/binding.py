@@ -1,0 +1,224 @@
+"""Thin ctypes binding of libhga.so (the C ABI declared in include/hga.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libhga.so.  torch provides the device memory (tensors are passed
+by data pointer) and the stream (the current torch stream unless one is
+given).  There is no fallback: if the library is missing or fails to load,
+every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+HGA_OK, HGA_ERR_INVALID_ARG, HGA_ERR_UNSUPPORTED, HGA_ERR_CUDA = 0, 1, 2, 3
+HGA_ALL = -1
+HGA_BF16, HGA_FP32 = 0, 1
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhga.so")
+
+EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_route_chunks",
+           "hga_route_groups", "hga_attn_fwd", "hga_attn_bwd", "hga_last_error", "hga_version")
+
+
+class HGAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[hga error {code}] {msg}")
+        self.code = code
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("d", ctypes.c_int), ("T_hist", ctypes.c_int64), ("T_seg", ctypes.c_int64),
+                ("chunk", ctypes.c_int), ("group", ctypes.c_int), ("qblock", ctypes.c_int),
+                ("k_c", ctypes.c_int), ("k_g", ctypes.c_int), ("scale", ctypes.c_float),
+                ("dtype", ctypes.c_int)]
+
+
+@dataclass
+class Params:
+    """Mirror of hga_params.  k_c / k_g may be HGA_ALL (-1)."""
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    T_hist: int
+    T_seg: int
+    k_c: int
+    k_g: int
+    dtype: int = HGA_BF16
+    scale: float = 0.0
+    chunk: int = 64
+    group: int = 8
+    qblock: int = 64
+
+    @staticmethod
+    def from_workload(w) -> "Params":
+        return Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T_hist=w.T_hist, T_seg=w.T_seg,
+                      k_c=w.k_c, k_g=w.k_g, dtype=HGA_BF16 if w.dtype == "bf16" else HGA_FP32)
+
+    @property
+    def T(self) -> int:
+        return self.T_hist + self.T_seg
+
+    @property
+    def nQB(self) -> int:
+        return self.T_seg // 64
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == HGA_BF16 else torch.float32
+
+    def c(self) -> _Params:
+        return _Params(self.B, self.Hq, self.Hkv, self.d, self.T_hist, self.T_seg, self.chunk,
+                       self.group, self.qblock, self.k_c, self.k_g, float(self.scale), self.dtype)
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libhga.so (built by hierarchical_routed_sparse_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m hierarchical_routed_sparse_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I64 = ctypes.c_void_p, ctypes.c_int64
+        PP = ctypes.POINTER(_Params)
+        sig = {
+            "hga_route_widths": ([PP, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)],
+                                 ctypes.c_int),
+            "hga_workspace_size": ([PP], ctypes.c_size_t),
+            "hga_build_summaries": ([PP, P, I64, I64, P, P, P], ctypes.c_int),
+            "hga_route_chunks": ([PP, P, P, P, P, P], ctypes.c_int),
+            "hga_route_groups": ([PP, P, P, P, P, P], ctypes.c_int),
+            "hga_attn_fwd": ([PP, P, P, P, P, P, P, P], ctypes.c_int),
+            "hga_attn_bwd": ([PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P],
+                             ctypes.c_int),
+            "hga_last_error": ([], ctypes.c_char_p),
+            "hga_version": ([], ctypes.c_char_p),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(lib, name)
+            f.argtypes, f.restype = args, res
+        _lib = lib
+    return _lib
+
+
+def _check(code: int) -> None:
+    if code != HGA_OK:
+        raise HGAError(code, load().hga_last_error().decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libhga takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libhga takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def version() -> str:
+    return load().hga_version().decode()
+
+
+def route_widths(p: Params) -> tuple[int, int]:
+    wc, wg = ctypes.c_int(), ctypes.c_int()
+    _check(load().hga_route_widths(ctypes.byref(p.c()), ctypes.byref(wc), ctypes.byref(wg)))
+    return wc.value, wg.value
+
+
+def workspace_size(p: Params) -> int:
+    return int(load().hga_workspace_size(ctypes.byref(p.c())))
+
+
+def build_summaries(p: Params, K, t_begin: int, t_end: int, csum, gsum, stream=None) -> None:
+    _check(load().hga_build_summaries(ctypes.byref(p.c()), _ptr(K), t_begin, t_end, _ptr(csum),
+                                      _ptr(gsum), _stream(stream)))
+
+
+def route_chunks(p: Params, Q, csum, qbar, cidx, stream=None) -> None:
+    _check(load().hga_route_chunks(ctypes.byref(p.c()), _ptr(Q), _ptr(csum), _ptr(qbar), _ptr(cidx),
+                                   _stream(stream)))
+
+
+def route_groups(p: Params, qbar, gsum, cidx, gidx, stream=None) -> None:
+    _check(load().hga_route_groups(ctypes.byref(p.c()), _ptr(qbar), _ptr(gsum), _ptr(cidx),
+                                   _ptr(gidx), _stream(stream)))
+
+
+def attn_fwd(p: Params, Q, K, V, gidx, O, lse, stream=None) -> None:
+    _check(load().hga_attn_fwd(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(gidx), _ptr(O),
+                               _ptr(lse), _stream(stream)))
+
+
+def attn_bwd(p: Params, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, workspace,
+             stream=None) -> None:
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load().hga_attn_bwd(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                               _ptr(dO), _ptr(gidx), _ptr(dQ), _ptr(dK_seg), _ptr(dV_seg),
+                               _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+class Buffers:
+    """Device buffers of one problem shape, allocated once with torch.
+
+    ``step`` runs one segment-wise training step of the hot path: the
+    summaries of the segment's keys (earlier summaries are kept), chunk and
+    group routing, the routed attention forward and its backward.
+    """
+
+    def __init__(self, p: Params, device="cuda"):
+        self.p = p
+        wc, wg = route_widths(p)
+        B, Hq, Hkv, d, T, Ts, nQB = p.B, p.Hq, p.Hkv, p.d, p.T, p.T_seg, p.nQB
+        f32 = dict(device=device, dtype=torch.float32)
+        i32 = dict(device=device, dtype=torch.int32)
+        self.csum = torch.zeros(B, Hkv, T // 64, d, **f32)
+        self.gsum = torch.zeros(B, Hkv, T // 8, d, **f32)
+        self.qbar = torch.empty(B, Hkv, nQB, d, **f32)
+        self.cidx = torch.empty(B, Hkv, nQB, wc, **i32)
+        self.gidx = torch.empty(B, Hkv, nQB, wg, **i32)
+        self.O = torch.empty(B, Hq, Ts, d, **f32)
+        self.lse = torch.empty(B, Hq, Ts, **f32)
+        self.dQ = torch.empty(B, Hq, Ts, d, **f32)
+        self.dK = torch.empty(B, Hkv, Ts, d, **f32)
+        self.dV = torch.empty(B, Hkv, Ts, d, **f32)
+        self.ws = torch.empty(max(1, math.ceil(workspace_size(p) / 4)), **f32)
+
+    def summaries(self, K, t_begin=None, t_end=None, stream=None):
+        t_begin = self.p.T_hist if t_begin is None else t_begin
+        t_end = self.p.T if t_end is None else t_end
+        build_summaries(self.p, K, t_begin, t_end, self.csum, self.gsum, stream)
+
+    def route(self, Q, stream=None):
+        route_chunks(self.p, Q, self.csum, self.qbar, self.cidx, stream)
+        route_groups(self.p, self.qbar, self.gsum, self.cidx, self.gidx, stream)
+
+    def forward(self, Q, K, V, gidx=None, stream=None):
+        attn_fwd(self.p, Q, K, V, self.gidx if gidx is None else gidx, self.O, self.lse, stream)
+
+    def backward(self, Q, K, V, dO, gidx=None, stream=None):
+        attn_bwd(self.p, Q, K, V, self.O, self.lse, dO, self.gidx if gidx is None else gidx,
+                 self.dQ, self.dK, self.dV, self.ws, stream)
+
+    def step(self, Q, K, V, dO=None, stream=None):
+        self.summaries(K, stream=stream)
+        self.route(Q, stream)
+        self.forward(Q, K, V, stream=stream)
+        if dO is not None:
+            self.backward(Q, K, V, dO, stream=stream)

@@ -1,0 +1,214 @@
+// hga_api.cu -- the C ABI of libhga.so (declared in include/hga.h).
+//
+// Every entry point validates its arguments on the host, turns them into a
+// hga::Shape and enqueues kernels on the caller's stream.  Nothing here
+// allocates device memory or synchronises.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "hga_internal.cuh"
+
+namespace hga {
+size_t route_chunks_smem(const Shape& s);
+size_t route_groups_smem(const Shape& s);
+size_t attn_simt_smem(const Shape& s, bool backward);
+}
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where)
+{
+    return fail(HGA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+constexpr size_t kMaxSmem = 227 * 1024;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define CHECK_PTR(ptr)                                                                   \
+    do {                                                                                 \
+        if ((ptr) == nullptr) return fail(HGA_ERR_INVALID_ARG, "%s is NULL", #ptr);      \
+        if (!aligned16(ptr)) return fail(HGA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #ptr); \
+    } while (0)
+
+// Validate the parameter block and derive the shape.  Returns HGA_OK or an
+// error code with the message set.
+int make_shape(const hga_params* p, hga::Shape* s)
+{
+    if (!p) return fail(HGA_ERR_INVALID_ARG, "params is NULL");
+    if (p->B < 1 || p->Hq < 1 || p->Hkv < 1)
+        return fail(HGA_ERR_INVALID_ARG, "B, Hq, Hkv must be >= 1 (got %d, %d, %d)", p->B, p->Hq, p->Hkv);
+    if (p->Hq % p->Hkv != 0)
+        return fail(HGA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", p->Hq, p->Hkv);
+    if (p->d != 64 && p->d != 128) return fail(HGA_ERR_UNSUPPORTED, "head dim d=%d (supported: 64, 128)", p->d);
+    if (p->chunk != hga::kChunk || p->group != hga::kGroup || p->qblock != hga::kChunk)
+        return fail(HGA_ERR_UNSUPPORTED, "chunk/group/qblock must be 64/8/64 (got %d/%d/%d)", p->chunk,
+                    p->group, p->qblock);
+    if (p->T_hist < 0 || p->T_seg < 0 || p->T_hist % 64 || p->T_seg % 64)
+        return fail(HGA_ERR_INVALID_ARG, "T_hist (%lld) and T_seg (%lld) must be non-negative multiples of 64",
+                    (long long)p->T_hist, (long long)p->T_seg);
+    if ((p->k_c < 1 && p->k_c != HGA_ALL) || (p->k_g < 1 && p->k_g != HGA_ALL))
+        return fail(HGA_ERR_INVALID_ARG, "k_c (%d) and k_g (%d) must be >= 1 or HGA_ALL", p->k_c, p->k_g);
+    if (p->dtype != HGA_BF16 && p->dtype != HGA_FP32)
+        return fail(HGA_ERR_INVALID_ARG, "dtype %d is neither HGA_BF16 nor HGA_FP32", p->dtype);
+    if (!std::isfinite(p->scale) || p->scale < 0.f)
+        return fail(HGA_ERR_INVALID_ARG, "scale must be finite and >= 0 (0 selects 1/sqrt(d))");
+    const int64_t T = p->T_hist + p->T_seg;
+    if (T / hga::kGroup > INT32_MAX)
+        return fail(HGA_ERR_UNSUPPORTED, "context of %lld tokens overflows int32 group indices", (long long)T);
+    s->B = p->B; s->Hq = p->Hq; s->Hkv = p->Hkv; s->G = p->Hq / p->Hkv; s->d = p->d;
+    s->T_hist = p->T_hist; s->T_seg = p->T_seg; s->T = T;
+    s->nC = T / hga::kChunk; s->nG = T / hga::kGroup; s->nQB = p->T_seg / hga::kChunk;
+    s->k_c = p->k_c == HGA_ALL ? 0 : p->k_c;
+    s->k_g = p->k_g == HGA_ALL ? 0 : p->k_g;
+    const int64_t wc = p->k_c == HGA_ALL ? (s->nC > 0 ? s->nC : 1) : p->k_c;
+    const int64_t wg = p->k_g == HGA_ALL ? wc * hga::kGroupsPerChunk : p->k_g;
+    if (wc > INT32_MAX / 64 || wg > INT32_MAX / 64)
+        return fail(HGA_ERR_UNSUPPORTED, "routing widths too large (wc=%lld, wg=%lld)", (long long)wc,
+                    (long long)wg);
+    s->wc = (int)wc; s->wg = (int)wg;
+    s->scale = p->scale == 0.f ? 1.0f / std::sqrt((float)p->d) : p->scale;
+    s->dtype = p->dtype;
+    const int64_t units = (int64_t)s->B * s->Hq * (s->nQB > 0 ? s->nQB : 1);
+    if (units > INT32_MAX || (int64_t)s->B * s->Hkv * (s->nC > 0 ? s->nC : 1) > INT32_MAX)
+        return fail(HGA_ERR_UNSUPPORTED, "problem too large for one launch grid");
+    return HGA_OK;
+}
+
+
+}  // namespace
+
+extern "C" {
+
+const char* hga_last_error(void) { return g_err; }
+
+const char* hga_version(void) { return "hga-b200 0.1 (sm_100a)"; }
+
+int hga_route_widths(const hga_params* p, int* wc, int* wg)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (!wc || !wg) return fail(HGA_ERR_INVALID_ARG, "wc / wg output pointer is NULL");
+    *wc = s.wc;
+    *wg = s.wg;
+    return HGA_OK;
+}
+
+size_t hga_workspace_size(const hga_params* p)
+{
+    hga::Shape s;
+    if (make_shape(p, &s)) return 0;
+    return sizeof(float) * (size_t)s.B * s.Hq * s.T_seg;
+}
+
+int hga_build_summaries(const hga_params* p, const void* K, int64_t t_begin, int64_t t_end,
+                        float* csum, float* gsum, hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (t_begin < 0 || t_end < t_begin || t_end > s.T || t_begin % 64 || t_end % 64)
+        return fail(HGA_ERR_INVALID_ARG, "need 0 <= t_begin <= t_end <= T with multiples of 64 (got %lld, %lld, T=%lld)",
+                    (long long)t_begin, (long long)t_end, (long long)s.T);
+    if (t_end == t_begin) return HGA_OK;
+    CHECK_PTR(K);
+    CHECK_PTR(csum);
+    CHECK_PTR(gsum);
+    cudaError_t e = hga::launch_summaries(s, K, t_begin / 64, t_end / 64, csum, gsum,
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_build_summaries");
+}
+
+int hga_route_chunks(const hga_params* p, const void* Q, const float* csum, float* qbar,
+                     int32_t* cidx, hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    CHECK_PTR(Q);
+    CHECK_PTR(csum);
+    CHECK_PTR(qbar);
+    CHECK_PTR(cidx);
+    if (hga::route_chunks_smem(s) > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "context of %lld chunks exceeds the chunk router's shared memory",
+                    (long long)s.nC);
+    cudaError_t e = hga::launch_route_chunks(s, Q, csum, qbar, cidx, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route_chunks");
+}
+
+int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum, const int32_t* cidx,
+                     int32_t* gidx, hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    CHECK_PTR(qbar);
+    CHECK_PTR(gsum);
+    CHECK_PTR(cidx);
+    CHECK_PTR(gidx);
+    if (hga::route_groups_smem(s) > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "k_c=%d gives too many candidate groups for the group router", s.wc);
+    cudaError_t e = hga::launch_route_groups(s, qbar, gsum, cidx, gidx, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route_groups");
+}
+
+int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* V,
+                 const int32_t* gidx, float* O, float* lse, hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(gidx);
+    CHECK_PTR(O);
+    CHECK_PTR(lse);
+    if (hga::attn_simt_smem(s, false) > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "k_g=%d too large for the attention kernel", s.wg);
+    cudaError_t e = hga::launch_attn_fwd_simt(s, Q, K, V, gidx, O, lse, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_fwd");
+}
+
+int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* V, const float* O,
+                 const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK_seg,
+                 float* dV_seg, void* workspace, size_t ws_bytes, hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(O);
+    CHECK_PTR(lse);
+    CHECK_PTR(dO);
+    CHECK_PTR(gidx);
+    CHECK_PTR(dQ);
+    CHECK_PTR(dK_seg);
+    CHECK_PTR(dV_seg);
+    CHECK_PTR(workspace);
+    const size_t need = sizeof(float) * (size_t)s.B * s.Hq * s.T_seg;
+    if (ws_bytes < need)
+        return fail(HGA_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, need);
+    if (hga::attn_simt_smem(s, true) > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "k_g=%d too large for the attention kernel", s.wg);
+    cudaError_t e = hga::launch_attn_bwd_simt(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg,
+                                              static_cast<float*>(workspace),
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_bwd");
+}
+
+}  // extern "C"

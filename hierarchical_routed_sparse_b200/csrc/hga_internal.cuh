@@ -1,0 +1,93 @@
+// hga_internal.cuh -- device helpers and kernel launchers shared by the
+// translation units of libhga.so.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hga.h"
+
+namespace hga {
+
+constexpr int kChunk = 64;   // tokens per chunk == queries per block
+constexpr int kGroup = 8;    // tokens per group
+constexpr int kGroupsPerChunk = kChunk / kGroup;
+
+// Validated problem shape handed to every launcher.
+struct Shape {
+    int B, Hq, Hkv, G, d;
+    int64_t T_hist, T_seg, T;
+    int64_t nC, nG, nQB;     // chunks, groups (whole context), query blocks
+    int k_c, k_g;            // <= 0: keep all eligible
+    int wc, wg;              // index row widths
+    float scale;
+    int dtype;
+};
+
+// ---- element loads --------------------------------------------------------
+// 16-byte vector of inputs widened to float32 (8 bf16 or 4 float).
+template <typename T> struct Vec16;
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int E = 8;
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* out) {
+        const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            out[2 * i] = __uint_as_float(w[i] << 16);
+            out[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+template <> struct Vec16<float> {
+    static constexpr int E = 4;
+    static __device__ __forceinline__ void load(const float* p, float* out) {
+        const float4 r = __ldg(reinterpret_cast<const float4*>(p));
+        out[0] = r.x; out[1] = r.y; out[2] = r.z; out[3] = r.w;
+    }
+};
+
+// ---- routing keys -----------------------------------------------------------
+// A candidate (score, index) packed so that a larger 64-bit key means a higher
+// score, and among equal scores the lower index.  -0.0 is folded into +0.0 so
+// that the two compare equal, as they do in floating point.
+__device__ __forceinline__ unsigned long long pack_key(float s, int32_t idx) {
+    uint32_t u = __float_as_uint(s + 0.0f);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return (static_cast<unsigned long long>(u) << 32) | static_cast<uint32_t>(~idx);
+}
+__device__ __forceinline__ int32_t key_index(unsigned long long k) {
+    return static_cast<int32_t>(~static_cast<uint32_t>(k & 0xFFFFFFFFull));
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long w = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        v = w > v ? w : v;
+    }
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+// ---- launchers (each returns cudaError_t of its launch) ------------------------
+cudaError_t launch_summaries(const Shape& s, const void* K, int64_t c_begin, int64_t c_end,
+                             float* csum, float* gsum, cudaStream_t st);
+cudaError_t launch_route_chunks(const Shape& s, const void* Q, const float* csum, float* qbar,
+                                int32_t* cidx, cudaStream_t st);
+cudaError_t launch_route_groups(const Shape& s, const float* qbar, const float* gsum,
+                                const int32_t* cidx, int32_t* gidx, cudaStream_t st);
+cudaError_t launch_attn_fwd_simt(const Shape& s, const void* Q, const void* K, const void* V,
+                                 const int32_t* gidx, float* O, float* lse, cudaStream_t st);
+cudaError_t launch_attn_bwd_simt(const Shape& s, const void* Q, const void* K, const void* V,
+                                 const float* O, const float* lse, const void* dO,
+                                 const int32_t* gidx, float* dQ, float* dK_seg, float* dV_seg,
+                                 float* Drow, cudaStream_t st);
+
+}  // namespace hga

@@ -23,6 +23,8 @@ them.  Recipes:
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field, replace
 
 import numpy as np
@@ -45,9 +47,9 @@ def _rng(seed: int, tid: int, b: int, g: int) -> np.random.Generator:
 def round_bf16(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bf16 (ties to even), as float32."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32)
+    u = x.view(np.uint32)      # finite inputs: the sum below cannot wrap
+    u = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return u.view(np.float32)
 
 
 @dataclass(frozen=True)
@@ -125,14 +127,18 @@ class Workload:
         K = np.empty((self.B, self.Hkv, self.T, self.d), dtype=np.float32)
         V = np.empty_like(K)
         dO = np.empty_like(Q) if self.backward else None
-        for b in range(self.B):
-            for g in range(self.Hkv):
-                u = self.unit(b, g)
-                Q[b, g * G:(g + 1) * G] = u["Q"]
-                K[b, g] = u["K"]
-                V[b, g] = u["V"]
-                if dO is not None:
-                    dO[b, g * G:(g + 1) * G] = u["dO"]
+        def fill(bg):
+            b, g = divmod(bg, self.Hkv)
+            u = self.unit(b, g)
+            Q[b, g * G:(g + 1) * G] = u["Q"]
+            K[b, g] = u["K"]
+            V[b, g] = u["V"]
+            if dO is not None:
+                dO[b, g * G:(g + 1) * G] = u["dO"]
+
+        # Units are independent streams: fill them concurrently.
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(self.B * self.Hkv)))
         out = dict(Q=Q, K=K, V=V)
         if dO is not None:
             out["dO"] = dO

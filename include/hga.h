@@ -1,0 +1,150 @@
+/*
+ * hga.h -- C ABI of libhga.so: Hierarchical Global Attention (HGA), the
+ * two-level routed sparse attention, on NVIDIA B200 (sm_100a).
+ *
+ * Method source: the article "BMW's 16 GB GPU just did what needs an A100"
+ * (seventnews.com), section "What HGA does differently": the context is cut
+ * into 64-token chunks whose compact summary vectors stay in device memory;
+ * each query block scores the chunk summaries and keeps the top-k chunks,
+ * opens them at the level of 8-token groups and keeps the top-k groups, and
+ * attends the exact token K/V of the selected groups only.  Summaries steer
+ * selection and are never attended to; the router has no learned weights.
+ * The segment-wise backward of the same section detaches older KV: later
+ * segments attend earlier exact tokens, but no gradient reaches them.
+ *
+ * Readings where the article is silent: a summary is the arithmetic mean of
+ * the keys; a routing score is the plain dot product of the block query with
+ * a summary; the block query is the mean of the block's 64 queries over every
+ * q-head that shares the kv-head (GQA); routed chunks lie strictly before the
+ * block's own chunk, which is always attended with the token-causal mask;
+ * group routing is one top-k over all groups of the chosen chunks; equal
+ * scores go to the lower index; fewer eligible candidates than k keep them
+ * all and pad with -1.
+ *
+ * Conventions of every call
+ *   - All tensors are dense row-major arrays in device memory of the current
+ *     device, 16-byte aligned.  Shapes use: B batch, Hq q-heads, Hkv kv-heads
+ *     (q-head h uses kv-head h / (Hq/Hkv)), d head dim, T_hist detached
+ *     history length, T_seg active segment length, T = T_hist + T_seg,
+ *     nQB = T_seg / 64 query blocks.
+ *       Q, dO      [B][Hq][T_seg][d]    (dtype of hga_params.dtype)
+ *       K, V       [B][Hkv][T][d]       (dtype; segment keys at [T_hist, T))
+ *       csum       [B][Hkv][T/64][d]    float32 chunk summaries
+ *       gsum       [B][Hkv][T/8][d]     float32 group summaries
+ *       qbar       [B][Hkv][nQB][d]     float32 block queries
+ *       cidx       [B][Hkv][nQB][wc]    int32 chosen chunks (hga_route_widths)
+ *       gidx       [B][Hkv][nQB][wg]    int32 chosen groups
+ *       O          [B][Hq][T_seg][d]    float32
+ *       lse        [B][Hq][T_seg]       float32, natural log of sum exp
+ *       dQ         [B][Hq][T_seg][d]    float32
+ *       dK_seg, dV_seg [B][Hkv][T_seg][d] float32 (segment keys only)
+ *     Index rows hold global chunk / group numbers within their (b, kv-head),
+ *     ascending, then -1 padding.
+ *   - The caller owns all memory.  The library allocates nothing, never
+ *     synchronises, and enqueues its kernels on `stream` (a cudaStream_t;
+ *     NULL is the legacy default stream).  Calls return before the work is
+ *     done.
+ *   - Return value: HGA_OK, or an error code.  Arguments are validated on the
+ *     host before any launch; on error nothing is launched and
+ *     hga_last_error() gives a message (per calling thread).
+ */
+#ifndef HGA_H
+#define HGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HGA_OK               0
+#define HGA_ERR_INVALID_ARG  1  /* bad shape, pointer, alignment or range   */
+#define HGA_ERR_UNSUPPORTED  2  /* valid but not implemented (e.g. d = 96)  */
+#define HGA_ERR_CUDA         3  /* a launch failed (message has the detail) */
+
+#define HGA_ALL  (-1)           /* k_c / k_g: keep every eligible candidate */
+
+#define HGA_BF16 0              /* Q, K, V, dO are bfloat16                  */
+#define HGA_FP32 1              /* Q, K, V, dO are float32                   */
+
+typedef void* hga_stream_t;     /* a cudaStream_t                            */
+
+typedef struct hga_params {
+    int     B, Hq, Hkv, d;      /* d in {64, 128}; Hq % Hkv == 0             */
+    int64_t T_hist, T_seg;      /* multiples of 64; T_seg may be 0 (no work) */
+    int     chunk, group, qblock; /* must be 64, 8, 64                        */
+    int     k_c, k_g;           /* >= 1, or HGA_ALL                          */
+    float   scale;              /* softmax scale; 0 selects 1/sqrt(d)        */
+    int     dtype;              /* HGA_BF16 or HGA_FP32                      */
+} hga_params;
+
+/* Row widths of the index tables: wc = k_c (T/64 for HGA_ALL); wg = k_g
+ * (8 * wc for HGA_ALL).  Returns HGA_OK or HGA_ERR_INVALID_ARG. */
+int hga_route_widths(const hga_params* p, int* wc, int* wg);
+
+/* Bytes of device scratch that hga_attn_bwd needs (B*Hq*T_seg floats for
+ * the per-row sums D = rowsum(dO * O)).  0 on invalid parameters. */
+size_t hga_workspace_size(const hga_params* p);
+
+/* a1. Chunk and group summaries: the mean of each 64-token chunk and of each
+ * 8-token group of K (article section "What HGA does differently": compact
+ * summary vectors of each chunk stay in device memory).  Only tokens
+ * [t_begin, t_end) are summarised (multiples of 64, 0 <= t_begin <= t_end
+ * <= T); the other rows of csum / gsum are left untouched, so a segment
+ * step appends the summaries of its own keys to those kept from earlier
+ * segments.  Accumulates in float32. */
+int hga_build_summaries(const hga_params* p, const void* K, int64_t t_begin,
+                        int64_t t_end, float* csum, float* gsum,
+                        hga_stream_t stream);
+
+/* a2 + a3. Block queries and chunk routing (same section: the query scores
+ * the chunk summaries and picks the top-k chunks).  Writes qbar (the mean
+ * of the block's queries over the G q-heads of each kv-head) and cidx: for
+ * block qb with own chunk c0 = T_hist/64 + qb, the min(k_c, c0) chunks
+ * c < c0 of highest score qbar . csum[c] (float32), ties to the lower index,
+ * ascending, -1 padded to wc. */
+int hga_route_chunks(const hga_params* p, const void* Q, const float* csum,
+                     float* qbar, int32_t* cidx, hga_stream_t stream);
+
+/* a4. Group routing (same section: it opens those chunks at the level of
+ * 8-token groups).  Candidates are the 8 groups of every chunk in the cidx
+ * row; keeps the k_g of highest score qbar . gsum[j] (float32), ties to
+ * the lower index, ascending, -1 padded to wg. */
+int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum,
+                     const int32_t* cidx, int32_t* gidx, hga_stream_t stream);
+
+/* a5. Routed attention forward (same section: only the exact token K/V of
+ * the selected groups is loaded for the attention).  Query i of block qb
+ * (global position p = T_hist + 64 qb + i) of q-head h attends the 8 tokens
+ * of every group in gidx[b][h/G][qb] plus tokens 64*(p/64) .. p of its own
+ * chunk: O = softmax(scale * q K^T) V and lse = log sum exp(scale * q K^T).
+ * bf16 inputs use tensor-core MMAs with float32 accumulation and softmax. */
+int hga_attn_fwd(const hga_params* p, const void* Q, const void* K,
+                 const void* V, const int32_t* gidx, float* O, float* lse,
+                 hga_stream_t stream);
+
+/* a6. Routed attention backward with the routing of the forward frozen
+ * (same section: the router has no learned weights, so gradients reach the
+ * projections as in the dense case; older KV is detached).  Given O and lse
+ * of hga_attn_fwd and the upstream dO, writes dQ, and dK_seg / dV_seg for
+ * the segment keys T_hist .. T-1 (overwritten, not accumulated), summed over
+ * the G q-heads of each kv-head.  History keys receive no gradient.
+ * `workspace` must hold hga_workspace_size(p) bytes of device memory. */
+int hga_attn_bwd(const hga_params* p, const void* Q, const void* K,
+                 const void* V, const float* O, const float* lse,
+                 const void* dO, const int32_t* gidx, float* dQ,
+                 float* dK_seg, float* dV_seg, void* workspace,
+                 size_t ws_bytes, hga_stream_t stream);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* hga_last_error(void);
+
+/* Library version string. */
+const char* hga_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HGA_H */

@@ -1,0 +1,118 @@
+"""CPU checks of the C ABI: the library loads, exports every function that
+include/hga.h declares, and rejects bad arguments on the host before any
+launch (these calls never reach the GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hierarchical_routed_sparse_b200 as hga
+from hierarchical_routed_sparse_b200 import build as hbuild
+from hierarchical_routed_sparse_b200.binding import _Params
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "hga.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    hbuild.build()
+    return hga.load()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hga_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert "hga_attn_fwd" in names and "hga_attn_bwd" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(hga.EXPORTS) == set(names)
+    assert "sm_100a" in hga.version()
+
+
+def _p(**kw):
+    base = dict(B=1, Hq=32, Hkv=8, d=128, T_hist=14336, T_seg=2048, k_c=8, k_g=32)
+    base.update(kw)
+    return hga.Params(**base)
+
+
+def test_route_widths_and_workspace(lib):
+    assert hga.route_widths(_p()) == (8, 32)
+    assert hga.route_widths(_p(k_c=hga.HGA_ALL, k_g=hga.HGA_ALL)) == (256, 2048)
+    assert hga.route_widths(_p(k_c=4, k_g=hga.HGA_ALL)) == (4, 32)
+    assert hga.workspace_size(_p()) == 4 * 32 * 2048
+    assert hga.workspace_size(_p(d=96)) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), hga.HGA_ERR_UNSUPPORTED),
+    (dict(T_hist=100), hga.HGA_ERR_INVALID_ARG),
+    (dict(T_seg=2000), hga.HGA_ERR_INVALID_ARG),
+    (dict(Hq=30), hga.HGA_ERR_INVALID_ARG),
+    (dict(k_c=0), hga.HGA_ERR_INVALID_ARG),
+    (dict(k_g=-5), hga.HGA_ERR_INVALID_ARG),
+    (dict(dtype=7), hga.HGA_ERR_INVALID_ARG),
+    (dict(chunk=32), hga.HGA_ERR_UNSUPPORTED),
+    (dict(B=0), hga.HGA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), hga.HGA_ERR_INVALID_ARG),
+])
+def test_invalid_params_rejected(lib, kw, code):
+    p = _p(**kw).c()
+    wc, wg = ctypes.c_int(), ctypes.c_int()
+    assert lib.hga_route_widths(ctypes.byref(p), ctypes.byref(wc), ctypes.byref(wg)) == code
+    assert lib.hga_last_error().decode()
+    # The same validation guards every launching call: nothing is launched.
+    P = ctypes.c_void_p(16)
+    assert lib.hga_attn_fwd(ctypes.byref(p), P, P, P, P, P, P, None) == code
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    p = _p().c()
+    good = ctypes.c_void_p(1 << 20)
+    assert lib.hga_attn_fwd(ctypes.byref(p), None, good, good, good, good, good, None) == \
+        hga.HGA_ERR_INVALID_ARG
+    assert "Q is NULL" in lib.hga_last_error().decode()
+    bad = ctypes.c_void_p((1 << 20) + 4)
+    assert lib.hga_route_chunks(ctypes.byref(p), good, bad, good, good, None) == hga.HGA_ERR_INVALID_ARG
+    assert "csum is not 16-byte aligned" in lib.hga_last_error().decode()
+    # Summary range must be 64-aligned and inside the context.
+    assert lib.hga_build_summaries(ctypes.byref(p), good, 64, 100, good, good, None) == \
+        hga.HGA_ERR_INVALID_ARG
+    assert lib.hga_build_summaries(ctypes.byref(p), good, 0, 1 << 20, good, good, None) == \
+        hga.HGA_ERR_INVALID_ARG
+    # Workspace smaller than hga_workspace_size.
+    P = ctypes.c_void_p(1 << 20)
+    assert lib.hga_attn_bwd(ctypes.byref(p), P, P, P, P, P, P, P, P, P, P, P, 16, None) == \
+        hga.HGA_ERR_INVALID_ARG
+    assert "workspace" in lib.hga_last_error().decode()
+
+
+def test_empty_segment_is_a_no_op(lib):
+    # T_seg = 0: valid, nothing to do, no pointer is touched.
+    p = _p(T_seg=0).c()
+    assert lib.hga_route_chunks(ctypes.byref(p), None, None, None, None, None) == hga.HGA_OK
+    assert lib.hga_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, None) == hga.HGA_OK
+    assert lib.hga_build_summaries(ctypes.byref(p), None, 64, 64, None, None, None) == hga.HGA_OK
+
+
+def test_params_struct_layout_matches_header(lib, tmp_path):
+    # Compare the ctypes mirror with the C compiler's layout of hga_params.
+    import subprocess
+    fields = [f for f, _ in _Params._fields_]
+    prog = "#include <stdio.h>\n#include <stddef.h>\n#include \"hga.h\"\nint main(void){\n"
+    prog += 'printf("%zu\\n", sizeof(hga_params));\n'
+    prog += "".join(f'printf("%zu\\n", offsetof(hga_params, {f}));\n' for f in fields)
+    prog += "return 0;}\n"
+    src = tmp_path / "layout.c"
+    src.write_text(prog)
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    out = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    assert out[0] == ctypes.sizeof(_Params)
+    assert out[1:] == [getattr(_Params, f).offset for f in fields]
