@@ -231,6 +231,27 @@ def dist_env():
     return rank, world, local
 
 
+def rank_workload(w, rank: int):
+    """The independent problem of one rank: same shape, its own seed."""
+    return w.with_(seed=w.seed + rank)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank duration over all ranks (1 rank: the value itself)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """All ranks' tokens over the slowest rank's time (weak scaling)."""
+    return world * steps * tokens_per_rank_step / (max_ms * 1e-3)
+
+
 def config_of(w) -> dict:
     return dict(workload=w.name, B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T_hist=w.T_hist,
                 T_seg=w.T_seg, T=w.T, k_c=w.k_c, k_g=w.k_g, keys=w.keys,
@@ -264,7 +285,7 @@ def run_gpu(args, w) -> None:
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-    wr = w.with_(seed=w.seed + rank)                 # independent problem per rank
+    wr = rank_workload(w, rank)                      # independent problem per rank
     x = wr.full()
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     Q = torch.from_numpy(x["Q"]).to(dev, tdt)
@@ -319,13 +340,8 @@ def run_gpu(args, w) -> None:
         for j, s in enumerate(stages):
             per_stage[s].append(ev[j].elapsed_time(ev[j + 1]))
         totals.append(ev[0].elapsed_time(ev[4]))
-    total_ms = sum(totals)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
-    tokens = world * args.steps * w.B * w.T_seg
-    value = tokens / (total_ms * 1e-3)
+    total_ms = max_over_ranks(sum(totals), dev)
+    value = whole_job_rate(w.B * w.T_seg, args.steps, world, total_ms)
 
     # ---- end to end through the public API with host buffers ----------------------
     Qh = torch.from_numpy(x["Q"]).to(tdt).pin_memory()
@@ -358,10 +374,8 @@ def run_gpu(args, w) -> None:
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = tokens / (float(t.item()) * 1e-3)
+    e2e_value = whole_job_rate(w.B * w.T_seg, args.steps, world,
+                               max_over_ranks(e0.elapsed_time(e1), dev))
 
     if rank == 0:
         alg = algorithmic(w)
