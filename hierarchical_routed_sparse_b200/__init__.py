@@ -8,11 +8,12 @@ Method source: the article "BMW's 16 GB GPU just did what needs an A100"
 buffers of one problem shape and runs a whole segment step.
 """
 from .binding import (EXPORTS, HGA_ALL, HGA_BF16, HGA_ERR_CUDA, HGA_ERR_INVALID_ARG,
-                      HGA_ERR_UNSUPPORTED, HGA_FP32, HGA_OK, LIB_PATH, Buffers, HGAError, Params,
-                      attn_bwd, attn_fwd, build_summaries, load, route_chunks, route_groups,
+                      HGA_ERR_UNSUPPORTED, HGA_FP32, HGA_OK, LIB_PATH, NOALLOC_MAX_ROWS, Buffers,
+                      HGAError, Params,
+                      attn_bwd, attn_bwd_noalloc, attn_fwd, build_summaries, load, route_chunks, route_groups,
                       route_widths, version, workspace_size)
 
 __all__ = ["EXPORTS", "HGA_ALL", "HGA_BF16", "HGA_FP32", "HGA_OK", "HGA_ERR_CUDA",
-           "HGA_ERR_INVALID_ARG", "HGA_ERR_UNSUPPORTED", "LIB_PATH", "Buffers", "HGAError",
-           "Params", "attn_bwd", "attn_fwd", "build_summaries", "load", "route_chunks",
+           "HGA_ERR_INVALID_ARG", "HGA_ERR_UNSUPPORTED", "LIB_PATH", "NOALLOC_MAX_ROWS", "Buffers", "HGAError",
+           "Params", "attn_bwd", "attn_bwd_noalloc", "attn_fwd", "build_summaries", "load", "route_chunks",
            "route_groups", "route_widths", "version", "workspace_size"]

@@ -22,7 +22,9 @@ HGA_BF16, HGA_FP32 = 0, 1
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhga.so")
 
 EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_route_chunks",
-           "hga_route_groups", "hga_attn_fwd", "hga_attn_bwd", "hga_last_error", "hga_version")
+           "hga_route_groups", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
+           "hga_last_error", "hga_version")
+NOALLOC_MAX_ROWS = 1 << 20     # HGA_NOALLOC_MAX_ROWS
 
 
 class HGAError(RuntimeError):
@@ -101,6 +103,7 @@ def load() -> ctypes.CDLL:
             "hga_attn_fwd": ([PP, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_attn_bwd": ([PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P],
                              ctypes.c_int),
+            "hga_attn_bwd_noalloc": ([PP, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_last_error": ([], ctypes.c_char_p),
             "hga_version": ([], ctypes.c_char_p),
         }
@@ -172,6 +175,21 @@ def attn_bwd(p: Params, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, workspace
     _check(load().hga_attn_bwd(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
                                _ptr(dO), _ptr(gidx), _ptr(dQ), _ptr(dK_seg), _ptr(dV_seg),
                                _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def attn_bwd_noalloc(p: Params, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg,
+                     stream=None) -> None:
+    """hga_attn_bwd with the library's built-in scratch instead of a workspace.
+
+    For callers that cannot pass scratch memory (plugin interfaces that give
+    an operator only its inputs and outputs, hosts whose pool owns all device
+    memory, loops that must not call cudaMalloc / cudaFree).  Limited to
+    B*Hq*T_seg <= NOALLOC_MAX_ROWS; calls that overlap on the GPU share one
+    scratch array and race, so keep them on one stream.
+    """
+    _check(load().hga_attn_bwd_noalloc(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                                       _ptr(lse), _ptr(dO), _ptr(gidx), _ptr(dQ), _ptr(dK_seg),
+                                       _ptr(dV_seg), _stream(stream)))
 
 
 class Buffers:

@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "hga_internal.cuh"
 
@@ -212,3 +213,82 @@ int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* 
 }
 
 }  // extern "C"
+
+// ---- hga_attn_bwd_noalloc: the backward with built-in scratch -----------------
+//
+// Some callers cannot give this library a scratch buffer: plugin interfaces
+// that hand an operator only its inputs and outputs, hosts whose memory pool
+// owns every byte of device memory, and latency-bound loops that must not
+// call cudaMalloc / cudaFree (cudaFree waits for the whole device).  For
+// them the backward's only scratch, the per-row sums D = rowsum(dO * O), lives
+// in the fixed array below, which the CUDA runtime places in device memory
+// when the library's code is loaded on a device and frees at process exit.
+// Host code must not use the array's name as a pointer: on the host it is a
+// stand-in symbol, not a device address.  Its device address is looked up
+// once per device with cudaGetSymbolAddress, on the first call made while
+// that device is current, and cached.
+
+static __device__ __align__(256) float g_noalloc_rowsum[HGA_NOALLOC_MAX_ROWS];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_rowsum on the current device (looked up once).
+int noalloc_scratch(float** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "hga_attn_bwd_noalloc: cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(HGA_ERR_UNSUPPORTED, "hga_attn_bwd_noalloc: device %d beyond the %d supported", dev,
+                    kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, g_noalloc_rowsum);
+        if (e != cudaSuccess) return cuda_fail(e, "hga_attn_bwd_noalloc: cudaGetSymbolAddress");
+        g_noalloc_addr[dev] = static_cast<float*>(addr);
+    }
+    *out = g_noalloc_addr[dev];
+    return HGA_OK;
+}
+
+}  // namespace
+
+extern "C" int hga_attn_bwd_noalloc(const hga_params* p, const void* Q, const void* K, const void* V,
+                                    const float* O, const float* lse, const void* dO,
+                                    const int32_t* gidx, float* dQ, float* dK_seg, float* dV_seg,
+                                    hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(O);
+    CHECK_PTR(lse);
+    CHECK_PTR(dO);
+    CHECK_PTR(gidx);
+    CHECK_PTR(dQ);
+    CHECK_PTR(dK_seg);
+    CHECK_PTR(dV_seg);
+    const int64_t rows = (int64_t)s.B * s.Hq * s.T_seg;
+    if (rows > HGA_NOALLOC_MAX_ROWS)
+        return fail(HGA_ERR_INVALID_ARG,
+                    "hga_attn_bwd_noalloc: B*Hq*T_seg = %lld exceeds its built-in scratch of %d rows; "
+                    "use hga_attn_bwd with a caller-provided workspace", (long long)rows,
+                    HGA_NOALLOC_MAX_ROWS);
+    if (hga::attn_simt_smem(s, true) > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "k_g=%d too large for the attention kernel", s.wg);
+    float* scratch = nullptr;
+    if (int r = noalloc_scratch(&scratch)) return r;
+    // Every row sum the kernels read is first written by this call, so the
+    // scratch needs no clearing between calls.
+    cudaError_t e = hga::launch_attn_bwd_simt(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, scratch,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_bwd_noalloc");
+}

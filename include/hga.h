@@ -119,7 +119,7 @@ int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum,
  * (global position p = T_hist + 64 qb + i) of q-head h attends the 8 tokens
  * of every group in gidx[b][h/G][qb] plus tokens 64*(p/64) .. p of its own
  * chunk: O = softmax(scale * q K^T) V and lse = log sum exp(scale * q K^T).
- * bf16 inputs use tensor-core MMAs with float32 accumulation and softmax. */
+ * Accumulation and softmax are in float32. */
 int hga_attn_fwd(const hga_params* p, const void* Q, const void* K,
                  const void* V, const int32_t* gidx, float* O, float* lse,
                  hga_stream_t stream);
@@ -136,6 +136,33 @@ int hga_attn_bwd(const hga_params* p, const void* Q, const void* K,
                  const void* dO, const int32_t* gidx, float* dQ,
                  float* dK_seg, float* dV_seg, void* workspace,
                  size_t ws_bytes, hga_stream_t stream);
+
+/* Largest B*Hq*T_seg that hga_attn_bwd_noalloc accepts. */
+#define HGA_NOALLOC_MAX_ROWS 1048576
+
+/* hga_attn_bwd without the workspace argument.  The article has no
+ * counterpart: this entry point exists for callers that cannot hand the
+ * library any scratch memory -- plugin interfaces that pass an operator only
+ * its inputs and outputs, hosts whose memory pool owns all device memory,
+ * and loops that must not call cudaMalloc / cudaFree.  It computes what
+ * hga_attn_bwd computes and allocates nothing: its scratch (B*Hq*T_seg
+ * floats of row sums) is a fixed array of HGA_NOALLOC_MAX_ROWS floats (4 MiB)
+ * inside the library, held on every device that loads the library until the
+ * process exits.
+ *   - B*Hq*T_seg above HGA_NOALLOC_MAX_ROWS returns HGA_ERR_INVALID_ARG,
+ *     with nothing launched.
+ *   - The first call on a device (the calling thread's current device, which
+ *     must own every pointer and the stream) looks up the array's device
+ *     address with cudaGetSymbolAddress and caches it; make that first call
+ *     before any stream capture on that device.
+ *   - All calls on a device share the one array and every call overwrites
+ *     the entries it uses before reading them.  Calls whose kernels overlap
+ *     on the GPU (other streams, other threads) race on it: order them, e.g.
+ *     on one stream. */
+int hga_attn_bwd_noalloc(const hga_params* p, const void* Q, const void* K,
+                         const void* V, const float* O, const float* lse,
+                         const void* dO, const int32_t* gidx, float* dQ,
+                         float* dK_seg, float* dV_seg, hga_stream_t stream);
 
 /* Message of the last failed call on this thread ("" if none). */
 const char* hga_last_error(void);
