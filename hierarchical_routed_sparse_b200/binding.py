@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhga.so")
 
 EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_route_chunks",
            "hga_route_groups", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
-           "hga_last_error", "hga_version")
+           "hga_device_status", "hga_last_error", "hga_version")
 NOALLOC_MAX_ROWS = 1 << 20     # HGA_NOALLOC_MAX_ROWS
 
 
@@ -104,6 +104,7 @@ def load() -> ctypes.CDLL:
             "hga_attn_bwd": ([PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P],
                              ctypes.c_int),
             "hga_attn_bwd_noalloc": ([PP, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "hga_device_status": ([ctypes.POINTER(ctypes.c_int), ctypes.c_int], ctypes.c_int),
             "hga_last_error": ([], ctypes.c_char_p),
             "hga_version": ([], ctypes.c_char_p),
         }
@@ -137,6 +138,13 @@ def _stream(stream) -> ctypes.c_void_p:
 
 def version() -> str:
     return load().hga_version().decode()
+
+
+def device_status(clear: bool = False) -> int:
+    """Status word of the kernels' bounded waits (0: none ran out).  Syncs."""
+    v = ctypes.c_int()
+    _check(load().hga_device_status(ctypes.byref(v), int(clear)))
+    return v.value
 
 
 def route_widths(p: Params) -> tuple[int, int]:

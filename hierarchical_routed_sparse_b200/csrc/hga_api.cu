@@ -98,6 +98,15 @@ const char* hga_last_error(void) { return g_err; }
 
 const char* hga_version(void) { return "hga-b200 0.1 (sm_100a)"; }
 
+int hga_device_status(int* status, int clear)
+{
+    if (!status) return fail(HGA_ERR_INVALID_ARG, "status is NULL");
+    const int v = hga::attn_fwd_tc_status(clear != 0);
+    if (v < 0) return fail(HGA_ERR_CUDA, "hga_device_status: the status word could not be read");
+    *status = v;
+    return HGA_OK;
+}
+
 int hga_route_widths(const hga_params* p, int* wc, int* wg)
 {
     hga::Shape s;
@@ -179,7 +188,10 @@ int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* 
     CHECK_PTR(lse);
     if (hga::attn_simt_smem(s, false) > kMaxSmem)
         return fail(HGA_ERR_UNSUPPORTED, "k_g=%d too large for the attention kernel", s.wg);
-    cudaError_t e = hga::launch_attn_fwd_simt(s, Q, K, V, gidx, O, lse, static_cast<cudaStream_t>(stream));
+    // bf16: tcgen05 tensor-core kernel; float32: the FMA kernel (1e-4 gate).
+    cudaError_t e = hga::attn_fwd_tc_supported(s)
+                        ? hga::launch_attn_fwd_tc(s, Q, K, V, gidx, O, lse, static_cast<cudaStream_t>(stream))
+                        : hga::launch_attn_fwd_simt(s, Q, K, V, gidx, O, lse, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_fwd");
 }
 

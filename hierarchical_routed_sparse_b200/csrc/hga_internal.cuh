@@ -90,4 +90,12 @@ cudaError_t launch_attn_bwd_simt(const Shape& s, const void* Q, const void* K, c
                                  const int32_t* gidx, float* dQ, float* dK_seg, float* dV_seg,
                                  float* Drow, cudaStream_t st);
 
+// Tensor-core (tcgen05) path for bf16 inputs.
+bool attn_fwd_tc_supported(const Shape& s);
+cudaError_t launch_attn_fwd_tc(const Shape& s, const void* Q, const void* K, const void* V,
+                               const int32_t* gidx, float* O, float* lse, cudaStream_t st);
+// Status word of the tensor-core kernels' bounded waits (0 = none ran out;
+// -1 = could not be read).  Synchronises with the device.
+int attn_fwd_tc_status(bool clear);
+
 }  // namespace hga

@@ -119,7 +119,8 @@ int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum,
  * (global position p = T_hist + 64 qb + i) of q-head h attends the 8 tokens
  * of every group in gidx[b][h/G][qb] plus tokens 64*(p/64) .. p of its own
  * chunk: O = softmax(scale * q K^T) V and lse = log sum exp(scale * q K^T).
- * Accumulation and softmax are in float32. */
+ * bf16 inputs run on the tcgen05 tensor cores, float32 inputs on the CUDA
+ * cores; accumulation and softmax are in float32 either way. */
 int hga_attn_fwd(const hga_params* p, const void* Q, const void* K,
                  const void* V, const int32_t* gidx, float* O, float* lse,
                  hga_stream_t stream);
@@ -163,6 +164,13 @@ int hga_attn_bwd_noalloc(const hga_params* p, const void* Q, const void* K,
                          const void* V, const float* O, const float* lse,
                          const void* dO, const int32_t* gidx, float* dQ,
                          float* dK_seg, float* dV_seg, hga_stream_t stream);
+
+/* Status word of the kernels' bounded waits: every wait of a tensor-core
+ * kernel on a barrier gives up after one second, records the code of the wait
+ * in this word and lets the kernel return (its outputs are then invalid).
+ * *status = 0 when no wait ran out; `clear` != 0 resets the word.
+ * Synchronises with the device. */
+int hga_device_status(int* status, int clear);
 
 /* Message of the last failed call on this thread ("" if none). */
 const char* hga_last_error(void);

@@ -94,6 +94,7 @@ def run_gpu(w, x: dict, gidx_in: np.ndarray | None = None, full_summaries: bool 
         buf.backward(Q, K, V, dO, gidx=gidx)
         out.update(dQ=buf.dQ, dK=buf.dK, dV=buf.dV)
     torch.cuda.synchronize()
+    assert hga.device_status() == 0, "a kernel's bounded wait ran out"
     out.update(csum=buf.csum, gsum=buf.gsum, qbar=buf.qbar, cidx=buf.cidx, gidx=buf.gidx,
                O=buf.O, lse=buf.lse)
     return {k: v.cpu().numpy() for k, v in out.items()}, buf
