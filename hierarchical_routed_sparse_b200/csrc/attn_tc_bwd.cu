@@ -1,0 +1,481 @@
+// attn_tc_bwd.cu -- a6 routed attention backward on the tcgen05 tensor cores
+// (bf16 inputs, d = 128, float32 accumulation).
+//
+// Article "BMW's 16 GB GPU just did what needs an A100" (seventnews.com),
+// section "What HGA does differently": the router has no learned weights, so
+// the gradients reach Q, K and V exactly as in dense attention over the routed
+// key set; the segment-wise backward of the same section detaches older KV,
+// so key gradients are kept for the segment's own tokens only.  The routing
+// of the forward is reused unchanged.
+//
+// One CTA owns one (batch, kv-head, query block) and a pair of q-heads: one
+// M-tile of 128 query rows.  For each 64-key tile (8 routed groups, or the
+// own chunk with the causal mask):
+//     S   = Q K^T, dP = dO V^T        tcgen05.mma -> tensor memory
+//     P   = exp2(S*c - lse), dS = P (dP - D)   row per thread; both written
+//           to shared memory as bf16 hi + lo parts (~16-bit operands)
+//     dQ += dS K                      A = dS (K-major), B = K (MN-major)
+//     dV^T = dO^T P, dK^T = Q^T dS    A = dO / Q read MN-major, B = P / dS
+// dV^T and dK^T (d on the tensor-memory lanes, keys on the columns) are added
+// to the float32 dV_seg / dK_seg rows of the segment's keys with coalesced
+// atomics; tiles whose keys are all detached history skip both products
+// (routed groups are ascending, so history tiles come first).
+//
+// Warp roles (320 threads): warps 0-3 softmax-gradient rows and the dQ
+// epilogue, warps 4-7 the dK/dV epilogue, warp 8 TMA producer, warp 9
+// tensor-memory owner and MMA issuer.  Tensor memory (512 columns): S and dP
+// double-buffered (4 x 64), dQ (128), dV^T (64), dK^T (64).
+#include "hga_internal.cuh"
+#include "sm100.cuh"
+
+namespace hga {
+namespace {
+
+using namespace sm100;
+
+constexpr int D = 128;
+constexpr int H = 2;                  // 64-column halves of d
+constexpr int kStages = 2;
+constexpr int kKeys = 64;
+constexpr int kThreads = 320;
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum : int {
+    kSiteQ = 201, kSiteFull, kSiteEmpty, kSiteSdp, kSitePs, kSiteMm2, kSiteDrained, kSiteFinal, kSiteDrain
+};
+
+struct BwdSmem {
+    static constexpr int kRows128 = 128 * 128;        // 128 rows x 128 B
+    static constexpr int kKVHalf = kKeys * 128;       // 64 keys x 128 B
+    static constexpr int q_off = 0;                   // [2 halves][128 rows][64]
+    static constexpr int do_off = q_off + H * kRows128;
+    static constexpr int k_off = do_off + H * kRows128;
+    static constexpr int v_off = k_off + kStages * H * kKVHalf;
+    static constexpr int p_off = v_off + kStages * H * kKVHalf;   // P hi, P lo: [128 rows][64 keys]
+    static constexpr int ds_off = p_off + 2 * kRows128;           // dS hi, dS lo
+    static constexpr int bar_off = ds_off + 2 * kRows128;
+    // q, full[2], empty[2], sdp[2], ps, mm2, drained, final
+    static constexpr int n_bars = 1 + 2 * kStages + 2 + 4;
+    static constexpr int tmem_slot_off = bar_off + 8 * n_bars;
+    static constexpr int bytes = tmem_slot_off + 16;
+    static constexpr int alloc = bytes + 1024;
+};
+
+// Tensor-memory columns.
+constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDV = 384, kColDK = 448;
+
+struct BwdArgs {
+    const int32_t* gidx;
+    const float* lse;
+    const float* Drow;
+    float* dQ;
+    float* dK;
+    float* dV;
+    int Hq, Hkv, G, wg;
+    int64_t T_hist, T_seg, nQB;
+    int q_rows;
+    float scale, scale_log2;
+};
+
+// Routed groups form an ascending prefix of the index row.
+__device__ __forceinline__ int count_groups(const int32_t* grow, int wg)
+{
+    int n = 0;
+    while (n < wg && grow[n] >= 0) ++n;
+    return n;
+}
+
+// Does key tile t hold any segment token (position >= T_hist)?
+__device__ __forceinline__ bool tile_has_segment_keys(int t, int n_rt, int n_g, const int32_t* grow,
+                                                      int64_t T_hist)
+{
+    if (t == n_rt) return true;                              // own chunk
+    const int last = min(t * 8 + 7, n_g - 1);
+    return (int64_t)grow[last] * 8 + 7 >= T_hist;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                   const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ CUtensorMap tm_v8,
+                   const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v64,
+                   const BwdArgs a)
+{
+    using L = BwdSmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + L::bar_off;
+    const uint32_t bar_q = bar0;
+    auto bar_full = [&](int s) { return bar0 + 8 * (1 + s); };
+    auto bar_empty = [&](int s) { return bar0 + 8 * (1 + kStages + s); };
+    auto bar_sdp = [&](int b) { return bar0 + 8 * (1 + 2 * kStages + b); };
+    const uint32_t bar_ps = bar0 + 8 * (3 + 2 * kStages);
+    const uint32_t bar_mm2 = bar0 + 8 * (4 + 2 * kStages);
+    const uint32_t bar_drained = bar0 + 8 * (5 + 2 * kStages);
+    const uint32_t bar_final = bar0 + 8 * (6 + 2 * kStages);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::tmem_slot_off);
+    __shared__ int s_abort;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t u = blockIdx.x;                           // ((b*Hkv)+g)*nQB + qb
+    const int64_t qb = u % a.nQB, bg = u / a.nQB;
+    const int64_t b = bg / a.Hkv, g = bg % a.Hkv;
+    const int head0 = 2 * blockIdx.y;
+    const int64_t T = a.T_hist + a.T_seg;
+    const int64_t kv_base = bg * T;
+    const int64_t own_start = a.T_hist + qb * 64;
+
+    const int32_t* grow = a.gidx + u * a.wg;
+    const int n_g = count_groups(grow, a.wg);
+    const int n_rt = (n_g + 7) / 8;
+    const int nt = n_rt + 1;
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_empty(s), 1);
+        }
+        mbar_init(bar_sdp(0), 1);
+        mbar_init(bar_sdp(1), 1);
+        mbar_init(bar_ps, 128);
+        mbar_init(bar_mm2, 1);
+        mbar_init(bar_drained, 128);
+        mbar_init(bar_final, 1);
+        fence_mbar_init();
+    }
+    if (warp == 9) tmem_alloc(smem_u32(tmem_slot), 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_do);
+            prefetch_tmap(&tm_k8);
+            prefetch_tmap(&tm_v8);
+            prefetch_tmap(&tm_k64);
+            prefetch_tmap(&tm_v64);
+            mbar_expect_tx(bar_q, 2 * 2 * H * 64 * 128);
+            for (int hp = 0; hp < 2; ++hp) {
+                const int head = head0 + hp;
+                const int y = head < a.G ? int((b * a.Hq + g * a.G + head) * a.T_seg + qb * 64) : a.q_rows;
+                for (int c = 0; c < H; ++c) {
+                    const uint32_t off = c * L::kRows128 + hp * 64 * 128;
+                    tma_load_2d(sbase + L::q_off + off, &tm_q, 64 * c, y, bar_q);
+                    tma_load_2d(sbase + L::do_off + off, &tm_do, 64 * c, y, bar_q);
+                }
+            }
+            for (int t = 0; t < nt; ++t) {
+                const int s = t % kStages, r = t / kStages;
+                if (t >= kStages && !mbar_wait(bar_empty(s), (r - 1) & 1, kSiteEmpty)) {
+                    s_abort = 1;
+                    break;
+                }
+                mbar_expect_tx(bar_full(s), 2 * H * kKeys * 128);
+                const uint32_t kdst = sbase + L::k_off + s * H * L::kKVHalf;
+                const uint32_t vdst = sbase + L::v_off + s * H * L::kKVHalf;
+                if (t < n_rt) {
+                    for (int j = 0; j < 8; ++j) {
+                        const int gi = t * 8 + j;
+                        const int grp = grow[gi < n_g ? gi : 0];
+                        const int y = int(kv_base + (int64_t)grp * 8);
+                        for (int c = 0; c < H; ++c) {
+                            tma_load_2d(kdst + c * L::kKVHalf + j * 1024, &tm_k8, 64 * c, y, bar_full(s));
+                            tma_load_2d(vdst + c * L::kKVHalf + j * 1024, &tm_v8, 64 * c, y, bar_full(s));
+                        }
+                    }
+                } else {
+                    const int y = int(kv_base + own_start);
+                    for (int c = 0; c < H; ++c) {
+                        tma_load_2d(kdst + c * L::kKVHalf, &tm_k64, 64 * c, y, bar_full(s));
+                        tma_load_2d(vdst + c * L::kKVHalf, &tm_v64, 64 * c, y, bar_full(s));
+                    }
+                }
+            }
+        }
+    } else if (warp == 9) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_sdp = idesc_bf16(128, kKeys, 0, 0);   // S, dP
+            constexpr uint32_t id_dq = idesc_bf16(128, D, 0, 1);        // dQ: A dS K-major, B K MN-major
+            constexpr uint32_t id_kv = idesc_bf16(128, kKeys, 1, 1);    // dV^T, dK^T: both MN-major
+            bool ok = mbar_wait(bar_q, 0, kSiteQ);
+            auto issue_sdp = [&](int t) -> bool {
+                const int s = t % kStages, bb = t & 1;
+                if (!mbar_wait(bar_full(s), (t / kStages) & 1, kSiteFull)) return false;
+                tc_fence_after();
+                for (int kk = 0; kk < 4 * H; ++kk) {
+                    const uint32_t o = (kk / 4) * L::kRows128 + (kk % 4) * 32;
+                    const uint32_t ko = (s * H + kk / 4) * L::kKVHalf + (kk % 4) * 32;
+                    mma_ss(tmem + kColS + bb * kKeys, sdesc_sw128(sbase + L::q_off + o, 16, 1024),
+                           sdesc_sw128(sbase + L::k_off + ko, 16, 1024), id_sdp, kk > 0);
+                    mma_ss(tmem + kColDP + bb * kKeys, sdesc_sw128(sbase + L::do_off + o, 16, 1024),
+                           sdesc_sw128(sbase + L::v_off + ko, 16, 1024), id_sdp, kk > 0);
+                }
+                mma_commit(bar_sdp(bb));
+                return true;
+            };
+            if (ok) ok = issue_sdp(0);
+            for (int t = 0; ok && t < nt; ++t) {
+                if (t + 1 < nt && !(ok = issue_sdp(t + 1))) break;
+                const int s = t % kStages;
+                if (!(ok = mbar_wait(bar_ps, t & 1, kSitePs))) break;
+                tc_fence_after();
+                // dQ += dS K  (dS hi and lo against the same K)
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t kb = sdesc_sw128(sbase + L::k_off + s * H * L::kKVHalf + kk * 2048, L::kKVHalf, 1024);
+                    mma_ss(tmem + kColDQ, sdesc_sw128(sbase + L::ds_off + kk * 32, 16, 1024), kb, id_dq,
+                           t > 0 || kk > 0);
+                    mma_ss(tmem + kColDQ, sdesc_sw128(sbase + L::ds_off + L::kRows128 + kk * 32, 16, 1024), kb,
+                           id_dq, true);
+                }
+                if (tile_has_segment_keys(t, n_rt, n_g, grow, a.T_hist)) {
+                    if (t >= 1 && !(ok = mbar_wait(bar_drained, (t - 1) & 1, kSiteDrained))) break;
+                    tc_fence_after();
+                    // dV^T = dO^T P and dK^T = Q^T dS over the 128 query rows.
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t dOt = sdesc_sw128(sbase + L::do_off + kk * 2048, L::kRows128, 1024);
+                        const uint64_t Qt = sdesc_sw128(sbase + L::q_off + kk * 2048, L::kRows128, 1024);
+                        const uint64_t Ph = sdesc_sw128(sbase + L::p_off + kk * 2048, L::kRows128, 1024);
+                        const uint64_t Pl = sdesc_sw128(sbase + L::p_off + L::kRows128 + kk * 2048, L::kRows128, 1024);
+                        const uint64_t Sh = sdesc_sw128(sbase + L::ds_off + kk * 2048, L::kRows128, 1024);
+                        const uint64_t Sl = sdesc_sw128(sbase + L::ds_off + L::kRows128 + kk * 2048, L::kRows128, 1024);
+                        mma_ss(tmem + kColDV, dOt, Ph, id_kv, kk > 0);
+                        mma_ss(tmem + kColDV, dOt, Pl, id_kv, true);
+                        mma_ss(tmem + kColDK, Qt, Sh, id_kv, kk > 0);
+                        mma_ss(tmem + kColDK, Qt, Sl, id_kv, true);
+                    }
+                }
+                mma_commit(bar_mm2);
+                mma_commit(bar_empty(s));
+            }
+            if (!ok) s_abort = 1;
+            mma_commit(bar_final);
+            mbar_wait(bar_final, 0, kSiteFinal);
+        }
+    } else if (warp < 4) {
+        // ------------------------------------- P and dS rows, then dQ epilogue
+        const int r = threadIdx.x;                          // query row of the M-tile
+        const int i = r & 63, hp = r >> 6, head = head0 + hp;
+        const bool row_ok = head < a.G;
+        const int64_t row = (b * a.Hq + g * a.G + head) * a.T_seg + qb * 64 + i;
+        const float lse2 = row_ok ? a.lse[row] * kLog2e : 0.f;
+        const float Dr = row_ok ? a.Drow[row] : 0.f;
+        const uint32_t lane_off = uint32_t(warp * 32) << 16;
+        uint8_t* prow_hi = smem + L::p_off + r * 128;
+        uint8_t* prow_lo = prow_hi + L::kRows128;
+        uint8_t* srow_hi = smem + L::ds_off + r * 128;
+        uint8_t* srow_lo = srow_hi + L::kRows128;
+        bool ok = true;
+        for (int t = 0; t < nt && ok; ++t) {
+            const int bb = t & 1;
+            ok = mbar_wait(bar_sdp(bb), (t / 2) & 1, kSiteSdp);
+            if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[2][32], pr[2][32];
+            tmem_ld32(tmem + lane_off + kColS + bb * kKeys, sr[0]);
+            tmem_ld32(tmem + lane_off + kColS + bb * kKeys + 32, sr[1]);
+            tmem_ld32(tmem + lane_off + kColDP + bb * kKeys, pr[0]);
+            tmem_ld32(tmem + lane_off + kColDP + bb * kKeys + 32, pr[1]);
+            tmem_wait_ld();
+            const bool own = t == n_rt;
+            uint32_t ph[32], pl[32], dh[32], dl[32];
+#pragma unroll
+            for (int j2 = 0; j2 < 32; ++j2) {
+                float p[2], ds[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int j = 2 * j2 + e;
+                    const bool valid = row_ok && (own ? (j <= i) : (t * 8 + j / 8 < n_g));
+                    p[e] = valid ? exp2f(__uint_as_float(sr[j / 32][j % 32]) * a.scale_log2 - lse2) : 0.f;
+                    ds[e] = p[e] * (__uint_as_float(pr[j / 32][j % 32]) - Dr);
+                }
+                const __nv_bfloat162 hp2 = __floats2bfloat162_rn(p[0], p[1]);
+                const __nv_bfloat162 hd2 = __floats2bfloat162_rn(ds[0], ds[1]);
+                ph[j2] = *reinterpret_cast<const uint32_t*>(&hp2);
+                dh[j2] = *reinterpret_cast<const uint32_t*>(&hd2);
+                pl[j2] = pack_bf16x2(p[0] - __low2float(hp2), p[1] - __high2float(hp2));
+                dl[j2] = pack_bf16x2(ds[0] - __low2float(hd2), ds[1] - __high2float(hd2));
+            }
+            // The previous tile's MMAs read P / dS from shared memory.
+            if (t >= 1) {
+                ok = mbar_wait(bar_mm2, (t - 1) & 1, kSiteMm2);
+                if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
+            }
+            // Row r, 16-byte chunk c lives at chunk c ^ (r % 8) (128-byte swizzle).
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int pc = (c ^ (r & 7)) * 16;
+                *reinterpret_cast<uint4*>(prow_hi + pc) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+                *reinterpret_cast<uint4*>(prow_lo + pc) = make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+                *reinterpret_cast<uint4*>(srow_hi + pc) = make_uint4(dh[4 * c], dh[4 * c + 1], dh[4 * c + 2], dh[4 * c + 3]);
+                *reinterpret_cast<uint4*>(srow_lo + pc) = make_uint4(dl[4 * c], dl[4 * c + 1], dl[4 * c + 2], dl[4 * c + 3]);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_ps);
+        }
+        if (ok) {
+            ok = mbar_wait(bar_mm2, (nt - 1) & 1, kSiteMm2);
+            if (__any_sync(0xFFFFFFFFu, !ok)) ok = false;
+        }
+        if (ok) {
+            tc_fence_after();
+            float* dq = a.dQ + row * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + kColDQ + 32 * c, v);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(dq + 32 * c + j) =
+                            make_float4(__uint_as_float(v[j]) * a.scale, __uint_as_float(v[j + 1]) * a.scale,
+                                        __uint_as_float(v[j + 2]) * a.scale, __uint_as_float(v[j + 3]) * a.scale);
+                }
+            }
+        } else {
+            s_abort = 1;
+        }
+    } else {
+        // ------------------------------------------------- dK / dV epilogue
+        const int dd = (warp - 4) * 32 + lane;              // tensor-memory lane = d index
+        const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
+        bool ok = true;
+        for (int t = 0; t < nt && ok; ++t) {
+            ok = mbar_wait(bar_mm2, t & 1, kSiteMm2);
+            if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
+            if (tile_has_segment_keys(t, n_rt, n_g, grow, a.T_hist)) {
+                tc_fence_after();
+                uint32_t vv[2][32], kv[2][32];
+                tmem_ld32(tmem + lane_off + kColDV, vv[0]);
+                tmem_ld32(tmem + lane_off + kColDV + 32, vv[1]);
+                tmem_ld32(tmem + lane_off + kColDK, kv[0]);
+                tmem_ld32(tmem + lane_off + kColDK + 32, kv[1]);
+                tmem_wait_ld();
+                const bool own = t == n_rt;
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    int64_t key;
+                    if (own) {
+                        key = own_start + j;
+                    } else {
+                        const int gi = t * 8 + j / 8;
+                        key = gi < n_g ? (int64_t)grow[gi] * 8 + j % 8 : -1;
+                    }
+                    if (key < a.T_hist) continue;           // padding or detached history
+                    const int64_t o = (bg * a.T_seg + (key - a.T_hist)) * D + dd;
+                    atomicAdd(a.dV + o, __uint_as_float(vv[j / 32][j % 32]));
+                    atomicAdd(a.dK + o, __uint_as_float(kv[j / 32][j % 32]) * a.scale);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar_drained);
+        }
+        if (!ok) s_abort = 1;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (s_abort && warp == 8 && lane == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            int last = -1;
+            for (int t = s; t < nt; t += kStages) last = t;
+            if (last >= 0) mbar_wait(bar_full(s), (last / kStages) & 1, kSiteDrain);
+        }
+        mbar_wait(bar_q, 0, kSiteDrain);
+    }
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// D_row = sum_e dO[row][e] * O[row][e]: one warp per row, 16-byte loads of O
+// and 8-byte loads of dO.
+__global__ void __launch_bounds__(256)
+rowdot_kernel(const float* __restrict__ O, const __nv_bfloat16* __restrict__ dO, float* __restrict__ Drow,
+              int64_t rows)
+{
+    const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float4 o = __ldg(reinterpret_cast<const float4*>(O + row * D) + lane);
+    const uint2 w = __ldg(reinterpret_cast<const uint2*>(dO + row * D) + lane);
+    float acc = o.x * __uint_as_float(w.x << 16) + o.y * __uint_as_float(w.x & 0xFFFF0000u) +
+                o.z * __uint_as_float(w.y << 16) + o.w * __uint_as_float(w.y & 0xFFFF0000u);
+    acc = warp_sum(acc);
+    if (lane == 0) Drow[row] = acc;
+}
+
+}  // namespace
+
+int attn_bwd_tc_status(bool clear)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, sm100::g_status, sizeof v) != cudaSuccess) return -1;
+    if (clear && v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(sm100::g_status, &z, sizeof z);
+    }
+    return v;
+}
+
+bool attn_bwd_tc_supported(const Shape& s)
+{
+    const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
+    return s.dtype == HGA_BF16 && s.d == D && q_rows < (1ull << 31) && kv_rows < (1ull << 31) &&
+           tensor_maps_available();
+}
+
+cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, const void* V, const float* O,
+                               const float* lse, const void* dO, const int32_t* gidx, float* dQ,
+                               float* dK_seg, float* dV_seg, float* Drow, cudaStream_t st)
+{
+    const int64_t rows = (int64_t)s.B * s.Hq * s.T_seg;
+    rowdot_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, static_cast<const __nv_bfloat16*>(dO), Drow, rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t seg_bytes = sizeof(float) * (size_t)s.B * s.Hkv * s.T_seg * D;
+    if ((e = cudaMemsetAsync(dK_seg, 0, seg_bytes, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dV_seg, 0, seg_bytes, st)) != cudaSuccess) return e;
+    CUtensorMap tq, tdo, tk8, tv8, tk64, tv64;
+    const uint64_t q_rows = (uint64_t)rows, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
+    if (!make_bf16_map(&tq, Q, q_rows, D, 64) || !make_bf16_map(&tdo, dO, q_rows, D, 64) ||
+        !make_bf16_map(&tk8, K, kv_rows, D, 8) || !make_bf16_map(&tv8, V, kv_rows, D, 8) ||
+        !make_bf16_map(&tk64, K, kv_rows, D, 64) || !make_bf16_map(&tv64, V, kv_rows, D, 64))
+        return cudaErrorInvalidValue;
+    BwdArgs a;
+    a.gidx = gidx;
+    a.lse = lse;
+    a.Drow = Drow;
+    a.dQ = dQ;
+    a.dK = dK_seg;
+    a.dV = dV_seg;
+    a.Hq = s.Hq;
+    a.Hkv = s.Hkv;
+    a.G = s.G;
+    a.wg = s.wg;
+    a.T_hist = s.T_hist;
+    a.T_seg = s.T_seg;
+    a.nQB = s.nQB;
+    a.q_rows = (int)q_rows;
+    a.scale = s.scale;
+    a.scale_log2 = s.scale * kLog2e;
+    const int smem = BwdSmem::alloc;
+    if ((e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+        return e;
+    const dim3 grid((unsigned)(s.B * s.Hkv * s.nQB), (unsigned)((s.G + 1) / 2));
+    attn_bwd_tc_kernel<<<grid, kThreads, smem, st>>>(tq, tdo, tk8, tv8, tk64, tv64, a);
+    return cudaGetLastError();
+}
+
+}  // namespace hga

@@ -24,8 +24,6 @@
 // Tensor memory (512 columns): O of each M-tile (D columns), and two S/P
 // buffers of 64 columns per M-tile so that S of the next key tile is computed
 // while the softmax works on the current one.
-#include <cudaTypedefs.h>
-
 #include "hga_internal.cuh"
 #include "sm100.cuh"
 
@@ -352,43 +350,15 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 }
 
 // ---- host side -------------------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void* p = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// 2-D bf16 map over `rows` rows of `cols` elements, box of 64 columns x box_rows
-// rows, 128-byte swizzle (the layout the MMA descriptors above expect).
-bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows)
-{
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
 cudaError_t launch(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* gidx,
                    float* O, float* lse, cudaStream_t st)
 {
     CUtensorMap tq, tk8, tv8, tk64, tv64;
     const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
-    if (!make_map(&tq, Q, q_rows, D, 64) || !make_map(&tk8, K, kv_rows, D, 8) ||
-        !make_map(&tv8, V, kv_rows, D, 8) || !make_map(&tk64, K, kv_rows, D, 64) ||
-        !make_map(&tv64, V, kv_rows, D, 64))
+    if (!make_bf16_map(&tq, Q, q_rows, D, 64) || !make_bf16_map(&tk8, K, kv_rows, D, 8) ||
+        !make_bf16_map(&tv8, V, kv_rows, D, 8) || !make_bf16_map(&tk64, K, kv_rows, D, 64) ||
+        !make_bf16_map(&tv64, V, kv_rows, D, 64))
         return cudaErrorInvalidValue;
     FwdArgs a;
     a.gidx = gidx;
@@ -430,7 +400,7 @@ bool attn_fwd_tc_supported(const Shape& s)
 {
     const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
     return s.dtype == HGA_BF16 && (s.d == 128 || s.d == 64) && q_rows < (1ull << 31) &&
-           kv_rows < (1ull << 31) && encode_fn() != nullptr;
+           kv_rows < (1ull << 31) && tensor_maps_available();
 }
 
 cudaError_t launch_attn_fwd_tc(const Shape& s, const void* Q, const void* K, const void* V,

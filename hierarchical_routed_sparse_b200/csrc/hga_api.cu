@@ -90,6 +90,17 @@ int make_shape(const hga_params* p, hga::Shape* s)
 }
 
 
+// The backward kernels: bf16 with d = 128 on the tensor cores, everything
+// else on the FMA kernel.  Drow is the B*Hq*T_seg-float row-sum scratch.
+cudaError_t run_attn_bwd(const hga::Shape& s, const void* Q, const void* K, const void* V, const float* O,
+                         const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK_seg,
+                         float* dV_seg, float* Drow, cudaStream_t st)
+{
+    if (hga::attn_bwd_tc_supported(s))
+        return hga::launch_attn_bwd_tc(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, Drow, st);
+    return hga::launch_attn_bwd_simt(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, Drow, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -101,9 +112,10 @@ const char* hga_version(void) { return "hga-b200 0.1 (sm_100a)"; }
 int hga_device_status(int* status, int clear)
 {
     if (!status) return fail(HGA_ERR_INVALID_ARG, "status is NULL");
-    const int v = hga::attn_fwd_tc_status(clear != 0);
-    if (v < 0) return fail(HGA_ERR_CUDA, "hga_device_status: the status word could not be read");
-    *status = v;
+    const int vf = hga::attn_fwd_tc_status(clear != 0);
+    const int vb = hga::attn_bwd_tc_status(clear != 0);
+    if (vf < 0 || vb < 0) return fail(HGA_ERR_CUDA, "hga_device_status: the status word could not be read");
+    *status = vf ? vf : vb;
     return HGA_OK;
 }
 
@@ -186,7 +198,7 @@ int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* 
     CHECK_PTR(gidx);
     CHECK_PTR(O);
     CHECK_PTR(lse);
-    if (hga::attn_simt_smem(s, false) > kMaxSmem)
+    if (!hga::attn_fwd_tc_supported(s) && hga::attn_simt_smem(s, false) > kMaxSmem)
         return fail(HGA_ERR_UNSUPPORTED, "k_g=%d too large for the attention kernel", s.wg);
     // bf16: tcgen05 tensor-core kernel; float32: the FMA kernel (1e-4 gate).
     cudaError_t e = hga::attn_fwd_tc_supported(s)
@@ -216,11 +228,10 @@ int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* 
     const size_t need = sizeof(float) * (size_t)s.B * s.Hq * s.T_seg;
     if (ws_bytes < need)
         return fail(HGA_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, need);
-    if (hga::attn_simt_smem(s, true) > kMaxSmem)
+    if (!hga::attn_bwd_tc_supported(s) && hga::attn_simt_smem(s, true) > kMaxSmem)
         return fail(HGA_ERR_UNSUPPORTED, "k_g=%d too large for the attention kernel", s.wg);
-    cudaError_t e = hga::launch_attn_bwd_simt(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg,
-                                              static_cast<float*>(workspace),
-                                              static_cast<cudaStream_t>(stream));
+    cudaError_t e = run_attn_bwd(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, static_cast<float*>(workspace),
+                                 static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_bwd");
 }
 
@@ -294,13 +305,13 @@ extern "C" int hga_attn_bwd_noalloc(const hga_params* p, const void* Q, const vo
                     "hga_attn_bwd_noalloc: B*Hq*T_seg = %lld exceeds its built-in scratch of %d rows; "
                     "use hga_attn_bwd with a caller-provided workspace", (long long)rows,
                     HGA_NOALLOC_MAX_ROWS);
-    if (hga::attn_simt_smem(s, true) > kMaxSmem)
+    if (!hga::attn_bwd_tc_supported(s) && hga::attn_simt_smem(s, true) > kMaxSmem)
         return fail(HGA_ERR_UNSUPPORTED, "k_g=%d too large for the attention kernel", s.wg);
     float* scratch = nullptr;
     if (int r = noalloc_scratch(&scratch)) return r;
     // Every row sum the kernels read is first written by this call, so the
     // scratch needs no clearing between calls.
-    cudaError_t e = hga::launch_attn_bwd_simt(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, scratch,
-                                              static_cast<cudaStream_t>(stream));
+    cudaError_t e = run_attn_bwd(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, scratch,
+                                 static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_bwd_noalloc");
 }

@@ -2,6 +2,7 @@
 // translation units of libhga.so.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -90,6 +91,10 @@ cudaError_t launch_attn_bwd_simt(const Shape& s, const void* Q, const void* K, c
                                  const int32_t* gidx, float* dQ, float* dK_seg, float* dV_seg,
                                  float* Drow, cudaStream_t st);
 
+// TMA tensor maps (tma_map.cu).
+bool tensor_maps_available();
+bool make_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
 // Tensor-core (tcgen05) path for bf16 inputs.
 bool attn_fwd_tc_supported(const Shape& s);
 cudaError_t launch_attn_fwd_tc(const Shape& s, const void* Q, const void* K, const void* V,
@@ -97,5 +102,11 @@ cudaError_t launch_attn_fwd_tc(const Shape& s, const void* Q, const void* K, con
 // Status word of the tensor-core kernels' bounded waits (0 = none ran out;
 // -1 = could not be read).  Synchronises with the device.
 int attn_fwd_tc_status(bool clear);
+bool attn_bwd_tc_supported(const Shape& s);
+cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, const void* V,
+                               const float* O, const float* lse, const void* dO,
+                               const int32_t* gidx, float* dQ, float* dK_seg, float* dV_seg,
+                               float* Drow, cudaStream_t st);
+int attn_bwd_tc_status(bool clear);
 
 }  // namespace hga
