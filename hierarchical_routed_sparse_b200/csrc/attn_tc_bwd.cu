@@ -13,7 +13,7 @@
 // own chunk with the causal mask):
 //     S   = Q K^T, dP = dO V^T        tcgen05.mma -> tensor memory
 //     P   = exp2(S*c - lse), dS = P (dP - D)   row per thread; both written
-//           to shared memory as bf16 hi + lo parts (~16-bit operands)
+//           to shared memory as bf16 hi + lo parts (~14-bit operands)
 //     dQ += dS K                      A = dS (K-major), B = K (MN-major)
 //     dV^T = dO^T P, dK^T = Q^T dS    A = dO / Q read MN-major, B = P / dS
 // dV^T and dK^T (d on the tensor-memory lanes, keys on the columns) are added
@@ -21,8 +21,9 @@
 // atomics; tiles whose keys are all detached history skip both products
 // (routed groups are ascending, so history tiles come first).
 //
-// Warp roles (320 threads): warps 0-3 softmax-gradient rows and the dQ
-// epilogue, warps 4-7 the dK/dV epilogue, warp 8 TMA producer, warp 9
+// Warp roles (320 threads): warps 0-7 compute P and dS (row 32*(w%4)+lane,
+// key half w/4), add the previous tile's dK/dV while the MMAs of the current
+// one run, and write dQ at the end; warp 8 is the TMA producer, warp 9 the
 // tensor-memory owner and MMA issuer.  Tensor memory (512 columns): S and dP
 // double-buffered (4 x 64), dQ (128), dV^T (64), dK^T (64).
 #include "hga_internal.cuh"
@@ -77,14 +78,6 @@ struct BwdArgs {
     float scale, scale_log2;
 };
 
-// Routed groups form an ascending prefix of the index row.
-__device__ __forceinline__ int count_groups(const int32_t* grow, int wg)
-{
-    int n = 0;
-    while (n < wg && grow[n] >= 0) ++n;
-    return n;
-}
-
 // Does key tile t hold any segment token (position >= T_hist)?
 __device__ __forceinline__ bool tile_has_segment_keys(int t, int n_rt, int n_g, const int32_t* grow,
                                                       int64_t T_hist)
@@ -126,9 +119,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int64_t own_start = a.T_hist + qb * 64;
 
     const int32_t* grow = a.gidx + u * a.wg;
-    const int n_g = count_groups(grow, a.wg);
-    const int n_rt = (n_g + 7) / 8;
-    const int nt = n_rt + 1;
+    __shared__ int s_ng;
+    if (threadIdx.x == 0) s_ng = 0;
+    __syncthreads();
+    {
+        int c = 0;
+        for (int i = threadIdx.x; i < a.wg; i += kThreads) c += grow[i] >= 0;
+        c = __reduce_add_sync(0xFFFFFFFFu, c);
+        if (lane == 0 && c) atomicAdd(&s_ng, c);
+    }
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -139,9 +138,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         mbar_init(bar_sdp(0), 1);
         mbar_init(bar_sdp(1), 1);
-        mbar_init(bar_ps, 128);
+        mbar_init(bar_ps, 256);
         mbar_init(bar_mm2, 1);
-        mbar_init(bar_drained, 128);
+        mbar_init(bar_drained, 256);
         mbar_init(bar_final, 1);
         fence_mbar_init();
     }
@@ -150,6 +149,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const int n_g = s_ng;                                   // routed groups (an ascending prefix)
+    const int n_rt = (n_g + 7) / 8;
+    const int nt = n_rt + 1;
 
     if (warp == 8) {
         // ------------------------------------------------------------ producer
@@ -170,33 +172,38 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tma_load_2d(sbase + L::do_off + off, &tm_do, 64 * c, y, bar_q);
                 }
             }
-            for (int t = 0; t < nt; ++t) {
-                const int s = t % kStages, r = t / kStages;
-                if (t >= kStages && !mbar_wait(bar_empty(s), (r - 1) & 1, kSiteEmpty)) {
-                    s_abort = 1;
-                    break;
-                }
-                mbar_expect_tx(bar_full(s), 2 * H * kKeys * 128);
-                const uint32_t kdst = sbase + L::k_off + s * H * L::kKVHalf;
-                const uint32_t vdst = sbase + L::v_off + s * H * L::kKVHalf;
-                if (t < n_rt) {
-                    for (int j = 0; j < 8; ++j) {
-                        const int gi = t * 8 + j;
-                        const int grp = grow[gi < n_g ? gi : 0];
-                        const int y = int(kv_base + (int64_t)grp * 8);
-                        for (int c = 0; c < H; ++c) {
-                            tma_load_2d(kdst + c * L::kKVHalf + j * 1024, &tm_k8, 64 * c, y, bar_full(s));
-                            tma_load_2d(vdst + c * L::kKVHalf + j * 1024, &tm_v8, 64 * c, y, bar_full(s));
-                        }
-                    }
-                } else {
-                    const int y = int(kv_base + own_start);
+        }
+        for (int t = 0; t < nt; ++t) {
+            const int s = t % kStages, r = t / kStages;
+            bool ok = true;
+            if (lane == 0) {
+                ok = t < kStages || mbar_wait(bar_empty(s), (r - 1) & 1, kSiteEmpty);
+                if (ok) mbar_expect_tx(bar_full(s), 2 * H * kKeys * 128);
+            }
+            if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+                s_abort = 1;
+                break;
+            }
+            const uint32_t kdst = sbase + L::k_off + s * H * L::kKVHalf;
+            const uint32_t vdst = sbase + L::v_off + s * H * L::kKVHalf;
+            if (t < n_rt) {
+                if (lane < 8) {                               // one group per lane
+                    const int gi = t * 8 + lane;
+                    const int grp = __ldg(grow + (gi < n_g ? gi : 0));
+                    const int y = int(kv_base + (int64_t)grp * 8);
                     for (int c = 0; c < H; ++c) {
-                        tma_load_2d(kdst + c * L::kKVHalf, &tm_k64, 64 * c, y, bar_full(s));
-                        tma_load_2d(vdst + c * L::kKVHalf, &tm_v64, 64 * c, y, bar_full(s));
+                        tma_load_2d(kdst + c * L::kKVHalf + lane * 1024, &tm_k8, 64 * c, y, bar_full(s));
+                        tma_load_2d(vdst + c * L::kKVHalf + lane * 1024, &tm_v8, 64 * c, y, bar_full(s));
                     }
+                }
+            } else if (lane == 0) {
+                const int y = int(kv_base + own_start);
+                for (int c = 0; c < H; ++c) {
+                    tma_load_2d(kdst + c * L::kKVHalf, &tm_k64, 64 * c, y, bar_full(s));
+                    tma_load_2d(vdst + c * L::kKVHalf, &tm_v64, 64 * c, y, bar_full(s));
                 }
             }
+            __syncwarp();
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
@@ -258,49 +265,72 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mma_commit(bar_final);
             mbar_wait(bar_final, 0, kSiteFinal);
         }
-    } else if (warp < 4) {
-        // ------------------------------------- P and dS rows, then dQ epilogue
-        const int r = threadIdx.x;                          // query row of the M-tile
+    } else {
+        // ------------- P and dS, then the dK / dV atomics and the dQ epilogue
+        // Thread (warp w, lane l): query row r = 32*(w%4) + l of the M-tile
+        // (its tensor-memory lane) and the 32-key half kh = w/4 of each tile.
+        const int r = (warp % 4) * 32 + lane, kh = warp / 4;
         const int i = r & 63, hp = r >> 6, head = head0 + hp;
         const bool row_ok = head < a.G;
         const int64_t row = (b * a.Hq + g * a.G + head) * a.T_seg + qb * 64 + i;
         const float lse2 = row_ok ? a.lse[row] * kLog2e : 0.f;
         const float Dr = row_ok ? a.Drow[row] : 0.f;
-        const uint32_t lane_off = uint32_t(warp * 32) << 16;
+        const uint32_t lane_off = uint32_t((warp % 4) * 32) << 16;
         uint8_t* prow_hi = smem + L::p_off + r * 128;
         uint8_t* prow_lo = prow_hi + L::kRows128;
         uint8_t* srow_hi = smem + L::ds_off + r * 128;
         uint8_t* srow_lo = srow_hi + L::kRows128;
+        // dV^T / dK^T of tile te (d = tensor-memory lane r, keys of half kh)
+        // added to the segment's rows; history keys and padding are skipped.
+        auto dkv_epilogue = [&](int te) {
+            if (!tile_has_segment_keys(te, n_rt, n_g, grow, a.T_hist)) return;
+            tc_fence_after();
+            uint32_t vv[32], kv[32];
+            tmem_ld32(tmem + lane_off + kColDV + 32 * kh, vv);
+            tmem_ld32(tmem + lane_off + kColDK + 32 * kh, kv);
+            tmem_wait_ld();
+            const bool own = te == n_rt;
+            int64_t gbase[4];                               // first token of each group slot
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int gi = te * 8 + 4 * kh + q;
+                gbase[q] = own ? own_start + 32 * kh + 8 * q : (gi < n_g ? (int64_t)__ldg(grow + gi) * 8 : -64);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int64_t key = gbase[j / 8] + j % 8;
+                if (key < a.T_hist) continue;               // padding or detached history
+                const int64_t o = (bg * a.T_seg + (key - a.T_hist)) * D + r;
+                atomicAdd(a.dV + o, __uint_as_float(vv[j]));
+                atomicAdd(a.dK + o, __uint_as_float(kv[j]) * a.scale);
+            }
+        };
         bool ok = true;
         for (int t = 0; t < nt && ok; ++t) {
             const int bb = t & 1;
             ok = mbar_wait(bar_sdp(bb), (t / 2) & 1, kSiteSdp);
             if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
             tc_fence_after();
-            uint32_t sr[2][32], pr[2][32];
-            tmem_ld32(tmem + lane_off + kColS + bb * kKeys, sr[0]);
-            tmem_ld32(tmem + lane_off + kColS + bb * kKeys + 32, sr[1]);
-            tmem_ld32(tmem + lane_off + kColDP + bb * kKeys, pr[0]);
-            tmem_ld32(tmem + lane_off + kColDP + bb * kKeys + 32, pr[1]);
-            tmem_wait_ld();
             const bool own = t == n_rt;
-            uint32_t ph[32], pl[32], dh[32], dl[32];
+            // P is an MMA operand only for dV, i.e. for tiles holding segment keys.
+            const bool seg = tile_has_segment_keys(t, n_rt, n_g, grow, a.T_hist);
+            uint32_t sr[32], pr[32];
+            tmem_ld32(tmem + lane_off + kColS + bb * kKeys + 32 * kh, sr);
+            tmem_ld32(tmem + lane_off + kColDP + bb * kKeys + 32 * kh, pr);
+            tmem_wait_ld();
+            uint32_t ph[16], pl[16], dh[16], dl[16];
 #pragma unroll
-            for (int j2 = 0; j2 < 32; ++j2) {
+            for (int j2 = 0; j2 < 16; ++j2) {
                 float p[2], ds[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const int j = 2 * j2 + e;
+                    const int jj = 2 * j2 + e, j = 32 * kh + jj;
                     const bool valid = row_ok && (own ? (j <= i) : (t * 8 + j / 8 < n_g));
-                    p[e] = valid ? exp2f(__uint_as_float(sr[j / 32][j % 32]) * a.scale_log2 - lse2) : 0.f;
-                    ds[e] = p[e] * (__uint_as_float(pr[j / 32][j % 32]) - Dr);
+                    p[e] = valid ? fast_exp2(fmaf(__uint_as_float(sr[jj]), a.scale_log2, -lse2)) : 0.f;
+                    ds[e] = p[e] * (__uint_as_float(pr[jj]) - Dr);
                 }
-                const __nv_bfloat162 hp2 = __floats2bfloat162_rn(p[0], p[1]);
-                const __nv_bfloat162 hd2 = __floats2bfloat162_rn(ds[0], ds[1]);
-                ph[j2] = *reinterpret_cast<const uint32_t*>(&hp2);
-                dh[j2] = *reinterpret_cast<const uint32_t*>(&hd2);
-                pl[j2] = pack_bf16x2(p[0] - __low2float(hp2), p[1] - __high2float(hp2));
-                dl[j2] = pack_bf16x2(ds[0] - __low2float(hd2), ds[1] - __high2float(hd2));
+                split_bf16x2(ds[0], ds[1], dh[j2], dl[j2]);
+                if (seg) split_bf16x2(p[0], p[1], ph[j2], pl[j2]);
             }
             // The previous tile's MMAs read P / dS from shared memory.
             if (t >= 1) {
@@ -309,28 +339,37 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             // Row r, 16-byte chunk c lives at chunk c ^ (r % 8) (128-byte swizzle).
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int pc = (c ^ (r & 7)) * 16;
-                *reinterpret_cast<uint4*>(prow_hi + pc) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
-                *reinterpret_cast<uint4*>(prow_lo + pc) = make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
-                *reinterpret_cast<uint4*>(srow_hi + pc) = make_uint4(dh[4 * c], dh[4 * c + 1], dh[4 * c + 2], dh[4 * c + 3]);
-                *reinterpret_cast<uint4*>(srow_lo + pc) = make_uint4(dl[4 * c], dl[4 * c + 1], dl[4 * c + 2], dl[4 * c + 3]);
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const int pc = ((4 * kh + c4) ^ (r & 7)) * 16;
+                *reinterpret_cast<uint4*>(srow_hi + pc) = make_uint4(dh[4 * c4], dh[4 * c4 + 1], dh[4 * c4 + 2], dh[4 * c4 + 3]);
+                *reinterpret_cast<uint4*>(srow_lo + pc) = make_uint4(dl[4 * c4], dl[4 * c4 + 1], dl[4 * c4 + 2], dl[4 * c4 + 3]);
+                if (seg) {
+                    *reinterpret_cast<uint4*>(prow_hi + pc) = make_uint4(ph[4 * c4], ph[4 * c4 + 1], ph[4 * c4 + 2], ph[4 * c4 + 3]);
+                    *reinterpret_cast<uint4*>(prow_lo + pc) = make_uint4(pl[4 * c4], pl[4 * c4 + 1], pl[4 * c4 + 2], pl[4 * c4 + 3]);
+                }
             }
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(bar_ps);
+            // While the MMAs of tile t run: the dK / dV of tile t-1.
+            if (t >= 1) {
+                dkv_epilogue(t - 1);
+                tc_fence_before();
+                mbar_arrive(bar_drained);
+            }
         }
         if (ok) {
             ok = mbar_wait(bar_mm2, (nt - 1) & 1, kSiteMm2);
             if (__any_sync(0xFFFFFFFFu, !ok)) ok = false;
         }
         if (ok) {
+            dkv_epilogue(nt - 1);
             tc_fence_after();
-            float* dq = a.dQ + row * D;
+            float* dq = a.dQ + row * D + 64 * kh;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t v[32];
-                tmem_ld32(tmem + lane_off + kColDQ + 32 * c, v);
+                tmem_ld32(tmem + lane_off + kColDQ + 64 * kh + 32 * c, v);
                 tmem_wait_ld();
                 if (row_ok) {
 #pragma unroll
@@ -343,42 +382,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         } else {
             s_abort = 1;
         }
-    } else {
-        // ------------------------------------------------- dK / dV epilogue
-        const int dd = (warp - 4) * 32 + lane;              // tensor-memory lane = d index
-        const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
-        bool ok = true;
-        for (int t = 0; t < nt && ok; ++t) {
-            ok = mbar_wait(bar_mm2, t & 1, kSiteMm2);
-            if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
-            if (tile_has_segment_keys(t, n_rt, n_g, grow, a.T_hist)) {
-                tc_fence_after();
-                uint32_t vv[2][32], kv[2][32];
-                tmem_ld32(tmem + lane_off + kColDV, vv[0]);
-                tmem_ld32(tmem + lane_off + kColDV + 32, vv[1]);
-                tmem_ld32(tmem + lane_off + kColDK, kv[0]);
-                tmem_ld32(tmem + lane_off + kColDK + 32, kv[1]);
-                tmem_wait_ld();
-                const bool own = t == n_rt;
-#pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    int64_t key;
-                    if (own) {
-                        key = own_start + j;
-                    } else {
-                        const int gi = t * 8 + j / 8;
-                        key = gi < n_g ? (int64_t)grow[gi] * 8 + j % 8 : -1;
-                    }
-                    if (key < a.T_hist) continue;           // padding or detached history
-                    const int64_t o = (bg * a.T_seg + (key - a.T_hist)) * D + dd;
-                    atomicAdd(a.dV + o, __uint_as_float(vv[j / 32][j % 32]));
-                    atomicAdd(a.dK + o, __uint_as_float(kv[j / 32][j % 32]) * a.scale);
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(bar_drained);
-        }
-        if (!ok) s_abort = 1;
     }
 
     tc_fence_before();

@@ -13,7 +13,7 @@
 // or the own chunk (one box).  Per key tile and M-tile:
 //     S  = Q K^T            tcgen05.mma  A = Q (smem), B = K (smem) -> TMEM
 //     P  = exp2(S*c - m)    softmax warpgroup, row per thread, P -> TMEM as
-//                           two bf16 parts hi + lo (P to ~16 bits)
+//                           two bf16 parts hi + lo (P to ~14 bits)
 //     O += P V              tcgen05.mma  A = P hi, P lo (TMEM), B = V (smem)
 // The running maximum is only moved when a row's maximum grows by more than
 // 2^8 (then O is rescaled in TMEM); any fixed reference point gives the same
@@ -103,14 +103,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int n_mt = (n_heads + 1) / 2;
 
     const int32_t* grow = a.gidx + u * a.wg;
-    // Routed groups form a prefix of the row.
-    int n_g = 0;
-    for (int i = 0; i < a.wg; ++i) {
-        if (grow[i] < 0) break;
-        ++n_g;
+    __shared__ int s_ng;
+    if (threadIdx.x == 0) s_ng = 0;
+    __syncthreads();
+    // Routed groups form a prefix of the row: count them with one parallel pass.
+    {
+        int c = 0;
+        for (int i = threadIdx.x; i < a.wg; i += kThreads) c += grow[i] >= 0;
+        c = __reduce_add_sync(0xFFFFFFFFu, c);
+        if (lane == 0 && c) atomicAdd(&s_ng, c);
     }
-    const int n_rt = (n_g + 7) / 8;
-    const int nt = n_rt + 1;                                // + own chunk tile
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -133,6 +135,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const int n_g = s_ng;
+    const int n_rt = (n_g + 7) / 8;
+    const int nt = n_rt + 1;                                // + own chunk tile
     // Column map: O[m] at m*D, S/P[m][b] at 2*D + (2*m + b)*64.
     auto col_o = [&](int m) { return uint32_t(m * D); };
     auto col_s = [&](int m, int bb) { return uint32_t(2 * D + (2 * m + bb) * kKeys); };
@@ -141,6 +146,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     if (warp == 8) {
         // ------------------------------------------------------------ producer
+        // Lane 0 issues the Q boxes and arms the barriers; for a routed tile,
+        // lane j < 8 fetches group j's index and issues that group's boxes,
+        // so the eight index loads overlap.
         if (lane == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k8);
@@ -156,35 +164,40 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tma_load_2d(sbase + L::q_off + ((hh / 2) * H + c) * L::kQTile + (hh % 2) * 64 * 128,
                                 &tm_q, 64 * c, y, bar_q);
             }
-            for (int t = 0; t < nt; ++t) {
-                const int s = t % kStages, r = t / kStages;
-                if (t >= kStages && !mbar_wait(bar_empty(s), (r - 1) & 1, kSiteEmpty)) {
-                    s_abort = 1;
-                    break;
-                }
-                mbar_expect_tx(bar_full(s), 2 * H * kKeys * 128);
-                const uint32_t kdst = sbase + L::k_off + s * H * L::kKVHalf;
-                const uint32_t vdst = sbase + L::v_off + s * H * L::kKVHalf;
-                if (t < n_rt) {
-                    for (int j = 0; j < 8; ++j) {
-                        const int gi = t * 8 + j;
-                        // Slots past the last routed group repeat group 0: finite
-                        // data whose scores the softmax masks out.
-                        const int grp = grow[gi < n_g ? gi : 0];
-                        const int y = int(kv_base + (int64_t)grp * 8);
-                        for (int c = 0; c < H; ++c) {
-                            tma_load_2d(kdst + c * L::kKVHalf + j * 1024, &tm_k8, 64 * c, y, bar_full(s));
-                            tma_load_2d(vdst + c * L::kKVHalf + j * 1024, &tm_v8, 64 * c, y, bar_full(s));
-                        }
-                    }
-                } else {
-                    const int y = int(kv_base + a.T_hist + qb * 64);
+        }
+        for (int t = 0; t < nt; ++t) {
+            const int s = t % kStages, r = t / kStages;
+            bool ok = true;
+            if (lane == 0) {
+                ok = t < kStages || mbar_wait(bar_empty(s), (r - 1) & 1, kSiteEmpty);
+                if (ok) mbar_expect_tx(bar_full(s), 2 * H * kKeys * 128);
+            }
+            if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+                s_abort = 1;
+                break;
+            }
+            const uint32_t kdst = sbase + L::k_off + s * H * L::kKVHalf;
+            const uint32_t vdst = sbase + L::v_off + s * H * L::kKVHalf;
+            if (t < n_rt) {
+                if (lane < 8) {
+                    const int gi = t * 8 + lane;
+                    // Slots past the last routed group repeat group 0: finite
+                    // data whose scores the softmax masks out.
+                    const int grp = __ldg(grow + (gi < n_g ? gi : 0));
+                    const int y = int(kv_base + (int64_t)grp * 8);
                     for (int c = 0; c < H; ++c) {
-                        tma_load_2d(kdst + c * L::kKVHalf, &tm_k64, 64 * c, y, bar_full(s));
-                        tma_load_2d(vdst + c * L::kKVHalf, &tm_v64, 64 * c, y, bar_full(s));
+                        tma_load_2d(kdst + c * L::kKVHalf + lane * 1024, &tm_k8, 64 * c, y, bar_full(s));
+                        tma_load_2d(vdst + c * L::kKVHalf + lane * 1024, &tm_v8, 64 * c, y, bar_full(s));
                     }
+                }
+            } else if (lane == 0) {
+                const int y = int(kv_base + a.T_hist + qb * 64);
+                for (int c = 0; c < H; ++c) {
+                    tma_load_2d(kdst + c * L::kKVHalf, &tm_k64, 64 * c, y, bar_full(s));
+                    tma_load_2d(vdst + c * L::kKVHalf, &tm_v64, 64 * c, y, bar_full(s));
                 }
             }
+            __syncwarp();
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
@@ -263,7 +276,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const bool need = mx > m_run + kRescaleLog2;
             if (__any_sync(0xFFFFFFFFu, need)) {
                 const float m_new = need ? mx : m_run;
-                const float alpha = exp2f(m_run - m_new);      // 0 when m_run = -inf
+                const float alpha = fast_exp2(m_run - m_new);  // 0 when m_run = -inf
                 if (t > 0) {
                     ok = mbar_wait(bar_o(m, (t - 1) & 1), ((t - 1) / 2) & 1, kSiteO);
                     if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
@@ -282,17 +295,15 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 l_run *= alpha;
                 m_run = m_new;
             }
-            // P = hi + lo, both bf16: the two MMAs carry P to ~16 bits, where
+            // P = hi + lo, both bf16: the two MMAs carry P to ~14 bits, where
             // one bf16 operand alone (8 bits) misses the 2e-3 output bound.
             uint32_t pk_hi[32], pk_lo[32];
             float rs = 0.f;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float p0 = exp2f(sv[2 * j] - m_run), p1 = exp2f(sv[2 * j + 1] - m_run);
+                const float p0 = fast_exp2(sv[2 * j] - m_run), p1 = fast_exp2(sv[2 * j + 1] - m_run);
                 rs += p0 + p1;
-                const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                pk_hi[j] = *reinterpret_cast<const uint32_t*>(&h);
-                pk_lo[j] = pack_bf16x2(p0 - __low2float(h), p1 - __high2float(h));
+                split_bf16x2(p0, p1, pk_hi[j], pk_lo[j]);
             }
             l_run += rs;
             tmem_st32(tmem + lane_off + col_s(m, bb), pk_hi);

@@ -59,27 +59,32 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
                  : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
+// Test the phase; if it is not complete the thread may sleep in hardware
+// until it completes or `hint_ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity, uint32_t hint_ns)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }
 
-// Wait for the phase of parity `parity` to complete.  Gives up after
-// kWaitLimitNs, records `site` in g_status and returns false.
+// Wait for the phase of parity `parity` to complete.  The waiting warp sleeps
+// in hardware (no spinning on issue slots); the time bound is checked between
+// sleeps.  Gives up after kWaitLimitNs, records `site` in g_status and
+// returns false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int site)
 {
-    if (mbar_try(bar, parity)) return true;
+    constexpr uint32_t kHintNs = 100000;                 // 0.1 ms per sleep
+    if (mbar_try(bar, parity, kHintNs)) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
-        if (mbar_try(bar, parity)) return true;
+        if (mbar_try(bar, parity, kHintNs)) return true;
         if (global_ns() - t0 > kWaitLimitNs) {
             atomicCAS(&g_status, 0, site);
             return false;
@@ -209,6 +214,28 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
+}
+
+// 2^x by the MUFU.EX2 instruction (ex2.approx.ftz.f32): relative error about
+// 2^-22, far below the ~2^-16 at which the softmax weights enter the MMAs.
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Split two floats into bf16 parts x = hi + lo: hi is x truncated to bf16
+// (the top 16 bits), lo the exact fp32 remainder truncated to bf16, so that
+// hi + lo carries x to about 2^-14 relative.  Integer ops only (no float to
+// bf16 conversion instructions).  Element 0 goes to the low half of each word.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo)
+{
+    const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
+    hi = __byte_perm(b0, b1, 0x7632);
+    const float r0 = x0 - __uint_as_float(b0 & 0xFFFF0000u);
+    const float r1 = x1 - __uint_as_float(b1 & 0xFFFF0000u);
+    lo = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
