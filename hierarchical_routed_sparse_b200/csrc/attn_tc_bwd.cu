@@ -25,7 +25,9 @@
 // key half w/4), add the previous tile's dK/dV while the MMAs of the current
 // one run, and write dQ at the end; warp 8 is the TMA producer, warp 9 the
 // tensor-memory owner and MMA issuer.  Tensor memory (512 columns): S and dP
-// double-buffered (4 x 64), dQ (128), dV^T (64), dK^T (64).
+// double-buffered (4 x 64), dQ (128), dV^T (64), dK^T (64).  Three K/V
+// stages (224 KB of shared memory in all) keep the gathered loads two tiles
+// ahead of the MMAs.
 #include "hga_internal.cuh"
 #include "sm100.cuh"
 
@@ -36,7 +38,7 @@ using namespace sm100;
 
 constexpr int D = 128;
 constexpr int H = 2;                  // 64-column halves of d
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kKeys = 64;
 constexpr int kThreads = 320;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -227,9 +229,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 mma_commit(bar_sdp(bb));
                 return true;
             };
+            // S / dP run two tiles ahead (double-buffered): S(t+2) is issued
+            // right after the MMAs of tile t, so that its load wait never
+            // holds back the gradient MMAs of the tile the softmax finished.
             if (ok) ok = issue_sdp(0);
+            if (ok && nt > 1) ok = issue_sdp(1);
             for (int t = 0; ok && t < nt; ++t) {
-                if (t + 1 < nt && !(ok = issue_sdp(t + 1))) break;
                 const int s = t % kStages;
                 if (!(ok = mbar_wait(bar_ps, t & 1, kSitePs))) break;
                 tc_fence_after();
@@ -260,6 +265,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 mma_commit(bar_mm2);
                 mma_commit(bar_empty(s));
+                if (t + 2 < nt && !(ok = issue_sdp(t + 2))) break;
             }
             if (!ok) s_abort = 1;
             mma_commit(bar_final);
