@@ -28,6 +28,8 @@
 // double-buffered (4 x 64), dQ (128), dV^T (64), dK^T (64).  Three K/V
 // stages (224 KB of shared memory in all) keep the gathered loads two tiles
 // ahead of the MMAs.
+#include <algorithm>
+
 #include "hga_internal.cuh"
 #include "sm100.cuh"
 
@@ -44,7 +46,8 @@ constexpr int kThreads = 320;
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int {
-    kSiteQ = 201, kSiteFull, kSiteEmpty, kSiteSdp, kSitePs, kSiteMm2, kSiteDrained, kSiteFinal, kSiteDrain
+    kSiteQ = 201, kSiteFull, kSiteEmpty, kSiteSdp, kSitePs, kSiteMm2, kSiteDrained, kSiteFinal, kSiteDrain,
+    kSiteQfree, kSiteDqfree
 };
 
 struct BwdSmem {
@@ -57,8 +60,8 @@ struct BwdSmem {
     static constexpr int p_off = v_off + kStages * H * kKVHalf;   // P hi, P lo: [128 rows][64 keys]
     static constexpr int ds_off = p_off + 2 * kRows128;           // dS hi, dS lo
     static constexpr int bar_off = ds_off + 2 * kRows128;
-    // q, full[2], empty[2], sdp[2], ps, mm2, drained, final
-    static constexpr int n_bars = 1 + 2 * kStages + 2 + 4;
+    // q, full[S], empty[S], sdp[2], ps, mm2, drained, final, qfree, dqfree
+    static constexpr int n_bars = 1 + 2 * kStages + 2 + 6;
     static constexpr int tmem_slot_off = bar_off + 8 * n_bars;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;
@@ -75,7 +78,7 @@ struct BwdArgs {
     float* dK;
     float* dV;
     int Hq, Hkv, G, wg;
-    int64_t T_hist, T_seg, nQB;
+    int64_t T_hist, T_seg, nQB, n_items;
     int q_rows;
     float scale, scale_log2;
 };
@@ -89,6 +92,61 @@ __device__ __forceinline__ bool tile_has_segment_keys(int t, int n_rt, int n_g, 
     return (int64_t)grow[last] * 8 + 7 >= T_hist;
 }
 
+// One work item: a (batch, kv-head, query block) and a pair of its q-heads.
+struct Item {
+    int64_t bg, qb, b, g, kv_base, own_start, u;
+    int head0, n_g, n_rt, nt;
+    uint64_t seg;                   // bit t: key tile t holds segment tokens (t < 64)
+    const int32_t* grow;
+};
+
+// Decode item `it` and count its routed groups (an ascending prefix of the
+// index row).  Whole-warp call.
+__device__ __forceinline__ Item make_item(const BwdArgs& a, int64_t it, int lane)
+{
+    Item m;
+    const int n_pairs = (a.G + 1) / 2;
+    m.u = it / n_pairs;                                     // (b*Hkv + g)*nQB + qb
+    m.head0 = 2 * int(it % n_pairs);
+    m.qb = m.u % a.nQB;
+    m.bg = m.u / a.nQB;
+    m.b = m.bg / a.Hkv;
+    m.g = m.bg % a.Hkv;
+    m.kv_base = m.bg * (a.T_hist + a.T_seg);
+    m.own_start = a.T_hist + m.qb * 64;
+    m.grow = a.gidx + m.u * a.wg;
+    // Count the routed groups and mark the tiles holding segment groups
+    // (group j is a segment group when 8 j >= T_hist).
+    int c = 0;
+    uint64_t seg = 0;
+    const int64_t first_seg_group = a.T_hist / 8;
+    for (int base = 0; base < a.wg; base += 32) {
+        const int i = base + lane;
+        const int32_t j = i < a.wg ? __ldg(m.grow + i) : -1;
+        c += j >= 0;
+        const unsigned in_seg = __ballot_sync(0xFFFFFFFFu, j >= 0 && j >= first_seg_group);
+        for (int q = 0; q < 4 && base / 8 + q < 64; ++q)
+            if ((in_seg >> (8 * q)) & 0xFFu) seg |= 1ull << (base / 8 + q);
+    }
+    m.n_g = __reduce_add_sync(0xFFFFFFFFu, c);
+    m.n_rt = (m.n_g + 7) / 8;
+    m.nt = m.n_rt + 1;
+    if (m.n_rt < 64) seg |= 1ull << m.n_rt;                 // the own chunk
+    m.seg = seg;
+    return m;
+}
+
+// Does key tile t of item m hold any segment token (position >= T_hist)?
+__device__ __forceinline__ bool item_tile_has_segment_keys(const Item& m, int t, int64_t T_hist)
+{
+    if (t < 64) return (m.seg >> t) & 1ull;
+    return tile_has_segment_keys(t, m.n_rt, m.n_g, m.grow, T_hist);
+}
+
+// Persistent: CTA c processes items c, c + gridDim.x, ...  Barrier phases
+// run on a global key-tile counter (gt) and an item counter (k) that every
+// role advances identically, so the next item's loads and first S/dP MMAs
+// overlap the current item's dK/dV and dQ epilogues.
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ CUtensorMap tm_v8,
@@ -108,28 +166,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t bar_mm2 = bar0 + 8 * (4 + 2 * kStages);
     const uint32_t bar_drained = bar0 + 8 * (5 + 2 * kStages);
     const uint32_t bar_final = bar0 + 8 * (6 + 2 * kStages);
+    const uint32_t bar_qfree = bar0 + 8 * (7 + 2 * kStages);
+    const uint32_t bar_dqfree = bar0 + 8 * (8 + 2 * kStages);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::tmem_slot_off);
     __shared__ int s_abort;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t u = blockIdx.x;                           // ((b*Hkv)+g)*nQB + qb
-    const int64_t qb = u % a.nQB, bg = u / a.nQB;
-    const int64_t b = bg / a.Hkv, g = bg % a.Hkv;
-    const int head0 = 2 * blockIdx.y;
-    const int64_t T = a.T_hist + a.T_seg;
-    const int64_t kv_base = bg * T;
-    const int64_t own_start = a.T_hist + qb * 64;
-
-    const int32_t* grow = a.gidx + u * a.wg;
-    __shared__ int s_ng;
-    if (threadIdx.x == 0) s_ng = 0;
-    __syncthreads();
-    {
-        int c = 0;
-        for (int i = threadIdx.x; i < a.wg; i += kThreads) c += grow[i] >= 0;
-        c = __reduce_add_sync(0xFFFFFFFFu, c);
-        if (lane == 0 && c) atomicAdd(&s_ng, c);
-    }
+    const int64_t n_items = a.n_items;
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -144,6 +187,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_init(bar_mm2, 1);
         mbar_init(bar_drained, 256);
         mbar_init(bar_final, 1);
+        mbar_init(bar_qfree, 1);
+        mbar_init(bar_dqfree, 256);
         fence_mbar_init();
     }
     if (warp == 9) tmem_alloc(smem_u32(tmem_slot), 512);
@@ -151,9 +196,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_g = s_ng;                                   // routed groups (an ascending prefix)
-    const int n_rt = (n_g + 7) / 8;
-    const int nt = n_rt + 1;
 
     if (warp == 8) {
         // ------------------------------------------------------------ producer
@@ -164,110 +206,154 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             prefetch_tmap(&tm_v8);
             prefetch_tmap(&tm_k64);
             prefetch_tmap(&tm_v64);
-            mbar_expect_tx(bar_q, 2 * 2 * H * 64 * 128);
-            for (int hp = 0; hp < 2; ++hp) {
-                const int head = head0 + hp;
-                const int y = head < a.G ? int((b * a.Hq + g * a.G + head) * a.T_seg + qb * 64) : a.q_rows;
-                for (int c = 0; c < H; ++c) {
-                    const uint32_t off = c * L::kRows128 + hp * 64 * 128;
-                    tma_load_2d(sbase + L::q_off + off, &tm_q, 64 * c, y, bar_q);
-                    tma_load_2d(sbase + L::do_off + off, &tm_do, 64 * c, y, bar_q);
+        }
+        int last_gt[kStages] = {-1, -1, -1};                // last tile loaded per stage
+        int k_loaded = -1;                                  // last item whose Q/dO was loaded
+        uint32_t gt = 0;
+        bool ok = true;
+        int k = 0;
+        for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+            const Item m = make_item(a, it, lane);
+            for (int t = 0; t < m.nt && ok; ++t, ++gt) {
+                const int s = gt % kStages;
+                if (lane == 0) {
+                    ok = gt < kStages || mbar_wait(bar_empty(s), ((gt / kStages) - 1) & 1, kSiteEmpty);
+                    if (ok) mbar_expect_tx(bar_full(s), 2 * H * kKeys * 128);
+                }
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
+                last_gt[s] = gt;
+                const uint32_t kdst = sbase + L::k_off + s * H * L::kKVHalf;
+                const uint32_t vdst = sbase + L::v_off + s * H * L::kKVHalf;
+                if (t < m.n_rt) {
+                    if (lane < 8) {                           // one group per lane
+                        const int gi = t * 8 + lane;
+                        const int grp = __ldg(m.grow + (gi < m.n_g ? gi : 0));
+                        const int y = int(m.kv_base + (int64_t)grp * 8);
+                        for (int c = 0; c < H; ++c) {
+                            tma_load_2d(kdst + c * L::kKVHalf + lane * 1024, &tm_k8, 64 * c, y, bar_full(s));
+                            tma_load_2d(vdst + c * L::kKVHalf + lane * 1024, &tm_v8, 64 * c, y, bar_full(s));
+                        }
+                    }
+                } else if (lane == 0) {
+                    const int y = int(m.kv_base + m.own_start);
+                    for (int c = 0; c < H; ++c) {
+                        tma_load_2d(kdst + c * L::kKVHalf, &tm_k64, 64 * c, y, bar_full(s));
+                        tma_load_2d(vdst + c * L::kKVHalf, &tm_v64, 64 * c, y, bar_full(s));
+                    }
+                }
+                __syncwarp();
+                if (t == 0) {
+                    // Q and dO of this item once the previous item's MMAs are done.
+                    if (lane == 0) {
+                        ok = k == 0 || mbar_wait(bar_qfree, (k - 1) & 1, kSiteQfree);
+                        if (ok) {
+                            mbar_expect_tx(bar_q, 2 * 2 * H * 64 * 128);
+                            for (int hp = 0; hp < 2; ++hp) {
+                                const int head = m.head0 + hp;
+                                const int y = head < a.G
+                                                  ? int((m.b * a.Hq + m.g * a.G + head) * a.T_seg + m.qb * 64)
+                                                  : a.q_rows;
+                                for (int c = 0; c < H; ++c) {
+                                    const uint32_t off = c * L::kRows128 + hp * 64 * 128;
+                                    tma_load_2d(sbase + L::q_off + off, &tm_q, 64 * c, y, bar_q);
+                                    tma_load_2d(sbase + L::do_off + off, &tm_do, 64 * c, y, bar_q);
+                                }
+                            }
+                        }
+                    }
+                    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                    if (ok) k_loaded = k;
                 }
             }
         }
-        for (int t = 0; t < nt; ++t) {
-            const int s = t % kStages, r = t / kStages;
-            bool ok = true;
-            if (lane == 0) {
-                ok = t < kStages || mbar_wait(bar_empty(s), (r - 1) & 1, kSiteEmpty);
-                if (ok) mbar_expect_tx(bar_full(s), 2 * H * kKeys * 128);
-            }
-            if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
-                s_abort = 1;
-                break;
-            }
-            const uint32_t kdst = sbase + L::k_off + s * H * L::kKVHalf;
-            const uint32_t vdst = sbase + L::v_off + s * H * L::kKVHalf;
-            if (t < n_rt) {
-                if (lane < 8) {                               // one group per lane
-                    const int gi = t * 8 + lane;
-                    const int grp = __ldg(grow + (gi < n_g ? gi : 0));
-                    const int y = int(kv_base + (int64_t)grp * 8);
-                    for (int c = 0; c < H; ++c) {
-                        tma_load_2d(kdst + c * L::kKVHalf + lane * 1024, &tm_k8, 64 * c, y, bar_full(s));
-                        tma_load_2d(vdst + c * L::kKVHalf + lane * 1024, &tm_v8, 64 * c, y, bar_full(s));
-                    }
-                }
-            } else if (lane == 0) {
-                const int y = int(kv_base + own_start);
-                for (int c = 0; c < H; ++c) {
-                    tma_load_2d(kdst + c * L::kKVHalf, &tm_k64, 64 * c, y, bar_full(s));
-                    tma_load_2d(vdst + c * L::kKVHalf, &tm_v64, 64 * c, y, bar_full(s));
-                }
-            }
-            __syncwarp();
+        if (!ok) s_abort = 1;
+        // Wind down: every copy issued has landed before the CTA exits.
+        __syncwarp();
+        if (lane == 0 && !ok) {
+            for (int s = 0; s < kStages; ++s)
+                if (last_gt[s] >= 0) mbar_wait(bar_full(s), (last_gt[s] / kStages) & 1, kSiteDrain);
+            if (k_loaded >= 0) mbar_wait(bar_q, k_loaded & 1, kSiteDrain);
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t id_sdp = idesc_bf16(128, kKeys, 0, 0);   // S, dP
-            constexpr uint32_t id_dq = idesc_bf16(128, D, 0, 1);        // dQ: A dS K-major, B K MN-major
-            constexpr uint32_t id_kv = idesc_bf16(128, kKeys, 1, 1);    // dV^T, dK^T: both MN-major
-            bool ok = mbar_wait(bar_q, 0, kSiteQ);
-            auto issue_sdp = [&](int t) -> bool {
-                const int s = t % kStages, bb = t & 1;
-                if (!mbar_wait(bar_full(s), (t / kStages) & 1, kSiteFull)) return false;
-                tc_fence_after();
-                for (int kk = 0; kk < 4 * H; ++kk) {
-                    const uint32_t o = (kk / 4) * L::kRows128 + (kk % 4) * 32;
-                    const uint32_t ko = (s * H + kk / 4) * L::kKVHalf + (kk % 4) * 32;
-                    mma_ss(tmem + kColS + bb * kKeys, sdesc_sw128(sbase + L::q_off + o, 16, 1024),
-                           sdesc_sw128(sbase + L::k_off + ko, 16, 1024), id_sdp, kk > 0);
-                    mma_ss(tmem + kColDP + bb * kKeys, sdesc_sw128(sbase + L::do_off + o, 16, 1024),
-                           sdesc_sw128(sbase + L::v_off + ko, 16, 1024), id_sdp, kk > 0);
-                }
-                mma_commit(bar_sdp(bb));
-                return true;
-            };
-            // S / dP run two tiles ahead (double-buffered): S(t+2) is issued
-            // right after the MMAs of tile t, so that its load wait never
-            // holds back the gradient MMAs of the tile the softmax finished.
-            if (ok) ok = issue_sdp(0);
-            if (ok && nt > 1) ok = issue_sdp(1);
-            for (int t = 0; ok && t < nt; ++t) {
-                const int s = t % kStages;
-                if (!(ok = mbar_wait(bar_ps, t & 1, kSitePs))) break;
-                tc_fence_after();
-                // dQ += dS K  (dS hi and lo against the same K)
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t kb = sdesc_sw128(sbase + L::k_off + s * H * L::kKVHalf + kk * 2048, L::kKVHalf, 1024);
-                    mma_ss(tmem + kColDQ, sdesc_sw128(sbase + L::ds_off + kk * 32, 16, 1024), kb, id_dq,
-                           t > 0 || kk > 0);
-                    mma_ss(tmem + kColDQ, sdesc_sw128(sbase + L::ds_off + L::kRows128 + kk * 32, 16, 1024), kb,
-                           id_dq, true);
-                }
-                if (tile_has_segment_keys(t, n_rt, n_g, grow, a.T_hist)) {
-                    if (t >= 1 && !(ok = mbar_wait(bar_drained, (t - 1) & 1, kSiteDrained))) break;
+        constexpr uint32_t id_sdp = idesc_bf16(128, kKeys, 0, 0);   // S, dP
+        constexpr uint32_t id_dq = idesc_bf16(128, D, 0, 1);        // dQ: A dS K-major, B K MN-major
+        constexpr uint32_t id_kv = idesc_bf16(128, kKeys, 1, 1);    // dV^T, dK^T: both MN-major
+        uint32_t gt = 0;
+        bool ok = true;
+        int k = 0;
+        for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+            const Item m = make_item(a, it, lane);
+            if (lane == 0) {
+                auto issue_sdp = [&](uint32_t gtt) -> bool {
+                    const int s = gtt % kStages, bb = gtt & 1;
+                    if (!mbar_wait(bar_full(s), (gtt / kStages) & 1, kSiteFull)) return false;
                     tc_fence_after();
-                    // dV^T = dO^T P and dK^T = Q^T dS over the 128 query rows.
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t dOt = sdesc_sw128(sbase + L::do_off + kk * 2048, L::kRows128, 1024);
-                        const uint64_t Qt = sdesc_sw128(sbase + L::q_off + kk * 2048, L::kRows128, 1024);
-                        const uint64_t Ph = sdesc_sw128(sbase + L::p_off + kk * 2048, L::kRows128, 1024);
-                        const uint64_t Pl = sdesc_sw128(sbase + L::p_off + L::kRows128 + kk * 2048, L::kRows128, 1024);
-                        const uint64_t Sh = sdesc_sw128(sbase + L::ds_off + kk * 2048, L::kRows128, 1024);
-                        const uint64_t Sl = sdesc_sw128(sbase + L::ds_off + L::kRows128 + kk * 2048, L::kRows128, 1024);
-                        mma_ss(tmem + kColDV, dOt, Ph, id_kv, kk > 0);
-                        mma_ss(tmem + kColDV, dOt, Pl, id_kv, true);
-                        mma_ss(tmem + kColDK, Qt, Sh, id_kv, kk > 0);
-                        mma_ss(tmem + kColDK, Qt, Sl, id_kv, true);
+                    for (int kk = 0; kk < 4 * H; ++kk) {
+                        const uint32_t o = (kk / 4) * L::kRows128 + (kk % 4) * 32;
+                        const uint32_t ko = (s * H + kk / 4) * L::kKVHalf + (kk % 4) * 32;
+                        mma_ss(tmem + kColS + bb * kKeys, sdesc_sw128(sbase + L::q_off + o, 16, 1024),
+                               sdesc_sw128(sbase + L::k_off + ko, 16, 1024), id_sdp, kk > 0);
+                        mma_ss(tmem + kColDP + bb * kKeys, sdesc_sw128(sbase + L::do_off + o, 16, 1024),
+                               sdesc_sw128(sbase + L::v_off + ko, 16, 1024), id_sdp, kk > 0);
                     }
+                    mma_commit(bar_sdp(bb));
+                    return true;
+                };
+                ok = mbar_wait(bar_q, k & 1, kSiteQ);
+                // S / dP run two tiles ahead (double-buffered): S(t+2) is
+                // issued right after the MMAs of tile t, so its load wait never
+                // holds back the gradient MMAs of the tile the softmax finished.
+                if (ok) ok = issue_sdp(gt);
+                if (ok && m.nt > 1) ok = issue_sdp(gt + 1);
+                for (int t = 0; ok && t < m.nt; ++t) {
+                    const uint32_t gtt = gt + t;
+                    const int s = gtt % kStages;
+                    if (!(ok = mbar_wait(bar_ps, gtt & 1, kSitePs))) break;
+                    // dQ accumulates from zero: the previous item's dQ is read out.
+                    if (t == 0 && k > 0 && !(ok = mbar_wait(bar_dqfree, (k - 1) & 1, kSiteDqfree))) break;
+                    tc_fence_after();
+                    // dQ += dS K  (dS hi and lo against the same K)
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t kb =
+                            sdesc_sw128(sbase + L::k_off + s * H * L::kKVHalf + kk * 2048, L::kKVHalf, 1024);
+                        mma_ss(tmem + kColDQ, sdesc_sw128(sbase + L::ds_off + kk * 32, 16, 1024), kb, id_dq,
+                               t > 0 || kk > 0);
+                        mma_ss(tmem + kColDQ, sdesc_sw128(sbase + L::ds_off + L::kRows128 + kk * 32, 16, 1024), kb,
+                               id_dq, true);
+                    }
+                    if (item_tile_has_segment_keys(m, t, a.T_hist)) {
+                        if (gtt >= 1 && !(ok = mbar_wait(bar_drained, (gtt - 1) & 1, kSiteDrained))) break;
+                        tc_fence_after();
+                        // dV^T = dO^T P and dK^T = Q^T dS over the 128 query rows.
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t dOt = sdesc_sw128(sbase + L::do_off + kk * 2048, L::kRows128, 1024);
+                            const uint64_t Qt = sdesc_sw128(sbase + L::q_off + kk * 2048, L::kRows128, 1024);
+                            const uint64_t Ph = sdesc_sw128(sbase + L::p_off + kk * 2048, L::kRows128, 1024);
+                            const uint64_t Pl =
+                                sdesc_sw128(sbase + L::p_off + L::kRows128 + kk * 2048, L::kRows128, 1024);
+                            const uint64_t Sh = sdesc_sw128(sbase + L::ds_off + kk * 2048, L::kRows128, 1024);
+                            const uint64_t Sl =
+                                sdesc_sw128(sbase + L::ds_off + L::kRows128 + kk * 2048, L::kRows128, 1024);
+                            mma_ss(tmem + kColDV, dOt, Ph, id_kv, kk > 0);
+                            mma_ss(tmem + kColDV, dOt, Pl, id_kv, true);
+                            mma_ss(tmem + kColDK, Qt, Sh, id_kv, kk > 0);
+                            mma_ss(tmem + kColDK, Qt, Sl, id_kv, true);
+                        }
+                    }
+                    mma_commit(bar_mm2);
+                    mma_commit(bar_empty(s));
+                    if (t == m.nt - 1) mma_commit(bar_qfree);          // Q / dO of this item no longer read
+                    if (t + 2 < m.nt && !(ok = issue_sdp(gtt + 2))) break;
                 }
-                mma_commit(bar_mm2);
-                mma_commit(bar_empty(s));
-                if (t + 2 < nt && !(ok = issue_sdp(t + 2))) break;
             }
-            if (!ok) s_abort = 1;
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            gt += m.nt;
+        }
+        if (!ok) s_abort = 1;
+        if (lane == 0) {
+            // Every MMA issued is complete before tensor memory is released.
             mma_commit(bar_final);
             mbar_wait(bar_final, 0, kSiteFinal);
         }
@@ -276,130 +362,174 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // Thread (warp w, lane l): query row r = 32*(w%4) + l of the M-tile
         // (its tensor-memory lane) and the 32-key half kh = w/4 of each tile.
         const int r = (warp % 4) * 32 + lane, kh = warp / 4;
-        const int i = r & 63, hp = r >> 6, head = head0 + hp;
-        const bool row_ok = head < a.G;
-        const int64_t row = (b * a.Hq + g * a.G + head) * a.T_seg + qb * 64 + i;
-        const float lse2 = row_ok ? a.lse[row] * kLog2e : 0.f;
-        const float Dr = row_ok ? a.Drow[row] : 0.f;
+        const int i = r & 63, hp = r >> 6;
         const uint32_t lane_off = uint32_t((warp % 4) * 32) << 16;
         uint8_t* prow_hi = smem + L::p_off + r * 128;
         uint8_t* prow_lo = prow_hi + L::kRows128;
         uint8_t* srow_hi = smem + L::ds_off + r * 128;
         uint8_t* srow_lo = srow_hi + L::kRows128;
-        // dV^T / dK^T of tile te (d = tensor-memory lane r, keys of half kh)
-        // added to the segment's rows; history keys and padding are skipped.
-        auto dkv_epilogue = [&](int te) {
-            if (!tile_has_segment_keys(te, n_rt, n_g, grow, a.T_hist)) return;
+        // dV^T / dK^T of tile te of item m (d = tensor-memory lane r, keys of
+        // half kh) added to the segment's rows; history keys and padding are
+        // skipped.
+        auto dkv_epilogue = [&](const Item& m, int te) {
+            if (!item_tile_has_segment_keys(m, te, a.T_hist)) return;
             tc_fence_after();
             uint32_t vv[32], kv[32];
             tmem_ld32(tmem + lane_off + kColDV + 32 * kh, vv);
             tmem_ld32(tmem + lane_off + kColDK + 32 * kh, kv);
             tmem_wait_ld();
-            const bool own = te == n_rt;
+            const bool own = te == m.n_rt;
             int64_t gbase[4];                               // first token of each group slot
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int gi = te * 8 + 4 * kh + q;
-                gbase[q] = own ? own_start + 32 * kh + 8 * q : (gi < n_g ? (int64_t)__ldg(grow + gi) * 8 : -64);
+                gbase[q] = own ? m.own_start + 32 * kh + 8 * q : (gi < m.n_g ? (int64_t)__ldg(m.grow + gi) * 8 : -64);
             }
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int64_t key = gbase[j / 8] + j % 8;
                 if (key < a.T_hist) continue;               // padding or detached history
-                const int64_t o = (bg * a.T_seg + (key - a.T_hist)) * D + r;
+                const int64_t o = (m.bg * a.T_seg + (key - a.T_hist)) * D + r;
                 atomicAdd(a.dV + o, __uint_as_float(vv[j]));
                 atomicAdd(a.dK + o, __uint_as_float(kv[j]) * a.scale);
             }
         };
+        // Per-row constants of an item.
+        struct RowInfo { int64_t row; bool ok; float lse2, Dr; };
+        auto row_info = [&](const Item& m) {
+            RowInfo ri;
+            const int head = m.head0 + hp;
+            ri.ok = head < a.G;
+            ri.row = (m.b * a.Hq + m.g * a.G + head) * a.T_seg + m.qb * 64 + i;
+            ri.lse2 = ri.ok ? __ldg(a.lse + ri.row) * kLog2e : 0.f;
+            ri.Dr = ri.ok ? __ldg(a.Drow + ri.row) : 0.f;
+            return ri;
+        };
+        // dQ staging: the P / dS region (64 KB) is free once an item's last
+        // MMAs are done; rows of 512 B, 16-byte chunks XOR-swizzled by row.
+        float* stage = reinterpret_cast<float*>(smem + L::p_off);
+        uint32_t gt = 0;
         bool ok = true;
-        for (int t = 0; t < nt && ok; ++t) {
-            const int bb = t & 1;
-            ok = mbar_wait(bar_sdp(bb), (t / 2) & 1, kSiteSdp);
-            if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
-            tc_fence_after();
-            const bool own = t == n_rt;
-            // P is an MMA operand only for dV, i.e. for tiles holding segment keys.
-            const bool seg = tile_has_segment_keys(t, n_rt, n_g, grow, a.T_hist);
-            uint32_t sr[32], pr[32];
-            tmem_ld32(tmem + lane_off + kColS + bb * kKeys + 32 * kh, sr);
-            tmem_ld32(tmem + lane_off + kColDP + bb * kKeys + 32 * kh, pr);
-            tmem_wait_ld();
-            uint32_t ph[16], pl[16], dh[16], dl[16];
-#pragma unroll
-            for (int j2 = 0; j2 < 16; ++j2) {
-                float p[2], ds[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int jj = 2 * j2 + e, j = 32 * kh + jj;
-                    const bool valid = row_ok && (own ? (j <= i) : (t * 8 + j / 8 < n_g));
-                    p[e] = valid ? fast_exp2(fmaf(__uint_as_float(sr[jj]), a.scale_log2, -lse2)) : 0.f;
-                    ds[e] = p[e] * (__uint_as_float(pr[jj]) - Dr);
-                }
-                split_bf16x2(ds[0], ds[1], dh[j2], dl[j2]);
-                if (seg) split_bf16x2(p[0], p[1], ph[j2], pl[j2]);
-            }
-            // The previous tile's MMAs read P / dS from shared memory.
-            if (t >= 1) {
-                ok = mbar_wait(bar_mm2, (t - 1) & 1, kSiteMm2);
+        int k = 0;
+        int64_t it = blockIdx.x;
+        Item m = make_item(a, it < n_items ? it : 0, lane);
+        RowInfo ri = row_info(m);
+        for (; it < n_items && ok; ++k) {
+            const int64_t row = ri.row;
+            const bool row_ok = ri.ok;
+            const float lse2 = ri.lse2, Dr = ri.Dr;
+            for (int t = 0; t < m.nt && ok; ++t) {
+                const uint32_t gtt = gt + t;
+                const int bb = gtt & 1;
+                ok = mbar_wait(bar_sdp(bb), (gtt / 2) & 1, kSiteSdp);
                 if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
-            }
-            // Row r, 16-byte chunk c lives at chunk c ^ (r % 8) (128-byte swizzle).
+                tc_fence_after();
+                const bool own = t == m.n_rt;
+                // P is an MMA operand only for dV, i.e. for tiles holding segment keys.
+                const bool seg = item_tile_has_segment_keys(m, t, a.T_hist);
+                uint32_t sr[32], pr[32];
+                tmem_ld32(tmem + lane_off + kColS + bb * kKeys + 32 * kh, sr);
+                tmem_ld32(tmem + lane_off + kColDP + bb * kKeys + 32 * kh, pr);
+                tmem_wait_ld();
+                uint32_t ph[16], pl[16], dh[16], dl[16];
+                // Every key of a full routed tile is valid for every row:
+                // no masks there; partial tiles and the own chunk mask keys.
+                const bool full = row_ok && !own && t * 8 + 8 <= m.n_g;
+                const float2 c2 = make_float2(a.scale_log2, a.scale_log2);
+                const float2 l2 = make_float2(-lse2, -lse2), d2 = make_float2(-Dr, -Dr);
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const int pc = ((4 * kh + c4) ^ (r & 7)) * 16;
-                *reinterpret_cast<uint4*>(srow_hi + pc) = make_uint4(dh[4 * c4], dh[4 * c4 + 1], dh[4 * c4 + 2], dh[4 * c4 + 3]);
-                *reinterpret_cast<uint4*>(srow_lo + pc) = make_uint4(dl[4 * c4], dl[4 * c4 + 1], dl[4 * c4 + 2], dl[4 * c4 + 3]);
-                if (seg) {
-                    *reinterpret_cast<uint4*>(prow_hi + pc) = make_uint4(ph[4 * c4], ph[4 * c4 + 1], ph[4 * c4 + 2], ph[4 * c4 + 3]);
-                    *reinterpret_cast<uint4*>(prow_lo + pc) = make_uint4(pl[4 * c4], pl[4 * c4 + 1], pl[4 * c4 + 2], pl[4 * c4 + 3]);
+                for (int j2 = 0; j2 < 16; ++j2) {
+                    const int j0 = 32 * kh + 2 * j2;
+                    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1])),
+                                                c2, l2);
+                    float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                    if (!full) {
+                        const bool v0 = row_ok && (own ? (j0 <= i) : (t * 8 + j0 / 8 < m.n_g));
+                        const bool v1 = row_ok && (own ? (j0 + 1 <= i) : (t * 8 + (j0 + 1) / 8 < m.n_g));
+                        p.x = v0 ? p.x : 0.f;
+                        p.y = v1 ? p.y : 0.f;
+                    }
+                    const float2 ds = __fmul2_rn(
+                        p, __fadd2_rn(make_float2(__uint_as_float(pr[2 * j2]), __uint_as_float(pr[2 * j2 + 1])), d2));
+                    split_bf16x2(ds.x, ds.y, dh[j2], dl[j2]);
+                    if (seg) split_bf16x2(p.x, p.y, ph[j2], pl[j2]);
+                }
+                // The previous tile's MMAs read P / dS from shared memory.
+                if (gtt >= 1) {
+                    ok = mbar_wait(bar_mm2, (gtt - 1) & 1, kSiteMm2);
+                    if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
+                }
+                // Row r, 16-byte chunk c lives at chunk c ^ (r % 8) (128-byte swizzle).
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int pc = ((4 * kh + c4) ^ (r & 7)) * 16;
+                    *reinterpret_cast<uint4*>(srow_hi + pc) = make_uint4(dh[4 * c4], dh[4 * c4 + 1], dh[4 * c4 + 2], dh[4 * c4 + 3]);
+                    *reinterpret_cast<uint4*>(srow_lo + pc) = make_uint4(dl[4 * c4], dl[4 * c4 + 1], dl[4 * c4 + 2], dl[4 * c4 + 3]);
+                    if (seg) {
+                        *reinterpret_cast<uint4*>(prow_hi + pc) = make_uint4(ph[4 * c4], ph[4 * c4 + 1], ph[4 * c4 + 2], ph[4 * c4 + 3]);
+                        *reinterpret_cast<uint4*>(prow_lo + pc) = make_uint4(pl[4 * c4], pl[4 * c4 + 1], pl[4 * c4 + 2], pl[4 * c4 + 3]);
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(bar_ps);
+                // While the MMAs of tile t run: the dK / dV of tile t-1.
+                if (t >= 1) {
+                    dkv_epilogue(m, t - 1);
+                    tc_fence_before();
+                    mbar_arrive(bar_drained);
                 }
             }
-            fence_async_smem();
+            if (!ok) break;
+            // The next item's index row and row constants load meanwhile.
+            const int64_t it_next = it + gridDim.x;
+            const Item m_next = make_item(a, it_next < n_items ? it_next : it, lane);
+            const RowInfo ri_next = row_info(m_next);
+            const uint32_t last = gt + m.nt - 1;
+            ok = mbar_wait(bar_mm2, last & 1, kSiteMm2);
+            if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
+            dkv_epilogue(m, m.nt - 1);
             tc_fence_before();
-            mbar_arrive(bar_ps);
-            // While the MMAs of tile t run: the dK / dV of tile t-1.
-            if (t >= 1) {
-                dkv_epilogue(t - 1);
-                tc_fence_before();
-                mbar_arrive(bar_drained);
-            }
-        }
-        if (ok) {
-            ok = mbar_wait(bar_mm2, (nt - 1) & 1, kSiteMm2);
-            if (__any_sync(0xFFFFFFFFu, !ok)) ok = false;
-        }
-        if (ok) {
-            dkv_epilogue(nt - 1);
+            mbar_arrive(bar_drained);
             tc_fence_after();
-            float* dq = a.dQ + row * D + 64 * kh;
+            // dQ (times the softmax scale): tensor memory -> swizzled shared rows.
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tmem + lane_off + kColDQ + 64 * kh + 32 * c, v);
                 tmem_wait_ld();
-                if (row_ok) {
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4*>(dq + 32 * c + j) =
-                            make_float4(__uint_as_float(v[j]) * a.scale, __uint_as_float(v[j + 1]) * a.scale,
-                                        __uint_as_float(v[j + 2]) * a.scale, __uint_as_float(v[j + 3]) * a.scale);
+                for (int j = 0; j < 32; j += 4) {
+                    const int ch = (64 * kh + 32 * c + j) / 4;     // 16-byte chunk of the row
+                    const int pch = (ch & ~7) | ((ch ^ r) & 7);
+                    *reinterpret_cast<float4*>(stage + r * D + 4 * pch) =
+                        make_float4(__uint_as_float(v[j]) * a.scale, __uint_as_float(v[j + 1]) * a.scale,
+                                    __uint_as_float(v[j + 2]) * a.scale, __uint_as_float(v[j + 3]) * a.scale);
                 }
             }
-        } else {
-            s_abort = 1;
+            tc_fence_before();
+            mbar_arrive(bar_dqfree);
+            named_barrier_sync(1, 256);
+            // Coalesced rows: warp w writes rows w, w+8, ...; lane l the l-th 16 bytes.
+            for (int rr = warp; rr < 128; rr += 8) {
+                const int head = m.head0 + (rr >> 6);
+                if (head >= a.G) continue;
+                const int64_t grow_ = (m.b * a.Hq + m.g * a.G + head) * a.T_seg + m.qb * 64 + (rr & 63);
+                const int pch = (lane & ~7) | ((lane ^ rr) & 7);
+                *reinterpret_cast<float4*>(a.dQ + grow_ * D + 4 * lane) =
+                    *reinterpret_cast<const float4*>(stage + rr * D + 4 * pch);
+            }
+            named_barrier_sync(1, 256);             // staging rows read before P / dS reuse them
+            (void)row;
+            gt += m.nt;
+            it = it_next;
+            m = m_next;
+            ri = ri_next;
         }
+        if (!ok) s_abort = 1;
     }
 
     tc_fence_before();
-    __syncthreads();
-    if (s_abort && warp == 8 && lane == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            int last = -1;
-            for (int t = s; t < nt; t += kStages) last = t;
-            if (last >= 0) mbar_wait(bar_full(s), (last / kStages) & 1, kSiteDrain);
-        }
-        mbar_wait(bar_q, 0, kSiteDrain);
-    }
     __syncthreads();
     if (warp == 9) {
         tc_fence_after();
@@ -482,8 +612,9 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
     if ((e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
         return e;
-    const dim3 grid((unsigned)(s.B * s.Hkv * s.nQB), (unsigned)((s.G + 1) / 2));
-    attn_bwd_tc_kernel<<<grid, kThreads, smem, st>>>(tq, tdo, tk8, tv8, tk64, tv64, a);
+    a.n_items = (int64_t)s.B * s.Hkv * s.nQB * ((s.G + 1) / 2);
+    const int64_t grid = std::min<int64_t>(a.n_items, sm_count());
+    attn_bwd_tc_kernel<<<(unsigned)grid, kThreads, smem, st>>>(tq, tdo, tk8, tv8, tk64, tv64, a);
     return cudaGetLastError();
 }
 

@@ -267,12 +267,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             float sv[64];
             float mx = -INFINITY;
             const bool own = t == n_rt;
+            // Full routed tiles need no masks; the scale is applied after the
+            // maximum (it is positive) and folded into the exponent's FMA.
+            const bool full = !own && t * 8 + 8 <= n_g;
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
-                const bool valid = own ? (j <= i) : (t * 8 + j / 8 < n_g);
-                sv[j] = valid ? __uint_as_float(raw[j / 32][j % 32]) * a.scale_log2 : -INFINITY;
+                sv[j] = __uint_as_float(raw[j / 32][j % 32]);
+                if (!full && !(own ? (j <= i) : (t * 8 + j / 8 < n_g))) sv[j] = -INFINITY;
                 mx = fmaxf(mx, sv[j]);
             }
+            mx *= a.scale_log2;
             const bool need = mx > m_run + kRescaleLog2;
             if (__any_sync(0xFFFFFFFFu, need)) {
                 const float m_new = need ? mx : m_run;
@@ -298,14 +302,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // P = hi + lo, both bf16: the two MMAs carry P to ~14 bits, where
             // one bf16 operand alone (8 bits) misses the 2e-3 output bound.
             uint32_t pk_hi[32], pk_lo[32];
-            float rs = 0.f;
+            float2 rs = make_float2(0.f, 0.f);
+            const float2 c2 = make_float2(a.scale_log2, a.scale_log2), nm = make_float2(-m_run, -m_run);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float p0 = fast_exp2(sv[2 * j] - m_run), p1 = fast_exp2(sv[2 * j + 1] - m_run);
-                rs += p0 + p1;
-                split_bf16x2(p0, p1, pk_hi[j], pk_lo[j]);
+                const float2 x = __ffma2_rn(make_float2(sv[2 * j], sv[2 * j + 1]), c2, nm);
+                const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                rs = __fadd2_rn(rs, p);
+                split_bf16x2(p.x, p.y, pk_hi[j], pk_lo[j]);
             }
-            l_run += rs;
+            l_run += rs.x + rs.y;
             tmem_st32(tmem + lane_off + col_s(m, bb), pk_hi);
             tmem_st32(tmem + lane_off + col_s(m, bb) + 32, pk_lo);
             tmem_wait_st();

@@ -91,6 +91,9 @@ cudaError_t launch_attn_bwd_simt(const Shape& s, const void* Q, const void* K, c
                                  const int32_t* gidx, float* dQ, float* dK_seg, float* dV_seg,
                                  float* Drow, cudaStream_t st);
 
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count();
+
 // TMA tensor maps (tma_map.cu).
 bool tensor_maps_available();
 bool make_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);

@@ -113,6 +113,12 @@ __device__ __forceinline__ void fence_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Named barrier `id` over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ---- tensor memory -------------------------------------------------------------------
 // Whole-warp operations.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
@@ -233,9 +239,10 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
 {
     const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
     hi = __byte_perm(b0, b1, 0x7632);
-    const float r0 = x0 - __uint_as_float(b0 & 0xFFFF0000u);
-    const float r1 = x1 - __uint_as_float(b1 & 0xFFFF0000u);
-    lo = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+    // remainder x - trunc(x), exact in fp32, with one packed FMA
+    const float2 r = __ffma2_rn(make_float2(__uint_as_float(b0 & 0xFFFF0000u), __uint_as_float(b1 & 0xFFFF0000u)),
+                                make_float2(-1.f, -1.f), make_float2(x0, x1));
+    lo = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)

@@ -26,6 +26,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 
 bool tensor_maps_available() { return encode_fn() != nullptr; }
 
+int sm_count()
+{
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 // 2-D bf16 map over `rows` rows of `cols` elements; box of 64 columns x
 // box_rows rows, 128-byte swizzle (the shared-memory layout the MMA operand
 // descriptors of the tensor-core kernels describe).  Out-of-range boxes read
