@@ -47,7 +47,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int {
     kSiteQ = 201, kSiteFull, kSiteEmpty, kSiteSdp, kSitePs, kSiteMm2, kSiteDrained, kSiteFinal, kSiteDrain,
-    kSiteQfree, kSiteDqfree
+    kSiteQfree, kSiteDqfree, kSiteStage
 };
 
 struct BwdSmem {
@@ -60,8 +60,8 @@ struct BwdSmem {
     static constexpr int p_off = v_off + kStages * H * kKVHalf;   // P hi, P lo: [128 rows][64 keys]
     static constexpr int ds_off = p_off + 2 * kRows128;           // dS hi, dS lo
     static constexpr int bar_off = ds_off + 2 * kRows128;
-    // q, full[S], empty[S], sdp[2], ps, mm2, drained, final, qfree, dqfree
-    static constexpr int n_bars = 1 + 2 * kStages + 2 + 6;
+    // q, full[S], empty[S], sdp[2], ps, mm2, drained, final, qfree, dqfree, stage
+    static constexpr int n_bars = 1 + 2 * kStages + 2 + 7;
     static constexpr int tmem_slot_off = bar_off + 8 * n_bars;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;
@@ -168,6 +168,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t bar_final = bar0 + 8 * (6 + 2 * kStages);
     const uint32_t bar_qfree = bar0 + 8 * (7 + 2 * kStages);
     const uint32_t bar_dqfree = bar0 + 8 * (8 + 2 * kStages);
+    const uint32_t bar_stage = bar0 + 8 * (9 + 2 * kStages);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::tmem_slot_off);
     __shared__ int s_abort;
 
@@ -189,6 +190,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_init(bar_final, 1);
         mbar_init(bar_qfree, 1);
         mbar_init(bar_dqfree, 256);
+        mbar_init(bar_stage, 256);
         fence_mbar_init();
     }
     if (warp == 9) tmem_alloc(smem_u32(tmem_slot), 512);
@@ -509,7 +511,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             tc_fence_before();
             mbar_arrive(bar_dqfree);
-            named_barrier_sync(1, 256);
+            // All 256 compute threads have staged their dQ parts (bounded wait).
+            mbar_arrive(bar_stage);
+            if (!mbar_wait(bar_stage, (2 * k) & 1, kSiteStage)) { ok = false; break; }
             // Coalesced rows: warp w writes rows w, w+8, ...; lane l the l-th 16 bytes.
             for (int rr = warp; rr < 128; rr += 8) {
                 const int head = m.head0 + (rr >> 6);
@@ -519,7 +523,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 *reinterpret_cast<float4*>(a.dQ + grow_ * D + 4 * lane) =
                     *reinterpret_cast<const float4*>(stage + rr * D + 4 * pch);
             }
-            named_barrier_sync(1, 256);             // staging rows read before P / dS reuse them
+            // The staging rows are read before P / dS of the next item reuse them.
+            mbar_arrive(bar_stage);
+            if (!mbar_wait(bar_stage, (2 * k + 1) & 1, kSiteStage)) { ok = false; break; }
             (void)row;
             gt += m.nt;
             it = it_next;

@@ -42,7 +42,7 @@ constexpr float kRescaleLog2 = 8.0f;
 
 // Status codes of the bounded waits (site of the wait that ran out).
 enum : int {
-    kSiteQ = 101, kSiteFull, kSiteEmpty, kSiteS, kSiteP, kSiteO, kSiteFinal, kSiteDrain
+    kSiteQ = 101, kSiteFull, kSiteEmpty, kSiteS, kSiteP, kSiteO, kSiteFinal, kSiteDrain, kSiteStage
 };
 
 template <int D>
@@ -54,8 +54,8 @@ struct FwdSmem {
     static constexpr int k_off = q_off + 2 * H * kQTile;
     static constexpr int v_off = k_off + kStages * H * kKVHalf;
     static constexpr int bar_off = v_off + kStages * H * kKVHalf;
-    // barriers: q, full[S], empty[S], s[2][2], p[2][2], o[2][2], final
-    static constexpr int n_bars = 1 + 2 * kStages + 4 + 4 + 4 + 1;
+    // barriers: q, full[S], empty[S], s[2][2], p[2][2], o[2][2], final, stage
+    static constexpr int n_bars = 1 + 2 * kStages + 4 + 4 + 4 + 2;
     static constexpr int tmem_slot_off = bar_off + 8 * n_bars;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;        // room to align the base to 1 KB
@@ -91,6 +91,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     auto bar_p = [&](int m, int b) { return bar0 + 8 * (5 + 2 * kStages + 2 * m + b); };
     auto bar_o = [&](int m, int b) { return bar0 + 8 * (9 + 2 * kStages + 2 * m + b); };
     const uint32_t bar_final = bar0 + 8 * (13 + 2 * kStages);
+    const uint32_t bar_stage = bar0 + 8 * (14 + 2 * kStages);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::tmem_slot_off);
     __shared__ int s_abort;
 
@@ -128,6 +129,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 mbar_init(bar_o(m, bb), 1);
             }
         mbar_init(bar_final, 1);
+        mbar_init(bar_stage, 128 * n_mt);
         fence_mbar_init();
     }
     if (warp == 9) tmem_alloc(smem_u32(tmem_slot), 512);
@@ -323,25 +325,46 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (__any_sync(0xFFFFFFFFu, !ok)) ok = false;
         }
         if (ok) {
+            // O = acc / l through a swizzled shared-memory stage (the Q and
+            // K/V buffers are free once the last PV is done), then coalesced
+            // row stores.  Row rr of the stage is M-tile rr/128, row rr%128.
             tc_fence_after();
-            const bool store = head < a.G;
-            const int64_t row = ((b * a.Hq + g * a.G + head) * a.T_seg + qb * 64 + i);
+            float* stage = reinterpret_cast<float*>(smem + L::q_off);
+            const int sr_ = m * 128 + r;
             const float inv = 1.f / l_run;
-            float* orow = a.O + row * D;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t ov[32];
                 tmem_ld32(tmem + lane_off + col_o(m) + 32 * c, ov);
                 tmem_wait_ld();
-                if (store) {
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4*>(orow + 32 * c + j) =
-                            make_float4(__uint_as_float(ov[j]) * inv, __uint_as_float(ov[j + 1]) * inv,
-                                        __uint_as_float(ov[j + 2]) * inv, __uint_as_float(ov[j + 3]) * inv);
+                for (int j = 0; j < 32; j += 4) {
+                    const int ch = (32 * c + j) / 4;
+                    const int pch = (ch & ~7) | ((ch ^ sr_) & 7);
+                    *reinterpret_cast<float4*>(stage + sr_ * D + 4 * pch) =
+                        make_float4(__uint_as_float(ov[j]) * inv, __uint_as_float(ov[j + 1]) * inv,
+                                    __uint_as_float(ov[j + 2]) * inv, __uint_as_float(ov[j + 3]) * inv);
                 }
             }
-            if (store) a.lse[row] = (m_run + log2f(l_run)) * kLn2;
+            if (head < a.G) {
+                const int64_t row = ((b * a.Hq + g * a.G + head) * a.T_seg + qb * 64 + i);
+                a.lse[row] = (m_run + log2f(l_run)) * kLn2;
+            }
+            // All softmax threads have staged their rows (bounded wait).
+            mbar_arrive(bar_stage);
+            if (!mbar_wait(bar_stage, 0, kSiteStage)) s_abort = 1;
+            constexpr int C4 = D / 4;                      // 16-byte chunks per row
+            for (int rr = warp; rr < 128 * n_mt; rr += 4 * n_mt) {
+                const int hh = rr / 64;                    // head within the CTA
+                const int head_r = head0 + hh;
+                if (head_r >= a.G) continue;
+                const int64_t grow_ = (b * a.Hq + g * a.G + head_r) * a.T_seg + qb * 64 + (rr & 63);
+                for (int ch = lane; ch < C4; ch += 32) {
+                    const int pch = (ch & ~7) | ((ch ^ rr) & 7);
+                    *reinterpret_cast<float4*>(a.O + grow_ * D + 4 * ch) =
+                        *reinterpret_cast<const float4*>(stage + rr * D + 4 * pch);
+                }
+            }
         } else {
             s_abort = 1;
         }
