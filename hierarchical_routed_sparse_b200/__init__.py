@@ -10,10 +10,10 @@ buffers of one problem shape and runs a whole segment step.
 from .binding import (EXPORTS, HGA_ALL, HGA_BF16, HGA_ERR_CUDA, HGA_ERR_INVALID_ARG,
                       HGA_ERR_UNSUPPORTED, HGA_FP32, HGA_OK, LIB_PATH, NOALLOC_MAX_ROWS, Buffers,
                       HGAError, Params,
-                      attn_bwd, attn_bwd_noalloc, attn_fwd, build_summaries, device_status, load, route_chunks, route_groups,
+                      attn_bwd, attn_bwd_noalloc, attn_fwd, build_summaries, device_status, load, route, route_chunks, route_groups,
                       route_widths, version, workspace_size)
 
 __all__ = ["EXPORTS", "HGA_ALL", "HGA_BF16", "HGA_FP32", "HGA_OK", "HGA_ERR_CUDA",
            "HGA_ERR_INVALID_ARG", "HGA_ERR_UNSUPPORTED", "LIB_PATH", "NOALLOC_MAX_ROWS", "Buffers", "HGAError",
-           "Params", "attn_bwd", "attn_bwd_noalloc", "attn_fwd", "build_summaries", "device_status", "load", "route_chunks",
+           "Params", "attn_bwd", "attn_bwd_noalloc", "attn_fwd", "build_summaries", "device_status", "load", "route", "route_chunks",
            "route_groups", "route_widths", "version", "workspace_size"]

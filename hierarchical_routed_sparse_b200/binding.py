@@ -22,7 +22,7 @@ HGA_BF16, HGA_FP32 = 0, 1
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhga.so")
 
 EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_route_chunks",
-           "hga_route_groups", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
+           "hga_route_groups", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
            "hga_device_status", "hga_last_error", "hga_version")
 NOALLOC_MAX_ROWS = 1 << 20     # HGA_NOALLOC_MAX_ROWS
 
@@ -100,6 +100,7 @@ def load() -> ctypes.CDLL:
             "hga_build_summaries": ([PP, P, I64, I64, P, P, P], ctypes.c_int),
             "hga_route_chunks": ([PP, P, P, P, P, P], ctypes.c_int),
             "hga_route_groups": ([PP, P, P, P, P, P], ctypes.c_int),
+            "hga_route": ([PP, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_attn_fwd": ([PP, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_attn_bwd": ([PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P],
                              ctypes.c_int),
@@ -172,6 +173,12 @@ def route_groups(p: Params, qbar, gsum, cidx, gidx, stream=None) -> None:
                                    _ptr(gidx), _stream(stream)))
 
 
+def route(p: Params, Q, csum, gsum, qbar, cidx, gidx, stream=None) -> None:
+    """Block queries, chunk routing and group routing in one launch."""
+    _check(load().hga_route(ctypes.byref(p.c()), _ptr(Q), _ptr(csum), _ptr(gsum), _ptr(qbar), _ptr(cidx),
+                            _ptr(gidx), _stream(stream)))
+
+
 def attn_fwd(p: Params, Q, K, V, gidx, O, lse, stream=None) -> None:
     _check(load().hga_attn_fwd(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(gidx), _ptr(O),
                                _ptr(lse), _stream(stream)))
@@ -231,9 +238,12 @@ class Buffers:
         t_end = self.p.T if t_end is None else t_end
         build_summaries(self.p, K, t_begin, t_end, self.csum, self.gsum, stream)
 
-    def route(self, Q, stream=None):
-        route_chunks(self.p, Q, self.csum, self.qbar, self.cidx, stream)
-        route_groups(self.p, self.qbar, self.gsum, self.cidx, self.gidx, stream)
+    def route(self, Q, stream=None, fused=True):
+        if fused:
+            route(self.p, Q, self.csum, self.gsum, self.qbar, self.cidx, self.gidx, stream)
+        else:
+            route_chunks(self.p, Q, self.csum, self.qbar, self.cidx, stream)
+            route_groups(self.p, self.qbar, self.gsum, self.cidx, self.gidx, stream)
 
     def forward(self, Q, K, V, gidx=None, stream=None):
         attn_fwd(self.p, Q, K, V, self.gidx if gidx is None else gidx, self.O, self.lse, stream)

@@ -186,6 +186,25 @@ int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum, 
     return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route_groups");
 }
 
+int hga_route(const hga_params* p, const void* Q, const float* csum, const float* gsum, float* qbar,
+              int32_t* cidx, int32_t* gidx, hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    CHECK_PTR(Q);
+    CHECK_PTR(csum);
+    CHECK_PTR(gsum);
+    CHECK_PTR(qbar);
+    CHECK_PTR(cidx);
+    CHECK_PTR(gidx);
+    if (hga::route_fused_smem(s) > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "routing of %lld chunks / k_c=%d exceeds the router's shared memory",
+                    (long long)s.nC, s.wc);
+    cudaError_t e = hga::launch_route_fused(s, Q, csum, gsum, qbar, cidx, gidx, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route");
+}
+
 int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* V,
                  const int32_t* gidx, float* O, float* lse, hga_stream_t stream)
 {

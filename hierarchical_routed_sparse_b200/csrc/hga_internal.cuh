@@ -84,6 +84,9 @@ cudaError_t launch_route_chunks(const Shape& s, const void* Q, const float* csum
                                 int32_t* cidx, cudaStream_t st);
 cudaError_t launch_route_groups(const Shape& s, const float* qbar, const float* gsum,
                                 const int32_t* cidx, int32_t* gidx, cudaStream_t st);
+cudaError_t launch_route_fused(const Shape& s, const void* Q, const float* csum, const float* gsum,
+                               float* qbar, int32_t* cidx, int32_t* gidx, cudaStream_t st);
+size_t route_fused_smem(const Shape& s);
 cudaError_t launch_attn_fwd_simt(const Shape& s, const void* Q, const void* K, const void* V,
                                  const int32_t* gidx, float* O, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Shape& s, const void* Q, const void* K, const void* V,

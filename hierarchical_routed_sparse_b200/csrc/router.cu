@@ -18,30 +18,122 @@ namespace hga {
 
 size_t route_chunks_smem(const Shape& s);
 size_t route_groups_smem(const Shape& s);
+size_t route_fused_smem(const Shape& s);
 
 namespace {
 
 constexpr int kRouterThreads = 256;
 constexpr int kRouterWarps = kRouterThreads / 32;
+constexpr int kBatch = 16;          // candidates a warp scores at once
 
-// Dot product of the block query in shared memory with one summary row, by
-// one warp: lane l owns elements [l*D/32, (l+1)*D/32).
-template <int D>
-__device__ __forceinline__ float warp_dot(const float* __restrict__ qs, const float* __restrict__ row,
-                                          int lane)
+// Scores of candidates 0..n-1 against the block query qs (shared memory):
+// score(c) = qs . row(c), written as a selection key into keys[c].  Warp w
+// takes batches of 16 candidates w, w+8, ...; for each batch every lane
+// issues its 16 coalesced loads (lane l holds elements [l*P, (l+1)*P) of each
+// row) before any arithmetic, so a batch costs one memory round trip, and
+// the 16 partial sums are reduced across the warp with 16 shuffles (each
+// step halves the values a lane carries).
+template <int D, typename RowFn>
+__device__ __forceinline__ void score_candidates(const float* __restrict__ qs, int n, RowFn row_of,
+                                                 unsigned long long* keys, int warp, int lane)
 {
     constexpr int P = D / 32;
-    float a = 0.f;
-    if constexpr (P == 4) {
-        const float4 r = __ldg(reinterpret_cast<const float4*>(row) + lane);
-        const float4 q = reinterpret_cast<const float4*>(qs)[lane];
-        a = r.x * q.x + r.y * q.y + r.z * q.z + r.w * q.w;
-    } else {
-        const float2 r = __ldg(reinterpret_cast<const float2*>(row) + lane);
-        const float2 q = reinterpret_cast<const float2*>(qs)[lane];
-        a = r.x * q.x + r.y * q.y;
+    float q[P];
+#pragma unroll
+    for (int e = 0; e < P; ++e) q[e] = qs[lane * P + e];
+    for (int base = warp * kBatch; base < n; base += kRouterWarps * kBatch) {
+        float v[kBatch];
+        int32_t id[kBatch];
+        float x[kBatch][P];
+#pragma unroll
+        for (int c = 0; c < kBatch; ++c) {
+            const int cc = base + c < n ? base + c : base;
+            const float* row;
+            id[c] = row_of(cc, row);
+            if constexpr (P == 4) {
+                const float4 t = __ldg(reinterpret_cast<const float4*>(row) + lane);
+                x[c][0] = t.x; x[c][1] = t.y; x[c][2] = t.z; x[c][3] = t.w;
+            } else {
+                const float2 t = __ldg(reinterpret_cast<const float2*>(row) + lane);
+                x[c][0] = t.x; x[c][1] = t.y;
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < kBatch; ++c) {
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < P; ++e) a = fmaf(x[c][e], q[e], a);
+            v[c] = a;
+        }
+        // Transpose-reduce: after the step with offset o the lane keeps the
+        // half of its values selected by its lane bit o.
+#pragma unroll
+        for (int o = 16, m = kBatch / 2; o >= 2; o >>= 1, m >>= 1) {
+            const bool up = lane & o;
+#pragma unroll
+            for (int c = 0; c < m; ++c) {
+                const float send = up ? v[c] : v[c + m];
+                const float keep = up ? v[c + m] : v[c];
+                v[c] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+            }
+        }
+        v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], 1);
+        // Lane l now holds the full score of candidate ((l >> 1) & 15) in
+        // bit order 16, 8, 4, 2 -> 8, 4, 2, 1.
+        const int c = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+        int32_t my_id = id[0];
+#pragma unroll
+        for (int k = 1; k < kBatch; ++k) my_id = c == k ? id[k] : my_id;
+        if ((lane & 1) == 0 && base + c < n) keys[base + c] = pack_key(v[0], my_id);
     }
-    return warp_sum(a);
+}
+
+// Block query into qs (and qbar[u]): the mean of the block's 64 queries over
+// the G q-heads of the kv-head.  Every thread owns one 16-byte column vector
+// and issues the loads of up to 8 of its rows before adding them.
+template <typename TIn, int D>
+__device__ __forceinline__ void block_query(const TIn* __restrict__ Q, float* __restrict__ qbar_row,
+                                            float* qs, float (*part)[D], int64_t b, int64_t g, int64_t qb,
+                                            int Hq, int G, int64_t T_seg, float inv_rows, int tid)
+{
+    constexpr int E = Vec16<TIn>::E;
+    constexpr int V16 = D / E;
+    constexpr int RL = kRouterThreads / V16;          // row lanes
+    const int v = tid % V16, rl = tid / V16;
+    const int rows = G * kChunk;
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (int r0 = rl; r0 < rows; r0 += 8 * RL) {
+        float x[8][E];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int r = r0 + q * RL;
+            if (r < rows) {
+                const int64_t h = (int64_t)g * G + r / kChunk;
+                Vec16<TIn>::load(Q + ((b * Hq + h) * T_seg + qb * kChunk + r % kChunk) * D + v * E, x[q]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) x[q][e] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] += x[q][e];
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) part[rl][v * E + e] = acc[e];
+    __syncthreads();
+    for (int col = tid; col < D; col += kRouterThreads) {
+        float a = 0.f;
+#pragma unroll 8
+        for (int r = 0; r < RL; ++r) a += part[r][col];
+        a *= inv_rows;
+        qs[col] = a;
+        qbar_row[col] = a;
+    }
+    __syncthreads();
 }
 
 // Write the selected candidates (key == 0 marks a selected slot) in
@@ -60,126 +152,73 @@ __device__ __forceinline__ void compact_selected(const unsigned long long* keys,
     for (int i = pos + lane; i < width; i += 32) out[i] = -1;
 }
 
-// ---- a2 + a3: one CTA per (batch, kv-head, query block) ----------------------
-template <typename TIn, int D>
-__global__ void __launch_bounds__(kRouterThreads)
-route_chunks_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum,
-                    float* __restrict__ qbar, int32_t* __restrict__ cidx,
-                    int Hq, int Hkv, int G, int64_t T_seg, int64_t nQB, int64_t nC,
-                    int64_t c_hist, int k_c, int wc, float inv_rows)
+// a3: chunk routing of one block: scores of the eligible chunks c < c0, then
+// a warp-level top-k (k rounds of a warp arg-max on warp 0; the winner's key
+// is cleared to 0, which marks it selected).  Writes the row to cidx_row and
+// (if not null) to crow_smem.
+template <int D>
+__device__ __forceinline__ void route_chunks_block(const float* qs, const float* __restrict__ cs, int c0, int k_c,
+                                                   int wc, unsigned long long* keys, int32_t* cidx_row,
+                                                   int32_t* crow_smem, int tid)
 {
-    constexpr int E = Vec16<TIn>::E;
-    constexpr int V16 = D / E;
-    constexpr int RL = kRouterThreads / V16;          // row lanes
-    extern __shared__ unsigned long long keys[];      // [nC]
-    __shared__ float part[RL][D];
-    __shared__ __align__(16) float qs[D];
-
-    const int64_t u = blockIdx.x;                      // ((b*Hkv)+g)*nQB + qb
-    const int64_t qb = u % nQB, bg = u / nQB;
-    const int64_t b = bg / Hkv, g = bg % Hkv;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-    // a2: block query = mean over G heads x 64 queries.
-    {
-        const int v = tid % V16, rl = tid / V16;
-        float acc[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = 0.f;
-        for (int r = rl; r < G * kChunk; r += RL) {
-            const int64_t h = g * G + r / kChunk;
-            const TIn* src = Q + ((b * Hq + h) * T_seg + qb * kChunk + r % kChunk) * D + v * E;
-            float x[E];
-            Vec16<TIn>::load(src, x);
-#pragma unroll
-            for (int e = 0; e < E; ++e) acc[e] += x[e];
-        }
-#pragma unroll
-        for (int e = 0; e < E; ++e) part[rl][v * E + e] = acc[e];
-    }
-    __syncthreads();
-    for (int col = tid; col < D; col += kRouterThreads) {
-        float a = 0.f;
-#pragma unroll 8
-        for (int r = 0; r < RL; ++r) a += part[r][col];
-        a *= inv_rows;
-        qs[col] = a;
-        qbar[u * D + col] = a;
-    }
-    __syncthreads();
-
-    // a3: scores of the eligible chunks c < c0 (strictly before the own chunk).
-    const int c0 = static_cast<int>(c_hist + qb);
-    int32_t* out = cidx + u * wc;
+    const int lane = tid & 31, warp = tid >> 5;
     if (k_c <= 0 || k_c >= c0) {                       // keep every eligible chunk
-        for (int i = tid; i < wc; i += kRouterThreads) out[i] = i < c0 ? i : -1;
+        for (int i = tid; i < wc; i += kRouterThreads) {
+            const int32_t v = i < c0 ? i : -1;
+            cidx_row[i] = v;
+            if (crow_smem) crow_smem[i] = v;
+        }
+        __syncthreads();
         return;
     }
-    const float* cs = csum + bg * nC * D;
-    for (int c = warp; c < c0; c += kRouterWarps) {
-        const float sc = warp_dot<D>(qs, cs + (int64_t)c * D, lane);
-        if (lane == 0) keys[c] = pack_key(sc, c);
+    score_candidates<D>(qs, c0, [&](int c, const float*& row) { row = cs + (int64_t)c * D; return c; }, keys,
+                        warp, lane);
+    __syncthreads();
+    if (warp == 0) {
+        for (int round = 0; round < k_c; ++round) {
+            unsigned long long best = 0ull;
+            for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
+            best = warp_max_u64(best);
+            __syncwarp();
+            if (lane == 0) keys[key_index(best)] = 0ull;
+            __syncwarp();
+        }
+        compact_selected(keys, nullptr, c0, cidx_row, wc, lane);
+        if (crow_smem) compact_selected(keys, nullptr, c0, crow_smem, wc, lane);
     }
     __syncthreads();
-    if (warp != 0) return;
-    // Warp-level top-k: k rounds of a warp arg-max; the winner's key is
-    // cleared to 0, which marks it selected.
-    for (int round = 0; round < k_c; ++round) {
-        unsigned long long best = 0ull;
-        for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
-        best = warp_max_u64(best);
-        __syncwarp();
-        if (lane == 0) keys[key_index(best)] = 0ull;
-        __syncwarp();
-    }
-    compact_selected(keys, nullptr, c0, out, wc, lane);
 }
 
-// ---- a4: one CTA per (batch, kv-head, query block) ---------------------------
+// a4: group routing of one block: the 8 groups of every chunk in crow (an
+// ascending prefix of valid chunks), scored and ranked; a candidate is kept
+// when fewer than k_g candidates beat it.
 template <int D>
-__global__ void __launch_bounds__(kRouterThreads)
-route_groups_kernel(const float* __restrict__ qbar, const float* __restrict__ gsum,
-                    const int32_t* __restrict__ cidx, int32_t* __restrict__ gidx,
-                    int64_t nQB, int64_t nG, int wc, int k_g, int wg)
+__device__ __forceinline__ void route_groups_block(const float* qs, const float* __restrict__ gs,
+                                                   const int32_t* crow, int wc, int k_g, int wg,
+                                                   unsigned long long* keys, int32_t* ids, uint8_t* flags,
+                                                   int* s_count, int32_t* gidx_row, int tid)
 {
-    extern __shared__ unsigned long long keys[];      // [8*wc], ids [8*wc], flags [8*wc]
-    int32_t* ids = reinterpret_cast<int32_t*>(keys + (size_t)kGroupsPerChunk * wc);
-    uint8_t* flags = reinterpret_cast<uint8_t*>(ids + (size_t)kGroupsPerChunk * wc);
-    __shared__ __align__(16) float qs[D];
-    __shared__ int n_valid;
-
-    const int64_t u = blockIdx.x;
-    const int64_t bg = u / nQB;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int32_t* crow = cidx + u * wc;
-
-    for (int col = tid; col < D; col += kRouterThreads) qs[col] = qbar[u * D + col];
+    const int lane = tid & 31, warp = tid >> 5;
     if (warp == 0) {                                   // valid chunks form a prefix
         int n = 0;
         for (int base = 0; base < wc; base += 32) {
             const int i = base + lane;
             n += __popc(__ballot_sync(0xFFFFFFFFu, i < wc && crow[i] >= 0));
         }
-        if (lane == 0) n_valid = n;
+        if (lane == 0) *s_count = n;
     }
     __syncthreads();
-    const int n = n_valid * kGroupsPerChunk;           // candidate groups
+    const int n = *s_count * kGroupsPerChunk;          // candidate groups
     for (int i = tid; i < n; i += kRouterThreads)
         ids[i] = crow[i / kGroupsPerChunk] * kGroupsPerChunk + i % kGroupsPerChunk;
-    int32_t* out = gidx + u * wg;
     __syncthreads();
     if (k_g <= 0 || k_g >= n) {                        // keep every candidate
-        for (int i = tid; i < wg; i += kRouterThreads) out[i] = i < n ? ids[i] : -1;
+        for (int i = tid; i < wg; i += kRouterThreads) gidx_row[i] = i < n ? ids[i] : -1;
         return;
     }
-    const float* gs = gsum + bg * nG * D;
-    for (int i = warp; i < n; i += kRouterWarps) {
-        const float sc = warp_dot<D>(qs, gs + (int64_t)ids[i] * D, lane);
-        if (lane == 0) keys[i] = pack_key(sc, ids[i]);
-    }
+    score_candidates<D>(qs, n, [&](int c, const float*& row) { row = gs + (int64_t)ids[c] * D; return ids[c]; },
+                        keys, warp, lane);
     __syncthreads();
-    // Rank selection: a candidate is kept when fewer than k_g keys beat it.
-    // Flags are gathered first, then written as key 0 for the compaction.
     for (int i = tid; i < n; i += kRouterThreads) {
         const unsigned long long ki = keys[i];
         int rank = 0;
@@ -190,7 +229,75 @@ route_groups_kernel(const float* __restrict__ qbar, const float* __restrict__ gs
     for (int i = tid; i < n; i += kRouterThreads)
         if (flags[i]) keys[i] = 0ull;
     __syncthreads();
-    if (warp == 0) compact_selected(keys, ids, n, out, wg, lane);
+    if (warp == 0) compact_selected(keys, ids, n, gidx_row, wg, lane);
+}
+
+// ---- a2 + a3: one CTA per (batch, kv-head, query block) ----------------------
+template <typename TIn, int D>
+__global__ void __launch_bounds__(kRouterThreads, 2)
+route_chunks_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum,
+                    float* __restrict__ qbar, int32_t* __restrict__ cidx,
+                    int Hq, int Hkv, int G, int64_t T_seg, int64_t nQB, int64_t nC,
+                    int64_t c_hist, int k_c, int wc, float inv_rows)
+{
+    constexpr int RL = kRouterThreads / (D / Vec16<TIn>::E);
+    extern __shared__ unsigned long long keys[];      // [nC]
+    __shared__ float part[RL][D];
+    __shared__ __align__(16) float qs[D];
+    const int64_t u = blockIdx.x;                      // ((b*Hkv)+g)*nQB + qb
+    const int64_t qb = u % nQB, bg = u / nQB;
+    const int64_t b = bg / Hkv, g = bg % Hkv;
+    block_query<TIn, D>(Q, qbar + u * D, qs, part, b, g, qb, Hq, G, T_seg, inv_rows, threadIdx.x);
+    route_chunks_block<D>(qs, csum + bg * nC * D, static_cast<int>(c_hist + qb), k_c, wc, keys, cidx + u * wc,
+                          nullptr, threadIdx.x);
+}
+
+// ---- a4: one CTA per (batch, kv-head, query block) ---------------------------
+template <int D>
+__global__ void __launch_bounds__(kRouterThreads, 2)
+route_groups_kernel(const float* __restrict__ qbar, const float* __restrict__ gsum,
+                    const int32_t* __restrict__ cidx, int32_t* __restrict__ gidx,
+                    int64_t nQB, int64_t nG, int wc, int k_g, int wg)
+{
+    extern __shared__ unsigned long long keys[];      // [8*wc], ids [8*wc], flags [8*wc]
+    int32_t* ids = reinterpret_cast<int32_t*>(keys + (size_t)kGroupsPerChunk * wc);
+    uint8_t* flags = reinterpret_cast<uint8_t*>(ids + (size_t)kGroupsPerChunk * wc);
+    __shared__ __align__(16) float qs[D];
+    __shared__ int n_valid;
+    const int64_t u = blockIdx.x;
+    const int64_t bg = u / nQB;
+    for (int col = threadIdx.x; col < D; col += kRouterThreads) qs[col] = qbar[u * D + col];
+    __syncthreads();
+    route_groups_block<D>(qs, gsum + bg * nG * D, cidx + u * wc, wc, k_g, wg, keys, ids, flags, &n_valid,
+                          gidx + u * wg, threadIdx.x);
+}
+
+// ---- a2 + a3 + a4 in one launch ------------------------------------------------
+template <typename TIn, int D>
+__global__ void __launch_bounds__(kRouterThreads, 2)
+route_fused_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, const float* __restrict__ gsum,
+                   float* __restrict__ qbar, int32_t* __restrict__ cidx, int32_t* __restrict__ gidx,
+                   int Hq, int Hkv, int G, int64_t T_seg, int64_t nQB, int64_t nC, int64_t nG,
+                   int64_t c_hist, int k_c, int wc, int k_g, int wg, float inv_rows)
+{
+    constexpr int RL = kRouterThreads / (D / Vec16<TIn>::E);
+    // keys [max(nC, 8*wc)], ids [8*wc], flags [8*wc], crow [wc]
+    extern __shared__ unsigned long long keys[];
+    const size_t nk = (size_t)(nC > kGroupsPerChunk * wc ? nC : kGroupsPerChunk * wc);
+    int32_t* ids = reinterpret_cast<int32_t*>(keys + nk);
+    int32_t* crow = ids + (size_t)kGroupsPerChunk * wc;
+    uint8_t* flags = reinterpret_cast<uint8_t*>(crow + wc);
+    __shared__ float part[RL][D];
+    __shared__ __align__(16) float qs[D];
+    __shared__ int n_valid;
+    const int64_t u = blockIdx.x;
+    const int64_t qb = u % nQB, bg = u / nQB;
+    const int64_t b = bg / Hkv, g = bg % Hkv;
+    block_query<TIn, D>(Q, qbar + u * D, qs, part, b, g, qb, Hq, G, T_seg, inv_rows, threadIdx.x);
+    route_chunks_block<D>(qs, csum + bg * nC * D, static_cast<int>(c_hist + qb), k_c, wc, keys, cidx + u * wc,
+                          crow, threadIdx.x);
+    route_groups_block<D>(qs, gsum + bg * nG * D, crow, wc, k_g, wg, keys, ids, flags, &n_valid, gidx + u * wg,
+                          threadIdx.x);
 }
 
 template <typename TIn, int D>
@@ -226,7 +333,41 @@ cudaError_t launch_rg(const Shape& s, const float* qbar, const float* gsum, cons
     return cudaGetLastError();
 }
 
+template <typename TIn, int D>
+cudaError_t launch_rf(const Shape& s, const void* Q, const float* csum, const float* gsum, float* qbar,
+                      int32_t* cidx, int32_t* gidx, cudaStream_t st)
+{
+    const size_t smem = route_fused_smem(s);
+    auto k = route_fused_kernel<TIn, D>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t blocks = (int64_t)s.B * s.Hkv * s.nQB;
+    k<<<(unsigned)blocks, kRouterThreads, smem, st>>>(
+        static_cast<const TIn*>(Q), csum, gsum, qbar, cidx, gidx, s.Hq, s.Hkv, s.G, s.T_seg, s.nQB, s.nC, s.nG,
+        s.T_hist / kChunk, s.k_c, s.wc, s.k_g, s.wg, 1.0f / (float)(s.G * kChunk));
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+size_t route_fused_smem(const Shape& s)
+{
+    const size_t nk = (size_t)(s.nC > kGroupsPerChunk * (int64_t)s.wc ? s.nC : kGroupsPerChunk * (int64_t)s.wc);
+    return sizeof(unsigned long long) * nk + (sizeof(int32_t) + 1) * kGroupsPerChunk * (size_t)s.wc +
+           sizeof(int32_t) * (size_t)s.wc;
+}
+
+cudaError_t launch_route_fused(const Shape& s, const void* Q, const float* csum, const float* gsum, float* qbar,
+                               int32_t* cidx, int32_t* gidx, cudaStream_t st)
+{
+    if (s.dtype == HGA_BF16)
+        return s.d == 128 ? launch_rf<__nv_bfloat16, 128>(s, Q, csum, gsum, qbar, cidx, gidx, st)
+                          : launch_rf<__nv_bfloat16, 64>(s, Q, csum, gsum, qbar, cidx, gidx, st);
+    return s.d == 128 ? launch_rf<float, 128>(s, Q, csum, gsum, qbar, cidx, gidx, st)
+                      : launch_rf<float, 64>(s, Q, csum, gsum, qbar, cidx, gidx, st);
+}
 
 size_t route_chunks_smem(const Shape& s) { return sizeof(unsigned long long) * (size_t)s.nC; }
 size_t route_groups_smem(const Shape& s)

@@ -114,6 +114,13 @@ int hga_route_chunks(const hga_params* p, const void* Q, const float* csum,
 int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum,
                      const int32_t* cidx, int32_t* gidx, hga_stream_t stream);
 
+/* a2 + a3 + a4 in one launch: the same qbar, cidx and gidx as
+ * hga_route_chunks followed by hga_route_groups (bit for bit), without the
+ * round trip of qbar and cidx through device memory between the stages. */
+int hga_route(const hga_params* p, const void* Q, const float* csum,
+              const float* gsum, float* qbar, int32_t* cidx, int32_t* gidx,
+              hga_stream_t stream);
+
 /* a5. Routed attention forward (same section: only the exact token K/V of
  * the selected groups is loaded for the attention).  Query i of block qb
  * (global position p = T_hist + 64 qb + i) of q-head h attends the 8 tokens

@@ -183,3 +183,21 @@ def test_sweep_sampled_units(w):
         # wherever its routing matched.
         if (got_g == orc["gidx"]).all():
             assert maxabs(buf.O[b:b + 1, g * G:(g + 1) * G].cpu().numpy(), orc["O"]) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[3], W.QWEN3_CTX16K_FWD], ids=lambda w: w.name)
+def test_fused_router_equals_separate_calls(w):
+    """hga_route gives bit for bit the outputs of hga_route_chunks followed by
+    hga_route_groups."""
+    x = w.full()
+    p = hga.Params.from_workload(w)
+    Q, K = to_dev(x["Q"], w.dtype), to_dev(x["K"], w.dtype)
+    a, b = hga.Buffers(p), hga.Buffers(p)
+    a.summaries(K, 0, w.T)
+    b.summaries(K, 0, w.T)
+    a.route(Q, fused=True)
+    b.route(Q, fused=False)
+    torch.cuda.synchronize()
+    assert torch.equal(a.qbar, b.qbar)
+    assert torch.equal(a.cidx, b.cidx)
+    assert torch.equal(a.gidx, b.gidx)
