@@ -21,9 +21,10 @@
 // atomics; tiles whose keys are all detached history skip both products
 // (routed groups are ascending, so history tiles come first).
 //
-// Warp roles (320 threads): warps 0-7 compute P and dS (row 32*(w%4)+lane,
-// key half w/4), add the previous tile's dK/dV while the MMAs of the current
-// one run, and write dQ at the end; warp 8 is the TMA producer, warp 9 the
+// Warp roles (576 threads): warps 0-15 compute P and dS (row 32*(w%4)+lane,
+// 16-key quarter w/4; four warps per scheduler hide each other's latency),
+// add the previous tile's dK/dV while the MMAs of the current one run, and
+// write dQ at the end; warp 16 is the TMA producer, warp 17 the
 // tensor-memory owner and MMA issuer.  Tensor memory (512 columns): S and dP
 // double-buffered (4 x 64), dQ (128), dV^T (64), dK^T (64).  Three K/V
 // stages (224 KB of shared memory in all) keep the gathered loads two tiles
@@ -42,7 +43,10 @@ constexpr int D = 128;
 constexpr int H = 2;                  // 64-column halves of d
 constexpr int kStages = 3;
 constexpr int kKeys = 64;
-constexpr int kThreads = 320;
+constexpr int kComputeWarps = 16;     // 4 per lane quadrant, one 16-key quarter each
+constexpr int kCompute = 32 * kComputeWarps;
+constexpr int kProducerWarp = kComputeWarps, kMmaWarp = kComputeWarps + 1;
+constexpr int kThreads = 32 * (kComputeWarps + 2);
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int {
@@ -184,22 +188,22 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         mbar_init(bar_sdp(0), 1);
         mbar_init(bar_sdp(1), 1);
-        mbar_init(bar_ps, 256);
+        mbar_init(bar_ps, kCompute);
         mbar_init(bar_mm2, 1);
-        mbar_init(bar_drained, 256);
+        mbar_init(bar_drained, kCompute);
         mbar_init(bar_final, 1);
         mbar_init(bar_qfree, 1);
-        mbar_init(bar_dqfree, 256);
-        mbar_init(bar_stage, 256);
+        mbar_init(bar_dqfree, kCompute);
+        mbar_init(bar_stage, kCompute);
         fence_mbar_init();
     }
-    if (warp == 9) tmem_alloc(smem_u32(tmem_slot), 512);
+    if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tm_q);
@@ -277,7 +281,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (last_gt[s] >= 0) mbar_wait(bar_full(s), (last_gt[s] / kStages) & 1, kSiteDrain);
             if (k_loaded >= 0) mbar_wait(bar_q, k_loaded & 1, kSiteDrain);
         }
-    } else if (warp == 9) {
+    } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
         constexpr uint32_t id_sdp = idesc_bf16(128, kKeys, 0, 0);   // S, dP
         constexpr uint32_t id_dq = idesc_bf16(128, D, 0, 1);        // dQ: A dS K-major, B K MN-major
@@ -362,8 +366,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     } else {
         // ------------- P and dS, then the dK / dV atomics and the dQ epilogue
         // Thread (warp w, lane l): query row r = 32*(w%4) + l of the M-tile
-        // (its tensor-memory lane) and the 32-key half kh = w/4 of each tile.
-        const int r = (warp % 4) * 32 + lane, kh = warp / 4;
+        // (its tensor-memory lane) and the 16-key quarter kq = w/4 of each tile.
+        const int r = (warp % 4) * 32 + lane, kq = warp / 4;
         const int i = r & 63, hp = r >> 6;
         const uint32_t lane_off = uint32_t((warp % 4) * 32) << 16;
         uint8_t* prow_hi = smem + L::p_off + r * 128;
@@ -371,24 +375,24 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         uint8_t* srow_hi = smem + L::ds_off + r * 128;
         uint8_t* srow_lo = srow_hi + L::kRows128;
         // dV^T / dK^T of tile te of item m (d = tensor-memory lane r, keys of
-        // half kh) added to the segment's rows; history keys and padding are
-        // skipped.
+        // quarter kq) added to the segment's rows; history keys and padding
+        // are skipped.
         auto dkv_epilogue = [&](const Item& m, int te) {
             if (!item_tile_has_segment_keys(m, te, a.T_hist)) return;
             tc_fence_after();
-            uint32_t vv[32], kv[32];
-            tmem_ld32(tmem + lane_off + kColDV + 32 * kh, vv);
-            tmem_ld32(tmem + lane_off + kColDK + 32 * kh, kv);
+            uint32_t vv[16], kv[16];
+            tmem_ld16(tmem + lane_off + kColDV + 16 * kq, vv);
+            tmem_ld16(tmem + lane_off + kColDK + 16 * kq, kv);
             tmem_wait_ld();
             const bool own = te == m.n_rt;
-            int64_t gbase[4];                               // first token of each group slot
+            int64_t gbase[2];                               // first token of each group slot
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int gi = te * 8 + 4 * kh + q;
-                gbase[q] = own ? m.own_start + 32 * kh + 8 * q : (gi < m.n_g ? (int64_t)__ldg(m.grow + gi) * 8 : -64);
+            for (int q = 0; q < 2; ++q) {
+                const int gi = te * 8 + 2 * kq + q;
+                gbase[q] = own ? m.own_start + 16 * kq + 8 * q : (gi < m.n_g ? (int64_t)__ldg(m.grow + gi) * 8 : -64);
             }
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < 16; ++j) {
                 const int64_t key = gbase[j / 8] + j % 8;
                 if (key < a.T_hist) continue;               // padding or detached history
                 const int64_t o = (m.bg * a.T_seg + (key - a.T_hist)) * D + r;
@@ -429,19 +433,19 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const bool own = t == m.n_rt;
                 // P is an MMA operand only for dV, i.e. for tiles holding segment keys.
                 const bool seg = item_tile_has_segment_keys(m, t, a.T_hist);
-                uint32_t sr[32], pr[32];
-                tmem_ld32(tmem + lane_off + kColS + bb * kKeys + 32 * kh, sr);
-                tmem_ld32(tmem + lane_off + kColDP + bb * kKeys + 32 * kh, pr);
+                uint32_t sr[16], pr[16];
+                tmem_ld16(tmem + lane_off + kColS + bb * kKeys + 16 * kq, sr);
+                tmem_ld16(tmem + lane_off + kColDP + bb * kKeys + 16 * kq, pr);
                 tmem_wait_ld();
-                uint32_t ph[16], pl[16], dh[16], dl[16];
+                uint32_t ph[8], pl[8], dh[8], dl[8];
                 // Every key of a full routed tile is valid for every row:
                 // no masks there; partial tiles and the own chunk mask keys.
                 const bool full = row_ok && !own && t * 8 + 8 <= m.n_g;
                 const float2 c2 = make_float2(a.scale_log2, a.scale_log2);
                 const float2 l2 = make_float2(-lse2, -lse2), d2 = make_float2(-Dr, -Dr);
 #pragma unroll
-                for (int j2 = 0; j2 < 16; ++j2) {
-                    const int j0 = 32 * kh + 2 * j2;
+                for (int j2 = 0; j2 < 8; ++j2) {
+                    const int j0 = 16 * kq + 2 * j2;
                     const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1])),
                                                 c2, l2);
                     float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
@@ -463,13 +467,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 // Row r, 16-byte chunk c lives at chunk c ^ (r % 8) (128-byte swizzle).
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const int pc = ((4 * kh + c4) ^ (r & 7)) * 16;
-                    *reinterpret_cast<uint4*>(srow_hi + pc) = make_uint4(dh[4 * c4], dh[4 * c4 + 1], dh[4 * c4 + 2], dh[4 * c4 + 3]);
-                    *reinterpret_cast<uint4*>(srow_lo + pc) = make_uint4(dl[4 * c4], dl[4 * c4 + 1], dl[4 * c4 + 2], dl[4 * c4 + 3]);
+                for (int c2i = 0; c2i < 2; ++c2i) {
+                    const int pc = ((2 * kq + c2i) ^ (r & 7)) * 16;
+                    *reinterpret_cast<uint4*>(srow_hi + pc) = make_uint4(dh[4 * c2i], dh[4 * c2i + 1], dh[4 * c2i + 2], dh[4 * c2i + 3]);
+                    *reinterpret_cast<uint4*>(srow_lo + pc) = make_uint4(dl[4 * c2i], dl[4 * c2i + 1], dl[4 * c2i + 2], dl[4 * c2i + 3]);
                     if (seg) {
-                        *reinterpret_cast<uint4*>(prow_hi + pc) = make_uint4(ph[4 * c4], ph[4 * c4 + 1], ph[4 * c4 + 2], ph[4 * c4 + 3]);
-                        *reinterpret_cast<uint4*>(prow_lo + pc) = make_uint4(pl[4 * c4], pl[4 * c4 + 1], pl[4 * c4 + 2], pl[4 * c4 + 3]);
+                        *reinterpret_cast<uint4*>(prow_hi + pc) = make_uint4(ph[4 * c2i], ph[4 * c2i + 1], ph[4 * c2i + 2], ph[4 * c2i + 3]);
+                        *reinterpret_cast<uint4*>(prow_lo + pc) = make_uint4(pl[4 * c2i], pl[4 * c2i + 1], pl[4 * c2i + 2], pl[4 * c2i + 3]);
                     }
                 }
                 fence_async_smem();
@@ -495,14 +499,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_arrive(bar_drained);
             tc_fence_after();
             // dQ (times the softmax scale): tensor memory -> swizzled shared rows.
-#pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
+            {
                 uint32_t v[32];
-                tmem_ld32(tmem + lane_off + kColDQ + 64 * kh + 32 * c, v);
+                tmem_ld32(tmem + lane_off + kColDQ + 32 * kq, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
-                    const int ch = (64 * kh + 32 * c + j) / 4;     // 16-byte chunk of the row
+                    const int ch = (32 * kq + j) / 4;              // 16-byte chunk of the row
                     const int pch = (ch & ~7) | ((ch ^ r) & 7);
                     *reinterpret_cast<float4*>(stage + r * D + 4 * pch) =
                         make_float4(__uint_as_float(v[j]) * a.scale, __uint_as_float(v[j + 1]) * a.scale,
@@ -511,11 +514,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             tc_fence_before();
             mbar_arrive(bar_dqfree);
-            // All 256 compute threads have staged their dQ parts (bounded wait).
+            // All compute threads have staged their dQ parts (bounded wait).
             mbar_arrive(bar_stage);
             if (!mbar_wait(bar_stage, (2 * k) & 1, kSiteStage)) { ok = false; break; }
-            // Coalesced rows: warp w writes rows w, w+8, ...; lane l the l-th 16 bytes.
-            for (int rr = warp; rr < 128; rr += 8) {
+            // Coalesced rows: warp w writes rows w, w+16, ...; lane l the l-th 16 bytes.
+            for (int rr = warp; rr < 128; rr += kComputeWarps) {
                 const int head = m.head0 + (rr >> 6);
                 if (head >= a.G) continue;
                 const int64_t grow_ = (m.b * a.Hq + m.g * a.G + head) * a.T_seg + m.qb * 64 + (rr & 63);
@@ -537,7 +540,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
