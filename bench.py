@@ -252,10 +252,11 @@ def whole_job_rate(tokens_per_rank_step: int, steps: int, world: int, max_ms: fl
     return world * steps * tokens_per_rank_step / (max_ms * 1e-3)
 
 
-def config_of(w) -> dict:
+def config_of(w, graph: bool = True) -> dict:
     return dict(workload=w.name, B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T_hist=w.T_hist,
                 T_seg=w.T_seg, T=w.T, k_c=w.k_c, k_g=w.k_g, keys=w.keys,
-                l2="flushed between timed steps (256 MiB write)")
+                l2="flushed between timed steps (256 MiB write)",
+                launch="CUDA graph of the step" if graph else "eager")
 
 
 def run_reference(args, w) -> None:
@@ -300,28 +301,58 @@ def run_gpu(args, w) -> None:
 
     stages = ["summaries", "route", "attn_fwd", "attn_bwd"]
 
-    def step(ev=None):
+    def step_on(st, ev=None):
         if ev is not None:
-            ev[0].record(stream)
-        buf.summaries(K, stream=stream)
+            ev[0].record(st)
+        buf.summaries(K, stream=st)
         if ev is not None:
-            ev[1].record(stream)
-        buf.route(Q, stream)
+            ev[1].record(st)
+        buf.route(Q, st)
         if ev is not None:
-            ev[2].record(stream)
-        buf.forward(Q, K, V, stream=stream)
+            ev[2].record(st)
+        buf.forward(Q, K, V, stream=st)
         if ev is not None:
-            ev[3].record(stream)
+            ev[3].record(st)
         if dO is not None:
-            buf.backward(Q, K, V, dO, stream=stream)
+            buf.backward(Q, K, V, dO, stream=st)
         if ev is not None:
-            ev[4].record(stream)
+            ev[4].record(st)
+
+    def step(ev=None):
+        step_on(stream, ev)
 
     for _ in range(args.warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # Events recorded inside a captured graph must be "external" to be timed
+    # from outside it.
+    events = [[torch.cuda.Event(enable_timing=True, external=not args.no_graph) for _ in range(5)]
+              for _ in range(args.steps)]
+    run_step = step
+    if not args.no_graph:
+        # One segment step captured as a CUDA graph (with its stage events),
+        # replayed per timed step: the device time of the kernels themselves,
+        # without host launch gaps between them.
+        graphs = []
+        cap_stream = torch.cuda.Stream(dev)
+        cap_stream.wait_stream(stream)
+        with torch.cuda.stream(cap_stream):
+            for i in range(args.steps):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap_stream):
+                    step_on(cap_stream, events[i])
+                graphs.append(g)
+        stream.wait_stream(cap_stream)
+        torch.cuda.synchronize()
+        for _ in range(args.warmup):
+            flush.zero_()
+            graphs[0].replay()
+        torch.cuda.synchronize()
+
+        def run_step(ev, i=[0]):
+            graphs[i[0] % len(graphs)].replay()
+            i[0] += 1
     clocks_path = os.path.join(ROOT, "gpurun_out", "clocks.csv") if os.path.isdir(
         os.path.join(ROOT, "gpurun_out")) else None
     if world > 1:
@@ -330,7 +361,7 @@ def run_gpu(args, w) -> None:
     with ClockSampler(local, clocks_path) as clk:
         for i in range(args.steps):
             flush.zero_()                            # outside the timed events
-            step(events[i])
+            run_step(events[i])
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -402,7 +433,7 @@ def run_gpu(args, w) -> None:
         line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype=w.dtype, data="synthetic",
-                    config=config_of(w), stage_ms=stage_ms, roofline=roof,
+                    config=config_of(w, not args.no_graph), stage_ms=stage_ms, roofline=roof,
                     gpu_launches=(LAUNCHES_PER_STEP if w.backward else 4) * args.steps,
                     e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d,
                              d2h_bytes_per_step=d2h),
@@ -425,6 +456,8 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=10.0,
                     help="seconds of oracle work in the CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager launches instead of a CUDA graph of the step")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu DRAM bytes per launch of the dominant kernel, if captured")
     args = ap.parse_args()
