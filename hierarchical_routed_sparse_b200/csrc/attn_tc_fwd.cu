@@ -19,9 +19,8 @@
 // 2^8 (then O is rescaled in TMEM); any fixed reference point gives the same
 // O / l, and it spares most rescales.
 //
-// Warp roles (576 threads): warps 0-7 softmax of M-tile 0 and warps 8-15 of
-// M-tile 1 (two warps per row quadrant, one per 32-key half), warp 16 TMA
-// producer, warp 17 tensor-memory owner and MMA issuer.
+// Warp roles (320 threads): warps 0-3 softmax of M-tile 0, warps 4-7 of
+// M-tile 1, warp 8 TMA producer, warp 9 tensor-memory owner and MMA issuer.
 // Tensor memory (512 columns): O of each M-tile (D columns), and two S/P
 // buffers of 64 columns per M-tile so that S of the next key tile is computed
 // while the softmax works on the current one.
@@ -36,16 +35,14 @@ using namespace sm100;
 
 constexpr int kStages = 3;          // K/V tiles in flight
 constexpr int kKeys = 64;           // keys per tile
-constexpr int kSoftmaxWarps = 16;     // per M-tile: 4 lane quadrants x 2 key halves
-constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
-constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+constexpr int kThreads = 320;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;
 
 // Status codes of the bounded waits (site of the wait that ran out).
 enum : int {
-    kSiteQ = 101, kSiteFull, kSiteEmpty, kSiteS, kSiteP, kSiteO, kSiteFinal, kSiteDrain, kSiteStage, kSiteX
+    kSiteQ = 101, kSiteFull, kSiteEmpty, kSiteS, kSiteP, kSiteO, kSiteFinal, kSiteDrain, kSiteStage
 };
 
 template <int D>
@@ -57,12 +54,9 @@ struct FwdSmem {
     static constexpr int k_off = q_off + 2 * H * kQTile;
     static constexpr int v_off = k_off + kStages * H * kKVHalf;
     static constexpr int bar_off = v_off + kStages * H * kKVHalf;
-    // barriers: q, full[S], empty[S], s[2][2], p[2][2], o[2][2], final, stage, x[2]
-    static constexpr int n_bars = 1 + 2 * kStages + 4 + 4 + 4 + 2 + 2;
-    // row-maximum / row-sum exchange between the two key halves of a row:
-    // [tile parity][M-tile][half][128 rows] floats
-    static constexpr int x_off = bar_off + 8 * n_bars;
-    static constexpr int tmem_slot_off = x_off + 4 * 2 * 2 * 2 * 128;
+    // barriers: q, full[S], empty[S], s[2][2], p[2][2], o[2][2], final, stage
+    static constexpr int n_bars = 1 + 2 * kStages + 4 + 4 + 4 + 2;
+    static constexpr int tmem_slot_off = bar_off + 8 * n_bars;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;        // room to align the base to 1 KB
 };
@@ -98,8 +92,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     auto bar_o = [&](int m, int b) { return bar0 + 8 * (9 + 2 * kStages + 2 * m + b); };
     const uint32_t bar_final = bar0 + 8 * (13 + 2 * kStages);
     const uint32_t bar_stage = bar0 + 8 * (14 + 2 * kStages);
-    auto bar_x = [&](int m) { return bar0 + 8 * (15 + 2 * kStages + m); };
-    float* xbuf = reinterpret_cast<float*>(smem + L::x_off);   // [2][2][2][128]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::tmem_slot_off);
     __shared__ int s_abort;
 
@@ -133,16 +125,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int m = 0; m < 2; ++m)
             for (int bb = 0; bb < 2; ++bb) {
                 mbar_init(bar_s(m, bb), 1);
-                mbar_init(bar_p(m, bb), 256);
+                mbar_init(bar_p(m, bb), 128);
                 mbar_init(bar_o(m, bb), 1);
             }
         mbar_init(bar_final, 1);
-        mbar_init(bar_stage, 256 * n_mt);
-        mbar_init(bar_x(0), 256);
-        mbar_init(bar_x(1), 256);
+        mbar_init(bar_stage, 128 * n_mt);
         fence_mbar_init();
     }
-    if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
+    if (warp == 9) tmem_alloc(smem_u32(tmem_slot), 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -156,7 +146,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     const int64_t kv_base = bg * (a.T_hist + a.T_seg);      // first K/V row of (b, g)
 
-    if (warp == kProducerWarp) {
+    if (warp == 8) {
         // ------------------------------------------------------------ producer
         // Lane 0 issues the Q boxes and arms the barriers; for a routed tile,
         // lane j < 8 fetches group j's index and issues that group's boxes,
@@ -211,7 +201,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             __syncwarp();
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_bf16(128, kKeys, 0, 0);
@@ -259,17 +249,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mma_commit(bar_final);
             mbar_wait(bar_final, 0, kSiteFinal);
         }
-    } else if (warp / 8 < n_mt) {
+    } else if (warp / 4 < n_mt) {
         // ------------------------------------------------ softmax + epilogue
-        // Warp w: M-tile m = w/8, key half h = (w/4)%2 (keys 32h..32h+31 of
-        // every tile), lane quadrant w%4 (rows 32*(w%4) .. +31).  The two
-        // halves of a row agree on its running maximum through xbuf once per
-        // key tile and add their partial row sums at the end.
-        const int m = warp / 8, h = (warp / 4) % 2, r = (warp % 4) * 32 + lane;
+        const int m = warp / 4, r = threadIdx.x % 128;     // row of the M-tile
         const int i = r & 63, hp = r >> 6;                 // query in block, head in pair
         const int head = head0 + 2 * m + hp;
         const uint32_t lane_off = uint32_t((warp % 4) * 32) << 16;
-        auto xslot = [&](int parity, int half) { return xbuf + ((parity * 2 + m) * 2 + half) * 128 + r; };
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int t = 0; t < nt && ok; ++t) {
@@ -277,27 +262,23 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ok = mbar_wait(bar_s(m, bb), (t / 2) & 1, kSiteS);
             if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
             tc_fence_after();
-            uint32_t raw[32];
-            tmem_ld32(tmem + lane_off + col_s(m, bb) + 32 * h, raw);
+            uint32_t raw[2][32];
+            tmem_ld32(tmem + lane_off + col_s(m, bb), raw[0]);
+            tmem_ld32(tmem + lane_off + col_s(m, bb) + 32, raw[1]);
             tmem_wait_ld();
-            float sv[32];
+            float sv[64];
             float mx = -INFINITY;
             const bool own = t == n_rt;
             // Full routed tiles need no masks; the scale is applied after the
             // maximum (it is positive) and folded into the exponent's FMA.
             const bool full = !own && t * 8 + 8 <= n_g;
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) {
-                const int j = 32 * h + jj;
-                sv[jj] = __uint_as_float(raw[jj]);
-                if (!full && !(own ? (j <= i) : (t * 8 + j / 8 < n_g))) sv[jj] = -INFINITY;
-                mx = fmaxf(mx, sv[jj]);
+            for (int j = 0; j < 64; ++j) {
+                sv[j] = __uint_as_float(raw[j / 32][j % 32]);
+                if (!full && !(own ? (j <= i) : (t * 8 + j / 8 < n_g))) sv[j] = -INFINITY;
+                mx = fmaxf(mx, sv[j]);
             }
-            *xslot(t & 1, h) = mx;
-            mbar_arrive(bar_x(m));
-            ok = mbar_wait(bar_x(m), t & 1, kSiteX);
-            if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
-            mx = fmaxf(mx, *xslot(t & 1, 1 - h)) * a.scale_log2;
+            mx *= a.scale_log2;
             const bool need = mx > m_run + kRescaleLog2;
             if (__any_sync(0xFFFFFFFFu, need)) {
                 const float m_new = need ? mx : m_run;
@@ -307,13 +288,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll 1
-                    for (int c = 0; c < D / 64; ++c) {           // this half's columns of O
+                    for (int c = 0; c < D / 32; ++c) {
                         uint32_t ov[32];
-                        tmem_ld32(tmem + lane_off + col_o(m) + (D / 2) * h + 32 * c, ov);
+                        tmem_ld32(tmem + lane_off + col_o(m) + 32 * c, ov);
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-                        tmem_st32(tmem + lane_off + col_o(m) + (D / 2) * h + 32 * c, ov);
+                        tmem_st32(tmem + lane_off + col_o(m) + 32 * c, ov);
                     }
                     tmem_wait_st();
                 }
@@ -322,19 +303,19 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             // P = hi + lo, both bf16: the two MMAs carry P to ~14 bits, where
             // one bf16 operand alone (8 bits) misses the 2e-3 output bound.
-            uint32_t pk_hi[16], pk_lo[16];
+            uint32_t pk_hi[32], pk_lo[32];
             float2 rs = make_float2(0.f, 0.f);
             const float2 c2 = make_float2(a.scale_log2, a.scale_log2), nm = make_float2(-m_run, -m_run);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 32; ++j) {
                 const float2 x = __ffma2_rn(make_float2(sv[2 * j], sv[2 * j + 1]), c2, nm);
                 const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
                 rs = __fadd2_rn(rs, p);
                 split_bf16x2(p.x, p.y, pk_hi[j], pk_lo[j]);
             }
             l_run += rs.x + rs.y;
-            tmem_st16(tmem + lane_off + col_s(m, bb) + 16 * h, pk_hi);
-            tmem_st16(tmem + lane_off + col_s(m, bb) + 32 + 16 * h, pk_lo);
+            tmem_st32(tmem + lane_off + col_s(m, bb), pk_hi);
+            tmem_st32(tmem + lane_off + col_s(m, bb) + 32, pk_lo);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p(m, bb));
@@ -344,41 +325,36 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (__any_sync(0xFFFFFFFFu, !ok)) ok = false;
         }
         if (ok) {
-            // Row sum of both halves.
-            *xslot(nt & 1, h) = l_run;
-            mbar_arrive(bar_x(m));
-            if (!mbar_wait(bar_x(m), nt & 1, kSiteX)) s_abort = 1;
-            const float l_tot = l_run + *xslot(nt & 1, 1 - h);
             // O = acc / l through a swizzled shared-memory stage (the Q and
             // K/V buffers are free once the last PV is done), then coalesced
             // row stores.  Row rr of the stage is M-tile rr/128, row rr%128.
             tc_fence_after();
             float* stage = reinterpret_cast<float*>(smem + L::q_off);
             const int sr_ = m * 128 + r;
-            const float inv = 1.f / l_tot;
+            const float inv = 1.f / l_run;
 #pragma unroll 1
-            for (int c = 0; c < D / 64; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t ov[32];
-                tmem_ld32(tmem + lane_off + col_o(m) + (D / 2) * h + 32 * c, ov);
+                tmem_ld32(tmem + lane_off + col_o(m) + 32 * c, ov);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
-                    const int ch = ((D / 2) * h + 32 * c + j) / 4;
+                    const int ch = (32 * c + j) / 4;
                     const int pch = (ch & ~7) | ((ch ^ sr_) & 7);
                     *reinterpret_cast<float4*>(stage + sr_ * D + 4 * pch) =
                         make_float4(__uint_as_float(ov[j]) * inv, __uint_as_float(ov[j + 1]) * inv,
                                     __uint_as_float(ov[j + 2]) * inv, __uint_as_float(ov[j + 3]) * inv);
                 }
             }
-            if (h == 0 && head < a.G) {
+            if (head < a.G) {
                 const int64_t row = ((b * a.Hq + g * a.G + head) * a.T_seg + qb * 64 + i);
-                a.lse[row] = (m_run + log2f(l_tot)) * kLn2;
+                a.lse[row] = (m_run + log2f(l_run)) * kLn2;
             }
             // All softmax threads have staged their rows (bounded wait).
             mbar_arrive(bar_stage);
             if (!mbar_wait(bar_stage, 0, kSiteStage)) s_abort = 1;
             constexpr int C4 = D / 4;                      // 16-byte chunks per row
-            for (int rr = warp; rr < 128 * n_mt; rr += 8 * n_mt) {
+            for (int rr = warp; rr < 128 * n_mt; rr += 4 * n_mt) {
                 const int hh = rr / 64;                    // head within the CTA
                 const int head_r = head0 + hh;
                 if (head_r >= a.G) continue;
@@ -397,7 +373,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // ---- wind down: every TMA copy this CTA issued has landed before exit
     tc_fence_before();
     __syncthreads();
-    if (s_abort && warp == kProducerWarp && lane == 0) {
+    if (s_abort && warp == 8 && lane == 0) {
         for (int s = 0; s < kStages; ++s) {
             // Loads issued for stage s: tiles s, s+S, ... < nt; wait for the last.
             int last = -1;
@@ -407,7 +383,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_wait(bar_q, 0, kSiteDrain);
     }
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
