@@ -36,9 +36,11 @@ from hierarchical_routed_sparse_b200 import workloads as W  # noqa: E402
 METRIC = "HGA routed-attention fwd+bwd tokens/s at 16K ctx; % of roofline (TFLOP/s or HBM GB/s)"
 DEFAULT_WORKLOAD = W.QWEN3_CTX16K_TRAIN.name
 L2_FLUSH_BYTES = 256 << 20
-# Kernels of this library launched per step: summaries, chunk router, group
-# router, attention forward, backward row-dot, attention backward.
-LAUNCHES_PER_STEP = 6
+# Kernels of this library launched per step: segment summaries, fused
+# chunk+group router, attention forward, and with a backward the row-dot
+# (which also zeroes dK/dV) and the attention backward.
+LAUNCHES_FWD = 3
+LAUNCHES_BWD = 2
 
 
 def peaks() -> dict:
@@ -434,7 +436,7 @@ def run_gpu(args, w) -> None:
                     warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype=w.dtype, data="synthetic",
                     config=config_of(w, not args.no_graph), stage_ms=stage_ms, roofline=roof,
-                    gpu_launches=(LAUNCHES_PER_STEP if w.backward else 4) * args.steps,
+                    gpu_launches=(LAUNCHES_FWD + (LAUNCHES_BWD if w.backward else 0)) * args.steps,
                     e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d,
                              d2h_bytes_per_step=d2h),
                     clocks=clk.summary())

@@ -12,23 +12,33 @@
 // M-tile of 128 query rows.  For each 64-key tile (8 routed groups, or the
 // own chunk with the causal mask):
 //     S   = Q K^T, dP = dO V^T        tcgen05.mma -> tensor memory
-//     P   = exp2(S*c - lse), dS = P (dP - D)   row per thread; both written
-//           to shared memory as bf16 hi + lo parts (~14-bit operands)
-//     dQ += dS K                      A = dS (K-major), B = K (MN-major)
+//     P   = exp2(S*c - lse), dS = P (dP - D)   row per thread; dS goes back
+//           over S in tensor memory as bf16 hi + lo parts (~14-bit operand)
+//     dQ += dS K                      A = dS (tensor memory), B = K (MN-major)
+// and for the tiles holding segment keys, with P and dS also written to
+// shared memory (hi + lo):
 //     dV^T = dO^T P, dK^T = Q^T dS    A = dO / Q read MN-major, B = P / dS
 // dV^T and dK^T (d on the tensor-memory lanes, keys on the columns) are added
 // to the float32 dV_seg / dK_seg rows of the segment's keys with coalesced
-// atomics; tiles whose keys are all detached history skip both products
-// (routed groups are ascending, so history tiles come first).
+// atomics; tiles of detached history skip both products.
+//
+// Tile order: an item runs its tiles from the own chunk down to the first
+// routed tile, so the tiles holding segment keys (the own chunk and the last
+// routed tiles, groups being ascending) come first.  Once their products are
+// done the item's P/dS buffer is free and the next item's Q and dO load into
+// it: two 64 KB buffers swap the Q/dO and P/dS roles from item to item, and
+// the next item's S/dP products start while this item's history tiles run.
 //
 // Warp roles (576 threads): warps 0-15 compute P and dS (row 32*(w%4)+lane,
-// 16-key quarter w/4; four warps per scheduler hide each other's latency),
-// add the previous tile's dK/dV while the MMAs of the current one run, and
-// write dQ at the end; warp 16 is the TMA producer, warp 17 the
-// tensor-memory owner and MMA issuer.  Tensor memory (512 columns): S and dP
-// double-buffered (4 x 64), dQ (128), dV^T (64), dK^T (64).  Three K/V
-// stages (224 KB of shared memory in all) keep the gathered loads two tiles
-// ahead of the MMAs.
+// 16-key quarter w/4), add a segment tile's dK/dV while the next tile's MMAs
+// run and write dQ at the end of an item; warp 16 loads Q / dO and the K/V
+// tiles (TMA gathers of 8-row groups), warp 17 owns tensor memory and issues
+// the MMAs.  Tensor memory (512 columns): S and dP
+// double-buffered (4 x 64), dQ (128), dV^T (64), dK^T (64).  K and V load
+// into separate rings: four K stages (K is read by S, two tiles ahead, and
+// by dQ) and two V stages (V is read by dP only and released as S / dP
+// complete), so each load is issued about two tiles before its use; with
+// the two Q/dO <-> P/dS buffers they fill 224 KB of shared memory.
 #include <algorithm>
 
 #include "hga_internal.cuh"
@@ -41,7 +51,8 @@ using namespace sm100;
 
 constexpr int D = 128;
 constexpr int H = 2;                  // 64-column halves of d
-constexpr int kStages = 3;
+constexpr int kKStages = 4;            // K is read by S (issued two tiles ahead) and dQ
+constexpr int kVStages = 2;            // V only by dP: released as S / dP complete
 constexpr int kKeys = 64;
 constexpr int kComputeWarps = 16;     // 4 per lane quadrant, one 16-key quarter each
 constexpr int kCompute = 32 * kComputeWarps;
@@ -50,26 +61,36 @@ constexpr int kThreads = 32 * (kComputeWarps + 2);
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int {
-    kSiteQ = 201, kSiteFull, kSiteEmpty, kSiteSdp, kSitePs, kSiteMm2, kSiteDrained, kSiteFinal, kSiteDrain,
-    kSiteQfree, kSiteDqfree, kSiteStage
+    kSiteQ = 201, kSiteFull, kSiteEmpty, kSiteSdp, kSitePs, kSiteKv, kSiteDrained, kSiteFinal, kSiteDrain,
+    kSiteQfree, kSiteDqfree, kSitePfree, kSiteDqs
 };
 
 struct BwdSmem {
     static constexpr int kRows128 = 128 * 128;        // 128 rows x 128 B
     static constexpr int kKVHalf = kKeys * 128;       // 64 keys x 128 B
-    static constexpr int q_off = 0;                   // [2 halves][128 rows][64]
-    static constexpr int do_off = q_off + H * kRows128;
-    static constexpr int k_off = do_off + H * kRows128;
-    static constexpr int v_off = k_off + kStages * H * kKVHalf;
-    static constexpr int p_off = v_off + kStages * H * kKVHalf;   // P hi, P lo: [128 rows][64 keys]
-    static constexpr int ds_off = p_off + 2 * kRows128;           // dS hi, dS lo
-    static constexpr int bar_off = ds_off + 2 * kRows128;
-    // q, full[S], empty[S], sdp[2], ps, mm2, drained, final, qfree, dqfree, stage
-    static constexpr int n_bars = 1 + 2 * kStages + 2 + 7;
-    static constexpr int tmem_slot_off = bar_off + 8 * n_bars;
+    // Two buffers of 64 KB.  As Q/dO: Q [2 halves][128 rows][64], then dO
+    // alike.  As P/dS: P hi, P lo, dS hi, dS lo, each [128 rows][64 keys].
+    static constexpr int kX = 4 * kRows128;
+    static constexpr int x_off = 0;
+    static constexpr int k_off = x_off + 2 * kX;
+    static constexpr int v_off = k_off + kKStages * H * kKVHalf;
+    static constexpr int bar_off = v_off + kVStages * H * kKVHalf;
+    static constexpr int n_bars = 26;
+    static constexpr int tab_off = bar_off + 8 * n_bars;       // (n_g, n_seg) of the CTA's first items
+    static constexpr int tmem_slot_off = tab_off + 8 * 64;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;
 };
+static_assert(BwdSmem::alloc <= 227 * 1024, "shared memory");
+
+// mbarriers: q[2], kfull / kempty[kKStages], vfull / vempty[kVStages], sdp[2],
+// ps[2], kv, drained, pfree, qfree, dqfree, final, dqs_full, dqs_free.
+constexpr int kBarQ = 0, kBarKFull = 2, kBarKEmpty = kBarKFull + kKStages, kBarVFull = kBarKEmpty + kKStages,
+              kBarVEmpty = kBarVFull + kVStages, kBarSdp = kBarVEmpty + kVStages, kBarPs = kBarSdp + 2,
+              kBarKv = kBarPs + 2, kBarDrained = kBarKv + 1, kBarPfree = kBarKv + 2, kBarQfree = kBarKv + 3,
+              kBarDqfree = kBarKv + 4, kBarFinal = kBarKv + 5, kBarDqsFull = kBarKv + 6,
+              kBarDqsFree = kBarKv + 7;
+static_assert(kBarDqsFree + 1 == BwdSmem::n_bars, "barrier count");
 
 // Tensor-memory columns.
 constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDV = 384, kColDK = 448;
@@ -87,92 +108,92 @@ struct BwdArgs {
     float scale, scale_log2;
 };
 
-// Does key tile t hold any segment token (position >= T_hist)?
-__device__ __forceinline__ bool tile_has_segment_keys(int t, int n_rt, int n_g, const int32_t* grow,
-                                                      int64_t T_hist)
-{
-    if (t == n_rt) return true;                              // own chunk
-    const int last = min(t * 8 + 7, n_g - 1);
-    return (int64_t)grow[last] * 8 + 7 >= T_hist;
-}
-
 // One work item: a (batch, kv-head, query block) and a pair of its q-heads.
+// Processing index p visits key tile t = nt - 1 - p; tiles p < n_seg hold
+// segment keys.
 struct Item {
-    int64_t bg, qb, b, g, kv_base, own_start, u;
-    int head0, n_g, n_rt, nt;
-    uint64_t seg;                   // bit t: key tile t holds segment tokens (t < 64)
-    const int32_t* grow;
+    int u, bg, qb, head0, n_g, n_seg;   // u = bg * nQB + qb, bg = b * Hkv + g
+    __device__ __forceinline__ int n_rt() const { return (n_g + 7) / 8; }
+    __device__ __forceinline__ int nt() const { return n_rt() + 1; }
+    __device__ __forceinline__ const int32_t* grow(const struct BwdArgs& a) const;
+    __device__ __forceinline__ int own_start(const struct BwdArgs& a) const;
 };
 
-// Decode item `it` and count its routed groups (an ascending prefix of the
-// index row).  Whole-warp call.
-__device__ __forceinline__ Item make_item(const BwdArgs& a, int64_t it, int lane)
+__device__ __forceinline__ const int32_t* Item::grow(const BwdArgs& a) const { return a.gidx + (int64_t)u * a.wg; }
+__device__ __forceinline__ int Item::own_start(const BwdArgs& a) const { return int(a.T_hist) + qb * 64; }
+
+// Routed-group count n_g and segment-tile count n_seg of item `it`.  The
+// routed groups are an ascending prefix of the index row: of the n_g, c_hist
+// lie wholly in detached history (group j holds segment tokens iff
+// 8 j >= T_hist), so the tiles from c_hist / 8 on, and the own chunk, hold
+// segment keys.  Whole-warp call.
+__device__ __forceinline__ int2 count_row(const BwdArgs& a, int64_t it, int lane)
+{
+    const int32_t* grow = a.gidx + (it / ((a.G + 1) / 2)) * a.wg;
+    const int64_t first_seg_group = a.T_hist / 8;
+    int n_g = 0, c_hist = 0;
+    for (int base = 0; base < a.wg; base += 32) {
+        const int i = base + lane;
+        const int32_t j = i < a.wg ? __ldg(grow + i) : -1;
+        n_g += __popc(__ballot_sync(0xFFFFFFFFu, j >= 0));
+        c_hist += __popc(__ballot_sync(0xFFFFFFFFu, j >= 0 && j < first_seg_group));
+    }
+    const int n_rt = (n_g + 7) / 8;
+    return make_int2(n_g, c_hist < n_g ? n_rt - c_hist / 8 + 1 : 1);
+}
+
+// Items a CTA decodes once, in its prologue, into shared memory; later ones
+// (more than kItemTab items per CTA) are counted when reached.
+constexpr int kItemTab = 64;
+
+// Item k of this CTA (global index it).  Whole-warp call.
+__device__ __forceinline__ Item make_item(const BwdArgs& a, const int2* tab, int k, int64_t it, int lane)
 {
     Item m;
     const int n_pairs = (a.G + 1) / 2;
-    m.u = it / n_pairs;                                     // (b*Hkv + g)*nQB + qb
-    m.head0 = 2 * int(it % n_pairs);
-    m.qb = m.u % a.nQB;
-    m.bg = m.u / a.nQB;
-    m.b = m.bg / a.Hkv;
-    m.g = m.bg % a.Hkv;
-    m.kv_base = m.bg * (a.T_hist + a.T_seg);
-    m.own_start = a.T_hist + m.qb * 64;
-    m.grow = a.gidx + m.u * a.wg;
-    // Count the routed groups and mark the tiles holding segment groups
-    // (group j is a segment group when 8 j >= T_hist).
-    int c = 0;
-    uint64_t seg = 0;
-    const int64_t first_seg_group = a.T_hist / 8;
-    for (int base = 0; base < a.wg; base += 32) {
-        const int i = base + lane;
-        const int32_t j = i < a.wg ? __ldg(m.grow + i) : -1;
-        c += j >= 0;
-        const unsigned in_seg = __ballot_sync(0xFFFFFFFFu, j >= 0 && j >= first_seg_group);
-        for (int q = 0; q < 4 && base / 8 + q < 64; ++q)
-            if ((in_seg >> (8 * q)) & 0xFFu) seg |= 1ull << (base / 8 + q);
-    }
-    m.n_g = __reduce_add_sync(0xFFFFFFFFu, c);
-    m.n_rt = (m.n_g + 7) / 8;
-    m.nt = m.n_rt + 1;
-    if (m.n_rt < 64) seg |= 1ull << m.n_rt;                 // the own chunk
-    m.seg = seg;
+    const int iit = int(it);
+    m.u = iit / n_pairs;
+    m.head0 = 2 * (iit % n_pairs);
+    m.qb = m.u % int(a.nQB);
+    m.bg = m.u / int(a.nQB);
+    const int2 c = k < kItemTab ? tab[k] : count_row(a, it, lane);
+    m.n_g = c.x;
+    m.n_seg = c.y;
     return m;
 }
 
-// Does key tile t of item m hold any segment token (position >= T_hist)?
-__device__ __forceinline__ bool item_tile_has_segment_keys(const Item& m, int t, int64_t T_hist)
-{
-    if (t < 64) return (m.seg >> t) & 1ull;
-    return tile_has_segment_keys(t, m.n_rt, m.n_g, m.grow, T_hist);
-}
-
 // Persistent: CTA c processes items c, c + gridDim.x, ...  Barrier phases
-// run on a global key-tile counter (gt) and an item counter (k) that every
-// role advances identically, so the next item's loads and first S/dP MMAs
-// overlap the current item's dK/dV and dQ epilogues.
+// run on a global key-tile counter (gt), a segment-tile counter (gs) and an
+// item counter (k) that every role advances identically.
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ CUtensorMap tm_v8,
                    const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v64,
-                   const BwdArgs a)
+                   const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a)
 {
     using L = BwdSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar0 = sbase + L::bar_off;
-    const uint32_t bar_q = bar0;
-    auto bar_full = [&](int s) { return bar0 + 8 * (1 + s); };
-    auto bar_empty = [&](int s) { return bar0 + 8 * (1 + kStages + s); };
-    auto bar_sdp = [&](int b) { return bar0 + 8 * (1 + 2 * kStages + b); };
-    const uint32_t bar_ps = bar0 + 8 * (3 + 2 * kStages);
-    const uint32_t bar_mm2 = bar0 + 8 * (4 + 2 * kStages);
-    const uint32_t bar_drained = bar0 + 8 * (5 + 2 * kStages);
-    const uint32_t bar_final = bar0 + 8 * (6 + 2 * kStages);
-    const uint32_t bar_qfree = bar0 + 8 * (7 + 2 * kStages);
-    const uint32_t bar_dqfree = bar0 + 8 * (8 + 2 * kStages);
-    const uint32_t bar_stage = bar0 + 8 * (9 + 2 * kStages);
+    auto bar_q = [&](int b) { return bar0 + 8 * (kBarQ + b); };
+    auto bar_kfull = [&](int s) { return bar0 + 8 * (kBarKFull + s); };
+    auto bar_kempty = [&](int s) { return bar0 + 8 * (kBarKEmpty + s); };
+    auto bar_vfull = [&](int s) { return bar0 + 8 * (kBarVFull + s); };
+    auto bar_vempty = [&](int s) { return bar0 + 8 * (kBarVEmpty + s); };
+    auto bar_sdp = [&](int b) { return bar0 + 8 * (kBarSdp + b); };
+    auto bar_ps = [&](int b) { return bar0 + 8 * (kBarPs + b); };
+    const uint32_t bar_kv = bar0 + 8 * kBarKv;
+    const uint32_t bar_drained = bar0 + 8 * kBarDrained;
+    const uint32_t bar_pfree = bar0 + 8 * kBarPfree;
+    const uint32_t bar_qfree = bar0 + 8 * kBarQfree;
+    const uint32_t bar_dqfree = bar0 + 8 * kBarDqfree;
+    const uint32_t bar_final = bar0 + 8 * kBarFinal;
+    const uint32_t bar_dqs_full = bar0 + 8 * kBarDqsFull;     // dQ staged in shared memory
+    const uint32_t bar_dqs_free = bar0 + 8 * kBarDqsFree;     // its bulk stores have read it
+    int2* tab = reinterpret_cast<int2*>(smem + L::tab_off);
+    // Item k's Q/dO live in buffer k & 1, its P/dS in buffer (k + 1) & 1.
+    auto xbuf = [&](int k) { return sbase + L::x_off + uint32_t(k & 1) * L::kX; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::tmem_slot_off);
     __shared__ int s_abort;
 
@@ -181,21 +202,37 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     if (threadIdx.x == 0) {
         s_abort = 0;
-        mbar_init(bar_q, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar_full(s), 1);
-            mbar_init(bar_empty(s), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_q(b), 1);
+            mbar_init(bar_sdp(b), 1);
+            mbar_init(bar_ps(b), kCompute);
         }
-        mbar_init(bar_sdp(0), 1);
-        mbar_init(bar_sdp(1), 1);
-        mbar_init(bar_ps, kCompute);
-        mbar_init(bar_mm2, 1);
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(bar_kfull(s), 1);
+            mbar_init(bar_kempty(s), 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(bar_vfull(s), 1);
+            mbar_init(bar_vempty(s), 1);
+        }
+        mbar_init(bar_kv, 1);
         mbar_init(bar_drained, kCompute);
-        mbar_init(bar_final, 1);
+        mbar_init(bar_pfree, 1);
         mbar_init(bar_qfree, 1);
         mbar_init(bar_dqfree, kCompute);
-        mbar_init(bar_stage, kCompute);
+        mbar_init(bar_final, 1);
+        mbar_init(bar_dqs_full, kCompute);
+        mbar_init(bar_dqs_free, 1);
         fence_mbar_init();
+    }
+    // Decode the CTA's first items (warp w: items w, w + 18, ...).
+    {
+        const int64_t n_mine = (n_items - blockIdx.x + gridDim.x - 1) / gridDim.x;
+        const int n_tab = int(n_mine < kItemTab ? n_mine : kItemTab);
+        for (int k = warp; k < n_tab; k += kThreads / 32) {
+            const int2 c = count_row(a, blockIdx.x + (int64_t)k * gridDim.x, lane);
+            if (lane == 0) tab[k] = c;
+        }
     }
     if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
     tc_fence_before();
@@ -213,149 +250,221 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             prefetch_tmap(&tm_k64);
             prefetch_tmap(&tm_v64);
         }
-        int last_gt[kStages] = {-1, -1, -1};                // last tile loaded per stage
-        int k_loaded = -1;                                  // last item whose Q/dO was loaded
+        // Q / dO of item kq_ (lane 0) into buffer kq_ & 1, which held item
+        // kq_-1's P / dS.
+        const int n_pairs = (a.G + 1) / 2;
+        auto load_q = [&](int kq_) {
+            const int64_t itq = blockIdx.x + (int64_t)kq_ * gridDim.x;
+            const int64_t u = itq / n_pairs, qb = u % a.nQB, bg = u / a.nQB;
+            const int64_t b = bg / a.Hkv, g = bg % a.Hkv;
+            const int head0 = 2 * int(itq % n_pairs);
+            mbar_expect_tx(bar_q(kq_ & 1), 2 * 2 * H * 64 * 128);
+            for (int hp = 0; hp < 2; ++hp) {
+                const int head = head0 + hp;
+                const int y = head < a.G ? int((b * a.Hq + g * a.G + head) * a.T_seg + qb * 64) : a.q_rows;
+                for (int c = 0; c < H; ++c) {
+                    const uint32_t off = c * L::kRows128 + hp * 64 * 128;
+                    tma_load_2d(xbuf(kq_) + off, &tm_q, 64 * c, y, bar_q(kq_ & 1));
+                    tma_load_2d(xbuf(kq_) + 2 * L::kRows128 + off, &tm_do, 64 * c, y, bar_q(kq_ & 1));
+                }
+            }
+        };
+        int last_k[kKStages], last_v[kVStages];              // last tile loaded per stage
+        for (int j = 0; j < kKStages; ++j) last_k[j] = -1;
+        for (int j = 0; j < kVStages; ++j) last_v[j] = -1;
+        int q_issued = -1;                                  // last item whose Q / dO load was issued
         uint32_t gt = 0;
         bool ok = true;
         int k = 0;
-        for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
-            const Item m = make_item(a, it, lane);
-            for (int t = 0; t < m.nt && ok; ++t, ++gt) {
-                const int s = gt % kStages;
+        int64_t it = blockIdx.x;
+        for (; it < n_items && ok; it += gridDim.x, ++k) {
+            const Item m = make_item(a, tab, k, it, lane);
+            const int nt = m.nt(), n_rt = m.n_rt();
+            const int32_t* grow = m.grow(a);
+            const int64_t kv_base = (int64_t)m.bg * (a.T_hist + a.T_seg);
+            for (int p = 0; p < nt && ok; ++p, ++gt) {
+                const int t = nt - 1 - p;
+                const int ks = gt % kKStages, vs = gt % kVStages;
+                // Rows of the tile: lane l < 8 holds group slot l (a routed
+                // tile) or lane 0 the own chunk's first row.
+                int y = 0;
+                if (t < n_rt) {
+                    const int gi = t * 8 + lane;
+                    if (lane < 8) y = int(kv_base + (int64_t)__ldg(grow + (gi < m.n_g ? gi : 0)) * 8);
+                } else {
+                    y = int(kv_base + m.own_start(a));
+                }
+                // K (or V) of the tile into stage `st` of `base`: 8-row
+                // gathers, or the own chunk's two 64-row boxes.
+                auto load_tile = [&](const CUtensorMap* m8, const CUtensorMap* m64, uint32_t dst, uint32_t bar) {
+                    if (t < n_rt) {
+                        if (lane < 8)
+                            for (int c = 0; c < H; ++c) tma_load_2d(dst + c * L::kKVHalf + lane * 1024, m8, 64 * c, y, bar);
+                    } else if (lane == 0) {
+                        for (int c = 0; c < H; ++c) tma_load_2d(dst + c * L::kKVHalf, m64, 64 * c, y, bar);
+                    }
+                };
                 if (lane == 0) {
-                    ok = gt < kStages || mbar_wait(bar_empty(s), ((gt / kStages) - 1) & 1, kSiteEmpty);
-                    if (ok) mbar_expect_tx(bar_full(s), 2 * H * kKeys * 128);
+                    // This item's Q / dO before any wait that their MMAs
+                    // gate; the next item's as soon as this one's P / dS are
+                    // released (tested without blocking).
+                    if (q_issued < k) {
+                        ok = k == 0 || mbar_wait(bar_pfree, (k - 1) & 1, kSitePfree);
+                        if (ok) load_q(k);
+                        q_issued = k;
+                    }
+                    if (ok && q_issued == k && it + gridDim.x < n_items && mbar_test(bar_pfree, k & 1)) {
+                        load_q(k + 1);
+                        q_issued = k + 1;
+                    }
+                    if (ok) ok = gt < kKStages || mbar_wait(bar_kempty(ks), ((gt / kKStages) - 1) & 1, kSiteEmpty);
+                    if (ok) mbar_expect_tx(bar_kfull(ks), H * kKeys * 128);
                 }
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
                 if (!ok) break;
-                last_gt[s] = gt;
-                const uint32_t kdst = sbase + L::k_off + s * H * L::kKVHalf;
-                const uint32_t vdst = sbase + L::v_off + s * H * L::kKVHalf;
-                if (t < m.n_rt) {
-                    if (lane < 8) {                           // one group per lane
-                        const int gi = t * 8 + lane;
-                        const int grp = __ldg(m.grow + (gi < m.n_g ? gi : 0));
-                        const int y = int(m.kv_base + (int64_t)grp * 8);
-                        for (int c = 0; c < H; ++c) {
-                            tma_load_2d(kdst + c * L::kKVHalf + lane * 1024, &tm_k8, 64 * c, y, bar_full(s));
-                            tma_load_2d(vdst + c * L::kKVHalf + lane * 1024, &tm_v8, 64 * c, y, bar_full(s));
-                        }
-                    }
-                } else if (lane == 0) {
-                    const int y = int(m.kv_base + m.own_start);
-                    for (int c = 0; c < H; ++c) {
-                        tma_load_2d(kdst + c * L::kKVHalf, &tm_k64, 64 * c, y, bar_full(s));
-                        tma_load_2d(vdst + c * L::kKVHalf, &tm_v64, 64 * c, y, bar_full(s));
-                    }
-                }
+                last_k[ks] = gt;
+                load_tile(&tm_k8, &tm_k64, sbase + L::k_off + ks * H * L::kKVHalf, bar_kfull(ks));
                 __syncwarp();
-                if (t == 0) {
-                    // Q and dO of this item once the previous item's MMAs are done.
-                    if (lane == 0) {
-                        ok = k == 0 || mbar_wait(bar_qfree, (k - 1) & 1, kSiteQfree);
-                        if (ok) {
-                            mbar_expect_tx(bar_q, 2 * 2 * H * 64 * 128);
-                            for (int hp = 0; hp < 2; ++hp) {
-                                const int head = m.head0 + hp;
-                                const int y = head < a.G
-                                                  ? int((m.b * a.Hq + m.g * a.G + head) * a.T_seg + m.qb * 64)
-                                                  : a.q_rows;
-                                for (int c = 0; c < H; ++c) {
-                                    const uint32_t off = c * L::kRows128 + hp * 64 * 128;
-                                    tma_load_2d(sbase + L::q_off + off, &tm_q, 64 * c, y, bar_q);
-                                    tma_load_2d(sbase + L::do_off + off, &tm_do, 64 * c, y, bar_q);
-                                }
-                            }
-                        }
-                    }
-                    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-                    if (ok) k_loaded = k;
+                if (lane == 0) {
+                    ok = gt < kVStages || mbar_wait(bar_vempty(vs), ((gt / kVStages) - 1) & 1, kSiteEmpty);
+                    if (ok) mbar_expect_tx(bar_vfull(vs), H * kKeys * 128);
                 }
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
+                last_v[vs] = gt;
+                load_tile(&tm_v8, &tm_v64, sbase + L::v_off + vs * H * L::kKVHalf, bar_vfull(vs));
+                __syncwarp();
             }
         }
         if (!ok) s_abort = 1;
-        // Wind down: every copy issued has landed before the CTA exits.
+        // Wind down: every copy issued has landed before the CTA exits (the
+        // Q / dO loads before the last one were read by MMAs pfree tracked).
         __syncwarp();
         if (lane == 0 && !ok) {
-            for (int s = 0; s < kStages; ++s)
-                if (last_gt[s] >= 0) mbar_wait(bar_full(s), (last_gt[s] / kStages) & 1, kSiteDrain);
-            if (k_loaded >= 0) mbar_wait(bar_q, k_loaded & 1, kSiteDrain);
+            for (int j = 0; j < kKStages; ++j)
+                if (last_k[j] >= 0) mbar_wait(bar_kfull(j), (last_k[j] / kKStages) & 1, kSiteDrain);
+            for (int j = 0; j < kVStages; ++j)
+                if (last_v[j] >= 0) mbar_wait(bar_vfull(j), (last_v[j] / kVStages) & 1, kSiteDrain);
+            if (q_issued >= 0) mbar_wait(bar_q(q_issued & 1), (q_issued >> 1) & 1, kSiteDrain);
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
         constexpr uint32_t id_sdp = idesc_bf16(128, kKeys, 0, 0);   // S, dP
-        constexpr uint32_t id_dq = idesc_bf16(128, D, 0, 1);        // dQ: A dS K-major, B K MN-major
+        constexpr uint32_t id_dq = idesc_bf16(128, D, 0, 1);        // dQ: A dS (tensor memory), B K MN-major
         constexpr uint32_t id_kv = idesc_bf16(128, kKeys, 1, 1);    // dV^T, dK^T: both MN-major
-        uint32_t gt = 0;
         bool ok = true;
-        int k = 0;
-        for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
-            const Item m = make_item(a, it, lane);
+        // Cursor A walks the tiles whose S / dP are issued next, up to two
+        // tiles ahead of the tile whose gradient MMAs run.
+        int64_t itA = blockIdx.x;
+        int kA = 0, pA = 0, ntA = 0;
+        uint32_t gtA = 0;
+        auto enter_A = [&]() { ntA = make_item(a, tab, kA, itA, lane).nt(); };
+        int pfree_k = -1;                                   // last item whose pfree was committed
+        // S / dP of an item's first tile need its Q / dO, which load once the
+        // previous item's P / dS are no longer read (pfree).
+        auto can_issue = [&]() { return itA < n_items && (pA > 0 || kA == 0 || pfree_k >= kA - 1); };
+        auto issue_sdp = [&]() -> bool {
+            bool r = true;
             if (lane == 0) {
-                auto issue_sdp = [&](uint32_t gtt) -> bool {
-                    const int s = gtt % kStages, bb = gtt & 1;
-                    if (!mbar_wait(bar_full(s), (gtt / kStages) & 1, kSiteFull)) return false;
+                const int ks = gtA % kKStages, vs = gtA % kVStages, bb = gtA & 1;
+                if (pA == 0) r = mbar_wait(bar_q(kA & 1), (kA >> 1) & 1, kSiteQ);
+                if (r) r = mbar_wait(bar_kfull(ks), (gtA / kKStages) & 1, kSiteFull);
+                if (r) r = mbar_wait(bar_vfull(vs), (gtA / kVStages) & 1, kSiteFull);
+                if (r) {
                     tc_fence_after();
+                    // Descriptors of the operand bases; a K step adds its
+                    // byte offset / 16 to the address field.
+                    const uint32_t qa = xbuf(kA);
+                    const uint64_t dq = sdesc_sw128(qa, 16, 1024), ddo = sdesc_sw128(qa + 2 * L::kRows128, 16, 1024);
+                    const uint64_t dk = sdesc_sw128(sbase + L::k_off + ks * H * L::kKVHalf, 16, 1024);
+                    const uint64_t dv = sdesc_sw128(sbase + L::v_off + vs * H * L::kKVHalf, 16, 1024);
+                    const uint32_t ts = tmem + kColS + bb * kKeys, tdp = tmem + kColDP + bb * kKeys;
+#pragma unroll
                     for (int kk = 0; kk < 4 * H; ++kk) {
-                        const uint32_t o = (kk / 4) * L::kRows128 + (kk % 4) * 32;
-                        const uint32_t ko = (s * H + kk / 4) * L::kKVHalf + (kk % 4) * 32;
-                        mma_ss(tmem + kColS + bb * kKeys, sdesc_sw128(sbase + L::q_off + o, 16, 1024),
-                               sdesc_sw128(sbase + L::k_off + ko, 16, 1024), id_sdp, kk > 0);
-                        mma_ss(tmem + kColDP + bb * kKeys, sdesc_sw128(sbase + L::do_off + o, 16, 1024),
-                               sdesc_sw128(sbase + L::v_off + ko, 16, 1024), id_sdp, kk > 0);
+                        const uint32_t o = ((kk / 4) * L::kRows128 + (kk % 4) * 32) >> 4;
+                        const uint32_t ko = ((kk / 4) * L::kKVHalf + (kk % 4) * 32) >> 4;
+                        mma_ss(ts, dq + o, dk + ko, id_sdp, kk > 0);
+                        mma_ss(tdp, ddo + o, dv + ko, id_sdp, kk > 0);
                     }
                     mma_commit(bar_sdp(bb));
-                    return true;
-                };
-                ok = mbar_wait(bar_q, k & 1, kSiteQ);
-                // S / dP run two tiles ahead (double-buffered): S(t+2) is
-                // issued right after the MMAs of tile t, so its load wait never
-                // holds back the gradient MMAs of the tile the softmax finished.
-                if (ok) ok = issue_sdp(gt);
-                if (ok && m.nt > 1) ok = issue_sdp(gt + 1);
-                for (int t = 0; ok && t < m.nt; ++t) {
-                    const uint32_t gtt = gt + t;
-                    const int s = gtt % kStages;
-                    if (!(ok = mbar_wait(bar_ps, gtt & 1, kSitePs))) break;
-                    // dQ accumulates from zero: the previous item's dQ is read out.
-                    if (t == 0 && k > 0 && !(ok = mbar_wait(bar_dqfree, (k - 1) & 1, kSiteDqfree))) break;
-                    tc_fence_after();
-                    // dQ += dS K  (dS hi and lo against the same K)
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t kb =
-                            sdesc_sw128(sbase + L::k_off + s * H * L::kKVHalf + kk * 2048, L::kKVHalf, 1024);
-                        mma_ss(tmem + kColDQ, sdesc_sw128(sbase + L::ds_off + kk * 32, 16, 1024), kb, id_dq,
-                               t > 0 || kk > 0);
-                        mma_ss(tmem + kColDQ, sdesc_sw128(sbase + L::ds_off + L::kRows128 + kk * 32, 16, 1024), kb,
-                               id_dq, true);
-                    }
-                    if (item_tile_has_segment_keys(m, t, a.T_hist)) {
-                        if (gtt >= 1 && !(ok = mbar_wait(bar_drained, (gtt - 1) & 1, kSiteDrained))) break;
-                        tc_fence_after();
-                        // dV^T = dO^T P and dK^T = Q^T dS over the 128 query rows.
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t dOt = sdesc_sw128(sbase + L::do_off + kk * 2048, L::kRows128, 1024);
-                            const uint64_t Qt = sdesc_sw128(sbase + L::q_off + kk * 2048, L::kRows128, 1024);
-                            const uint64_t Ph = sdesc_sw128(sbase + L::p_off + kk * 2048, L::kRows128, 1024);
-                            const uint64_t Pl =
-                                sdesc_sw128(sbase + L::p_off + L::kRows128 + kk * 2048, L::kRows128, 1024);
-                            const uint64_t Sh = sdesc_sw128(sbase + L::ds_off + kk * 2048, L::kRows128, 1024);
-                            const uint64_t Sl =
-                                sdesc_sw128(sbase + L::ds_off + L::kRows128 + kk * 2048, L::kRows128, 1024);
-                            mma_ss(tmem + kColDV, dOt, Ph, id_kv, kk > 0);
-                            mma_ss(tmem + kColDV, dOt, Pl, id_kv, true);
-                            mma_ss(tmem + kColDK, Qt, Sh, id_kv, kk > 0);
-                            mma_ss(tmem + kColDK, Qt, Sl, id_kv, true);
-                        }
-                    }
-                    mma_commit(bar_mm2);
-                    mma_commit(bar_empty(s));
-                    if (t == m.nt - 1) mma_commit(bar_qfree);          // Q / dO of this item no longer read
-                    if (t + 2 < m.nt && !(ok = issue_sdp(gtt + 2))) break;
+                    mma_commit(bar_vempty(vs));                 // V is read by dP only
                 }
             }
-            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-            gt += m.nt;
+            r = __shfl_sync(0xFFFFFFFFu, r, 0);
+            ++gtA;
+            if (++pA == ntA) {
+                pA = 0;
+                ++kA;
+                itA += gridDim.x;
+                if (itA < n_items) enter_A();
+            }
+            return r;
+        };
+        if (itA < n_items) enter_A();
+        uint32_t gt = 0, gs = 0;
+        int k = 0;
+        for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+            const Item mc = make_item(a, tab, k, it, lane);
+            const int nt = mc.nt(), n_seg = mc.n_seg;
+            for (int p = 0; ok && p < nt; ++p, ++gt) {
+                // S / dP up to two tiles ahead (this tile's always: its
+                // item's Q / dO were released during the previous item).
+                while (ok && can_issue() && gtA <= gt + 1) ok = issue_sdp();
+                if (!ok) break;
+                const int ks = gt % kKStages, bb = gt & 1;
+                const bool seg = p < n_seg;
+                if (lane == 0) {
+                    ok = mbar_wait(bar_ps(bb), (gt >> 1) & 1, kSitePs);
+                    // dQ accumulates from zero: the previous item's dQ is read out.
+                    if (ok && p == 0 && k > 0) ok = mbar_wait(bar_dqfree, (k - 1) & 1, kSiteDqfree);
+                    if (ok) {
+                        tc_fence_after();
+                        // dQ += dS K, dS hi and lo from tensor memory (over S).
+                        const uint64_t kb = sdesc_sw128(sbase + L::k_off + ks * H * L::kKVHalf, L::kKVHalf, 1024);
+                        const uint32_t ds = tmem + kColS + bb * kKeys;
+                        const bool acc = p > 0;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            mma_ts(tmem + kColDQ, ds + 16 * kk, kb + (kk * 2048 >> 4), id_dq, acc || kk > 0);
+                            mma_ts(tmem + kColDQ, ds + 16 * kk + 8, kb + (kk * 2048 >> 4), id_dq, true);
+                        }
+                    }
+                    if (ok && seg) {
+                        // dV^T = dO^T P and dK^T = Q^T dS over the 128 query
+                        // rows, once the previous segment tile's are read out.
+                        if (gs >= 1) ok = mbar_wait(bar_drained, (gs - 1) & 1, kSiteDrained);
+                        if (ok) {
+                            tc_fence_after();
+                            const uint32_t qa = xbuf(k), pa = xbuf(k + 1);
+                            const uint64_t dOt = sdesc_sw128(qa + 2 * L::kRows128, L::kRows128, 1024);
+                            const uint64_t Qt = sdesc_sw128(qa, L::kRows128, 1024);
+                            const uint64_t Ph = sdesc_sw128(pa, L::kRows128, 1024);
+                            const uint64_t Pl = sdesc_sw128(pa + L::kRows128, L::kRows128, 1024);
+                            const uint64_t Sh = sdesc_sw128(pa + 2 * L::kRows128, L::kRows128, 1024);
+                            const uint64_t Sl = sdesc_sw128(pa + 3 * L::kRows128, L::kRows128, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t o = (kk * 2048) >> 4;
+                                mma_ss(tmem + kColDV, dOt + o, Ph + o, id_kv, kk > 0);
+                                mma_ss(tmem + kColDV, dOt + o, Pl + o, id_kv, true);
+                                mma_ss(tmem + kColDK, Qt + o, Sh + o, id_kv, kk > 0);
+                                mma_ss(tmem + kColDK, Qt + o, Sl + o, id_kv, true);
+                            }
+                            mma_commit(bar_kv);
+                            if (p == n_seg - 1) mma_commit(bar_pfree);   // P / dS no longer read
+                        }
+                    }
+                    if (ok) {
+                        mma_commit(bar_kempty(ks));
+                        if (p == nt - 1) mma_commit(bar_qfree);          // Q / dO no longer read
+                    }
+                }
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (seg) {
+                    if (p == n_seg - 1) pfree_k = k;
+                    ++gs;
+                }
+            }
         }
         if (!ok) s_abort = 1;
         if (lane == 0) {
@@ -370,74 +479,79 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int r = (warp % 4) * 32 + lane, kq = warp / 4;
         const int i = r & 63, hp = r >> 6;
         const uint32_t lane_off = uint32_t((warp % 4) * 32) << 16;
-        uint8_t* prow_hi = smem + L::p_off + r * 128;
-        uint8_t* prow_lo = prow_hi + L::kRows128;
-        uint8_t* srow_hi = smem + L::ds_off + r * 128;
-        uint8_t* srow_lo = srow_hi + L::kRows128;
-        // dV^T / dK^T of tile te of item m (d = tensor-memory lane r, keys of
+        // First token of the quarter's two group slots of tile t (-64: padding).
+        auto group_bases = [&](const Item& m, int t, int (&gb)[2]) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int gi = t * 8 + 2 * kq + q;
+                gb[q] = t == m.n_rt() ? m.own_start(a) + 16 * kq + 8 * q
+                                      : (gi < m.n_g ? __ldg(m.grow(a) + gi) * 8 : -64);
+            }
+        };
+        // dV^T / dK^T of a segment tile (d = tensor-memory lane r, keys of
         // quarter kq) added to the segment's rows; history keys and padding
-        // are skipped.
-        auto dkv_epilogue = [&](const Item& m, int te) {
-            if (!item_tile_has_segment_keys(m, te, a.T_hist)) return;
+        // are skipped.  Tensor memory is released before the atomics.
+        auto dkv_epilogue = [&](int bg, const int (&gb)[2]) {
             tc_fence_after();
             uint32_t vv[16], kv[16];
             tmem_ld16(tmem + lane_off + kColDV + 16 * kq, vv);
             tmem_ld16(tmem + lane_off + kColDK + 16 * kq, kv);
             tmem_wait_ld();
-            const bool own = te == m.n_rt;
-            int64_t gbase[2];                               // first token of each group slot
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int gi = te * 8 + 2 * kq + q;
-                gbase[q] = own ? m.own_start + 16 * kq + 8 * q : (gi < m.n_g ? (int64_t)__ldg(m.grow + gi) * 8 : -64);
-            }
+            tc_fence_before();
+            mbar_arrive(bar_drained);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const int64_t key = gbase[j / 8] + j % 8;
+                const int key = gb[j / 8] + j % 8;
                 if (key < a.T_hist) continue;               // padding or detached history
-                const int64_t o = (m.bg * a.T_seg + (key - a.T_hist)) * D + r;
+                const int64_t o = ((int64_t)bg * a.T_seg + (key - a.T_hist)) * D + r;
                 atomicAdd(a.dV + o, __uint_as_float(vv[j]));
                 atomicAdd(a.dK + o, __uint_as_float(kv[j]) * a.scale);
             }
         };
         // Per-row constants of an item.
-        struct RowInfo { int64_t row; bool ok; float lse2, Dr; };
+        struct RowInfo { int row; bool ok; float lse2, Dr; };
         auto row_info = [&](const Item& m) {
             RowInfo ri;
             const int head = m.head0 + hp;
             ri.ok = head < a.G;
-            ri.row = (m.b * a.Hq + m.g * a.G + head) * a.T_seg + m.qb * 64 + i;
+            const int b = m.bg / a.Hkv, g = m.bg % a.Hkv;
+            ri.row = int((b * a.Hq + g * a.G + head) * a.T_seg) + m.qb * 64 + i;
             ri.lse2 = ri.ok ? __ldg(a.lse + ri.row) * kLog2e : 0.f;
             ri.Dr = ri.ok ? __ldg(a.Drow + ri.row) : 0.f;
             return ri;
         };
-        // dQ staging: the P / dS region (64 KB) is free once an item's last
-        // MMAs are done; rows of 512 B, 16-byte chunks XOR-swizzled by row.
-        float* stage = reinterpret_cast<float*>(smem + L::p_off);
-        uint32_t gt = 0;
+        uint32_t gt = 0, gs = 0;
         bool ok = true;
         int k = 0;
         int64_t it = blockIdx.x;
-        Item m = make_item(a, it < n_items ? it : 0, lane);
+        Item m = make_item(a, tab, 0, it, lane);           // gridDim.x <= n_items
         RowInfo ri = row_info(m);
         for (; it < n_items && ok; ++k) {
-            const int64_t row = ri.row;
             const bool row_ok = ri.ok;
             const float lse2 = ri.lse2, Dr = ri.Dr;
-            for (int t = 0; t < m.nt && ok; ++t) {
-                const uint32_t gtt = gt + t;
-                const int bb = gtt & 1;
-                ok = mbar_wait(bar_sdp(bb), (gtt / 2) & 1, kSiteSdp);
+            const uint32_t pd = xbuf(k + 1) - sbase;        // this item's P / dS buffer
+            uint8_t* prow_hi = smem + pd + r * 128;
+            uint8_t* prow_lo = prow_hi + L::kRows128;
+            uint8_t* srow_hi = prow_hi + 2 * L::kRows128;
+            uint8_t* srow_lo = prow_hi + 3 * L::kRows128;
+            int gb_prev[2] = {-64, -64};
+            bool pending = false;                           // a segment tile's dK / dV are due
+            const int nt = m.nt(), n_rt = m.n_rt();
+            for (int p = 0; p < nt && ok; ++p, ++gt) {
+                const int t = nt - 1 - p;
+                const int bb = gt & 1;
+                const bool seg = p < m.n_seg;
+                int gb[2] = {-64, -64};
+                if (seg) group_bases(m, t, gb);             // in flight during the tile
+                ok = mbar_wait(bar_sdp(bb), (gt >> 1) & 1, kSiteSdp);
                 if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
                 tc_fence_after();
-                const bool own = t == m.n_rt;
-                // P is an MMA operand only for dV, i.e. for tiles holding segment keys.
-                const bool seg = item_tile_has_segment_keys(m, t, a.T_hist);
+                const bool own = t == n_rt;
                 uint32_t sr[16], pr[16];
                 tmem_ld16(tmem + lane_off + kColS + bb * kKeys + 16 * kq, sr);
                 tmem_ld16(tmem + lane_off + kColDP + bb * kKeys + 16 * kq, pr);
                 tmem_wait_ld();
-                uint32_t ph[8], pl[8], dh[8], dl[8];
+                uint32_t ph[8], pl[8], dsw[16];             // dsw: dS hi (8), then dS lo (8)
                 // Every key of a full routed tile is valid for every row:
                 // no masks there; partial tiles and the own chunk mask keys.
                 const bool full = row_ok && !own && t * 8 + 8 <= m.n_g;
@@ -448,93 +562,126 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const int j0 = 16 * kq + 2 * j2;
                     const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1])),
                                                 c2, l2);
-                    float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                    float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
                     if (!full) {
                         const bool v0 = row_ok && (own ? (j0 <= i) : (t * 8 + j0 / 8 < m.n_g));
                         const bool v1 = row_ok && (own ? (j0 + 1 <= i) : (t * 8 + (j0 + 1) / 8 < m.n_g));
-                        p.x = v0 ? p.x : 0.f;
-                        p.y = v1 ? p.y : 0.f;
+                        pv.x = v0 ? pv.x : 0.f;
+                        pv.y = v1 ? pv.y : 0.f;
                     }
                     const float2 ds = __fmul2_rn(
-                        p, __fadd2_rn(make_float2(__uint_as_float(pr[2 * j2]), __uint_as_float(pr[2 * j2 + 1])), d2));
-                    split_bf16x2(ds.x, ds.y, dh[j2], dl[j2]);
-                    if (seg) split_bf16x2(p.x, p.y, ph[j2], pl[j2]);
+                        pv, __fadd2_rn(make_float2(__uint_as_float(pr[2 * j2]), __uint_as_float(pr[2 * j2 + 1])), d2));
+                    split_bf16x2(ds.x, ds.y, dsw[j2], dsw[8 + j2]);
+                    if (seg) split_bf16x2(pv.x, pv.y, ph[j2], pl[j2]);
                 }
-                // The previous tile's MMAs read P / dS from shared memory.
-                if (gtt >= 1) {
-                    ok = mbar_wait(bar_mm2, (gtt - 1) & 1, kSiteMm2);
-                    if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
-                }
-                // Row r, 16-byte chunk c lives at chunk c ^ (r % 8) (128-byte swizzle).
-#pragma unroll
-                for (int c2i = 0; c2i < 2; ++c2i) {
-                    const int pc = ((2 * kq + c2i) ^ (r & 7)) * 16;
-                    *reinterpret_cast<uint4*>(srow_hi + pc) = make_uint4(dh[4 * c2i], dh[4 * c2i + 1], dh[4 * c2i + 2], dh[4 * c2i + 3]);
-                    *reinterpret_cast<uint4*>(srow_lo + pc) = make_uint4(dl[4 * c2i], dl[4 * c2i + 1], dl[4 * c2i + 2], dl[4 * c2i + 3]);
-                    if (seg) {
-                        *reinterpret_cast<uint4*>(prow_hi + pc) = make_uint4(ph[4 * c2i], ph[4 * c2i + 1], ph[4 * c2i + 2], ph[4 * c2i + 3]);
-                        *reinterpret_cast<uint4*>(prow_lo + pc) = make_uint4(pl[4 * c2i], pl[4 * c2i + 1], pl[4 * c2i + 2], pl[4 * c2i + 3]);
+                // dS over this quarter's S columns: hi for keys 16kq.. at
+                // column 16kq, lo at 16kq + 8 (the dQ MMA's A operand).
+                tmem_st16(tmem + lane_off + kColS + bb * kKeys + 16 * kq, dsw);
+                if (seg) {
+                    // The previous segment tile's dK / dV MMAs read P / dS
+                    // from this buffer (the item's first segment tile reuses
+                    // the previous item's Q / dO, released at its end).
+                    if (p > 0) {
+                        ok = mbar_wait(bar_kv, (gs - 1) & 1, kSiteKv);
+                        if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
+                    } else if (k > 0) {
+                        // The previous item's dQ boxes, staged here, have
+                        // been read by their bulk stores.
+                        if (threadIdx.x == 0) {
+                            bulk_wait_read();
+                            mbar_arrive(bar_dqs_free);
+                        }
+                        ok = mbar_wait(bar_dqs_free, (k - 1) & 1, kSiteDqs);
+                        if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
                     }
+                    // Row r, 16-byte chunk c lives at chunk c ^ (r % 8) (128-byte swizzle).
+#pragma unroll
+                    for (int c2i = 0; c2i < 2; ++c2i) {
+                        const int pc = ((2 * kq + c2i) ^ (r & 7)) * 16;
+                        *reinterpret_cast<uint4*>(srow_hi + pc) =
+                            make_uint4(dsw[4 * c2i], dsw[4 * c2i + 1], dsw[4 * c2i + 2], dsw[4 * c2i + 3]);
+                        *reinterpret_cast<uint4*>(srow_lo + pc) =
+                            make_uint4(dsw[8 + 4 * c2i], dsw[9 + 4 * c2i], dsw[10 + 4 * c2i], dsw[11 + 4 * c2i]);
+                        *reinterpret_cast<uint4*>(prow_hi + pc) =
+                            make_uint4(ph[4 * c2i], ph[4 * c2i + 1], ph[4 * c2i + 2], ph[4 * c2i + 3]);
+                        *reinterpret_cast<uint4*>(prow_lo + pc) =
+                            make_uint4(pl[4 * c2i], pl[4 * c2i + 1], pl[4 * c2i + 2], pl[4 * c2i + 3]);
+                    }
+                    fence_async_smem();
                 }
-                fence_async_smem();
+                tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(bar_ps);
-                // While the MMAs of tile t run: the dK / dV of tile t-1.
-                if (t >= 1) {
-                    dkv_epilogue(m, t - 1);
-                    tc_fence_before();
-                    mbar_arrive(bar_drained);
+                mbar_arrive(bar_ps(bb));
+                // While this tile's MMAs run: the previous segment tile's dK / dV.
+                if (pending) {
+                    if (!seg) {
+                        ok = mbar_wait(bar_kv, (gs - 1) & 1, kSiteKv);
+                        if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
+                    }
+                    dkv_epilogue(m.bg, gb_prev);
+                    pending = false;
+                }
+                if (seg) {
+                    gb_prev[0] = gb[0];
+                    gb_prev[1] = gb[1];
+                    pending = true;
+                    ++gs;
                 }
             }
             if (!ok) break;
             // The next item's index row and row constants load meanwhile.
             const int64_t it_next = it + gridDim.x;
-            const Item m_next = make_item(a, it_next < n_items ? it_next : it, lane);
+            const Item m_next = it_next < n_items ? make_item(a, tab, k + 1, it_next, lane) : m;
             const RowInfo ri_next = row_info(m_next);
-            const uint32_t last = gt + m.nt - 1;
-            ok = mbar_wait(bar_mm2, last & 1, kSiteMm2);
+            if (pending) {
+                ok = mbar_wait(bar_kv, (gs - 1) & 1, kSiteKv);
+                if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
+                dkv_epilogue(m.bg, gb_prev);
+            }
+            // dQ (times the softmax scale), columns 32kq.. of row r: into
+            // this item's Q / dO buffer (free once its last MMAs completed) as
+            // eight 64-row x 32-column boxes in the 128-byte-swizzled layout
+            // of the dQ tensor map; thread 0 stores the boxes with bulk copies
+            // that run on while the next item starts.
+            ok = mbar_wait(bar_qfree, k & 1, kSiteQfree);
             if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
-            dkv_epilogue(m, m.nt - 1);
-            tc_fence_before();
-            mbar_arrive(bar_drained);
             tc_fence_after();
-            // dQ (times the softmax scale): tensor memory -> swizzled shared rows.
             {
                 uint32_t v[32];
                 tmem_ld32(tmem + lane_off + kColDQ + 32 * kq, v);
                 tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar_dqfree);
+                uint8_t* box = smem + (xbuf(k) - sbase) + (hp * 4 + kq) * 8192 + i * 128;
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const int ch = (32 * kq + j) / 4;              // 16-byte chunk of the row
-                    const int pch = (ch & ~7) | ((ch ^ r) & 7);
-                    *reinterpret_cast<float4*>(stage + r * D + 4 * pch) =
-                        make_float4(__uint_as_float(v[j]) * a.scale, __uint_as_float(v[j + 1]) * a.scale,
-                                    __uint_as_float(v[j + 2]) * a.scale, __uint_as_float(v[j + 3]) * a.scale);
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<float4*>(box + ((j ^ (i & 7)) * 16)) =
+                        make_float4(__uint_as_float(v[4 * j]) * a.scale, __uint_as_float(v[4 * j + 1]) * a.scale,
+                                    __uint_as_float(v[4 * j + 2]) * a.scale, __uint_as_float(v[4 * j + 3]) * a.scale);
+                fence_async_smem();
+                mbar_arrive(bar_dqs_full);
+            }
+            if (threadIdx.x == 0) {
+                ok = mbar_wait(bar_dqs_full, k & 1, kSiteDqs);
+                if (ok) {
+                    const int b = m.bg / a.Hkv, g = m.bg % a.Hkv;
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int head = m.head0 + h2;
+                        if (head >= a.G) continue;           // no such head: nothing to store
+                        const int y = int((b * a.Hq + g * a.G + head) * a.T_seg) + m.qb * 64;
+                        for (int c = 0; c < 4; ++c) tma_store_2d(&tm_dq, 32 * c, y, xbuf(k) + (h2 * 4 + c) * 8192);
+                    }
+                    bulk_commit();
                 }
             }
-            tc_fence_before();
-            mbar_arrive(bar_dqfree);
-            // All compute threads have staged their dQ parts (bounded wait).
-            mbar_arrive(bar_stage);
-            if (!mbar_wait(bar_stage, (2 * k) & 1, kSiteStage)) { ok = false; break; }
-            // Coalesced rows: warp w writes rows w, w+16, ...; lane l the l-th 16 bytes.
-            for (int rr = warp; rr < 128; rr += kComputeWarps) {
-                const int head = m.head0 + (rr >> 6);
-                if (head >= a.G) continue;
-                const int64_t grow_ = (m.b * a.Hq + m.g * a.G + head) * a.T_seg + m.qb * 64 + (rr & 63);
-                const int pch = (lane & ~7) | ((lane ^ rr) & 7);
-                *reinterpret_cast<float4*>(a.dQ + grow_ * D + 4 * lane) =
-                    *reinterpret_cast<const float4*>(stage + rr * D + 4 * pch);
-            }
-            // The staging rows are read before P / dS of the next item reuse them.
-            mbar_arrive(bar_stage);
-            if (!mbar_wait(bar_stage, (2 * k + 1) & 1, kSiteStage)) { ok = false; break; }
-            (void)row;
-            gt += m.nt;
+            if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
             it = it_next;
             m = m_next;
             ri = ri_next;
         }
+        // The dQ bulk stores are complete (and have read shared memory)
+        // before the CTA exits.
+        if (threadIdx.x == 0) bulk_wait_all();
         if (!ok) s_abort = 1;
     }
 
@@ -547,11 +694,18 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 }
 
 // D_row = sum_e dO[row][e] * O[row][e]: one warp per row, 16-byte loads of O
-// and 8-byte loads of dO.
+// and 8-byte loads of dO.  The same launch zeroes dK_seg and dV_seg (the
+// backward kernel adds into them), n floats each, grid-stride.
 __global__ void __launch_bounds__(256)
 rowdot_kernel(const float* __restrict__ O, const __nv_bfloat16* __restrict__ dO, float* __restrict__ Drow,
-              int64_t rows)
+              int64_t rows, float* __restrict__ dK, float* __restrict__ dV, int64_t n)
 {
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t j = tid; j < n; j += nthreads) {
+        dK[j] = 0.f;
+        dV[j] = 0.f;
+    }
     const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -588,17 +742,17 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
                                float* dK_seg, float* dV_seg, float* Drow, cudaStream_t st)
 {
     const int64_t rows = (int64_t)s.B * s.Hq * s.T_seg;
-    rowdot_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, static_cast<const __nv_bfloat16*>(dO), Drow, rows);
+    const int64_t n = (int64_t)s.B * s.Hkv * s.T_seg * D;
+    rowdot_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, static_cast<const __nv_bfloat16*>(dO), Drow, rows,
+                                                             dK_seg, dV_seg, n);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t seg_bytes = sizeof(float) * (size_t)s.B * s.Hkv * s.T_seg * D;
-    if ((e = cudaMemsetAsync(dK_seg, 0, seg_bytes, st)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(dV_seg, 0, seg_bytes, st)) != cudaSuccess) return e;
-    CUtensorMap tq, tdo, tk8, tv8, tk64, tv64;
+    CUtensorMap tq, tdo, tk8, tv8, tk64, tv64, tdq;
     const uint64_t q_rows = (uint64_t)rows, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
     if (!make_bf16_map(&tq, Q, q_rows, D, 64) || !make_bf16_map(&tdo, dO, q_rows, D, 64) ||
         !make_bf16_map(&tk8, K, kv_rows, D, 8) || !make_bf16_map(&tv8, V, kv_rows, D, 8) ||
-        !make_bf16_map(&tk64, K, kv_rows, D, 64) || !make_bf16_map(&tv64, V, kv_rows, D, 64))
+        !make_bf16_map(&tk64, K, kv_rows, D, 64) || !make_bf16_map(&tv64, V, kv_rows, D, 64) ||
+        !make_f32_map(&tdq, dQ, q_rows, D, 64))
         return cudaErrorInvalidValue;
     BwdArgs a;
     a.gidx = gidx;
@@ -623,7 +777,7 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
         return e;
     a.n_items = (int64_t)s.B * s.Hkv * s.nQB * ((s.G + 1) / 2);
     const int64_t grid = std::min<int64_t>(a.n_items, sm_count());
-    attn_bwd_tc_kernel<<<(unsigned)grid, kThreads, smem, st>>>(tq, tdo, tk8, tv8, tk64, tv64, a);
+    attn_bwd_tc_kernel<<<(unsigned)grid, kThreads, smem, st>>>(tq, tdo, tk8, tv8, tk64, tv64, tdq, a);
     return cudaGetLastError();
 }
 

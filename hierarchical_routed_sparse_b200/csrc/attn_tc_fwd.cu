@@ -216,12 +216,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     // The buffer held P(t-2), read by PV(t-2).
                     if (t >= 2 && !mbar_wait(bar_o(m, bb), ((t - 2) / 2) & 1, kSiteO)) return false;
                     tc_fence_after();
-                    for (int kk = 0; kk < 4 * H; ++kk) {
-                        const uint32_t qa = sbase + L::q_off + (m * H + kk / 4) * L::kQTile + (kk % 4) * 32;
-                        const uint32_t ka = sbase + L::k_off + (s * H + kk / 4) * L::kKVHalf + (kk % 4) * 32;
-                        mma_ss(tmem + col_s(m, bb), sdesc_sw128(qa, 16, 1024), sdesc_sw128(ka, 16, 1024),
-                               id_s, kk > 0);
-                    }
+                    // Descriptors of the operand bases, stepped by constants.
+                    const uint64_t dq = sdesc_sw128(sbase + L::q_off + m * H * L::kQTile, 16, 1024);
+                    const uint64_t dk = sdesc_sw128(sbase + L::k_off + s * H * L::kKVHalf, 16, 1024);
+                    const uint32_t ts = tmem + col_s(m, bb);
+#pragma unroll
+                    for (int kk = 0; kk < 4 * H; ++kk)
+                        mma_ss(ts, dq + (((kk / 4) * L::kQTile + (kk % 4) * 32) >> 4),
+                               dk + (((kk / 4) * L::kKVHalf + (kk % 4) * 32) >> 4), id_s, kk > 0);
                     mma_commit(bar_s(m, bb));
                 }
                 return true;
@@ -233,11 +235,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 for (int m = 0; m < n_mt; ++m) {
                     if (!(ok = mbar_wait(bar_p(m, bb), (t / 2) & 1, kSiteP))) break;
                     tc_fence_after();
+                    const uint64_t vd = sdesc_sw128(sbase + L::v_off + s * H * L::kKVHalf, L::kKVHalf, 1024);
+                    const uint32_t to = tmem + col_o(m), tp = tmem + col_s(m, bb);
+                    const bool acc = t > 0;
+#pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t va = sbase + L::v_off + s * H * L::kKVHalf + kk * 16 * 128;
-                        const uint64_t vd = sdesc_sw128(va, L::kKVHalf, 1024);
-                        mma_ts(tmem + col_o(m), tmem + col_s(m, bb) + kk * 8, vd, id_o, t > 0 || kk > 0);
-                        mma_ts(tmem + col_o(m), tmem + col_s(m, bb) + 32 + kk * 8, vd, id_o, true);
+                        mma_ts(to, tp + kk * 8, vd + (kk * 16 * 128 >> 4), id_o, acc || kk > 0);
+                        mma_ts(to, tp + 32 + kk * 8, vd + (kk * 16 * 128 >> 4), id_o, true);
                     }
                     mma_commit(bar_o(m, bb));
                 }

@@ -100,6 +100,7 @@ int sm_count();
 // TMA tensor maps (tma_map.cu).
 bool tensor_maps_available();
 bool make_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool make_f32_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // Tensor-core (tcgen05) path for bf16 inputs.
 bool attn_fwd_tc_supported(const Shape& s);

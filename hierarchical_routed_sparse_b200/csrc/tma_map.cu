@@ -56,4 +56,20 @@ bool make_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t c
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D float32 map over `rows` rows of `cols` elements; box of 32 columns
+// (128 bytes) x box_rows rows, 128-byte swizzle.  Used for bulk stores:
+// elements of a box outside the tensor are not written.
+bool make_f32_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 4};
+    const cuuint32_t box[2] = {32, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace hga
