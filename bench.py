@@ -258,7 +258,8 @@ def config_of(w, graph: bool = True) -> dict:
     return dict(workload=w.name, B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T_hist=w.T_hist,
                 T_seg=w.T_seg, T=w.T, k_c=w.k_c, k_g=w.k_g, keys=w.keys,
                 l2="flushed between timed steps (256 MiB write)",
-                launch="CUDA graph of the step" if graph else "eager")
+                launch=("CUDA graph of the step, events around its replay; stage_ms from a second "
+                        "capture with events between the stages") if graph else "eager")
 
 
 def run_reference(args, w) -> None:
@@ -331,11 +332,18 @@ def run_gpu(args, w) -> None:
     # from outside it.
     events = [[torch.cuda.Event(enable_timing=True, external=not args.no_graph) for _ in range(5)]
               for _ in range(args.steps)]
+    # Whole-step timing: events on the stream around each step (the L2 flush
+    # before the first event).  With graphs, the step is one CUDA graph and
+    # the events bracket its replay, graph launch included.
+    outer = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
     run_step = step
+    run_plain = step
     if not args.no_graph:
-        # One segment step captured as a CUDA graph (with its stage events),
-        # replayed per timed step: the device time of the kernels themselves,
-        # without host launch gaps between them.
+        # Two captures of one segment step: a plain graph, timed from outside
+        # for the headline, and one graph per timed step with stage events
+        # recorded inside it for the per-stage breakdown (each event node
+        # adds a few microseconds between the kernels it separates).
         graphs = []
         cap_stream = torch.cuda.Stream(dev)
         cap_stream.wait_stream(stream)
@@ -345,16 +353,24 @@ def run_gpu(args, w) -> None:
                 with torch.cuda.graph(g, stream=cap_stream):
                     step_on(cap_stream, events[i])
                 graphs.append(g)
+            plain = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(plain, stream=cap_stream):
+                step_on(cap_stream)
         stream.wait_stream(cap_stream)
         torch.cuda.synchronize()
         for _ in range(args.warmup):
             flush.zero_()
             graphs[0].replay()
+            flush.zero_()
+            plain.replay()
         torch.cuda.synchronize()
 
         def run_step(ev, i=[0]):
             graphs[i[0] % len(graphs)].replay()
             i[0] += 1
+
+        def run_plain():
+            plain.replay()
     clocks_path = os.path.join(ROOT, "gpurun_out", "clocks.csv") if os.path.isdir(
         os.path.join(ROOT, "gpurun_out")) else None
     if world > 1:
@@ -363,17 +379,24 @@ def run_gpu(args, w) -> None:
     with ClockSampler(local, clocks_path) as clk:
         for i in range(args.steps):
             flush.zero_()                            # outside the timed events
+            outer[i][0].record(stream)
+            run_plain()
+            outer[i][1].record(stream)
+        for i in range(args.steps):
+            flush.zero_()
             run_step(events[i])
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     per_stage = {s: [] for s in stages}
-    totals = []
+    staged_totals = []
     for ev in events:
         for j, s in enumerate(stages):
             per_stage[s].append(ev[j].elapsed_time(ev[j + 1]))
-        totals.append(ev[0].elapsed_time(ev[4]))
+        staged_totals.append(ev[0].elapsed_time(ev[4]))
+    totals = [a.elapsed_time(b) for a, b in outer]
     total_ms = max_over_ranks(sum(totals), dev)
+    staged_ms = max_over_ranks(sum(staged_totals), dev)
     value = whole_job_rate(w.B * w.T_seg, args.steps, world, total_ms)
 
     # ---- end to end through the public API with host buffers ----------------------
@@ -435,7 +458,8 @@ def run_gpu(args, w) -> None:
         line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype=w.dtype, data="synthetic",
-                    config=config_of(w, not args.no_graph), stage_ms=stage_ms, roofline=roof,
+                    config=config_of(w, not args.no_graph), stage_ms=stage_ms,
+                    ms_per_step_with_stage_events=staged_ms / args.steps, roofline=roof,
                     gpu_launches=(LAUNCHES_FWD + (LAUNCHES_BWD if w.backward else 0)) * args.steps,
                     e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d,
                              d2h_bytes_per_step=d2h),

@@ -88,9 +88,27 @@ __device__ __forceinline__ void score_candidates(const float* __restrict__ qs, i
     }
 }
 
+// 16 bytes of inputs widened to float32 (8 bf16 or 4 float).
+template <typename T> __device__ __forceinline__ void widen16(const uint4 r, float* out);
+template <> __device__ __forceinline__ void widen16<__nv_bfloat16>(const uint4 r, float* out)
+{
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        out[2 * i] = __uint_as_float(w[i] << 16);
+        out[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+template <> __device__ __forceinline__ void widen16<float>(const uint4 r, float* out)
+{
+    out[0] = __uint_as_float(r.x); out[1] = __uint_as_float(r.y);
+    out[2] = __uint_as_float(r.z); out[3] = __uint_as_float(r.w);
+}
+
 // Block query into qs (and qbar[u]): the mean of the block's 64 queries over
 // the G q-heads of the kv-head.  Every thread owns one 16-byte column vector
-// and issues the loads of up to 8 of its rows before adding them.
+// and issues the loads of up to 16 of its rows (kept as raw 16-byte words)
+// before widening and adding them: one memory round trip for G = 4.
 template <typename TIn, int D>
 __device__ __forceinline__ void block_query(const TIn* __restrict__ Q, float* __restrict__ qbar_row,
                                             float* qs, float (*part)[D], int64_t b, int64_t g, int64_t qb,
@@ -104,23 +122,27 @@ __device__ __forceinline__ void block_query(const TIn* __restrict__ Q, float* __
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int r0 = rl; r0 < rows; r0 += 8 * RL) {
-        float x[8][E];
+    constexpr int kLoads = 16;
+    for (int r0 = rl; r0 < rows; r0 += kLoads * RL) {
+        uint4 raw[kLoads];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < kLoads; ++q) {
             const int r = r0 + q * RL;
             if (r < rows) {
                 const int64_t h = (int64_t)g * G + r / kChunk;
-                Vec16<TIn>::load(Q + ((b * Hq + h) * T_seg + qb * kChunk + r % kChunk) * D + v * E, x[q]);
+                raw[q] = __ldg(reinterpret_cast<const uint4*>(
+                    Q + ((b * Hq + h) * T_seg + qb * kChunk + r % kChunk) * D + v * E));
             } else {
-#pragma unroll
-                for (int e = 0; e < E; ++e) x[q][e] = 0.f;
+                raw[q] = make_uint4(0u, 0u, 0u, 0u);        // zero bits widen to 0.0f
             }
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
+        for (int q = 0; q < kLoads; ++q) {
+            float x[E];
+            widen16<TIn>(raw[q], x);
 #pragma unroll
-            for (int e = 0; e < E; ++e) acc[e] += x[q][e];
+            for (int e = 0; e < E; ++e) acc[e] += x[e];
+        }
     }
 #pragma unroll
     for (int e = 0; e < E; ++e) part[rl][v * E + e] = acc[e];
@@ -152,10 +174,66 @@ __device__ __forceinline__ void compact_selected(const unsigned long long* keys,
     for (int i = pos + lane; i < width; i += 32) out[i] = -1;
 }
 
+// Warp-level top-k over candidate keys held in registers: lane l holds the
+// keys of candidates l + 32 m (m < kRegCand; 0 = none).  A round takes the
+// warp maximum with two 32-bit reductions (score bits, then the inverted
+// index among equal scores); the winning lane marks its candidate (bit m of
+// sel) and recomputes its maximum from registers.  Then the selected
+// candidates are written in ascending candidate order, -1 up to `width`,
+// to out0 and (if not null) out1.
+constexpr int kRegCand = 8;
+
+__device__ __forceinline__ void warp_topk_regs(unsigned long long (&ck)[kRegCand], int k, int32_t* out0,
+                                               int32_t* out1, int width, int lane)
+{
+    auto lane_max = [&]() {
+        unsigned long long b = ck[0];
+#pragma unroll
+        for (int m = 1; m < kRegCand; ++m) b = ck[m] > b ? ck[m] : b;
+        return b;
+    };
+    unsigned long long best = lane_max();
+    uint32_t sel = 0;
+    for (int round = 0; round < k; ++round) {
+        const uint32_t hi = uint32_t(best >> 32), lo = uint32_t(best);
+        const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
+        const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+        if (best != 0ull && hi == mhi && lo == mlo) {       // keys are distinct: one lane wins
+#pragma unroll
+            for (int m = 0; m < kRegCand; ++m)
+                if (ck[m] == best) {
+                    ck[m] = 0ull;
+                    sel |= 1u << m;
+                }
+            best = lane_max();
+        }
+    }
+    const unsigned below = (1u << lane) - 1u;
+    int pos = 0;
+#pragma unroll
+    for (int m = 0; m < kRegCand; ++m) {
+        const bool mine = (sel >> m) & 1u;
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, mine);
+        if (mine) {
+            const int at = pos + __popc(bal & below);
+            out0[at] = lane + 32 * m;
+            if (out1) out1[at] = lane + 32 * m;
+        }
+        pos += __popc(bal);
+    }
+    for (int i = pos + lane; i < width; i += 32) {
+        out0[i] = -1;
+        if (out1) out1[i] = -1;
+    }
+}
+
 // a3: chunk routing of one block: scores of the eligible chunks c < c0, then
-// a warp-level top-k (k rounds of a warp arg-max on warp 0; the winner's key
-// is cleared to 0, which marks it selected).  Writes the row to cidx_row and
-// (if not null) to crow_smem.
+// a warp-level top-k on warp 0 -- from registers (warp_topk_regs) when
+// c0 <= 256, else by rounds over shared memory: lane l keeps the largest key
+// among its candidates l, l+32, ...; a round takes the warp maximum as above
+// and the winning lane clears the winner's key (0 marks it selected) and
+// rescans its candidates.  Writes the row to cidx_row and (if not null) to
+// crow_smem.
 template <int D>
 __device__ __forceinline__ void route_chunks_block(const float* qs, const float* __restrict__ cs, int c0, int k_c,
                                                    int wc, unsigned long long* keys, int32_t* cidx_row,
@@ -174,15 +252,25 @@ __device__ __forceinline__ void route_chunks_block(const float* qs, const float*
     score_candidates<D>(qs, c0, [&](int c, const float*& row) { row = cs + (int64_t)c * D; return c; }, keys,
                         warp, lane);
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 0 && c0 <= 32 * kRegCand) {
+        unsigned long long ck[kRegCand];
+#pragma unroll
+        for (int m = 0; m < kRegCand; ++m) ck[m] = lane + 32 * m < c0 ? keys[lane + 32 * m] : 0ull;
+        warp_topk_regs(ck, k_c, cidx_row, crow_smem, wc, lane);
+    } else if (warp == 0) {
+        unsigned long long best = 0ull;
+        for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
         for (int round = 0; round < k_c; ++round) {
-            unsigned long long best = 0ull;
-            for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
-            best = warp_max_u64(best);
-            __syncwarp();
-            if (lane == 0) keys[key_index(best)] = 0ull;
-            __syncwarp();
+            const uint32_t hi = uint32_t(best >> 32), lo = uint32_t(best);
+            const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
+            const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+            if (best != 0ull && hi == mhi && lo == mlo) {   // keys are distinct: one lane wins
+                keys[key_index(best)] = 0ull;
+                best = 0ull;
+                for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
+            }
         }
+        __syncwarp();
         compact_selected(keys, nullptr, c0, cidx_row, wc, lane);
         if (crow_smem) compact_selected(keys, nullptr, c0, crow_smem, wc, lane);
     }
