@@ -225,6 +225,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_init(bar_dqs_free, 1);
         fence_mbar_init();
     }
+    if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
+    // Setup above touches no global memory; the inputs are read from here on.
+    pdl_wait();
+    pdl_trigger();
     // Decode the CTA's first items (warp w: items w, w + 18, ...).
     {
         const int64_t n_mine = (n_items - blockIdx.x + gridDim.x - 1) / gridDim.x;
@@ -234,7 +238,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (lane == 0) tab[k] = c;
         }
     }
-    if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -700,6 +703,8 @@ __global__ void __launch_bounds__(256)
 rowdot_kernel(const float* __restrict__ O, const __nv_bfloat16* __restrict__ dO, float* __restrict__ Drow,
               int64_t rows, float* __restrict__ dK, float* __restrict__ dV, int64_t n)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
     for (int64_t j = tid; j < n; j += nthreads) {
@@ -743,9 +748,8 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
 {
     const int64_t rows = (int64_t)s.B * s.Hq * s.T_seg;
     const int64_t n = (int64_t)s.B * s.Hkv * s.T_seg * D;
-    rowdot_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, static_cast<const __nv_bfloat16*>(dO), Drow, rows,
-                                                             dK_seg, dV_seg, n);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(rowdot_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, st, O,
+                               static_cast<const __nv_bfloat16*>(dO), Drow, rows, dK_seg, dV_seg, n);
     if (e != cudaSuccess) return e;
     CUtensorMap tq, tdo, tk8, tv8, tk64, tv64, tdq;
     const uint64_t q_rows = (uint64_t)rows, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
@@ -777,8 +781,8 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
         return e;
     a.n_items = (int64_t)s.B * s.Hkv * s.nQB * ((s.G + 1) / 2);
     const int64_t grid = std::min<int64_t>(a.n_items, sm_count());
-    attn_bwd_tc_kernel<<<(unsigned)grid, kThreads, smem, st>>>(tq, tdo, tk8, tv8, tk64, tv64, tdq, a);
-    return cudaGetLastError();
+    return launch_pdl(attn_bwd_tc_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st, tq, tdo, tk8, tv8,
+                      tk64, tv64, tdq, a);
 }
 
 }  // namespace hga

@@ -77,6 +77,33 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// ---- programmatic dependent launch ------------------------------------------------
+// The library's kernels are launched so that each may start while the kernel
+// before it on the stream finishes (its launch and setup overlap that
+// kernel's last CTAs).  A kernel calls pdl_wait() before its first access to
+// global memory -- the previous kernel, the library's or the caller's, may be
+// writing any of its inputs -- and pdl_trigger() right after, which lets the
+// next kernel launch.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---- launchers (each returns cudaError_t of its launch) ------------------------
 cudaError_t launch_summaries(const Shape& s, const void* K, int64_t c_begin, int64_t c_end,
                              float* csum, float* gsum, cudaStream_t st);

@@ -332,6 +332,8 @@ route_chunks_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum,
     extern __shared__ unsigned long long keys[];      // [nC]
     __shared__ float part[RL][D];
     __shared__ __align__(16) float qs[D];
+    pdl_wait();
+    pdl_trigger();
     const int64_t u = blockIdx.x;                      // ((b*Hkv)+g)*nQB + qb
     const int64_t qb = u % nQB, bg = u / nQB;
     const int64_t b = bg / Hkv, g = bg % Hkv;
@@ -352,6 +354,8 @@ route_groups_kernel(const float* __restrict__ qbar, const float* __restrict__ gs
     uint8_t* flags = reinterpret_cast<uint8_t*>(ids + (size_t)kGroupsPerChunk * wc);
     __shared__ __align__(16) float qs[D];
     __shared__ int n_valid;
+    pdl_wait();
+    pdl_trigger();
     const int64_t u = blockIdx.x;
     const int64_t bg = u / nQB;
     for (int col = threadIdx.x; col < D; col += kRouterThreads) qs[col] = qbar[u * D + col];
@@ -378,6 +382,8 @@ route_fused_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, co
     __shared__ float part[RL][D];
     __shared__ __align__(16) float qs[D];
     __shared__ int n_valid;
+    pdl_wait();
+    pdl_trigger();
     const int64_t u = blockIdx.x;
     const int64_t qb = u % nQB, bg = u / nQB;
     const int64_t b = bg / Hkv, g = bg % Hkv;
@@ -399,10 +405,9 @@ cudaError_t launch_rc(const Shape& s, const void* Q, const float* csum, float* q
         if (e != cudaSuccess) return e;
     }
     const int64_t blocks = (int64_t)s.B * s.Hkv * s.nQB;
-    k<<<(unsigned)blocks, kRouterThreads, smem, st>>>(
-        static_cast<const TIn*>(Q), csum, qbar, cidx, s.Hq, s.Hkv, s.G, s.T_seg, s.nQB, s.nC,
-        s.T_hist / kChunk, s.k_c, s.wc, 1.0f / (float)(s.G * kChunk));
-    return cudaGetLastError();
+    return launch_pdl(k, dim3((unsigned)blocks), dim3(kRouterThreads), smem, st, static_cast<const TIn*>(Q), csum,
+                      qbar, cidx, s.Hq, s.Hkv, s.G, s.T_seg, s.nQB, s.nC, s.T_hist / kChunk, s.k_c, s.wc,
+                      1.0f / (float)(s.G * kChunk));
 }
 
 template <int D>
@@ -416,9 +421,8 @@ cudaError_t launch_rg(const Shape& s, const float* qbar, const float* gsum, cons
         if (e != cudaSuccess) return e;
     }
     const int64_t blocks = (int64_t)s.B * s.Hkv * s.nQB;
-    k<<<(unsigned)blocks, kRouterThreads, smem, st>>>(qbar, gsum, cidx, gidx, s.nQB, s.nG, s.wc,
-                                                      s.k_g, s.wg);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3((unsigned)blocks), dim3(kRouterThreads), smem, st, qbar, gsum, cidx, gidx, s.nQB,
+                      s.nG, s.wc, s.k_g, s.wg);
 }
 
 template <typename TIn, int D>
@@ -432,10 +436,9 @@ cudaError_t launch_rf(const Shape& s, const void* Q, const float* csum, const fl
         if (e != cudaSuccess) return e;
     }
     const int64_t blocks = (int64_t)s.B * s.Hkv * s.nQB;
-    k<<<(unsigned)blocks, kRouterThreads, smem, st>>>(
-        static_cast<const TIn*>(Q), csum, gsum, qbar, cidx, gidx, s.Hq, s.Hkv, s.G, s.T_seg, s.nQB, s.nC, s.nG,
-        s.T_hist / kChunk, s.k_c, s.wc, s.k_g, s.wg, 1.0f / (float)(s.G * kChunk));
-    return cudaGetLastError();
+    return launch_pdl(k, dim3((unsigned)blocks), dim3(kRouterThreads), smem, st, static_cast<const TIn*>(Q), csum,
+                      gsum, qbar, cidx, gidx, s.Hq, s.Hkv, s.G, s.T_seg, s.nQB, s.nC, s.nG, s.T_hist / kChunk,
+                      s.k_c, s.wc, s.k_g, s.wg, 1.0f / (float)(s.G * kChunk));
 }
 
 }  // namespace

@@ -26,6 +26,8 @@ summaries_kernel(const TIn* __restrict__ K, int64_t T, int64_t c_begin, int64_t 
     constexpr int V16 = D / E;                  // 16-byte vectors per row
     __shared__ float part[kGroupsPerChunk][D];
 
+    pdl_wait();
+    pdl_trigger();
     const int64_t bg = blockIdx.x / n_chunks;   // (batch, kv-head)
     const int64_t c = c_begin + blockIdx.x % n_chunks;
     const int r = threadIdx.x / V16, v = threadIdx.x % V16;
@@ -65,9 +67,8 @@ cudaError_t launch(const Shape& s, const void* K, int64_t c_begin, int64_t c_end
     const int64_t n = c_end - c_begin;
     const int64_t blocks = n * s.B * s.Hkv;
     constexpr int threads = kGroupsPerChunk * D / Vec16<TIn>::E;
-    summaries_kernel<TIn, D><<<(unsigned)blocks, threads, 0, st>>>(
-        static_cast<const TIn*>(K), s.T, c_begin, n, csum, gsum);
-    return cudaGetLastError();
+    return launch_pdl(summaries_kernel<TIn, D>, dim3((unsigned)blocks), dim3(threads), 0, st,
+                      static_cast<const TIn*>(K), s.T, c_begin, n, csum, gsum);
 }
 
 }  // namespace
