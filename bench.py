@@ -101,8 +101,8 @@ def algorithmic(w) -> dict:
 # Source files of each timed kernel: a recorded ncu traffic figure is used
 # only while these files are unchanged since the capture.
 KERNEL_SOURCES = {
-    "attn_fwd": ["attn_tc_fwd.cu", "sm100.cuh"],
-    "attn_bwd": ["attn_tc_bwd.cu", "sm100.cuh"],
+    "attn_fwd": ["attn_tc_fwd.cu", "sm100.cuh", "hga_internal.cuh"],
+    "attn_bwd": ["attn_tc_bwd.cu", "sm100.cuh", "hga_internal.cuh"],
 }
 
 

@@ -696,30 +696,47 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
 }
 
-// D_row = sum_e dO[row][e] * O[row][e]: one warp per row, 16-byte loads of O
-// and 8-byte loads of dO.  The same launch zeroes dK_seg and dV_seg (the
-// backward kernel adds into them), n floats each, grid-stride.
+// D_row = sum_e dO[row][e] * O[row][e]: one warp per four rows, whose
+// 16-byte loads of O and 8-byte loads of dO are all issued before the sums.
+// The same launch zeroes dK_seg and dV_seg (the backward kernel adds into
+// them), n4 float4s each, grid-stride.
+constexpr int kRowdotRows = 4;
+
 __global__ void __launch_bounds__(256)
 rowdot_kernel(const float* __restrict__ O, const __nv_bfloat16* __restrict__ dO, float* __restrict__ Drow,
-              int64_t rows, float* __restrict__ dK, float* __restrict__ dV, int64_t n)
+              int64_t rows, float4* __restrict__ dK, float4* __restrict__ dV, int64_t n4)
 {
     pdl_wait();
     pdl_trigger();
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t j = tid; j < n; j += nthreads) {
-        dK[j] = 0.f;
-        dV[j] = 0.f;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t j = tid; j < n4; j += nthreads) {
+        dK[j] = z;
+        dV[j] = z;
     }
-    const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
+    const int64_t row0 = ((int64_t)blockIdx.x * 8 + threadIdx.x / 32) * kRowdotRows;
     const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    const float4 o = __ldg(reinterpret_cast<const float4*>(O + row * D) + lane);
-    const uint2 w = __ldg(reinterpret_cast<const uint2*>(dO + row * D) + lane);
-    float acc = o.x * __uint_as_float(w.x << 16) + o.y * __uint_as_float(w.x & 0xFFFF0000u) +
-                o.z * __uint_as_float(w.y << 16) + o.w * __uint_as_float(w.y & 0xFFFF0000u);
-    acc = warp_sum(acc);
-    if (lane == 0) Drow[row] = acc;
+    float4 o[kRowdotRows];
+    uint2 w[kRowdotRows];
+#pragma unroll
+    for (int q = 0; q < kRowdotRows; ++q) {
+        const int64_t row = row0 + q;
+        if (row < rows) {
+            o[q] = __ldg(reinterpret_cast<const float4*>(O + row * D) + lane);
+            w[q] = __ldg(reinterpret_cast<const uint2*>(dO + row * D) + lane);
+        } else {
+            o[q] = z;
+            w[q] = make_uint2(0u, 0u);
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < kRowdotRows; ++q) {
+        float acc = o[q].x * __uint_as_float(w[q].x << 16) + o[q].y * __uint_as_float(w[q].x & 0xFFFF0000u) +
+                    o[q].z * __uint_as_float(w[q].y << 16) + o[q].w * __uint_as_float(w[q].y & 0xFFFF0000u);
+        acc = warp_sum(acc);
+        if (lane == 0 && row0 + q < rows) Drow[row0 + q] = acc;
+    }
 }
 
 }  // namespace
@@ -747,9 +764,11 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
                                float* dK_seg, float* dV_seg, float* Drow, cudaStream_t st)
 {
     const int64_t rows = (int64_t)s.B * s.Hq * s.T_seg;
-    const int64_t n = (int64_t)s.B * s.Hkv * s.T_seg * D;
-    cudaError_t e = launch_pdl(rowdot_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, st, O,
-                               static_cast<const __nv_bfloat16*>(dO), Drow, rows, dK_seg, dV_seg, n);
+    const int64_t n4 = (int64_t)s.B * s.Hkv * s.T_seg * D / 4;   // D = 128: whole float4s
+    const int64_t rows_per_cta = 8 * kRowdotRows;
+    cudaError_t e = launch_pdl(rowdot_kernel, dim3((unsigned)((rows + rows_per_cta - 1) / rows_per_cta)), dim3(256),
+                               0, st, O, static_cast<const __nv_bfloat16*>(dO), Drow, rows,
+                               reinterpret_cast<float4*>(dK_seg), reinterpret_cast<float4*>(dV_seg), n4);
     if (e != cudaSuccess) return e;
     CUtensorMap tq, tdo, tk8, tv8, tk64, tv64, tdq;
     const uint64_t q_rows = (uint64_t)rows, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
