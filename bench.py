@@ -472,6 +472,121 @@ def run_gpu(args, w) -> None:
         dist.destroy_process_group()
 
 
+def run_host_tier(args, w) -> None:
+    """The segment step with the history K/V rows in pinned host memory: the
+    segment's summaries come from its own rows (hga_build_summaries_rows),
+    the routed history groups are staged in device memory over the host link
+    after routing (hga_stage_routed), and the attention runs on the staged
+    problem.  One JSON line with config.kv_tier = "host"."""
+    import torch
+    import torch.distributed as dist
+
+    import hierarchical_routed_sparse_b200 as hga
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    wr = rank_workload(w, rank)
+    x = wr.full()
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    p = hga.Params.from_workload(w)
+    buf = hga.Buffers(p, device=dev)
+    # History summaries persist in HBM (built once, from the history rows).
+    Kh = torch.from_numpy(np.ascontiguousarray(x["K"][:, :, :w.T_hist])).to(tdt).pin_memory()
+    Vh = torch.from_numpy(np.ascontiguousarray(x["V"][:, :, :w.T_hist])).to(tdt).pin_memory()
+    hga.build_summaries_rows(p, Kh.to(dev), 0, w.T_hist, buf.csum, buf.gsum)
+    Q = torch.from_numpy(x["Q"]).to(dev, tdt)
+    Ks = torch.from_numpy(np.ascontiguousarray(x["K"][:, :, w.T_hist:])).to(dev, tdt)
+    Vs = torch.from_numpy(np.ascontiguousarray(x["V"][:, :, w.T_hist:])).to(dev, tdt)
+    dO = torch.from_numpy(x["dO"]).to(dev, tdt) if w.backward else None
+    skv = hga.StagedKV(p, device=dev)
+    sbuf = hga.Buffers(skv.ps, device=dev)           # outputs of the staged attention
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize()
+    stages = ["summaries", "route", "stage", "attn_fwd", "attn_bwd"]
+
+    def step_on(st, ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(st)
+        mark(0)
+        hga.build_summaries_rows(p, Ks, w.T_hist, w.T, buf.csum, buf.gsum, st)
+        mark(1)
+        buf.route(Q, st)
+        mark(2)
+        skv.stage(Kh, Vh, Ks, Vs, buf.gidx, st)
+        mark(3)
+        sbuf.forward(Q, skv.K, skv.V, gidx=skv.gidx, stream=st)
+        mark(4)
+        if dO is not None:
+            sbuf.backward(Q, skv.K, skv.V, dO, gidx=skv.gidx, stream=st)
+        mark(5)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step_on(stream)
+    torch.cuda.synchronize()
+    events = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)] for _ in range(args.steps)]
+    outer = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    graphs = []
+    with torch.cuda.stream(cap):
+        for i in range(args.steps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                step_on(cap, events[i])
+            graphs.append(g)
+        plain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(plain, stream=cap):
+            step_on(cap)
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        flush.zero_()
+        plain.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    with ClockSampler(local, None) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            outer[i][0].record(stream)
+            plain.replay()
+            outer[i][1].record(stream)
+        for i in range(args.steps):
+            flush.zero_()
+            graphs[i].replay()
+        torch.cuda.synchronize()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in outer), dev)
+    stage_ms = {s: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in events) for j, s in enumerate(stages)}
+    value = whole_job_rate(w.B * w.T_seg, args.steps, world, total_ms)
+    # Host bytes read per step: 8 rows of K and of V per routed history group.
+    gidx = buf.gidx.cpu().numpy()
+    n_hist = int(((gidx >= 0) & (gidx < w.T_hist // 8)).sum())
+    host_bytes = n_hist * 8 * w.d * (2 if w.dtype == "bf16" else 4) * 2
+    if rank == 0:
+        line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
+                    warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
+                    scaling="weak", vs_baseline=None, dtype=w.dtype, data="synthetic",
+                    config=dict(config_of(w), kv_tier="host",
+                                history="pinned host memory, routed groups staged in HBM per step"),
+                    stage_ms=stage_ms,
+                    host_link=dict(bytes_per_step=host_bytes,
+                                   gb_per_s=host_bytes / (stage_ms["stage"] * 1e-3) / 1e9),
+                    gpu_launches=(LAUNCHES_FWD + 1 + (LAUNCHES_BWD if w.backward else 0)) * args.steps,
+                    clocks=clk.summary())
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -484,12 +599,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager launches instead of a CUDA graph of the step")
+    ap.add_argument("--kv-tier", choices=["hbm", "host"], default="hbm",
+                    help="host: history K/V in pinned host memory, routed groups staged per step")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu DRAM bytes per launch of the dominant kernel, if captured")
     args = ap.parse_args()
     w = W.BY_NAME[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.kv_tier == "host":
+        run_host_tier(args, w)
     else:
         run_gpu(args, w)
 

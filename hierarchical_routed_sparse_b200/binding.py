@@ -9,6 +9,7 @@ every call raises.
 from __future__ import annotations
 
 import ctypes
+import dataclasses
 import math
 import os
 from dataclasses import dataclass
@@ -21,9 +22,11 @@ HGA_BF16, HGA_FP32 = 0, 1
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhga.so")
 
-EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_route_chunks",
+EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_build_summaries_rows",
+           "hga_route_chunks",
            "hga_route_groups", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
-           "hga_device_status", "hga_last_error", "hga_version")
+           "hga_stage_params", "hga_stage_routed", "hga_device_status", "hga_last_error",
+           "hga_version")
 NOALLOC_MAX_ROWS = 1 << 20     # HGA_NOALLOC_MAX_ROWS
 
 
@@ -98,6 +101,7 @@ def load() -> ctypes.CDLL:
                                  ctypes.c_int),
             "hga_workspace_size": ([PP], ctypes.c_size_t),
             "hga_build_summaries": ([PP, P, I64, I64, P, P, P], ctypes.c_int),
+            "hga_build_summaries_rows": ([PP, P, I64, I64, P, P, P], ctypes.c_int),
             "hga_route_chunks": ([PP, P, P, P, P, P], ctypes.c_int),
             "hga_route_groups": ([PP, P, P, P, P, P], ctypes.c_int),
             "hga_route": ([PP, P, P, P, P, P, P, P], ctypes.c_int),
@@ -105,6 +109,8 @@ def load() -> ctypes.CDLL:
             "hga_attn_bwd": ([PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P],
                              ctypes.c_int),
             "hga_attn_bwd_noalloc": ([PP, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "hga_stage_params": ([PP, PP], ctypes.c_int),
+            "hga_stage_routed": ([PP, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_device_status": ([ctypes.POINTER(ctypes.c_int), ctypes.c_int], ctypes.c_int),
             "hga_last_error": ([], ctypes.c_char_p),
             "hga_version": ([], ctypes.c_char_p),
@@ -163,6 +169,12 @@ def build_summaries(p: Params, K, t_begin: int, t_end: int, csum, gsum, stream=N
                                       _ptr(gsum), _stream(stream)))
 
 
+def build_summaries_rows(p: Params, K_rows, t_begin: int, t_end: int, csum, gsum, stream=None) -> None:
+    """Summaries of tokens [t_begin, t_end) from a K holding only those rows."""
+    _check(load().hga_build_summaries_rows(ctypes.byref(p.c()), _ptr(K_rows), t_begin, t_end, _ptr(csum),
+                                           _ptr(gsum), _stream(stream)))
+
+
 def route_chunks(p: Params, Q, csum, qbar, cidx, stream=None) -> None:
     _check(load().hga_route_chunks(ctypes.byref(p.c()), _ptr(Q), _ptr(csum), _ptr(qbar), _ptr(cidx),
                                    _stream(stream)))
@@ -205,6 +217,54 @@ def attn_bwd_noalloc(p: Params, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg,
     _check(load().hga_attn_bwd_noalloc(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
                                        _ptr(lse), _ptr(dO), _ptr(gidx), _ptr(dQ), _ptr(dK_seg),
                                        _ptr(dV_seg), _stream(stream)))
+
+
+def stage_params(p: Params) -> Params:
+    """The parameter block of the staged problem (host-RAM KV tier): p with
+    T_hist replaced by the staged history rows round_up_64(nQB * wg * 8) and
+    k_c, k_g by p's index-row widths (so HGA_ALL keeps the same widths)."""
+    out = _Params()
+    _check(load().hga_stage_params(ctypes.byref(p.c()), ctypes.byref(out)))
+    return dataclasses.replace(p, T_hist=int(out.T_hist), k_c=int(out.k_c), k_g=int(out.k_g))
+
+
+def _hist_ptr(t: torch.Tensor | None):
+    """History rows may be a device tensor or a pinned host tensor."""
+    if t is None or t.numel() == 0:                  # no history rows (T_hist = 0)
+        return None
+    if not t.is_contiguous():
+        raise ValueError("libhga takes contiguous tensors")
+    if not t.is_cuda and not t.is_pinned():
+        raise ValueError("host-resident history must be in pinned memory")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def stage_routed(p: Params, K_hist, V_hist, K_seg, V_seg, gidx, K_stage, V_stage, gidx_stage,
+                 stream=None) -> None:
+    """Gather the routed history groups into K_stage / V_stage and remap gidx."""
+    _check(load().hga_stage_routed(ctypes.byref(p.c()), _hist_ptr(K_hist), _hist_ptr(V_hist), _ptr(K_seg),
+                                   _ptr(V_seg), _ptr(gidx), _ptr(K_stage), _ptr(V_stage), _ptr(gidx_stage),
+                                   _stream(stream)))
+
+
+class StagedKV:
+    """Host-RAM KV tier: history K/V rows stay in (pinned) host memory; after
+    routing on the full problem, the routed groups are staged in device
+    memory and the attention runs on the staged problem (``ps``), whose
+    results equal those of the full problem."""
+
+    def __init__(self, p: Params, device="cuda"):
+        self.p = p
+        self.ps = stage_params(p)
+        _, wg = route_widths(p)
+        B, Hkv, d, nQB = p.B, p.Hkv, p.d, p.nQB
+        rows = self.ps.T_hist + p.T_seg
+        self.K = torch.empty(B, Hkv, rows, d, device=device, dtype=p.torch_dtype)
+        self.V = torch.empty(B, Hkv, rows, d, device=device, dtype=p.torch_dtype)
+        self.gidx = torch.empty(B, Hkv, nQB, wg, device=device, dtype=torch.int32)
+
+    def stage(self, K_hist, V_hist, K_seg, V_seg, gidx, stream=None) -> None:
+        stage_routed(self.p, K_hist, V_hist, K_seg, V_seg, gidx, self.K, self.V, self.gidx, stream)
 
 
 class Buffers:

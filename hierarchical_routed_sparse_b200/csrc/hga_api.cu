@@ -101,7 +101,36 @@ cudaError_t run_attn_bwd(const hga::Shape& s, const void* Q, const void* K, cons
     return hga::launch_attn_bwd_simt(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, Drow, st);
 }
 
+// A pointer the device can load from: device (or managed) memory as it is,
+// device-mapped host memory by its device address; pageable host memory is
+// refused.
+int device_addressable(const void* ptr, const void** dev, const char* name)
+{
+    cudaPointerAttributes at;
+    const cudaError_t e = cudaPointerGetAttributes(&at, ptr);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(HGA_ERR_INVALID_ARG, "%s: the pointer is unknown to CUDA (%s)", name, cudaGetErrorName(e));
+    }
+    if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) {
+        *dev = ptr;
+        return HGA_OK;
+    }
+    if (at.type == cudaMemoryTypeHost && at.devicePointer != nullptr) {
+        *dev = at.devicePointer;
+        return HGA_OK;
+    }
+    return fail(HGA_ERR_INVALID_ARG, "%s: host memory the device cannot address (pin and map it)", name);
+}
+
 }  // namespace
+
+namespace hga {
+int64_t stage_hist_rows(const Shape& s);
+cudaError_t launch_stage(const Shape& s, const void* K_hist, const void* V_hist, const void* K_seg,
+                         const void* V_seg, const int32_t* gidx, void* K_stage, void* V_stage,
+                         int32_t* gidx_stage, cudaStream_t st);
+}
 
 extern "C" {
 
@@ -148,9 +177,26 @@ int hga_build_summaries(const hga_params* p, const void* K, int64_t t_begin, int
     CHECK_PTR(K);
     CHECK_PTR(csum);
     CHECK_PTR(gsum);
-    cudaError_t e = hga::launch_summaries(s, K, t_begin / 64, t_end / 64, csum, gsum,
+    cudaError_t e = hga::launch_summaries(s, K, s.T, 0, t_begin / 64, t_end / 64, csum, gsum,
                                           static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_build_summaries");
+}
+
+int hga_build_summaries_rows(const hga_params* p, const void* K_rows, int64_t t_begin, int64_t t_end,
+                             float* csum, float* gsum, hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (t_begin < 0 || t_end < t_begin || t_end > s.T || t_begin % 64 || t_end % 64)
+        return fail(HGA_ERR_INVALID_ARG, "need 0 <= t_begin <= t_end <= T with multiples of 64 (got %lld, %lld, T=%lld)",
+                    (long long)t_begin, (long long)t_end, (long long)s.T);
+    if (t_end == t_begin) return HGA_OK;
+    CHECK_PTR(K_rows);
+    CHECK_PTR(csum);
+    CHECK_PTR(gsum);
+    cudaError_t e = hga::launch_summaries(s, K_rows, t_end - t_begin, t_begin, t_begin / 64, t_end / 64, csum,
+                                          gsum, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_build_summaries_rows");
 }
 
 int hga_route_chunks(const hga_params* p, const void* Q, const float* csum, float* qbar,
@@ -203,6 +249,48 @@ int hga_route(const hga_params* p, const void* Q, const float* csum, const float
                     (long long)s.nC, s.wc);
     cudaError_t e = hga::launch_route_fused(s, Q, csum, gsum, qbar, cidx, gidx, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route");
+}
+
+int hga_stage_params(const hga_params* p, hga_params* staged)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (!staged) return fail(HGA_ERR_INVALID_ARG, "staged is NULL");
+    *staged = *p;
+    staged->T_hist = hga::stage_hist_rows(s);
+    // The staged problem keeps the routing's row widths: with HGA_ALL they
+    // would otherwise follow the staged T.
+    staged->k_c = s.wc;
+    staged->k_g = s.wg;
+    return HGA_OK;
+}
+
+int hga_stage_routed(const hga_params* p, const void* K_hist, const void* V_hist, const void* K_seg,
+                     const void* V_seg, const int32_t* gidx, void* K_stage, void* V_stage, int32_t* gidx_stage,
+                     hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    if (s.T_hist > 0) {
+        CHECK_PTR(K_hist);
+        CHECK_PTR(V_hist);
+    }
+    CHECK_PTR(K_seg);
+    CHECK_PTR(V_seg);
+    CHECK_PTR(gidx);
+    CHECK_PTR(K_stage);
+    CHECK_PTR(V_stage);
+    CHECK_PTR(gidx_stage);
+    const void* kh = K_hist;
+    const void* vh = V_hist;
+    if (s.T_hist > 0) {
+        if (int r = device_addressable(K_hist, &kh, "K_hist")) return r;
+        if (int r = device_addressable(V_hist, &vh, "V_hist")) return r;
+    }
+    const cudaError_t e = hga::launch_stage(s, kh, vh, K_seg, V_seg, gidx, K_stage, V_stage, gidx_stage,
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_stage_routed");
 }
 
 int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* V,

@@ -105,8 +105,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 // ---- launchers (each returns cudaError_t of its launch) ------------------------
-cudaError_t launch_summaries(const Shape& s, const void* K, int64_t c_begin, int64_t c_end,
-                             float* csum, float* gsum, cudaStream_t st);
+// K holds T_src rows per (batch, kv-head), the first of them at position row0.
+cudaError_t launch_summaries(const Shape& s, const void* K, int64_t T_src, int64_t row0, int64_t c_begin,
+                             int64_t c_end, float* csum, float* gsum, cudaStream_t st);
 cudaError_t launch_route_chunks(const Shape& s, const void* Q, const float* csum, float* qbar,
                                 int32_t* cidx, cudaStream_t st);
 cudaError_t launch_route_groups(const Shape& s, const float* qbar, const float* gsum,

@@ -19,8 +19,8 @@ namespace {
 
 template <typename TIn, int D>
 __global__ void __launch_bounds__(kGroupsPerChunk * D / Vec16<TIn>::E)
-summaries_kernel(const TIn* __restrict__ K, int64_t T, int64_t c_begin, int64_t n_chunks,
-                 float* __restrict__ csum, float* __restrict__ gsum)
+summaries_kernel(const TIn* __restrict__ K, int64_t T, int64_t T_src, int64_t row0, int64_t c_begin,
+                 int64_t n_chunks, float* __restrict__ csum, float* __restrict__ gsum)
 {
     constexpr int E = Vec16<TIn>::E;
     constexpr int V16 = D / E;                  // 16-byte vectors per row
@@ -32,7 +32,8 @@ summaries_kernel(const TIn* __restrict__ K, int64_t T, int64_t c_begin, int64_t 
     const int64_t c = c_begin + blockIdx.x % n_chunks;
     const int r = threadIdx.x / V16, v = threadIdx.x % V16;
 
-    const TIn* src = K + (bg * T + c * kChunk + r * kGroup) * D + v * E;
+    // K holds T_src rows per (batch, kv-head), the first at position row0.
+    const TIn* src = K + (bg * T_src + c * kChunk - row0 + r * kGroup) * D + v * E;
     float x[kGroup][E];
 #pragma unroll
     for (int t = 0; t < kGroup; ++t) Vec16<TIn>::load(src + t * D, x[t]);
@@ -61,26 +62,26 @@ summaries_kernel(const TIn* __restrict__ K, int64_t T, int64_t c_begin, int64_t 
 }
 
 template <typename TIn, int D>
-cudaError_t launch(const Shape& s, const void* K, int64_t c_begin, int64_t c_end, float* csum,
-                   float* gsum, cudaStream_t st)
+cudaError_t launch(const Shape& s, const void* K, int64_t T_src, int64_t row0, int64_t c_begin, int64_t c_end,
+                   float* csum, float* gsum, cudaStream_t st)
 {
     const int64_t n = c_end - c_begin;
     const int64_t blocks = n * s.B * s.Hkv;
     constexpr int threads = kGroupsPerChunk * D / Vec16<TIn>::E;
     return launch_pdl(summaries_kernel<TIn, D>, dim3((unsigned)blocks), dim3(threads), 0, st,
-                      static_cast<const TIn*>(K), s.T, c_begin, n, csum, gsum);
+                      static_cast<const TIn*>(K), s.T, T_src, row0, c_begin, n, csum, gsum);
 }
 
 }  // namespace
 
-cudaError_t launch_summaries(const Shape& s, const void* K, int64_t c_begin, int64_t c_end,
-                             float* csum, float* gsum, cudaStream_t st)
+cudaError_t launch_summaries(const Shape& s, const void* K, int64_t T_src, int64_t row0, int64_t c_begin,
+                             int64_t c_end, float* csum, float* gsum, cudaStream_t st)
 {
     if (s.dtype == HGA_BF16)
-        return s.d == 128 ? launch<__nv_bfloat16, 128>(s, K, c_begin, c_end, csum, gsum, st)
-                          : launch<__nv_bfloat16, 64>(s, K, c_begin, c_end, csum, gsum, st);
-    return s.d == 128 ? launch<float, 128>(s, K, c_begin, c_end, csum, gsum, st)
-                      : launch<float, 64>(s, K, c_begin, c_end, csum, gsum, st);
+        return s.d == 128 ? launch<__nv_bfloat16, 128>(s, K, T_src, row0, c_begin, c_end, csum, gsum, st)
+                          : launch<__nv_bfloat16, 64>(s, K, T_src, row0, c_begin, c_end, csum, gsum, st);
+    return s.d == 128 ? launch<float, 128>(s, K, T_src, row0, c_begin, c_end, csum, gsum, st)
+                      : launch<float, 64>(s, K, T_src, row0, c_begin, c_end, csum, gsum, st);
 }
 
 }  // namespace hga

@@ -98,6 +98,14 @@ int hga_build_summaries(const hga_params* p, const void* K, int64_t t_begin,
                         int64_t t_end, float* csum, float* gsum,
                         hga_stream_t stream);
 
+/* a1 for callers that hold only the rows being summarised on the device
+ * (e.g. with the history in host memory, see hga_stage_routed): the same as
+ * hga_build_summaries, but K_rows is [B][Hkv][t_end - t_begin][d] and holds
+ * tokens t_begin .. t_end-1 only. */
+int hga_build_summaries_rows(const hga_params* p, const void* K_rows,
+                             int64_t t_begin, int64_t t_end, float* csum,
+                             float* gsum, hga_stream_t stream);
+
 /* a2 + a3. Block queries and chunk routing (same section: the query scores
  * the chunk summaries and picks the top-k chunks).  Writes qbar (the mean
  * of the block's queries over the G q-heads of each kv-head) and cidx: for
@@ -171,6 +179,46 @@ int hga_attn_bwd_noalloc(const hga_params* p, const void* Q, const void* K,
                          const void* V, const float* O, const float* lse,
                          const void* dO, const int32_t* gidx, float* dQ,
                          float* dK_seg, float* dV_seg, hga_stream_t stream);
+
+/* Host-RAM KV tier (article section "How it fits in 16 GB": older KV can be
+ * held in host RAM; after routing only the selected groups' exact tokens are
+ * brought to the GPU).  The history rows of K and V (positions < T_hist)
+ * may live in pinned host memory that the device can address (memory from
+ * cudaHostAlloc / cudaMallocHost, or registered with cudaHostRegister with
+ * the mapped flag) or in device memory; the segment rows, the summaries and
+ * the index rows live in device memory as usual.
+ *
+ * hga_stage_params: the parameter block of the staged problem -- *staged =
+ * *p with T_hist replaced by T_stage = round_up_64(nQB * wg * 8), the
+ * number of staged history rows per (batch, kv-head), and k_c, k_g replaced
+ * by the row widths wc, wg of p (hga_route_widths), so that the staged index
+ * rows keep their width also under HGA_ALL. */
+int hga_stage_params(const hga_params* p, hga_params* staged);
+
+/* Gather, after routing, every routed history group into a device staging
+ * buffer and rewrite the index rows, so that hga_attn_fwd / hga_attn_bwd
+ * with the staged parameter block (hga_stage_params), K_stage, V_stage and
+ * gidx_stage compute exactly what they compute on the full K, V and gidx.
+ *   K_hist, V_hist  [B][Hkv][T_hist][d]  history rows (host-mapped or device)
+ *   K_seg, V_seg    [B][Hkv][T_seg][d]   segment rows (device)
+ *   gidx            [B][Hkv][nQB][wg]    routing of hga_route (device)
+ *   K_stage, V_stage [B][Hkv][T_stage + T_seg][d] (device, written): slot j
+ *       of block qb holds the 8 rows of that block's j-th routed history
+ *       group at rows (qb*wg + j)*8; the segment rows follow at T_stage.
+ *       Slots of padding or of segment groups are left untouched and are
+ *       never read by the attention kernels.
+ *   gidx_stage      [B][Hkv][nQB][wg] (device, written): a history group
+ *       becomes qb*wg + j, a segment group j' becomes T_stage/8 + j' -
+ *       T_hist/8, padding stays -1; rows stay ascending.
+ * The segment keys keep their offsets past the (staged) history, so
+ * dK_seg / dV_seg of the staged backward are those of the full problem.
+ * Host-resident history is read over the host link with plain loads.
+ * HGA_ERR_INVALID_ARG if K_hist / V_hist are neither device memory nor
+ * device-addressable host memory. */
+int hga_stage_routed(const hga_params* p, const void* K_hist, const void* V_hist,
+                     const void* K_seg, const void* V_seg, const int32_t* gidx,
+                     void* K_stage, void* V_stage, int32_t* gidx_stage,
+                     hga_stream_t stream);
 
 /* Status word of the kernels' bounded waits: every wait of a tensor-core
  * kernel on a barrier gives up after one second, records the code of the wait

@@ -116,3 +116,37 @@ def test_params_struct_layout_matches_header(lib, tmp_path):
                                           check=True).stdout.split()]
     assert out[0] == ctypes.sizeof(_Params)
     assert out[1:] == [getattr(_Params, f).offset for f in fields]
+
+
+def test_stage_params_round_history_to_whole_chunks(lib):
+    # T_stage = round_up_64(nQB * wg * 8); every other field unchanged.
+    p = _p()
+    ps = hga.stage_params(p)
+    assert ps.T_hist == 32 * 32 * 8 and (ps.T_seg, ps.k_c, ps.k_g, ps.d) == (p.T_seg, p.k_c, p.k_g, p.d)
+    ps = hga.stage_params(_p(T_seg=128, k_g=5))                  # 2 blocks x 5 groups x 8 = 80 -> 128
+    assert ps.T_hist == 128
+    ps = hga.stage_params(_p(T_hist=0, T_seg=64, k_g=3))          # 24 -> 64
+    assert ps.T_hist == 64
+    wg = hga.route_widths(_p(k_c=4, k_g=hga.HGA_ALL))[1]          # all groups of the chosen chunks
+    assert hga.stage_params(_p(k_c=4, k_g=hga.HGA_ALL)).T_hist == -(-32 * wg * 8 // 64) * 64
+    # The staged problem keeps the index-row widths (HGA_ALL would follow T).
+    for kw in (dict(), dict(k_c=hga.HGA_ALL, k_g=hga.HGA_ALL), dict(k_c=4, k_g=hga.HGA_ALL),
+               dict(T_hist=192, T_seg=256, k_c=hga.HGA_ALL, k_g=hga.HGA_ALL)):
+        assert hga.route_widths(hga.stage_params(_p(**kw))) == hga.route_widths(_p(**kw)), kw
+    assert lib.hga_stage_params(ctypes.byref(_p(T_hist=100).c()), ctypes.byref(_Params())) == \
+        hga.HGA_ERR_INVALID_ARG
+    assert lib.hga_stage_params(ctypes.byref(_p().c()), None) == hga.HGA_ERR_INVALID_ARG
+
+
+def test_stage_routed_rejects_bad_pointers_on_the_host(lib):
+    p = _p()
+    P = ctypes.c_void_p
+    ok, mis = P(0x10000), P(0x10008)
+    args = [ok] * 8
+    # NULL segment rows and a misaligned staging buffer are refused before
+    # any CUDA call (the history pointers are checked first only when set).
+    for i, bad in ((2, None), (6, mis)):
+        a = list(args)
+        a[i] = bad
+        assert lib.hga_stage_routed(ctypes.byref(p.c()), *a, None) == hga.HGA_ERR_INVALID_ARG
+    assert lib.hga_stage_routed(ctypes.byref(_p(T_seg=0).c()), *([None] * 8), None) == hga.HGA_OK
