@@ -587,6 +587,65 @@ def run_host_tier(args, w) -> None:
         dist.destroy_process_group()
 
 
+def run_layer(args, w) -> None:
+    """Segment-wise (TBPTT) training of one attention layer with HGA as its
+    attention: Q / K / V / O projections of the workload's head layout over
+    d_model = Hq * d (bf16 autocast), HGA forward and backward per segment,
+    an SGD step per segment.  The sequence is the workload's T tokens in
+    T / T_seg segments, so the last segment sees the workload's history.
+    One JSON line, config.mode = "layer_tbptt"."""
+    import torch
+
+    import hierarchical_routed_sparse_b200 as hga
+    from hierarchical_routed_sparse_b200.segment import HGASegmentLayer
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    d_model = w.Hq * w.d
+    layer = HGASegmentLayer(d_model, w.Hq, w.Hkv, w.d, k_c=w.k_c, k_g=w.k_g)
+    opt = torch.optim.SGD(layer.parameters(), lr=1e-4)
+    x = torch.randn(w.B, w.T, d_model, device=dev, generator=g)
+    target = torch.randn(w.B, w.T, d_model, device=dev, generator=g)
+    n_seg = w.T // w.T_seg
+    stream = torch.cuda.current_stream(dev)
+
+    def sequence():
+        layer.cache.reset()
+        for s in range(n_seg):
+            xs = x[:, s * w.T_seg:(s + 1) * w.T_seg]
+            ts = target[:, s * w.T_seg:(s + 1) * w.T_seg]
+            with torch.autocast("cuda", dtype=torch.bfloat16):
+                out = layer.segment(xs)
+                loss = 0.5 * (out.float() - ts).pow(2).mean()
+            loss.backward()
+            opt.step()
+            opt.zero_grad(set_to_none=True)
+
+    for _ in range(args.warmup):
+        sequence()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(0, None) as clk:
+        for a, b in ev:
+            a.record(stream)
+            sequence()
+            b.record(stream)
+        torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    assert hga.device_status() == 0
+    line = dict(metric="HGA attention layer, segment-wise training: tokens/s", value=w.B * w.T / (ms * 1e-3),
+                unit="tokens/s", n_gpus=1, steps=args.steps, warmup=args.warmup, ms_per_step=ms,
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16 (autocast projections)",
+                data="synthetic",
+                config=dict(config_of(w), mode="layer_tbptt", d_model=d_model, segments=n_seg,
+                            l2="not flushed (a pass streams far more than L2)",
+                            launch="eager PyTorch autograd, events around each pass",
+                            step="one pass over the T tokens: per segment projections, HGA fwd + bwd, SGD"),
+                clocks=clk.summary())
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -599,6 +658,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager launches instead of a CUDA graph of the step")
+    ap.add_argument("--layer", action="store_true",
+                    help="segment-wise training of one attention layer with HGA (f4 integration)")
     ap.add_argument("--kv-tier", choices=["hbm", "host"], default="hbm",
                     help="host: history K/V in pinned host memory, routed groups staged per step")
     ap.add_argument("--traffic", type=float, default=None,
@@ -607,6 +668,8 @@ def main():
     w = W.BY_NAME[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.layer:
+        run_layer(args, w)
     elif args.kv_tier == "host":
         run_host_tier(args, w)
     else:

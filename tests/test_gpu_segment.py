@@ -1,0 +1,162 @@
+"""HGA as a drop-in attention module in a segment-wise (TBPTT) training loop
+(article "BMW's 16 GB GPU just did what needs an A100", section "What HGA
+does differently": HGA replaces the attention module; segments attend the
+exact tokens of earlier segments; older KV is detached).
+
+The layer's losses and weight gradients, summed over the segments of a
+sequence, are compared with the same layer whose attention is an
+independent float32 PyTorch computation of the routed attention: a dense
+masked softmax over the history (detached) and the segment, the mask built
+from the routing the HGA layer used (frozen, so only the attention and its
+autograd wiring are under test; the routing itself is checked against the
+oracle elsewhere).  The reference sees the same bf16-rounded Q / K / V,
+and, like the layer, passes the attention backward a bf16 dO.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import hierarchical_routed_sparse_b200 as hga
+from hierarchical_routed_sparse_b200.segment import HGASegmentLayer, run_tbptt
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from hierarchical_routed_sparse_b200 import build
+    build.build()
+    hga.load()
+
+
+class _Cast(torch.autograd.Function):
+    """float32 -> dtype -> float32 both ways, as the layer's activation cast:
+    the value is rounded to dtype and so is the gradient that flows back
+    (autograd hands a dtype input a dtype gradient)."""
+
+    @staticmethod
+    def forward(ctx, t, dtype):
+        ctx.dtype = dtype
+        return t.to(dtype).float()
+
+    @staticmethod
+    def backward(ctx, g):
+        return g.to(ctx.dtype).float(), None
+
+
+def _round(t, dtype):
+    return _Cast.apply(t, dtype)
+
+
+class _GradCast(torch.autograd.Function):
+    """Identity forward; the gradient is rounded to dtype -- the layer hands
+    the attention backward dO in the activations' dtype."""
+
+    @staticmethod
+    def forward(ctx, t, dtype):
+        ctx.dtype = dtype
+        return t.view_as(t)
+
+    @staticmethod
+    def backward(ctx, g):
+        return g.to(ctx.dtype).float(), None
+
+
+def _mask(gidx, T_hist, Ts, T):
+    """allowed[b, g, i, t]: key t is in a routed group of query i's block, or
+    in i's own chunk at or before i."""
+    Bn, Hkv, nQB, wg = gidx.shape
+    allowed = torch.zeros(Bn, Hkv, Ts, T, dtype=torch.bool, device=gidx.device)
+    i = torch.arange(Ts, device=gidx.device)
+    t = torch.arange(T, device=gidx.device)
+    own = (t[None, :] >= T_hist + 64 * (i[:, None] // 64)) & (t[None, :] <= T_hist + i[:, None])
+    allowed |= own[None, None]
+    g = gidx.clamp(min=0).long()
+    valid = gidx >= 0
+    grp_of_t = t // 8
+    for qb in range(nQB):
+        sel = torch.zeros(Bn, Hkv, T // 8 + 1, dtype=torch.bool, device=gidx.device)
+        sel.scatter_(2, torch.where(valid[:, :, qb], g[:, :, qb], T // 8), True)
+        allowed[:, :, 64 * qb:64 * qb + 64, :] |= sel[:, :, grp_of_t][:, :, None, :]
+    return allowed
+
+
+def _reference_tbptt(layer, x, target, seg_len, gidx_list):
+    """Same projections and loss; routed attention written as a masked dense
+    softmax in float32 with autograd."""
+    Hq, Hkv, d = layer.Hq, layer.Hkv, layer.d
+    G = Hq // Hkv
+    Kh = Vh = None
+    losses = []
+    for s_i, s in enumerate(range(0, x.shape[1], seg_len)):
+        xs, ts = x[:, s:s + seg_len], target[:, s:s + seg_len]
+        Bn, Ts, _ = xs.shape
+        q = _round(layer.wq(xs).view(Bn, Ts, Hq, d).transpose(1, 2), layer.act_dtype)
+        k = _round(layer.wk(xs).view(Bn, Ts, Hkv, d).transpose(1, 2), layer.act_dtype)
+        v = _round(layer.wv(xs).view(Bn, Ts, Hkv, d).transpose(1, 2), layer.act_dtype)
+        T_hist = 0 if Kh is None else Kh.shape[2]
+        Kall = k if Kh is None else torch.cat([Kh, k], dim=2)
+        Vall = v if Vh is None else torch.cat([Vh, v], dim=2)
+        T = T_hist + Ts
+        allowed = _mask(gidx_list[s_i], T_hist, Ts, T)                     # [B][Hkv][Ts][T]
+        Kr = Kall.repeat_interleave(G, dim=1)
+        Vr = Vall.repeat_interleave(G, dim=1)
+        S = torch.einsum("bhid,bhtd->bhit", q, Kr) / math.sqrt(d)
+        S = S.masked_fill(~allowed.repeat_interleave(G, dim=1), float("-inf"))
+        O = _GradCast.apply(torch.einsum("bhit,bhtd->bhid", torch.softmax(S, dim=-1), Vr), layer.act_dtype)
+        out = layer.wo(O.transpose(1, 2).reshape(Bn, Ts, Hq * d))
+        loss = 0.5 * (out - ts).pow(2).mean()
+        loss.backward()
+        losses.append(float(loss.detach()))
+        Kh = Kall.detach()
+        Vh = Vall.detach()
+    return losses
+
+
+@pytest.mark.parametrize("dtype,d,k_c,k_g", [(torch.bfloat16, 128, 3, 12), (torch.float32, 64, 2, 7),
+                                             (torch.bfloat16, 128, hga.HGA_ALL, hga.HGA_ALL)],
+                         ids=["bf16_d128", "fp32_d64", "bf16_all_routing"])
+def test_tbptt_layer_matches_masked_reference(dtype, d, k_c, k_g):
+    torch.manual_seed(0)
+    d_model, Hq, Hkv, seg, T = 192, 4, 2, 256, 1024
+    layer = HGASegmentLayer(d_model, Hq, Hkv, d, k_c=k_c, k_g=k_g, dtype=dtype)
+    x = torch.randn(2, T, d_model, device="cuda")
+    target = torch.randn(2, T, d_model, device="cuda")
+    gidx_list = []
+    layer.cache.reset()
+    losses = []
+    for s in range(0, T, seg):                     # run_tbptt, keeping each segment's routing
+        out = layer.segment(x[:, s:s + seg])
+        gidx_list.append(layer.last_gidx)
+        loss = 0.5 * (out - target[:, s:s + seg]).pow(2).mean()
+        loss.backward()
+        losses.append(float(loss.detach()))
+    torch.cuda.synchronize()
+    assert hga.device_status() == 0
+    got = {n: p.grad.clone() for n, p in layer.named_parameters()}
+    for p in layer.parameters():
+        p.grad = None
+    ref_losses = _reference_tbptt(layer, x, target, seg, gidx_list)
+    np.testing.assert_allclose(losses, ref_losses, rtol=1e-4)
+    for n, p in layer.named_parameters():
+        rel = float((got[n] - p.grad).norm() / p.grad.norm())
+        assert rel < 2e-3, f"{n}: relative gradient error {rel:.3g}"
+
+
+def test_history_is_detached_and_run_tbptt_trains():
+    # Only the last segment's loss reaches the weights through that segment;
+    # gradients of a later segment do not change with the earlier segments'
+    # inputs once the history K/V are fixed.  And an optimiser loop runs.
+    torch.manual_seed(1)
+    layer = HGASegmentLayer(128, 2, 1, 128, k_c=2, k_g=8)
+    x = torch.randn(1, 512, 128, device="cuda")
+    target = torch.randn(1, 512, 128, device="cuda")
+    opt = torch.optim.SGD(layer.parameters(), lr=1e-2)
+    l0 = run_tbptt(layer, x, target, 256, opt)
+    l1 = run_tbptt(layer, x, target, 256, opt)
+    assert len(l0) == 2 and all(np.isfinite(l0 + l1))
+    assert layer.cache.T_hist == 512
