@@ -102,10 +102,11 @@ def _load():
         lib.oracle_route_groups.argtypes = [D, P, P, P, P, P]
         lib.oracle_attn_fwd.argtypes = [D, P, P, P, P, P, P]
         lib.oracle_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, P]
+        lib.oracle_decode.argtypes = [D, ctypes.c_int64, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         for f in ("oracle_build_summaries", "oracle_block_query", "oracle_route_chunks",
-                  "oracle_route_groups", "oracle_attn_fwd", "oracle_attn_bwd",
+                  "oracle_route_groups", "oracle_attn_fwd", "oracle_attn_bwd", "oracle_decode",
                   "oracle_set_num_threads"):
             getattr(lib, f).restype = None
         _lib = lib
@@ -198,6 +199,24 @@ def attn_bwd(dims: Dims, Q, K, V, dO, gidx):
     _load().oracle_attn_bwd(ctypes.byref(dims._c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(dO),
                             _ptr(gidx), _ptr(dQ), _ptr(dK), _ptr(dV))
     return dQ, dK, dV
+
+
+def decode(dims: Dims, pos: int, q, K, V, csum, gsum):
+    """One generation step for the token at position pos (a query block of
+    one): q [B,Hq,d]; K, V [B,Hkv,T,d] with rows 0..pos valid; csum / gsum of
+    the complete chunks.  Returns dict(O [B,Hq,d], lse [B,Hq], cidx, gidx
+    [B,Hkv,w], cgap, ggap [B,Hkv])."""
+    q, K, V, csum, gsum = _f64(q), _f64(K), _f64(V), _f64(csum), _f64(gsum)
+    B, Hq, Hkv, d = dims.B, dims.Hq, dims.Hkv, dims.d
+    O = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    cidx = np.full((B, Hkv, dims.wc), -7, dtype=np.int32)
+    gidx = np.full((B, Hkv, dims.wg), -7, dtype=np.int32)
+    cgap = np.zeros((B, Hkv))
+    ggap = np.zeros((B, Hkv))
+    _load().oracle_decode(ctypes.byref(dims._c()), int(pos), _ptr(q), _ptr(K), _ptr(V), _ptr(csum),
+                          _ptr(gsum), _ptr(O), _ptr(lse), _ptr(cidx), _ptr(gidx), _ptr(cgap), _ptr(ggap))
+    return dict(O=O, lse=lse, cidx=cidx, gidx=gidx, cgap=cgap, ggap=ggap)
 
 
 def route(dims: Dims, Q, K):

@@ -359,6 +359,94 @@ void oracle_attn_bwd(const oracle_dims* p, const double* Q, const double* K,
     }
 }
 
+/* ------------------------------------------------------------ decode ---- */
+/* One generation step (article section "Retrieval: no degradation in the
+ * dense baseline": HGA itself can also do generation): the new token at position pos
+ * is a query block of one.  q [B][Hq][d]; K, V [B][Hkv][T][d] with rows
+ * 0..pos valid (pos < T = T_hist + T_seg, the capacity); csum / gsum as for
+ * the segment calls, rows of the complete chunks < pos/chunk used.
+ *   qbar  = mean of the token's query over the G q-heads of the kv-head (R3
+ *           with a block of one);
+ *   chunks c < c0 = pos / chunk eligible (R4), top-k_c (R6, R7), gap (R8);
+ *   groups of the chosen chunks, top-k_g (R5);
+ *   O, lse: exact softmax over the routed groups' tokens and the own chunk's
+ *           tokens c0*chunk .. pos (R9).
+ * Outputs: O [B][Hq][d], lse [B][Hq], cidx [B][Hkv][wc], gidx [B][Hkv][wg],
+ * cgap, ggap [B][Hkv]. */
+void oracle_decode(const oracle_dims* p, int64_t pos, const double* q, const double* K,
+                   const double* V, const double* csum, const double* gsum, double* O,
+                   double* lse, int32_t* cidx, int32_t* gidx, double* cgap, double* ggap)
+{
+    const int G = p->Hq / p->Hkv, d = p->d, gpc = p->chunk / p->group;
+    const int64_t T = total_len(p), nC = T / p->chunk, nG = T / p->group;
+    const int64_t c0 = pos / p->chunk;
+    const int64_t units = (int64_t)p->B * p->Hkv;
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t u = 0; u < units; ++u) {
+        const int64_t b = u / p->Hkv, g = u % p->Hkv;
+        double* qbar = (double*)malloc(sizeof(double) * (size_t)d);
+        for (int e = 0; e < d; ++e) {
+            double a = 0.0;
+            for (int h = 0; h < G; ++h) a += q[((b * p->Hq) + g * G + h) * d + e];
+            qbar[e] = a / (double)G;
+        }
+        /* chunk routing */
+        cand* list = (cand*)malloc(sizeof(cand) * (size_t)((c0 > 0 ? c0 : 1) + p->wc * gpc + 1));
+        for (int64_t c = 0; c < c0; ++c) {
+            list[c].s = dot(qbar, csum + (u * nC + c) * d, d);
+            list[c].idx = c;
+        }
+        cgap[u] = select_top(list, c0, p->k_c, cidx + u * p->wc, p->wc);
+        /* group routing */
+        int64_t n = 0;
+        for (int i = 0; i < p->wc; ++i) {
+            const int32_t c = cidx[u * p->wc + i];
+            if (c < 0) continue;
+            for (int r = 0; r < gpc; ++r) {
+                const int64_t j = (int64_t)c * gpc + r;
+                list[n].s = dot(qbar, gsum + (u * nG + j) * d, d);
+                list[n].idx = j;
+                ++n;
+            }
+        }
+        ggap[u] = select_top(list, n, p->k_g, gidx + u * p->wg, p->wg);
+        free(list);
+        /* attention of each q-head of the kv-head */
+        const int32_t* grow = gidx + u * p->wg;
+        int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * (size_t)(p->wg * p->group + p->chunk));
+        double* s = (double*)malloc(sizeof(double) * (size_t)(p->wg * p->group + p->chunk));
+        int64_t nk = 0;
+        for (int r = 0; r < p->wg; ++r) {
+            if (grow[r] < 0) continue;
+            for (int t = 0; t < p->group; ++t) keys[nk++] = (int64_t)grow[r] * p->group + t;
+        }
+        for (int64_t t = c0 * p->chunk; t <= pos; ++t) keys[nk++] = t;
+        const double* Kh = K + u * T * d;
+        const double* Vh = V + u * T * d;
+        for (int h = 0; h < G; ++h) {
+            const int64_t row = b * p->Hq + g * G + h;
+            const double* qh = q + row * d;
+            double m = -INFINITY;
+            for (int64_t j = 0; j < nk; ++j) {
+                s[j] = p->scale * dot(qh, Kh + keys[j] * d, d);
+                if (s[j] > m) m = s[j];
+            }
+            double l = 0.0;
+            for (int64_t j = 0; j < nk; ++j) { s[j] = exp(s[j] - m); l += s[j]; }
+            double* o = O + row * d;
+            for (int e = 0; e < d; ++e) o[e] = 0.0;
+            for (int64_t j = 0; j < nk; ++j) {
+                const double w = s[j] / l;
+                for (int e = 0; e < d; ++e) o[e] += w * Vh[keys[j] * d + e];
+            }
+            lse[row] = m + log(l);
+        }
+        free(keys);
+        free(s);
+        free(qbar);
+    }
+}
+
 /* Number of worker threads the oracle runs with. */
 int oracle_num_threads(void)
 {
