@@ -646,6 +646,150 @@ def run_layer(args, w) -> None:
     print(json.dumps(line), flush=True)
 
 
+def decode_algorithmic(w, pos: int) -> dict:
+    """Algorithmic bytes of one hga_decode call at position pos: the token's
+    queries, the eligible chunk summaries, the group summaries of the routed
+    chunks, the routed groups' and the own chunk's K / V rows, and the
+    outputs (O, lse, cidx, gidx)."""
+    el = 2 if w.dtype == "bf16" else 4
+    c0 = pos // 64
+    nc = c0 if w.k_c <= 0 else min(w.k_c, c0)
+    ng = 8 * nc if w.k_g <= 0 else min(w.k_g, 8 * nc)
+    n_keys = 8 * ng + pos - 64 * c0 + 1
+    wc = w.k_c if w.k_c > 0 else w.T // 64
+    wg = w.k_g if w.k_g > 0 else 8 * wc
+    per_unit = (w.G * w.d * el + c0 * w.d * 4 + 8 * nc * w.d * 4 + 2 * n_keys * w.d * el
+                + w.G * (w.d + 1) * 4 + (wc + wg) * 4)
+    return dict(bytes=w.B * w.Hkv * per_unit, n_keys=n_keys)
+
+
+def oracle_decode_rate(w, pos0: int, min_seconds: float = 10.0, max_reps: int = 1_000_000) -> dict:
+    """The oracle's decode step on the first sequence of the batch, at the
+    positions the GPU run decodes, repeated for about min_seconds."""
+    import oracle
+    oracle.build()
+    w1 = w.with_(B=1)
+    x = w1.full()
+    K, V = x["K"].astype(np.float64), x["V"].astype(np.float64)
+    dims = oracle.Dims(B=1, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T_hist=w.T_hist, T_seg=w.T_seg, k_c=w.k_c, k_g=w.k_g)
+    csum, gsum = oracle.build_summaries(dims, K)
+    q = x["Q"][:, :, 0].astype(np.float64)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode(dims, pos0 + reps % 64, q, K, V, csum, gsum)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= max_reps:
+            break
+    return dict(value=reps / el, unit="tokens/s", cores=oracle.num_threads(), kind="oracle", seconds=el,
+                sample=f"{reps} decode steps of one sequence ({w.Hq} q-heads, {w.Hkv} kv-heads, ctx {w.T}), "
+                       "float64, OpenMP over kv-heads",
+                cpu=_cpu_model())
+
+
+def run_decode(args, w) -> None:
+    """Generation with HGA: one decode step per token (hga_decode) over a
+    KV cache of the workload's T rows, for a batch of sequences.  The timed
+    steps decode the last 64 positions of the cache (T-64 .. T-1) in order;
+    the step that completes the chunk also appends its summaries
+    (hga_build_summaries).  Each step is timed alone with CUDA events, L2
+    flushed before it.  One JSON line, config.mode = "decode"."""
+    import torch
+
+    import hierarchical_routed_sparse_b200 as hga
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wd = w.with_(B=args.decode_batch, backward=False)
+    x = wd.full()
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    p = hga.Params.from_workload(wd)
+    st = hga.DecodeState(p, device=dev)
+    K = torch.from_numpy(x["K"]).to(dev, tdt)
+    V = torch.from_numpy(x["V"]).to(dev, tdt)
+    pos0 = wd.T - 64
+    st.prefill(K[:, :, :pos0], V[:, :, :pos0])
+    st.K.copy_(K)                                   # rows of the timed tokens already in place
+    st.V.copy_(V)
+    del K, V
+    qs = [torch.from_numpy(np.ascontiguousarray(x["Q"][:, :, i])).to(dev, tdt) for i in range(64)]
+    del x
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, s=None):
+        pos = pos0 + i % 64
+        hga.decode(p, pos, qs[i % 64], st.K, st.V, st.csum, st.gsum, st.O, st.lse, st.cidx, st.gidx, s)
+        if (pos + 1) % 64 == 0:
+            hga.build_summaries(p, st.K, pos + 1 - 64, pos + 1, st.csum, st.gsum, s)
+
+    for i in range(max(args.warmup, 3)):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    n = max(args.steps, 64)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    launches = 0
+    with ClockSampler(0, None) as clk:
+        # A decode call is shorter than its host-side launch path (Python
+        # marshalling + C-ABI checks): a GPU-side delay first lets the host
+        # queue every timed step ahead, so the events time the device work.
+        torch.cuda._sleep(int(1e8))
+        for i in range(n):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
+            launches += 1 + ((pos0 + i % 64 + 1) % 64 == 0)
+        torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    ms_step = statistics.mean(ms)
+    # Decode calls alone (steps that do not append summaries).
+    dec_ms = statistics.mean(m for i, m in enumerate(ms) if (pos0 + i % 64 + 1) % 64 != 0)
+    # End to end through the public API: q from pinned host memory, O back;
+    # no delay ahead, so the host's launch path counts.
+    el = 2 if w.dtype == "bf16" else 4
+    q_host = [q.cpu().pin_memory() for q in qs]
+    o_host = torch.empty(st.O.shape, dtype=torch.float32).pin_memory()
+    q_dev = torch.empty_like(qs[0])
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        flush.zero_()
+        ev2[i][0].record(stream)
+        q_dev.copy_(q_host[i % 64], non_blocking=True)
+        pos = pos0 + i % 64
+        hga.decode(p, pos, q_dev, st.K, st.V, st.csum, st.gsum, st.O, st.lse, st.cidx, st.gidx)
+        if (pos + 1) % 64 == 0:
+            hga.build_summaries(p, st.K, pos + 1 - 64, pos + 1, st.csum, st.gsum)
+        o_host.copy_(st.O, non_blocking=True)
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in ev2)
+    assert hga.device_status() == 0
+    pk = peaks()
+    alg = statistics.mean(decode_algorithmic(wd, pos0 + i)["bytes"] for i in range(63))
+    achieved = alg / (dec_ms * 1e-3) / 1e9
+    line = dict(metric="HGA decode tokens/s at 16K ctx (one token per sequence per step)",
+                value=wd.B / (ms_step * 1e-3), unit="tokens/s", n_gpus=1, steps=n, warmup=args.warmup,
+                ms_per_step=ms_step, higher_is_better=True, scaling="weak", vs_baseline=None, dtype=w.dtype,
+                data="synthetic",
+                config=dict(config_of(wd, graph=False), mode="decode", decode_batch=wd.B,
+                            positions=f"{pos0}..{wd.T - 1}, summaries appended at chunk end",
+                            l2="flushed before every step (256 MiB write)",
+                            launch="eager, CUDA events around each step"),
+                decode_call_ms=dec_ms,
+                roofline=dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
+                              frac=achieved / pk["hbm_gbs"], traffic=None,
+                              kernel="decode_kernel", algorithmic_bytes_per_call=alg,
+                              peak_source=pk["source"] + " (burst copy)"),
+                e2e=dict(value=wd.B / (e2e_ms * 1e-3), unit="tokens/s", h2d_bytes_per_step=wd.B * wd.Hq * wd.d * el,
+                         d2h_bytes_per_step=wd.B * wd.Hq * wd.d * 4),
+                gpu_launches=launches, clocks=clk.summary())
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_decode_rate(wd, pos0)
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -662,12 +806,17 @@ def main():
                     help="segment-wise training of one attention layer with HGA (f4 integration)")
     ap.add_argument("--kv-tier", choices=["hbm", "host"], default="hbm",
                     help="host: history K/V in pinned host memory, routed groups staged per step")
+    ap.add_argument("--decode", action="store_true",
+                    help="generation: one hga_decode step per token over the workload's context (f3)")
+    ap.add_argument("--decode-batch", type=int, default=1, help="sequences decoded per step")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu DRAM bytes per launch of the dominant kernel, if captured")
     args = ap.parse_args()
     w = W.BY_NAME[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.decode:
+        run_decode(args, w)
     elif args.layer:
         run_layer(args, w)
     elif args.kv_tier == "host":

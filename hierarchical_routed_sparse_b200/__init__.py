@@ -6,15 +6,16 @@ Method source: the article "BMW's 16 GB GPU just did what needs an A100"
 (``build_summaries``, ``route_chunks``, ``route_groups``, ``attn_fwd``,
 ``attn_bwd``, ``stage_routed`` ...) mirror the C ABI one to one; ``Buffers``
 holds the device buffers of one problem shape and runs a whole segment step;
-``StagedKV`` runs the attention on history kept in host memory.
+``StagedKV`` runs the attention on history kept in host memory;
+``DecodeState`` generates token by token (hga_decode).
 """
 from .binding import (EXPORTS, HGA_ALL, HGA_BF16, HGA_ERR_CUDA, HGA_ERR_INVALID_ARG,
                       HGA_ERR_UNSUPPORTED, HGA_FP32, HGA_OK, LIB_PATH, NOALLOC_MAX_ROWS, Buffers,
-                      HGAError, Params, StagedKV,
-                      attn_bwd, attn_bwd_noalloc, attn_fwd, build_summaries, build_summaries_rows, device_status, load, route, route_chunks, route_groups,
+                      DecodeState, HGAError, Params, StagedKV,
+                      attn_bwd, attn_bwd_noalloc, attn_fwd, build_summaries, decode, build_summaries_rows, device_status, load, route, route_chunks, route_groups,
                       route_widths, stage_params, stage_routed, version, workspace_size)
 
 __all__ = ["EXPORTS", "HGA_ALL", "HGA_BF16", "HGA_FP32", "HGA_OK", "HGA_ERR_CUDA",
            "HGA_ERR_INVALID_ARG", "HGA_ERR_UNSUPPORTED", "LIB_PATH", "NOALLOC_MAX_ROWS", "Buffers", "HGAError",
-           "Params", "StagedKV", "stage_params", "stage_routed", "attn_bwd", "attn_bwd_noalloc", "attn_fwd", "build_summaries", "build_summaries_rows", "device_status", "load", "route", "route_chunks",
+           "DecodeState", "Params", "StagedKV", "decode", "stage_params", "stage_routed", "attn_bwd", "attn_bwd_noalloc", "attn_fwd", "build_summaries", "build_summaries_rows", "device_status", "load", "route", "route_chunks",
            "route_groups", "route_widths", "version", "workspace_size"]

@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhga.so")
 EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_build_summaries_rows",
            "hga_route_chunks",
            "hga_route_groups", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
-           "hga_stage_params", "hga_stage_routed", "hga_device_status", "hga_last_error",
+           "hga_stage_params", "hga_stage_routed", "hga_decode", "hga_device_status", "hga_last_error",
            "hga_version")
 NOALLOC_MAX_ROWS = 1 << 20     # HGA_NOALLOC_MAX_ROWS
 
@@ -111,6 +111,7 @@ def load() -> ctypes.CDLL:
             "hga_attn_bwd_noalloc": ([PP, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_stage_params": ([PP, PP], ctypes.c_int),
             "hga_stage_routed": ([PP, P, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "hga_decode": ([PP, I64, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_device_status": ([ctypes.POINTER(ctypes.c_int), ctypes.c_int], ctypes.c_int),
             "hga_last_error": ([], ctypes.c_char_p),
             "hga_version": ([], ctypes.c_char_p),
@@ -245,6 +246,66 @@ def stage_routed(p: Params, K_hist, V_hist, K_seg, V_seg, gidx, K_stage, V_stage
     _check(load().hga_stage_routed(ctypes.byref(p.c()), _hist_ptr(K_hist), _hist_ptr(V_hist), _ptr(K_seg),
                                    _ptr(V_seg), _ptr(gidx), _ptr(K_stage), _ptr(V_stage), _ptr(gidx_stage),
                                    _stream(stream)))
+
+
+def decode(p: Params, pos: int, q, K, V, csum, gsum, O, lse, cidx, gidx, stream=None) -> None:
+    """One decode step of the token at position ``pos`` (rows 0..pos of K / V
+    valid, summaries of the chunks before pos // 64 built)."""
+    _check(load().hga_decode(ctypes.byref(p.c()), int(pos), _ptr(q), _ptr(K), _ptr(V), _ptr(csum), _ptr(gsum),
+                             _ptr(O), _ptr(lse), _ptr(cidx), _ptr(gidx), _stream(stream)))
+
+
+class DecodeState:
+    """Generation with HGA: a KV cache of ``p.T`` rows and its summaries.
+
+    ``prefill`` fills the first rows; each ``step`` writes the new token's
+    K / V row, runs hga_decode for it, and appends the summaries of its chunk
+    once the chunk's 64 tokens are in the cache."""
+
+    def __init__(self, p: Params, device="cuda"):
+        self.p = p
+        wc, wg = route_widths(p)
+        B, Hq, Hkv, d, T = p.B, p.Hq, p.Hkv, p.d, p.T
+        f32 = dict(device=device, dtype=torch.float32)
+        i32 = dict(device=device, dtype=torch.int32)
+        self.K = torch.zeros(B, Hkv, T, d, device=device, dtype=p.torch_dtype)
+        self.V = torch.zeros(B, Hkv, T, d, device=device, dtype=p.torch_dtype)
+        self.csum = torch.zeros(B, Hkv, T // 64, d, **f32)
+        self.gsum = torch.zeros(B, Hkv, T // 8, d, **f32)
+        self.O = torch.empty(B, Hq, d, **f32)
+        self.lse = torch.empty(B, Hq, **f32)
+        self.cidx = torch.empty(B, Hkv, wc, **i32)
+        self.gidx = torch.empty(B, Hkv, wg, **i32)
+        self.pos = 0                               # tokens in the cache
+
+    def prefill(self, K, V, stream=None) -> None:
+        """Rows [0, n) of the cache from K, V [B][Hkv][n][d]; summaries of the
+        complete chunks among them."""
+        n = K.shape[2]
+        if n > self.p.T:
+            raise ValueError(f"prefill of {n} rows exceeds the cache of {self.p.T}")
+        self.K[:, :, :n] = K
+        self.V[:, :, :n] = V
+        full = n - n % 64
+        if full:
+            build_summaries(self.p, self.K, 0, full, self.csum, self.gsum, stream)
+        self.pos = n
+
+    def step(self, q, k, v, stream=None):
+        """Decode the token with queries q [B][Hq][d] and key / value rows
+        k, v [B][Hkv][d]; returns O [B][Hq][d] (float32, a view of the
+        state's buffer)."""
+        pos = self.pos
+        if pos >= self.p.T:
+            raise ValueError(f"the cache of {self.p.T} rows is full")
+        self.K[:, :, pos] = k
+        self.V[:, :, pos] = v
+        decode(self.p, pos, q, self.K, self.V, self.csum, self.gsum, self.O, self.lse, self.cidx, self.gidx,
+               stream)
+        if (pos + 1) % 64 == 0:
+            build_summaries(self.p, self.K, pos + 1 - 64, pos + 1, self.csum, self.gsum, stream)
+        self.pos = pos + 1
+        return self.O
 
 
 class StagedKV:

@@ -293,6 +293,34 @@ int hga_stage_routed(const hga_params* p, const void* K_hist, const void* V_hist
     return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_stage_routed");
 }
 
+int hga_decode(const hga_params* p, int64_t pos, const void* q, const void* K, const void* V,
+               const float* csum, const float* gsum, float* O, float* lse, int32_t* cidx, int32_t* gidx,
+               hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = make_shape(p, &s)) return r;
+    if (pos < 0 || pos >= s.T)
+        return fail(HGA_ERR_INVALID_ARG, "pos (%lld) must lie in [0, T=%lld)", (long long)pos, (long long)s.T);
+    CHECK_PTR(q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(csum);
+    CHECK_PTR(gsum);
+    CHECK_PTR(O);
+    CHECK_PTR(lse);
+    CHECK_PTR(cidx);
+    CHECK_PTR(gidx);
+    if (s.G > hga::decode_max_heads())
+        return fail(HGA_ERR_UNSUPPORTED, "decode takes at most %d q-heads per kv-head (got %d)",
+                    hga::decode_max_heads(), s.G);
+    if (hga::decode_smem(s) > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "decode of %lld chunks / k_g=%d exceeds the kernel's shared memory",
+                    (long long)s.nC, s.wg);
+    cudaError_t e = hga::launch_decode(s, pos, q, K, V, csum, gsum, O, lse, cidx, gidx,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_decode");
+}
+
 int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* V,
                  const int32_t* gidx, float* O, float* lse, hga_stream_t stream)
 {

@@ -1,6 +1,7 @@
 // hga_internal.cuh -- device helpers and kernel launchers shared by the
 // translation units of libhga.so.  Not part of the public ABI.
 #pragma once
+#include <atomic>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -104,6 +105,25 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Raise a kernel's dynamic shared memory limit to at least `bytes`, calling
+// the driver only when the limit set so far (per kernel and device) is
+// lower: a repeated launch path makes no driver call besides the launch.
+template <typename Kern>
+cudaError_t allow_smem(Kern kernel, int bytes)
+{
+    static std::atomic<int> limit[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && limit[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev < 64) {
+        int cur = limit[dev].load(std::memory_order_relaxed);
+        while (cur < bytes && !limit[dev].compare_exchange_weak(cur, bytes)) {}
+    }
+    return e;
+}
+
 // ---- launchers (each returns cudaError_t of its launch) ------------------------
 // K holds T_src rows per (batch, kv-head), the first of them at position row0.
 cudaError_t launch_summaries(const Shape& s, const void* K, int64_t T_src, int64_t row0, int64_t c_begin,
@@ -115,6 +135,12 @@ cudaError_t launch_route_groups(const Shape& s, const float* qbar, const float* 
 cudaError_t launch_route_fused(const Shape& s, const void* Q, const float* csum, const float* gsum,
                                float* qbar, int32_t* cidx, int32_t* gidx, cudaStream_t st);
 size_t route_fused_smem(const Shape& s);
+// One decode step of the token at position pos (decode.cu).
+cudaError_t launch_decode(const Shape& s, int64_t pos, const void* q, const void* K, const void* V,
+                          const float* csum, const float* gsum, float* O, float* lse, int32_t* cidx,
+                          int32_t* gidx, cudaStream_t st);
+size_t decode_smem(const Shape& s);
+int decode_max_heads();
 cudaError_t launch_attn_fwd_simt(const Shape& s, const void* Q, const void* K, const void* V,
                                  const int32_t* gidx, float* O, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Shape& s, const void* Q, const void* K, const void* V,

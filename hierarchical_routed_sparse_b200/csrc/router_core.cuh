@@ -1,0 +1,247 @@
+// router_core.cuh -- device pieces of the routing (a3, a4) shared by the
+// segment router (router.cu) and the decode step (decode.cu): candidate
+// scoring, warp-level top-k and the chunk / group selection of one block.
+//
+// Article "BMW's 16 GB GPU just did what needs an A100" (seventnews.com),
+// section "What HGA does differently": the block query scores the chunk
+// summaries and keeps the top-k chunks, then the top-k groups of those
+// chunks.  Selection uses 64-bit keys (order-preserving score bits, then the
+// inverted index), so "higher score, then lower index" is one unsigned
+// comparison and every candidate key is distinct.  Not part of the ABI.
+#pragma once
+
+#include "hga_internal.cuh"
+
+namespace hga {
+namespace rt {
+
+constexpr int kRouterThreads = 256;
+constexpr int kRouterWarps = kRouterThreads / 32;
+constexpr int kBatch = 16;          // candidates a warp scores at once
+
+// Scores of candidates 0..n-1 against the block query qs (shared memory):
+// score(c) = qs . row(c), written as a selection key into keys[c].  Warp w
+// takes batches of 16 candidates w, w+8, ...; for each batch every lane
+// issues its 16 coalesced loads (lane l holds elements [l*P, (l+1)*P) of each
+// row) before any arithmetic, so a batch costs one memory round trip, and
+// the 16 partial sums are reduced across the warp with 16 shuffles (each
+// step halves the values a lane carries).
+template <int D, typename RowFn>
+__device__ __forceinline__ void score_candidates(const float* __restrict__ qs, int n, RowFn row_of,
+                                                 unsigned long long* keys, int warp, int lane)
+{
+    constexpr int P = D / 32;
+    float q[P];
+#pragma unroll
+    for (int e = 0; e < P; ++e) q[e] = qs[lane * P + e];
+    for (int base = warp * kBatch; base < n; base += kRouterWarps * kBatch) {
+        float v[kBatch];
+        int32_t id[kBatch];
+        float x[kBatch][P];
+#pragma unroll
+        for (int c = 0; c < kBatch; ++c) {
+            const int cc = base + c < n ? base + c : base;
+            const float* row;
+            id[c] = row_of(cc, row);
+            if constexpr (P == 4) {
+                const float4 t = __ldg(reinterpret_cast<const float4*>(row) + lane);
+                x[c][0] = t.x; x[c][1] = t.y; x[c][2] = t.z; x[c][3] = t.w;
+            } else {
+                const float2 t = __ldg(reinterpret_cast<const float2*>(row) + lane);
+                x[c][0] = t.x; x[c][1] = t.y;
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < kBatch; ++c) {
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < P; ++e) a = fmaf(x[c][e], q[e], a);
+            v[c] = a;
+        }
+        // Transpose-reduce: after the step with offset o the lane keeps the
+        // half of its values selected by its lane bit o.
+#pragma unroll
+        for (int o = 16, m = kBatch / 2; o >= 2; o >>= 1, m >>= 1) {
+            const bool up = lane & o;
+#pragma unroll
+            for (int c = 0; c < m; ++c) {
+                const float send = up ? v[c] : v[c + m];
+                const float keep = up ? v[c + m] : v[c];
+                v[c] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+            }
+        }
+        v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], 1);
+        // Lane l now holds the full score of candidate ((l >> 1) & 15) in
+        // bit order 16, 8, 4, 2 -> 8, 4, 2, 1.
+        const int c = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+        int32_t my_id = id[0];
+#pragma unroll
+        for (int k = 1; k < kBatch; ++k) my_id = c == k ? id[k] : my_id;
+        if ((lane & 1) == 0 && base + c < n) keys[base + c] = pack_key(v[0], my_id);
+    }
+}
+
+// Write the selected candidates (key == 0 marks a selected slot) in
+// ascending candidate order, then -1 up to the row width.  One warp.
+__device__ __forceinline__ void compact_selected(const unsigned long long* keys, const int32_t* ids,
+                                                 int n, int32_t* out, int width, int lane)
+{
+    int pos = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        const bool sel = i < n && keys[i] == 0ull;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, sel);
+        if (sel) out[pos + __popc(m & ((1u << lane) - 1u))] = ids ? ids[i] : i;
+        pos += __popc(m);
+    }
+    for (int i = pos + lane; i < width; i += 32) out[i] = -1;
+}
+
+// Warp-level top-k over candidate keys held in registers: lane l holds the
+// keys of candidates l + 32 m (m < kRegCand; 0 = none).  A round takes the
+// warp maximum with two 32-bit reductions (score bits, then the inverted
+// index among equal scores); the winning lane marks its candidate (bit m of
+// sel) and recomputes its maximum from registers.  Then the selected
+// candidates are written in ascending candidate order, -1 up to `width`,
+// to out0 and (if not null) out1.
+constexpr int kRegCand = 8;
+
+__device__ __forceinline__ void warp_topk_regs(unsigned long long (&ck)[kRegCand], int k, int32_t* out0,
+                                               int32_t* out1, int width, int lane)
+{
+    auto lane_max = [&]() {
+        unsigned long long b = ck[0];
+#pragma unroll
+        for (int m = 1; m < kRegCand; ++m) b = ck[m] > b ? ck[m] : b;
+        return b;
+    };
+    unsigned long long best = lane_max();
+    uint32_t sel = 0;
+    for (int round = 0; round < k; ++round) {
+        const uint32_t hi = uint32_t(best >> 32), lo = uint32_t(best);
+        const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
+        const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+        if (best != 0ull && hi == mhi && lo == mlo) {       // keys are distinct: one lane wins
+#pragma unroll
+            for (int m = 0; m < kRegCand; ++m)
+                if (ck[m] == best) {
+                    ck[m] = 0ull;
+                    sel |= 1u << m;
+                }
+            best = lane_max();
+        }
+    }
+    const unsigned below = (1u << lane) - 1u;
+    int pos = 0;
+#pragma unroll
+    for (int m = 0; m < kRegCand; ++m) {
+        const bool mine = (sel >> m) & 1u;
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, mine);
+        if (mine) {
+            const int at = pos + __popc(bal & below);
+            out0[at] = lane + 32 * m;
+            if (out1) out1[at] = lane + 32 * m;
+        }
+        pos += __popc(bal);
+    }
+    for (int i = pos + lane; i < width; i += 32) {
+        out0[i] = -1;
+        if (out1) out1[i] = -1;
+    }
+}
+
+// a3: chunk routing of one block: scores of the eligible chunks c < c0, then
+// a warp-level top-k on warp 0 -- from registers (warp_topk_regs) when
+// c0 <= 256, else by rounds over shared memory: lane l keeps the largest key
+// among its candidates l, l+32, ...; a round takes the warp maximum as above
+// and the winning lane clears the winner's key (0 marks it selected) and
+// rescans its candidates.  Writes the row to cidx_row and (if not null) to
+// crow_smem.
+template <int D>
+__device__ __forceinline__ void route_chunks_block(const float* qs, const float* __restrict__ cs, int c0, int k_c,
+                                                   int wc, unsigned long long* keys, int32_t* cidx_row,
+                                                   int32_t* crow_smem, int tid)
+{
+    const int lane = tid & 31, warp = tid >> 5;
+    if (k_c <= 0 || k_c >= c0) {                       // keep every eligible chunk
+        for (int i = tid; i < wc; i += kRouterThreads) {
+            const int32_t v = i < c0 ? i : -1;
+            cidx_row[i] = v;
+            if (crow_smem) crow_smem[i] = v;
+        }
+        __syncthreads();
+        return;
+    }
+    score_candidates<D>(qs, c0, [&](int c, const float*& row) { row = cs + (int64_t)c * D; return c; }, keys,
+                        warp, lane);
+    __syncthreads();
+    if (warp == 0 && c0 <= 32 * kRegCand) {
+        unsigned long long ck[kRegCand];
+#pragma unroll
+        for (int m = 0; m < kRegCand; ++m) ck[m] = lane + 32 * m < c0 ? keys[lane + 32 * m] : 0ull;
+        warp_topk_regs(ck, k_c, cidx_row, crow_smem, wc, lane);
+    } else if (warp == 0) {
+        unsigned long long best = 0ull;
+        for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
+        for (int round = 0; round < k_c; ++round) {
+            const uint32_t hi = uint32_t(best >> 32), lo = uint32_t(best);
+            const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
+            const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+            if (best != 0ull && hi == mhi && lo == mlo) {   // keys are distinct: one lane wins
+                keys[key_index(best)] = 0ull;
+                best = 0ull;
+                for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
+            }
+        }
+        __syncwarp();
+        compact_selected(keys, nullptr, c0, cidx_row, wc, lane);
+        if (crow_smem) compact_selected(keys, nullptr, c0, crow_smem, wc, lane);
+    }
+    __syncthreads();
+}
+
+// a4: group routing of one block: the 8 groups of every chunk in crow (an
+// ascending prefix of valid chunks), scored and ranked; a candidate is kept
+// when fewer than k_g candidates beat it.
+template <int D>
+__device__ __forceinline__ void route_groups_block(const float* qs, const float* __restrict__ gs,
+                                                   const int32_t* crow, int wc, int k_g, int wg,
+                                                   unsigned long long* keys, int32_t* ids, uint8_t* flags,
+                                                   int* s_count, int32_t* gidx_row, int tid)
+{
+    const int lane = tid & 31, warp = tid >> 5;
+    if (warp == 0) {                                   // valid chunks form a prefix
+        int n = 0;
+        for (int base = 0; base < wc; base += 32) {
+            const int i = base + lane;
+            n += __popc(__ballot_sync(0xFFFFFFFFu, i < wc && crow[i] >= 0));
+        }
+        if (lane == 0) *s_count = n;
+    }
+    __syncthreads();
+    const int n = *s_count * kGroupsPerChunk;          // candidate groups
+    for (int i = tid; i < n; i += kRouterThreads)
+        ids[i] = crow[i / kGroupsPerChunk] * kGroupsPerChunk + i % kGroupsPerChunk;
+    __syncthreads();
+    if (k_g <= 0 || k_g >= n) {                        // keep every candidate
+        for (int i = tid; i < wg; i += kRouterThreads) gidx_row[i] = i < n ? ids[i] : -1;
+        return;
+    }
+    score_candidates<D>(qs, n, [&](int c, const float*& row) { row = gs + (int64_t)ids[c] * D; return ids[c]; },
+                        keys, warp, lane);
+    __syncthreads();
+    for (int i = tid; i < n; i += kRouterThreads) {
+        const unsigned long long ki = keys[i];
+        int rank = 0;
+        for (int j = 0; j < n; ++j) rank += keys[j] > ki;
+        flags[i] = rank < k_g;
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += kRouterThreads)
+        if (flags[i]) keys[i] = 0ull;
+    __syncthreads();
+    if (warp == 0) compact_selected(keys, ids, n, gidx_row, wg, lane);
+}
+
+}  // namespace rt
+}  // namespace hga

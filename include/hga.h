@@ -220,6 +220,29 @@ int hga_stage_routed(const hga_params* p, const void* K_hist, const void* V_hist
                      void* K_stage, void* V_stage, int32_t* gidx_stage,
                      hga_stream_t stream);
 
+/* f3. One decode step (article section "Retrieval: no degradation in the
+ * dense baseline": HGA can generate too).  The token at position pos is a
+ * query block of one: its block query is the mean of its G q-heads' queries
+ * (per kv-head); chunks c < pos / 64 are routed on csum (top k_c), their
+ * groups on gsum (top k_g), and each q-head attends the routed groups' exact
+ * tokens plus its own chunk's tokens 64 * (pos / 64) .. pos.  The shapes of
+ * hga_params describe the cache: T = T_hist + T_seg rows of capacity.
+ *   q          [B][Hq][d]          dtype, the new token's queries
+ *   K, V       [B][Hkv][T][d]      dtype, rows 0 .. pos valid (pos included)
+ *   csum, gsum as above; rows of chunks c < pos / 64 (groups of them) valid
+ *              -- append a chunk's summaries with hga_build_summaries (or
+ *              hga_build_summaries_rows) once its 64 tokens are in the cache
+ *   O          [B][Hq][d]          float32
+ *   lse        [B][Hq]             float32, natural log
+ *   cidx       [B][Hkv][wc]        int32 (widths of hga_route_widths)
+ *   gidx       [B][Hkv][wg]        int32
+ * Rows outside 0 .. pos are never read.  HGA_ERR_INVALID_ARG if pos is not
+ * in [0, T); HGA_ERR_UNSUPPORTED for more than 8 q-heads per kv-head or when
+ * the key list (8 wg + 64 scores per q-head) exceeds shared memory. */
+int hga_decode(const hga_params* p, int64_t pos, const void* q, const void* K,
+               const void* V, const float* csum, const float* gsum, float* O,
+               float* lse, int32_t* cidx, int32_t* gidx, hga_stream_t stream);
+
 /* Status word of the kernels' bounded waits: every wait of a tensor-core
  * kernel on a barrier gives up after one second, records the code of the wait
  * in this word and lets the kernel return (its outputs are then invalid).

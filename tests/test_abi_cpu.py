@@ -150,3 +150,23 @@ def test_stage_routed_rejects_bad_pointers_on_the_host(lib):
         a[i] = bad
         assert lib.hga_stage_routed(ctypes.byref(p.c()), *a, None) == hga.HGA_ERR_INVALID_ARG
     assert lib.hga_stage_routed(ctypes.byref(_p(T_seg=0).c()), *([None] * 8), None) == hga.HGA_OK
+
+
+def test_decode_rejects_bad_arguments_on_the_host(lib):
+    p = _p().c()
+    P = ctypes.c_void_p
+    ok = P(1 << 20)
+    T = p.T_hist + p.T_seg
+    for pos in (-1, T, T + 5):
+        assert lib.hga_decode(ctypes.byref(p), pos, *([ok] * 10), None) == hga.HGA_ERR_INVALID_ARG
+        assert "pos" in lib.hga_last_error().decode()
+    a = [ok] * 10
+    a[0] = None
+    assert lib.hga_decode(ctypes.byref(p), 3, *a, None) == hga.HGA_ERR_INVALID_ARG
+    assert "q is NULL" in lib.hga_last_error().decode()
+    a[0], a[7] = ok, P((1 << 20) + 8)
+    assert lib.hga_decode(ctypes.byref(p), 3, *a, None) == hga.HGA_ERR_INVALID_ARG
+    assert "cidx is not 16-byte aligned" in lib.hga_last_error().decode()
+    # More than 8 q-heads per kv-head: refused before any launch.
+    p9 = hga.Params(B=1, Hq=9, Hkv=1, d=128, T_hist=64, T_seg=64, k_c=2, k_g=4, dtype=hga.HGA_BF16).c()
+    assert lib.hga_decode(ctypes.byref(p9), 3, *([ok] * 10), None) == hga.HGA_ERR_UNSUPPORTED
