@@ -11,229 +11,386 @@
 // A chunk's summaries exist once the chunk is complete (the caller appends
 // them with hga_build_summaries as decoding fills it).
 //
-// One CTA per (batch, kv-head), 256 threads: routing with the segment
-// router's pieces, then the G heads' scores (keys spread over the 8 warps,
-// four rows in flight per warp), a softmax per head and O = P V with a
-// cross-warp reduction in shared memory.  Float32 arithmetic throughout.
+// One thread-block cluster of kS = 8 CTAs per (batch, kv-head), 256 threads
+// each.  A decode step is a chain of dependent memory round trips (query ->
+// chunk scores -> group scores -> K / V rows), so the cluster splits every
+// link of the chain:
+//   * chunk and group scoring: CTA r scores the r-th eighth of the
+//     candidates and writes the keys into every peer's shared memory
+//     (distributed shared memory); after a cluster barrier each CTA holds
+//     all keys and runs the same selection, so all hold the same routing;
+//   * attention: the keys come in 8-token units (the own chunk's tokens up
+//     to pos, then the routed groups, 8 contiguous rows each); CTA r takes
+//     units r, r + 8, ..., stages them into shared memory with bulk copies
+//     (tiles of 8 units, one mbarrier) and keeps a running softmax per head;
+//     the own chunk's unit is fetched at kernel start, before the routing;
+//   * combine: every CTA writes (max, sum, unnormalised O) of each head into
+//     CTA 0's shared memory; CTA 0 merges them (log-sum-exp) and stores O
+//     and lse.
+// Float32 arithmetic throughout.
 #include "hga_internal.cuh"
 #include "router_core.cuh"
+#include "sm100.cuh"
 
 namespace hga {
 namespace {
 
 using namespace rt;
+using namespace sm100;
 
-constexpr int kMaxG = 8;            // q-heads per kv-head handled by one CTA
-constexpr int kRowsInFlight = 4;    // K / V rows a warp loads before using them
+constexpr int kS = 8;                       // CTAs per (batch, kv-head): one cluster
+constexpr int kMaxG = 8;                    // q-heads per kv-head
+constexpr int kTileUnits = 8;               // 8-token units a CTA stages at once
+constexpr int kTileRows = kTileUnits * kGroup;
+constexpr int kSiteOwn = 0x301, kSiteTile = 0x302;   // bounded-wait sites
 
 struct DecodeLayout {
-    size_t keys, ids, flags, crow, grow, qh, sc, red, total;
+    size_t ckeys, gkeys, ids, flags, crow, grow, qh, kv, sc, hs, part, bar, total;
 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+__host__ __device__ inline size_t align128(size_t x) { return (x + 127) & ~size_t(127); }
 
-// Dynamic shared memory of the decode kernel.
-__host__ __device__ inline DecodeLayout decode_layout(int64_t nC, int wc, int wg, int G, int D)
+// Floats per CTA in the combine area: O [G][D], then max [G] and sum [G]
+// padded to a multiple of 4 (each CTA's block starts 16-byte aligned).
+__host__ __device__ inline int part_stride(int G, int D) { return G * D + ((2 * G + 3) & ~3); }
+
+// Dynamic shared memory of the decode kernel (el = bytes per K / V element).
+//   ckeys [nC] / gkeys [8 wc]   selection keys of chunks / groups (u64)
+//   ids [8 wc], flags [8 wc]    group candidates, their keep flags
+//   crow [wc], grow [wg]        the routing rows
+//   qh [G][D]                   the token's queries (float)
+//   kv                          K tile [64][D] then V tile [64][D] (input dtype)
+//   sc [G][64]                  scores, then weights, of the tile
+//   hs [3][G]                   running max, sum and rescale factor per head
+//   part [kS][part_stride]      per-CTA O [G][D], max [G], sum [G] read by CTA 0
+//   bar                         two mbarriers (own unit, tiles)
+__host__ __device__ inline DecodeLayout decode_layout(int64_t nC, int wc, int wg, int G, int D, int el)
 {
     DecodeLayout L;
-    const size_t nk = (size_t)(nC > 8 * (int64_t)wc ? nC : 8 * (int64_t)wc);
-    const size_t maxkeys = 8 * (size_t)wg + kChunk;
-    L.keys = 0;
-    L.ids = align16(L.keys + 8 * nk);
+    L.ckeys = 0;
+    L.gkeys = align16(L.ckeys + 8 * (size_t)(nC > 0 ? nC : 1));
+    L.ids = align16(L.gkeys + 8 * 8 * (size_t)wc);
     L.flags = align16(L.ids + 4 * 8 * (size_t)wc);
     L.crow = align16(L.flags + 8 * (size_t)wc);
     L.grow = align16(L.crow + 4 * (size_t)wc);
     L.qh = align16(L.grow + 4 * (size_t)wg);
-    L.sc = align16(L.qh + 4 * (size_t)G * D);
-    L.red = align16(L.sc + 4 * (size_t)G * maxkeys);
-    L.total = align16(L.red + 4 * (size_t)kRouterWarps * G * D);
+    L.kv = align128(L.qh + 4 * (size_t)G * D);
+    L.sc = align16(L.kv + 2 * (size_t)kTileRows * D * el);
+    L.hs = align16(L.sc + 4 * (size_t)G * kTileRows);
+    L.part = align16(L.hs + 4 * 3 * (size_t)G);
+    L.bar = align16(L.part + 4 * (size_t)kS * part_stride(G, D));
+    L.total = align16(L.bar + 16);
     return L;
 }
 
-// P consecutive elements widened to float32 (P = 2 or 4; 4- to 16-byte loads).
-template <typename TIn, int P> struct RowLoad;
-template <> struct RowLoad<__nv_bfloat16, 4> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* o) {
-        const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
-        o[0] = __uint_as_float(r.x << 16); o[1] = __uint_as_float(r.x & 0xFFFF0000u);
-        o[2] = __uint_as_float(r.y << 16); o[3] = __uint_as_float(r.y & 0xFFFF0000u);
-    }
-};
-template <> struct RowLoad<__nv_bfloat16, 2> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* o) {
-        const uint32_t r = __ldg(reinterpret_cast<const unsigned int*>(p));
-        o[0] = __uint_as_float(r << 16); o[1] = __uint_as_float(r & 0xFFFF0000u);
-    }
-};
-template <> struct RowLoad<float, 4> {
-    static __device__ __forceinline__ void load(const float* p, float* o) {
-        const float4 r = __ldg(reinterpret_cast<const float4*>(p));
-        o[0] = r.x; o[1] = r.y; o[2] = r.z; o[3] = r.w;
-    }
-};
-template <> struct RowLoad<float, 2> {
-    static __device__ __forceinline__ void load(const float* p, float* o) {
-        const float2 r = __ldg(reinterpret_cast<const float2*>(p));
-        o[0] = r.x; o[1] = r.y;
-    }
-};
+// P consecutive elements of a shared-memory row widened to float32.
+template <typename TIn, int P> __device__ __forceinline__ void smem_row(const TIn* p, float* o);
+template <> __device__ __forceinline__ void smem_row<__nv_bfloat16, 4>(const __nv_bfloat16* p, float* o)
+{
+    const uint2 r = *reinterpret_cast<const uint2*>(p);
+    o[0] = __uint_as_float(r.x << 16); o[1] = __uint_as_float(r.x & 0xFFFF0000u);
+    o[2] = __uint_as_float(r.y << 16); o[3] = __uint_as_float(r.y & 0xFFFF0000u);
+}
+template <> __device__ __forceinline__ void smem_row<__nv_bfloat16, 2>(const __nv_bfloat16* p, float* o)
+{
+    const uint32_t r = *reinterpret_cast<const uint32_t*>(p);
+    o[0] = __uint_as_float(r << 16); o[1] = __uint_as_float(r & 0xFFFF0000u);
+}
+template <> __device__ __forceinline__ void smem_row<float, 4>(const float* p, float* o)
+{
+    const float4 r = *reinterpret_cast<const float4*>(p);
+    o[0] = r.x; o[1] = r.y; o[2] = r.z; o[3] = r.w;
+}
+template <> __device__ __forceinline__ void smem_row<float, 2>(const float* p, float* o)
+{
+    const float2 r = *reinterpret_cast<const float2*>(p);
+    o[0] = r.x; o[1] = r.y;
+}
 
 template <typename TIn> __device__ __forceinline__ float to_f32(TIn x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
+// keys[b, e) of this CTA, written into the same slots of every peer.
+__device__ __forceinline__ void push_keys(unsigned long long* keys, int b, int e, uint32_t rank, int tid)
+{
+    for (int i = b + tid; i < e; i += kRouterThreads) {
+        const unsigned long long v = keys[i];
+        const uint32_t a = smem_u32(keys + i);
+#pragma unroll
+        for (uint32_t p = 0; p < kS; ++p)
+            if (p != rank) st_cluster_u64(peer_addr(a, p), v);
+    }
+}
+
 template <typename TIn, int D>
-__global__ void __launch_bounds__(kRouterThreads, 1)
+__global__ void __launch_bounds__(kRouterThreads, 2)
 decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ K, const TIn* __restrict__ V,
               const float* __restrict__ csum, const float* __restrict__ gsum, float* __restrict__ O,
               float* __restrict__ lse, int32_t* __restrict__ cidx, int32_t* __restrict__ gidx, int Hq, int Hkv,
               int G, int64_t T, int64_t pos, int k_c, int wc, int k_g, int wg, float scale)
 {
-    pdl_wait();
-    pdl_trigger();
     constexpr int P = D / 32;                        // elements of a row per lane
-    constexpr int R = kRowsInFlight;
-    extern __shared__ __align__(16) uint8_t sm[];
+    constexpr uint32_t kRowBytes = D * sizeof(TIn);
+    extern __shared__ __align__(128) uint8_t sm[];
     const int64_t nC = T / kChunk, nG = T / kGroup;
-    const DecodeLayout L = decode_layout(nC, wc, wg, G, D);
-    unsigned long long* keys = reinterpret_cast<unsigned long long*>(sm + L.keys);
+    const DecodeLayout L = decode_layout(nC, wc, wg, G, D, (int)sizeof(TIn));
+    unsigned long long* ckeys = reinterpret_cast<unsigned long long*>(sm + L.ckeys);
+    unsigned long long* gkeys = reinterpret_cast<unsigned long long*>(sm + L.gkeys);
     int32_t* ids = reinterpret_cast<int32_t*>(sm + L.ids);
     uint8_t* flags = sm + L.flags;
     int32_t* crow = reinterpret_cast<int32_t*>(sm + L.crow);
     int32_t* grow = reinterpret_cast<int32_t*>(sm + L.grow);
-    float* qh = reinterpret_cast<float*>(sm + L.qh);     // [G][D] the token's queries
-    float* sc = reinterpret_cast<float*>(sm + L.sc);     // [G][maxkeys] scores, then weights
-    float* red = reinterpret_cast<float*>(sm + L.red);   // [warps][G][D] partial outputs
+    float* qh = reinterpret_cast<float*>(sm + L.qh);
+    TIn* kt = reinterpret_cast<TIn*>(sm + L.kv);
+    TIn* vt = kt + kTileRows * D;
+    float* sc = reinterpret_cast<float*>(sm + L.sc);
+    float* hm = reinterpret_cast<float*>(sm + L.hs);   // running max per head
+    float* hl = hm + G;                                // running sum
+    float* ha = hl + G;                                // rescale of the current tile
+    float* part = reinterpret_cast<float*>(sm + L.part);
+    const uint32_t bar_own = smem_u32(sm + L.bar), bar_tile = bar_own + 8;
     __shared__ __align__(16) float qs[D];
-    __shared__ int n_valid, s_ng;
-    const int maxkeys = 8 * wg + kChunk;
+    __shared__ int s_cnt, s_ng;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t bg = blockIdx.x;
+    const uint32_t r = cluster_rank();
+    const int64_t bg = blockIdx.x / kS;
     const int64_t b = bg / Hkv, g = bg % Hkv;
+    const TIn* Kb = K + bg * T * D;
+    const TIn* Vb = V + bg * T * D;
 
-    // The token's queries of the G heads, and their mean (the block query).
+    if (tid == 0) {
+        mbar_init(bar_own, 1);
+        mbar_init(bar_tile, 1);
+        fence_mbar_init();
+    }
+    if (tid < G) {
+        hm[tid] = -INFINITY;
+        hl[tid] = 0.f;
+    }
+    pdl_wait();
+    pdl_trigger();
+
+    // The own chunk's tokens 64 c0 .. pos form units 0 .. n_ou-1 (n_ou <= 8):
+    // CTA r's is unit r, slot 0 of its first tile; fetch it now.  Also bring
+    // this CTA's slice of the chunk summaries into L2 ahead of the scoring.
+    const int c0 = int(pos / kChunk);
+    const int own_rows = int(pos - (int64_t)c0 * kChunk) + 1;
+    const int n_ou = (own_rows + kGroup - 1) / kGroup;
+    const bool has_own = (int)r < n_ou;
+    const int own_r = has_own ? min(kGroup, own_rows - kGroup * (int)r) : 0;
+    const bool score_c = k_c > 0 && k_c < c0;
+    const int cb = (int)r * c0 / kS, ce = ((int)r + 1) * c0 / kS;
+    const float* cs = csum + bg * nC * D;
+    if (tid == 0) {
+        if (has_own) {
+            const int64_t t0 = (int64_t)c0 * kChunk + kGroup * r;
+            mbar_expect_tx(bar_own, 2 * own_r * kRowBytes);
+            bulk_load(smem_u32(kt), Kb + t0 * D, own_r * kRowBytes, bar_own);
+            bulk_load(smem_u32(vt), Vb + t0 * D, own_r * kRowBytes, bar_own);
+        }
+        if (score_c && ce > cb) bulk_prefetch_l2(cs + (int64_t)cb * D, (uint32_t)(ce - cb) * D * 4u);
+    }
+    // The token's queries of the G heads (loads overlap the cluster barrier).
     for (int i = tid; i < G * D; i += kRouterThreads) qh[i] = to_f32<TIn>(q[(b * Hq + g * G) * D + i]);
-    __syncthreads();
+    cluster_sync();                                  // all CTAs run; barriers initialised; qh complete
+
+    // The block query: mean of the G heads' queries.
     for (int e = tid; e < D; e += kRouterThreads) {
         float a = 0.f;
         for (int h = 0; h < G; ++h) a += qh[h * D + e];
         qs[e] = a / (float)G;
     }
     __syncthreads();
-    // Chunk and group routing of the one-token block.
-    const int c0 = int(pos / kChunk);
-    int32_t* gout = gidx + bg * wg;
-    route_chunks_block<D>(qs, csum + bg * nC * D, c0, k_c, wc, keys, cidx + bg * wc, crow, tid);
-    route_groups_block<D>(qs, gsum + bg * nG * D, crow, wc, k_g, wg, keys, ids, flags, &n_valid, grow, tid);
-    __syncthreads();
-    for (int i = tid; i < wg; i += kRouterThreads) gout[i] = grow[i];
-    if (warp == 0) {                                 // routed groups: an ascending prefix
-        int n = 0;
-        for (int base = 0; base < wg; base += 32) {
-            const int i = base + lane;
-            n += __popc(__ballot_sync(0xFFFFFFFFu, i < wg && grow[i] >= 0));
+
+    // a3: chunk routing.  CTA r scores chunks [r c0 / 8, (r+1) c0 / 8).
+    if (score_c) {
+        score_candidates<D>(qs, ce - cb, [&](int c, const float*& row) { row = cs + (int64_t)(cb + c) * D; return cb + c; },
+                            ckeys + cb, warp, lane);
+        __syncthreads();
+        push_keys(ckeys, cb, ce, r, tid);
+    }
+    cluster_sync();
+    if (score_c) {
+        select_chunks(ckeys, c0, k_c, wc, crow, r == 0 ? cidx + bg * wc : nullptr, warp, lane);
+    } else {
+        for (int i = tid; i < wc; i += kRouterThreads) {
+            const int32_t v = i < c0 ? i : -1;
+            crow[i] = v;
+            if (r == 0) cidx[bg * wc + i] = v;
         }
+    }
+    __syncthreads();
+
+    // a4: group routing over the 8 groups of every routed chunk.  CTA r
+    // scores candidates [r n / 8, (r+1) n / 8).
+    if (warp == 0) {
+        const int n = prefix_count(crow, wc, lane);
+        if (lane == 0) s_cnt = n;
+    }
+    __syncthreads();
+    const int n_cand = s_cnt * kGroupsPerChunk;
+    for (int i = tid; i < n_cand; i += kRouterThreads)
+        ids[i] = crow[i / kGroupsPerChunk] * kGroupsPerChunk + i % kGroupsPerChunk;
+    __syncthreads();
+    const bool score_g = k_g > 0 && k_g < n_cand;
+    if (score_g) {
+        const int gb = (int)r * n_cand / kS, ge = ((int)r + 1) * n_cand / kS;
+        const float* gs = gsum + bg * nG * D;
+        score_candidates<D>(qs, ge - gb,
+                            [&](int c, const float*& row) { row = gs + (int64_t)ids[gb + c] * D; return ids[gb + c]; },
+                            gkeys + gb, warp, lane);
+        __syncthreads();
+        push_keys(gkeys, gb, ge, r, tid);
+    }
+    cluster_sync();
+    if (score_g) {
+        select_groups(gkeys, ids, n_cand, k_g, flags, grow, wg, tid);
+    } else {
+        for (int i = tid; i < wg; i += kRouterThreads) grow[i] = i < n_cand ? ids[i] : -1;
+    }
+    __syncthreads();
+    if (r == 0)
+        for (int i = tid; i < wg; i += kRouterThreads) gidx[bg * wg + i] = grow[i];
+    if (warp == 0) {
+        const int n = prefix_count(grow, wg, lane);
         if (lane == 0) s_ng = n;
     }
     __syncthreads();
-    const int n_g = s_ng;
-    const int n_keys = kGroup * n_g + int(pos - (int64_t)c0 * kChunk) + 1;
-    const TIn* Kb = K + bg * T * D + lane * P;
-    const TIn* Vb = V + bg * T * D + lane * P;
-    // Key k: the tokens of the routed groups in order, then the own chunk's
-    // tokens 64 c0 .. pos.
-    auto token = [&](int k) -> int64_t {
-        return k < kGroup * n_g ? (int64_t)grow[k / kGroup] * kGroup + k % kGroup
-                                : (int64_t)c0 * kChunk + (k - kGroup * n_g);
-    };
-    // Scores: warp w takes keys w + 8 j; lane l holds elements lP .. lP+P-1
-    // of the key row and of every head's query.
+
+    // Attention.  Units: 0 .. n_ou-1 the own chunk's, then the routed groups;
+    // CTA r takes units r + 8 j, tile t holding j = 8 t .. 8 t + 7 (slot j - 8 t).
+    const int n_u = n_ou + s_ng;
+    const int my_units = n_u > (int)r ? (n_u - (int)r + kS - 1) / kS : 0;
+    const int n_tiles = (my_units + kTileUnits - 1) / kTileUnits;
+    // Rows of a partial own unit past pos are zero in the V tile (their
+    // weight is 0, and 0 times stale shared memory could be NaN).
+    if (has_own && own_r < kGroup) {
+        for (int i = own_r * D + tid; i < kGroup * D; i += kRouterThreads) vt[i] = TIn(0.f);
+        fence_async_smem();                          // ordered before later bulk copies into the slot
+    }
     float qv[kMaxG][P];
 #pragma unroll
     for (int h = 0; h < kMaxG; ++h)
 #pragma unroll
         for (int e = 0; e < P; ++e) qv[h][e] = h < G ? qh[h * D + lane * P + e] : 0.f;
-    for (int k0 = warp; k0 < n_keys; k0 += R * kRouterWarps) {
-        float kv[R][P];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int k = k0 + r * kRouterWarps;
-            if (k < n_keys) RowLoad<TIn, P>::load(Kb + token(k) * D, kv[r]);
+    // P V: thread tid accumulates outputs 4 tid .. 4 tid + 3 of [G][D].
+    const int i4 = 4 * tid;
+    const bool pv_on = i4 < G * D;
+    const int ph = pv_on ? i4 / D : 0, pe = i4 % D;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    bool ok = true;
+    for (int t = 0; t < n_tiles; ++t) {
+        const int slots = min(kTileUnits, my_units - t * kTileUnits);
+        if (tid == 0) {
+            uint32_t bytes = 0;
+            for (int i = 0; i < slots; ++i)
+                if ((int)r + kS * (t * kTileUnits + i) >= n_ou) bytes += kGroup * kRowBytes;
+            mbar_expect_tx(bar_tile, 2 * bytes);
+            for (int i = 0; i < slots; ++i) {
+                const int u = (int)r + kS * (t * kTileUnits + i);
+                if (u < n_ou) continue;
+                const int64_t t0 = (int64_t)grow[u - n_ou] * kGroup;
+                bulk_load(smem_u32(kt + i * kGroup * D), Kb + t0 * D, kGroup * kRowBytes, bar_tile);
+                bulk_load(smem_u32(vt + i * kGroup * D), Vb + t0 * D, kGroup * kRowBytes, bar_tile);
+            }
         }
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int k = k0 + r * kRouterWarps;
-            if (k >= n_keys) break;
+        bool w = true;
+        if (t == 0 && has_own) w = mbar_wait(bar_own, 0, kSiteOwn);
+        w = mbar_wait(bar_tile, t & 1, kSiteTile) && w;
+        if (!__syncthreads_and(w)) {                 // a copy did not land in time
+            ok = false;
+            break;
+        }
+        // Scores of the tile's rows: warp w takes rows w, w + 8, ...
+        const int nrows = slots * kGroup;
+        for (int j = warp; j < nrows; j += kRouterWarps) {
+            const bool valid = !(t == 0 && j < kGroup && has_own) || j < own_r;
+            float kv[P];
+            smem_row<TIn, P>(kt + j * D + lane * P, kv);
 #pragma unroll
             for (int h = 0; h < kMaxG; ++h) {
                 if (h >= G) break;
                 float a = 0.f;
 #pragma unroll
-                for (int e = 0; e < P; ++e) a = fmaf(qv[h][e], kv[r][e], a);
+                for (int e = 0; e < P; ++e) a = fmaf(qv[h][e], kv[e], a);
                 a = warp_sum(a);
-                if (lane == 0) sc[h * maxkeys + k] = a * scale;
+                if (lane == 0) sc[h * kTileRows + j] = valid ? a * scale : -INFINITY;
             }
         }
-    }
-    __syncthreads();
-    // Softmax of each head (warp h, h + 8, ...): weights in place, lse.
-    for (int h = warp; h < G; h += kRouterWarps) {
-        float* s = sc + h * maxkeys;
-        float m = -INFINITY;
-        for (int k = lane; k < n_keys; k += 32) m = fmaxf(m, s[k]);
+        __syncthreads();
+        // Running softmax per head (warp h): weights of the tile, rescale.
+        for (int h = warp; h < G; h += kRouterWarps) {
+            float* s = sc + h * kTileRows;
+            float mt = -INFINITY;
+            for (int j = lane; j < nrows; j += 32) mt = fmaxf(mt, s[j]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        float l = 0.f;
-        for (int k = lane; k < n_keys; k += 32) {
-            const float w = expf(s[k] - m);
-            s[k] = w;
-            l += w;
-        }
-        l = warp_sum(l);
-        const float inv = 1.0f / l;
-        for (int k = lane; k < n_keys; k += 32) s[k] *= inv;
-        if (lane == 0) lse[b * Hq + g * G + h] = m + logf(l);
-    }
-    __syncthreads();
-    // O = P V: warp w accumulates keys w + 8 j for every head, then the 8
-    // warps' partial sums are added.
-    float acc[kMaxG][P];
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h)
-#pragma unroll
-        for (int e = 0; e < P; ++e) acc[h][e] = 0.f;
-    for (int k0 = warp; k0 < n_keys; k0 += R * kRouterWarps) {
-        float vv[R][P];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int k = k0 + r * kRouterWarps;
-            if (k < n_keys) RowLoad<TIn, P>::load(Vb + token(k) * D, vv[r]);
-        }
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int k = k0 + r * kRouterWarps;
-            if (k >= n_keys) break;
-#pragma unroll
-            for (int h = 0; h < kMaxG; ++h) {
-                if (h >= G) break;
-                const float w = sc[h * maxkeys + k];
-#pragma unroll
-                for (int e = 0; e < P; ++e) acc[h][e] = fmaf(w, vv[r][e], acc[h][e]);
+            for (int o = 16; o > 0; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, o));
+            const float mo = hm[h], mn = fmaxf(mo, mt);
+            float ls = 0.f;
+            for (int j = lane; j < nrows; j += 32) {
+                const float p = expf(s[j] - mn);
+                s[j] = p;
+                ls += p;
+            }
+            ls = warp_sum(ls);
+            if (lane == 0) {
+                const float a = expf(mo - mn);
+                ha[h] = a;
+                hl[h] = hl[h] * a + ls;
+                hm[h] = mn;
             }
         }
+        __syncthreads();
+        if (pv_on) {
+            const float a = ha[ph];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] *= a;
+            const float* wts = sc + ph * kTileRows;
+            for (int j = 0; j < nrows; ++j) {
+                float v[4];
+                smem_row<TIn, 4>(vt + j * D + pe, v);
+                const float p = wts[j];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc[k] = fmaf(p, v[k], acc[k]);
+            }
+        }
+        __syncthreads();                             // the tile is free for the next copies
     }
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) {
-        if (h >= G) break;
-#pragma unroll
-        for (int e = 0; e < P; ++e) red[(warp * G + h) * D + lane * P + e] = acc[h][e];
+
+    // Combine in CTA 0: O = sum_r O_r e^(m_r - M) / sum_r l_r e^(m_r - M).
+    const int stride = part_stride(G, D);
+    float* mine = part + (int)r * stride;
+    if (tid < G) {
+        st_cluster_f32(peer_addr(smem_u32(mine + G * D + tid), 0), ok ? hm[tid] : -INFINITY);
+        st_cluster_f32(peer_addr(smem_u32(mine + G * D + G + tid), 0), ok ? hl[tid] : 0.f);
     }
-    __syncthreads();
-    for (int i = tid; i < G * D; i += kRouterThreads) {
-        float a = 0.f;
+    if (pv_on) {
+        const float z = ok ? 1.f : 0.f;
+        st_cluster_v4(peer_addr(smem_u32(mine + i4), 0), acc[0] * z, acc[1] * z, acc[2] * z, acc[3] * z);
+    }
+    cluster_sync();
+    if (r == 0 && pv_on) {
+        float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kRouterWarps; ++w) a += red[w * G * D + i];
-        O[(b * Hq + g * G) * D + i] = a;
+        for (int c = 0; c < kS; ++c) M = fmaxf(M, part[c * stride + G * D + ph]);
+        float Ls = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < kS; ++c) {
+            const float* pc = part + c * stride;
+            const float f = expf(pc[G * D + ph] - M);
+            Ls = fmaf(pc[G * D + G + ph], f, Ls);
+            const float4 oc = *reinterpret_cast<const float4*>(pc + i4);
+            o[0] = fmaf(oc.x, f, o[0]);
+            o[1] = fmaf(oc.y, f, o[1]);
+            o[2] = fmaf(oc.z, f, o[2]);
+            o[3] = fmaf(oc.w, f, o[3]);
+        }
+        const float inv = 1.0f / Ls;
+        *reinterpret_cast<float4*>(O + (b * Hq + g * G) * D + i4) =
+            make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
+        if (pe == 0) lse[b * Hq + g * G + ph] = M + logf(Ls);
     }
 }
 
@@ -241,18 +398,33 @@ template <typename TIn, int D>
 cudaError_t launch(const Shape& s, int64_t pos, const void* q, const void* K, const void* V, const float* csum,
                    const float* gsum, float* O, float* lse, int32_t* cidx, int32_t* gidx, cudaStream_t st)
 {
-    const size_t smem = decode_layout(s.nC, s.wc, s.wg, s.G, D).total;
+    const size_t smem = decode_layout(s.nC, s.wc, s.wg, s.G, D, (int)sizeof(TIn)).total;
     auto k = decode_kernel<TIn, D>;
     cudaError_t e = allow_smem(k, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(k, dim3((unsigned)(s.B * s.Hkv)), dim3(kRouterThreads), smem, st,
-                      static_cast<const TIn*>(q), static_cast<const TIn*>(K), static_cast<const TIn*>(V), csum,
-                      gsum, O, lse, cidx, gidx, s.Hq, s.Hkv, s.G, s.T, pos, s.k_c, s.wc, s.k_g, s.wg, s.scale);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(s.B * s.Hkv * kS));
+    cfg.blockDim = dim3(kRouterThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, static_cast<const TIn*>(q), static_cast<const TIn*>(K),
+                              static_cast<const TIn*>(V), csum, gsum, O, lse, cidx, gidx, s.Hq, s.Hkv, s.G, s.T,
+                              pos, s.k_c, s.wc, s.k_g, s.wg, s.scale);
 }
 
 }  // namespace
 
-size_t decode_smem(const Shape& s) { return decode_layout(s.nC, s.wc, s.wg, s.G, s.d).total; }
+size_t decode_smem(const Shape& s)
+{
+    return decode_layout(s.nC, s.wc, s.wg, s.G, s.d, s.dtype == HGA_BF16 ? 2 : 4).total;
+}
 int decode_max_heads() { return kMaxG; }
 
 cudaError_t launch_decode(const Shape& s, int64_t pos, const void* q, const void* K, const void* V,
@@ -264,6 +436,18 @@ cudaError_t launch_decode(const Shape& s, int64_t pos, const void* q, const void
                           : launch<__nv_bfloat16, 64>(s, pos, q, K, V, csum, gsum, O, lse, cidx, gidx, st);
     return s.d == 128 ? launch<float, 128>(s, pos, q, K, V, csum, gsum, O, lse, cidx, gidx, st)
                       : launch<float, 64>(s, pos, q, K, V, csum, gsum, O, lse, cidx, gidx, st);
+}
+
+// Status word of the decode kernel's bounded waits (0 = none ran out).
+int decode_status(bool clear)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, sm100::g_status, sizeof v) != cudaSuccess) return -1;
+    if (clear && v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(sm100::g_status, &z, sizeof z);
+    }
+    return v;
 }
 
 }  // namespace hga

@@ -143,8 +143,10 @@ int hga_device_status(int* status, int clear)
     if (!status) return fail(HGA_ERR_INVALID_ARG, "status is NULL");
     const int vf = hga::attn_fwd_tc_status(clear != 0);
     const int vb = hga::attn_bwd_tc_status(clear != 0);
-    if (vf < 0 || vb < 0) return fail(HGA_ERR_CUDA, "hga_device_status: the status word could not be read");
-    *status = vf ? vf : vb;
+    const int vd = hga::decode_status(clear != 0);
+    if (vf < 0 || vb < 0 || vd < 0)
+        return fail(HGA_ERR_CUDA, "hga_device_status: the status word could not be read");
+    *status = vf ? vf : (vb ? vb : vd);
     return HGA_OK;
 }
 
@@ -313,7 +315,7 @@ int hga_decode(const hga_params* p, int64_t pos, const void* q, const void* K, c
     if (s.G > hga::decode_max_heads())
         return fail(HGA_ERR_UNSUPPORTED, "decode takes at most %d q-heads per kv-head (got %d)",
                     hga::decode_max_heads(), s.G);
-    if (hga::decode_smem(s) > kMaxSmem)
+    if (hga::decode_smem(s) + 1024 > kMaxSmem)      // + the kernel's static shared memory
         return fail(HGA_ERR_UNSUPPORTED, "decode of %lld chunks / k_g=%d exceeds the kernel's shared memory",
                     (long long)s.nC, s.wg);
     cudaError_t e = hga::launch_decode(s, pos, q, K, V, csum, gsum, O, lse, cidx, gidx,

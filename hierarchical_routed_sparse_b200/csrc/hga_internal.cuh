@@ -141,6 +141,7 @@ cudaError_t launch_decode(const Shape& s, int64_t pos, const void* q, const void
                           int32_t* gidx, cudaStream_t st);
 size_t decode_smem(const Shape& s);
 int decode_max_heads();
+int decode_status(bool clear);   // status word of decode.cu's bounded waits
 cudaError_t launch_attn_fwd_simt(const Shape& s, const void* Q, const void* K, const void* V,
                                  const int32_t* gidx, float* O, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Shape& s, const void* Q, const void* K, const void* V,

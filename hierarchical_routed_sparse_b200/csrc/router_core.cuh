@@ -150,13 +150,43 @@ __device__ __forceinline__ void warp_topk_regs(unsigned long long (&ck)[kRegCand
     }
 }
 
+// a3 selection: the top-k_c of the chunk keys keys[0..c0) (all scored, block
+// synchronised) on warp 0 -- from registers (warp_topk_regs) when c0 <= 256,
+// else by rounds over shared memory: lane l keeps the largest key among its
+// candidates l, l+32, ...; a round takes the warp maximum as above and the
+// winning lane clears the winner's key (0 marks it selected) and rescans its
+// candidates.  Writes the row to out0 and (if not null) out1.  Other warps
+// return at once.
+__device__ __forceinline__ void select_chunks(unsigned long long* keys, int c0, int k_c, int wc, int32_t* out0,
+                                              int32_t* out1, int warp, int lane)
+{
+    if (warp != 0) return;
+    if (c0 <= 32 * kRegCand) {
+        unsigned long long ck[kRegCand];
+#pragma unroll
+        for (int m = 0; m < kRegCand; ++m) ck[m] = lane + 32 * m < c0 ? keys[lane + 32 * m] : 0ull;
+        warp_topk_regs(ck, k_c, out0, out1, wc, lane);
+        return;
+    }
+    unsigned long long best = 0ull;
+    for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
+    for (int round = 0; round < k_c; ++round) {
+        const uint32_t hi = uint32_t(best >> 32), lo = uint32_t(best);
+        const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
+        const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+        if (best != 0ull && hi == mhi && lo == mlo) {   // keys are distinct: one lane wins
+            keys[key_index(best)] = 0ull;
+            best = 0ull;
+            for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
+        }
+    }
+    __syncwarp();
+    compact_selected(keys, nullptr, c0, out0, wc, lane);
+    if (out1) compact_selected(keys, nullptr, c0, out1, wc, lane);
+}
+
 // a3: chunk routing of one block: scores of the eligible chunks c < c0, then
-// a warp-level top-k on warp 0 -- from registers (warp_topk_regs) when
-// c0 <= 256, else by rounds over shared memory: lane l keeps the largest key
-// among its candidates l, l+32, ...; a round takes the warp maximum as above
-// and the winning lane clears the winner's key (0 marks it selected) and
-// rescans its candidates.  Writes the row to cidx_row and (if not null) to
-// crow_smem.
+// select_chunks.  Writes the row to cidx_row and (if not null) to crow_smem.
 template <int D>
 __device__ __forceinline__ void route_chunks_block(const float* qs, const float* __restrict__ cs, int c0, int k_c,
                                                    int wc, unsigned long long* keys, int32_t* cidx_row,
@@ -175,34 +205,43 @@ __device__ __forceinline__ void route_chunks_block(const float* qs, const float*
     score_candidates<D>(qs, c0, [&](int c, const float*& row) { row = cs + (int64_t)c * D; return c; }, keys,
                         warp, lane);
     __syncthreads();
-    if (warp == 0 && c0 <= 32 * kRegCand) {
-        unsigned long long ck[kRegCand];
-#pragma unroll
-        for (int m = 0; m < kRegCand; ++m) ck[m] = lane + 32 * m < c0 ? keys[lane + 32 * m] : 0ull;
-        warp_topk_regs(ck, k_c, cidx_row, crow_smem, wc, lane);
-    } else if (warp == 0) {
-        unsigned long long best = 0ull;
-        for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
-        for (int round = 0; round < k_c; ++round) {
-            const uint32_t hi = uint32_t(best >> 32), lo = uint32_t(best);
-            const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
-            const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
-            if (best != 0ull && hi == mhi && lo == mlo) {   // keys are distinct: one lane wins
-                keys[key_index(best)] = 0ull;
-                best = 0ull;
-                for (int c = lane; c < c0; c += 32) best = keys[c] > best ? keys[c] : best;
-            }
-        }
-        __syncwarp();
-        compact_selected(keys, nullptr, c0, cidx_row, wc, lane);
-        if (crow_smem) compact_selected(keys, nullptr, c0, crow_smem, wc, lane);
-    }
+    select_chunks(keys, c0, k_c, wc, cidx_row, crow_smem, warp, lane);
     __syncthreads();
 }
 
+// Number of valid entries of an index row (an ascending prefix); one warp.
+__device__ __forceinline__ int prefix_count(const int32_t* row, int w, int lane)
+{
+    int n = 0;
+    for (int base = 0; base < w; base += 32) {
+        const int i = base + lane;
+        n += __popc(__ballot_sync(0xFFFFFFFFu, i < w && row[i] >= 0));
+    }
+    return n;
+}
+
+// a4 selection: of the n scored group candidates (keys, ids; block
+// synchronised) a candidate is kept when fewer than k_g candidates beat it;
+// the kept ids are written in candidate order to gidx_row.
+__device__ __forceinline__ void select_groups(unsigned long long* keys, const int32_t* ids, int n, int k_g,
+                                              uint8_t* flags, int32_t* gidx_row, int wg, int tid)
+{
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < n; i += kRouterThreads) {
+        const unsigned long long ki = keys[i];
+        int rank = 0;
+        for (int j = 0; j < n; ++j) rank += keys[j] > ki;
+        flags[i] = rank < k_g;
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += kRouterThreads)
+        if (flags[i]) keys[i] = 0ull;
+    __syncthreads();
+    if (warp == 0) compact_selected(keys, ids, n, gidx_row, wg, lane);
+}
+
 // a4: group routing of one block: the 8 groups of every chunk in crow (an
-// ascending prefix of valid chunks), scored and ranked; a candidate is kept
-// when fewer than k_g candidates beat it.
+// ascending prefix of valid chunks), scored and ranked (select_groups).
 template <int D>
 __device__ __forceinline__ void route_groups_block(const float* qs, const float* __restrict__ gs,
                                                    const int32_t* crow, int wc, int k_g, int wg,
@@ -210,12 +249,8 @@ __device__ __forceinline__ void route_groups_block(const float* qs, const float*
                                                    int* s_count, int32_t* gidx_row, int tid)
 {
     const int lane = tid & 31, warp = tid >> 5;
-    if (warp == 0) {                                   // valid chunks form a prefix
-        int n = 0;
-        for (int base = 0; base < wc; base += 32) {
-            const int i = base + lane;
-            n += __popc(__ballot_sync(0xFFFFFFFFu, i < wc && crow[i] >= 0));
-        }
+    if (warp == 0) {
+        const int n = prefix_count(crow, wc, lane);
         if (lane == 0) *s_count = n;
     }
     __syncthreads();
@@ -230,17 +265,7 @@ __device__ __forceinline__ void route_groups_block(const float* qs, const float*
     score_candidates<D>(qs, n, [&](int c, const float*& row) { row = gs + (int64_t)ids[c] * D; return ids[c]; },
                         keys, warp, lane);
     __syncthreads();
-    for (int i = tid; i < n; i += kRouterThreads) {
-        const unsigned long long ki = keys[i];
-        int rank = 0;
-        for (int j = 0; j < n; ++j) rank += keys[j] > ki;
-        flags[i] = rank < k_g;
-    }
-    __syncthreads();
-    for (int i = tid; i < n; i += kRouterThreads)
-        if (flags[i]) keys[i] = 0ull;
-    __syncthreads();
-    if (warp == 0) compact_selected(keys, ids, n, gidx_row, wg, lane);
+    select_groups(keys, ids, n, k_g, flags, gidx_row, wg, tid);
 }
 
 }  // namespace rt

@@ -238,13 +238,15 @@ int hga_stage_routed(const hga_params* p, const void* K_hist, const void* V_hist
  *   gidx       [B][Hkv][wg]        int32
  * Rows outside 0 .. pos are never read.  HGA_ERR_INVALID_ARG if pos is not
  * in [0, T); HGA_ERR_UNSUPPORTED for more than 8 q-heads per kv-head or when
- * the key list (8 wg + 64 scores per q-head) exceeds shared memory. */
+ * the routing state (8 bytes per chunk of T, about 70 bytes per unit of
+ * wc) exceeds shared memory.  Runs as one 8-CTA cluster per (batch,
+ * kv-head). */
 int hga_decode(const hga_params* p, int64_t pos, const void* q, const void* K,
                const void* V, const float* csum, const float* gsum, float* O,
                float* lse, int32_t* cidx, int32_t* gidx, hga_stream_t stream);
 
 /* Status word of the kernels' bounded waits: every wait of a tensor-core
- * kernel on a barrier gives up after one second, records the code of the wait
+ * kernel or of the decode kernel on a barrier gives up after one second, records the code of the wait
  * in this word and lets the kernel return (its outputs are then invalid).
  * *status = 0 when no wait ran out; `clear` != 0 resets the word.
  * Synchronises with the device. */
