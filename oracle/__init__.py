@@ -103,10 +103,14 @@ def _load():
         lib.oracle_attn_fwd.argtypes = [D, P, P, P, P, P, P]
         lib.oracle_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, P]
         lib.oracle_decode.argtypes = [D, ctypes.c_int64, P, P, P, P, P, P, P, P, P, P, P]
+        lib.oracle_causal_route.argtypes = [D, P, P, P, P, P, P, P]
+        lib.oracle_causal_attn_fwd.argtypes = [D, P, P, P, P, P, P]
+        lib.oracle_causal_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         for f in ("oracle_build_summaries", "oracle_block_query", "oracle_route_chunks",
                   "oracle_route_groups", "oracle_attn_fwd", "oracle_attn_bwd", "oracle_decode",
+                  "oracle_causal_route", "oracle_causal_attn_fwd", "oracle_causal_attn_bwd",
                   "oracle_set_num_threads"):
             getattr(lib, f).restype = None
         _lib = lib
@@ -217,6 +221,42 @@ def decode(dims: Dims, pos: int, q, K, V, csum, gsum):
     _load().oracle_decode(ctypes.byref(dims._c()), int(pos), _ptr(q), _ptr(K), _ptr(V), _ptr(csum),
                           _ptr(gsum), _ptr(O), _ptr(lse), _ptr(cidx), _ptr(gidx), _ptr(cgap), _ptr(ggap))
     return dict(O=O, lse=lse, cidx=cidx, gidx=gidx, cgap=cgap, ggap=ggap)
+
+
+def causal_route(dims: Dims, Q, csum, gsum):
+    """Strictly causal routing: every query position routes on its own query
+    (mean over the G q-heads), a block of one.  Returns dict(cidx [B,Hkv,
+    T_seg,wc], gidx [B,Hkv,T_seg,wg], cgap, ggap [B,Hkv,T_seg])."""
+    Q, csum, gsum = _f64(Q), _f64(csum), _f64(gsum)
+    B, Hkv, Ts = dims.B, dims.Hkv, dims.T_seg
+    cidx = np.full((B, Hkv, Ts, dims.wc), -7, dtype=np.int32)
+    gidx = np.full((B, Hkv, Ts, dims.wg), -7, dtype=np.int32)
+    cgap = np.zeros((B, Hkv, Ts))
+    ggap = np.zeros((B, Hkv, Ts))
+    _load().oracle_causal_route(ctypes.byref(dims._c()), _ptr(Q), _ptr(csum), _ptr(gsum), _ptr(cidx),
+                                _ptr(gidx), _ptr(cgap), _ptr(ggap))
+    return dict(cidx=cidx, gidx=gidx, cgap=cgap, ggap=ggap)
+
+
+def causal_attn_fwd(dims: Dims, Q, K, V, gidx):
+    """Attention of the causal variant (gidx per position).  Returns (O, lse)."""
+    Q, K, V, gidx = _f64(Q), _f64(K), _f64(V), _i32(gidx)
+    O = np.zeros((dims.B, dims.Hq, dims.T_seg, dims.d))
+    lse = np.zeros((dims.B, dims.Hq, dims.T_seg))
+    _load().oracle_causal_attn_fwd(ctypes.byref(dims._c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(gidx),
+                                   _ptr(O), _ptr(lse))
+    return O, lse
+
+
+def causal_attn_bwd(dims: Dims, Q, K, V, dO, gidx):
+    """Backward of the causal variant (routing frozen).  Returns (dQ, dK_seg, dV_seg)."""
+    Q, K, V, dO, gidx = _f64(Q), _f64(K), _f64(V), _f64(dO), _i32(gidx)
+    dQ = np.zeros((dims.B, dims.Hq, dims.T_seg, dims.d))
+    dK = np.zeros((dims.B, dims.Hkv, dims.T_seg, dims.d))
+    dV = np.zeros((dims.B, dims.Hkv, dims.T_seg, dims.d))
+    _load().oracle_causal_attn_bwd(ctypes.byref(dims._c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(dO),
+                                   _ptr(gidx), _ptr(dQ), _ptr(dK), _ptr(dV))
+    return dQ, dK, dV
 
 
 def route(dims: Dims, Q, K):

@@ -249,11 +249,14 @@ static int64_t key_set(const oracle_dims* p, const int32_t* grow, int64_t i,
 /* ---------------------------------------------------------------- a5 ---- */
 /* Exact softmax attention over the routed key set (reading R9).  The softmax
  * is evaluated directly: scores, their maximum, exponentials, their sum. */
-void oracle_attn_fwd(const oracle_dims* p, const double* Q, const double* K,
-                     const double* V, const int32_t* gidx, double* O, double* lse)
+static void attn_fwd_rows(const oracle_dims* p, const double* Q, const double* K,
+                          const double* V, const int32_t* gidx, int per_row, double* O,
+                          double* lse)
 {
     const int G = p->Hq / p->Hkv, d = p->d;
-    const int64_t T = total_len(p), nQB = p->T_seg / p->chunk;
+    const int64_t T = total_len(p);
+    /* routing rows per (b, kv-head): one per block, or one per position */
+    const int64_t nR = per_row ? p->T_seg : p->T_seg / p->chunk;
     const int64_t maxkeys = (int64_t)p->wg * p->group + p->chunk;
     const int64_t rows = (int64_t)p->B * p->Hq * p->T_seg;
 #pragma omp parallel
@@ -264,8 +267,8 @@ void oracle_attn_fwd(const oracle_dims* p, const double* Q, const double* K,
         for (int64_t r = 0; r < rows; ++r) {
             const int64_t i = r % p->T_seg, bh = r / p->T_seg;
             const int b = (int)(bh / p->Hq), h = (int)(bh % p->Hq), g = h / G;
-            const int64_t qb = i / p->chunk;
-            const int32_t* grow = gidx + (((int64_t)b * p->Hkv + g) * nQB + qb) * p->wg;
+            const int64_t qr = per_row ? i : i / p->chunk;
+            const int32_t* grow = gidx + (((int64_t)b * p->Hkv + g) * nR + qr) * p->wg;
             const double* q = Q + r * d;
             const double* Kh = K + ((int64_t)b * p->Hkv + g) * T * d;
             const double* Vh = V + ((int64_t)b * p->Hkv + g) * T * d;
@@ -290,17 +293,24 @@ void oracle_attn_fwd(const oracle_dims* p, const double* Q, const double* K,
     }
 }
 
+void oracle_attn_fwd(const oracle_dims* p, const double* Q, const double* K,
+                     const double* V, const int32_t* gidx, double* O, double* lse)
+{
+    attn_fwd_rows(p, Q, K, V, gidx, 0, O, lse);
+}
+
 /* ---------------------------------------------------------------- a6 ---- */
 /* Backward of a5 with the routing frozen (R10).  P is recomputed from the
  * inputs (not from a stored O or LSE) and the softmax Jacobian is applied
  * in its textbook form dS_j = P_j (dP_j - sum_k P_k dP_k).  Gradients of
  * keys before T_hist (detached history) are dropped. */
-void oracle_attn_bwd(const oracle_dims* p, const double* Q, const double* K,
-                     const double* V, const double* dO, const int32_t* gidx,
-                     double* dQ, double* dK_seg, double* dV_seg)
+static void attn_bwd_rows(const oracle_dims* p, const double* Q, const double* K,
+                          const double* V, const double* dO, const int32_t* gidx,
+                          int per_row, double* dQ, double* dK_seg, double* dV_seg)
 {
     const int G = p->Hq / p->Hkv, d = p->d;
-    const int64_t T = total_len(p), nQB = p->T_seg / p->chunk;
+    const int64_t T = total_len(p);
+    const int64_t nR = per_row ? p->T_seg : p->T_seg / p->chunk;
     const int64_t maxkeys = (int64_t)p->wg * p->group + p->chunk;
     const int64_t units = (int64_t)p->B * p->Hkv;
     memset(dK_seg, 0, sizeof(double) * (size_t)(units * p->T_seg * d));
@@ -320,7 +330,7 @@ void oracle_attn_bwd(const oracle_dims* p, const double* Q, const double* K,
             const int h = g * G + hh;
             for (int64_t i = 0; i < p->T_seg; ++i) {
                 const int64_t r = ((int64_t)b * p->Hq + h) * p->T_seg + i;
-                const int32_t* grow = gidx + (u * nQB + i / p->chunk) * p->wg;
+                const int32_t* grow = gidx + (u * nR + (per_row ? i : i / p->chunk)) * p->wg;
                 const double* q = Q + r * d;
                 const double* dout = dO + r * d;
                 const int64_t n = key_set(p, grow, i, keys);
@@ -359,6 +369,43 @@ void oracle_attn_bwd(const oracle_dims* p, const double* Q, const double* K,
     }
 }
 
+void oracle_attn_bwd(const oracle_dims* p, const double* Q, const double* K,
+                     const double* V, const double* dO, const int32_t* gidx,
+                     double* dQ, double* dK_seg, double* dV_seg)
+{
+    attn_bwd_rows(p, Q, K, V, dO, gidx, 0, dQ, dK_seg, dV_seg);
+}
+
+/* Routing of one query block of a single position whose own chunk is c0:
+ * qbar (d values) against the chunk summaries csu [nC][d] and the group
+ * summaries gsu [nG][d] of one (b, kv-head).  Chunks c < c0 (R4), top-k_c
+ * (R6, R7) into crow [wc]; groups of the chosen chunks, top-k_g (R5) into
+ * grow [wg]; gaps (R8) into *cgap, *ggap.  list: scratch of at least
+ * max(c0, 1) + wc * (chunk / group) + 1 candidates. */
+static void route_single(const oracle_dims* p, const double* qbar, const double* csu,
+                         const double* gsu, int64_t c0, cand* list, int32_t* crow,
+                         int32_t* grow, double* cgap, double* ggap)
+{
+    const int d = p->d, gpc = p->chunk / p->group;
+    for (int64_t c = 0; c < c0; ++c) {
+        list[c].s = dot(qbar, csu + c * d, d);
+        list[c].idx = c;
+    }
+    *cgap = select_top(list, c0, p->k_c, crow, p->wc);
+    int64_t n = 0;
+    for (int i = 0; i < p->wc; ++i) {
+        const int32_t c = crow[i];
+        if (c < 0) continue;
+        for (int r = 0; r < gpc; ++r) {
+            const int64_t j = (int64_t)c * gpc + r;
+            list[n].s = dot(qbar, gsu + j * d, d);
+            list[n].idx = j;
+            ++n;
+        }
+    }
+    *ggap = select_top(list, n, p->k_g, grow, p->wg);
+}
+
 /* ------------------------------------------------------------ decode ---- */
 /* One generation step (article section "Retrieval: no degradation in the
  * dense baseline": HGA itself can also do generation): the new token at position pos
@@ -390,26 +437,10 @@ void oracle_decode(const oracle_dims* p, int64_t pos, const double* q, const dou
             for (int h = 0; h < G; ++h) a += q[((b * p->Hq) + g * G + h) * d + e];
             qbar[e] = a / (double)G;
         }
-        /* chunk routing */
+        /* chunk and group routing */
         cand* list = (cand*)malloc(sizeof(cand) * (size_t)((c0 > 0 ? c0 : 1) + p->wc * gpc + 1));
-        for (int64_t c = 0; c < c0; ++c) {
-            list[c].s = dot(qbar, csum + (u * nC + c) * d, d);
-            list[c].idx = c;
-        }
-        cgap[u] = select_top(list, c0, p->k_c, cidx + u * p->wc, p->wc);
-        /* group routing */
-        int64_t n = 0;
-        for (int i = 0; i < p->wc; ++i) {
-            const int32_t c = cidx[u * p->wc + i];
-            if (c < 0) continue;
-            for (int r = 0; r < gpc; ++r) {
-                const int64_t j = (int64_t)c * gpc + r;
-                list[n].s = dot(qbar, gsum + (u * nG + j) * d, d);
-                list[n].idx = j;
-                ++n;
-            }
-        }
-        ggap[u] = select_top(list, n, p->k_g, gidx + u * p->wg, p->wg);
+        route_single(p, qbar, csum + u * nC * d, gsum + u * nG * d, c0, list, cidx + u * p->wc,
+                     gidx + u * p->wg, &cgap[u], &ggap[u]);
         free(list);
         /* attention of each q-head of the kv-head */
         const int32_t* grow = gidx + u * p->wg;
@@ -445,6 +476,63 @@ void oracle_decode(const oracle_dims* p, int64_t pos, const double* q, const dou
         free(s);
         free(qbar);
     }
+}
+
+/* ------------------------------------------------------------ causal ---- */
+/* Strictly causal variant.  Article section "The one real caveat: causal
+ * leakage": a block's routing depends on the scores of several query
+ * positions, so through the routing an earlier token sees the queries of
+ * later tokens of its block; the authors mention a strictly causal variant
+ * in the works without describing it.  Reading R11: every query position
+ * routes on its own query, a query block of one exactly as in the decode
+ * step -- qbar_i = mean of Q[., i] over the G q-heads of the kv-head, chunks
+ * c < (T_hist + i) / chunk eligible (R4), groups of the chosen chunks (R5),
+ * attention over the routed groups' tokens and the own chunk up to i (R9).
+ * Then the output at position i depends on positions <= i only.
+ * Routing rows per position: cidx [B][Hkv][T_seg][wc], gidx [B][Hkv][T_seg][wg],
+ * cgap, ggap [B][Hkv][T_seg]. */
+void oracle_causal_route(const oracle_dims* p, const double* Q, const double* csum,
+                         const double* gsum, int32_t* cidx, int32_t* gidx, double* cgap,
+                         double* ggap)
+{
+    const int G = p->Hq / p->Hkv, d = p->d, gpc = p->chunk / p->group;
+    const int64_t T = total_len(p), nC = T / p->chunk, nG = T / p->group;
+    const int64_t rows = (int64_t)p->B * p->Hkv * p->T_seg;
+#pragma omp parallel
+    {
+        double* qbar = (double*)malloc(sizeof(double) * (size_t)d);
+        cand* list = (cand*)malloc(sizeof(cand) * (size_t)(nC + 1 + p->wc * gpc));
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < rows; ++r) {
+            const int64_t u = r / p->T_seg, i = r % p->T_seg;
+            const int64_t b = u / p->Hkv, g = u % p->Hkv;
+            for (int e = 0; e < d; ++e) {
+                double a = 0.0;
+                for (int h = 0; h < G; ++h) a += Q[((b * p->Hq + g * G + h) * p->T_seg + i) * d + e];
+                qbar[e] = a / (double)G;
+            }
+            const int64_t c0 = (p->T_hist + i) / p->chunk;
+            route_single(p, qbar, csum + u * nC * d, gsum + u * nG * d, c0, list, cidx + r * p->wc,
+                         gidx + r * p->wg, &cgap[r], &ggap[r]);
+        }
+        free(qbar);
+        free(list);
+    }
+}
+
+/* Attention forward / backward of the causal variant: as a5 / a6 with the
+ * routing row of position i (gidx [B][Hkv][T_seg][wg]). */
+void oracle_causal_attn_fwd(const oracle_dims* p, const double* Q, const double* K,
+                            const double* V, const int32_t* gidx, double* O, double* lse)
+{
+    attn_fwd_rows(p, Q, K, V, gidx, 1, O, lse);
+}
+
+void oracle_causal_attn_bwd(const oracle_dims* p, const double* Q, const double* K,
+                            const double* V, const double* dO, const int32_t* gidx,
+                            double* dQ, double* dK_seg, double* dV_seg)
+{
+    attn_bwd_rows(p, Q, K, V, dO, gidx, 1, dQ, dK_seg, dV_seg);
 }
 
 /* Number of worker threads the oracle runs with. */
