@@ -646,6 +646,147 @@ def run_layer(args, w) -> None:
     print(json.dumps(line), flush=True)
 
 
+def causal_algorithmic(w) -> dict:
+    """Algorithmic bytes of the causal variant's attention kernels: every
+    input row read once (Q, dO, O, lse and the whole K / V context of each
+    (batch, kv-head)), every output written once, the per-position routing
+    rows read once."""
+    el = 2 if w.dtype == "bf16" else 4
+    B, Hq, Hkv, d, Ts, T = w.B, w.Hq, w.Hkv, w.d, w.T_seg, w.T
+    wc = w.k_c if w.k_c > 0 else T // 64
+    wg = w.k_g if w.k_g > 0 else 8 * wc
+    q = B * Hq * Ts * d * el
+    kv = 2 * B * Hkv * T * d * el
+    o = B * Hq * Ts * d * 4
+    l_ = B * Hq * Ts * 4
+    gi = B * Hkv * Ts * wg * 4
+    seg = 2 * B * Hkv * Ts * d * 4
+    return dict(attn_fwd_causal=q + kv + o + l_ + gi,
+                attn_bwd_causal=q + q + o + l_ + kv + gi + o + seg,
+                route_causal=q + B * Hkv * (T // 64 + T // 8) * d * 4 + B * Hkv * Ts * (wc + wg) * 4)
+
+
+def run_causal(args, w) -> None:
+    """The segment training step of the strictly causal variant (every query
+    position routes on its own query): segment summaries, per-position
+    routing, the causal attention forward and backward.  CUDA graph of the
+    step, events around its replay, L2 flushed between steps; stage_ms from a
+    second capture with events between the stages.  One JSON line,
+    config.mode = "causal"."""
+    import torch
+
+    import hierarchical_routed_sparse_b200 as hga
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    x = w.full()
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    p = hga.Params.from_workload(w)
+    cb = hga.CausalBuffers(p, device=dev)
+    Q, K, V = (torch.from_numpy(x[k]).to(dev, tdt) for k in ("Q", "K", "V"))
+    dO = torch.from_numpy(x["dO"]).to(dev, tdt)
+    cb.summaries(K, 0, w.T_hist)                     # history summaries persist
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    stages = ["summaries", "route_causal", "attn_fwd_causal", "attn_bwd_causal"]
+
+    def step_on(st, ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(st)
+        mark(0)
+        cb.summaries(K, stream=st)
+        mark(1)
+        cb.route(Q, st)
+        mark(2)
+        cb.forward(Q, K, V, stream=st)
+        mark(3)
+        cb.backward(Q, K, V, dO, stream=st)
+        mark(4)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step_on(stream)
+    torch.cuda.synchronize()
+    events = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)] for _ in range(args.steps)]
+    outer = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    graphs = []
+    with torch.cuda.stream(cap):
+        for i in range(args.steps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                step_on(cap, events[i])
+            graphs.append(g)
+        plain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(plain, stream=cap):
+            step_on(cap)
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        flush.zero_()
+        plain.replay()
+    torch.cuda.synchronize()
+    with ClockSampler(0, None) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            outer[i][0].record(stream)
+            plain.replay()
+            outer[i][1].record(stream)
+        for i in range(args.steps):
+            flush.zero_()
+            graphs[i].replay()
+        torch.cuda.synchronize()
+    total_ms = sum(a.elapsed_time(b) for a, b in outer)
+    stage_ms = {s_: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in events) for j, s_ in enumerate(stages)}
+    assert hga.device_status() == 0
+    ms = total_ms / args.steps
+    alg = causal_algorithmic(w)
+    pk = peaks()
+    dom = max(("attn_fwd_causal", "attn_bwd_causal"), key=lambda k: stage_ms[k])
+    achieved = alg[dom] / (stage_ms[dom] * 1e-3) / 1e9
+    # End to end through the public API: Q / K_seg / V_seg / dO from pinned
+    # host memory each step, the loss-side dQ read back.
+    el = 2 if w.dtype == "bf16" else 4
+    seg = slice(w.T_hist, w.T)
+    hosts = {k: v.cpu().pin_memory() for k, v in (("Q", Q), ("dO", dO))}
+    ks_h = K[:, :, seg].contiguous().cpu().pin_memory()
+    vs_h = V[:, :, seg].contiguous().cpu().pin_memory()
+    dq_h = torch.empty(cb.dQ.shape, dtype=torch.float32).pin_memory()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        ev2[i][0].record(stream)
+        Q.copy_(hosts["Q"], non_blocking=True)
+        dO.copy_(hosts["dO"], non_blocking=True)
+        K[:, :, seg].copy_(ks_h, non_blocking=True)
+        V[:, :, seg].copy_(vs_h, non_blocking=True)
+        step_on(stream)
+        dq_h.copy_(cb.dQ, non_blocking=True)
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in ev2)
+    h2d = (2 * w.B * w.Hq * w.T_seg + 2 * w.B * w.Hkv * w.T_seg) * w.d * el
+    d2h = w.B * w.Hq * w.T_seg * w.d * 4
+    line = dict(metric="HGA strictly causal variant, segment fwd+bwd tokens/s at 16K ctx",
+                value=w.B * w.T_seg / (ms * 1e-3), unit="tokens/s", n_gpus=1, steps=args.steps,
+                warmup=args.warmup, ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype=w.dtype, data="synthetic",
+                config=dict(config_of(w), mode="causal",
+                            routing="per query position (a block of one); per-row key sets"),
+                stage_ms=stage_ms,
+                roofline=dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
+                              frac=achieved / pk["hbm_gbs"], traffic=None, kernel=dom,
+                              algorithmic_bytes_per_launch=alg[dom],
+                              peak_source=pk["source"] + " (burst copy)"),
+                e2e=dict(value=w.B * w.T_seg / (e2e_ms * 1e-3), unit="tokens/s", h2d_bytes_per_step=h2d,
+                         d2h_bytes_per_step=d2h),
+                gpu_launches=(1 + 1 + 1 + 1) * args.steps, clocks=clk.summary())
+    print(json.dumps(line), flush=True)
+
+
 def decode_algorithmic(w, pos: int) -> dict:
     """Algorithmic bytes of one hga_decode call at position pos: the token's
     queries, the eligible chunk summaries, the group summaries of the routed
@@ -806,6 +947,8 @@ def main():
                     help="segment-wise training of one attention layer with HGA (f4 integration)")
     ap.add_argument("--kv-tier", choices=["hbm", "host"], default="hbm",
                     help="host: history K/V in pinned host memory, routed groups staged per step")
+    ap.add_argument("--causal", action="store_true",
+                    help="the strictly causal variant: routing per query position (f1)")
     ap.add_argument("--decode", action="store_true",
                     help="generation: one hga_decode step per token over the workload's context (f3)")
     ap.add_argument("--decode-batch", type=int, default=1, help="sequences decoded per step")
@@ -815,6 +958,8 @@ def main():
     w = W.BY_NAME[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.causal:
+        run_causal(args, w)
     elif args.decode:
         run_decode(args, w)
     elif args.layer:

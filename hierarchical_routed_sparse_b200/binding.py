@@ -25,7 +25,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhga.so")
 EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_build_summaries_rows",
            "hga_route_chunks",
            "hga_route_groups", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
-           "hga_stage_params", "hga_stage_routed", "hga_decode", "hga_device_status", "hga_last_error",
+           "hga_stage_params", "hga_stage_routed", "hga_decode", "hga_route_causal", "hga_attn_fwd_causal",
+           "hga_attn_bwd_causal", "hga_device_status", "hga_last_error",
            "hga_version")
 NOALLOC_MAX_ROWS = 1 << 20     # HGA_NOALLOC_MAX_ROWS
 
@@ -112,6 +113,9 @@ def load() -> ctypes.CDLL:
             "hga_stage_params": ([PP, PP], ctypes.c_int),
             "hga_stage_routed": ([PP, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_decode": ([PP, I64, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "hga_route_causal": ([PP, P, P, P, P, P, P], ctypes.c_int),
+            "hga_attn_fwd_causal": ([PP, P, P, P, P, P, P, P], ctypes.c_int),
+            "hga_attn_bwd_causal": ([PP, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_device_status": ([ctypes.POINTER(ctypes.c_int), ctypes.c_int], ctypes.c_int),
             "hga_last_error": ([], ctypes.c_char_p),
             "hga_version": ([], ctypes.c_char_p),
@@ -253,6 +257,68 @@ def decode(p: Params, pos: int, q, K, V, csum, gsum, O, lse, cidx, gidx, stream=
     valid, summaries of the chunks before pos // 64 built)."""
     _check(load().hga_decode(ctypes.byref(p.c()), int(pos), _ptr(q), _ptr(K), _ptr(V), _ptr(csum), _ptr(gsum),
                              _ptr(O), _ptr(lse), _ptr(cidx), _ptr(gidx), _stream(stream)))
+
+
+def route_causal(p: Params, Q, csum, gsum, cidx, gidx, stream=None) -> None:
+    """Strictly causal routing: one routing row per query position
+    (cidx [B][Hkv][T_seg][wc], gidx [B][Hkv][T_seg][wg])."""
+    _check(load().hga_route_causal(ctypes.byref(p.c()), _ptr(Q), _ptr(csum), _ptr(gsum), _ptr(cidx), _ptr(gidx),
+                                   _stream(stream)))
+
+
+def attn_fwd_causal(p: Params, Q, K, V, gidx, O, lse, stream=None) -> None:
+    _check(load().hga_attn_fwd_causal(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(gidx), _ptr(O),
+                                      _ptr(lse), _stream(stream)))
+
+
+def attn_bwd_causal(p: Params, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, stream=None) -> None:
+    _check(load().hga_attn_bwd_causal(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                                      _ptr(dO), _ptr(gidx), _ptr(dQ), _ptr(dK_seg), _ptr(dV_seg),
+                                      _stream(stream)))
+
+
+class CausalBuffers:
+    """Device buffers of the strictly causal variant for one problem shape:
+    routing rows per query position; ``step`` runs summaries, routing,
+    forward and (with dO) backward."""
+
+    def __init__(self, p: Params, device="cuda"):
+        self.p = p
+        wc, wg = route_widths(p)
+        B, Hq, Hkv, d, T, Ts = p.B, p.Hq, p.Hkv, p.d, p.T, p.T_seg
+        f32 = dict(device=device, dtype=torch.float32)
+        i32 = dict(device=device, dtype=torch.int32)
+        self.csum = torch.zeros(B, Hkv, T // 64, d, **f32)
+        self.gsum = torch.zeros(B, Hkv, T // 8, d, **f32)
+        self.cidx = torch.empty(B, Hkv, Ts, wc, **i32)
+        self.gidx = torch.empty(B, Hkv, Ts, wg, **i32)
+        self.O = torch.empty(B, Hq, Ts, d, **f32)
+        self.lse = torch.empty(B, Hq, Ts, **f32)
+        self.dQ = torch.empty(B, Hq, Ts, d, **f32)
+        self.dK = torch.empty(B, Hkv, Ts, d, **f32)
+        self.dV = torch.empty(B, Hkv, Ts, d, **f32)
+
+    def summaries(self, K, t_begin=None, t_end=None, stream=None):
+        t_begin = self.p.T_hist if t_begin is None else t_begin
+        t_end = self.p.T if t_end is None else t_end
+        build_summaries(self.p, K, t_begin, t_end, self.csum, self.gsum, stream)
+
+    def route(self, Q, stream=None):
+        route_causal(self.p, Q, self.csum, self.gsum, self.cidx, self.gidx, stream)
+
+    def forward(self, Q, K, V, gidx=None, stream=None):
+        attn_fwd_causal(self.p, Q, K, V, self.gidx if gidx is None else gidx, self.O, self.lse, stream)
+
+    def backward(self, Q, K, V, dO, gidx=None, stream=None):
+        attn_bwd_causal(self.p, Q, K, V, self.O, self.lse, dO, self.gidx if gidx is None else gidx, self.dQ,
+                        self.dK, self.dV, stream)
+
+    def step(self, Q, K, V, dO=None, stream=None):
+        self.summaries(K, stream=stream)
+        self.route(Q, stream)
+        self.forward(Q, K, V, stream=stream)
+        if dO is not None:
+            self.backward(Q, K, V, dO, stream=stream)
 
 
 class DecodeState:

@@ -1,0 +1,474 @@
+// causal.cu -- the strictly causal variant: routing per query position.
+//
+// Article "BMW's 16 GB GPU just did what needs an A100" (seventnews.com),
+// section "The one real caveat: causal leakage": with block routing the
+// routing of a block depends on the scores of several query positions, so an
+// earlier token sees later tokens through it; the authors mention a strictly
+// causal variant in the works.  This variant routes every query position on
+// its own query -- a query block of one, as the decode step does: the mean of
+// its G q-heads' queries scores the chunks before its own chunk (top k_c),
+// then the groups of those chunks (top k_g); each q-head attends the routed
+// groups' exact tokens and its own chunk up to itself.  The output at a
+// position then depends on earlier positions only.
+//
+// Every row has its own key set, so there is no key tile shared by the rows
+// of a block: the kernels work per (row, kv-head) on the FMA pipes.
+//   causal_route_kernel  one warp per row: block query of one, chunk scores
+//                        (the 8 rows of a CTA share the summaries through
+//                        L1), warp top-k, group scores, warp rank selection;
+//   causal_fwd_kernel    one warp per (row, kv-head), the G heads together:
+//                        keys in batches of 4 (K and V rows in flight),
+//                        running softmax, O and lse;
+//   causal_bwd_kernel    one warp per (row, kv-head): P from lse, dP, dS,
+//                        dQ in registers; dK / dV of segment keys added with
+//                        vector float atomics.
+// Float32 arithmetic; bf16 or float32 inputs.
+#include "hga_internal.cuh"
+#include "router_core.cuh"
+
+namespace hga {
+namespace {
+
+using namespace rt;
+
+constexpr int kWarps = 8;                   // rows (warps) per CTA
+constexpr int kThreads = 32 * kWarps;
+constexpr int kMaxG = 8;                    // q-heads per kv-head
+constexpr int kKeysInFlight = 4;            // K / V rows a warp loads before using them
+
+__host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~size_t(15); }
+
+// Per-warp shared memory of the routing kernel.
+struct RouteWarpLayout {
+    size_t keys, ids, flags, crow, qs, total;
+};
+__host__ __device__ inline RouteWarpLayout route_warp_layout(int64_t nC, int wc, int D)
+{
+    RouteWarpLayout L;
+    const size_t nk = (size_t)(nC > 8 * (int64_t)wc ? nC : 8 * (int64_t)wc);
+    L.keys = 0;
+    L.ids = al16(L.keys + 8 * nk);
+    L.flags = al16(L.ids + 4 * 8 * (size_t)wc);
+    L.crow = al16(L.flags + 8 * (size_t)wc);
+    L.qs = al16(L.crow + 4 * (size_t)wc);
+    L.total = al16(L.qs + 4 * (size_t)D);
+    return L;
+}
+
+// P consecutive elements widened to float32 (4- to 16-byte loads).
+template <typename TIn, int P> struct Row;
+template <> struct Row<__nv_bfloat16, 4> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* o) {
+        const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
+        o[0] = __uint_as_float(r.x << 16); o[1] = __uint_as_float(r.x & 0xFFFF0000u);
+        o[2] = __uint_as_float(r.y << 16); o[3] = __uint_as_float(r.y & 0xFFFF0000u);
+    }
+};
+template <> struct Row<__nv_bfloat16, 2> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* o) {
+        const uint32_t r = __ldg(reinterpret_cast<const unsigned int*>(p));
+        o[0] = __uint_as_float(r << 16); o[1] = __uint_as_float(r & 0xFFFF0000u);
+    }
+};
+template <> struct Row<float, 4> {
+    static __device__ __forceinline__ void load(const float* p, float* o) {
+        const float4 r = __ldg(reinterpret_cast<const float4*>(p));
+        o[0] = r.x; o[1] = r.y; o[2] = r.z; o[3] = r.w;
+    }
+};
+template <> struct Row<float, 2> {
+    static __device__ __forceinline__ void load(const float* p, float* o) {
+        const float2 r = __ldg(reinterpret_cast<const float2*>(p));
+        o[0] = r.x; o[1] = r.y;
+    }
+};
+
+// a4 selection inside one warp: of the n scored candidates (keys, ids) keep
+// those beaten by fewer than k_g others; kept ids in candidate order to out.
+__device__ __forceinline__ void warp_select_groups(unsigned long long* keys, const int32_t* ids, int n, int k_g,
+                                                   uint8_t* flags, int32_t* out, int wg, int lane)
+{
+    for (int i = lane; i < n; i += 32) {
+        const unsigned long long ki = keys[i];
+        int rank = 0;
+        for (int j = 0; j < n; ++j) rank += keys[j] > ki;
+        flags[i] = rank < k_g;
+    }
+    __syncwarp();
+    for (int i = lane; i < n; i += 32)
+        if (flags[i]) keys[i] = 0ull;
+    __syncwarp();
+    compact_selected(keys, ids, n, out, wg, lane);
+}
+
+// Routing of every query position: warp w of CTA x routes row
+// 8 x + w of the (batch, kv-head, row) grid.  cidx [B][Hkv][T_seg][wc],
+// gidx [B][Hkv][T_seg][wg].
+template <typename TIn, int D>
+__global__ void __launch_bounds__(kThreads)
+causal_route_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, const float* __restrict__ gsum,
+                    int32_t* __restrict__ cidx, int32_t* __restrict__ gidx, int Hq, int Hkv, int G,
+                    int64_t T_hist, int64_t T_seg, int k_c, int wc, int k_g, int wg)
+{
+    pdl_wait();
+    pdl_trigger();
+    constexpr int P = D / 32;
+    extern __shared__ __align__(16) uint8_t sm[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t T = T_hist + T_seg, nC = T / kChunk, nG = T / kGroup;
+    const RouteWarpLayout L = route_warp_layout(nC, wc, D);
+    uint8_t* ws = sm + (size_t)warp * L.total;
+    unsigned long long* keys = reinterpret_cast<unsigned long long*>(ws + L.keys);
+    int32_t* ids = reinterpret_cast<int32_t*>(ws + L.ids);
+    uint8_t* flags = ws + L.flags;
+    int32_t* crow = reinterpret_cast<int32_t*>(ws + L.crow);
+    float* qs = reinterpret_cast<float*>(ws + L.qs);
+    const int64_t row = (int64_t)blockIdx.x * kWarps + warp;      // (b, g, i) flattened
+    const int64_t bg = row / T_seg, i = row % T_seg;
+    const int64_t b = bg / Hkv, g = bg % Hkv;
+    // Block query of one: the mean of the row's G q-heads' queries.
+    float a[P];
+#pragma unroll
+    for (int e = 0; e < P; ++e) a[e] = 0.f;
+    for (int h = 0; h < G; ++h) {
+        float x[P];
+        Row<TIn, P>::load(Q + ((b * Hq + g * G + h) * T_seg + i) * D + lane * P, x);
+#pragma unroll
+        for (int e = 0; e < P; ++e) a[e] += x[e];
+    }
+#pragma unroll
+    for (int e = 0; e < P; ++e) qs[lane * P + e] = a[e] / (float)G;
+    __syncwarp();
+    // a3: chunks before the row's own chunk.
+    const int c0 = int((T_hist + i) / kChunk);
+    int32_t* crow_out = cidx + row * wc;
+    if (k_c <= 0 || k_c >= c0) {
+        for (int j = lane; j < wc; j += 32) {
+            const int32_t v = j < c0 ? j : -1;
+            crow[j] = v;
+            crow_out[j] = v;
+        }
+    } else {
+        const float* cs = csum + bg * nC * D;
+        score_candidates<D, 1>(qs, c0, [&](int c, const float*& r) { r = cs + (int64_t)c * D; return c; }, keys, 0,
+                               lane);
+        __syncwarp();
+        select_chunks(keys, c0, k_c, wc, crow, crow_out, 0, lane);
+    }
+    __syncwarp();
+    // a4: the groups of the chosen chunks.
+    const int n = prefix_count(crow, wc, lane) * kGroupsPerChunk;
+    for (int j = lane; j < n; j += 32) ids[j] = crow[j / kGroupsPerChunk] * kGroupsPerChunk + j % kGroupsPerChunk;
+    __syncwarp();
+    int32_t* grow_out = gidx + row * wg;
+    if (k_g <= 0 || k_g >= n) {
+        for (int j = lane; j < wg; j += 32) grow_out[j] = j < n ? ids[j] : -1;
+    } else {
+        const float* gs = gsum + bg * nG * D;
+        score_candidates<D, 1>(qs, n, [&](int c, const float*& r) { r = gs + (int64_t)ids[c] * D; return ids[c]; },
+                               keys, 0, lane);
+        __syncwarp();
+        warp_select_groups(keys, ids, n, k_g, flags, grow_out, wg, lane);
+    }
+}
+
+// Key k of a row: the routed groups' tokens in order, then the own chunk's
+// tokens own0 .. pos.
+__device__ __forceinline__ int64_t row_token(const int32_t* grow, int n_g, int64_t own0, int k)
+{
+    return k < kGroup * n_g ? (int64_t)__ldg(grow + k / kGroup) * kGroup + k % kGroup
+                            : own0 + (k - kGroup * n_g);
+}
+
+// Forward: warp w of CTA x takes row 8 x + w of the (batch, kv-head, row)
+// grid, for the G q-heads of the kv-head.  GM >= G bounds the heads held in
+// registers.
+template <typename TIn, int D, int GM>
+__global__ void __launch_bounds__(kThreads)
+causal_fwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TIn* __restrict__ V,
+                  const int32_t* __restrict__ gidx, float* __restrict__ O, float* __restrict__ lse, int Hq, int Hkv,
+                  int G, int64_t T_hist, int64_t T_seg, int wg, float scale)
+{
+    pdl_wait();
+    pdl_trigger();
+    constexpr int P = D / 32, R = kKeysInFlight;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
+    const int64_t bg = row / T_seg, i = row % T_seg;
+    const int64_t b = bg / Hkv, g = bg % Hkv;
+    const int64_t T = T_hist + T_seg, pos = T_hist + i, own0 = pos / kChunk * kChunk;
+    const int32_t* grow = gidx + row * wg;
+    const int n_g = prefix_count(grow, wg, lane);
+    const int n_keys = kGroup * n_g + int(pos - own0) + 1;
+    const TIn* Kb = K + bg * T * D + lane * P;
+    const TIn* Vb = V + bg * T * D + lane * P;
+    float qv[GM][P], acc[GM][P], m[GM], l[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+        m[h] = -INFINITY;
+        l[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < P; ++e) acc[h][e] = 0.f;
+        if (h < G) Row<TIn, P>::load(Q + ((b * Hq + g * G + h) * T_seg + i) * D + lane * P, qv[h]);
+    }
+    for (int k0 = 0; k0 < n_keys; k0 += R) {
+        float kv[R][P], vv[R][P];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            if (k0 + r < n_keys) {
+                const int64_t t = row_token(grow, n_g, own0, k0 + r);
+                Row<TIn, P>::load(Kb + t * D, kv[r]);
+                Row<TIn, P>::load(Vb + t * D, vv[r]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < P; ++e) kv[r][e] = vv[r][e] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+            if (h >= G) break;
+            float s[R], mb = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                float a = 0.f;
+#pragma unroll
+                for (int e = 0; e < P; ++e) a = fmaf(qv[h][e], kv[r][e], a);
+                a = warp_sum(a) * scale;
+                s[r] = k0 + r < n_keys ? a : -INFINITY;
+                mb = fmaxf(mb, s[r]);
+            }
+            const float mn = fmaxf(m[h], mb), c = expf(m[h] - mn);
+            l[h] *= c;
+#pragma unroll
+            for (int e = 0; e < P; ++e) acc[h][e] *= c;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float p = expf(s[r] - mn);
+                l[h] += p;
+#pragma unroll
+                for (int e = 0; e < P; ++e) acc[h][e] = fmaf(p, vv[r][e], acc[h][e]);
+            }
+            m[h] = mn;
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+        if (h >= G) break;
+        const int64_t orow = (b * Hq + g * G + h) * T_seg + i;
+        const float inv = 1.0f / l[h];
+#pragma unroll
+        for (int e = 0; e < P; ++e) O[orow * D + lane * P + e] = acc[h][e] * inv;
+        if (lane == 0) lse[orow] = m[h] + logf(l[h]);
+    }
+}
+
+// Vector float atomic add of P consecutive values (16- or 8-byte aligned).
+template <int P> __device__ __forceinline__ void atomic_add_vec(float* p, const float* v);
+template <> __device__ __forceinline__ void atomic_add_vec<4>(float* p, const float* v)
+{
+    atomicAdd(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
+}
+template <> __device__ __forceinline__ void atomic_add_vec<2>(float* p, const float* v)
+{
+    atomicAdd(reinterpret_cast<float2*>(p), make_float2(v[0], v[1]));
+}
+
+// Backward with the routing frozen: per key, P = exp(s - lse), dP = dO . V,
+// dS = P (dP - D) with D = dO . O; dQ += scale dS K in registers; the key's
+// dK (scale sum_h dS q_h) and dV (sum_h P dO_h) are added to dK_seg / dV_seg
+// when it is a segment key (history gets no gradient).
+template <typename TIn, int D, int GM>
+__global__ void __launch_bounds__(kThreads)
+causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TIn* __restrict__ V,
+                  const float* __restrict__ O, const float* __restrict__ lse, const TIn* __restrict__ dO,
+                  const int32_t* __restrict__ gidx, float* __restrict__ dQ, float* __restrict__ dK_seg,
+                  float* __restrict__ dV_seg, int Hq, int Hkv, int G, int64_t T_hist, int64_t T_seg, int wg,
+                  float scale)
+{
+    pdl_wait();
+    pdl_trigger();
+    constexpr int P = D / 32, R = 2;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
+    const int64_t bg = row / T_seg, i = row % T_seg;
+    const int64_t b = bg / Hkv, g = bg % Hkv;
+    const int64_t T = T_hist + T_seg, pos = T_hist + i, own0 = pos / kChunk * kChunk;
+    const int32_t* grow = gidx + row * wg;
+    const int n_g = prefix_count(grow, wg, lane);
+    const int n_keys = kGroup * n_g + int(pos - own0) + 1;
+    const TIn* Kb = K + bg * T * D + lane * P;
+    const TIn* Vb = V + bg * T * D + lane * P;
+    float* dKb = dK_seg + bg * T_seg * D + lane * P;
+    float* dVb = dV_seg + bg * T_seg * D + lane * P;
+    float qv[GM][P], dov[GM][P], dq[GM][P], Dh[GM], lh[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+#pragma unroll
+        for (int e = 0; e < P; ++e) dq[h][e] = 0.f;
+        Dh[h] = 0.f;
+        lh[h] = 0.f;
+        if (h < G) {
+            const int64_t qrow = (b * Hq + g * G + h) * T_seg + i;
+            Row<TIn, P>::load(Q + qrow * D + lane * P, qv[h]);
+            Row<TIn, P>::load(dO + qrow * D + lane * P, dov[h]);
+            float o[P];
+            Row<float, P>::load(O + qrow * D + lane * P, o);
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < P; ++e) a = fmaf(dov[h][e], o[e], a);
+            Dh[h] = warp_sum(a);
+            lh[h] = __ldg(lse + qrow);
+        } else {
+#pragma unroll
+            for (int e = 0; e < P; ++e) qv[h][e] = dov[h][e] = 0.f;
+        }
+    }
+    for (int k0 = 0; k0 < n_keys; k0 += R) {
+        float kv[R][P], vv[R][P];
+        int64_t tk[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            tk[r] = -1;
+            if (k0 + r < n_keys) {
+                tk[r] = row_token(grow, n_g, own0, k0 + r);
+                Row<TIn, P>::load(Kb + tk[r] * D, kv[r]);
+                Row<TIn, P>::load(Vb + tk[r] * D, vv[r]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            if (k0 + r >= n_keys) break;
+            float dk[P], dv[P];
+#pragma unroll
+            for (int e = 0; e < P; ++e) dk[e] = dv[e] = 0.f;
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
+                if (h >= G) break;
+                float s = 0.f, dp = 0.f;
+#pragma unroll
+                for (int e = 0; e < P; ++e) {
+                    s = fmaf(qv[h][e], kv[r][e], s);
+                    dp = fmaf(dov[h][e], vv[r][e], dp);
+                }
+                s = warp_sum(s) * scale;
+                dp = warp_sum(dp);
+                const float p = expf(s - lh[h]);
+                const float ds = p * (dp - Dh[h]);
+#pragma unroll
+                for (int e = 0; e < P; ++e) {
+                    dq[h][e] = fmaf(scale * ds, kv[r][e], dq[h][e]);
+                    dk[e] = fmaf(scale * ds, qv[h][e], dk[e]);
+                    dv[e] = fmaf(p, dov[h][e], dv[e]);
+                }
+            }
+            if (tk[r] >= T_hist) {
+                const int64_t t = tk[r] - T_hist;
+                atomic_add_vec<P>(dKb + t * D, dk);
+                atomic_add_vec<P>(dVb + t * D, dv);
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+        if (h >= G) break;
+        const int64_t qrow = (b * Hq + g * G + h) * T_seg + i;
+#pragma unroll
+        for (int e = 0; e < P; ++e) dQ[qrow * D + lane * P + e] = dq[h][e];
+    }
+}
+
+template <typename TIn, int D>
+cudaError_t launch_route(const Shape& s, const void* Q, const float* csum, const float* gsum, int32_t* cidx,
+                         int32_t* gidx, cudaStream_t st)
+{
+    const size_t smem = kWarps * route_warp_layout(s.nC, s.wc, D).total;
+    auto k = causal_route_kernel<TIn, D>;
+    cudaError_t e = allow_smem(k, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(s.B * s.Hkv * s.T_seg / kWarps);
+    return launch_pdl(k, dim3(grid), dim3(kThreads), smem, st, static_cast<const TIn*>(Q), csum, gsum, cidx, gidx,
+                      s.Hq, s.Hkv, s.G, s.T_hist, s.T_seg, s.k_c, s.wc, s.k_g, s.wg);
+}
+
+template <typename TIn, int D, int GM>
+cudaError_t launch_fwd(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* gidx, float* O,
+                       float* lse, cudaStream_t st)
+{
+    const unsigned grid = (unsigned)(s.B * s.Hkv * s.T_seg / kWarps);
+    return launch_pdl(causal_fwd_kernel<TIn, D, GM>, dim3(grid), dim3(kThreads), 0, st, static_cast<const TIn*>(Q),
+                      static_cast<const TIn*>(K), static_cast<const TIn*>(V), gidx, O, lse, s.Hq, s.Hkv, s.G,
+                      s.T_hist, s.T_seg, s.wg, s.scale);
+}
+
+template <typename TIn, int D, int GM>
+cudaError_t launch_bwd(const Shape& s, const void* Q, const void* K, const void* V, const float* O, const float* lse,
+                       const void* dO, const int32_t* gidx, float* dQ, float* dK, float* dV, cudaStream_t st)
+{
+    const size_t seg_bytes = sizeof(float) * (size_t)s.B * s.Hkv * s.T_seg * s.d;
+    cudaError_t e = cudaMemsetAsync(dK, 0, seg_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dV, 0, seg_bytes, st);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(s.B * s.Hkv * s.T_seg / kWarps);
+    return launch_pdl(causal_bwd_kernel<TIn, D, GM>, dim3(grid), dim3(kThreads), 0, st, static_cast<const TIn*>(Q),
+                      static_cast<const TIn*>(K), static_cast<const TIn*>(V), O, lse, static_cast<const TIn*>(dO),
+                      gidx, dQ, dK, dV, s.Hq, s.Hkv, s.G, s.T_hist, s.T_seg, s.wg, s.scale);
+}
+
+// Dispatch over input type, head dim and the bound on heads per kv-head.
+template <template <typename, int, int> class F, typename... A>
+cudaError_t dispatch(const Shape& s, A... a)
+{
+    const bool small = s.G <= 4;
+    if (s.dtype == HGA_BF16) {
+        if (s.d == 128) return small ? F<__nv_bfloat16, 128, 4>::run(s, a...) : F<__nv_bfloat16, 128, 8>::run(s, a...);
+        return small ? F<__nv_bfloat16, 64, 4>::run(s, a...) : F<__nv_bfloat16, 64, 8>::run(s, a...);
+    }
+    if (s.d == 128) return small ? F<float, 128, 4>::run(s, a...) : F<float, 128, 8>::run(s, a...);
+    return small ? F<float, 64, 4>::run(s, a...) : F<float, 64, 8>::run(s, a...);
+}
+
+template <typename TIn, int D, int GM> struct FwdOp {
+    static cudaError_t run(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* gidx, float* O,
+                           float* lse, cudaStream_t st)
+    {
+        return launch_fwd<TIn, D, GM>(s, Q, K, V, gidx, O, lse, st);
+    }
+};
+template <typename TIn, int D, int GM> struct BwdOp {
+    static cudaError_t run(const Shape& s, const void* Q, const void* K, const void* V, const float* O,
+                           const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK, float* dV,
+                           cudaStream_t st)
+    {
+        return launch_bwd<TIn, D, GM>(s, Q, K, V, O, lse, dO, gidx, dQ, dK, dV, st);
+    }
+};
+
+}  // namespace
+
+size_t route_causal_smem(const Shape& s) { return kWarps * route_warp_layout(s.nC, s.wc, s.d).total; }
+int causal_max_heads() { return kMaxG; }
+
+cudaError_t launch_route_causal(const Shape& s, const void* Q, const float* csum, const float* gsum, int32_t* cidx,
+                                int32_t* gidx, cudaStream_t st)
+{
+    if (s.dtype == HGA_BF16)
+        return s.d == 128 ? launch_route<__nv_bfloat16, 128>(s, Q, csum, gsum, cidx, gidx, st)
+                          : launch_route<__nv_bfloat16, 64>(s, Q, csum, gsum, cidx, gidx, st);
+    return s.d == 128 ? launch_route<float, 128>(s, Q, csum, gsum, cidx, gidx, st)
+                      : launch_route<float, 64>(s, Q, csum, gsum, cidx, gidx, st);
+}
+
+cudaError_t launch_attn_fwd_causal(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* gidx,
+                                   float* O, float* lse, cudaStream_t st)
+{
+    return dispatch<FwdOp>(s, Q, K, V, gidx, O, lse, st);
+}
+
+cudaError_t launch_attn_bwd_causal(const Shape& s, const void* Q, const void* K, const void* V, const float* O,
+                                   const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK,
+                                   float* dV, cudaStream_t st)
+{
+    return dispatch<BwdOp>(s, Q, K, V, O, lse, dO, gidx, dQ, dK, dV, st);
+}
+
+}  // namespace hga

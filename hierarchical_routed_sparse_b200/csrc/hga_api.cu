@@ -323,6 +323,72 @@ int hga_decode(const hga_params* p, int64_t pos, const void* q, const void* K, c
     return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_decode");
 }
 
+// Shared checks of the causal variant's calls.
+static int causal_shape(const hga_params* p, hga::Shape* s)
+{
+    if (int r = make_shape(p, s)) return r;
+    if (s->G > hga::causal_max_heads())
+        return fail(HGA_ERR_UNSUPPORTED, "the causal variant takes at most %d q-heads per kv-head (got %d)",
+                    hga::causal_max_heads(), s->G);
+    return HGA_OK;
+}
+
+int hga_route_causal(const hga_params* p, const void* Q, const float* csum, const float* gsum, int32_t* cidx,
+                     int32_t* gidx, hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = causal_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    CHECK_PTR(Q);
+    CHECK_PTR(csum);
+    CHECK_PTR(gsum);
+    CHECK_PTR(cidx);
+    CHECK_PTR(gidx);
+    if (hga::route_causal_smem(s) + 1024 > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "causal routing of %lld chunks / k_c=%d exceeds shared memory",
+                    (long long)s.nC, s.wc);
+    cudaError_t e = hga::launch_route_causal(s, Q, csum, gsum, cidx, gidx, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route_causal");
+}
+
+int hga_attn_fwd_causal(const hga_params* p, const void* Q, const void* K, const void* V, const int32_t* gidx,
+                        float* O, float* lse, hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = causal_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(gidx);
+    CHECK_PTR(O);
+    CHECK_PTR(lse);
+    cudaError_t e = hga::launch_attn_fwd_causal(s, Q, K, V, gidx, O, lse, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_fwd_causal");
+}
+
+int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K, const void* V, const float* O,
+                        const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK_seg,
+                        float* dV_seg, hga_stream_t stream)
+{
+    hga::Shape s;
+    if (int r = causal_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(O);
+    CHECK_PTR(lse);
+    CHECK_PTR(dO);
+    CHECK_PTR(gidx);
+    CHECK_PTR(dQ);
+    CHECK_PTR(dK_seg);
+    CHECK_PTR(dV_seg);
+    cudaError_t e = hga::launch_attn_bwd_causal(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg,
+                                                static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_bwd_causal");
+}
+
 int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* V,
                  const int32_t* gidx, float* O, float* lse, hga_stream_t stream)
 {

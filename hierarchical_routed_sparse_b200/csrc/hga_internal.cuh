@@ -142,6 +142,16 @@ cudaError_t launch_decode(const Shape& s, int64_t pos, const void* q, const void
 size_t decode_smem(const Shape& s);
 int decode_max_heads();
 int decode_status(bool clear);   // status word of decode.cu's bounded waits
+// Strictly causal variant: routing per query position (causal.cu).
+cudaError_t launch_route_causal(const Shape& s, const void* Q, const float* csum, const float* gsum, int32_t* cidx,
+                                int32_t* gidx, cudaStream_t st);
+cudaError_t launch_attn_fwd_causal(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* gidx,
+                                   float* O, float* lse, cudaStream_t st);
+cudaError_t launch_attn_bwd_causal(const Shape& s, const void* Q, const void* K, const void* V, const float* O,
+                                   const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK,
+                                   float* dV, cudaStream_t st);
+size_t route_causal_smem(const Shape& s);
+int causal_max_heads();
 cudaError_t launch_attn_fwd_simt(const Shape& s, const void* Q, const void* K, const void* V,
                                  const int32_t* gidx, float* O, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Shape& s, const void* Q, const void* K, const void* V,

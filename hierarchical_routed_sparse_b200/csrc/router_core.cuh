@@ -21,12 +21,12 @@ constexpr int kBatch = 16;          // candidates a warp scores at once
 
 // Scores of candidates 0..n-1 against the block query qs (shared memory):
 // score(c) = qs . row(c), written as a selection key into keys[c].  Warp w
-// takes batches of 16 candidates w, w+8, ...; for each batch every lane
+// of `Warps` takes batches of 16 candidates w, w+Warps, ...; for each batch every lane
 // issues its 16 coalesced loads (lane l holds elements [l*P, (l+1)*P) of each
 // row) before any arithmetic, so a batch costs one memory round trip, and
 // the 16 partial sums are reduced across the warp with 16 shuffles (each
 // step halves the values a lane carries).
-template <int D, typename RowFn>
+template <int D, int Warps = kRouterWarps, typename RowFn>
 __device__ __forceinline__ void score_candidates(const float* __restrict__ qs, int n, RowFn row_of,
                                                  unsigned long long* keys, int warp, int lane)
 {
@@ -34,7 +34,7 @@ __device__ __forceinline__ void score_candidates(const float* __restrict__ qs, i
     float q[P];
 #pragma unroll
     for (int e = 0; e < P; ++e) q[e] = qs[lane * P + e];
-    for (int base = warp * kBatch; base < n; base += kRouterWarps * kBatch) {
+    for (int base = warp * kBatch; base < n; base += Warps * kBatch) {
         float v[kBatch];
         int32_t id[kBatch];
         float x[kBatch][P];

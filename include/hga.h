@@ -245,6 +245,32 @@ int hga_decode(const hga_params* p, int64_t pos, const void* q, const void* K,
                const void* V, const float* csum, const float* gsum, float* O,
                float* lse, int32_t* cidx, int32_t* gidx, hga_stream_t stream);
 
+/* f1. Strictly causal variant (article section "The one real caveat:
+ * causal leakage": a block's routing depends on the scores of several query
+ * positions, so an earlier token sees later tokens through it; the authors
+ * mention a strictly causal variant).  Here every query position routes on
+ * its own query, a query block of one as in hga_decode: its block query is
+ * the mean of its G q-heads' queries; chunks c < (T_hist + i) / 64 are
+ * routed (top k_c), then their groups (top k_g); each q-head attends the
+ * routed groups' exact tokens and its own chunk up to itself.  The output
+ * at segment position i depends on positions <= i only.  Routing rows are
+ * per position:
+ *   cidx [B][Hkv][T_seg][wc], gidx [B][Hkv][T_seg][wg]   int32
+ * and the other tensors are as for the block calls.  hga_attn_bwd_causal
+ * zeroes dK_seg / dV_seg itself (they are accumulated with atomics, so
+ * their float32 sums are not bit-reproducible run to run).  At most 8
+ * q-heads per kv-head (HGA_ERR_UNSUPPORTED otherwise). */
+int hga_route_causal(const hga_params* p, const void* Q, const float* csum,
+                     const float* gsum, int32_t* cidx, int32_t* gidx,
+                     hga_stream_t stream);
+int hga_attn_fwd_causal(const hga_params* p, const void* Q, const void* K,
+                        const void* V, const int32_t* gidx, float* O,
+                        float* lse, hga_stream_t stream);
+int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K,
+                        const void* V, const float* O, const float* lse,
+                        const void* dO, const int32_t* gidx, float* dQ,
+                        float* dK_seg, float* dV_seg, hga_stream_t stream);
+
 /* Status word of the kernels' bounded waits: every wait of a tensor-core
  * kernel or of the decode kernel on a barrier gives up after one second, records the code of the wait
  * in this word and lets the kernel return (its outputs are then invalid).

@@ -170,3 +170,22 @@ def test_decode_rejects_bad_arguments_on_the_host(lib):
     # More than 8 q-heads per kv-head: refused before any launch.
     p9 = hga.Params(B=1, Hq=9, Hkv=1, d=128, T_hist=64, T_seg=64, k_c=2, k_g=4, dtype=hga.HGA_BF16).c()
     assert lib.hga_decode(ctypes.byref(p9), 3, *([ok] * 10), None) == hga.HGA_ERR_UNSUPPORTED
+
+
+def test_causal_calls_reject_bad_arguments_on_the_host(lib):
+    ok = ctypes.c_void_p(1 << 20)
+    p9 = hga.Params(B=1, Hq=9, Hkv=1, d=128, T_hist=64, T_seg=64, k_c=2, k_g=4, dtype=hga.HGA_BF16).c()
+    assert lib.hga_route_causal(ctypes.byref(p9), *([ok] * 5), None) == hga.HGA_ERR_UNSUPPORTED
+    assert lib.hga_attn_fwd_causal(ctypes.byref(p9), *([ok] * 6), None) == hga.HGA_ERR_UNSUPPORTED
+    assert lib.hga_attn_bwd_causal(ctypes.byref(p9), *([ok] * 10), None) == hga.HGA_ERR_UNSUPPORTED
+    p = _p().c()
+    a = [ok] * 10
+    a[6] = None
+    assert lib.hga_attn_bwd_causal(ctypes.byref(p), *a, None) == hga.HGA_ERR_INVALID_ARG
+    assert "gidx is NULL" in lib.hga_last_error().decode()
+    assert lib.hga_route_causal(ctypes.byref(p), ok, ok, ctypes.c_void_p((1 << 20) + 4), ok, ok, None) == \
+        hga.HGA_ERR_INVALID_ARG
+    assert "gsum is not 16-byte aligned" in lib.hga_last_error().decode()
+    # An empty segment is a no-op.
+    p0 = _p(T_seg=0).c()
+    assert lib.hga_attn_fwd_causal(ctypes.byref(p0), *([None] * 6), None) == hga.HGA_OK
