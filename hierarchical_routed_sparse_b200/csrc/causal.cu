@@ -34,7 +34,6 @@ using namespace rt;
 constexpr int kWarps = 8;                   // rows (warps) per CTA
 constexpr int kThreads = 32 * kWarps;
 constexpr int kMaxG = 8;                    // q-heads per kv-head
-constexpr int kKeysInFlight = 4;            // K / V rows a warp loads before using them
 
 __host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~size_t(15); }
 
@@ -180,18 +179,97 @@ __device__ __forceinline__ int64_t row_token(const int32_t* grow, int n_g, int64
                             : own0 + (k - kGroup * n_g);
 }
 
-// Forward: warp w of CTA x takes row 8 x + w of the (batch, kv-head, row)
-// grid, for the G q-heads of the kv-head.  GM >= G bounds the heads held in
-// registers.
+// 16 bytes of a row widened to float32 (8 bf16 or 4 float).
+template <typename TIn> struct U4;
+template <> struct U4<__nv_bfloat16> {
+    static constexpr int E = 8;
+    static __device__ __forceinline__ void unpack(const uint4& r, float* x) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+template <> struct U4<float> {
+    static constexpr int E = 4;
+    static __device__ __forceinline__ void unpack(const uint4& r, float* x) {
+        x[0] = __uint_as_float(r.x); x[1] = __uint_as_float(r.y);
+        x[2] = __uint_as_float(r.z); x[3] = __uint_as_float(r.w);
+    }
+};
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+// s[h] += x . rows[h][e0 .. e0+E) of the G rows held in shared memory (floats,
+// row stride D), for 16 bytes of a key row widened to x.
 template <typename TIn, int D, int GM>
-__global__ void __launch_bounds__(kThreads)
+__device__ __forceinline__ void dot16(const float* rows, int G, int e0, const uint4& raw, float* s)
+{
+    constexpr int E = U4<TIn>::E;
+    float x[E];
+    U4<TIn>::unpack(raw, x);
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+        if (h >= G) break;
+#pragma unroll
+        for (int v = 0; v < E; v += 4) {
+            const float4 q = *reinterpret_cast<const float4*>(rows + h * D + e0 + v);
+            s[h] = fmaf(q.x, x[v], s[h]);
+            s[h] = fmaf(q.y, x[v + 1], s[h]);
+            s[h] = fmaf(q.z, x[v + 2], s[h]);
+            s[h] = fmaf(q.w, x[v + 3], s[h]);
+        }
+    }
+}
+
+// s[h] = rows[h] . key row (all D elements), the key row read by this lane
+// alone in pieces of MaxInFlight loads of 16 bytes, each piece all in flight.
+template <typename TIn, int D, int GM, int MaxInFlight = 16>
+__device__ __forceinline__ void row_dots(const float* rows, int G, const TIn* krow, bool valid, float* s)
+{
+    constexpr int E = U4<TIn>::E;
+    constexpr int ROW_U4 = D / E;                    // 16-byte pieces of a row
+    constexpr int CH = ROW_U4 < MaxInFlight ? ROW_U4 : MaxInFlight;
+    const uint4* kr = reinterpret_cast<const uint4*>(krow);
+#pragma unroll
+    for (int h = 0; h < GM; ++h) s[h] = 0.f;
+#pragma unroll
+    for (int c = 0; c < ROW_U4; c += CH) {
+        uint4 r[CH];
+#pragma unroll
+        for (int u = 0; u < CH; ++u) r[u] = valid ? __ldg(kr + c + u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < CH; ++u) dot16<TIn, D, GM>(rows, G, (c + u) * E, r[u], s);
+    }
+}
+
+// V / K rows (dims layout) a warp loads at once: fewer when more heads'
+// state is held in registers.
+template <int GM> struct InFlight { static constexpr int fwd = GM <= 4 ? 16 : 8, bwd = GM <= 4 ? 8 : 4; };
+
+// Forward: warp w of CTA x takes row 8 x + w of the (batch, kv-head, row)
+// grid, for the G q-heads of the kv-head.  Keys go in batches of 32: lane j
+// reads key j's whole K row and scores it against the G queries (shared
+// memory); a running softmax per head (per-lane partial sums); then P V
+// with lanes over the head dims, 16 V rows in flight, each key's weights
+// broadcast from its lane.  GM >= G bounds the heads held in registers.
+template <typename TIn, int D, int GM>
+__global__ void __launch_bounds__(kThreads, GM <= 4 ? 2 : 1)
 causal_fwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TIn* __restrict__ V,
                   const int32_t* __restrict__ gidx, float* __restrict__ O, float* __restrict__ lse, int Hq, int Hkv,
                   int G, int64_t T_hist, int64_t T_seg, int wg, float scale)
 {
     pdl_wait();
     pdl_trigger();
-    constexpr int P = D / 32, R = kKeysInFlight;
+    constexpr int P = D / 32;
+    __shared__ __align__(16) float qsm[kWarps][GM * D];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
     const int64_t bg = row / T_seg, i = row % T_seg;
@@ -200,65 +278,76 @@ causal_fwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
     const int32_t* grow = gidx + row * wg;
     const int n_g = prefix_count(grow, wg, lane);
     const int n_keys = kGroup * n_g + int(pos - own0) + 1;
-    const TIn* Kb = K + bg * T * D + lane * P;
-    const TIn* Vb = V + bg * T * D + lane * P;
-    float qv[GM][P], acc[GM][P], m[GM], l[GM];
+    const TIn* Kb = K + bg * T * D;
+    const TIn* Vb = V + bg * T * D;
+    float* qw = qsm[warp];
+    for (int h = 0; h < G; ++h) {
+        float x[P];
+        Row<TIn, P>::load(Q + ((b * Hq + g * G + h) * T_seg + i) * D + lane * P, x);
+#pragma unroll
+        for (int e = 0; e < P; ++e) qw[h * D + lane * P + e] = x[e];
+    }
+    __syncwarp();
+    float m[GM], lp[GM], acc[GM][P];
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
         m[h] = -INFINITY;
-        l[h] = 0.f;
+        lp[h] = 0.f;
 #pragma unroll
         for (int e = 0; e < P; ++e) acc[h][e] = 0.f;
-        if (h < G) Row<TIn, P>::load(Q + ((b * Hq + g * G + h) * T_seg + i) * D + lane * P, qv[h]);
     }
-    for (int k0 = 0; k0 < n_keys; k0 += R) {
-        float kv[R][P], vv[R][P];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            if (k0 + r < n_keys) {
-                const int64_t t = row_token(grow, n_g, own0, k0 + r);
-                Row<TIn, P>::load(Kb + t * D, kv[r]);
-                Row<TIn, P>::load(Vb + t * D, vv[r]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < P; ++e) kv[r][e] = vv[r][e] = 0.f;
-            }
-        }
+    for (int k0 = 0; k0 < n_keys; k0 += 32) {
+        const bool valid = k0 + lane < n_keys;
+        const int64_t t = valid ? row_token(grow, n_g, own0, k0 + lane) : 0;
+        float s[GM], p[GM];
+        row_dots<TIn, D, GM>(qw, G, Kb + t * D, valid, s);
 #pragma unroll
         for (int h = 0; h < GM; ++h) {
             if (h >= G) break;
-            float s[R], mb = -INFINITY;
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                float a = 0.f;
-#pragma unroll
-                for (int e = 0; e < P; ++e) a = fmaf(qv[h][e], kv[r][e], a);
-                a = warp_sum(a) * scale;
-                s[r] = k0 + r < n_keys ? a : -INFINITY;
-                mb = fmaxf(mb, s[r]);
-            }
-            const float mn = fmaxf(m[h], mb), c = expf(m[h] - mn);
-            l[h] *= c;
+            const float sv = valid ? s[h] * scale : -INFINITY;
+            const float mn = fmaxf(m[h], warp_max(sv));
+            const float c = expf(m[h] - mn);
+            p[h] = expf(sv - mn);
+            lp[h] = fmaf(lp[h], c, p[h]);
 #pragma unroll
             for (int e = 0; e < P; ++e) acc[h][e] *= c;
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const float p = expf(s[r] - mn);
-                l[h] += p;
-#pragma unroll
-                for (int e = 0; e < P; ++e) acc[h][e] = fmaf(p, vv[r][e], acc[h][e]);
-            }
             m[h] = mn;
+        }
+        const int nb = min(32, n_keys - k0);
+        constexpr int NV = InFlight<GM>::fwd;
+        for (int j0 = 0; j0 < nb; j0 += NV) {
+            float vv[NV][P];
+#pragma unroll
+            for (int jj = 0; jj < NV; ++jj) {
+                const int64_t tj = __shfl_sync(0xFFFFFFFFu, t, (j0 + jj) & 31);
+                if (j0 + jj < nb) {
+                    Row<TIn, P>::load(Vb + tj * D + lane * P, vv[jj]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < P; ++e) vv[jj][e] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < NV; ++jj) {
+#pragma unroll
+                for (int h = 0; h < GM; ++h) {
+                    if (h >= G) break;
+                    const float pj = __shfl_sync(0xFFFFFFFFu, p[h], (j0 + jj) & 31);
+#pragma unroll
+                    for (int e = 0; e < P; ++e) acc[h][e] = fmaf(pj, vv[jj][e], acc[h][e]);
+                }
+            }
         }
     }
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
         if (h >= G) break;
+        const float l = warp_sum(lp[h]);
         const int64_t orow = (b * Hq + g * G + h) * T_seg + i;
-        const float inv = 1.0f / l[h];
+        const float inv = 1.0f / l;
 #pragma unroll
         for (int e = 0; e < P; ++e) O[orow * D + lane * P + e] = acc[h][e] * inv;
-        if (lane == 0) lse[orow] = m[h] + logf(l[h]);
+        if (lane == 0) lse[orow] = m[h] + logf(l);
     }
 }
 
@@ -273,12 +362,19 @@ template <> __device__ __forceinline__ void atomic_add_vec<2>(float* p, const fl
     atomicAdd(reinterpret_cast<float2*>(p), make_float2(v[0], v[1]));
 }
 
-// Backward with the routing frozen: per key, P = exp(s - lse), dP = dO . V,
-// dS = P (dP - D) with D = dO . O; dQ += scale dS K in registers; the key's
-// dK (scale sum_h dS q_h) and dV (sum_h P dO_h) are added to dK_seg / dV_seg
-// when it is a segment key (history gets no gradient).
+// Dynamic shared memory of the backward: per warp the G queries and the G
+// output gradients of its row (floats).
+__host__ __device__ inline size_t bwd_smem(int GM, int D) { return 2 * (size_t)kWarps * GM * D * sizeof(float); }
+
+// Backward with the routing frozen.  Keys in batches of 32: lane j reads key
+// j's K and V rows and forms, per head, P = exp(s - lse), dP = dO . V and
+// dS = P (dP - D) with D = dO . O.  Then, lanes over the head dims (K rows
+// 16 in flight), each key's dS and P broadcast from its lane: dQ += scale dS
+// K in registers; the key's dK = scale sum_h dS q_h and dV = sum_h P dO_h go
+// to dK_seg / dV_seg with vector atomics when it is a segment key (history
+// gets no gradient).
 template <typename TIn, int D, int GM>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, GM <= 4 ? 2 : 1)
 causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TIn* __restrict__ V,
                   const float* __restrict__ O, const float* __restrict__ lse, const TIn* __restrict__ dO,
                   const int32_t* __restrict__ gidx, float* __restrict__ dQ, float* __restrict__ dK_seg,
@@ -287,7 +383,8 @@ causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
 {
     pdl_wait();
     pdl_trigger();
-    constexpr int P = D / 32, R = 2;
+    constexpr int P = D / 32;
+    extern __shared__ __align__(16) float bsm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
     const int64_t bg = row / T_seg, i = row % T_seg;
@@ -296,17 +393,19 @@ causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
     const int32_t* grow = gidx + row * wg;
     const int n_g = prefix_count(grow, wg, lane);
     const int n_keys = kGroup * n_g + int(pos - own0) + 1;
-    const TIn* Kb = K + bg * T * D + lane * P;
-    const TIn* Vb = V + bg * T * D + lane * P;
+    const TIn* Kb = K + bg * T * D;
+    const TIn* Vb = V + bg * T * D;
     float* dKb = dK_seg + bg * T_seg * D + lane * P;
     float* dVb = dV_seg + bg * T_seg * D + lane * P;
+    float* qw = bsm + (size_t)warp * 2 * GM * D;
+    float* dow = qw + GM * D;
     float qv[GM][P], dov[GM][P], dq[GM][P], Dh[GM], lh[GM];
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
-#pragma unroll
-        for (int e = 0; e < P; ++e) dq[h][e] = 0.f;
         Dh[h] = 0.f;
         lh[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < P; ++e) qv[h][e] = dov[h][e] = dq[h][e] = 0.f;
         if (h < G) {
             const int64_t qrow = (b * Hq + g * G + h) * T_seg + i;
             Row<TIn, P>::load(Q + qrow * D + lane * P, qv[h]);
@@ -315,56 +414,64 @@ causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
             Row<float, P>::load(O + qrow * D + lane * P, o);
             float a = 0.f;
 #pragma unroll
-            for (int e = 0; e < P; ++e) a = fmaf(dov[h][e], o[e], a);
+            for (int e = 0; e < P; ++e) {
+                a = fmaf(dov[h][e], o[e], a);
+                qw[h * D + lane * P + e] = qv[h][e];
+                dow[h * D + lane * P + e] = dov[h][e];
+            }
             Dh[h] = warp_sum(a);
             lh[h] = __ldg(lse + qrow);
-        } else {
-#pragma unroll
-            for (int e = 0; e < P; ++e) qv[h][e] = dov[h][e] = 0.f;
         }
     }
-    for (int k0 = 0; k0 < n_keys; k0 += R) {
-        float kv[R][P], vv[R][P];
-        int64_t tk[R];
+    __syncwarp();
+    for (int k0 = 0; k0 < n_keys; k0 += 32) {
+        const bool valid = k0 + lane < n_keys;
+        const int64_t t = valid ? row_token(grow, n_g, own0, k0 + lane) : 0;
+        float s[GM], dp[GM], p[GM], ds[GM];
+        row_dots<TIn, D, GM, 8>(qw, G, Kb + t * D, valid, s);
+        row_dots<TIn, D, GM, 8>(dow, G, Vb + t * D, valid, dp);
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            tk[r] = -1;
-            if (k0 + r < n_keys) {
-                tk[r] = row_token(grow, n_g, own0, k0 + r);
-                Row<TIn, P>::load(Kb + tk[r] * D, kv[r]);
-                Row<TIn, P>::load(Vb + tk[r] * D, vv[r]);
-            }
+        for (int h = 0; h < GM; ++h) {
+            p[h] = valid && h < G ? expf(s[h] * scale - lh[h]) : 0.f;
+            ds[h] = p[h] * (dp[h] - Dh[h]);
         }
+        const int nb = min(32, n_keys - k0);
+        constexpr int NK = InFlight<GM>::bwd;
+        for (int j0 = 0; j0 < nb; j0 += NK) {
+            float kv[NK][P];
+            int64_t tj[NK];
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            if (k0 + r >= n_keys) break;
-            float dk[P], dv[P];
+            for (int jj = 0; jj < NK; ++jj) {
+                tj[jj] = __shfl_sync(0xFFFFFFFFu, t, (j0 + jj) & 31);
+                if (j0 + jj < nb) {
+                    Row<TIn, P>::load(Kb + tj[jj] * D + lane * P, kv[jj]);
+                } else {
 #pragma unroll
-            for (int e = 0; e < P; ++e) dk[e] = dv[e] = 0.f;
-#pragma unroll
-            for (int h = 0; h < GM; ++h) {
-                if (h >= G) break;
-                float s = 0.f, dp = 0.f;
-#pragma unroll
-                for (int e = 0; e < P; ++e) {
-                    s = fmaf(qv[h][e], kv[r][e], s);
-                    dp = fmaf(dov[h][e], vv[r][e], dp);
-                }
-                s = warp_sum(s) * scale;
-                dp = warp_sum(dp);
-                const float p = expf(s - lh[h]);
-                const float ds = p * (dp - Dh[h]);
-#pragma unroll
-                for (int e = 0; e < P; ++e) {
-                    dq[h][e] = fmaf(scale * ds, kv[r][e], dq[h][e]);
-                    dk[e] = fmaf(scale * ds, qv[h][e], dk[e]);
-                    dv[e] = fmaf(p, dov[h][e], dv[e]);
+                    for (int e = 0; e < P; ++e) kv[jj][e] = 0.f;
                 }
             }
-            if (tk[r] >= T_hist) {
-                const int64_t t = tk[r] - T_hist;
-                atomic_add_vec<P>(dKb + t * D, dk);
-                atomic_add_vec<P>(dVb + t * D, dv);
+#pragma unroll
+            for (int jj = 0; jj < NK; ++jj) {
+                float dk[P], dv[P];
+#pragma unroll
+                for (int e = 0; e < P; ++e) dk[e] = dv[e] = 0.f;
+#pragma unroll
+                for (int h = 0; h < GM; ++h) {
+                    if (h >= G) break;
+                    const float dsj = scale * __shfl_sync(0xFFFFFFFFu, ds[h], (j0 + jj) & 31);
+                    const float pj = __shfl_sync(0xFFFFFFFFu, p[h], (j0 + jj) & 31);
+#pragma unroll
+                    for (int e = 0; e < P; ++e) {
+                        dq[h][e] = fmaf(dsj, kv[jj][e], dq[h][e]);
+                        dk[e] = fmaf(dsj, qv[h][e], dk[e]);
+                        dv[e] = fmaf(pj, dov[h][e], dv[e]);
+                    }
+                }
+                if (j0 + jj < nb && tj[jj] >= T_hist) {
+                    const int64_t st = tj[jj] - T_hist;
+                    atomic_add_vec<P>(dKb + st * D, dk);
+                    atomic_add_vec<P>(dVb + st * D, dv);
+                }
             }
         }
     }
@@ -409,7 +516,10 @@ cudaError_t launch_bwd(const Shape& s, const void* Q, const void* K, const void*
     if (e == cudaSuccess) e = cudaMemsetAsync(dV, 0, seg_bytes, st);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)(s.B * s.Hkv * s.T_seg / kWarps);
-    return launch_pdl(causal_bwd_kernel<TIn, D, GM>, dim3(grid), dim3(kThreads), 0, st, static_cast<const TIn*>(Q),
+    const size_t smem = bwd_smem(GM, D);
+    auto k = causal_bwd_kernel<TIn, D, GM>;
+    if ((e = allow_smem(k, (int)smem)) != cudaSuccess) return e;
+    return launch_pdl(k, dim3(grid), dim3(kThreads), smem, st, static_cast<const TIn*>(Q),
                       static_cast<const TIn*>(K), static_cast<const TIn*>(V), O, lse, static_cast<const TIn*>(dO),
                       gidx, dQ, dK, dV, s.Hq, s.Hkv, s.G, s.T_hist, s.T_seg, s.wg, s.scale);
 }
