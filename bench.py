@@ -433,6 +433,18 @@ def run_gpu(args, w) -> None:
     e2e_value = whole_job_rate(w.B * w.T_seg, args.steps, world,
                                max_over_ranks(e0.elapsed_time(e1), dev))
 
+    # ---- the one-shot summaries of the whole context (not part of a step) ----------
+    full_ms = []
+    for _ in range(max(args.warmup, 3) + 5):
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        buf.summaries(K, 0, w.T, stream)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        full_ms.append(s0.elapsed_time(s1))
+    full_ms = statistics.median(full_ms[max(args.warmup, 3):])
+
     if rank == 0:
         alg = algorithmic(w)
         pk = peaks()
@@ -455,11 +467,29 @@ def run_gpu(args, w) -> None:
                     kernel=dom, launch_ms=dom_ms, algorithmic_bytes=a["bytes"],
                     algorithmic_flops=a["flops"], peak_source=pk["source"])
         stage_ms = {s: statistics.mean(v) for s, v in per_stage.items()}
+        # Every stage against the HBM roofline (algorithmic bytes / stage time;
+        # stage times carry the events' own cost of a few microseconds).
+        stage_bytes = dict(summaries=alg["summaries"]["bytes"],
+                           route=alg["route_chunks"]["bytes"] + alg["route_groups"]["bytes"],
+                           attn_fwd=alg["attn_fwd"]["bytes"], attn_bwd=alg["attn_bwd"]["bytes"])
+        stage_roof = {}
+        for s_, b_ in stage_bytes.items():
+            if s_ in stage_ms and stage_ms[s_] > 0:
+                gbs = b_ / (stage_ms[s_] * 1e-3) / 1e9
+                stage_roof[s_] = dict(ms=stage_ms[s_], algorithmic_bytes=b_, gb_per_s=gbs,
+                                      frac=gbs / pk["hbm_gbs"])
+        el = 2 if w.dtype == "bf16" else 4
+        full_bytes = w.B * w.Hkv * w.T * w.d * el + w.B * w.Hkv * (w.T // 64 + w.T // 8) * w.d * 4
+        stage_roof["summaries_full_history"] = dict(
+            ms=full_ms, algorithmic_bytes=full_bytes, gb_per_s=full_bytes / (full_ms * 1e-3) / 1e9,
+            frac=full_bytes / (full_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            note="one-shot build of all chunk / group summaries of the context, timed alone")
         line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype=w.dtype, data="synthetic",
                     config=config_of(w, not args.no_graph), stage_ms=stage_ms,
                     ms_per_step_with_stage_events=staged_ms / args.steps, roofline=roof,
+                    stage_roofline=stage_roof,
                     gpu_launches=(LAUNCHES_FWD + (LAUNCHES_BWD if w.backward else 0)) * args.steps,
                     e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d,
                              d2h_bytes_per_step=d2h),
