@@ -112,3 +112,29 @@ def test_outputs_do_not_see_later_positions(w):
     assert np.array_equal(a["O"][:, :, :p + 1], b["O"][:, :, :p + 1])
     assert np.array_equal(a["lse"][:, :, :p + 1], b["lse"][:, :, :p + 1])
     assert not np.array_equal(a["O"][:, :, p + 1:], b["O"][:, :, p + 1:])
+
+
+@pytest.mark.parametrize("T", [32768, 131072])
+def test_causal_long_context_sampled_units(T):
+    # Per-position routing over up to 511 / 2047 eligible chunks (the warp
+    # router's selection over shared memory), k_c 16, k_g 64: the whole
+    # problem on the GPU, two (batch, kv-head) units against the oracle.
+    from parity_util import unit_slice
+    w = W.sweep_point(T, 16, 64).with_(B=1)
+    x = w.full()
+    got = _run(w, x)
+    for g in (0, w.Hkv - 1):
+        wu, xu = unit_slice(w, x, 0, g)
+        orc = _oracle(wu, xu)
+        hs = slice(g * w.G, (g + 1) * w.G)
+        check_indices(got["cidx"][:, g:g + 1], orc["cidx"], orc["cgap"], "cidx")
+        same_c = (got["cidx"][:, g:g + 1] == orc["cidx"]).all(axis=-1)
+        check_indices(got["gidx"][:, g:g + 1], orc["gidx"], np.where(same_c, orc["ggap"], 0.0), "gidx")
+        att = _run(wu, xu, gidx_in=orc["gidx"])
+        for k in ("O", "lse", "dQ", "dK", "dV"):
+            err = maxabs(att[k], orc[k])
+            assert err <= TOL[w.dtype], f"{k}: {err:.3g}"
+        # The whole-problem run gives the same outputs on rows whose routing matched.
+        same = (got["gidx"][:, g:g + 1] == orc["gidx"]).all(axis=-1)       # [1, 1, T_seg]
+        rows = np.repeat(same, w.G, axis=1)
+        assert maxabs(got["O"][:, hs][rows], orc["O"][rows]) <= TOL[w.dtype]

@@ -193,3 +193,18 @@ def test_decode_rejects_bad_arguments():
     with pytest.raises(hga.HGAError) as e:
         hga.decode(p9, 10, q9, s9.K, s9.V, s9.csum, s9.gsum, s9.O, s9.lse, s9.cidx, s9.gidx)
     assert e.value.code == hga.HGA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("pos", [131071, 70000])
+def test_decode_long_context_sampled_units(pos):
+    # 128K context (2047 eligible chunks at the end: chunk selection over
+    # shared memory, not registers), k_c 16, k_g 64; two (batch, kv-head)
+    # units against the oracle.
+    from parity_util import unit_slice
+    w = W.sweep_point(131072, 16, 64).with_(B=1, backward=False)
+    x = w.full()
+    got, _ = _run_decode(w, x, pos)
+    for g in (0, w.Hkv - 1):
+        wu, xu = unit_slice(w, x, 0, g)
+        _compare(wu, xu, pos, {k: v[:, g:g + 1] if k in ("cidx", "gidx") else v[:, g * w.G:(g + 1) * w.G]
+                               for k, v in got.items()})
