@@ -419,17 +419,37 @@ def run_gpu(args, w) -> None:
         for hst, dv in zip(outs_h, outs_dev):
             hst.copy_(dv, non_blocking=True)
 
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    if w.backward:
+        # Training steps through hga.StepPipeline: the next step's uploads and
+        # the previous step's downloads overlap this step's compute (own
+        # streams, two device buffer sets); every step moves all its bytes.
+        pipe = hga.StepPipeline(p, K[:, :, :w.T_hist], V[:, :, :w.T_hist], device=dev)
+        outs_sets = [outs_h, [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs_dev]]
+        for i in range(args.warmup):
+            pipe.submit(Qh, Kh, Vh, dOh, outs_sets[i % 2])
+        pipe.synchronize()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(pipe.s_in)
+        for i in range(args.steps):
+            pipe.submit(Qh, Kh, Vh, dOh, outs_sets[i % 2])
+        e1.record(pipe.s_out)
+        torch.cuda.synchronize()
+        e2e_mode = "hga.StepPipeline: uploads, compute and downloads of consecutive steps overlapped"
+    else:
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_mode = "serial: upload, step, download on one stream"
     e2e_value = whole_job_rate(w.B * w.T_seg, args.steps, world,
                                max_over_ranks(e0.elapsed_time(e1), dev))
 
@@ -492,7 +512,7 @@ def run_gpu(args, w) -> None:
                     stage_roofline=stage_roof,
                     gpu_launches=(LAUNCHES_FWD + (LAUNCHES_BWD if w.backward else 0)) * args.steps,
                     e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d,
-                             d2h_bytes_per_step=d2h),
+                             d2h_bytes_per_step=d2h, mode=e2e_mode),
                     clocks=clk.summary())
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = oracle_step_rate(w, min_seconds=args.ref_seconds)

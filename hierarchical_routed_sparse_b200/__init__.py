@@ -8,8 +8,10 @@ Method source: the article "BMW's 16 GB GPU just did what needs an A100"
 holds the device buffers of one problem shape and runs a whole segment step;
 ``StagedKV`` runs the attention on history kept in host memory;
 ``DecodeState`` generates token by token (hga_decode); ``CausalBuffers``
-runs the strictly causal variant (routing per query position).
+runs the strictly causal variant (routing per query position);
+``StepPipeline`` overlaps host copies with the compute of segment steps.
 """
+from .pipeline import StepPipeline
 from .binding import (EXPORTS, HGA_ALL, HGA_BF16, HGA_ERR_CUDA, HGA_ERR_INVALID_ARG,
                       HGA_ERR_UNSUPPORTED, HGA_FP32, HGA_OK, LIB_PATH, NOALLOC_MAX_ROWS, Buffers,
                       CausalBuffers, DecodeState, HGAError, Params, StagedKV, attn_bwd_causal, attn_fwd_causal, route_causal,
@@ -18,5 +20,5 @@ from .binding import (EXPORTS, HGA_ALL, HGA_BF16, HGA_ERR_CUDA, HGA_ERR_INVALID_
 
 __all__ = ["EXPORTS", "HGA_ALL", "HGA_BF16", "HGA_FP32", "HGA_OK", "HGA_ERR_CUDA",
            "HGA_ERR_INVALID_ARG", "HGA_ERR_UNSUPPORTED", "LIB_PATH", "NOALLOC_MAX_ROWS", "Buffers", "HGAError",
-           "CausalBuffers", "DecodeState", "Params", "attn_bwd_causal", "attn_fwd_causal", "route_causal", "StagedKV", "decode", "stage_params", "stage_routed", "attn_bwd", "attn_bwd_noalloc", "attn_fwd", "build_summaries", "build_summaries_rows", "device_status", "load", "route", "route_chunks",
+           "CausalBuffers", "DecodeState", "Params", "StepPipeline", "attn_bwd_causal", "attn_fwd_causal", "route_causal", "StagedKV", "decode", "stage_params", "stage_routed", "attn_bwd", "attn_bwd_noalloc", "attn_fwd", "build_summaries", "build_summaries_rows", "device_status", "load", "route", "route_chunks",
            "route_groups", "route_widths", "version", "workspace_size"]
