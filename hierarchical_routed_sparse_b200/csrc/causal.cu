@@ -207,10 +207,11 @@ __device__ __forceinline__ float warp_max(float v)
     return v;
 }
 
-// s[h] += x . rows[h][e0 .. e0+E) of the G rows held in shared memory (floats,
-// row stride D), for 16 bytes of a key row widened to x.
+// s2[h] += x . rows[h][e0 .. e0+E) of the G rows held in shared memory
+// (floats, row stride D), for 16 bytes of a key row widened to x; packed
+// fp32x2 FMAs, the even and odd elements in the two halves of s2[h].
 template <typename TIn, int D, int GM>
-__device__ __forceinline__ void dot16(const float* rows, int G, int e0, const uint4& raw, float* s)
+__device__ __forceinline__ void dot16(const float* rows, int G, int e0, const uint4& raw, float2* s2)
 {
     constexpr int E = U4<TIn>::E;
     float x[E];
@@ -221,10 +222,8 @@ __device__ __forceinline__ void dot16(const float* rows, int G, int e0, const ui
 #pragma unroll
         for (int v = 0; v < E; v += 4) {
             const float4 q = *reinterpret_cast<const float4*>(rows + h * D + e0 + v);
-            s[h] = fmaf(q.x, x[v], s[h]);
-            s[h] = fmaf(q.y, x[v + 1], s[h]);
-            s[h] = fmaf(q.z, x[v + 2], s[h]);
-            s[h] = fmaf(q.w, x[v + 3], s[h]);
+            s2[h] = __ffma2_rn(make_float2(q.x, q.y), make_float2(x[v], x[v + 1]), s2[h]);
+            s2[h] = __ffma2_rn(make_float2(q.z, q.w), make_float2(x[v + 2], x[v + 3]), s2[h]);
         }
     }
 }
@@ -238,15 +237,30 @@ __device__ __forceinline__ void row_dots(const float* rows, int G, const TIn* kr
     constexpr int ROW_U4 = D / E;                    // 16-byte pieces of a row
     constexpr int CH = ROW_U4 < MaxInFlight ? ROW_U4 : MaxInFlight;
     const uint4* kr = reinterpret_cast<const uint4*>(krow);
+    float2 s2[GM];
 #pragma unroll
-    for (int h = 0; h < GM; ++h) s[h] = 0.f;
+    for (int h = 0; h < GM; ++h) s2[h] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int c = 0; c < ROW_U4; c += CH) {
         uint4 r[CH];
 #pragma unroll
         for (int u = 0; u < CH; ++u) r[u] = valid ? __ldg(kr + c + u) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int u = 0; u < CH; ++u) dot16<TIn, D, GM>(rows, G, (c + u) * E, r[u], s);
+        for (int u = 0; u < CH; ++u) dot16<TIn, D, GM>(rows, G, (c + u) * E, r[u], s2);
+    }
+#pragma unroll
+    for (int h = 0; h < GM; ++h) s[h] = s2[h].x + s2[h].y;
+}
+
+// acc[e] += w * v[e] for P (even) consecutive values, as packed fp32x2 FMAs.
+template <int P>
+__device__ __forceinline__ void axpy2(float w, const float* v, float* acc)
+{
+#pragma unroll
+    for (int e = 0; e < P; e += 2) {
+        const float2 r = __ffma2_rn(make_float2(w, w), make_float2(v[e], v[e + 1]), make_float2(acc[e], acc[e + 1]));
+        acc[e] = r.x;
+        acc[e + 1] = r.y;
     }
 }
 
@@ -333,8 +347,7 @@ causal_fwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
                 for (int h = 0; h < GM; ++h) {
                     if (h >= G) break;
                     const float pj = __shfl_sync(0xFFFFFFFFu, p[h], (j0 + jj) & 31);
-#pragma unroll
-                    for (int e = 0; e < P; ++e) acc[h][e] = fmaf(pj, vv[jj][e], acc[h][e]);
+                    axpy2<P>(pj, vv[jj], acc[h]);
                 }
             }
         }
@@ -460,12 +473,9 @@ causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
                     if (h >= G) break;
                     const float dsj = scale * __shfl_sync(0xFFFFFFFFu, ds[h], (j0 + jj) & 31);
                     const float pj = __shfl_sync(0xFFFFFFFFu, p[h], (j0 + jj) & 31);
-#pragma unroll
-                    for (int e = 0; e < P; ++e) {
-                        dq[h][e] = fmaf(dsj, kv[jj][e], dq[h][e]);
-                        dk[e] = fmaf(dsj, qv[h][e], dk[e]);
-                        dv[e] = fmaf(pj, dov[h][e], dv[e]);
-                    }
+                    axpy2<P>(dsj, kv[jj], dq[h]);
+                    axpy2<P>(dsj, qv[h], dk);
+                    axpy2<P>(pj, dov[h], dv);
                 }
                 if (j0 + jj < nb && tj[jj] >= T_hist) {
                     const int64_t st = tj[jj] - T_hist;
