@@ -616,9 +616,12 @@ def run_host_tier(args, w) -> None:
     total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in outer), dev)
     stage_ms = {s: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in events) for j, s in enumerate(stages)}
     value = whole_job_rate(w.B * w.T_seg, args.steps, world, total_ms)
-    # Host bytes read per step: 8 rows of K and of V per routed history group.
+    # Host bytes read per step: 8 rows of K and of V per staged history group.
     gidx = buf.gidx.cpu().numpy()
-    n_hist = int(((gidx >= 0) & (gidx < w.T_hist // 8)).sum())
+    # Distinct routed history groups per (batch, kv-head): each is staged once.
+    fsg = w.T_hist // 8
+    n_hist = sum(len(np.unique(gidx[b_, g_][(gidx[b_, g_] >= 0) & (gidx[b_, g_] < fsg)]))
+                 for b_ in range(gidx.shape[0]) for g_ in range(gidx.shape[1]))
     host_bytes = n_hist * 8 * w.d * (2 if w.dtype == "bf16" else 4) * 2
     if rank == 0:
         line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,

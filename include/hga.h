@@ -202,14 +202,15 @@ int hga_stage_params(const hga_params* p, hga_params* staged);
  *   K_hist, V_hist  [B][Hkv][T_hist][d]  history rows (host-mapped or device)
  *   K_seg, V_seg    [B][Hkv][T_seg][d]   segment rows (device)
  *   gidx            [B][Hkv][nQB][wg]    routing of hga_route (device)
- *   K_stage, V_stage [B][Hkv][T_stage + T_seg][d] (device, written): slot j
- *       of block qb holds the 8 rows of that block's j-th routed history
- *       group at rows (qb*wg + j)*8; the segment rows follow at T_stage.
- *       Slots of padding or of segment groups are left untouched and are
- *       never read by the attention kernels.
+ *   K_stage, V_stage [B][Hkv][T_stage + T_seg][d] (device, written): the
+ *       distinct history groups routed by any query block of the (batch,
+ *       kv-head), each copied once, in ascending group order: the k-th of
+ *       them at rows 8k .. 8k+7; the segment rows follow at T_stage.  Rows
+ *       past the last distinct group are left untouched and never read.
  *   gidx_stage      [B][Hkv][nQB][wg] (device, written): a history group
- *       becomes qb*wg + j, a segment group j' becomes T_stage/8 + j' -
- *       T_hist/8, padding stays -1; rows stay ascending.
+ *       becomes its rank k among the distinct routed history groups, a
+ *       segment group j' becomes T_stage/8 + j' - T_hist/8, padding stays
+ *       -1; rows stay ascending.
  * The segment keys keep their offsets past the (staged) history, so
  * dK_seg / dV_seg of the staged backward are those of the full problem.
  * Host-resident history is read over the host link with plain loads.

@@ -73,11 +73,17 @@ def _attention(p, Q, K, V, gidx, dO):
 
 
 def _check_stage_rows(w, gidx: np.ndarray, staged: np.ndarray, T_stage: int):
-    wg = gidx.shape[-1]
+    # A history group becomes its rank among the distinct routed history
+    # groups of its (batch, kv-head); a segment group moves past the staged
+    # history; padding stays -1.
     fsg = w.T_hist // 8
-    qb = np.arange(gidx.shape[2])[None, None, :, None]
-    j = np.arange(wg)[None, None, None, :]
-    want = np.where(gidx < 0, -1, np.where(gidx < fsg, qb * wg + j, T_stage // 8 + gidx - fsg))
+    want = np.full_like(gidx, -1)
+    for b in range(gidx.shape[0]):
+        for g in range(gidx.shape[1]):
+            row = gidx[b, g]
+            hist = np.unique(row[(row >= 0) & (row < fsg)])
+            assert 8 * len(hist) <= T_stage
+            want[b, g] = np.where(row < 0, -1, np.where(row < fsg, np.searchsorted(hist, row), T_stage // 8 + row - fsg))
     assert np.array_equal(staged, want)
 
 
