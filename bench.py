@@ -895,6 +895,8 @@ def run_decode(args, w) -> None:
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     wd = w.with_(B=args.decode_batch, backward=False)
+    if args.decode_layers > 1:
+        return run_decode_layers(args, wd)
     x = wd.full()
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     p = hga.Params.from_workload(wd)
@@ -984,6 +986,97 @@ def run_decode(args, w) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_decode_layers(args, wd) -> None:
+    """Decode through a stack of L attention layers per token: L caches (one
+    per layer, the workload's 16K context each), one CUDA graph per token
+    position holding the L hga_decode calls (and, at a chunk's last token,
+    the L summary appends), replayed with events around it; L2 flushed
+    before every token.  The decode kernels launch with programmatic
+    dependent launch, so each layer's launch overlaps the previous one's
+    tail.  One JSON line, config.mode = "decode_layers"."""
+    import torch
+
+    import hierarchical_routed_sparse_b200 as hga
+
+    dev = torch.device("cuda", 0)
+    L = args.decode_layers
+    x = wd.full()
+    tdt = torch.bfloat16 if wd.dtype == "bf16" else torch.float32
+    p = hga.Params.from_workload(wd)
+    K = torch.from_numpy(x["K"]).to(dev, tdt)
+    V = torch.from_numpy(x["V"]).to(dev, tdt)
+    pos0 = wd.T - 64
+    states = []
+    for _ in range(L):
+        st = hga.DecodeState(p, device=dev)
+        st.prefill(K[:, :, :pos0], V[:, :, :pos0])
+        st.K.copy_(K)
+        st.V.copy_(V)
+        states.append(st)
+    del K, V
+    qs = [torch.from_numpy(np.ascontiguousarray(x["Q"][:, :, i])).to(dev, tdt) for i in range(64)]
+    del x
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def token(i, st_):
+        pos = pos0 + i
+        for l_, sl in enumerate(states):
+            hga.decode(p, pos, qs[(i + l_) % 64], sl.K, sl.V, sl.csum, sl.gsum, sl.O, sl.lse, sl.cidx, sl.gidx, st_)
+        if (pos + 1) % 64 == 0:
+            for sl in states:
+                hga.build_summaries(p, sl.K, pos + 1 - 64, pos + 1, sl.csum, sl.gsum, st_)
+
+    for i in range(64):                              # warm-up, eager
+        token(i, stream)
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    graphs = []
+    with torch.cuda.stream(cap):
+        for i in range(64):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                token(i, cap)
+            graphs.append(g)
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+    for i in range(max(args.warmup, 3)):
+        flush.zero_()
+        graphs[i % 64].replay()
+    torch.cuda.synchronize()
+    n = max(args.steps, 64)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    with ClockSampler(0, None) as clk:
+        for i in range(n):
+            flush.zero_()
+            ev[i][0].record(stream)
+            graphs[i % 64].replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    ms_tok = statistics.mean(ms)
+    assert hga.device_status() == 0
+    pk = peaks()
+    alg = statistics.mean(decode_algorithmic(wd, pos0 + i)["bytes"] for i in range(63)) * L
+    achieved = alg / (ms_tok * 1e-3) / 1e9
+    line = dict(metric=f"HGA decode tokens/s at 16K ctx through {L} attention layers per token",
+                value=wd.B / (ms_tok * 1e-3), unit="tokens/s", n_gpus=1, steps=n, warmup=args.warmup,
+                ms_per_step=ms_tok, higher_is_better=True, scaling="weak", vs_baseline=None, dtype=wd.dtype,
+                data="synthetic",
+                config=dict(config_of(wd, graph=False), mode="decode_layers", decode_batch=wd.B, layers=L,
+                            positions=f"{pos0}..{wd.T - 1}, summaries appended at chunk end",
+                            l2="flushed before every token (256 MiB write)",
+                            launch="one CUDA graph per token position (L decode calls), events around its replay"),
+                us_per_layer=ms_tok * 1e3 / L,
+                roofline=dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
+                              frac=achieved / pk["hbm_gbs"], traffic=None, kernel="decode_kernel",
+                              algorithmic_bytes_per_step=alg, peak_source=pk["source"] + " (burst copy)"),
+                gpu_launches=sum(L + (L if (pos0 + i % 64 + 1) % 64 == 0 else 0) for i in range(n)),
+                clocks=clk.summary())
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -1005,6 +1098,8 @@ def main():
     ap.add_argument("--decode", action="store_true",
                     help="generation: one hga_decode step per token over the workload's context (f3)")
     ap.add_argument("--decode-batch", type=int, default=1, help="sequences decoded per step")
+    ap.add_argument("--decode-layers", type=int, default=1,
+                    help="attention layers per decoded token (one cache each; a CUDA graph per token)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu DRAM bytes per launch of the dominant kernel, if captured")
     args = ap.parse_args()

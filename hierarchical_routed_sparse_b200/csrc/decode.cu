@@ -407,13 +407,18 @@ cudaError_t launch(const Shape& s, int64_t pos, const void* q, const void* K, co
     cfg.blockDim = dim3(kRouterThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    // An 8-CTA cluster per (batch, kv-head); programmatic dependent launch,
+    // so that a step's launch overlaps the previous kernel's tail (the
+    // kernel reads no global memory before its griddepcontrol.wait).
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, k, static_cast<const TIn*>(q), static_cast<const TIn*>(K),
                               static_cast<const TIn*>(V), csum, gsum, O, lse, cidx, gidx, s.Hq, s.Hkv, s.G, s.T,
                               pos, s.k_c, s.wc, s.k_g, s.wg, s.scale);
