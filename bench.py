@@ -371,8 +371,7 @@ def run_gpu(args, w) -> None:
 
         def run_plain():
             plain.replay()
-    clocks_path = os.path.join(ROOT, "gpurun_out", "clocks.csv") if os.path.isdir(
-        os.path.join(ROOT, "gpurun_out")) else None
+    clocks_path = args.clocks_csv if rank == 0 else None
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -1100,6 +1099,8 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=1, help="sequences decoded per step")
     ap.add_argument("--decode-layers", type=int, default=1,
                     help="attention layers per decoded token (one cache each; a CUDA graph per token)")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="also write the nvidia-smi samples of the timed region to this file")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu DRAM bytes per launch of the dominant kernel, if captured")
     args = ap.parse_args()
