@@ -47,6 +47,8 @@ class StepPipeline:
             buf.summaries(K, 0, Th)                  # history summaries persist
             self.sets.append(dict(
                 Q=torch.empty(Bn, Hq, Ts, d, device=dev, dtype=dt), K=K, V=V,
+                Kseg=torch.empty(Bn, Hkv, Ts, d, device=dev, dtype=dt),
+                Vseg=torch.empty(Bn, Hkv, Ts, d, device=dev, dtype=dt),
                 dO=torch.empty(Bn, Hq, Ts, d, device=dev, dtype=dt), buf=buf,
                 in_done=torch.cuda.Event(), cmp_done=torch.cuda.Event(), out_done=torch.cuda.Event(),
                 used=False))
@@ -65,12 +67,14 @@ class StepPipeline:
         if S["used"]:
             self.s_in.wait_event(S["cmp_done"])
         with torch.cuda.stream(self.s_in):
+            # Four contiguous uploads; the segment rows then move into the
+            # caches' strided slots on the device.
             S["Q"].copy_(Qh, non_blocking=True)
             S["dO"].copy_(dOh, non_blocking=True)
-            for b in range(p.B):                     # contiguous rows per (b, kv-head)
-                for g in range(p.Hkv):
-                    S["K"][b, g, Th:].copy_(Kh_seg[b, g], non_blocking=True)
-                    S["V"][b, g, Th:].copy_(Vh_seg[b, g], non_blocking=True)
+            S["Kseg"].copy_(Kh_seg, non_blocking=True)
+            S["Vseg"].copy_(Vh_seg, non_blocking=True)
+            S["K"][:, :, Th:].copy_(S["Kseg"])
+            S["V"][:, :, Th:].copy_(S["Vseg"])
             S["in_done"].record(self.s_in)
         # Outputs of this set are free once the step two back is downloaded.
         self.s_cmp.wait_event(S["in_done"])
