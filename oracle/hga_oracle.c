@@ -483,7 +483,7 @@ void oracle_decode(const oracle_dims* p, int64_t pos, const double* q, const dou
  * leakage": a block's routing depends on the scores of several query
  * positions, so through the routing an earlier token sees the queries of
  * later tokens of its block; the authors mention a strictly causal variant
- * in the works without describing it.  Reading R11: every query position
+ * in the works without describing it.  Reading R14: every query position
  * routes on its own query, a query block of one exactly as in the decode
  * step -- qbar_i = mean of Q[., i] over the G q-heads of the kv-head, chunks
  * c < (T_hist + i) / chunk eligible (R4), groups of the chosen chunks (R5),
