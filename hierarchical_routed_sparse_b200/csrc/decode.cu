@@ -45,7 +45,7 @@ constexpr int kTileRows = kTileUnits * kGroup;
 constexpr int kSiteOwn = 0x301, kSiteTile = 0x302;   // bounded-wait sites
 
 struct DecodeLayout {
-    size_t ckeys, gkeys, ids, flags, crow, grow, qh, kv, sc, hs, part, bar, total;
+    size_t ckeys, gkeys, ids, flags, crow, grow, qh, kv, sc, hs, part, pvred, bar, total;
 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
@@ -64,6 +64,7 @@ __host__ __device__ inline int part_stride(int G, int D) { return G * D + ((2 * 
 //   sc [G][64]                  scores, then weights, of the tile
 //   hs [3][G]                   running max, sum and rescale factor per head
 //   part [kS][part_stride]      per-CTA O [G][D], max [G], sum [G] read by CTA 0
+//   pvred [256] float4          P V partial sums of the row slices
 //   bar                         two mbarriers (own unit, tiles)
 __host__ __device__ inline DecodeLayout decode_layout(int64_t nC, int wc, int wg, int G, int D, int el)
 {
@@ -79,7 +80,8 @@ __host__ __device__ inline DecodeLayout decode_layout(int64_t nC, int wc, int wg
     L.sc = align16(L.kv + 2 * (size_t)kTileRows * D * el);
     L.hs = align16(L.sc + 4 * (size_t)G * kTileRows);
     L.part = align16(L.hs + 4 * 3 * (size_t)G);
-    L.bar = align16(L.part + 4 * (size_t)kS * part_stride(G, D));
+    L.pvred = align16(L.part + 4 * (size_t)kS * part_stride(G, D));
+    L.bar = align16(L.pvred + 16 * (size_t)kRouterThreads);
     L.total = align16(L.bar + 16);
     return L;
 }
@@ -275,10 +277,15 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ K, const TIn* _
     for (int h = 0; h < kMaxG; ++h)
 #pragma unroll
         for (int e = 0; e < P; ++e) qv[h][e] = h < G ? qh[h * D + lane * P + e] : 0.f;
-    // P V: thread tid accumulates outputs 4 tid .. 4 tid + 3 of [G][D].
-    const int i4 = 4 * tid;
-    const bool pv_on = i4 < G * D;
-    const int ph = pv_on ? i4 / D : 0, pe = i4 % D;
+    // P V: the outputs [G][D] in nq quads of 4; thread tid takes quad
+    // tid % nq for the rows j = tid / nq (mod nh) of every tile, nh row
+    // slices in all; the slices' sums are added after the last tile.
+    const int nq = G * D / 4;
+    const int nh = kRouterThreads / nq;
+    const int slice = tid / nq;
+    const bool pv_on = slice < nh;
+    const int i4 = 4 * (tid % nq);
+    const int ph = i4 / D, pe = i4 % D;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     bool ok = true;
     for (int t = 0; t < n_tiles; ++t) {
@@ -348,7 +355,7 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ K, const TIn* _
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc[k] *= a;
             const float* wts = sc + ph * kTileRows;
-            for (int j = 0; j < nrows; ++j) {
+            for (int j = slice; j < nrows; j += nh) {
                 float v[4];
                 smem_row<TIn, 4>(vt + j * D + pe, v);
                 const float p = wts[j];
@@ -359,6 +366,21 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ K, const TIn* _
         __syncthreads();                             // the tile is free for the next copies
     }
 
+    // The row slices' partial sums, added in slice order by slice 0.
+    float4* pvred = reinterpret_cast<float4*>(sm + L.pvred);
+    if (pv_on && slice > 0) pvred[(slice - 1) * nq + tid % nq] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    __syncthreads();
+    const bool pv0 = slice == 0;
+    if (pv0) {
+        for (int sl = 1; sl < nh; ++sl) {
+            const float4 v = pvred[(sl - 1) * nq + tid];
+            acc[0] += v.x;
+            acc[1] += v.y;
+            acc[2] += v.z;
+            acc[3] += v.w;
+        }
+    }
+
     // Combine in CTA 0: O = sum_r O_r e^(m_r - M) / sum_r l_r e^(m_r - M).
     const int stride = part_stride(G, D);
     float* mine = part + (int)r * stride;
@@ -366,12 +388,12 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ K, const TIn* _
         st_cluster_f32(peer_addr(smem_u32(mine + G * D + tid), 0), ok ? hm[tid] : -INFINITY);
         st_cluster_f32(peer_addr(smem_u32(mine + G * D + G + tid), 0), ok ? hl[tid] : 0.f);
     }
-    if (pv_on) {
+    if (pv0) {
         const float z = ok ? 1.f : 0.f;
         st_cluster_v4(peer_addr(smem_u32(mine + i4), 0), acc[0] * z, acc[1] * z, acc[2] * z, acc[3] * z);
     }
     cluster_sync();
-    if (r == 0 && pv_on) {
+    if (r == 0 && pv0) {
         float M = -INFINITY;
 #pragma unroll
         for (int c = 0; c < kS; ++c) M = fmaxf(M, part[c * stride + G * D + ph]);
