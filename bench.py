@@ -497,6 +497,21 @@ def run_gpu(args, w) -> None:
                 gbs = b_ / (stage_ms[s_] * 1e-3) / 1e9
                 stage_roof[s_] = dict(ms=stage_ms[s_], algorithmic_bytes=b_, gb_per_s=gbs,
                                       frac=gbs / pk["hbm_gbs"])
+        # The routers' algorithmic bytes count every block's read of its
+        # eligible chunk summaries (per use); the distinct bytes -- Q, each
+        # (batch, kv-head)'s summaries once, the index rows -- bound what
+        # reaches HBM when L2 serves the re-reads.
+        el_ = 2 if w.dtype == "bf16" else 4
+        wc_ = w.k_c if w.k_c > 0 else w.T // 64
+        wg_ = w.k_g if w.k_g > 0 else 8 * wc_
+        uniq = (w.B * w.Hq * w.T_seg * w.d * el_ + w.B * w.Hkv * (w.T // 64 + w.T // 8) * w.d * 4
+                + w.B * w.Hkv * (w.T_seg // 64) * (w.d * 4 + (wc_ + wg_) * 4))
+        if "route" in stage_roof:
+            r_ = stage_roof["route"]
+            r_["unique_bytes"] = uniq
+            r_["frac_unique"] = uniq / (r_["ms"] * 1e-3) / 1e9 / pk["hbm_gbs"]
+            if r_["frac"] > 1.0:
+                r_["note"] = "per-use bytes above the copy peak: re-reads of the summaries hit L2"
         el = 2 if w.dtype == "bf16" else 4
         full_bytes = w.B * w.Hkv * w.T * w.d * el + w.B * w.Hkv * (w.T // 64 + w.T // 8) * w.d * 4
         stage_roof["summaries_full_history"] = dict(
