@@ -16,13 +16,19 @@
 //   causal_route_kernel  one warp per row: block query of one, chunk scores
 //                        (the 8 rows of a CTA share the summaries through
 //                        L1), warp top-k, group scores, warp rank selection;
-//   causal_fwd_kernel    one warp per (row, kv-head), the G heads together:
-//                        keys in batches of 4 (K and V rows in flight),
-//                        running softmax, O and lse;
-//   causal_bwd_kernel    one warp per (row, kv-head): P from lse, dP, dS,
-//                        dQ in registers; dK / dV of segment keys added with
-//                        vector float atomics.
-// Float32 arithmetic; bf16 or float32 inputs.
+//   causal_fwd_kernel    one warp per (row, kv-head), the G heads together,
+//                        keys in batches of 32: scores with one key per lane
+//                        (the lane reads the key's whole K row and dots it
+//                        with the G queries held in shared memory), a
+//                        running softmax per head, then P V with lanes over
+//                        the head dims (V rows in flight, each key's weight
+//                        broadcast from its lane); O and lse;
+//   causal_bwd_kernel    one warp per (row, kv-head), the same two layouts:
+//                        per key P from lse, dP, dS by lanes over keys; dQ
+//                        in registers and the key's dK / dV over head dims,
+//                        added to the segment's rows with vector float
+//                        atomics.
+// Float32 arithmetic (packed fp32x2 FMAs); bf16 or float32 inputs.
 #include "hga_internal.cuh"
 #include "router_core.cuh"
 
