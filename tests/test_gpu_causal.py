@@ -42,6 +42,8 @@ CASES = [
              keys="clustered", backward=True, seed=44),
     Workload("causal_no_history", B=1, Hq=2, Hkv=2, d=128, T_hist=0, T_seg=256, k_c=2, k_g=40,
              backward=True, seed=45),
+    Workload("causal_fp32_d128_k1", B=1, Hq=4, Hkv=1, d=128, T_hist=192, T_seg=128, k_c=1, k_g=1,
+             dtype="fp32", keys="clustered", backward=True, seed=46),
 ]
 
 

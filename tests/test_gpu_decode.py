@@ -46,6 +46,8 @@ CASES = [
     Workload("dec_gqa8_bf16", B=1, Hq=16, Hkv=2, d=128, T_hist=256, T_seg=64, k_c=2, k_g=6,
              keys="clustered", seed=34),
     Workload("dec_mha_bf16_d64", B=1, Hq=3, Hkv=3, d=64, T_hist=192, T_seg=64, k_c=4, k_g=40, seed=35),
+    Workload("dec_fp32_d128_k1", B=1, Hq=8, Hkv=2, d=128, T_hist=256, T_seg=64, k_c=1, k_g=1, dtype="fp32",
+             keys="clustered", seed=36),
 ]
 POSITIONS = [0, 5, 63, 64, 100, 127, 128, 250]
 
