@@ -76,8 +76,8 @@ struct BwdSmem {
     static constexpr int v_off = k_off + kKStages * H * kKVHalf;
     static constexpr int bar_off = v_off + kVStages * H * kKVHalf;
     static constexpr int n_bars = 26;
-    static constexpr int tab_off = bar_off + 8 * n_bars;       // (n_g, n_seg) of the CTA's first items
-    static constexpr int tmem_slot_off = tab_off + 8 * 64;
+    static constexpr int tab_off = bar_off + 8 * n_bars;       // (item, n_g, n_seg) of the CTA's first items
+    static constexpr int tmem_slot_off = tab_off + 16 * 64;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;
 };
@@ -97,6 +97,7 @@ constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDV = 384, kColDK =
 
 struct BwdArgs {
     const int32_t* gidx;
+    const int32_t* sched;      // CTA c's k-th item at sched[k * gridDim.x + c]
     const float* lse;
     const float* Drow;
     float* dQ;
@@ -143,28 +144,45 @@ __device__ __forceinline__ int2 count_row(const BwdArgs& a, int64_t it, int lane
 }
 
 // Items a CTA decodes once, in its prologue, into shared memory; later ones
-// (more than kItemTab items per CTA) are counted when reached.
+// (more than kItemTab items per CTA) are read and counted when reached.
 constexpr int kItemTab = 64;
 
-// Item k of this CTA (global index it).  Whole-warp call.
-__device__ __forceinline__ Item make_item(const BwdArgs& a, const int2* tab, int k, int64_t it, int lane)
+// Global index of CTA blockIdx.x's k-th item.
+__device__ __forceinline__ int item_at(const BwdArgs& a, const int4* tab, int k)
+{
+    return k < kItemTab ? tab[k].x : __ldg(a.sched + (int64_t)k * gridDim.x + blockIdx.x);
+}
+
+// Item k of this CTA.  Whole-warp call.
+__device__ __forceinline__ Item make_item(const BwdArgs& a, const int4* tab, int k, int lane)
 {
     Item m;
+    int it, n_g, n_seg;
+    if (k < kItemTab) {
+        const int4 e = tab[k];
+        it = e.x;
+        n_g = e.y;
+        n_seg = e.z;
+    } else {
+        it = __ldg(a.sched + (int64_t)k * gridDim.x + blockIdx.x);
+        const int2 c = count_row(a, it, lane);
+        n_g = c.x;
+        n_seg = c.y;
+    }
     const int n_pairs = (a.G + 1) / 2;
-    const int iit = int(it);
-    m.u = iit / n_pairs;
-    m.head0 = 2 * (iit % n_pairs);
+    m.u = it / n_pairs;
+    m.head0 = 2 * (it % n_pairs);
     m.qb = m.u % int(a.nQB);
     m.bg = m.u / int(a.nQB);
-    const int2 c = k < kItemTab ? tab[k] : count_row(a, it, lane);
-    m.n_g = c.x;
-    m.n_seg = c.y;
+    m.n_g = n_g;
+    m.n_seg = n_seg;
     return m;
 }
 
-// Persistent: CTA c processes items c, c + gridDim.x, ...  Barrier phases
-// run on a global key-tile counter (gt), a segment-tile counter (gs) and an
-// item counter (k) that every role advances identically.
+// Persistent: CTA c processes the items of its column of the schedule, as
+// many as round-robin would give it.  Barrier phases run on a global
+// key-tile counter (gt), a segment-tile counter (gs) and an item counter (k)
+// that every role advances identically.
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ CUtensorMap tm_v8,
@@ -191,14 +209,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t bar_final = bar0 + 8 * kBarFinal;
     const uint32_t bar_dqs_full = bar0 + 8 * kBarDqsFull;     // dQ staged in shared memory
     const uint32_t bar_dqs_free = bar0 + 8 * kBarDqsFree;     // its bulk stores have read it
-    int2* tab = reinterpret_cast<int2*>(smem + L::tab_off);
+    int4* tab = reinterpret_cast<int4*>(smem + L::tab_off);
     // Item k's Q/dO live in buffer k & 1, its P/dS in buffer (k + 1) & 1.
     auto xbuf = [&](int k) { return sbase + L::x_off + uint32_t(k & 1) * L::kX; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::tmem_slot_off);
     __shared__ int s_abort;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t n_items = a.n_items;
+    const int n_mine = int((a.n_items - blockIdx.x + gridDim.x - 1) / gridDim.x);
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -231,11 +249,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     pdl_trigger();
     // Decode the CTA's first items (warp w: items w, w + 18, ...).
     {
-        const int64_t n_mine = (n_items - blockIdx.x + gridDim.x - 1) / gridDim.x;
-        const int n_tab = int(n_mine < kItemTab ? n_mine : kItemTab);
+        const int n_tab = n_mine < kItemTab ? n_mine : kItemTab;
         for (int k = warp; k < n_tab; k += kThreads / 32) {
-            const int2 c = count_row(a, blockIdx.x + (int64_t)k * gridDim.x, lane);
-            if (lane == 0) tab[k] = c;
+            const int32_t it = __ldg(a.sched + (int64_t)k * gridDim.x + blockIdx.x);
+            const int2 c = count_row(a, it, lane);
+            if (lane == 0) tab[k] = make_int4(it, c.x, c.y, 0);
         }
     }
     tc_fence_before();
@@ -257,7 +275,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // kq_-1's P / dS.
         const int n_pairs = (a.G + 1) / 2;
         auto load_q = [&](int kq_) {
-            const int64_t itq = blockIdx.x + (int64_t)kq_ * gridDim.x;
+            const int64_t itq = item_at(a, tab, kq_);
             const int64_t u = itq / n_pairs, qb = u % a.nQB, bg = u / a.nQB;
             const int64_t b = bg / a.Hkv, g = bg % a.Hkv;
             const int head0 = 2 * int(itq % n_pairs);
@@ -278,10 +296,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         int q_issued = -1;                                  // last item whose Q / dO load was issued
         uint32_t gt = 0;
         bool ok = true;
-        int k = 0;
-        int64_t it = blockIdx.x;
-        for (; it < n_items && ok; it += gridDim.x, ++k) {
-            const Item m = make_item(a, tab, k, it, lane);
+        for (int k = 0; k < n_mine && ok; ++k) {
+            const Item m = make_item(a, tab, k, lane);
             const int nt = m.nt(), n_rt = m.n_rt();
             const int32_t* grow = m.grow(a);
             const int64_t kv_base = (int64_t)m.bg * (a.T_hist + a.T_seg);
@@ -316,7 +332,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         if (ok) load_q(k);
                         q_issued = k;
                     }
-                    if (ok && q_issued == k && it + gridDim.x < n_items && mbar_test(bar_pfree, k & 1)) {
+                    if (ok && q_issued == k && k + 1 < n_mine && mbar_test(bar_pfree, k & 1)) {
                         load_q(k + 1);
                         q_issued = k + 1;
                     }
@@ -358,14 +374,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         bool ok = true;
         // Cursor A walks the tiles whose S / dP are issued next, up to two
         // tiles ahead of the tile whose gradient MMAs run.
-        int64_t itA = blockIdx.x;
         int kA = 0, pA = 0, ntA = 0;
         uint32_t gtA = 0;
-        auto enter_A = [&]() { ntA = make_item(a, tab, kA, itA, lane).nt(); };
+        auto enter_A = [&]() { ntA = make_item(a, tab, kA, lane).nt(); };
         int pfree_k = -1;                                   // last item whose pfree was committed
         // S / dP of an item's first tile need its Q / dO, which load once the
         // previous item's P / dS are no longer read (pfree).
-        auto can_issue = [&]() { return itA < n_items && (pA > 0 || kA == 0 || pfree_k >= kA - 1); };
+        auto can_issue = [&]() { return kA < n_mine && (pA > 0 || kA == 0 || pfree_k >= kA - 1); };
         auto issue_sdp = [&]() -> bool {
             bool r = true;
             if (lane == 0) {
@@ -397,17 +412,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ++gtA;
             if (++pA == ntA) {
                 pA = 0;
-                ++kA;
-                itA += gridDim.x;
-                if (itA < n_items) enter_A();
+                if (++kA < n_mine) enter_A();
             }
             return r;
         };
-        if (itA < n_items) enter_A();
+        if (kA < n_mine) enter_A();
         uint32_t gt = 0, gs = 0;
-        int k = 0;
-        for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
-            const Item mc = make_item(a, tab, k, it, lane);
+        for (int k = 0; k < n_mine && ok; ++k) {
+            const Item mc = make_item(a, tab, k, lane);
             const int nt = mc.nt(), n_seg = mc.n_seg;
             for (int p = 0; ok && p < nt; ++p, ++gt) {
                 // S / dP up to two tiles ahead (this tile's always: its
@@ -525,11 +537,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         };
         uint32_t gt = 0, gs = 0;
         bool ok = true;
-        int k = 0;
-        int64_t it = blockIdx.x;
-        Item m = make_item(a, tab, 0, it, lane);           // gridDim.x <= n_items
+        Item m = make_item(a, tab, 0, lane);   // gridDim.x <= n_items
         RowInfo ri = row_info(m);
-        for (; it < n_items && ok; ++k) {
+        for (int k = 0; k < n_mine && ok; ++k) {
             const bool row_ok = ri.ok;
             const float lse2 = ri.lse2, Dr = ri.Dr;
             const uint32_t pd = xbuf(k + 1) - sbase;        // this item's P / dS buffer
@@ -633,8 +643,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             if (!ok) break;
             // The next item's index row and row constants load meanwhile.
-            const int64_t it_next = it + gridDim.x;
-            const Item m_next = it_next < n_items ? make_item(a, tab, k + 1, it_next, lane) : m;
+            const Item m_next = k + 1 < n_mine ? make_item(a, tab, k + 1, lane) : m;
             const RowInfo ri_next = row_info(m_next);
             if (pending) {
                 ok = mbar_wait(bar_kv, (gs - 1) & 1, kSiteKv);
@@ -678,7 +687,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
             }
             if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
-            it = it_next;
             m = m_next;
             ri = ri_next;
         }
@@ -696,26 +704,141 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
 }
 
+// ---------------------------------------------------------------- schedule
+// The backward kernel is persistent: its G CTAs take R = ceil(n / G) or R-1
+// items each.  An item's time grows with its key tiles and, more steeply,
+// with its segment tiles (their dK / dV products and atomics), which
+// depend on the routing.  Round-robin lets a CTA with R items draw heavy
+// ones and end well after the rest, so block 0 of the row-dot launch ranks
+// the items by estimated cost, heaviest first (ties by index), and deals
+// them out: the heaviest to the G - E CTAs that take R - 1 items, the
+// lightest to the E that take R, in rounds whose direction alternates.
+// sched[k * G + c] is CTA c's k-th item; CTA c takes the same number of
+// items as under round-robin.
+constexpr int kCostClasses = 64;
+
+struct SchedArgs {
+    const int32_t* gidx;
+    int32_t* sched;
+    int64_t n_items, first_seg_group;
+    int n_pairs, wg, G;
+};
+
+// Estimated cost of item `it`: key tiles plus segment tiles (each of those
+// costs about two), clamped to the class range.  Counts as count_row does,
+// one thread per item.
+__device__ __forceinline__ int item_cost(const SchedArgs& sa, int64_t it)
+{
+    const int32_t* row = sa.gidx + (it / sa.n_pairs) * sa.wg;
+    int n_g = 0, c_hist = 0;
+    if ((sa.wg & 3) == 0) {
+        for (int i = 0; i < sa.wg; i += 4) {
+            const int4 v = __ldg(reinterpret_cast<const int4*>(row + i));
+            const int j[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                n_g += j[q] >= 0;
+                c_hist += j[q] >= 0 && j[q] < sa.first_seg_group;
+            }
+        }
+    } else {
+        for (int i = 0; i < sa.wg; ++i) {
+            const int32_t j = __ldg(row + i);
+            n_g += j >= 0;
+            c_hist += j >= 0 && j < sa.first_seg_group;
+        }
+    }
+    const int n_rt = (n_g + 7) / 8;
+    const int n_seg = c_hist < n_g ? n_rt - c_hist / 8 + 1 : 1;
+    return min(n_rt + 1 + n_seg, kCostClasses - 1);
+}
+
+// Whole-block call (256 threads): counting sort of the items by cost class,
+// stable within a class, then the deal described above.
+__device__ void build_schedule(const SchedArgs& sa)
+{
+    __shared__ int hist[kCostClasses], next[kCostClasses];
+    __shared__ int wcnt[8][kCostClasses];
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int64_t n = sa.n_items;
+    for (int c = tid; c < kCostClasses; c += 256) hist[c] = 0;
+    __syncthreads();
+    for (int64_t i = tid; i < n; i += 256) atomicAdd(&hist[item_cost(sa, i)], 1);
+    __syncthreads();
+    // next[c] = items of classes above c (heaviest first): lane L sums
+    // classes 2L and 2L + 1, a suffix scan over the lanes does the rest.
+    if (warp == 0) {
+        const int h0 = hist[2 * lane], h1 = hist[2 * lane + 1];
+        const int own = h0 + h1;
+        int suf = own;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_down_sync(0xFFFFFFFFu, suf, o);
+            if (lane + o < 32) suf += v;
+        }
+        next[2 * lane + 1] = suf - own;
+        next[2 * lane] = suf - own + h1;
+    }
+    __syncthreads();
+    const int64_t G = sa.G, R = (n + G - 1) / G, E = n - (R - 1) * G, S = (G - E) * (R - 1);
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int64_t base = 0; base < n; base += 256) {
+        const int64_t i = base + tid;
+        const int c = i < n ? item_cost(sa, i) : -1;
+        for (int j = tid; j < 8 * kCostClasses; j += 256) (&wcnt[0][0])[j] = 0;
+        __syncthreads();
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, c);
+        const int below = __popc(peers & lt);
+        if (c >= 0 && below == 0) wcnt[warp][c] = __popc(peers);
+        __syncthreads();
+        if (c >= 0) {
+            int64_t rank = next[c] + below;
+            for (int w = 0; w < warp; ++w) rank += wcnt[w][c];
+            // Rank -> (CTA, round): ranks below S go to the CTAs E.. G-1
+            // (R - 1 items), the rest to CTAs 0 .. E-1 (R items).
+            const int64_t m = rank < S ? G - E : E, r = rank < S ? rank : rank - S;
+            const int64_t round = r / m;
+            int64_t pos = r % m;
+            if (round & 1) pos = m - 1 - pos;
+            const int64_t cta = rank < S ? E + pos : pos;
+            sa.sched[round * G + cta] = int32_t(i);
+        }
+        __syncthreads();
+        if (tid < kCostClasses) {
+            int add = 0;
+            for (int w = 0; w < 8; ++w) add += wcnt[w][tid];
+            next[tid] += add;
+        }
+        __syncthreads();
+    }
+}
+
 // D_row = sum_e dO[row][e] * O[row][e]: one warp per four rows, whose
 // 16-byte loads of O and 8-byte loads of dO are all issued before the sums.
 // The same launch zeroes dK_seg and dV_seg (the backward kernel adds into
-// them), n4 float4s each, grid-stride.
+// them), n4 float4s each, grid-stride; its block 0 builds the backward's
+// item schedule instead.
 constexpr int kRowdotRows = 4;
 
 __global__ void __launch_bounds__(256)
 rowdot_kernel(const float* __restrict__ O, const __nv_bfloat16* __restrict__ dO, float* __restrict__ Drow,
-              int64_t rows, float4* __restrict__ dK, float4* __restrict__ dV, int64_t n4)
+              int64_t rows, float4* __restrict__ dK, float4* __restrict__ dV, int64_t n4, const SchedArgs sa)
 {
     pdl_wait();
     pdl_trigger();
-    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+    if (blockIdx.x == 0) {
+        build_schedule(sa);
+        return;
+    }
+    const int64_t bx = blockIdx.x - 1;
+    const int64_t tid = bx * blockDim.x + threadIdx.x;
+    const int64_t nthreads = (int64_t)(gridDim.x - 1) * blockDim.x;
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int64_t j = tid; j < n4; j += nthreads) {
         dK[j] = z;
         dV[j] = z;
     }
-    const int64_t row0 = ((int64_t)blockIdx.x * 8 + threadIdx.x / 32) * kRowdotRows;
+    const int64_t row0 = (bx * 8 + threadIdx.x / 32) * kRowdotRows;
     const int lane = threadIdx.x & 31;
     float4 o[kRowdotRows];
     uint2 w[kRowdotRows];
@@ -766,9 +889,21 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
     const int64_t rows = (int64_t)s.B * s.Hq * s.T_seg;
     const int64_t n4 = (int64_t)s.B * s.Hkv * s.T_seg * D / 4;   // D = 128: whole float4s
     const int64_t rows_per_cta = 8 * kRowdotRows;
-    cudaError_t e = launch_pdl(rowdot_kernel, dim3((unsigned)((rows + rows_per_cta - 1) / rows_per_cta)), dim3(256),
-                               0, st, O, static_cast<const __nv_bfloat16*>(dO), Drow, rows,
-                               reinterpret_cast<float4*>(dK_seg), reinterpret_cast<float4*>(dV_seg), n4);
+    const int64_t n_items = bwd_items(s);
+    const int64_t grid = std::min<int64_t>(n_items, sm_count());
+    // The scratch holds the row sums, then the schedule (Drow + rows).
+    int32_t* sched = reinterpret_cast<int32_t*>(Drow + rows);
+    SchedArgs sa;
+    sa.gidx = gidx;
+    sa.sched = sched;
+    sa.n_items = n_items;
+    sa.first_seg_group = s.T_hist / 8;
+    sa.n_pairs = (s.G + 1) / 2;
+    sa.wg = s.wg;
+    sa.G = (int)grid;
+    cudaError_t e = launch_pdl(rowdot_kernel, dim3((unsigned)(1 + (rows + rows_per_cta - 1) / rows_per_cta)),
+                               dim3(256), 0, st, O, static_cast<const __nv_bfloat16*>(dO), Drow, rows,
+                               reinterpret_cast<float4*>(dK_seg), reinterpret_cast<float4*>(dV_seg), n4, sa);
     if (e != cudaSuccess) return e;
     CUtensorMap tq, tdo, tk8, tv8, tk64, tv64, tdq;
     const uint64_t q_rows = (uint64_t)rows, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
@@ -798,8 +933,8 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
     if ((e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
         return e;
-    a.n_items = (int64_t)s.B * s.Hkv * s.nQB * ((s.G + 1) / 2);
-    const int64_t grid = std::min<int64_t>(a.n_items, sm_count());
+    a.n_items = n_items;
+    a.sched = sched;
     return launch_pdl(attn_bwd_tc_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st, tq, tdo, tk8, tv8,
                       tk64, tv64, tdq, a);
 }

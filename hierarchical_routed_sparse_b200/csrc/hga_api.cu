@@ -91,7 +91,8 @@ int make_shape(const hga_params* p, hga::Shape* s)
 
 
 // The backward kernels: bf16 with d = 128 on the tensor cores, everything
-// else on the FMA kernel.  Drow is the B*Hq*T_seg-float row-sum scratch.
+// else on the FMA kernel.  Drow is the scratch of hga::bwd_scratch_floats:
+// row sums, then (tensor-core kernel only) the item schedule.
 cudaError_t run_attn_bwd(const hga::Shape& s, const void* Q, const void* K, const void* V, const float* O,
                          const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK_seg,
                          float* dV_seg, float* Drow, cudaStream_t st)
@@ -164,7 +165,7 @@ size_t hga_workspace_size(const hga_params* p)
 {
     hga::Shape s;
     if (make_shape(p, &s)) return 0;
-    return sizeof(float) * (size_t)s.B * s.Hq * s.T_seg;
+    return sizeof(float) * (size_t)hga::bwd_scratch_floats(s);
 }
 
 int hga_build_summaries(const hga_params* p, const void* K, int64_t t_begin, int64_t t_end,
@@ -428,7 +429,7 @@ int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* 
     CHECK_PTR(dK_seg);
     CHECK_PTR(dV_seg);
     CHECK_PTR(workspace);
-    const size_t need = sizeof(float) * (size_t)s.B * s.Hq * s.T_seg;
+    const size_t need = sizeof(float) * (size_t)hga::bwd_scratch_floats(s);
     if (ws_bytes < need)
         return fail(HGA_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, need);
     if (!hga::attn_bwd_tc_supported(s) && hga::attn_simt_smem(s, true) > kMaxSmem)
@@ -454,7 +455,8 @@ int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* 
 // once per device with cudaGetSymbolAddress, on the first call made while
 // that device is current, and cached.
 
-static __device__ __align__(256) float g_noalloc_rowsum[HGA_NOALLOC_MAX_ROWS];
+// Row sums, then the item schedule (at most one item per 64 rows).
+static __device__ __align__(256) float g_noalloc_rowsum[HGA_NOALLOC_MAX_ROWS + HGA_NOALLOC_MAX_ROWS / 64];
 
 namespace {
 

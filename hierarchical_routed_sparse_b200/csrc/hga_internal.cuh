@@ -27,6 +27,14 @@ struct Shape {
     int dtype;
 };
 
+// Work items of the tensor-core backward: one per (batch, kv-head, query
+// block) and pair of q-heads.  At most B*Hq*T_seg / 64.
+inline int64_t bwd_items(const Shape& s) { return (int64_t)s.B * s.Hkv * s.nQB * ((s.G + 1) / 2); }
+
+// Backward scratch, in floats: the row sums D (B*Hq*T_seg floats), then the
+// backward's item schedule (one int32 per item).
+inline int64_t bwd_scratch_floats(const Shape& s) { return (int64_t)s.B * s.Hq * s.T_seg + bwd_items(s); }
+
 // ---- element loads --------------------------------------------------------
 // 16-byte vector of inputs widened to float32 (8 bf16 or 4 float).
 template <typename T> struct Vec16;

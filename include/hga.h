@@ -83,8 +83,10 @@ typedef struct hga_params {
  * (8 * wc for HGA_ALL).  Returns HGA_OK or HGA_ERR_INVALID_ARG. */
 int hga_route_widths(const hga_params* p, int* wc, int* wg);
 
-/* Bytes of device scratch that hga_attn_bwd needs (B*Hq*T_seg floats for
- * the per-row sums D = rowsum(dO * O)).  0 on invalid parameters. */
+/* Bytes of device scratch that hga_attn_bwd needs: B*Hq*T_seg floats for
+ * the per-row sums D = rowsum(dO * O), then one int32 per work item of the
+ * backward (B*Hkv*(T_seg/64)*ceil(G/2), G = Hq/Hkv) for its schedule.  0 on
+ * invalid parameters. */
 size_t hga_workspace_size(const hga_params* p);
 
 /* a1. Chunk and group summaries: the mean of each 64-token chunk and of each
@@ -162,9 +164,9 @@ int hga_attn_bwd(const hga_params* p, const void* Q, const void* K,
  * its inputs and outputs, hosts whose memory pool owns all device memory,
  * and loops that must not call cudaMalloc / cudaFree.  It computes what
  * hga_attn_bwd computes and allocates nothing: its scratch (B*Hq*T_seg
- * floats of row sums) is a fixed array of HGA_NOALLOC_MAX_ROWS floats (4 MiB)
- * inside the library, held on every device that loads the library until the
- * process exits.
+ * floats of row sums, then the backward's item schedule) is a fixed array
+ * of HGA_NOALLOC_MAX_ROWS * 65 / 64 words (about 4 MiB) inside the library,
+ * held on every device that loads the library until the process exits.
  *   - B*Hq*T_seg above HGA_NOALLOC_MAX_ROWS returns HGA_ERR_INVALID_ARG,
  *     with nothing launched.
  *   - The first call on a device (the calling thread's current device, which

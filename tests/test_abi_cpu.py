@@ -45,7 +45,9 @@ def test_route_widths_and_workspace(lib):
     assert hga.route_widths(_p()) == (8, 32)
     assert hga.route_widths(_p(k_c=hga.HGA_ALL, k_g=hga.HGA_ALL)) == (256, 2048)
     assert hga.route_widths(_p(k_c=4, k_g=hga.HGA_ALL)) == (4, 32)
-    assert hga.workspace_size(_p()) == 4 * 32 * 2048
+    # Row sums (B*Hq*T_seg floats), then one int per backward item
+    # (B*Hkv*nQB*ceil(G/2) = 8 * 32 * 2).
+    assert hga.workspace_size(_p()) == 4 * (32 * 2048 + 8 * 32 * 2)
     assert hga.workspace_size(_p(d=96)) == 0
 
 
