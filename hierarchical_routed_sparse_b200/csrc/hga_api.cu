@@ -153,7 +153,7 @@ int hga_device_status(int* status, int clear)
 
 int hga_route_widths(const hga_params* p, int* wc, int* wg)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (!wc || !wg) return fail(HGA_ERR_INVALID_ARG, "wc / wg output pointer is NULL");
     *wc = s.wc;
@@ -163,7 +163,7 @@ int hga_route_widths(const hga_params* p, int* wc, int* wg)
 
 size_t hga_workspace_size(const hga_params* p)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (make_shape(p, &s)) return 0;
     return sizeof(float) * (size_t)hga::bwd_scratch_floats(s);
 }
@@ -171,7 +171,7 @@ size_t hga_workspace_size(const hga_params* p)
 int hga_build_summaries(const hga_params* p, const void* K, int64_t t_begin, int64_t t_end,
                         float* csum, float* gsum, hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (t_begin < 0 || t_end < t_begin || t_end > s.T || t_begin % 64 || t_end % 64)
         return fail(HGA_ERR_INVALID_ARG, "need 0 <= t_begin <= t_end <= T with multiples of 64 (got %lld, %lld, T=%lld)",
@@ -188,7 +188,7 @@ int hga_build_summaries(const hga_params* p, const void* K, int64_t t_begin, int
 int hga_build_summaries_rows(const hga_params* p, const void* K_rows, int64_t t_begin, int64_t t_end,
                              float* csum, float* gsum, hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (t_begin < 0 || t_end < t_begin || t_end > s.T || t_begin % 64 || t_end % 64)
         return fail(HGA_ERR_INVALID_ARG, "need 0 <= t_begin <= t_end <= T with multiples of 64 (got %lld, %lld, T=%lld)",
@@ -205,7 +205,7 @@ int hga_build_summaries_rows(const hga_params* p, const void* K_rows, int64_t t_
 int hga_route_chunks(const hga_params* p, const void* Q, const float* csum, float* qbar,
                      int32_t* cidx, hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
     CHECK_PTR(Q);
@@ -222,7 +222,7 @@ int hga_route_chunks(const hga_params* p, const void* Q, const float* csum, floa
 int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum, const int32_t* cidx,
                      int32_t* gidx, hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
     CHECK_PTR(qbar);
@@ -238,7 +238,7 @@ int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum, 
 int hga_route(const hga_params* p, const void* Q, const float* csum, const float* gsum, float* qbar,
               int32_t* cidx, int32_t* gidx, hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
     CHECK_PTR(Q);
@@ -256,7 +256,7 @@ int hga_route(const hga_params* p, const void* Q, const float* csum, const float
 
 int hga_stage_params(const hga_params* p, hga_params* staged)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (!staged) return fail(HGA_ERR_INVALID_ARG, "staged is NULL");
     *staged = *p;
@@ -272,7 +272,7 @@ int hga_stage_routed(const hga_params* p, const void* K_hist, const void* V_hist
                      const void* V_seg, const int32_t* gidx, void* K_stage, void* V_stage, int32_t* gidx_stage,
                      hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
     if (s.T_hist > 0) {
@@ -300,7 +300,7 @@ int hga_decode(const hga_params* p, int64_t pos, const void* q, const void* K, c
                const float* csum, const float* gsum, float* O, float* lse, int32_t* cidx, int32_t* gidx,
                hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (pos < 0 || pos >= s.T)
         return fail(HGA_ERR_INVALID_ARG, "pos (%lld) must lie in [0, T=%lld)", (long long)pos, (long long)s.T);
@@ -337,7 +337,7 @@ static int causal_shape(const hga_params* p, hga::Shape* s)
 int hga_route_causal(const hga_params* p, const void* Q, const float* csum, const float* gsum, int32_t* cidx,
                      int32_t* gidx, hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = causal_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
     CHECK_PTR(Q);
@@ -355,7 +355,7 @@ int hga_route_causal(const hga_params* p, const void* Q, const float* csum, cons
 int hga_attn_fwd_causal(const hga_params* p, const void* Q, const void* K, const void* V, const int32_t* gidx,
                         float* O, float* lse, hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = causal_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
     CHECK_PTR(Q);
@@ -372,7 +372,7 @@ int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K, const
                         const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK_seg,
                         float* dV_seg, hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = causal_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
     CHECK_PTR(Q);
@@ -393,7 +393,7 @@ int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K, const
 int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* V,
                  const int32_t* gidx, float* O, float* lse, hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
     CHECK_PTR(Q);
@@ -415,7 +415,7 @@ int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* 
                  const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK_seg,
                  float* dV_seg, void* workspace, size_t ws_bytes, hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
     CHECK_PTR(Q);
@@ -491,7 +491,7 @@ extern "C" int hga_attn_bwd_noalloc(const hga_params* p, const void* Q, const vo
                                     const int32_t* gidx, float* dQ, float* dK_seg, float* dV_seg,
                                     hga_stream_t stream)
 {
-    hga::Shape s;
+    hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
     CHECK_PTR(Q);
