@@ -7,10 +7,11 @@ CTA c's k-th item is sched[k * G + c].  Checked here from the workspace
 after a backward call, against the routing the call used:
   * the schedule is a permutation of the items and CTA c takes as many
     items as round-robin would give it (ceil((n - c) / G));
-  * items are ranked by estimated cost (key tiles plus segment tiles of
-    their index row) and the heaviest go to the CTAs that take one item
-    fewer: no item of a CTA with R items costs more than any item of a CTA
-    with R - 1 items.
+  * when a CTA takes at most 4 items (R <= 4), items are ranked by
+    estimated cost (key tiles plus segment tiles of their index row) and the
+    heaviest go to the CTAs that take one item fewer: no item of a CTA with
+    R items costs more than any item of a CTA with R - 1 items;
+  * with more items a CTA, the schedule is round-robin (the identity).
 The gradients themselves are the parity tests' subject.
 """
 import numpy as np
@@ -39,8 +40,10 @@ CASES = [
              keys="clustered", backward=True, seed=41),                # G 3: a pair with one head
     Workload("sched_few_items", B=1, Hq=4, Hkv=2, d=128, T_hist=256, T_seg=256, k_c=2, k_g=9,
              backward=True, seed=42),                                  # fewer items than SMs
-    Workload("sched_wide_rows", B=1, Hq=32, Hkv=8, d=128, T_hist=8192, T_seg=4096, k_c=4, k_g=19,
-             keys="clustered", backward=True, seed=43),                # 1024 items, wg not a multiple of 4
+    Workload("sched_wide_rows", B=1, Hq=32, Hkv=8, d=128, T_hist=8192, T_seg=2048, k_c=4, k_g=19,
+             keys="clustered", backward=True, seed=43),                # wg not a multiple of 4
+    Workload("sched_many_items", B=2, Hq=32, Hkv=8, d=128, T_hist=2048, T_seg=4096, k_c=4, k_g=16,
+             keys="clustered", backward=True, seed=44),                # 2048 items: round-robin
 ]
 
 
@@ -73,6 +76,9 @@ def test_schedule_is_a_balanced_permutation(w):
     sched = buf.ws.view(torch.int32)[rows:rows + n].cpu().numpy()
     assert sorted(sched.tolist()) == list(range(n))
     G = min(n, torch.cuda.get_device_properties(0).multi_processor_count)
+    if (n + G - 1) // G > 4:
+        assert np.array_equal(sched, np.arange(n)), w.name
+        return
     gidx = buf.gidx.cpu().numpy().reshape(-1, buf.gidx.shape[-1])
     cost = np.array([_cost(gidx[i // n_pairs], w.T_hist) for i in range(n)])
     R = (n + G - 1) // G
