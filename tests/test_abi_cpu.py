@@ -49,6 +49,9 @@ def test_route_widths_and_workspace(lib):
     # (B*Hkv*nQB*ceil(G/2) = 8 * 32 * 2).
     assert hga.workspace_size(_p()) == 4 * (32 * 2048 + 8 * 32 * 2)
     assert hga.workspace_size(_p(d=96)) == 0
+    # G = 3: two q-head pairs per (kv-head, block), the second with one head.
+    p3 = _p(B=2, Hq=6, Hkv=2, T_hist=1024, T_seg=640)
+    assert hga.workspace_size(p3) == 4 * (2 * 6 * 640 + 2 * 2 * 10 * 2)
 
 
 @pytest.mark.parametrize("kw,code", [
