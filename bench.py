@@ -183,10 +183,14 @@ class ClockSampler:
 
 
 # ---- the CPU oracle, timed on this host ------------------------------------------------------
-def oracle_step_rate(w, min_seconds: float = 10.0, max_reps: int = 50) -> dict:
+def oracle_step_rate(w, min_seconds: float = 10.0, max_reps: int = 50, one_thread: bool = False) -> dict:
     """Time the oracle's segment step (same stages as the GPU step) on the host.
 
-    The sample is the whole workload, repeated until min_seconds of CPU work.
+    The sample is the whole workload, repeated until min_seconds of CPU work,
+    on every core OpenMP uses.  With one_thread, the same step is also timed
+    on one thread over one (batch, kv-head) unit (the units are independent
+    and equal in work), repeated until a quarter of min_seconds, and scaled
+    to the workload's units.
     """
     import oracle
     oracle.build()
@@ -207,11 +211,39 @@ def oracle_step_rate(w, min_seconds: float = 10.0, max_reps: int = 50) -> dict:
         el = time.perf_counter() - t0
         if el >= min_seconds or reps >= max_reps:
             break
-    return dict(value=reps * w.B * w.T_seg / el, unit="tokens/s", cores=oracle.num_threads(),
-                kind="oracle", seconds=el,
-                sample=f"whole {w.name} step (all {w.B * w.Hkv} (batch, kv-head) units) "
-                       f"x {reps} repetitions, float64, OpenMP",
-                cpu=_cpu_model())
+    out = dict(value=reps * w.B * w.T_seg / el, unit="tokens/s", cores=oracle.num_threads(),
+               kind="oracle", seconds=el,
+               sample=f"whole {w.name} step (all {w.B * w.Hkv} (batch, kv-head) units) "
+                      f"x {reps} repetitions, float64, OpenMP",
+               cpu=_cpu_model())
+    if one_thread:
+        G, units = w.Hq // w.Hkv, w.B * w.Hkv
+        x1 = {k: np.ascontiguousarray(v[:1, :G] if k in ("Q", "dO") else v[:1, :1]) for k, v in x.items()}
+        d1 = oracle.Dims(B=1, Hq=G, Hkv=1, d=w.d, T_hist=w.T_hist, T_seg=w.T_seg, k_c=w.k_c, k_g=w.k_g)
+        n0 = oracle.num_threads()
+        oracle.set_num_threads(1)
+        try:
+            csum1, gsum1 = oracle.build_summaries(d1, x1["K"], 0, w.T_hist)
+            reps1, t1 = 0, time.perf_counter()
+            while True:
+                c, g = oracle.build_summaries(d1, x1["K"], w.T_hist, w.T, csum1, gsum1)
+                qbar = oracle.block_query(d1, x1["Q"])
+                cidx, _ = oracle.route_chunks(d1, qbar, c)
+                gidx, _ = oracle.route_groups(d1, qbar, g, cidx)
+                oracle.attn_fwd(d1, x1["Q"], x1["K"], x1["V"], gidx)
+                if w.backward:
+                    oracle.attn_bwd(d1, x1["Q"], x1["K"], x1["V"], x1["dO"], gidx)
+                reps1 += 1
+                el1 = time.perf_counter() - t1
+                if el1 >= min_seconds / 4 or reps1 >= max_reps:
+                    break
+        finally:
+            oracle.set_num_threads(n0)
+        out["one_thread"] = dict(value=reps1 * w.B * w.T_seg / (el1 * units), unit="tokens/s", cores=1,
+                                 seconds=el1,
+                                 sample=f"one (batch, kv-head) unit of {w.name} x {reps1} repetitions on one "
+                                        f"thread, scaled to the workload's {units} units")
+    return out
 
 
 def _cpu_model() -> str:
@@ -384,9 +416,20 @@ def run_gpu(args, w) -> None:
         for i in range(args.steps):
             flush.zero_()
             run_step(events[i])
+        # The same step with L2 left warm: plain replays back to back (one
+        # untimed replay first), events around each.
+        warm = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+        run_plain()
+        for a, b in warm:
+            a.record(stream)
+            run_plain()
+            b.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    warm_ms = [a.elapsed_time(b) for a, b in warm]
+    warm_total = max_over_ranks(sum(warm_ms), dev)
     per_stage = {s: [] for s in stages}
     staged_totals = []
     for ev in events:
@@ -522,14 +565,18 @@ def run_gpu(args, w) -> None:
                     warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype=w.dtype, data="synthetic",
                     config=config_of(w, not args.no_graph), stage_ms=stage_ms,
-                    ms_per_step_with_stage_events=staged_ms / args.steps, roofline=roof,
+                    ms_per_step_with_stage_events=staged_ms / args.steps,
+                    ms_per_step_median=statistics.median(totals),
+                    l2_warm=dict(ms_per_step=warm_total / args.steps, ms_median=statistics.median(warm_ms),
+                                 note="the same graph replayed back to back, L2 not flushed between steps"),
+                    roofline=roof,
                     stage_roofline=stage_roof,
                     gpu_launches=(LAUNCHES_FWD + (LAUNCHES_BWD if w.backward else 0)) * args.steps,
                     e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d,
                              d2h_bytes_per_step=d2h, mode=e2e_mode),
                     clocks=clk.summary())
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = oracle_step_rate(w, min_seconds=args.ref_seconds)
+            line["cpu_baseline"] = oracle_step_rate(w, min_seconds=args.ref_seconds, one_thread=True)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
