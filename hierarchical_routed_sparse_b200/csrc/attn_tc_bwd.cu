@@ -716,6 +716,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 // 14 items a CTA: 2-7 % on the backward), so sched is then the identity.
 constexpr int kCostClasses = 64;
 constexpr int kDealRounds = 4;
+constexpr int kMaxDealItems = 1024;
 
 struct SchedArgs {
     const int32_t* gidx;
@@ -759,6 +760,10 @@ __device__ void build_schedule(const SchedArgs& sa)
 {
     __shared__ int hist[kCostClasses], next[kCostClasses];
     __shared__ int wcnt[8][kCostClasses];
+    // Cost classes of the first kMaxDealItems items, read from the index
+    // rows once (the deal runs for at most kDealRounds items a CTA: 592
+    // items on 148 SMs); classes past it are recomputed.
+    __shared__ uint8_t cls[kMaxDealItems];
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int64_t n = sa.n_items;
     if ((n + sa.G - 1) / sa.G > kDealRounds) {
@@ -767,7 +772,11 @@ __device__ void build_schedule(const SchedArgs& sa)
     }
     for (int c = tid; c < kCostClasses; c += 256) hist[c] = 0;
     __syncthreads();
-    for (int64_t i = tid; i < n; i += 256) atomicAdd(&hist[item_cost(sa, i)], 1);
+    for (int64_t i = tid; i < n; i += 256) {
+        const int c = item_cost(sa, i);
+        if (i < kMaxDealItems) cls[i] = uint8_t(c);
+        atomicAdd(&hist[c], 1);
+    }
     __syncthreads();
     // next[c] = items of classes above c (heaviest first): lane L sums
     // classes 2L and 2L + 1, a suffix scan over the lanes does the rest.
@@ -788,7 +797,7 @@ __device__ void build_schedule(const SchedArgs& sa)
     const uint32_t lt = (1u << lane) - 1u;
     for (int64_t base = 0; base < n; base += 256) {
         const int64_t i = base + tid;
-        const int c = i < n ? item_cost(sa, i) : -1;
+        const int c = i >= n ? -1 : i < kMaxDealItems ? int(cls[i]) : item_cost(sa, i);
         for (int j = tid; j < 8 * kCostClasses; j += 256) (&wcnt[0][0])[j] = 0;
         __syncthreads();
         const uint32_t peers = __match_any_sync(0xFFFFFFFFu, c);
