@@ -237,6 +237,19 @@ def test_hand_worked_example(oracle_mod):
         den = 2 * a + (i + 1)
         np.testing.assert_allclose(O[0, 0, i], [a / den, a / den], rtol=1e-14)
         assert lse[0, 0, i] == pytest.approx(math.log(den), rel=1e-14)
+    # Backward closed forms of the fixture's backward derivation (dO_i = (1, 0)).
+    dO = np.array(ex["dO"], dtype=np.float64)[None, None]
+    dQ, dK, dV = oracle_mod.attn_bwd(dims, Q, K, V, dO, r["gidx"])
+    s = 1.0 / math.sqrt(2.0)
+    Z = [2 * a + (i + 1) for i in range(4)]
+    for i in range(4):
+        np.testing.assert_allclose(dQ[0, 0, i], [0.0, s * 2 * (a / Z[i]) * (1 - 2 * a / Z[i])],
+                                   rtol=1e-13, atol=1e-15)
+    for m in range(4):
+        k_m = -s * sum(a / Z[i] ** 2 for i in range(m, 4))
+        v_m = sum(1.0 / Z[i] for i in range(m, 4))
+        np.testing.assert_allclose(dK[0, 0, m], [k_m, k_m], rtol=1e-13)
+        np.testing.assert_allclose(dV[0, 0, m], [v_m, 0.0], rtol=1e-13, atol=1e-15)
 
 
 # ----------------------------------------------------- attention forward --
