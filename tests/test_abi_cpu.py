@@ -95,6 +95,12 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert lib.hga_attn_bwd(ctypes.byref(p), P, P, P, P, P, P, P, P, P, P, P, 16, None) == \
         hga.HGA_ERR_INVALID_ARG
     assert "workspace" in lib.hga_last_error().decode()
+    # The row sums alone (B*Hq*T_seg floats) are not enough: the workspace
+    # also holds the backward's item schedule.
+    rows_only = 4 * 32 * 2048
+    assert lib.hga_attn_bwd(ctypes.byref(p), P, P, P, P, P, P, P, P, P, P, P, rows_only, None) == \
+        hga.HGA_ERR_INVALID_ARG
+    assert str(hga.workspace_size(_p())) in lib.hga_last_error().decode()
 
 
 def test_empty_segment_is_a_no_op(lib):
