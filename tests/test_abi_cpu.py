@@ -200,3 +200,38 @@ def test_causal_calls_reject_bad_arguments_on_the_host(lib):
     # An empty segment is a no-op.
     p0 = _p(T_seg=0).c()
     assert lib.hga_attn_fwd_causal(ctypes.byref(p0), *([None] * 6), None) == hga.HGA_OK
+
+@pytest.mark.parametrize("compiler,suffix", [("gcc", ".c"), ("g++", ".cpp")])
+def test_plain_c_and_cpp_callers_link_and_call(lib, tmp_path, compiler, suffix):
+    # A caller written against include/hga.h alone, linked to libhga.so:
+    # host-only calls (version, workspace size, validation) need no GPU.
+    import subprocess
+    libdir = os.path.dirname(hga.LIB_PATH)
+    prog = r"""
+#include <stdio.h>
+#include <string.h>
+#include "hga.h"
+int main(void) {
+    hga_params p;
+    memset(&p, 0, sizeof p);
+    p.B = 1; p.Hq = 32; p.Hkv = 8; p.d = 128; p.T_hist = 14336; p.T_seg = 2048;
+    p.chunk = 64; p.group = 8; p.qblock = 64; p.k_c = 8; p.k_g = 32; p.dtype = HGA_BF16;
+    int wc = 0, wg = 0;
+    if (hga_route_widths(&p, &wc, &wg) != HGA_OK || wc != 8 || wg != 32) return 1;
+    if (hga_workspace_size(&p) != 4u * (32u * 2048u + 8u * 32u * 2u)) return 2;
+    if (hga_attn_fwd(&p, NULL, NULL, NULL, NULL, NULL, NULL, NULL) != HGA_ERR_INVALID_ARG) return 3;
+    if (strstr(hga_last_error(), "NULL") == NULL) return 4;
+    p.d = 96;
+    if (hga_workspace_size(&p) != 0) return 5;
+    puts(hga_version());
+    return 0;
+}
+"""
+    src = tmp_path / ("caller" + suffix)
+    src.write_text(prog)
+    exe = tmp_path / "caller"
+    subprocess.run([compiler, "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-L", libdir,
+                    "-lhga", "-Wl,-rpath," + libdir, "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert "sm_100a" in r.stdout
