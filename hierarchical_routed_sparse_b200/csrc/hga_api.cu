@@ -455,8 +455,14 @@ int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* 
 // once per device with cudaGetSymbolAddress, on the first call made while
 // that device is current, and cached.
 
-// Row sums, then the item schedule (at most one item per 64 rows).
-static __device__ __align__(256) float g_noalloc_rowsum[HGA_NOALLOC_MAX_ROWS + HGA_NOALLOC_MAX_ROWS / 64];
+// Size of the built-in scratch in 4-byte words: the row sums of up to
+// HGA_NOALLOC_MAX_ROWS rows, then the backward's item schedule.  An item is
+// a query block of 64 rows of at least one q-head, so the schedule holds at
+// most one word per 64 rows; the call below checks the exact need,
+// hga::bwd_scratch_floats, against this total, so a change in how items are
+// counted cannot overrun the array.
+constexpr int64_t kNoallocWords = (int64_t)HGA_NOALLOC_MAX_ROWS + HGA_NOALLOC_MAX_ROWS / 64;
+static __device__ __align__(256) float g_noalloc_rowsum[kNoallocWords];
 
 namespace {
 
@@ -505,11 +511,12 @@ extern "C" int hga_attn_bwd_noalloc(const hga_params* p, const void* Q, const vo
     CHECK_PTR(dK_seg);
     CHECK_PTR(dV_seg);
     const int64_t rows = (int64_t)s.B * s.Hq * s.T_seg;
-    if (rows > HGA_NOALLOC_MAX_ROWS)
+    if (rows > HGA_NOALLOC_MAX_ROWS || hga::bwd_scratch_floats(s) > kNoallocWords)
         return fail(HGA_ERR_INVALID_ARG,
-                    "hga_attn_bwd_noalloc: B*Hq*T_seg = %lld exceeds its built-in scratch of %d rows; "
-                    "use hga_attn_bwd with a caller-provided workspace", (long long)rows,
-                    HGA_NOALLOC_MAX_ROWS);
+                    "hga_attn_bwd_noalloc: B*Hq*T_seg = %lld (%lld scratch words) exceeds its built-in "
+                    "scratch of %d rows (%lld words); use hga_attn_bwd with a caller-provided workspace",
+                    (long long)rows, (long long)hga::bwd_scratch_floats(s), HGA_NOALLOC_MAX_ROWS,
+                    (long long)kNoallocWords);
     if (!hga::attn_bwd_tc_supported(s) && hga::attn_simt_smem(s, true) > kMaxSmem)
         return fail(HGA_ERR_UNSUPPORTED, "k_g=%d too large for the attention kernel", s.wg);
     float* scratch = nullptr;

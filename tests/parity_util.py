@@ -15,6 +15,8 @@ resolves the other way cannot leak into the attention comparison.
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 import torch
 
@@ -49,22 +51,139 @@ def unit_slice(w, x: dict, b: int, g: int) -> tuple:
     return w.with_(B=1, Hq=G, Hkv=1), sl
 
 
+def _format_ok(got: np.ndarray, what: str) -> None:
+    """Every row ascending, unique and -1 padded."""
+    for row in got.reshape(-1, got.shape[-1]):
+        v = row[row >= 0]
+        n = len(v)
+        assert (row[n:] == -1).all() and (np.diff(v) > 0).all(), f"{what}: malformed row {row}"
+
+
 def check_indices(got: np.ndarray, want: np.ndarray, gap: np.ndarray, what: str) -> int:
     """Exact equality except on rows whose oracle gap is below the exemption.
 
-    Returns the number of exempt rows that differ.
+    Only the format of an exempt row is checked here; check_routing also
+    proves that such a row is a valid top-k.  Returns the number of exempt
+    rows that differ.
     """
     diff = (got != want).any(axis=-1)
     bad = diff & ~(gap < GAP_EXEMPT)
     assert not bad.any(), (f"{what}: {int(bad.sum())} rows differ outside the gap exemption; "
                            f"first at {np.argwhere(bad)[0].tolist()}: gpu {got[bad][0].tolist()} "
                            f"oracle {want[bad][0].tolist()} gap {gap[bad][0]}")
-    # Every row, exempt or not, must still be ascending, unique and -1 padded.
-    for row in got.reshape(-1, got.shape[-1]):
-        v = row[row >= 0]
-        n = len(v)
-        assert (row[n:] == -1).all() and (np.diff(v) > 0).all(), f"{what}: malformed row {row}"
+    _format_ok(got, what)
     return int((diff & (gap < GAP_EXEMPT)).sum())
+
+
+def _band(s: np.ndarray, cand: np.ndarray, k: int):
+    """For candidate scores s (float64) and a requested k (<= 0: all): the
+    kept count, the reference top set (score descending, lower index first
+    on ties), the k-th and (k+1)-th scores and the relative gap's
+    denominator max(|s_k|, |s_k+1|, 1e-3 rms(s))."""
+    n = len(cand)
+    keep = n if (k <= 0 or k > n) else k
+    order = np.lexsort((cand, -s))
+    ref = np.sort(cand[order[:keep]])
+    if keep == 0 or keep >= n:
+        return keep, ref, None, None, None
+    a, b = float(s[order[keep - 1]]), float(s[order[keep]])
+    den = max(abs(a), abs(b), 1e-3 * math.sqrt(float(np.mean(s * s))))
+    return keep, ref, a, b, den
+
+
+def _valid_topk(row: np.ndarray, cand: np.ndarray, s: np.ndarray, k: int, what: str, where) -> bool:
+    """Assert that `row` is one of the valid answers of a top-k among
+    `cand` with scores `s`: it holds min(k, n) candidates, and every pick
+    and every dropped reference pick lies within 1e-4 (relative, reading R8)
+    of the boundary between the k-th and (k+1)-th scores.  Returns whether
+    the row equals the reference top set exactly."""
+    v = row[row >= 0]
+    keep, ref, a, b, den = _band(s, cand, k)
+    assert len(v) == keep, f"{what} {where}: {len(v)} entries, want min(k, eligible) = {keep}"
+    pos = {int(c): i for i, c in enumerate(cand)}
+    assert all(int(c) in pos for c in v), f"{what} {where}: {v.tolist()} not all eligible"
+    if np.array_equal(v, ref):
+        return True
+    assert a is not None, f"{what} {where}: every candidate kept, yet the row differs"
+    gap = (a - b) / den if den > 0 else 0.0
+    assert gap < GAP_EXEMPT, f"{what} {where}: differs from the top set outside the gap ({gap:.3g})"
+    eps = GAP_EXEMPT * den
+    picked = np.array([s[pos[int(c)]] for c in v])
+    assert picked.min() >= a - eps, f"{what} {where}: a pick scores {picked.min()} < s_k {a} - eps"
+    dropped = np.setdiff1d(ref, v)
+    if len(dropped):
+        ds = np.array([s[pos[int(c)]] for c in dropped])
+        assert ds.max() <= b + eps, f"{what} {where}: dropped {ds.max()} > s_k+1 {b} + eps"
+    return False
+
+
+def check_routing(got_c: np.ndarray, got_g: np.ndarray, q: np.ndarray, unit: np.ndarray,
+                  csum: np.ndarray, gsum: np.ndarray, n_elig: np.ndarray, k_c: int, k_g: int,
+                  what: str,
+                  want_c: np.ndarray, cgap: np.ndarray, want_g: np.ndarray | None = None,
+                  ggap: np.ndarray | None = None) -> dict:
+    """Routing rows of the GPU against the oracle, under the index gate.
+
+    Rows are flattened: got_c [N, wc], got_g [N, wg]; q [N, d] the row's
+    block query (float64, the oracle's); unit [N] the row's flat (batch,
+    kv-head) index into csum [U, nC, d] and gsum [U, nG, d]; n_elig [N] the
+    eligible chunk count (the own chunk's index).
+    A chunk row equals the oracle's exactly, or the oracle's gap is below
+    1e-4 and the row is a valid top-k_c of the eligible chunks (count, range,
+    scores within the tie band).  A group row is judged against the top-k_g
+    of the groups of the GPU's OWN chunk row: want_g / ggap when given (the
+    oracle's group routing run on the GPU's chunk rows), else recomputed
+    from the scores.  Returns the counts of differing (exempt) rows.
+    """
+    N = got_c.shape[0]
+    got_c, got_g = got_c.reshape(N, -1), got_g.reshape(N, -1)
+    want_c, cgap = want_c.reshape(N, -1), cgap.reshape(N)
+    _format_ok(got_c, what + " cidx")
+    _format_ok(got_g, what + " gidx")
+    gpc = 8
+    out = {"cidx_exempt_rows": 0, "gidx_exempt_rows": 0}
+    for i in range(N):
+        crow = got_c[i][got_c[i] >= 0]
+        if not np.array_equal(got_c[i], want_c[i]):
+            assert cgap[i] < GAP_EXEMPT, (f"{what} cidx row {i}: gpu {got_c[i].tolist()} oracle "
+                                          f"{want_c[i].tolist()} gap {cgap[i]}")
+            cand = np.arange(int(n_elig[i]))
+            s = csum[unit[i]][:len(cand)] @ q[i]
+            _valid_topk(crow, cand, s, k_c, what + " cidx", i)
+            out["cidx_exempt_rows"] += 1
+        if want_g is not None and np.array_equal(got_g[i], want_g.reshape(N, -1)[i]):
+            continue
+        if want_g is not None:
+            assert ggap.reshape(N)[i] < GAP_EXEMPT, (
+                f"{what} gidx row {i}: gpu {got_g[i].tolist()} oracle "
+                f"{want_g.reshape(N, -1)[i].tolist()} gap {ggap.reshape(N)[i]}")
+        gcand = (crow[:, None] * gpc + np.arange(gpc)[None, :]).reshape(-1)
+        s = gsum[unit[i]][gcand] @ q[i]
+        grow = got_g[i][got_g[i] >= 0]
+        if not _valid_topk(grow, gcand, s, k_g, what + " gidx", i):
+            out["gidx_exempt_rows"] += 1
+    return out
+
+
+def block_rows(w, orc: dict, gpu_cidx: np.ndarray):
+    """Flattened routing rows of the block path: for every (batch, kv-head,
+    query block) the oracle's block query, its summaries and eligible chunk
+    count, plus the oracle's group routing run on the GPU's chunk rows."""
+    nQB = w.T_seg // 64
+    N = w.B * w.Hkv * nQB
+    q = orc["qbar"].reshape(N, w.d)
+    unit = np.repeat(np.arange(w.B * w.Hkv), nQB)
+    csum = orc["csum"].reshape(w.B * w.Hkv, -1, w.d)
+    gsum = orc["gsum"].reshape(w.B * w.Hkv, -1, w.d)
+    n_elig = np.tile(w.T_hist // 64 + np.arange(nQB), w.B * w.Hkv)
+    want_g, ggap = oracle.route_groups(dims_of(w), orc["qbar"], orc["gsum"], gpu_cidx)
+    return q, unit, csum, gsum, n_elig, want_g, ggap
+
+
+def check_block_routing(w, gpu_cidx: np.ndarray, gpu_gidx: np.ndarray, orc: dict) -> dict:
+    q, unit, csum, gsum, n_elig, want_g, ggap = block_rows(w, orc, gpu_cidx)
+    return check_routing(gpu_cidx, gpu_gidx, q, unit, csum, gsum, n_elig, w.k_c, w.k_g, w.name,
+                         orc["cidx"], orc["cgap"], want_g, ggap)
 
 
 def maxabs(a, b) -> float:
@@ -119,14 +238,36 @@ def compare_all(w, gpu: dict, orc: dict, gpu_routed: dict | None = None) -> dict
     errs["gsum"] = maxabs(gpu["gsum"], orc["gsum"])
     errs["qbar"] = maxabs(gpu["qbar"], orc["qbar"])
     assert errs["csum"] < 1e-5 and errs["gsum"] < 1e-5 and errs["qbar"] < 1e-5, errs
-    errs["cidx_exempt_rows"] = check_indices(gpu["cidx"], orc["cidx"], orc["cgap"], "cidx")
-    # Group routing is compared on the rows whose chunk choice agrees (a
-    # different, exempt chunk choice gives different candidates).
-    same_c = (gpu["cidx"] == orc["cidx"]).all(axis=-1)
-    ggap = np.where(same_c, orc["ggap"], 0.0)
-    errs["gidx_exempt_rows"] = check_indices(gpu["gidx"], orc["gidx"], ggap, "gidx")
+    errs.update(check_block_routing(w, gpu["cidx"], gpu["gidx"], orc))
     for k in ("O", "lse", "dQ", "dK", "dV"):
         if k in gpu:
             errs[k] = maxabs(gpu[k], orc[k])
             assert errs[k] <= tol, f"{k}: max-abs error {errs[k]:.3g} > {tol}"
     return errs
+
+
+def check_causal_routing(w, got_c: np.ndarray, got_g: np.ndarray, Q64: np.ndarray,
+                         csum: np.ndarray, gsum: np.ndarray, orc: dict) -> dict:
+    """Routing rows of the strictly causal variant (one per query position):
+    the row's query is the mean of its G q-heads' queries at that position
+    and chunks before the position's own chunk are eligible.  Group rows are
+    judged on the GPU's own chunk rows."""
+    B, Hkv, Ts, d, G = w.B, w.Hkv, w.T_seg, w.d, w.G
+    q = Q64.reshape(B, Hkv, G, Ts, d).mean(axis=2).reshape(-1, d)
+    unit = np.repeat(np.arange(B * Hkv), Ts)
+    n_elig = np.tile((w.T_hist + np.arange(Ts)) // 64, B * Hkv)
+    return check_routing(got_c, got_g, q, unit, csum.reshape(B * Hkv, -1, d),
+                         gsum.reshape(B * Hkv, -1, d), n_elig, w.k_c, w.k_g, w.name + " causal",
+                         orc["cidx"], orc["cgap"])
+
+
+def check_decode_routing(w, pos: int, got_c: np.ndarray, got_g: np.ndarray, q64: np.ndarray,
+                         csum: np.ndarray, gsum: np.ndarray, orc: dict) -> dict:
+    """Routing rows of one decode step (a block of one at position pos)."""
+    B, Hkv, d, G = w.B, w.Hkv, w.d, w.G
+    q = q64.reshape(B, Hkv, G, d).mean(axis=2).reshape(-1, d)
+    unit = np.arange(B * Hkv)
+    n_elig = np.full(B * Hkv, pos // 64)
+    return check_routing(got_c, got_g, q, unit, csum.reshape(B * Hkv, -1, d),
+                         gsum.reshape(B * Hkv, -1, d), n_elig, w.k_c, w.k_g,
+                         f"{w.name} decode@{pos}", orc["cidx"], orc["cgap"])

@@ -23,7 +23,7 @@ from hierarchical_routed_sparse_b200 import workloads as W
 from hierarchical_routed_sparse_b200.workloads import Workload
 
 import oracle
-from parity_util import GAP_EXEMPT, TOL, check_indices, dims_of, maxabs, to_dev
+from parity_util import GAP_EXEMPT, TOL, check_decode_routing, dims_of, maxabs, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -90,9 +90,7 @@ def _compare(w, x, pos, got):
     q64 = x["Q"][:, :, pos % w.T_seg].astype(np.float64)
     csum, gsum = oracle.build_summaries(dims, K64)
     orc = oracle.decode(dims, pos, q64, K64, V64, csum, gsum)
-    check_indices(got["cidx"], orc["cidx"], orc["cgap"], "cidx")
-    same_c = (got["cidx"] == orc["cidx"]).all(axis=-1)
-    check_indices(got["gidx"], orc["gidx"], np.where(same_c, orc["ggap"], 0.0), "gidx")
+    check_decode_routing(w, pos, got["cidx"], got["gidx"], q64, csum, gsum, orc)
     tol = TOL[w.dtype]
     G, scale = w.G, 1.0 / math.sqrt(w.d)
     for b in range(w.B):
@@ -166,7 +164,7 @@ def test_generation_appends_summaries():
         orc = oracle.decode(dims, pos, q64, K64, V64, csum, gsum)
         cg = st.cidx.cpu().numpy()
         gg = st.gidx.cpu().numpy()
-        check_indices(cg, orc["cidx"], orc["cgap"], "cidx")
+        check_decode_routing(w, pos, cg, gg, q64, csum, gsum, orc)
         if np.array_equal(gg, orc["gidx"]):
             assert maxabs(O, orc["O"]) <= TOL[w.dtype], pos
     assert st.pos == n0 + 120

@@ -15,8 +15,8 @@ import hierarchical_routed_sparse_b200 as hga
 from hierarchical_routed_sparse_b200 import workloads as W
 from hierarchical_routed_sparse_b200.workloads import Workload
 
-from parity_util import (compare_all, f64, maxabs, run_gpu, run_oracle, to_dev, unit_slice,
-                         TOL)
+from parity_util import (check_block_routing, compare_all, f64, maxabs, run_gpu, run_oracle,
+                         to_dev, unit_slice, TOL)
 
 pytestmark = pytest.mark.gpu
 
@@ -164,11 +164,8 @@ def test_sweep_sampled_units(w):
         orc = run_oracle(wu, f64(xu), backward=True)
         G = w.G
         got_c = buf.cidx[b:b + 1, g:g + 1].cpu().numpy()
-        from parity_util import check_indices
-        check_indices(got_c, orc["cidx"], orc["cgap"], "cidx")
-        same_c = (got_c == orc["cidx"]).all(axis=-1)
         got_g = buf.gidx[b:b + 1, g:g + 1].cpu().numpy()
-        check_indices(got_g, orc["gidx"], np.where(same_c, orc["ggap"], 0.0), "gidx")
+        check_block_routing(wu, got_c, got_g, orc)
         # Attention with the oracle's routing, on this unit only.
         pu = hga.Params.from_workload(wu)
         bu = hga.Buffers(pu)
@@ -201,3 +198,51 @@ def test_fused_router_equals_separate_calls(w):
     assert torch.equal(a.qbar, b.qbar)
     assert torch.equal(a.cidx, b.cidx)
     assert torch.equal(a.gidx, b.gidx)
+
+
+# ---- whole-problem launches whose backward deals items round-robin --------------
+# The persistent backward ranks items by cost only when a CTA takes at most 4
+# of them; beyond that it deals them round-robin, and beyond 64 items a CTA
+# it reads its items from global memory instead of its prologue table.  The
+# gradients of those very launches are checked here on sampled (batch,
+# kv-head) units against the oracle's backward fed the launch's own routing
+# (once that routing has passed the index gate).
+ROUND_ROBIN = [
+    W.sweep_point(32768, 16, 64),                                         # 2048 items, 14 a CTA
+    Workload("bwd_items_beyond_table", B=10, Hq=32, Hkv=8, d=128, T_hist=0, T_seg=4096, k_c=8,
+             k_g=32, keys="clustered", backward=True, seed=51),           # 10240 items, 70 a CTA
+]
+
+
+@pytest.mark.parametrize("w", ROUND_ROBIN, ids=lambda w: w.name)
+def test_round_robin_backward_whole_launch(w):
+    import oracle
+    from parity_util import dims_of
+    n_items = w.B * w.Hkv * (w.T_seg // 64) * ((w.G + 1) // 2)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert n_items > 4 * sms
+    x = w.full()
+    p = hga.Params.from_workload(w)
+    buf = hga.Buffers(p)
+    Q, K, V, dO = (to_dev(x[k], "bf16") for k in ("Q", "K", "V", "dO"))
+    buf.summaries(K, 0, w.T)
+    buf.step(Q, K, V, dO)                       # routing, forward, backward: one problem
+    torch.cuda.synchronize()
+    assert hga.device_status() == 0
+    units = [(0, 0), (w.B // 2, 3), (w.B - 1, w.Hkv - 1)]
+    for (b, g) in units:
+        wu, xu = unit_slice(w, x, b, g)
+        x64 = f64(xu)
+        dims = dims_of(wu)
+        orc = oracle.route(dims, x64["Q"], x64["K"])
+        got_c = buf.cidx[b:b + 1, g:g + 1].cpu().numpy()
+        got_g = buf.gidx[b:b + 1, g:g + 1].cpu().numpy()
+        check_block_routing(wu, got_c, got_g, orc)
+        O, lse = oracle.attn_fwd(dims, x64["Q"], x64["K"], x64["V"], got_g)
+        dQ, dK, dV = oracle.attn_bwd(dims, x64["Q"], x64["K"], x64["V"], x64["dO"], got_g)
+        hs = slice(g * w.G, (g + 1) * w.G)
+        for k, got, want in (("O", buf.O[b:b + 1, hs], O), ("lse", buf.lse[b:b + 1, hs], lse),
+                             ("dQ", buf.dQ[b:b + 1, hs], dQ), ("dK", buf.dK[b:b + 1, g:g + 1], dK),
+                             ("dV", buf.dV[b:b + 1, g:g + 1], dV)):
+            err = maxabs(got.cpu().numpy(), want)
+            assert err <= TOL["bf16"], (w.name, b, g, k, err)

@@ -214,6 +214,42 @@ def test_routing_gap_definition(oracle_mod):
     assert math.isinf(oracle_mod.route(dims, Q, K)["cgap"][0, 0, 0])
 
 
+def test_routing_gap_floor_decides_near_zero_scores(oracle_mod):
+    # Chunk scores 10, 2e-6, 1e-6, -30 with k_c 2: the k-th and (k+1)-th
+    # scores are near zero, so the floor tau = 1e-3 * rms of ALL four
+    # eligible scores sets the denominator:
+    #   rms = sqrt((100 + 4e-12 + 1e-12 + 900) / 4) = sqrt(250.00000000000125)
+    #   gap = (2e-6 - 1e-6) / (1e-3 * rms) = 6.32455532e-5  (exempt: < 1e-4).
+    # Plausible slips give other values: no floor -> 0.5; rms over the kept
+    # scores only -> 1.414e-4 (not exempt); no square root -> 4e-6; a floor
+    # factor of 1e-4 -> 6.3e-4.
+    K = np.zeros((1, 1, 5 * 64, 4))
+    for c, s in enumerate([10.0, 2e-6, 1e-6, -30.0]):
+        K[0, 0, 64 * c:64 * c + 64, 0] = s
+    Q = np.zeros((1, 1, 64, 4))
+    Q[..., 0] = 1.0
+    dims = oracle_mod.Dims(B=1, Hq=1, Hkv=1, d=4, T_hist=256, T_seg=64, k_c=2, k_g=1)
+    r = oracle_mod.route(dims, Q, K)
+    assert list(r["cidx"][0, 0, 0]) == [0, 1]
+    want = 1e-6 / (1e-3 * math.sqrt((100.0 + 4e-12 + 1e-12 + 900.0) / 4.0))
+    assert want == pytest.approx(6.32455532e-5, rel=1e-8)
+    assert r["cgap"][0, 0, 0] == pytest.approx(want, rel=1e-6)
+    assert r["cgap"][0, 0, 0] < 1e-4
+    # The same floor at group level: the one eligible chunk's eight groups
+    # score 10, 2e-6, 1e-6, -30, 0, 0, 0, 0 (k_g 2); rms over the eight
+    # candidates is sqrt(1000 / 8) = sqrt(125), so the gap is
+    # 1e-6 / (1e-3 * sqrt(125)) = 8.94427191e-5.
+    K = np.zeros((1, 1, 128, 4))
+    for j, s in enumerate([10.0, 2e-6, 1e-6, -30.0, 0.0, 0.0, 0.0, 0.0]):
+        K[0, 0, 8 * j:8 * j + 8, 0] = s
+    dims = oracle_mod.Dims(B=1, Hq=1, Hkv=1, d=4, T_hist=64, T_seg=64, k_c=1, k_g=2)
+    r = oracle_mod.route(dims, Q, K)
+    assert list(r["gidx"][0, 0, 0]) == [0, 1]
+    want = 1e-6 / (1e-3 * math.sqrt((100.0 + 4e-12 + 1e-12 + 900.0) / 8.0))
+    assert want == pytest.approx(8.94427191e-5, rel=1e-8)
+    assert r["ggap"][0, 0, 0] == pytest.approx(want, rel=1e-6)
+
+
 def test_hand_worked_example(oracle_mod):
     """Tiny example worked by hand (chunk 4, group 2, d 2); see the fixture."""
     with open(os.path.join(GOLDEN, "hand_worked_example.json")) as f:

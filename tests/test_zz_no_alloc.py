@@ -6,7 +6,10 @@ hosts whose memory pool owns all device memory, loops that must not call
 cudaMalloc / cudaFree).  It keeps its scratch in a fixed array inside the
 library.  Its results must match the workspace entry point's within the
 parity tolerance, call after call: the array keeps the previous call's
-contents, and two calls in a row must not see each other.
+contents, so between the two compared calls another problem (a different
+upstream gradient, then another head layout whose item schedule sits at a
+different offset) leaves different row sums and a different schedule in it,
+and the second call must overwrite every entry it reads.
 
 The file name sorts last so that a run stopping at the first failure has
 already run every other test.
@@ -43,7 +46,27 @@ CASES = [
     Workload("noalloc_fp32_d64", B=1, Hq=4, Hkv=2, d=64, T_hist=256, T_seg=256, k_c=2, k_g=9,
              dtype="fp32", backward=True, seed=22),
     W.QWEN3_CTX16K_TRAIN,
+    # 2048 backward items, 14 a CTA: the round-robin schedule (262144 rows)
+    Workload("noalloc_round_robin", B=2, Hq=32, Hkv=8, d=128, T_hist=2048, T_seg=4096, k_c=4,
+             k_g=16, keys="clustered", backward=True, seed=23),
 ]
+
+# The problem run between the two compared calls: G = 3 (a pair with one
+# head) and another row count, so its row sums and schedule land elsewhere.
+OTHER = Workload("noalloc_other", B=1, Hq=6, Hkv=2, d=128, T_hist=1024, T_seg=640, k_c=4, k_g=17,
+                 keys="clustered", backward=True, seed=24)
+
+
+def _other_problem_call():
+    x = OTHER.full()
+    p = hga.Params.from_workload(OTHER)
+    Q, K, V, dO = (_dev(x[k], OTHER.dtype) for k in ("Q", "K", "V", "dO"))
+    b = hga.Buffers(p)
+    b.summaries(K, 0, OTHER.T)
+    b.route(Q)
+    b.forward(Q, K, V)
+    hga.attn_bwd_noalloc(p, Q, K, V, b.O, b.lse, dO, b.gidx, b.dQ, b.dK, b.dV)
+    torch.cuda.synchronize()
 
 
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
@@ -59,6 +82,12 @@ def test_noalloc_matches_workspace_backward_twice(w):
     torch.cuda.synchronize()
     ref = [t.cpu().numpy() for t in (buf.dQ, buf.dK, buf.dV)]
     for call in range(2):
+        if call == 1:
+            # Same problem, another dO: different row sums in the same slots.
+            dO2 = _dev(np.ascontiguousarray(x["dO"][..., ::-1]), w.dtype)
+            junk = [torch.empty_like(t) for t in (buf.dQ, buf.dK, buf.dV)]
+            hga.attn_bwd_noalloc(p, Q, K, V, buf.O, buf.lse, dO2, buf.gidx, *junk)
+            _other_problem_call()
         outs = [torch.full_like(t, float("nan")) for t in (buf.dQ, buf.dK, buf.dV)]
         hga.attn_bwd_noalloc(p, Q, K, V, buf.O, buf.lse, dO, buf.gidx, *outs)
         torch.cuda.synchronize()
