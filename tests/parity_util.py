@@ -135,7 +135,7 @@ def check_routing(got_c: np.ndarray, got_g: np.ndarray, q: np.ndarray, unit: np.
     oracle's group routing run on the GPU's chunk rows), else recomputed
     from the scores.  Returns the counts of differing (exempt) rows.
     """
-    N = got_c.shape[0]
+    N = int(np.prod(got_c.shape[:-1]))
     got_c, got_g = got_c.reshape(N, -1), got_g.reshape(N, -1)
     want_c, cgap = want_c.reshape(N, -1), cgap.reshape(N)
     _format_ok(got_c, what + " cidx")

@@ -117,3 +117,21 @@ def test_decode_rows(oracle_mod):
     bad[0, 0] = [0, 3]
     with pytest.raises(AssertionError):
         check_decode_routing(wd, 300, bad, orc["gidx"], q, csum, gsum, orc)
+
+
+def test_many_rows_of_real_workloads(oracle_mod):
+    # The oracle's own routing of multi-row problems passes as it stands
+    # (block path and strictly causal path); one planted row fails.
+    from parity_util import check_causal_routing, dims_of
+    w = Workload("rows", B=2, Hq=4, Hkv=2, d=16, T_hist=256, T_seg=256, k_c=2, k_g=5,
+                 dtype="fp32", keys="clustered", seed=3)
+    x = {k: v.astype(np.float64) for k, v in w.full().items()}
+    dims = dims_of(w)
+    orc = oracle_mod.route(dims, x["Q"], x["K"])
+    check_block_routing(w, orc["cidx"], orc["gidx"], orc)
+    rc = oracle_mod.causal_route(dims, x["Q"], orc["csum"], orc["gsum"])
+    check_causal_routing(w, rc["cidx"], rc["gidx"], x["Q"], orc["csum"], orc["gsum"], rc)
+    bad = rc["gidx"].copy()
+    bad[1, 1, 200, 0] = bad[1, 1, 200, 1]                  # a duplicate: malformed
+    with pytest.raises(AssertionError):
+        check_causal_routing(w, rc["cidx"], bad, x["Q"], orc["csum"], orc["gsum"], rc)
