@@ -29,11 +29,17 @@
 // it: two 64 KB buffers swap the Q/dO and P/dS roles from item to item, and
 // the next item's S/dP products start while this item's history tiles run.
 //
-// Warp roles (576 threads): warps 0-15 compute P and dS (row 32*(w%4)+lane,
+// Warp roles (608 threads): warps 0-15 compute P and dS (row 32*(w%4)+lane,
 // 16-key quarter w/4), add a segment tile's dK/dV while the next tile's MMAs
 // run and write dQ at the end of an item; warp 16 loads Q / dO and the K/V
-// tiles (TMA gathers of 8-row groups), warp 17 owns tensor memory and issues
-// the MMAs.  Tensor memory (512 columns): S and dP
+// tiles (TMA gathers of 8-row groups); warp 17 owns tensor memory and issues
+// the gradient MMAs (dQ, dV^T, dK^T); warp 18 issues S / dP.  A single
+// issuing thread serialised the two streams: each tcgen05.mma takes it
+// 70-90 cycles to issue, and its waits (the compute warps' hand-off, the
+// next tile's K / V) delayed everything queued behind them.  With two
+// issuers, S / dP of tile t + 2 go out as soon as its operands have landed
+// and dQ of tile t, which reads dS from the same tensor-memory buffer, has
+// completed (an mbarrier the gradient issuer commits).  Tensor memory (512 columns): S and dP
 // double-buffered (4 x 64), dQ (128), dV^T (64), dK^T (64).  K and V load
 // into separate rings: four K stages (K is read by S, two tiles ahead, and
 // by dQ) and two V stages (V is read by dP only and released as S / dP
@@ -56,13 +62,13 @@ constexpr int kVStages = 2;            // V only by dP: released as S / dP compl
 constexpr int kKeys = 64;
 constexpr int kComputeWarps = 16;     // 4 per lane quadrant, one 16-key quarter each
 constexpr int kCompute = 32 * kComputeWarps;
-constexpr int kProducerWarp = kComputeWarps, kMmaWarp = kComputeWarps + 1;
-constexpr int kThreads = 32 * (kComputeWarps + 2);
+constexpr int kProducerWarp = kComputeWarps, kMmaWarp = kComputeWarps + 1, kSdpWarp = kComputeWarps + 2;
+constexpr int kThreads = 32 * (kComputeWarps + 3);
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int {
     kSiteQ = 201, kSiteFull, kSiteEmpty, kSiteSdp, kSitePs, kSiteKv, kSiteDrained, kSiteFinal, kSiteDrain,
-    kSiteQfree, kSiteDqfree, kSitePfree, kSiteDqs
+    kSiteQfree, kSiteDqfree, kSitePfree, kSiteDqs, kSiteSfree, kSiteFinalSdp
 };
 
 struct BwdSmem {
@@ -75,22 +81,24 @@ struct BwdSmem {
     static constexpr int k_off = x_off + 2 * kX;
     static constexpr int v_off = k_off + kKStages * H * kKVHalf;
     static constexpr int bar_off = v_off + kVStages * H * kKVHalf;
-    static constexpr int n_bars = 26;
-    static constexpr int tab_off = bar_off + 8 * n_bars;       // (item, n_g, n_seg) of the CTA's first items
+    static constexpr int n_bars = 29;
+    static constexpr int tab_off = (bar_off + 8 * n_bars + 15) & ~15;   // int4 (item, n_g, n_seg) of the CTA's first items
     static constexpr int tmem_slot_off = tab_off + 16 * 64;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;
 };
 static_assert(BwdSmem::alloc <= 227 * 1024, "shared memory");
+static_assert(BwdSmem::tab_off % 16 == 0 && BwdSmem::bar_off % 8 == 0, "int4 table and mbarrier alignment");
 
 // mbarriers: q[2], kfull / kempty[kKStages], vfull / vempty[kVStages], sdp[2],
-// ps[2], kv, drained, pfree, qfree, dqfree, final, dqs_full, dqs_free.
+// ps[2], kv, drained, pfree, qfree, dqfree, final, dqs_full, dqs_free, sfree[2],
+// final_sdp.
 constexpr int kBarQ = 0, kBarKFull = 2, kBarKEmpty = kBarKFull + kKStages, kBarVFull = kBarKEmpty + kKStages,
               kBarVEmpty = kBarVFull + kVStages, kBarSdp = kBarVEmpty + kVStages, kBarPs = kBarSdp + 2,
               kBarKv = kBarPs + 2, kBarDrained = kBarKv + 1, kBarPfree = kBarKv + 2, kBarQfree = kBarKv + 3,
               kBarDqfree = kBarKv + 4, kBarFinal = kBarKv + 5, kBarDqsFull = kBarKv + 6,
-              kBarDqsFree = kBarKv + 7;
-static_assert(kBarDqsFree + 1 == BwdSmem::n_bars, "barrier count");
+              kBarDqsFree = kBarKv + 7, kBarSfree = kBarKv + 8, kBarFinalSdp = kBarSfree + 2;
+static_assert(kBarFinalSdp + 1 == BwdSmem::n_bars, "barrier count");
 
 // Tensor-memory columns.
 constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDV = 384, kColDK = 448;
@@ -201,6 +209,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     auto bar_vempty = [&](int s) { return bar0 + 8 * (kBarVEmpty + s); };
     auto bar_sdp = [&](int b) { return bar0 + 8 * (kBarSdp + b); };
     auto bar_ps = [&](int b) { return bar0 + 8 * (kBarPs + b); };
+    auto bar_sfree = [&](int b) { return bar0 + 8 * (kBarSfree + b); };   // dQ of the buffer's tile done
+    const uint32_t bar_final_sdp = bar0 + 8 * kBarFinalSdp;
     const uint32_t bar_kv = bar0 + 8 * kBarKv;
     const uint32_t bar_drained = bar0 + 8 * kBarDrained;
     const uint32_t bar_pfree = bar0 + 8 * kBarPfree;
@@ -222,6 +232,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(bar_q(b), 1);
             mbar_init(bar_sdp(b), 1);
             mbar_init(bar_ps(b), kCompute);
+            mbar_init(bar_sfree(b), 1);
         }
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(bar_kfull(s), 1);
@@ -239,6 +250,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_init(bar_final, 1);
         mbar_init(bar_dqs_full, kCompute);
         mbar_init(bar_dqs_free, 1);
+        mbar_init(bar_final_sdp, 1);
         fence_mbar_init();
     }
     if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
@@ -363,66 +375,62 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (last_v[j] >= 0) mbar_wait(bar_vfull(j), (last_v[j] / kVStages) & 1, kSiteDrain);
             if (q_issued >= 0) mbar_wait(bar_q(q_issued & 1), (q_issued >> 1) & 1, kSiteDrain);
         }
+    } else if (warp == kSdpWarp) {
+        // --------------------------------------------------- S / dP issuer
+        // Tile g (the CTA's g-th key tile over all its items) writes S and
+        // dP into buffer g & 1, which tile g - 2's dS still occupies until
+        // that tile's dQ MMAs complete (sfree).
+        constexpr uint32_t id_sdp = idesc_bf16(128, kKeys, 0, 0);
+        bool ok = true;
+        uint32_t g = 0;
+        for (int k = 0; k < n_mine && ok; ++k) {
+            const int nt = make_item(a, tab, k, lane).nt();
+            for (int p = 0; p < nt && ok; ++p, ++g) {
+                bool r = true;
+                if (lane == 0) {
+                    const int ks = g % kKStages, vs = g % kVStages, bb = g & 1;
+                    if (p == 0) r = mbar_wait(bar_q(k & 1), (k >> 1) & 1, kSiteQ);
+                    if (r && g >= 2) r = mbar_wait(bar_sfree(bb), ((g - 2) >> 1) & 1, kSiteSfree);
+                    if (r) r = mbar_wait(bar_kfull(ks), (g / kKStages) & 1, kSiteFull);
+                    if (r) r = mbar_wait(bar_vfull(vs), (g / kVStages) & 1, kSiteFull);
+                    if (r) {
+                        tc_fence_after();
+                        // Descriptors of the operand bases; a K step adds its
+                        // byte offset / 16 to the address field.
+                        const uint32_t qa = xbuf(k);
+                        const uint64_t dq = sdesc_sw128(qa, 16, 1024), ddo = sdesc_sw128(qa + 2 * L::kRows128, 16, 1024);
+                        const uint64_t dk = sdesc_sw128(sbase + L::k_off + ks * H * L::kKVHalf, 16, 1024);
+                        const uint64_t dv = sdesc_sw128(sbase + L::v_off + vs * H * L::kKVHalf, 16, 1024);
+                        const uint32_t ts = tmem + kColS + bb * kKeys, tdp = tmem + kColDP + bb * kKeys;
+#pragma unroll
+                        for (int kk = 0; kk < 4 * H; ++kk) {
+                            const uint32_t o = ((kk / 4) * L::kRows128 + (kk % 4) * 32) >> 4;
+                            const uint32_t ko = ((kk / 4) * L::kKVHalf + (kk % 4) * 32) >> 4;
+                            mma_ss(ts, dq + o, dk + ko, id_sdp, kk > 0);
+                            mma_ss(tdp, ddo + o, dv + ko, id_sdp, kk > 0);
+                        }
+                        mma_commit(bar_sdp(bb));
+                        mma_commit(bar_vempty(vs));                 // V is read by dP only
+                    }
+                }
+                ok = __shfl_sync(0xFFFFFFFFu, r, 0);
+            }
+        }
+        if (lane == 0) {
+            // Every MMA issued here is complete before tensor memory is released.
+            mma_commit(bar_final_sdp);
+            mbar_wait(bar_final_sdp, 0, kSiteFinalSdp);
+        }
     } else if (warp == kMmaWarp) {
-        // ---------------------------------------------------------- MMA issuer
-        constexpr uint32_t id_sdp = idesc_bf16(128, kKeys, 0, 0);   // S, dP
+        // --------------------------------------------------- gradient issuer
         constexpr uint32_t id_dq = idesc_bf16(128, D, 0, 1);        // dQ: A dS (tensor memory), B K MN-major
         constexpr uint32_t id_kv = idesc_bf16(128, kKeys, 1, 1);    // dV^T, dK^T: both MN-major
         bool ok = true;
-        // Cursor A walks the tiles whose S / dP are issued next, up to two
-        // tiles ahead of the tile whose gradient MMAs run.
-        int kA = 0, pA = 0, ntA = 0;
-        uint32_t gtA = 0;
-        auto enter_A = [&]() { ntA = make_item(a, tab, kA, lane).nt(); };
-        int pfree_k = -1;                                   // last item whose pfree was committed
-        // S / dP of an item's first tile need its Q / dO, which load once the
-        // previous item's P / dS are no longer read (pfree).
-        auto can_issue = [&]() { return kA < n_mine && (pA > 0 || kA == 0 || pfree_k >= kA - 1); };
-        auto issue_sdp = [&]() -> bool {
-            bool r = true;
-            if (lane == 0) {
-                const int ks = gtA % kKStages, vs = gtA % kVStages, bb = gtA & 1;
-                if (pA == 0) r = mbar_wait(bar_q(kA & 1), (kA >> 1) & 1, kSiteQ);
-                if (r) r = mbar_wait(bar_kfull(ks), (gtA / kKStages) & 1, kSiteFull);
-                if (r) r = mbar_wait(bar_vfull(vs), (gtA / kVStages) & 1, kSiteFull);
-                if (r) {
-                    tc_fence_after();
-                    // Descriptors of the operand bases; a K step adds its
-                    // byte offset / 16 to the address field.
-                    const uint32_t qa = xbuf(kA);
-                    const uint64_t dq = sdesc_sw128(qa, 16, 1024), ddo = sdesc_sw128(qa + 2 * L::kRows128, 16, 1024);
-                    const uint64_t dk = sdesc_sw128(sbase + L::k_off + ks * H * L::kKVHalf, 16, 1024);
-                    const uint64_t dv = sdesc_sw128(sbase + L::v_off + vs * H * L::kKVHalf, 16, 1024);
-                    const uint32_t ts = tmem + kColS + bb * kKeys, tdp = tmem + kColDP + bb * kKeys;
-#pragma unroll
-                    for (int kk = 0; kk < 4 * H; ++kk) {
-                        const uint32_t o = ((kk / 4) * L::kRows128 + (kk % 4) * 32) >> 4;
-                        const uint32_t ko = ((kk / 4) * L::kKVHalf + (kk % 4) * 32) >> 4;
-                        mma_ss(ts, dq + o, dk + ko, id_sdp, kk > 0);
-                        mma_ss(tdp, ddo + o, dv + ko, id_sdp, kk > 0);
-                    }
-                    mma_commit(bar_sdp(bb));
-                    mma_commit(bar_vempty(vs));                 // V is read by dP only
-                }
-            }
-            r = __shfl_sync(0xFFFFFFFFu, r, 0);
-            ++gtA;
-            if (++pA == ntA) {
-                pA = 0;
-                if (++kA < n_mine) enter_A();
-            }
-            return r;
-        };
-        if (kA < n_mine) enter_A();
         uint32_t gt = 0, gs = 0;
         for (int k = 0; k < n_mine && ok; ++k) {
             const Item mc = make_item(a, tab, k, lane);
             const int nt = mc.nt(), n_seg = mc.n_seg;
             for (int p = 0; ok && p < nt; ++p, ++gt) {
-                // S / dP up to two tiles ahead (this tile's always: its
-                // item's Q / dO were released during the previous item).
-                while (ok && can_issue() && gtA <= gt + 1) ok = issue_sdp();
-                if (!ok) break;
                 const int ks = gt % kKStages, bb = gt & 1;
                 const bool seg = p < n_seg;
                 if (lane == 0) {
@@ -440,6 +448,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             mma_ts(tmem + kColDQ, ds + 16 * kk, kb + (kk * 2048 >> 4), id_dq, acc || kk > 0);
                             mma_ts(tmem + kColDQ, ds + 16 * kk + 8, kb + (kk * 2048 >> 4), id_dq, true);
                         }
+                        mma_commit(bar_sfree(bb));                  // S / dP buffer bb reusable
                     }
                     if (ok && seg) {
                         // dV^T = dO^T P and dK^T = Q^T dS over the 128 query
@@ -467,19 +476,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                     }
                     if (ok) {
-                        mma_commit(bar_kempty(ks));
+                        mma_commit(bar_kempty(ks));                      // K read by S (done) and dQ
                         if (p == nt - 1) mma_commit(bar_qfree);          // Q / dO no longer read
                     }
                 }
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-                if (seg) {
-                    if (p == n_seg - 1) pfree_k = k;
-                    ++gs;
-                }
+                if (seg) ++gs;
             }
         }
         if (lane == 0) {
-            // Every MMA issued is complete before tensor memory is released.
+            // Every MMA issued here is complete before tensor memory is released.
             mma_commit(bar_final);
             mbar_wait(bar_final, 0, kSiteFinal);
         }
@@ -650,7 +656,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // this item's Q / dO buffer (free once its last MMAs completed) as
             // eight 64-row x 32-column boxes in the 128-byte-swizzled layout
             // of the dQ tensor map; thread 0 stores the boxes with bulk copies
-            // that run on while the next item starts.
+            // that run on while the next item starts.  (Stores straight from
+            // registers measured slower.)
             ok = mbar_wait(bar_qfree, k & 1, kSiteQfree);
             if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
             tc_fence_after();
