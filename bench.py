@@ -86,14 +86,24 @@ def algorithmic(w) -> dict:
                  + gidx_bytes)
     seg_keys = B * Hkv * Ts * d * el
     summ_bytes = seg_keys + B * Hkv * (Ts // 64 + Ts // 8) * d * 4
-    csum_read = B * Hkv * nQB * (w.T_hist // 64 + nQB / 2) * d * 4    # eligible chunks
-    rc_bytes = q_bytes + csum_read + B * Hkv * nQB * (d * 4 + wc * 4)
+    # Routers: the block query reads all of Q; chunk routing reads the
+    # context's chunk summaries (each once per (batch, kv-head)); group
+    # routing gathers the 8 group summaries of each chosen chunk per block;
+    # plus qbar and the index rows written and read back.  The per-use
+    # figure instead counts every block's own read of its eligible chunk
+    # summaries (most of them served by L2).
+    n_chunks = w.T // 64
+    csum_once = B * Hkv * n_chunks * d * 4
+    csum_per_use = B * Hkv * sum(w.T_hist // 64 + qb for qb in range(nQB)) * d * 4
+    small = B * Hkv * nQB * (d * 4 + wc * 4)                           # qbar and cidx written
+    rc_bytes = q_bytes + csum_once + small
     rg_bytes = B * Hkv * nQB * (d * 4 + wc * 4 + 8 * wc * d * 4 + wg * 4)
     return dict(
         attn_fwd=dict(bytes=fwd_bytes, flops=4.0 * d * B * Hq * key_pairs),
         attn_bwd=dict(bytes=bwd_bytes, flops=10.0 * d * B * Hq * key_pairs),
         summaries=dict(bytes=summ_bytes, flops=0.0),
-        route_chunks=dict(bytes=rc_bytes, flops=0.0),
+        route_chunks=dict(bytes=rc_bytes, flops=0.0,
+                          per_use_bytes=q_bytes + csum_per_use + small),
         route_groups=dict(bytes=rg_bytes, flops=0.0),
     )
 
@@ -540,20 +550,15 @@ def run_gpu(args, w) -> None:
                 gbs = b_ / (stage_ms[s_] * 1e-3) / 1e9
                 stage_roof[s_] = dict(ms=stage_ms[s_], algorithmic_bytes=b_, gb_per_s=gbs,
                                       frac=gbs / pk["hbm_gbs"])
-        # The routers' algorithmic bytes count every block's read of its
-        # eligible chunk summaries (per use); the distinct bytes -- Q, each
-        # (batch, kv-head)'s summaries once, the index rows -- bound what
-        # reaches HBM when L2 serves the re-reads.
-        el_ = 2 if w.dtype == "bf16" else 4
-        wc_ = w.k_c if w.k_c > 0 else w.T // 64
-        wg_ = w.k_g if w.k_g > 0 else 8 * wc_
-        uniq = (w.B * w.Hq * w.T_seg * w.d * el_ + w.B * w.Hkv * (w.T // 64 + w.T // 8) * w.d * 4
-                + w.B * w.Hkv * (w.T_seg // 64) * (w.d * 4 + (wc_ + wg_) * 4))
+        # The routers' roofline counts each byte once (Q, the chunk summaries,
+        # the gathered group summaries, index rows); the per-use figure counts
+        # every block's read of its eligible chunk summaries.
         if "route" in stage_roof:
             r_ = stage_roof["route"]
-            r_["unique_bytes"] = uniq
-            r_["frac_unique"] = uniq / (r_["ms"] * 1e-3) / 1e9 / pk["hbm_gbs"]
-            if r_["frac"] > 1.0:
+            per_use = alg["route_chunks"]["per_use_bytes"] + alg["route_groups"]["bytes"]
+            r_["per_use_bytes"] = per_use
+            r_["frac_per_use"] = per_use / (r_["ms"] * 1e-3) / 1e9 / pk["hbm_gbs"]
+            if r_["frac_per_use"] > 1.0:
                 r_["note"] = "per-use bytes above the copy peak: re-reads of the summaries hit L2"
         el = 2 if w.dtype == "bf16" else 4
         full_bytes = w.B * w.Hkv * w.T * w.d * el + w.B * w.Hkv * (w.T // 64 + w.T // 8) * w.d * 4

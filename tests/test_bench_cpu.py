@@ -68,3 +68,22 @@ def test_sweep_work_is_constant_in_context(bench, k_g):
         assert len({(x[stage]["bytes"], x[stage]["flops"]) for x in works}) == 1
     pairs = 2048 * 8 * k_g + 32 * 2080
     assert works[0]["attn_fwd"]["flops"] == 4 * 128 * 4 * 32 * pairs
+
+
+def test_router_bytes_count_each_byte_once(bench):
+    # 16K step: Q (bf16) read once; the 256 chunk summaries of each of the
+    # 8 kv-heads read once; per block the 8 groups of each of the 8 chosen
+    # chunks gathered; qbar (128 floats) and the index rows written and read
+    # back: 16.8 + 1.0 + 8.4 MB plus the small terms, about 26.6 MB.
+    a = bench.algorithmic(W.QWEN3_CTX16K_TRAIN)
+    q = 32 * 2048 * 128 * 2
+    csum = 8 * 256 * 128 * 4
+    blocks = 8 * 32
+    rc = q + csum + blocks * (128 * 4 + 8 * 4)
+    rg = blocks * (128 * 4 + 8 * 4 + 8 * 8 * 128 * 4 + 32 * 4)
+    assert a["route_chunks"]["bytes"] == rc
+    assert a["route_groups"]["bytes"] == rg
+    assert 26.5e6 < rc + rg < 26.7e6
+    # Per use, block qb reads its 224 + qb eligible chunk summaries.
+    per_use = q + 8 * sum(224 + qb for qb in range(32)) * 128 * 4 + blocks * (128 * 4 + 8 * 4)
+    assert a["route_chunks"]["per_use_bytes"] == per_use
