@@ -16,17 +16,20 @@ from dataclasses import dataclass
 
 import torch
 
-HGA_OK, HGA_ERR_INVALID_ARG, HGA_ERR_UNSUPPORTED, HGA_ERR_CUDA = 0, 1, 2, 3
+HGA_OK, HGA_ERR_INVALID_ARG, HGA_ERR_UNSUPPORTED, HGA_ERR_CUDA, HGA_ERR_DEVICE_CHECK = 0, 1, 2, 3, 4
 HGA_ALL = -1
 HGA_BF16, HGA_FP32 = 0, 1
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhga.so")
+# The bounds-checked build of the same library (-DHGA_CHECK_BOUNDS).
+CHECKED_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhga_checked.so")
 
 EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_build_summaries_rows",
            "hga_route_chunks",
            "hga_route_groups", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
            "hga_stage_params", "hga_stage_routed", "hga_decode", "hga_route_causal", "hga_attn_fwd_causal",
-           "hga_attn_bwd_causal", "hga_device_status", "hga_last_error",
+           "hga_attn_bwd_causal", "hga_device_status", "hga_device_check", "hga_checked_build",
+           "hga_selftest_wait", "hga_last_error",
            "hga_version")
 NOALLOC_MAX_ROWS = 1 << 20     # HGA_NOALLOC_MAX_ROWS
 
@@ -117,6 +120,9 @@ def load() -> ctypes.CDLL:
             "hga_attn_fwd_causal": ([PP, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_attn_bwd_causal": ([PP, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_device_status": ([ctypes.POINTER(ctypes.c_int), ctypes.c_int], ctypes.c_int),
+            "hga_selftest_wait": ([ctypes.c_int, ctypes.POINTER(ctypes.c_int), P], ctypes.c_int),
+            "hga_device_check": ([ctypes.POINTER(ctypes.c_int), ctypes.c_int], ctypes.c_int),
+            "hga_checked_build": ([], ctypes.c_int),
             "hga_last_error": ([], ctypes.c_char_p),
             "hga_version": ([], ctypes.c_char_p),
         }
@@ -157,6 +163,34 @@ def device_status(clear: bool = False) -> int:
     v = ctypes.c_int()
     _check(load().hga_device_status(ctypes.byref(v), int(clear)))
     return v.value
+
+
+def use_library(path: str) -> None:
+    """Route every later call through the library at `path` (for instance
+    CHECKED_LIB_PATH, the bounds-checked build); the next call loads it."""
+    global _lib, LIB_PATH
+    LIB_PATH = path
+    _lib = None
+
+
+def checked_build() -> bool:
+    """Whether the loaded library checks index rows on the device."""
+    return bool(load().hga_checked_build())
+
+
+def device_check(clear: bool = False) -> int:
+    """First failed device bounds check's site code (0: none).  Syncs."""
+    v = ctypes.c_int()
+    _check(load().hga_device_check(ctypes.byref(v), int(clear)))
+    return v.value
+
+
+def selftest_wait(limit_us: int, stream=None) -> int:
+    """Launch the failure-path self-test (a bounded wait that runs out after
+    limit_us); returns the code it records in the status word."""
+    site = ctypes.c_int()
+    _check(load().hga_selftest_wait(int(limit_us), ctypes.byref(site), _stream(stream)))
+    return site.value
 
 
 def route_widths(p: Params) -> tuple[int, int]:

@@ -19,6 +19,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libhga.so")
+# The bounds-checked build (device checks of the caller's index rows).
+BUILD_CHECKED = os.path.join(PKG, "_build_checked")
+LIB_CHECKED = os.path.join(PKG, "libhga_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
@@ -37,15 +40,18 @@ def _deps_mtime() -> float:
     return max((os.path.getmtime(f) for f in files), default=0.0)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
-    """Compile stale objects and relink libhga.so; returns the library path."""
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None,
+          checked: bool = False) -> str:
+    """Compile stale objects and relink libhga.so (libhga_checked.so with
+    checked=True: compiled with -DHGA_CHECK_BOUNDS); returns the library path."""
+    build_dir, lib_path = (BUILD_CHECKED, LIB_CHECKED) if checked else (BUILD, LIB)
+    os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr = _deps_mtime()
-    flags = NVCC_FLAGS + (extra_flags or [])
+    flags = NVCC_FLAGS + (["-DHGA_CHECK_BOUNDS"] if checked else []) + (extra_flags or [])
     procs, objs = [], []
     for src in sources:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), hdr):
             cmd = [nvcc(), *flags, "-c", src, "-o", obj]
@@ -61,14 +67,14 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
             failed.append(src)
     if failed:
         raise RuntimeError(f"nvcc failed for {', '.join(os.path.basename(f) for f in failed)}")
-    if procs or force or not os.path.exists(LIB) or \
-            os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        tmp = LIB + ".tmp"
+    if procs or force or not os.path.exists(lib_path) or \
+            os.path.getmtime(lib_path) < max(os.path.getmtime(o) for o in objs):
+        tmp = lib_path + ".tmp"
         cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
         subprocess.run(cmd, check=True)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, checked="--checked" in sys.argv))

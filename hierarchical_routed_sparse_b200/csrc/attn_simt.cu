@@ -13,6 +13,7 @@
 // routed groups (8 groups each), then the own chunk with the token-causal
 // mask.  Thread (ty, tx) of a 16 x 16 grid owns rows 4ty..4ty+3 and the
 // columns tx + 16c, which keeps the shared-memory reads conflict-free.
+#include "check.cuh"
 #include "hga_internal.cuh"
 
 namespace hga {
@@ -82,7 +83,9 @@ __device__ __forceinline__ float half_warp_sum(float v)
 }
 
 // Number of valid (non -1) entries of an index row; they form a prefix.
-__device__ __forceinline__ int count_valid(const int32_t* row, int w, int* s_groups)
+// In checked builds the n entries used are range-checked (0 <= j < limit,
+// limit = 8 * own chunk), which also catches a -1 inside the prefix.
+__device__ __forceinline__ int count_valid(const int32_t* row, int w, int* s_groups, int64_t limit, int site)
 {
     __shared__ int n;
     if (threadIdx.x == 0) n = 0;
@@ -93,6 +96,10 @@ __device__ __forceinline__ int count_valid(const int32_t* row, int w, int* s_gro
         if (j >= 0) atomicAdd(&n, 1);
     }
     __syncthreads();
+    if (chk::kEnabled) {
+        for (int i = threadIdx.x; i < n; i += kThreads) s_groups[i] = chk::group(s_groups[i], limit, site);
+        __syncthreads();
+    }
     return n;
 }
 
@@ -134,7 +141,8 @@ attn_fwd_simt_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K,
     const TIn* Qrow0 = Q + (bh * T_seg + qb * kTile) * D;
     const TIn* Kh = K + (b * Hkv + g) * T * D;
     const TIn* Vh = V + (b * Hkv + g) * T * D;
-    const int n_groups = count_valid(gidx + ((b * Hkv + g) * nQB + qb) * wg, wg, s_groups);
+    const int n_groups = count_valid(gidx + ((b * Hkv + g) * nQB + qb) * wg, wg, s_groups,
+                                     (T_hist + qb * kTile) / kGroup, chk::kSiteSimtFwd);
     const int n_routed_tiles = (n_groups + 7) / 8;
     const int64_t own_start = T_hist + qb * kTile;
 
@@ -261,7 +269,8 @@ attn_bwd_simt_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K,
     const TIn* Vh = V + (b * Hkv + g) * T * D;
     float* dKh = dK_seg + (b * Hkv + g) * T_seg * D;
     float* dVh = dV_seg + (b * Hkv + g) * T_seg * D;
-    const int n_groups = count_valid(gidx + ((b * Hkv + g) * nQB + qb) * wg, wg, s_groups);
+    const int n_groups = count_valid(gidx + ((b * Hkv + g) * nQB + qb) * wg, wg, s_groups,
+                                     (T_hist + qb * kTile) / kGroup, chk::kSiteSimtBwd);
     const int n_routed_tiles = (n_groups + 7) / 8;
     const int64_t own_start = T_hist + qb * kTile;
 
@@ -445,5 +454,8 @@ cudaError_t launch_attn_bwd_simt(const Shape& s, const void* Q, const void* K, c
                       : launch_bwd<float, 64>(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg,
                                               Drow, st);
 }
+
+// Check word of this translation unit's bounds checks (checked builds).
+HGA_CHECK_WORD_READER(check_word_attn_simt)
 
 }  // namespace hga

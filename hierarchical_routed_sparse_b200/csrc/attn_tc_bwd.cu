@@ -47,6 +47,7 @@
 // the two Q/dO <-> P/dS buffers they fill 224 KB of shared memory.
 #include <algorithm>
 
+#include "check.cuh"
 #include "hga_internal.cuh"
 #include "sm100.cuh"
 
@@ -319,7 +320,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 int y = 0;
                 if (t < n_rt) {
                     const int gi = t * 8 + lane;
-                    if (lane < 8) y = int(kv_base + (int64_t)__ldg(grow + (gi < m.n_g ? gi : 0)) * 8);
+                    if (lane < 8)
+                        y = int(kv_base + (int64_t)chk::group(__ldg(grow + (gi < m.n_g ? gi : 0)),
+                                                              8 * (a.T_hist / 64 + m.qb), chk::kSiteBwdTcLoad) * 8);
                 } else {
                     y = int(kv_base + m.own_start(a));
                 }
@@ -502,7 +505,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int q = 0; q < 2; ++q) {
                 const int gi = t * 8 + 2 * kq + q;
                 gb[q] = t == m.n_rt() ? m.own_start(a) + 16 * kq + 8 * q
-                                      : (gi < m.n_g ? __ldg(m.grow(a) + gi) * 8 : -64);
+                                      : (gi < m.n_g ? chk::group(__ldg(m.grow(a) + gi), 8 * (a.T_hist / 64 + m.qb),
+                                                                 chk::kSiteBwdTcKeys) * 8
+                                                    : -64);
             }
         };
         // dV^T / dK^T of a segment tile (d = tensor-memory lane r, keys of
@@ -958,5 +963,8 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
     return launch_pdl(attn_bwd_tc_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st, tq, tdo, tk8, tv8,
                       tk64, tv64, tdq, a);
 }
+
+// Check word of this translation unit's bounds checks (checked builds).
+HGA_CHECK_WORD_READER(check_word_attn_tc_bwd)
 
 }  // namespace hga

@@ -29,6 +29,7 @@
 // the softmax works on the current one.  With 97 KB of shared memory and 256
 // columns, two CTAs share an SM: one's prologue and epilogue overlap the
 // other's key loop.
+#include "check.cuh"
 #include "hga_internal.cuh"
 #include "sm100.cuh"
 
@@ -210,7 +211,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const int gi = t * 8 + gl;
                     // Slots past the last routed group repeat group 0: finite
                     // data whose scores the softmax masks out.
-                    const int grp = __ldg(grow + (gi < n_g ? gi : 0));
+                    const int grp = chk::group(__ldg(grow + (gi < n_g ? gi : 0)), 8 * (a.T_hist / 64 + qb),
+                                               chk::kSiteFwdTc);
                     const int y = int(kv_base + (int64_t)grp * 8);
                     for (int c = 0; c < H; ++c)
                         tma_load_2d(dst + c * L::kKVHalf + gl * 1024, m8, 64 * c, y, bar_full(ring, s));
@@ -496,5 +498,8 @@ cudaError_t launch_attn_fwd_tc(const Shape& s, const void* Q, const void* K, con
 {
     return s.d == 128 ? launch<128>(s, Q, K, V, gidx, O, lse, st) : launch<64>(s, Q, K, V, gidx, O, lse, st);
 }
+
+// Check word of this translation unit's bounds checks (checked builds).
+HGA_CHECK_WORD_READER(check_word_attn_tc_fwd)
 
 }  // namespace hga

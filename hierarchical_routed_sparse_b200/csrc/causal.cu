@@ -29,6 +29,7 @@
 //                        added to the segment's rows with vector float
 //                        atomics.
 // Float32 arithmetic (packed fp32x2 FMAs); bf16 or float32 inputs.
+#include "check.cuh"
 #include "hga_internal.cuh"
 #include "router_core.cuh"
 
@@ -179,9 +180,9 @@ causal_route_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, c
 
 // Key k of a row: the routed groups' tokens in order, then the own chunk's
 // tokens own0 .. pos.
-__device__ __forceinline__ int64_t row_token(const int32_t* grow, int n_g, int64_t own0, int k)
+__device__ __forceinline__ int64_t row_token(const int32_t* grow, int n_g, int64_t own0, int k, int site)
 {
-    return k < kGroup * n_g ? (int64_t)__ldg(grow + k / kGroup) * kGroup + k % kGroup
+    return k < kGroup * n_g ? (int64_t)chk::group(__ldg(grow + k / kGroup), own0 / kGroup, site) * kGroup + k % kGroup
                             : own0 + (k - kGroup * n_g);
 }
 
@@ -318,7 +319,7 @@ causal_fwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
     }
     for (int k0 = 0; k0 < n_keys; k0 += 32) {
         const bool valid = k0 + lane < n_keys;
-        const int64_t t = valid ? row_token(grow, n_g, own0, k0 + lane) : 0;
+        const int64_t t = valid ? row_token(grow, n_g, own0, k0 + lane, chk::kSiteCausalFwd) : 0;
         float s[GM], p[GM];
         row_dots<TIn, D, GM>(qw, G, Kb + t * D, valid, s);
 #pragma unroll
@@ -445,7 +446,7 @@ causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
     __syncwarp();
     for (int k0 = 0; k0 < n_keys; k0 += 32) {
         const bool valid = k0 + lane < n_keys;
-        const int64_t t = valid ? row_token(grow, n_g, own0, k0 + lane) : 0;
+        const int64_t t = valid ? row_token(grow, n_g, own0, k0 + lane, chk::kSiteCausalBwd) : 0;
         float s[GM], dp[GM], p[GM], ds[GM];
         row_dots<TIn, D, GM, 8>(qw, G, Kb + t * D, valid, s);
         row_dots<TIn, D, GM, 8>(dow, G, Vb + t * D, valid, dp);
@@ -596,5 +597,8 @@ cudaError_t launch_attn_bwd_causal(const Shape& s, const void* Q, const void* K,
 {
     return dispatch<BwdOp>(s, Q, K, V, O, lse, dO, gidx, dQ, dK, dV, st);
 }
+
+// Check word of this translation unit's bounds checks (checked builds).
+HGA_CHECK_WORD_READER(check_word_causal)
 
 }  // namespace hga

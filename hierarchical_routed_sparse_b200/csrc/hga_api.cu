@@ -37,6 +37,44 @@ int cuda_fail(cudaError_t e, const char* where)
 
 constexpr size_t kMaxSmem = 227 * 1024;
 
+// First nonzero check word of the translation units that read caller index
+// rows (-1 if one could not be read); cleared when `clear`.
+int read_check_words(bool clear)
+{
+    int (*const readers[])(bool) = {hga::check_word_attn_tc_fwd, hga::check_word_attn_tc_bwd,
+                                    hga::check_word_attn_simt,   hga::check_word_causal,
+                                    hga::check_word_router,      hga::check_word_stage};
+    int first = 0;
+    for (auto f : readers) {
+        const int v = f(clear);
+        if (v < 0) return -1;
+        if (!first) first = v;
+    }
+    return first;
+}
+
+// Result of a call that enqueued its kernels with launch status `e`.  In a
+// build with HGA_CHECK_BOUNDS the call waits for its stream and reports a
+// failed device bounds check as HGA_ERR_DEVICE_CHECK (the word is cleared);
+// release builds return at once.
+int finish(cudaError_t e, cudaStream_t st, const char* name)
+{
+    if (e != cudaSuccess) return cuda_fail(e, name);
+#ifdef HGA_CHECK_BOUNDS
+    e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, name);
+    const int w = read_check_words(true);
+    if (w < 0) return fail(HGA_ERR_CUDA, "%s: the bounds-check word could not be read", name);
+    if (w)
+        return fail(HGA_ERR_DEVICE_CHECK,
+                    "%s: device bounds check %d failed: an index row holds an entry outside its valid range "
+                    "(outputs are invalid)", name, w);
+#else
+    (void)st;
+#endif
+    return HGA_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 #define CHECK_PTR(ptr)                                                                   \
@@ -145,10 +183,39 @@ int hga_device_status(int* status, int clear)
     const int vf = hga::attn_fwd_tc_status(clear != 0);
     const int vb = hga::attn_bwd_tc_status(clear != 0);
     const int vd = hga::decode_status(clear != 0);
-    if (vf < 0 || vb < 0 || vd < 0)
+    const int vs = hga::selftest_status(clear != 0);
+    if (vf < 0 || vb < 0 || vd < 0 || vs < 0)
         return fail(HGA_ERR_CUDA, "hga_device_status: the status word could not be read");
-    *status = vf ? vf : (vb ? vb : vd);
+    *status = vf ? vf : (vb ? vb : (vd ? vd : vs));
     return HGA_OK;
+}
+
+int hga_device_check(int* word, int clear)
+{
+    if (!word) return fail(HGA_ERR_INVALID_ARG, "word is NULL");
+    const int w = read_check_words(clear != 0);
+    if (w < 0) return fail(HGA_ERR_CUDA, "hga_device_check: the check word could not be read");
+    *word = w;
+    return HGA_OK;
+}
+
+int hga_checked_build(void)
+{
+#ifdef HGA_CHECK_BOUNDS
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+int hga_selftest_wait(int limit_us, int* site, hga_stream_t stream)
+{
+    if (limit_us < 1 || limit_us > 1000000)
+        return fail(HGA_ERR_INVALID_ARG, "limit_us=%d outside [1, 1000000]", limit_us);
+    if (site) *site = hga::selftest_site();
+    const cudaError_t e = hga::launch_selftest_wait(1000ull * (unsigned long long)limit_us,
+                                                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_selftest_wait");
 }
 
 int hga_route_widths(const hga_params* p, int* wc, int* wg)
@@ -232,7 +299,7 @@ int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum, 
     if (hga::route_groups_smem(s) > kMaxSmem)
         return fail(HGA_ERR_UNSUPPORTED, "k_c=%d gives too many candidate groups for the group router", s.wc);
     cudaError_t e = hga::launch_route_groups(s, qbar, gsum, cidx, gidx, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route_groups");
+    return finish(e, static_cast<cudaStream_t>(stream), "hga_route_groups");
 }
 
 int hga_route(const hga_params* p, const void* Q, const float* csum, const float* gsum, float* qbar,
@@ -293,7 +360,7 @@ int hga_stage_routed(const hga_params* p, const void* K_hist, const void* V_hist
     }
     const cudaError_t e = hga::launch_stage(s, kh, vh, K_seg, V_seg, gidx, K_stage, V_stage, gidx_stage,
                                             static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_stage_routed");
+    return finish(e, static_cast<cudaStream_t>(stream), "hga_stage_routed");
 }
 
 int hga_decode(const hga_params* p, int64_t pos, const void* q, const void* K, const void* V,
@@ -365,7 +432,7 @@ int hga_attn_fwd_causal(const hga_params* p, const void* Q, const void* K, const
     CHECK_PTR(O);
     CHECK_PTR(lse);
     cudaError_t e = hga::launch_attn_fwd_causal(s, Q, K, V, gidx, O, lse, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_fwd_causal");
+    return finish(e, static_cast<cudaStream_t>(stream), "hga_attn_fwd_causal");
 }
 
 int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K, const void* V, const float* O,
@@ -387,7 +454,7 @@ int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K, const
     CHECK_PTR(dV_seg);
     cudaError_t e = hga::launch_attn_bwd_causal(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg,
                                                 static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_bwd_causal");
+    return finish(e, static_cast<cudaStream_t>(stream), "hga_attn_bwd_causal");
 }
 
 int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* V,
@@ -408,7 +475,7 @@ int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* 
     cudaError_t e = hga::attn_fwd_tc_supported(s)
                         ? hga::launch_attn_fwd_tc(s, Q, K, V, gidx, O, lse, static_cast<cudaStream_t>(stream))
                         : hga::launch_attn_fwd_simt(s, Q, K, V, gidx, O, lse, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_fwd");
+    return finish(e, static_cast<cudaStream_t>(stream), "hga_attn_fwd");
 }
 
 int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* V, const float* O,
@@ -436,7 +503,7 @@ int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* 
         return fail(HGA_ERR_UNSUPPORTED, "k_g=%d too large for the attention kernel", s.wg);
     cudaError_t e = run_attn_bwd(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, static_cast<float*>(workspace),
                                  static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_bwd");
+    return finish(e, static_cast<cudaStream_t>(stream), "hga_attn_bwd");
 }
 
 }  // extern "C"
@@ -525,5 +592,5 @@ extern "C" int hga_attn_bwd_noalloc(const hga_params* p, const void* Q, const vo
     // scratch needs no clearing between calls.
     cudaError_t e = run_attn_bwd(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, scratch,
                                  static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attn_bwd_noalloc");
+    return finish(e, static_cast<cudaStream_t>(stream), "hga_attn_bwd_noalloc");
 }

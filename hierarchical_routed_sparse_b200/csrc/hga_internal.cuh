@@ -150,6 +150,17 @@ cudaError_t launch_decode(const Shape& s, int64_t pos, const void* q, const void
 size_t decode_smem(const Shape& s);
 int decode_max_heads();
 int decode_status(bool clear);   // status word of decode.cu's bounded waits
+// Check words of the bounds checks (checked builds; 0 otherwise), one per
+// translation unit that reads caller index rows.
+int check_word_attn_tc_fwd(bool clear);
+int check_word_attn_tc_bwd(bool clear);
+int check_word_attn_simt(bool clear);
+int check_word_causal(bool clear);
+int check_word_router(bool clear);
+int check_word_stage(bool clear);
+int selftest_status(bool clear); // status word of selftest.cu
+int selftest_site();             // the code its wait records
+cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t st);
 // Strictly causal variant: routing per query position (causal.cu).
 cudaError_t launch_route_causal(const Shape& s, const void* Q, const float* csum, const float* gsum, int32_t* cidx,
                                 int32_t* gidx, cudaStream_t st);

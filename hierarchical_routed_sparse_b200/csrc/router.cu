@@ -122,7 +122,7 @@ template <int D>
 __global__ void __launch_bounds__(kRouterThreads, 2)
 route_groups_kernel(const float* __restrict__ qbar, const float* __restrict__ gsum,
                     const int32_t* __restrict__ cidx, int32_t* __restrict__ gidx,
-                    int64_t nQB, int64_t nG, int wc, int k_g, int wg)
+                    int64_t nQB, int64_t nG, int wc, int k_g, int wg, int64_t c_hist)
 {
     extern __shared__ unsigned long long keys[];      // [8*wc], ids [8*wc], flags [8*wc]
     int32_t* ids = reinterpret_cast<int32_t*>(keys + (size_t)kGroupsPerChunk * wc);
@@ -135,8 +135,9 @@ route_groups_kernel(const float* __restrict__ qbar, const float* __restrict__ gs
     const int64_t bg = u / nQB;
     for (int col = threadIdx.x; col < D; col += kRouterThreads) qs[col] = qbar[u * D + col];
     __syncthreads();
+    // The caller's chunk row: valid chunks lie before the block's own chunk.
     route_groups_block<D>(qs, gsum + bg * nG * D, cidx + u * wc, wc, k_g, wg, keys, ids, flags, &n_valid,
-                          gidx + u * wg, threadIdx.x);
+                          gidx + u * wg, threadIdx.x, c_hist + u % nQB);
 }
 
 // ---- a2 + a3 + a4 in one launch ------------------------------------------------
@@ -197,7 +198,7 @@ cudaError_t launch_rg(const Shape& s, const float* qbar, const float* gsum, cons
     }
     const int64_t blocks = (int64_t)s.B * s.Hkv * s.nQB;
     return launch_pdl(k, dim3((unsigned)blocks), dim3(kRouterThreads), smem, st, qbar, gsum, cidx, gidx, s.nQB,
-                      s.nG, s.wc, s.k_g, s.wg);
+                      s.nG, s.wc, s.k_g, s.wg, s.T_hist / kChunk);
 }
 
 template <typename TIn, int D>
@@ -257,5 +258,8 @@ cudaError_t launch_route_groups(const Shape& s, const float* qbar, const float* 
     return s.d == 128 ? launch_rg<128>(s, qbar, gsum, cidx, gidx, st)
                       : launch_rg<64>(s, qbar, gsum, cidx, gidx, st);
 }
+
+// Check word of this translation unit's bounds checks (checked builds).
+HGA_CHECK_WORD_READER(check_word_router)
 
 }  // namespace hga

@@ -10,6 +10,10 @@
 // comparison and every candidate key is distinct.  Not part of the ABI.
 #pragma once
 
+#include <stdint.h>
+
+#include "check.cuh"
+
 #include "hga_internal.cuh"
 
 namespace hga {
@@ -246,7 +250,8 @@ template <int D>
 __device__ __forceinline__ void route_groups_block(const float* qs, const float* __restrict__ gs,
                                                    const int32_t* crow, int wc, int k_g, int wg,
                                                    unsigned long long* keys, int32_t* ids, uint8_t* flags,
-                                                   int* s_count, int32_t* gidx_row, int tid)
+                                                   int* s_count, int32_t* gidx_row, int tid,
+                                                   int64_t c_limit = INT64_MAX)
 {
     const int lane = tid & 31, warp = tid >> 5;
     if (warp == 0) {
@@ -256,7 +261,8 @@ __device__ __forceinline__ void route_groups_block(const float* qs, const float*
     __syncthreads();
     const int n = *s_count * kGroupsPerChunk;          // candidate groups
     for (int i = tid; i < n; i += kRouterThreads)
-        ids[i] = crow[i / kGroupsPerChunk] * kGroupsPerChunk + i % kGroupsPerChunk;
+        ids[i] = chk::chunk(crow[i / kGroupsPerChunk], c_limit, chk::kSiteRouteGroups) * kGroupsPerChunk +
+                 i % kGroupsPerChunk;
     __syncthreads();
     if (k_g <= 0 || k_g >= n) {                        // keep every candidate
         for (int i = tid; i < wg; i += kRouterThreads) gidx_row[i] = i < n ? ids[i] : -1;

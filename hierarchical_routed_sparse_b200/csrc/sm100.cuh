@@ -92,18 +92,24 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
 // in hardware (no spinning on issue slots); the time bound is checked between
 // sleeps.  Gives up after kWaitLimitNs, records `site` in g_status and
 // returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int site)
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, int site,
+                                                unsigned long long limit_ns)
 {
-    constexpr uint32_t kHintNs = 100000;                 // 0.1 ms per sleep
-    if (mbar_try(bar, parity, kHintNs)) return true;
+    const uint32_t hint_ns = limit_ns < 100000ull ? uint32_t(limit_ns / 4 + 1) : 100000u;   // per sleep
+    if (mbar_try(bar, parity, hint_ns)) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
-        if (mbar_try(bar, parity, kHintNs)) return true;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (mbar_try(bar, parity, hint_ns)) return true;
+        if (global_ns() - t0 > limit_ns) {
             atomicCAS(&g_status, 0, site);
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int site)
+{
+    return mbar_wait_limit(bar, parity, site, kWaitLimitNs);
 }
 
 // ---- TMA ----------------------------------------------------------------------------

@@ -20,6 +20,7 @@
 // stays -1.  The map is increasing, so every row stays ascending with
 // history before segment, and the segment keys keep their offsets past the
 // history, so the backward's dK_seg / dV_seg are unchanged.
+#include "check.cuh"
 #include "hga_internal.cuh"
 
 namespace hga {
@@ -82,6 +83,9 @@ stage_unique_kernel(const uint8_t* __restrict__ Kh, const uint8_t* __restrict__ 
         if (g < 0) {
             out = -1;
         } else if (g >= ng_hist) {
+            // A segment group: in the staged problem it follows the T_stage
+            // history rows.  Valid groups lie before the row's own chunk.
+            chk::flag_if(g >= ng_hist + T_seg / 8, chk::kSiteStage);
             out = int32_t(T_stage / 8 + (g - ng_hist));
         } else {
             const uint32_t word = bm[g >> 5];
@@ -160,5 +164,8 @@ cudaError_t launch_stage(const Shape& s, const void* K_hist, const void* V_hist,
     }
     return cudaSuccess;
 }
+
+// Check word of this translation unit's bounds checks (checked builds).
+HGA_CHECK_WORD_READER(check_word_stage)
 
 }  // namespace hga

@@ -62,6 +62,7 @@ extern "C" {
 #define HGA_ERR_INVALID_ARG  1  /* bad shape, pointer, alignment or range   */
 #define HGA_ERR_UNSUPPORTED  2  /* valid but not implemented (e.g. d = 96)  */
 #define HGA_ERR_CUDA         3  /* a launch failed (message has the detail) */
+#define HGA_ERR_DEVICE_CHECK 4  /* checked build: a device bounds check failed */
 
 #define HGA_ALL  (-1)           /* k_c / k_g: keep every eligible candidate */
 
@@ -280,6 +281,32 @@ int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K,
  * *status = 0 when no wait ran out; `clear` != 0 resets the word.
  * Synchronises with the device. */
 int hga_device_status(int* status, int clear);
+
+/* Bounds-check build.  A library compiled with -DHGA_CHECK_BOUNDS
+ * (libhga_checked.so) checks, on the device, every routed group or chunk
+ * index it reads from a caller's index row before using it as an address
+ * (valid: 0 <= index < the row's own chunk, in chunks or groups); an index
+ * outside records a site code in a device check word and is replaced by
+ * index 0 of the same (batch, kv-head), so no access leaves the tensors.
+ * In that build hga_route_groups, hga_attn_fwd, hga_attn_bwd,
+ * hga_attn_bwd_noalloc, hga_stage_routed, hga_attn_fwd_causal and
+ * hga_attn_bwd_causal wait for their stream and return HGA_ERR_DEVICE_CHECK
+ * (outputs invalid, word cleared) when a check failed.  Release builds skip
+ * the checks and return without waiting.
+ * hga_checked_build: 1 in a checked build, else 0.
+ * hga_device_check: *word = the first failed check's site code (0: none);
+ * `clear` != 0 resets it.  Synchronises with the device. */
+int hga_checked_build(void);
+int hga_device_check(int* word, int clear);
+
+/* Failure-path self-test.  The article has no counterpart: this call lets a
+ * caller (or a test) check that the library's bounded waits end cleanly.
+ * It launches one CTA on `stream` that allocates tensor memory, waits on an
+ * mbarrier nothing arrives at until `limit_us` microseconds pass, records
+ * its code (written to *site when site is not NULL) in the status word that
+ * hga_device_status reads, frees the tensor memory and returns.  The device
+ * stays usable.  HGA_ERR_INVALID_ARG unless 1 <= limit_us <= 1000000. */
+int hga_selftest_wait(int limit_us, int* site, hga_stream_t stream);
 
 /* Message of the last failed call on this thread ("" if none). */
 const char* hga_last_error(void);
