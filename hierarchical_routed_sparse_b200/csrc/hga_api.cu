@@ -9,6 +9,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "hga_internal.cuh"
 
 namespace hga {
@@ -20,6 +22,16 @@ size_t attn_simt_smem(const Shape& s, bool backward);
 namespace {
 
 thread_local char g_err[512] = "";
+
+// An NVTX range around one ABI call, named after it: profilers (ncu --nvtx,
+// Nsight Systems) show the call and can select its kernels by the range.
+// Without a tool attached a push / pop is a test of a null function pointer.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 int fail(int code, const char* fmt, ...)
 {
@@ -179,6 +191,7 @@ const char* hga_version(void) { return "hga-b200 0.1 (sm_100a)"; }
 
 int hga_device_status(int* status, int clear)
 {
+    const NvtxRange nvtx_range("hga_device_status");
     if (!status) return fail(HGA_ERR_INVALID_ARG, "status is NULL");
     const int vf = hga::attn_fwd_tc_status(clear != 0);
     const int vb = hga::attn_bwd_tc_status(clear != 0);
@@ -192,6 +205,7 @@ int hga_device_status(int* status, int clear)
 
 int hga_device_check(int* word, int clear)
 {
+    const NvtxRange nvtx_range("hga_device_check");
     if (!word) return fail(HGA_ERR_INVALID_ARG, "word is NULL");
     const int w = read_check_words(clear != 0);
     if (w < 0) return fail(HGA_ERR_CUDA, "hga_device_check: the check word could not be read");
@@ -210,6 +224,7 @@ int hga_checked_build(void)
 
 int hga_selftest_wait(int limit_us, int* site, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_selftest_wait");
     if (limit_us < 1 || limit_us > 1000000)
         return fail(HGA_ERR_INVALID_ARG, "limit_us=%d outside [1, 1000000]", limit_us);
     if (site) *site = hga::selftest_site();
@@ -238,6 +253,7 @@ size_t hga_workspace_size(const hga_params* p)
 int hga_build_summaries(const hga_params* p, const void* K, int64_t t_begin, int64_t t_end,
                         float* csum, float* gsum, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_build_summaries");
     hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (t_begin < 0 || t_end < t_begin || t_end > s.T || t_begin % 64 || t_end % 64)
@@ -255,6 +271,7 @@ int hga_build_summaries(const hga_params* p, const void* K, int64_t t_begin, int
 int hga_build_summaries_rows(const hga_params* p, const void* K_rows, int64_t t_begin, int64_t t_end,
                              float* csum, float* gsum, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_build_summaries_rows");
     hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (t_begin < 0 || t_end < t_begin || t_end > s.T || t_begin % 64 || t_end % 64)
@@ -272,6 +289,7 @@ int hga_build_summaries_rows(const hga_params* p, const void* K_rows, int64_t t_
 int hga_route_chunks(const hga_params* p, const void* Q, const float* csum, float* qbar,
                      int32_t* cidx, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_route_chunks");
     hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
@@ -289,6 +307,7 @@ int hga_route_chunks(const hga_params* p, const void* Q, const float* csum, floa
 int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum, const int32_t* cidx,
                      int32_t* gidx, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_route_groups");
     hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
@@ -305,6 +324,7 @@ int hga_route_groups(const hga_params* p, const float* qbar, const float* gsum, 
 int hga_route(const hga_params* p, const void* Q, const float* csum, const float* gsum, float* qbar,
               int32_t* cidx, int32_t* gidx, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_route");
     hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
@@ -339,6 +359,7 @@ int hga_stage_routed(const hga_params* p, const void* K_hist, const void* V_hist
                      const void* V_seg, const int32_t* gidx, void* K_stage, void* V_stage, int32_t* gidx_stage,
                      hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_stage_routed");
     hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
@@ -367,6 +388,7 @@ int hga_decode(const hga_params* p, int64_t pos, const void* q, const void* K, c
                const float* csum, const float* gsum, float* O, float* lse, int32_t* cidx, int32_t* gidx,
                hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_decode");
     hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (pos < 0 || pos >= s.T)
@@ -404,6 +426,7 @@ static int causal_shape(const hga_params* p, hga::Shape* s)
 int hga_route_causal(const hga_params* p, const void* Q, const float* csum, const float* gsum, int32_t* cidx,
                      int32_t* gidx, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_route_causal");
     hga::Shape s{};
     if (int r = causal_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
@@ -422,6 +445,7 @@ int hga_route_causal(const hga_params* p, const void* Q, const float* csum, cons
 int hga_attn_fwd_causal(const hga_params* p, const void* Q, const void* K, const void* V, const int32_t* gidx,
                         float* O, float* lse, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_attn_fwd_causal");
     hga::Shape s{};
     if (int r = causal_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
@@ -439,6 +463,7 @@ int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K, const
                         const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK_seg,
                         float* dV_seg, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_attn_bwd_causal");
     hga::Shape s{};
     if (int r = causal_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
@@ -460,6 +485,7 @@ int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K, const
 int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* V,
                  const int32_t* gidx, float* O, float* lse, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_attn_fwd");
     hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
@@ -482,6 +508,7 @@ int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* 
                  const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK_seg,
                  float* dV_seg, void* workspace, size_t ws_bytes, hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_attn_bwd");
     hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
@@ -564,6 +591,7 @@ extern "C" int hga_attn_bwd_noalloc(const hga_params* p, const void* Q, const vo
                                     const int32_t* gidx, float* dQ, float* dK_seg, float* dV_seg,
                                     hga_stream_t stream)
 {
+    const NvtxRange nvtx_range("hga_attn_bwd_noalloc");
     hga::Shape s{};
     if (int r = make_shape(p, &s)) return r;
     if (s.nQB == 0) return HGA_OK;
