@@ -45,7 +45,7 @@ class _Params(ctypes.Structure):
                 ("d", ctypes.c_int), ("T_hist", ctypes.c_int64), ("T_seg", ctypes.c_int64),
                 ("chunk", ctypes.c_int), ("group", ctypes.c_int), ("qblock", ctypes.c_int),
                 ("k_c", ctypes.c_int), ("k_g", ctypes.c_int), ("scale", ctypes.c_float),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("kv_capacity", ctypes.c_int64)]
 
 
 @dataclass
@@ -64,6 +64,7 @@ class Params:
     chunk: int = 64
     group: int = 8
     qblock: int = 64
+    kv_capacity: int = 0     # rows per (batch, kv-head) of K / V / summaries; 0 = T
 
     @staticmethod
     def from_workload(w) -> "Params":
@@ -79,12 +80,19 @@ class Params:
         return self.T_seg // 64
 
     @property
+    def cap(self) -> int:
+        """Rows per (batch, kv-head) of the K / V buffers (and 64x / 8x the
+        rows of the chunk / group summaries)."""
+        return self.kv_capacity or self.T
+
+    @property
     def torch_dtype(self):
         return torch.bfloat16 if self.dtype == HGA_BF16 else torch.float32
 
     def c(self) -> _Params:
         return _Params(self.B, self.Hq, self.Hkv, self.d, self.T_hist, self.T_seg, self.chunk,
-                       self.group, self.qblock, self.k_c, self.k_g, float(self.scale), self.dtype)
+                       self.group, self.qblock, self.k_c, self.k_g, float(self.scale), self.dtype,
+                       self.kv_capacity)
 
 
 _lib = None
@@ -322,8 +330,8 @@ class CausalBuffers:
         B, Hq, Hkv, d, T, Ts = p.B, p.Hq, p.Hkv, p.d, p.T, p.T_seg
         f32 = dict(device=device, dtype=torch.float32)
         i32 = dict(device=device, dtype=torch.int32)
-        self.csum = torch.zeros(B, Hkv, T // 64, d, **f32)
-        self.gsum = torch.zeros(B, Hkv, T // 8, d, **f32)
+        self.csum = torch.zeros(B, Hkv, p.cap // 64, d, **f32)
+        self.gsum = torch.zeros(B, Hkv, p.cap // 8, d, **f32)
         self.cidx = torch.empty(B, Hkv, Ts, wc, **i32)
         self.gidx = torch.empty(B, Hkv, Ts, wg, **i32)
         self.O = torch.empty(B, Hq, Ts, d, **f32)
@@ -368,10 +376,10 @@ class DecodeState:
         B, Hq, Hkv, d, T = p.B, p.Hq, p.Hkv, p.d, p.T
         f32 = dict(device=device, dtype=torch.float32)
         i32 = dict(device=device, dtype=torch.int32)
-        self.K = torch.zeros(B, Hkv, T, d, device=device, dtype=p.torch_dtype)
-        self.V = torch.zeros(B, Hkv, T, d, device=device, dtype=p.torch_dtype)
-        self.csum = torch.zeros(B, Hkv, T // 64, d, **f32)
-        self.gsum = torch.zeros(B, Hkv, T // 8, d, **f32)
+        self.K = torch.zeros(B, Hkv, p.cap, d, device=device, dtype=p.torch_dtype)
+        self.V = torch.zeros(B, Hkv, p.cap, d, device=device, dtype=p.torch_dtype)
+        self.csum = torch.zeros(B, Hkv, p.cap // 64, d, **f32)
+        self.gsum = torch.zeros(B, Hkv, p.cap // 8, d, **f32)
         self.O = torch.empty(B, Hq, d, **f32)
         self.lse = torch.empty(B, Hq, **f32)
         self.cidx = torch.empty(B, Hkv, wc, **i32)
@@ -442,8 +450,8 @@ class Buffers:
         B, Hq, Hkv, d, T, Ts, nQB = p.B, p.Hq, p.Hkv, p.d, p.T, p.T_seg, p.nQB
         f32 = dict(device=device, dtype=torch.float32)
         i32 = dict(device=device, dtype=torch.int32)
-        self.csum = torch.zeros(B, Hkv, T // 64, d, **f32)
-        self.gsum = torch.zeros(B, Hkv, T // 8, d, **f32)
+        self.csum = torch.zeros(B, Hkv, p.cap // 64, d, **f32)
+        self.gsum = torch.zeros(B, Hkv, p.cap // 8, d, **f32)
         self.qbar = torch.empty(B, Hkv, nQB, d, **f32)
         self.cidx = torch.empty(B, Hkv, nQB, wc, **i32)
         self.gidx = torch.empty(B, Hkv, nQB, wg, **i32)

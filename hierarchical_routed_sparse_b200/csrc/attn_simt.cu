@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads)
 attn_fwd_simt_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K,
                      const TIn* __restrict__ V, const int32_t* __restrict__ gidx,
                      float* __restrict__ O, float* __restrict__ lse,
-                     int Hq, int Hkv, int G, int64_t T_hist, int64_t T_seg, int64_t nQB, int wg,
+                     int Hq, int Hkv, int G, int64_t T_hist, int64_t T_seg, int64_t nQB, int64_t cap, int wg,
                      float scale_log2)
 {
     constexpr int DP = padded<D>(), NC = D / 16;
@@ -135,12 +135,11 @@ attn_fwd_simt_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K,
     const int64_t bhq = blockIdx.x;               // ((b*Hq)+h)*nQB + qb
     const int64_t qb = bhq % nQB, bh = bhq / nQB;
     const int64_t b = bh / Hq, h = bh % Hq, g = h / G;
-    const int64_t T = T_hist + T_seg;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
 
     const TIn* Qrow0 = Q + (bh * T_seg + qb * kTile) * D;
-    const TIn* Kh = K + (b * Hkv + g) * T * D;
-    const TIn* Vh = V + (b * Hkv + g) * T * D;
+    const TIn* Kh = K + (b * Hkv + g) * cap * D;     // K / V rows of (b, g): cap apart
+    const TIn* Vh = V + (b * Hkv + g) * cap * D;
     const int n_groups = count_valid(gidx + ((b * Hkv + g) * nQB + qb) * wg, wg, s_groups,
                                      (T_hist + qb * kTile) / kGroup, chk::kSiteSimtFwd);
     const int n_routed_tiles = (n_groups + 7) / 8;
@@ -245,7 +244,7 @@ attn_bwd_simt_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K,
                      const TIn* __restrict__ dO, const float* __restrict__ Drow,
                      const int32_t* __restrict__ gidx, float* __restrict__ dQ,
                      float* __restrict__ dK_seg, float* __restrict__ dV_seg,
-                     int Hq, int Hkv, int G, int64_t T_hist, int64_t T_seg, int64_t nQB, int wg,
+                     int Hq, int Hkv, int G, int64_t T_hist, int64_t T_seg, int64_t nQB, int64_t cap, int wg,
                      float scale, float scale_log2)
 {
     constexpr int DP = padded<D>(), NC = D / 16, PP = kTile + 1;
@@ -261,12 +260,11 @@ attn_bwd_simt_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K,
     const int64_t bhq = blockIdx.x;
     const int64_t qb = bhq % nQB, bh = bhq / nQB;
     const int64_t b = bh / Hq, h = bh % Hq, g = h / G;
-    const int64_t T = T_hist + T_seg;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
 
     const int64_t row0 = bh * T_seg + qb * kTile;
-    const TIn* Kh = K + (b * Hkv + g) * T * D;
-    const TIn* Vh = V + (b * Hkv + g) * T * D;
+    const TIn* Kh = K + (b * Hkv + g) * cap * D;     // K / V rows of (b, g): cap apart
+    const TIn* Vh = V + (b * Hkv + g) * cap * D;
     float* dKh = dK_seg + (b * Hkv + g) * T_seg * D;
     float* dVh = dV_seg + (b * Hkv + g) * T_seg * D;
     const int n_groups = count_valid(gidx + ((b * Hkv + g) * nQB + qb) * wg, wg, s_groups,
@@ -392,7 +390,7 @@ cudaError_t launch_fwd(const Shape& s, const void* Q, const void* K, const void*
     const int64_t blocks = (int64_t)s.B * s.Hq * s.nQB;
     k<<<(unsigned)blocks, kThreads, smem, st>>>(
         static_cast<const TIn*>(Q), static_cast<const TIn*>(K), static_cast<const TIn*>(V), gidx, O,
-        lse, s.Hq, s.Hkv, s.G, s.T_hist, s.T_seg, s.nQB, s.wg, s.scale * kLog2e);
+        lse, s.Hq, s.Hkv, s.G, s.T_hist, s.T_seg, s.nQB, s.cap, s.wg, s.scale * kLog2e);
     return cudaGetLastError();
 }
 
@@ -417,7 +415,7 @@ cudaError_t launch_bwd(const Shape& s, const void* Q, const void* K, const void*
     k<<<(unsigned)blocks, kThreads, smem, st>>>(
         static_cast<const TIn*>(Q), static_cast<const TIn*>(K), static_cast<const TIn*>(V), lse,
         static_cast<const TIn*>(dO), Drow, gidx, dQ, dK_seg, dV_seg, s.Hq, s.Hkv, s.G, s.T_hist,
-        s.T_seg, s.nQB, s.wg, s.scale, s.scale * kLog2e);
+        s.T_seg, s.nQB, s.cap, s.wg, s.scale, s.scale * kLog2e);
     return cudaGetLastError();
 }
 

@@ -114,6 +114,7 @@ struct BwdArgs {
     float* dV;
     int Hq, Hkv, G, wg;
     int64_t T_hist, T_seg, nQB, n_items;
+    int64_t cap;               // K / V rows per (batch, kv-head)
     int q_rows;
     float scale, scale_log2;
 };
@@ -311,7 +312,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const Item m = make_item(a, tab, k, lane);
             const int nt = m.nt(), n_rt = m.n_rt();
             const int32_t* grow = m.grow(a);
-            const int64_t kv_base = (int64_t)m.bg * (a.T_hist + a.T_seg);
+            const int64_t kv_base = (int64_t)m.bg * a.cap;
             for (int p = 0; p < nt && ok; ++p, ++gt) {
                 const int t = nt - 1 - p;
                 const int ks = gt % kKStages, vs = gt % kVStages;
@@ -902,7 +903,7 @@ int attn_bwd_tc_status(bool clear)
 
 bool attn_bwd_tc_supported(const Shape& s)
 {
-    const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
+    const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.cap;
     return s.dtype == HGA_BF16 && s.d == D && q_rows < (1ull << 31) && kv_rows < (1ull << 31) &&
            tensor_maps_available();
 }
@@ -931,7 +932,7 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
                                reinterpret_cast<float4*>(dK_seg), reinterpret_cast<float4*>(dV_seg), n4, sa);
     if (e != cudaSuccess) return e;
     CUtensorMap tq, tdo, tk8, tv8, tk64, tv64, tdq;
-    const uint64_t q_rows = (uint64_t)rows, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
+    const uint64_t q_rows = (uint64_t)rows, kv_rows = (uint64_t)s.B * s.Hkv * s.cap;
     if (!make_bf16_map(&tq, Q, q_rows, D, 64) || !make_bf16_map(&tdo, dO, q_rows, D, 64) ||
         !make_bf16_map(&tk8, K, kv_rows, D, 8) || !make_bf16_map(&tv8, V, kv_rows, D, 8) ||
         !make_bf16_map(&tk64, K, kv_rows, D, 64) || !make_bf16_map(&tv64, V, kv_rows, D, 64) ||
@@ -951,6 +952,7 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
     a.T_hist = s.T_hist;
     a.T_seg = s.T_seg;
     a.nQB = s.nQB;
+    a.cap = s.cap;
     a.q_rows = (int)q_rows;
     a.scale = s.scale;
     a.scale_log2 = s.scale * kLog2e;

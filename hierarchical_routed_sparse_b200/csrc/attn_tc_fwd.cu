@@ -82,7 +82,8 @@ struct FwdArgs {
     int Hq, Hkv, G, wg;
     int64_t T_hist, T_seg, nQB;
     int q_rows;          // B*Hq*T_seg (rows of the Q map)
-    int kv_rows;         // B*Hkv*T
+    int kv_rows;         // B*Hkv*cap (rows of the K / V maps)
+    int64_t cap;         // K / V rows per (batch, kv-head)
     float scale_log2;
 };
 
@@ -165,7 +166,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     constexpr uint32_t kColO = 0;
     auto col_s = [&](int bb) { return uint32_t(D + bb * kKeys); };
 
-    const int64_t kv_base = bg * (a.T_hist + a.T_seg);      // first K/V row of (b, g)
+    const int64_t kv_base = bg * a.cap;                      // first K/V row of (b, g)
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
@@ -445,7 +446,7 @@ cudaError_t launch(const Shape& s, const void* Q, const void* K, const void* V, 
                    float* O, float* lse, cudaStream_t st)
 {
     CUtensorMap tq, tk8, tv8, tk64, tv64;
-    const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
+    const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.cap;
     if (!make_bf16_map(&tq, Q, q_rows, D, 64) || !make_bf16_map(&tk8, K, kv_rows, D, 8) ||
         !make_bf16_map(&tv8, V, kv_rows, D, 8) || !make_bf16_map(&tk64, K, kv_rows, D, 64) ||
         !make_bf16_map(&tv64, V, kv_rows, D, 64))
@@ -463,6 +464,7 @@ cudaError_t launch(const Shape& s, const void* Q, const void* K, const void* V, 
     a.nQB = s.nQB;
     a.q_rows = (int)q_rows;
     a.kv_rows = (int)kv_rows;
+    a.cap = s.cap;
     a.scale_log2 = s.scale * kLog2e;
     // One head pair per CTA, two CTAs per SM.
     auto k = attn_fwd_tc_kernel<D>;
@@ -488,7 +490,7 @@ int attn_fwd_tc_status(bool clear)
 
 bool attn_fwd_tc_supported(const Shape& s)
 {
-    const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.T;
+    const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.cap;
     return s.dtype == HGA_BF16 && (s.d == 128 || s.d == 64) && q_rows < (1ull << 31) &&
            kv_rows < (1ull << 31) && tensor_maps_available();
 }

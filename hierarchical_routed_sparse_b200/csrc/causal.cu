@@ -114,14 +114,14 @@ template <typename TIn, int D>
 __global__ void __launch_bounds__(kThreads)
 causal_route_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, const float* __restrict__ gsum,
                     int32_t* __restrict__ cidx, int32_t* __restrict__ gidx, int Hq, int Hkv, int G,
-                    int64_t T_hist, int64_t T_seg, int k_c, int wc, int k_g, int wg)
+                    int64_t T_hist, int64_t T_seg, int64_t cap, int k_c, int wc, int k_g, int wg)
 {
     pdl_wait();
     pdl_trigger();
     constexpr int P = D / 32;
     extern __shared__ __align__(16) uint8_t sm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t T = T_hist + T_seg, nC = T / kChunk, nG = T / kGroup;
+    const int64_t T = T_hist + T_seg, nC = T / kChunk, nCs = cap / kChunk, nGs = cap / kGroup;
     const RouteWarpLayout L = route_warp_layout(nC, wc, D);
     uint8_t* ws = sm + (size_t)warp * L.total;
     unsigned long long* keys = reinterpret_cast<unsigned long long*>(ws + L.keys);
@@ -155,7 +155,7 @@ causal_route_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, c
             crow_out[j] = v;
         }
     } else {
-        const float* cs = csum + bg * nC * D;
+        const float* cs = csum + bg * nCs * D;
         score_candidates<D, 1>(qs, c0, [&](int c, const float*& r) { r = cs + (int64_t)c * D; return c; }, keys, 0,
                                lane);
         __syncwarp();
@@ -170,7 +170,7 @@ causal_route_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, c
     if (k_g <= 0 || k_g >= n) {
         for (int j = lane; j < wg; j += 32) grow_out[j] = j < n ? ids[j] : -1;
     } else {
-        const float* gs = gsum + bg * nG * D;
+        const float* gs = gsum + bg * nGs * D;
         score_candidates<D, 1>(qs, n, [&](int c, const float*& r) { r = gs + (int64_t)ids[c] * D; return ids[c]; },
                                keys, 0, lane);
         __syncwarp();
@@ -285,7 +285,7 @@ template <typename TIn, int D, int GM>
 __global__ void __launch_bounds__(kThreads, GM <= 4 ? 2 : 1)
 causal_fwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TIn* __restrict__ V,
                   const int32_t* __restrict__ gidx, float* __restrict__ O, float* __restrict__ lse, int Hq, int Hkv,
-                  int G, int64_t T_hist, int64_t T_seg, int wg, float scale)
+                  int G, int64_t T_hist, int64_t T_seg, int64_t cap, int wg, float scale)
 {
     pdl_wait();
     pdl_trigger();
@@ -299,8 +299,8 @@ causal_fwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
     const int32_t* grow = gidx + row * wg;
     const int n_g = prefix_count(grow, wg, lane);
     const int n_keys = kGroup * n_g + int(pos - own0) + 1;
-    const TIn* Kb = K + bg * T * D;
-    const TIn* Vb = V + bg * T * D;
+    const TIn* Kb = K + bg * cap * D;            // K / V rows of (b, g): cap apart
+    const TIn* Vb = V + bg * cap * D;
     float* qw = qsm[warp];
     for (int h = 0; h < G; ++h) {
         float x[P];
@@ -398,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, GM <= 4 ? 2 : 1)
 causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TIn* __restrict__ V,
                   const float* __restrict__ O, const float* __restrict__ lse, const TIn* __restrict__ dO,
                   const int32_t* __restrict__ gidx, float* __restrict__ dQ, float* __restrict__ dK_seg,
-                  float* __restrict__ dV_seg, int Hq, int Hkv, int G, int64_t T_hist, int64_t T_seg, int wg,
-                  float scale)
+                  float* __restrict__ dV_seg, int Hq, int Hkv, int G, int64_t T_hist, int64_t T_seg, int64_t cap,
+                  int wg, float scale)
 {
     pdl_wait();
     pdl_trigger();
@@ -413,8 +413,8 @@ causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
     const int32_t* grow = gidx + row * wg;
     const int n_g = prefix_count(grow, wg, lane);
     const int n_keys = kGroup * n_g + int(pos - own0) + 1;
-    const TIn* Kb = K + bg * T * D;
-    const TIn* Vb = V + bg * T * D;
+    const TIn* Kb = K + bg * cap * D;            // K / V rows of (b, g): cap apart
+    const TIn* Vb = V + bg * cap * D;
     float* dKb = dK_seg + bg * T_seg * D + lane * P;
     float* dVb = dV_seg + bg * T_seg * D + lane * P;
     float* qw = bsm + (size_t)warp * 2 * GM * D;
@@ -511,7 +511,7 @@ cudaError_t launch_route(const Shape& s, const void* Q, const float* csum, const
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)(s.B * s.Hkv * s.T_seg / kWarps);
     return launch_pdl(k, dim3(grid), dim3(kThreads), smem, st, static_cast<const TIn*>(Q), csum, gsum, cidx, gidx,
-                      s.Hq, s.Hkv, s.G, s.T_hist, s.T_seg, s.k_c, s.wc, s.k_g, s.wg);
+                      s.Hq, s.Hkv, s.G, s.T_hist, s.T_seg, s.cap, s.k_c, s.wc, s.k_g, s.wg);
 }
 
 template <typename TIn, int D, int GM>
@@ -521,7 +521,7 @@ cudaError_t launch_fwd(const Shape& s, const void* Q, const void* K, const void*
     const unsigned grid = (unsigned)(s.B * s.Hkv * s.T_seg / kWarps);
     return launch_pdl(causal_fwd_kernel<TIn, D, GM>, dim3(grid), dim3(kThreads), 0, st, static_cast<const TIn*>(Q),
                       static_cast<const TIn*>(K), static_cast<const TIn*>(V), gidx, O, lse, s.Hq, s.Hkv, s.G,
-                      s.T_hist, s.T_seg, s.wg, s.scale);
+                      s.T_hist, s.T_seg, s.cap, s.wg, s.scale);
 }
 
 template <typename TIn, int D, int GM>
@@ -538,7 +538,7 @@ cudaError_t launch_bwd(const Shape& s, const void* Q, const void* K, const void*
     if ((e = allow_smem(k, (int)smem)) != cudaSuccess) return e;
     return launch_pdl(k, dim3(grid), dim3(kThreads), smem, st, static_cast<const TIn*>(Q),
                       static_cast<const TIn*>(K), static_cast<const TIn*>(V), O, lse, static_cast<const TIn*>(dO),
-                      gidx, dQ, dK, dV, s.Hq, s.Hkv, s.G, s.T_hist, s.T_seg, s.wg, s.scale);
+                      gidx, dQ, dK, dV, s.Hq, s.Hkv, s.G, s.T_hist, s.T_seg, s.cap, s.wg, s.scale);
 }
 
 // Dispatch over input type, head dim and the bound on heads per kv-head.

@@ -131,12 +131,12 @@ __global__ void __launch_bounds__(kRouterThreads, 2)
 decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ K, const TIn* __restrict__ V,
               const float* __restrict__ csum, const float* __restrict__ gsum, float* __restrict__ O,
               float* __restrict__ lse, int32_t* __restrict__ cidx, int32_t* __restrict__ gidx, int Hq, int Hkv,
-              int G, int64_t T, int64_t pos, int k_c, int wc, int k_g, int wg, float scale)
+              int G, int64_t T, int64_t cap, int64_t pos, int k_c, int wc, int k_g, int wg, float scale)
 {
     constexpr int P = D / 32;                        // elements of a row per lane
     constexpr uint32_t kRowBytes = D * sizeof(TIn);
     extern __shared__ __align__(128) uint8_t sm[];
-    const int64_t nC = T / kChunk, nG = T / kGroup;
+    const int64_t nC = T / kChunk, nCs = cap / kChunk, nGs = cap / kGroup;
     const DecodeLayout L = decode_layout(nC, wc, wg, G, D, (int)sizeof(TIn));
     unsigned long long* ckeys = reinterpret_cast<unsigned long long*>(sm + L.ckeys);
     unsigned long long* gkeys = reinterpret_cast<unsigned long long*>(sm + L.gkeys);
@@ -159,8 +159,8 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ K, const TIn* _
     const uint32_t r = cluster_rank();
     const int64_t bg = blockIdx.x / kS;
     const int64_t b = bg / Hkv, g = bg % Hkv;
-    const TIn* Kb = K + bg * T * D;
-    const TIn* Vb = V + bg * T * D;
+    const TIn* Kb = K + bg * cap * D;                // K / V rows of (b, g): cap apart
+    const TIn* Vb = V + bg * cap * D;
 
     if (tid == 0) {
         mbar_init(bar_own, 1);
@@ -184,7 +184,7 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ K, const TIn* _
     const int own_r = has_own ? min(kGroup, own_rows - kGroup * (int)r) : 0;
     const bool score_c = k_c > 0 && k_c < c0;
     const int cb = (int)r * c0 / kS, ce = ((int)r + 1) * c0 / kS;
-    const float* cs = csum + bg * nC * D;
+    const float* cs = csum + bg * nCs * D;
     if (tid == 0) {
         if (has_own) {
             const int64_t t0 = (int64_t)c0 * kChunk + kGroup * r;
@@ -239,7 +239,7 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ K, const TIn* _
     const bool score_g = k_g > 0 && k_g < n_cand;
     if (score_g) {
         const int gb = (int)r * n_cand / kS, ge = ((int)r + 1) * n_cand / kS;
-        const float* gs = gsum + bg * nG * D;
+        const float* gs = gsum + bg * nGs * D;
         score_candidates<D>(qs, ge - gb,
                             [&](int c, const float*& row) { row = gs + (int64_t)ids[gb + c] * D; return ids[gb + c]; },
                             gkeys + gb, warp, lane);
@@ -443,7 +443,7 @@ cudaError_t launch(const Shape& s, int64_t pos, const void* q, const void* K, co
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, k, static_cast<const TIn*>(q), static_cast<const TIn*>(K),
                               static_cast<const TIn*>(V), csum, gsum, O, lse, cidx, gidx, s.Hq, s.Hkv, s.G, s.T,
-                              pos, s.k_c, s.wc, s.k_g, s.wg, s.scale);
+                              s.cap, pos, s.k_c, s.wc, s.k_g, s.wg, s.scale);
 }
 
 }  // namespace

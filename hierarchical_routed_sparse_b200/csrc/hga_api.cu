@@ -123,6 +123,13 @@ int make_shape(const hga_params* p, hga::Shape* s)
     s->B = p->B; s->Hq = p->Hq; s->Hkv = p->Hkv; s->G = p->Hq / p->Hkv; s->d = p->d;
     s->T_hist = p->T_hist; s->T_seg = p->T_seg; s->T = T;
     s->nC = T / hga::kChunk; s->nG = T / hga::kGroup; s->nQB = p->T_seg / hga::kChunk;
+    if (p->kv_capacity != 0 && (p->kv_capacity < T || p->kv_capacity % 64))
+        return fail(HGA_ERR_INVALID_ARG, "kv_capacity (%lld) must be 0 or a multiple of 64 >= T_hist + T_seg (%lld)",
+                    (long long)p->kv_capacity, (long long)T);
+    s->cap = p->kv_capacity ? p->kv_capacity : T;
+    if (s->cap / hga::kGroup > INT32_MAX)
+        return fail(HGA_ERR_UNSUPPORTED, "kv_capacity of %lld rows overflows int32 group indices", (long long)s->cap);
+    s->nCs = s->cap / hga::kChunk; s->nGs = s->cap / hga::kGroup;
     s->k_c = p->k_c == HGA_ALL ? 0 : p->k_c;
     s->k_g = p->k_g == HGA_ALL ? 0 : p->k_g;
     const int64_t wc = p->k_c == HGA_ALL ? (s->nC > 0 ? s->nC : 1) : p->k_c;
@@ -263,7 +270,7 @@ int hga_build_summaries(const hga_params* p, const void* K, int64_t t_begin, int
     CHECK_PTR(K);
     CHECK_PTR(csum);
     CHECK_PTR(gsum);
-    cudaError_t e = hga::launch_summaries(s, K, s.T, 0, t_begin / 64, t_end / 64, csum, gsum,
+    cudaError_t e = hga::launch_summaries(s, K, s.cap, 0, t_begin / 64, t_end / 64, csum, gsum,
                                           static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_build_summaries");
 }
@@ -348,6 +355,7 @@ int hga_stage_params(const hga_params* p, hga_params* staged)
     if (!staged) return fail(HGA_ERR_INVALID_ARG, "staged is NULL");
     *staged = *p;
     staged->T_hist = hga::stage_hist_rows(s);
+    staged->kv_capacity = 0;                   // the staging buffers are dense
     // The staged problem keeps the routing's row widths: with HGA_ALL they
     // would otherwise follow the staged T.
     staged->k_c = s.wc;

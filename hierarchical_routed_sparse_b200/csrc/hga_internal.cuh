@@ -21,6 +21,8 @@ struct Shape {
     int B, Hq, Hkv, G, d;
     int64_t T_hist, T_seg, T;
     int64_t nC, nG, nQB;     // chunks, groups (whole context), query blocks
+    int64_t cap;             // K / V rows per (batch, kv-head) (row stride of K, V)
+    int64_t nCs, nGs;        // row strides of csum / gsum per (batch, kv-head): cap / 64, cap / 8
     int k_c, k_g;            // <= 0: keep all eligible
     int wc, wg;              // index row widths
     float scale;

@@ -100,7 +100,7 @@ template <typename TIn, int D>
 __global__ void __launch_bounds__(kRouterThreads, 2)
 route_chunks_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum,
                     float* __restrict__ qbar, int32_t* __restrict__ cidx,
-                    int Hq, int Hkv, int G, int64_t T_seg, int64_t nQB, int64_t nC,
+                    int Hq, int Hkv, int G, int64_t T_seg, int64_t nQB, int64_t nCs,
                     int64_t c_hist, int k_c, int wc, float inv_rows)
 {
     constexpr int RL = kRouterThreads / (D / Vec16<TIn>::E);
@@ -113,7 +113,7 @@ route_chunks_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum,
     const int64_t qb = u % nQB, bg = u / nQB;
     const int64_t b = bg / Hkv, g = bg % Hkv;
     block_query<TIn, D>(Q, qbar + u * D, qs, part, b, g, qb, Hq, G, T_seg, inv_rows, threadIdx.x);
-    route_chunks_block<D>(qs, csum + bg * nC * D, static_cast<int>(c_hist + qb), k_c, wc, keys, cidx + u * wc,
+    route_chunks_block<D>(qs, csum + bg * nCs * D, static_cast<int>(c_hist + qb), k_c, wc, keys, cidx + u * wc,
                           nullptr, threadIdx.x);
 }
 
@@ -122,7 +122,7 @@ template <int D>
 __global__ void __launch_bounds__(kRouterThreads, 2)
 route_groups_kernel(const float* __restrict__ qbar, const float* __restrict__ gsum,
                     const int32_t* __restrict__ cidx, int32_t* __restrict__ gidx,
-                    int64_t nQB, int64_t nG, int wc, int k_g, int wg, int64_t c_hist)
+                    int64_t nQB, int64_t nGs, int wc, int k_g, int wg, int64_t c_hist)
 {
     extern __shared__ unsigned long long keys[];      // [8*wc], ids [8*wc], flags [8*wc]
     int32_t* ids = reinterpret_cast<int32_t*>(keys + (size_t)kGroupsPerChunk * wc);
@@ -136,7 +136,7 @@ route_groups_kernel(const float* __restrict__ qbar, const float* __restrict__ gs
     for (int col = threadIdx.x; col < D; col += kRouterThreads) qs[col] = qbar[u * D + col];
     __syncthreads();
     // The caller's chunk row: valid chunks lie before the block's own chunk.
-    route_groups_block<D>(qs, gsum + bg * nG * D, cidx + u * wc, wc, k_g, wg, keys, ids, flags, &n_valid,
+    route_groups_block<D>(qs, gsum + bg * nGs * D, cidx + u * wc, wc, k_g, wg, keys, ids, flags, &n_valid,
                           gidx + u * wg, threadIdx.x, c_hist + u % nQB);
 }
 
@@ -145,7 +145,7 @@ template <typename TIn, int D>
 __global__ void __launch_bounds__(kRouterThreads, 2)
 route_fused_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, const float* __restrict__ gsum,
                    float* __restrict__ qbar, int32_t* __restrict__ cidx, int32_t* __restrict__ gidx,
-                   int Hq, int Hkv, int G, int64_t T_seg, int64_t nQB, int64_t nC, int64_t nG,
+                   int Hq, int Hkv, int G, int64_t T_seg, int64_t nQB, int64_t nC, int64_t nCs, int64_t nGs,
                    int64_t c_hist, int k_c, int wc, int k_g, int wg, float inv_rows)
 {
     constexpr int RL = kRouterThreads / (D / Vec16<TIn>::E);
@@ -164,9 +164,9 @@ route_fused_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, co
     const int64_t qb = u % nQB, bg = u / nQB;
     const int64_t b = bg / Hkv, g = bg % Hkv;
     block_query<TIn, D>(Q, qbar + u * D, qs, part, b, g, qb, Hq, G, T_seg, inv_rows, threadIdx.x);
-    route_chunks_block<D>(qs, csum + bg * nC * D, static_cast<int>(c_hist + qb), k_c, wc, keys, cidx + u * wc,
+    route_chunks_block<D>(qs, csum + bg * nCs * D, static_cast<int>(c_hist + qb), k_c, wc, keys, cidx + u * wc,
                           crow, threadIdx.x);
-    route_groups_block<D>(qs, gsum + bg * nG * D, crow, wc, k_g, wg, keys, ids, flags, &n_valid, gidx + u * wg,
+    route_groups_block<D>(qs, gsum + bg * nGs * D, crow, wc, k_g, wg, keys, ids, flags, &n_valid, gidx + u * wg,
                           threadIdx.x);
 }
 
@@ -182,7 +182,7 @@ cudaError_t launch_rc(const Shape& s, const void* Q, const float* csum, float* q
     }
     const int64_t blocks = (int64_t)s.B * s.Hkv * s.nQB;
     return launch_pdl(k, dim3((unsigned)blocks), dim3(kRouterThreads), smem, st, static_cast<const TIn*>(Q), csum,
-                      qbar, cidx, s.Hq, s.Hkv, s.G, s.T_seg, s.nQB, s.nC, s.T_hist / kChunk, s.k_c, s.wc,
+                      qbar, cidx, s.Hq, s.Hkv, s.G, s.T_seg, s.nQB, s.nCs, s.T_hist / kChunk, s.k_c, s.wc,
                       1.0f / (float)(s.G * kChunk));
 }
 
@@ -198,7 +198,7 @@ cudaError_t launch_rg(const Shape& s, const float* qbar, const float* gsum, cons
     }
     const int64_t blocks = (int64_t)s.B * s.Hkv * s.nQB;
     return launch_pdl(k, dim3((unsigned)blocks), dim3(kRouterThreads), smem, st, qbar, gsum, cidx, gidx, s.nQB,
-                      s.nG, s.wc, s.k_g, s.wg, s.T_hist / kChunk);
+                      s.nGs, s.wc, s.k_g, s.wg, s.T_hist / kChunk);
 }
 
 template <typename TIn, int D>
@@ -213,8 +213,8 @@ cudaError_t launch_rf(const Shape& s, const void* Q, const float* csum, const fl
     }
     const int64_t blocks = (int64_t)s.B * s.Hkv * s.nQB;
     return launch_pdl(k, dim3((unsigned)blocks), dim3(kRouterThreads), smem, st, static_cast<const TIn*>(Q), csum,
-                      gsum, qbar, cidx, gidx, s.Hq, s.Hkv, s.G, s.T_seg, s.nQB, s.nC, s.nG, s.T_hist / kChunk,
-                      s.k_c, s.wc, s.k_g, s.wg, 1.0f / (float)(s.G * kChunk));
+                      gsum, qbar, cidx, gidx, s.Hq, s.Hkv, s.G, s.T_seg, s.nQB, s.nC, s.nCs, s.nGs,
+                      s.T_hist / kChunk, s.k_c, s.wc, s.k_g, s.wg, 1.0f / (float)(s.G * kChunk));
 }
 
 }  // namespace

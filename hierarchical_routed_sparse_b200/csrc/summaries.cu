@@ -19,8 +19,8 @@ namespace {
 
 template <typename TIn, int D>
 __global__ void __launch_bounds__(kGroupsPerChunk * D / Vec16<TIn>::E)
-summaries_kernel(const TIn* __restrict__ K, int64_t T, int64_t T_src, int64_t row0, int64_t c_begin,
-                 int64_t n_chunks, float* __restrict__ csum, float* __restrict__ gsum)
+summaries_kernel(const TIn* __restrict__ K, int64_t nCs, int64_t nGs, int64_t T_src, int64_t row0,
+                 int64_t c_begin, int64_t n_chunks, float* __restrict__ csum, float* __restrict__ gsum)
 {
     constexpr int E = Vec16<TIn>::E;
     constexpr int V16 = D / E;                  // 16-byte vectors per row
@@ -45,7 +45,7 @@ summaries_kernel(const TIn* __restrict__ K, int64_t T, int64_t T_src, int64_t ro
         for (int t = 0; t < kGroup; ++t) a += x[t][e];
         acc[e] = a;
     }
-    float* gdst = gsum + (bg * (T / kGroup) + c * kGroupsPerChunk + r) * D + v * E;
+    float* gdst = gsum + (bg * nGs + c * kGroupsPerChunk + r) * D + v * E;
 #pragma unroll
     for (int e = 0; e < E; e += 4)
         *reinterpret_cast<float4*>(gdst + e) =
@@ -57,7 +57,7 @@ summaries_kernel(const TIn* __restrict__ K, int64_t T, int64_t T_src, int64_t ro
         float a = 0.f;
 #pragma unroll
         for (int q = 0; q < kGroupsPerChunk; ++q) a += part[q][col];
-        csum[(bg * (T / kChunk) + c) * D + col] = a * (1.0f / kChunk);
+        csum[(bg * nCs + c) * D + col] = a * (1.0f / kChunk);
     }
 }
 
@@ -69,7 +69,7 @@ cudaError_t launch(const Shape& s, const void* K, int64_t T_src, int64_t row0, i
     const int64_t blocks = n * s.B * s.Hkv;
     constexpr int threads = kGroupsPerChunk * D / Vec16<TIn>::E;
     return launch_pdl(summaries_kernel<TIn, D>, dim3((unsigned)blocks), dim3(threads), 0, st,
-                      static_cast<const TIn*>(K), s.T, T_src, row0, c_begin, n, csum, gsum);
+                      static_cast<const TIn*>(K), s.nCs, s.nGs, T_src, row0, c_begin, n, csum, gsum);
 }
 
 }  // namespace

@@ -11,7 +11,8 @@ the segment's summaries, the routing and the routed attention forward of
 libhga; its backward runs the routed backward with the forward's routing
 frozen and returns gradients for the segment's Q, K and V (history gets
 none).  ``HGASegmentLayer`` wraps it between real Q / K / V / O projections
-and keeps the KV cache and the summaries of the segments seen so far;
+and keeps the KV cache and the summaries of the segments seen so far in
+buffers that grow by doubling (the library reads them in place);
 ``run_tbptt`` trains a sequence segment by segment (truncated
 back-propagation through time).
 """
@@ -26,63 +27,113 @@ from . import binding as B
 
 
 class KVCache:
-    """History of one layer: K / V rows [B][Hkv][T_hist][d] (no gradient)
-    and their chunk / group summaries."""
+    """History of one layer, kept in preallocated buffers that grow by
+    doubling: K / V [B][Hkv][cap][d] (rows 0 .. n-1 in use, no gradient) and
+    their chunk / group summaries [B][Hkv][cap/64][d], [B][Hkv][cap/8][d].
+    A segment writes only its own rows, and the library reads the buffers in
+    place (hga_params.kv_capacity = cap), so a sequence of segments costs no
+    copies of the history beyond the occasional doubling."""
 
     def __init__(self):
-        self.K = None
-        self.V = None
-        self.csum = None
-        self.gsum = None
-        self.pending = None      # summaries including the segment in flight
+        self.K = self.V = self.csum = self.gsum = None
+        self.n = 0
 
     @property
     def T_hist(self) -> int:
+        return self.n
+
+    @property
+    def cap(self) -> int:
         return 0 if self.K is None else self.K.shape[2]
 
     def reset(self):
         self.__init__()
 
+    @torch.no_grad()
+    def reserve(self, B: int, Hkv: int, d: int, dtype, rows: int, device):
+        """Capacity for `rows` rows (a multiple of 64), keeping the rows in use."""
+        if self.K is not None and self.K.shape[2] >= rows:
+            return
+        cap = max(rows, 2 * self.cap)
+        K = torch.empty(B, Hkv, cap, d, device=device, dtype=dtype)
+        V = torch.empty_like(K)
+        csum = torch.zeros(B, Hkv, cap // 64, d, device=device, dtype=torch.float32)
+        gsum = torch.zeros(B, Hkv, cap // 8, d, device=device, dtype=torch.float32)
+        if self.n:
+            K[:, :, :self.n] = self.K[:, :, :self.n]
+            V[:, :, :self.n] = self.V[:, :, :self.n]
+            csum[:, :, :self.n // 64] = self.csum[:, :, :self.n // 64]
+            gsum[:, :, :self.n // 8] = self.gsum[:, :, :self.n // 8]
+        self.K, self.V, self.csum, self.gsum = K, V, csum, gsum
+
+
+class _SegmentBuffers:
+    """Per-segment outputs and scratch of one shape, reused segment after
+    segment (their sizes depend on the segment length and the routing
+    widths, not on the history)."""
+
+    def __init__(self, p: B.Params, device):
+        wc, wg = B.route_widths(p)
+        Bn, Hq, Hkv, d, Ts, nQB = p.B, p.Hq, p.Hkv, p.d, p.T_seg, p.nQB
+        f32 = dict(device=device, dtype=torch.float32)
+        i32 = dict(device=device, dtype=torch.int32)
+        self.key = (Bn, Hq, Hkv, d, Ts, wc, wg)
+        self.qbar = torch.empty(Bn, Hkv, nQB, d, **f32)
+        self.cidx = torch.empty(Bn, Hkv, nQB, wc, **i32)
+        self.gidx = torch.empty(Bn, Hkv, nQB, wg, **i32)
+        self.O = torch.empty(Bn, Hq, Ts, d, **f32)
+        self.lse = torch.empty(Bn, Hq, Ts, **f32)
+        self.dQ = torch.empty(Bn, Hq, Ts, d, **f32)
+        self.dK = torch.empty(Bn, Hkv, Ts, d, **f32)
+        self.dV = torch.empty(Bn, Hkv, Ts, d, **f32)
+        self.ws = torch.empty(max(1, math.ceil(B.workspace_size(p) / 4)), **f32)
+
 
 class HGAAttention(torch.autograd.Function):
     """O = routed attention of the segment's queries over the history and the
-    segment's own keys (forward of libhga); float32 output."""
+    segment's own keys (forward of libhga); float32 output.  The segment's
+    keys and values are written into the cache (rows T_hist .. T_hist + T_seg)
+    before the routing; the caller then advances the cache by T_seg rows."""
 
     @staticmethod
-    def forward(ctx, q, k, v, cache: KVCache, k_c: int, k_g: int):
+    def forward(ctx, q, k, v, cache: KVCache, k_c: int, k_g: int, bufs: dict):
         Bn, Hq, Ts, d = q.shape
         Hkv = k.shape[1]
         dtype = B.HGA_BF16 if q.dtype == torch.bfloat16 else B.HGA_FP32
-        p = B.Params(B=Bn, Hq=Hq, Hkv=Hkv, d=d, T_hist=cache.T_hist, T_seg=Ts, k_c=k_c, k_g=k_g, dtype=dtype)
-        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        Kall = k if cache.K is None else torch.cat([cache.K, k.detach()], dim=2).contiguous()
-        Vall = v if cache.V is None else torch.cat([cache.V, v.detach()], dim=2).contiguous()
-        buf = B.Buffers(p, device=q.device)
-        if cache.csum is not None:                    # history summaries are kept
-            buf.csum[:, :, :cache.csum.shape[2]] = cache.csum
-            buf.gsum[:, :, :cache.gsum.shape[2]] = cache.gsum
-        B.build_summaries_rows(p, k.detach(), p.T_hist, p.T, buf.csum, buf.gsum)
-        buf.route(q)
-        buf.forward(q, Kall, Vall)
-        ctx.p = p
-        ctx.buf = buf
-        ctx.save_for_backward(q, Kall, Vall)
+        T_hist = cache.n
+        cache.reserve(Bn, Hkv, d, q.dtype, T_hist + Ts, q.device)
+        p = B.Params(B=Bn, Hq=Hq, Hkv=Hkv, d=d, T_hist=T_hist, T_seg=Ts, k_c=k_c, k_g=k_g, dtype=dtype,
+                     kv_capacity=cache.cap)
+        q = q.contiguous()
+        with torch.no_grad():
+            cache.K[:, :, T_hist:T_hist + Ts] = k
+            cache.V[:, :, T_hist:T_hist + Ts] = v
+        wc, wg = B.route_widths(p)
+        key = (Bn, Hq, Hkv, d, Ts, wc, wg)
+        buf = bufs.get(key)
+        if buf is None or buf.ws.numel() * 4 < B.workspace_size(p):
+            buf = bufs[key] = _SegmentBuffers(p, q.device)
+        # The segment's summaries go next to the history's, in the cache.
+        B.build_summaries_rows(p, k.detach().contiguous(), T_hist, T_hist + Ts, cache.csum, cache.gsum)
+        B.route(p, q, cache.csum, cache.gsum, buf.qbar, buf.cidx, buf.gidx)
+        B.attn_fwd(p, q, cache.K, cache.V, buf.gidx, buf.O, buf.lse)
+        O, lse, gidx = buf.O.clone(), buf.lse.clone(), buf.gidx.clone()
+        ctx.p, ctx.buf = p, buf
+        ctx.K, ctx.V = cache.K, cache.V          # the buffers this segment's rows live in
+        ctx.save_for_backward(q, O, lse, gidx)
         ctx.dtypes = (q.dtype, k.dtype, v.dtype)
-        # Summaries of history + segment: the cache takes them when the
-        # layer appends the segment.
-        cache.pending = (buf.csum, buf.gsum)
-        gidx = buf.gidx.clone()
         ctx.mark_non_differentiable(gidx)
-        return buf.O.clone(), gidx
+        return O, gidx
 
     @staticmethod
     def backward(ctx, dO, _dgidx):
-        q, Kall, Vall = ctx.saved_tensors
+        q, O, lse, gidx = ctx.saved_tensors
         buf, p = ctx.buf, ctx.p
         dO = dO.to(q.dtype).contiguous()
-        buf.backward(q, Kall, Vall, dO)
+        B.attn_bwd(p, q, ctx.K, ctx.V, O, lse, dO, gidx, buf.dQ, buf.dK, buf.dV, buf.ws)
         tq, tk, tv = ctx.dtypes
-        return buf.dQ.to(tq), buf.dK.to(tk), buf.dV.to(tv), None, None, None
+        return (buf.dQ.to(tq, copy=True), buf.dK.to(tk, copy=True), buf.dV.to(tv, copy=True),
+                None, None, None, None)
 
 
 class HGASegmentLayer(nn.Module):
@@ -103,6 +154,7 @@ class HGASegmentLayer(nn.Module):
         for m in (self.wq, self.wk, self.wv, self.wo):
             nn.init.normal_(m.weight, std=1.0 / math.sqrt(m.in_features))
         self.cache = KVCache()
+        self.bufs = {}                                # per-segment buffers, by shape
         self.last_gidx = None
 
     def project(self, x):
@@ -117,19 +169,10 @@ class HGASegmentLayer(nn.Module):
     def segment(self, x):
         Bn, Ts, _ = x.shape
         q, k, v = self.project(x)
-        O, gidx = HGAAttention.apply(q, k, v, self.cache, self.k_c, self.k_g)
+        O, gidx = HGAAttention.apply(q, k, v, self.cache, self.k_c, self.k_g, self.bufs)
+        self.cache.n += Ts                            # the segment's rows join the history
         self.last_gidx = gidx
-        out = self.wo(O.transpose(1, 2).reshape(Bn, Ts, self.Hq * self.d))
-        self._append(k.detach(), v.detach())
-        return out
-
-    @torch.no_grad()
-    def _append(self, k, v):
-        c = self.cache
-        c.K = k.clone() if c.K is None else torch.cat([c.K, k], dim=2).contiguous()
-        c.V = v.clone() if c.V is None else torch.cat([c.V, v], dim=2).contiguous()
-        c.csum, c.gsum = c.pending                    # built by the segment's forward
-        c.pending = None
+        return self.wo(O.transpose(1, 2).reshape(Bn, Ts, self.Hq * self.d))
 
 
 def run_tbptt(layer: HGASegmentLayer, x, target, seg_len: int, optimizer=None):

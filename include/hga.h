@@ -78,7 +78,18 @@ typedef struct hga_params {
     int     k_c, k_g;           /* >= 1, or HGA_ALL                          */
     float   scale;              /* softmax scale; 0 selects 1/sqrt(d)        */
     int     dtype;              /* HGA_BF16 or HGA_FP32                      */
+    int64_t kv_capacity;        /* rows per (batch, kv-head) of the K / V
+                                 * buffers; 0 = T_hist + T_seg (see below)   */
 } hga_params;
+
+/* kv_capacity lets a caller keep K / V in a preallocated cache that grows
+ * segment by segment: K and V are [B][Hkv][kv_capacity][d] with rows
+ * 0 .. T_hist + T_seg - 1 of each (batch, kv-head) in use, and the chunk /
+ * group summaries are [B][Hkv][kv_capacity / 64][d] and
+ * [B][Hkv][kv_capacity / 8][d].  It must be 0 or a multiple of 64 that is
+ * at least T_hist + T_seg.  It applies to every K, V, csum and gsum
+ * argument below, except K_rows of hga_build_summaries_rows (its own rows)
+ * and the history / segment rows that hga_stage_routed reads (dense). */
 
 /* Row widths of the index tables: wc = k_c (T/64 for HGA_ALL); wg = k_g
  * (8 * wc for HGA_ALL).  Returns HGA_OK or HGA_ERR_INVALID_ARG. */

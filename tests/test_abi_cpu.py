@@ -235,3 +235,17 @@ int main(void) {
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     assert "sm_100a" in r.stdout
+
+
+def test_kv_capacity_is_validated_on_the_host(lib):
+    import ctypes
+    from hierarchical_routed_sparse_b200.binding import Params
+    p = Params(B=1, Hq=4, Hkv=2, d=128, T_hist=128, T_seg=128, k_c=2, k_g=8)
+    wc, wg = ctypes.c_int(), ctypes.c_int()
+    for bad in (192, 256 + 32, -64):          # below T = 256, not a multiple of 64, negative
+        p.kv_capacity = bad
+        assert lib.hga_route_widths(ctypes.byref(p.c()), ctypes.byref(wc), ctypes.byref(wg)) == 1
+        assert b"kv_capacity" in lib.hga_last_error()
+    for good in (0, 256, 1024):
+        p.kv_capacity = good
+        assert lib.hga_route_widths(ctypes.byref(p.c()), ctypes.byref(wc), ctypes.byref(wg)) == 0

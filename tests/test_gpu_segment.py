@@ -160,3 +160,26 @@ def test_history_is_detached_and_run_tbptt_trains():
     l1 = run_tbptt(layer, x, target, 256, opt)
     assert len(l0) == 2 and all(np.isfinite(l0 + l1))
     assert layer.cache.T_hist == 512
+
+
+def test_layer_segment_attention_matches_oracle(oracle_mod):
+    # Two segments through the layer's autograd function, the history kept
+    # in the growing cache: the second segment's attention output against
+    # the oracle's routed attention over the same 512 keys, fed the routing
+    # the layer used (the routing itself is gated elsewhere).
+    from hierarchical_routed_sparse_b200.segment import HGAAttention, KVCache
+    from hierarchical_routed_sparse_b200.workloads import Workload
+    from parity_util import TOL, dims_of, maxabs, to_dev
+    w = Workload("layer_oracle", B=1, Hq=4, Hkv=2, d=128, T_hist=256, T_seg=256, k_c=3, k_g=12,
+                 keys="clustered", seed=81)
+    x = w.full()
+    Q, K, V = (to_dev(x[k], "bf16") for k in ("Q", "K", "V"))
+    cache, bufs = KVCache(), {}
+    q1 = torch.randn(1, 4, 256, 128, device="cuda").to(torch.bfloat16)
+    HGAAttention.apply(q1, K[:, :, :256].contiguous(), V[:, :, :256].contiguous(), cache, 3, 12, bufs)
+    cache.n += 256
+    O2, gidx = HGAAttention.apply(Q, K[:, :, 256:].contiguous(), V[:, :, 256:].contiguous(), cache, 3, 12, bufs)
+    torch.cuda.synchronize()
+    assert cache.cap >= 512
+    O_ref, _ = oracle_mod.attn_fwd(dims_of(w), x["Q"], x["K"], x["V"], gidx.cpu().numpy())
+    assert maxabs(O2.cpu().numpy(), O_ref) <= TOL["bf16"]
