@@ -1,5 +1,5 @@
 // attn_tc_bwd.cu -- a6 routed attention backward on the tcgen05 tensor cores
-// (bf16 inputs, d = 128, float32 accumulation).
+// (bf16 inputs, d = 64 or 128, float32 accumulation).
 //
 // Article "BMW's 16 GB GPU just did what needs an A100" (seventnews.com),
 // section "What HGA does differently": the router has no learned weights, so
@@ -56,6 +56,10 @@ namespace {
 
 using namespace sm100;
 
+// The kernel's layout is 128 columns wide.  With d = 64 the second 64-column
+// half of every Q / dO / K / V box lies past the tensor maps' width and the
+// TMA fills it with zeros, so S, dP and the products stay exact; dQ and the
+// dK / dV rows are written for the first d columns only.
 constexpr int D = 128;
 constexpr int H = 2;                  // 64-column halves of d
 constexpr int kKStages = 4;            // K is read by S (issued two tiles ahead) and dQ
@@ -112,7 +116,7 @@ struct BwdArgs {
     float* dQ;
     float* dK;
     float* dV;
-    int Hq, Hkv, G, wg;
+    int Hq, Hkv, G, wg, d;     // d: head dim of the tensors (64 or 128)
     int64_t T_hist, T_seg, nQB, n_items;
     int64_t cap;               // K / V rows per (batch, kv-head)
     int q_rows;
@@ -525,8 +529,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int key = gb[j / 8] + j % 8;
-                if (key < a.T_hist) continue;               // padding or detached history
-                const int64_t o = ((int64_t)bg * a.T_seg + (key - a.T_hist)) * D + r;
+                if (key < a.T_hist || r >= a.d) continue;   // padding, detached history, zero columns
+                const int64_t o = ((int64_t)bg * a.T_seg + (key - a.T_hist)) * a.d + r;
                 atomicAdd(a.dV + o, __uint_as_float(vv[j]));
                 atomicAdd(a.dK + o, __uint_as_float(kv[j]) * a.scale);
             }
@@ -690,7 +694,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         const int head = m.head0 + h2;
                         if (head >= a.G) continue;           // no such head: nothing to store
                         const int y = int((b * a.Hq + g * a.G + head) * a.T_seg) + m.qb * 64;
-                        for (int c = 0; c < 4; ++c) tma_store_2d(&tm_dq, 32 * c, y, xbuf(k) + (h2 * 4 + c) * 8192);
+                        for (int c = 0; c < a.d / 32; ++c)
+                            tma_store_2d(&tm_dq, 32 * c, y, xbuf(k) + (h2 * 4 + c) * 8192);
                     }
                     bulk_commit();
                 }
@@ -846,6 +851,7 @@ __device__ void build_schedule(const SchedArgs& sa)
 // item schedule instead.
 constexpr int kRowdotRows = 4;
 
+template <int DH>
 __global__ void __launch_bounds__(256)
 rowdot_kernel(const float* __restrict__ O, const __nv_bfloat16* __restrict__ dO, float* __restrict__ Drow,
               int64_t rows, float4* __restrict__ dK, float4* __restrict__ dV, int64_t n4, const SchedArgs sa)
@@ -866,25 +872,37 @@ rowdot_kernel(const float* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
     }
     const int64_t row0 = (bx * 8 + threadIdx.x / 32) * kRowdotRows;
     const int lane = threadIdx.x & 31;
-    float4 o[kRowdotRows];
-    uint2 w[kRowdotRows];
+    float acc[kRowdotRows];
+    if constexpr (DH == 128) {          // a lane: 4 columns (16 bytes of O, 8 of dO)
+        float4 o[kRowdotRows];
+        uint2 w[kRowdotRows];
 #pragma unroll
-    for (int q = 0; q < kRowdotRows; ++q) {
-        const int64_t row = row0 + q;
-        if (row < rows) {
-            o[q] = __ldg(reinterpret_cast<const float4*>(O + row * D) + lane);
-            w[q] = __ldg(reinterpret_cast<const uint2*>(dO + row * D) + lane);
-        } else {
-            o[q] = z;
-            w[q] = make_uint2(0u, 0u);
+        for (int q = 0; q < kRowdotRows; ++q) {
+            const int64_t row = row0 + q;
+            o[q] = row < rows ? __ldg(reinterpret_cast<const float4*>(O + row * DH) + lane) : z;
+            w[q] = row < rows ? __ldg(reinterpret_cast<const uint2*>(dO + row * DH) + lane) : make_uint2(0u, 0u);
         }
+#pragma unroll
+        for (int q = 0; q < kRowdotRows; ++q)
+            acc[q] = o[q].x * __uint_as_float(w[q].x << 16) + o[q].y * __uint_as_float(w[q].x & 0xFFFF0000u) +
+                     o[q].z * __uint_as_float(w[q].y << 16) + o[q].w * __uint_as_float(w[q].y & 0xFFFF0000u);
+    } else {                            // d = 64: 2 columns a lane
+        float2 o[kRowdotRows];
+        uint32_t w[kRowdotRows];
+#pragma unroll
+        for (int q = 0; q < kRowdotRows; ++q) {
+            const int64_t row = row0 + q;
+            o[q] = row < rows ? __ldg(reinterpret_cast<const float2*>(O + row * DH) + lane) : make_float2(0.f, 0.f);
+            w[q] = row < rows ? __ldg(reinterpret_cast<const uint32_t*>(dO + row * DH) + lane) : 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < kRowdotRows; ++q)
+            acc[q] = o[q].x * __uint_as_float(w[q] << 16) + o[q].y * __uint_as_float(w[q] & 0xFFFF0000u);
     }
 #pragma unroll
     for (int q = 0; q < kRowdotRows; ++q) {
-        float acc = o[q].x * __uint_as_float(w[q].x << 16) + o[q].y * __uint_as_float(w[q].x & 0xFFFF0000u) +
-                    o[q].z * __uint_as_float(w[q].y << 16) + o[q].w * __uint_as_float(w[q].y & 0xFFFF0000u);
-        acc = warp_sum(acc);
-        if (lane == 0 && row0 + q < rows) Drow[row0 + q] = acc;
+        const float v = warp_sum(acc[q]);
+        if (lane == 0 && row0 + q < rows) Drow[row0 + q] = v;
     }
 }
 
@@ -904,7 +922,7 @@ int attn_bwd_tc_status(bool clear)
 bool attn_bwd_tc_supported(const Shape& s)
 {
     const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.cap;
-    return s.dtype == HGA_BF16 && s.d == D && q_rows < (1ull << 31) && kv_rows < (1ull << 31) &&
+    return s.dtype == HGA_BF16 && (s.d == 64 || s.d == 128) && q_rows < (1ull << 31) && kv_rows < (1ull << 31) &&
            tensor_maps_available();
 }
 
@@ -913,7 +931,7 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
                                float* dK_seg, float* dV_seg, float* Drow, cudaStream_t st)
 {
     const int64_t rows = (int64_t)s.B * s.Hq * s.T_seg;
-    const int64_t n4 = (int64_t)s.B * s.Hkv * s.T_seg * D / 4;   // D = 128: whole float4s
+    const int64_t n4 = (int64_t)s.B * s.Hkv * s.T_seg * s.d / 4;   // d = 64 or 128: whole float4s
     const int64_t rows_per_cta = 8 * kRowdotRows;
     const int64_t n_items = bwd_items(s);
     const int64_t grid = std::min<int64_t>(n_items, sm_count());
@@ -927,16 +945,18 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
     sa.n_pairs = (s.G + 1) / 2;
     sa.wg = s.wg;
     sa.G = (int)grid;
-    cudaError_t e = launch_pdl(rowdot_kernel, dim3((unsigned)(1 + (rows + rows_per_cta - 1) / rows_per_cta)),
+    auto rowdot = s.d == 128 ? rowdot_kernel<128> : rowdot_kernel<64>;
+    cudaError_t e = launch_pdl(rowdot, dim3((unsigned)(1 + (rows + rows_per_cta - 1) / rows_per_cta)),
                                dim3(256), 0, st, O, static_cast<const __nv_bfloat16*>(dO), Drow, rows,
                                reinterpret_cast<float4*>(dK_seg), reinterpret_cast<float4*>(dV_seg), n4, sa);
     if (e != cudaSuccess) return e;
     CUtensorMap tq, tdo, tk8, tv8, tk64, tv64, tdq;
     const uint64_t q_rows = (uint64_t)rows, kv_rows = (uint64_t)s.B * s.Hkv * s.cap;
-    if (!make_bf16_map(&tq, Q, q_rows, D, 64) || !make_bf16_map(&tdo, dO, q_rows, D, 64) ||
-        !make_bf16_map(&tk8, K, kv_rows, D, 8) || !make_bf16_map(&tv8, V, kv_rows, D, 8) ||
-        !make_bf16_map(&tk64, K, kv_rows, D, 64) || !make_bf16_map(&tv64, V, kv_rows, D, 64) ||
-        !make_f32_map(&tdq, dQ, q_rows, D, 64))
+    // Maps of the tensors' own width d: boxes past it (d = 64) read zeros.
+    if (!make_bf16_map(&tq, Q, q_rows, s.d, 64) || !make_bf16_map(&tdo, dO, q_rows, s.d, 64) ||
+        !make_bf16_map(&tk8, K, kv_rows, s.d, 8) || !make_bf16_map(&tv8, V, kv_rows, s.d, 8) ||
+        !make_bf16_map(&tk64, K, kv_rows, s.d, 64) || !make_bf16_map(&tv64, V, kv_rows, s.d, 64) ||
+        !make_f32_map(&tdq, dQ, q_rows, s.d, 64))
         return cudaErrorInvalidValue;
     BwdArgs a;
     a.gidx = gidx;
@@ -949,6 +969,7 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
     a.Hkv = s.Hkv;
     a.G = s.G;
     a.wg = s.wg;
+    a.d = s.d;
     a.T_hist = s.T_hist;
     a.T_seg = s.T_seg;
     a.nQB = s.nQB;

@@ -1,4 +1,4 @@
-"""The backward's item schedule (bf16, d 128 tensor-core path), on the GPU.
+"""The backward's item schedule (bf16 tensor-core path, d 64 and 128), on the GPU.
 
 The row-dot launch of hga_attn_bwd writes, after the row sums in the
 workspace, the order in which the persistent backward's G CTAs take the
@@ -44,6 +44,9 @@ CASES = [
              keys="clustered", backward=True, seed=43),                # wg not a multiple of 4
     Workload("sched_many_items", B=2, Hq=32, Hkv=8, d=128, T_hist=2048, T_seg=4096, k_c=4, k_g=16,
              keys="clustered", backward=True, seed=44),                # 2048 items: round-robin
+    # d = 64 runs on the same tensor-core kernel (only it writes a schedule)
+    Workload("sched_d64", B=1, Hq=4, Hkv=2, d=64, T_hist=512, T_seg=256, k_c=3, k_g=13,
+             keys="clustered", backward=True, seed=45),
 ]
 
 
