@@ -32,6 +32,7 @@
 #include "check.cuh"
 #include "hga_internal.cuh"
 #include "sm100.cuh"
+#include "window_union.cuh"
 
 namespace hga {
 
@@ -71,6 +72,8 @@ struct FwdSmem {
     static constexpr int tmem_slot_off = bar_off + 8 * n_bars;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;        // room to align the base to 1 KB
+    // Strictly causal variant: the window's union of routed groups follows.
+    static constexpr int union_off = (bytes + 15) & ~15;
     // The O stage of the epilogue (128 rows x D floats) reuses Q and K/V.
     static_assert(128 * D * 4 <= xmax_off, "O stage");
 };
@@ -81,13 +84,21 @@ struct FwdArgs {
     float* lse;
     int Hq, Hkv, G, wg;
     int64_t T_hist, T_seg, nQB;
+    int64_t nWin;        // strictly causal variant: windows of wu::kWin positions per (b, g)
+    int64_t n_groups;    // groups of the context (T / 8): bounds the union's bitmap
     int q_rows;          // B*Hq*T_seg (rows of the Q map)
     int kv_rows;         // B*Hkv*cap (rows of the K / V maps)
     int64_t cap;         // K / V rows per (batch, kv-head)
     float scale_log2;
 };
 
-template <int D>
+// CAUSAL: the strictly causal variant.  A CTA then owns wu::kWin
+// neighbouring query positions of one (batch, kv-head) and four of its
+// q-heads (row r: head r / 32, position r % 32 of the window); its key tiles
+// are the union of the positions' routed groups, built in shared memory, and
+// every row keeps only the groups its own position routed (a bit of the
+// group's mask) plus its own chunk up to itself.  Q boxes are 32 rows.
+template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k8,
                    const __grid_constant__ CUtensorMap tm_v8, const __grid_constant__ CUtensorMap tm_k64,
@@ -114,15 +125,26 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __shared__ int s_abort;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    // CTAs of one query block are adjacent, so they run together and share
-    // the K/V tiles through L2.
-    const int n_y = (a.G + 1) / 2;
-    const int64_t u = blockIdx.x / n_y;                     // ((b*Hkv)+g)*nQB + qb
-    const int64_t qb = u % a.nQB, bg = u / a.nQB;
+    // CTAs of one query block (window) are adjacent, so they run together and
+    // share the K/V tiles through L2.
+    constexpr int kHeads = CAUSAL ? 4 : 2;                  // q-heads of the M-tile
+    constexpr int kRows = 128 / kHeads;                     // query rows of each head
+    const int n_y = (a.G + kHeads - 1) / kHeads;
+    const int64_t u = blockIdx.x / n_y;                     // ((b*Hkv)+g)*nQB + qb, or the window
+    int64_t bg, w0, c0;                                     // first query of the tile; own chunk
+    if constexpr (CAUSAL) {
+        bg = u / a.nWin;
+        w0 = (u % a.nWin) * wu::kWin;
+        c0 = (a.T_hist + w0) / 64;
+    } else {
+        bg = u / a.nQB;
+        w0 = (u % a.nQB) * 64;
+        c0 = a.T_hist / 64 + u % a.nQB;
+    }
     const int64_t b = bg / a.Hkv, g = bg % a.Hkv;
-    const int head0 = 2 * int(blockIdx.x % n_y);            // first q-head (within kv-head) of this CTA
+    const int head0 = kHeads * int(blockIdx.x % n_y);       // first q-head (within kv-head) of this CTA
 
-    const int32_t* grow = a.gidx + u * a.wg;
+    const int32_t* grow = a.gidx + u * a.wg;                // block path's index row
     __shared__ int s_ng;
     if (threadIdx.x == 0) {
         s_ng = 0;
@@ -148,8 +170,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     pdl_wait();
     pdl_trigger();
     __syncthreads();
-    // Routed groups form a prefix of the row: count them with one parallel pass.
-    {
+    wu::View uv{};
+    if constexpr (CAUSAL) {
+        // The union of the window's routed groups (eligible: before the own chunk).
+        uv = wu::view(smem + L::union_off, a.n_groups, a.wg);
+        wu::build(a.gidx + (bg * a.T_seg + w0) * a.wg, a.wg, 8 * c0, uv, &s_ng, chk::kSiteCausalFwd);
+    } else {
+        // Routed groups form a prefix of the row: count them with one parallel pass.
         int c = 0;
         for (int i = threadIdx.x; i < a.wg; i += kThreads) c += grow[i] >= 0;
         c = __reduce_add_sync(0xFFFFFFFFu, c);
@@ -180,12 +207,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             prefetch_tmap(&tm_k64);
             prefetch_tmap(&tm_v64);
             mbar_expect_tx(bar_q, 2 * H * 64 * 128);
-            for (int hh = 0; hh < 2; ++hh) {
+            for (int hh = 0; hh < kHeads; ++hh) {
                 const int head = head0 + hh;
-                // A missing head (odd count) is read past the end: zeros.
-                const int y = head < a.G ? int((b * a.Hq + g * a.G + head) * a.T_seg + qb * 64) : a.q_rows;
+                // A missing head (G not a multiple) is read past the end: zeros.
+                const int y = head < a.G ? int((b * a.Hq + g * a.G + head) * a.T_seg + w0) : a.q_rows;
                 for (int c = 0; c < H; ++c)
-                    tma_load_2d(sbase + L::q_off + c * L::kQTile + hh * 64 * 128, &tm_q, 64 * c, y, bar_q);
+                    tma_load_2d(sbase + L::q_off + c * L::kQTile + hh * kRows * 128, &tm_q, 64 * c, y, bar_q);
             }
         }
         // Lanes 0-7 load the K ring, lanes 8-15 the V ring, each at its own
@@ -212,13 +239,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const int gi = t * 8 + gl;
                     // Slots past the last routed group repeat group 0: finite
                     // data whose scores the softmax masks out.
-                    const int grp = chk::group(__ldg(grow + (gi < n_g ? gi : 0)), 8 * (a.T_hist / 64 + qb),
-                                               chk::kSiteFwdTc);
+                    int grp;
+                    if constexpr (CAUSAL) grp = uv.list[gi < n_g ? gi : 0];   // checked when built
+                    else grp = chk::group(__ldg(grow + (gi < n_g ? gi : 0)), 8 * c0, chk::kSiteFwdTc);
                     const int y = int(kv_base + (int64_t)grp * 8);
                     for (int c = 0; c < H; ++c)
                         tma_load_2d(dst + c * L::kKVHalf + gl * 1024, m8, 64 * c, y, bar_full(ring, s));
                 } else if (lane == leader) {
-                    const int y = int(kv_base + a.T_hist + qb * 64);
+                    const int y = int(kv_base + 64 * c0);
                     for (int c = 0; c < H; ++c) tma_load_2d(dst + c * L::kKVHalf, m64, 64 * c, y, bar_full(ring, s));
                 }
                 __syncwarp(mask);
@@ -279,7 +307,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // tensor-memory lane) and keys 32 hk.. of each tile, hk = w/4.
         const int q = warp % 4, hk = warp / 4;
         const int r = 32 * q + lane;
-        const int i = r & 63, hp = r >> 6;                 // query in block, head in pair
+        const int hp = r / kRows, pl = r % kRows;          // head within the tile, query within its rows
+        const int i = int(w0) + pl;                        // query position within the segment
+        const int own_lim = int(a.T_hist + i - 64 * c0);   // own-chunk keys 0 .. own_lim are visible
         const int head = head0 + hp;
         const uint32_t lane_off = uint32_t(32 * q) << 16;
         float m_run = -INFINITY;                           // same in both warps of the row
@@ -295,15 +325,30 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tmem_wait_ld();
             float sv[32];
             const bool own = t == n_rt;
-            // Full routed tiles need no masks; the scale is applied after the
-            // maximum (it is positive) and folded into the exponent's FMA.
-            const bool full = !own && t * 8 + 8 <= n_g;
+            // Full routed tiles need no masks (block path); the scale is applied
+            // after the maximum (it is positive) and folded into the exponent's FMA.
+            const bool full = !CAUSAL && !own && t * 8 + 8 <= n_g;
+            // Causal: the masks of this warp's four group slots of the tile.
+            uint32_t mb[4] = {0u, 0u, 0u, 0u};
+            if constexpr (CAUSAL) {
+                if (!own) {
+#pragma unroll
+                    for (int s4 = 0; s4 < 4; ++s4) {
+                        const int slot = t * 8 + 4 * hk + s4;
+                        mb[s4] = slot < n_g ? uv.mask[slot] : 0u;
+                    }
+                }
+            }
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int jj = 32 * hk + j;                // key within the tile
                 sv[j] = __uint_as_float(raw[j]);
-                if (!full && !(own ? (jj <= i) : (t * 8 + jj / 8 < n_g))) sv[j] = -INFINITY;
+                bool vis;
+                if (own) vis = jj <= own_lim;
+                else if constexpr (CAUSAL) vis = (mb[j / 8] >> pl) & 1u;
+                else vis = t * 8 + jj / 8 < n_g;
+                if (!full && !vis) sv[j] = -INFINITY;
                 m4[j & 3] = fmaxf(m4[j & 3], sv[j]);
             }
             const float pm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
@@ -318,7 +363,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const bool need = mx > m_run + kRescaleLog2;
             if (__any_sync(0xFFFFFFFFu, need)) {
                 const float m_new = need ? mx : m_run;
-                const float alpha = fast_exp2(m_run - m_new);  // 0 when m_run = -inf
+                // 0 when m_run = -inf; 1 for a lane that keeps its maximum (also
+                // one that has seen no visible key yet: -inf - -inf is no number).
+                const float alpha = need ? fast_exp2(m_run - m_new) : 1.f;
                 if (t > 0) {
                     ok = mbar_wait(bar_o((t - 1) & 1), ((t - 1) / 2) & 1, kSiteO);
                     if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
@@ -345,7 +392,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // the warp writes only the 32 columns it read.
             uint32_t pk[32];
             float2 rs = make_float2(0.f, 0.f);
-            const float2 c2 = make_float2(a.scale_log2, a.scale_log2), nm = make_float2(-m_run, -m_run);
+            // No visible key yet (a causal row whose position routed none of the
+            // tiles so far): every score is -inf, and subtracting 0 keeps
+            // exp2(-inf) = 0 rather than -inf + inf.
+            const float mz = m_run == -INFINITY ? 0.f : -m_run;
+            const float2 c2 = make_float2(a.scale_log2, a.scale_log2), nm = make_float2(mz, mz);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const float2 x = __ffma2_rn(make_float2(sv[2 * j], sv[2 * j + 1]), c2, nm);
@@ -398,7 +449,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
             }
             if (hk == 0 && head < a.G) {
-                const int64_t row = ((b * a.Hq + g * a.G + head) * a.T_seg + qb * 64 + i);
+                const int64_t row = ((b * a.Hq + g * a.G + head) * a.T_seg + i);
                 a.lse[row] = (m_run + log2f(l_row)) * kLn2;
             }
             // All softmax threads have staged their rows (bounded wait).
@@ -406,9 +457,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (!mbar_wait(bar_stage, 0, kSiteStage)) s_abort = 1;
             constexpr int C4 = D / 4;                      // 16-byte chunks per row
             for (int rr = warp; rr < 128; rr += kSoftmaxWarps) {
-                const int head_r = head0 + rr / 64;
+                const int head_r = head0 + rr / kRows;
                 if (head_r >= a.G) continue;
-                const int64_t grow_ = (b * a.Hq + g * a.G + head_r) * a.T_seg + qb * 64 + (rr & 63);
+                const int64_t grow_ = (b * a.Hq + g * a.G + head_r) * a.T_seg + w0 + rr % kRows;
                 for (int ch = lane; ch < C4; ch += 32) {
                     const int pch = (ch & ~7) | ((ch ^ rr) & 7);
                     *reinterpret_cast<float4*>(a.O + grow_ * D + 4 * ch) =
@@ -441,13 +492,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 }
 
 // ---- host side -------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool CAUSAL>
 cudaError_t launch(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* gidx,
                    float* O, float* lse, cudaStream_t st)
 {
     CUtensorMap tq, tk8, tv8, tk64, tv64;
+    constexpr int kRows = CAUSAL ? wu::kWin : 64;           // query rows of a head in a tile
     const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.cap;
-    if (!make_bf16_map(&tq, Q, q_rows, D, 64) || !make_bf16_map(&tk8, K, kv_rows, D, 8) ||
+    if (!make_bf16_map(&tq, Q, q_rows, D, kRows) || !make_bf16_map(&tk8, K, kv_rows, D, 8) ||
         !make_bf16_map(&tv8, V, kv_rows, D, 8) || !make_bf16_map(&tk64, K, kv_rows, D, 64) ||
         !make_bf16_map(&tv64, V, kv_rows, D, 64))
         return cudaErrorInvalidValue;
@@ -466,12 +518,16 @@ cudaError_t launch(const Shape& s, const void* Q, const void* K, const void* V, 
     a.kv_rows = (int)kv_rows;
     a.cap = s.cap;
     a.scale_log2 = s.scale * kLog2e;
-    // One head pair per CTA, two CTAs per SM.
-    auto k = attn_fwd_tc_kernel<D>;
-    const int smem = FwdSmem<D>::alloc;
+    a.nWin = s.T_seg / wu::kWin;
+    a.n_groups = s.nG;
+    // One tile (a head pair of a query block, or four heads of a causal
+    // window) per CTA, two CTAs per SM when shared memory allows.
+    auto k = attn_fwd_tc_kernel<D, CAUSAL>;
+    const int smem = CAUSAL ? int(FwdSmem<D>::union_off + wu::bytes(s.nG, s.wg) + 1024) : FwdSmem<D>::alloc;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const int64_t ctas = (int64_t)s.B * s.Hkv * s.nQB * ((s.G + 1) / 2);
+    const int64_t ctas = CAUSAL ? (int64_t)s.B * s.Hkv * a.nWin * ((s.G + 3) / 4)
+                                : (int64_t)s.B * s.Hkv * s.nQB * ((s.G + 1) / 2);
     return launch_pdl(k, dim3((unsigned)ctas), dim3(kThreads), (size_t)smem, st, tq, tk8, tv8, tk64, tv64, a);
 }
 
@@ -498,7 +554,24 @@ bool attn_fwd_tc_supported(const Shape& s)
 cudaError_t launch_attn_fwd_tc(const Shape& s, const void* Q, const void* K, const void* V,
                                const int32_t* gidx, float* O, float* lse, cudaStream_t st)
 {
-    return s.d == 128 ? launch<128>(s, Q, K, V, gidx, O, lse, st) : launch<64>(s, Q, K, V, gidx, O, lse, st);
+    return s.d == 128 ? launch<128, false>(s, Q, K, V, gidx, O, lse, st)
+                      : launch<64, false>(s, Q, K, V, gidx, O, lse, st);
+}
+
+// Strictly causal variant on the tensor cores: bf16, index rows of at most
+// 64 groups (a window's union of at most 2048), shared memory permitting.
+bool attn_fwd_tc_causal_supported(const Shape& s)
+{
+    const size_t smem = (size_t)(s.d == 128 ? FwdSmem<128>::union_off : FwdSmem<64>::union_off) +
+                        wu::bytes(s.nG, s.wg) + 1024;
+    return attn_fwd_tc_supported(s) && s.wg <= 64 && s.T_seg % wu::kWin == 0 && smem <= 227 * 1024;
+}
+
+cudaError_t launch_attn_fwd_tc_causal(const Shape& s, const void* Q, const void* K, const void* V,
+                                      const int32_t* gidx, float* O, float* lse, cudaStream_t st)
+{
+    return s.d == 128 ? launch<128, true>(s, Q, K, V, gidx, O, lse, st)
+                      : launch<64, true>(s, Q, K, V, gidx, O, lse, st);
 }
 
 // Check word of this translation unit's bounds checks (checked builds).

@@ -588,6 +588,9 @@ cudaError_t launch_route_causal(const Shape& s, const void* Q, const float* csum
 cudaError_t launch_attn_fwd_causal(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* gidx,
                                    float* O, float* lse, cudaStream_t st)
 {
+    // bf16 on the tensor cores (windows of neighbouring positions over the
+    // union of their routed groups); otherwise one warp per position.
+    if (attn_fwd_tc_causal_supported(s)) return launch_attn_fwd_tc_causal(s, Q, K, V, gidx, O, lse, st);
     return dispatch<FwdOp>(s, Q, K, V, gidx, O, lse, st);
 }
 

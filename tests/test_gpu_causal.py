@@ -6,7 +6,10 @@ Gates as for the block path: routing rows equal to the oracle's except on
 rows whose oracle gap is below 1e-4; the attention stages run on the
 oracle's routing and meet 2e-3 (bf16) / 1e-4 (float32) max-abs on O, lse,
 dQ, dK, dV.  A property check runs on the GPU alone: changing the inputs
-after position p leaves the outputs at positions <= p bit for bit.
+after position p leaves the routing at positions <= p bit for bit and the
+outputs there bit for bit (float32, one warp per position) or within float
+rounding (bf16 on the tensor cores, where windows of 32 positions share key
+tiles: see the test).
 """
 import numpy as np
 import pytest
@@ -94,7 +97,7 @@ def test_causal_full_size_workload():
     _compare(W.QWEN3_CTX16K_TRAIN, W.QWEN3_CTX16K_TRAIN.full())
 
 
-@pytest.mark.parametrize("w", [CASES[0], W.QWEN3_CTX16K_TRAIN], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [CASES[0], CASES[1], W.QWEN3_CTX16K_TRAIN], ids=lambda w: w.name)
 def test_outputs_do_not_see_later_positions(w):
     x = w.full()
     a = _run(w, x)
@@ -108,10 +111,20 @@ def test_outputs_do_not_see_later_positions(w):
         for k in ("Q", "K", "V"):
             y[k] = W.round_bf16(y[k])
     b = _run(w, y)
+    assert np.array_equal(a["cidx"][:, :, :p + 1], b["cidx"][:, :, :p + 1])
     assert np.array_equal(a["gidx"][:, :, :p + 1], b["gidx"][:, :, :p + 1])
-    assert np.array_equal(a["O"][:, :, :p + 1], b["O"][:, :, :p + 1])
-    assert np.array_equal(a["lse"][:, :, :p + 1], b["lse"][:, :, :p + 1])
-    assert not np.array_equal(a["O"][:, :, p + 1:], b["O"][:, :, p + 1:])
+    if w.dtype == "fp32":        # one warp per position: bit for bit
+        assert np.array_equal(a["O"][:, :, :p + 1], b["O"][:, :, :p + 1])
+        assert np.array_equal(a["lse"][:, :, :p + 1], b["lse"][:, :, :p + 1])
+    else:
+        # Tensor cores: a window of 32 positions runs over the union of their
+        # routed groups, so a later position of the same window can change
+        # which tile holds a key; its own keys are masked to exactly zero, but
+        # the order in which a row's keys are summed may move.  Equal within
+        # float rounding, far below any real change of the inputs' effect.
+        assert maxabs(a["O"][:, :, :p + 1], b["O"][:, :, :p + 1]) <= 1e-5
+        assert maxabs(a["lse"][:, :, :p + 1], b["lse"][:, :, :p + 1]) <= 1e-5
+    assert maxabs(a["O"][:, :, p + 1:], b["O"][:, :, p + 1:]) > 1e-2
 
 
 @pytest.mark.parametrize("T", [32768, 131072])
