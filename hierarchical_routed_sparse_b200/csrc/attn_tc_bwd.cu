@@ -50,6 +50,7 @@
 #include "check.cuh"
 #include "hga_internal.cuh"
 #include "sm100.cuh"
+#include "window_union.cuh"
 
 namespace hga {
 namespace {
@@ -76,6 +77,7 @@ enum : int {
     kSiteQfree, kSiteDqfree, kSitePfree, kSiteDqs, kSiteSfree, kSiteFinalSdp
 };
 
+template <int KST>                   // K stages
 struct BwdSmem {
     static constexpr int kRows128 = 128 * 128;        // 128 rows x 128 B
     static constexpr int kKVHalf = kKeys * 128;       // 64 keys x 128 B
@@ -84,16 +86,22 @@ struct BwdSmem {
     static constexpr int kX = 4 * kRows128;
     static constexpr int x_off = 0;
     static constexpr int k_off = x_off + 2 * kX;
-    static constexpr int v_off = k_off + kKStages * H * kKVHalf;
+    static constexpr int v_off = k_off + KST * H * kKVHalf;
     static constexpr int bar_off = v_off + kVStages * H * kKVHalf;
     static constexpr int n_bars = 29;
     static constexpr int tab_off = (bar_off + 8 * n_bars + 15) & ~15;   // int4 (item, n_g, n_seg) of the CTA's first items
     static constexpr int tmem_slot_off = tab_off + 16 * 64;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;
+    // Strictly causal variant: the row sums D of the CTA's 128 rows, then the
+    // window's union of routed groups (wu::bytes, sized at launch).
+    static constexpr int ds_off = bytes;
+    static constexpr int union_off = ds_off + 128 * 4;
 };
-static_assert(BwdSmem::alloc <= 227 * 1024, "shared memory");
-static_assert(BwdSmem::tab_off % 16 == 0 && BwdSmem::bar_off % 8 == 0, "int4 table and mbarrier alignment");
+static_assert(BwdSmem<kKStages>::alloc <= 227 * 1024, "shared memory");
+static_assert(BwdSmem<kKStages>::tab_off % 16 == 0 && BwdSmem<kKStages>::bar_off % 8 == 0,
+              "int4 table and mbarrier alignment");
+static_assert(BwdSmem<3>::union_off % 16 == 0, "union alignment");
 
 // mbarriers: q[2], kfull / kempty[kKStages], vfull / vempty[kVStages], sdp[2],
 // ps[2], kv, drained, pfree, qfree, dqfree, final, dqs_full, dqs_free, sfree[2],
@@ -103,7 +111,7 @@ constexpr int kBarQ = 0, kBarKFull = 2, kBarKEmpty = kBarKFull + kKStages, kBarV
               kBarKv = kBarPs + 2, kBarDrained = kBarKv + 1, kBarPfree = kBarKv + 2, kBarQfree = kBarKv + 3,
               kBarDqfree = kBarKv + 4, kBarFinal = kBarKv + 5, kBarDqsFull = kBarKv + 6,
               kBarDqsFree = kBarKv + 7, kBarSfree = kBarKv + 8, kBarFinalSdp = kBarSfree + 2;
-static_assert(kBarFinalSdp + 1 == BwdSmem::n_bars, "barrier count");
+static_assert(kBarFinalSdp + 1 == BwdSmem<kKStages>::n_bars, "barrier count");
 
 // Tensor-memory columns.
 constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDV = 384, kColDK = 448;
@@ -119,6 +127,9 @@ struct BwdArgs {
     int Hq, Hkv, G, wg, d;     // d: head dim of the tensors (64 or 128)
     int64_t T_hist, T_seg, nQB, n_items;
     int64_t cap;               // K / V rows per (batch, kv-head)
+    int64_t nWin, n_groups;    // strictly causal variant: windows per (b, g); groups of the context
+    const float* O;            // strictly causal variant: O and dO for the row sums
+    const __nv_bfloat16* dO;
     int q_rows;
     float scale, scale_log2;
 };
@@ -128,6 +139,7 @@ struct BwdArgs {
 // segment keys.
 struct Item {
     int u, bg, qb, head0, n_g, n_seg;   // u = bg * nQB + qb, bg = b * Hkv + g
+    int w0, own0;                       // first query (in the segment) of the rows; first token of the own chunk
     __device__ __forceinline__ int n_rt() const { return (n_g + 7) / 8; }
     __device__ __forceinline__ int nt() const { return n_rt() + 1; }
     __device__ __forceinline__ const int32_t* grow(const struct BwdArgs& a) const;
@@ -135,7 +147,31 @@ struct Item {
 };
 
 __device__ __forceinline__ const int32_t* Item::grow(const BwdArgs& a) const { return a.gidx + (int64_t)u * a.wg; }
-__device__ __forceinline__ int Item::own_start(const BwdArgs& a) const { return int(a.T_hist) + qb * 64; }
+__device__ __forceinline__ int Item::own_start(const BwdArgs&) const { return own0; }
+
+// Item `it` of the block path: a query block and a pair of its q-heads; of
+// the strictly causal variant: a window of wu::kWin positions and four q-heads.
+template <bool CAUSAL>
+__device__ __forceinline__ void decode_item(const BwdArgs& a, int it, Item& m)
+{
+    if constexpr (CAUSAL) {
+        const int n_y = (a.G + 3) / 4;
+        m.u = it / n_y;
+        m.head0 = 4 * (it % n_y);
+        m.bg = m.u / int(a.nWin);
+        m.w0 = (m.u % int(a.nWin)) * wu::kWin;
+        m.qb = 0;
+        m.own0 = int(64 * ((a.T_hist + m.w0) / 64));
+    } else {
+        const int n_pairs = (a.G + 1) / 2;
+        m.u = it / n_pairs;
+        m.head0 = 2 * (it % n_pairs);
+        m.qb = m.u % int(a.nQB);
+        m.bg = m.u / int(a.nQB);
+        m.w0 = m.qb * 64;
+        m.own0 = int(a.T_hist) + m.qb * 64;
+    }
+}
 
 // Routed-group count n_g and segment-tile count n_seg of item `it`.  The
 // routed groups are an ascending prefix of the index row: of the n_g, c_hist
@@ -168,6 +204,7 @@ __device__ __forceinline__ int item_at(const BwdArgs& a, const int4* tab, int k)
 }
 
 // Item k of this CTA.  Whole-warp call.
+template <bool CAUSAL>
 __device__ __forceinline__ Item make_item(const BwdArgs& a, const int4* tab, int k, int lane)
 {
     Item m;
@@ -183,11 +220,7 @@ __device__ __forceinline__ Item make_item(const BwdArgs& a, const int4* tab, int
         n_g = c.x;
         n_seg = c.y;
     }
-    const int n_pairs = (a.G + 1) / 2;
-    m.u = it / n_pairs;
-    m.head0 = 2 * (it % n_pairs);
-    m.qb = m.u % int(a.nQB);
-    m.bg = m.u / int(a.nQB);
+    decode_item<CAUSAL>(a, it, m);
     m.n_g = n_g;
     m.n_seg = n_seg;
     return m;
@@ -197,13 +230,21 @@ __device__ __forceinline__ Item make_item(const BwdArgs& a, const int4* tab, int
 // many as round-robin would give it.  Barrier phases run on a global
 // key-tile counter (gt), a segment-tile counter (gs) and an item counter (k)
 // that every role advances identically.
+// CAUSAL: the strictly causal variant, one window item per CTA: its key tiles
+// are the union of the window's routed groups (built in the prologue with
+// the rows' sums D), rows are masked by their position's routing, and the
+// K ring has 3 stages to make room for the union.
+template <bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ CUtensorMap tm_v8,
                    const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v64,
                    const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a)
 {
-    using L = BwdSmem;
+    constexpr int KST = CAUSAL ? 3 : kKStages;         // K stages
+    constexpr int kHeads = CAUSAL ? 4 : 2;              // q-heads of the M-tile
+    constexpr int kRows = 128 / kHeads;                 // query rows of each head
+    using L = BwdSmem<KST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -240,7 +281,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(bar_ps(b), kCompute);
             mbar_init(bar_sfree(b), 1);
         }
-        for (int s = 0; s < kKStages; ++s) {
+        for (int s = 0; s < KST; ++s) {
             mbar_init(bar_kfull(s), 1);
             mbar_init(bar_kempty(s), 1);
         }
@@ -263,8 +304,44 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // Setup above touches no global memory; the inputs are read from here on.
     pdl_wait();
     pdl_trigger();
-    // Decode the CTA's first items (warp w: items w, w + 18, ...).
-    {
+    float* Ds = reinterpret_cast<float*>(smem + L::ds_off);      // causal: row sums D
+    wu::View uv{};
+    if constexpr (CAUSAL) {
+        // The CTA's one item: the union of its window's routed groups, its
+        // segment tiles and the row sums D = rowsum(dO * O) of its rows.
+        __shared__ int s_n, s_hist;
+        Item m0;
+        decode_item<true>(a, blockIdx.x, m0);
+        uv = wu::view(smem + L::union_off, a.n_groups, a.wg);
+        if (threadIdx.x == 0) s_hist = 0;
+        const int n = wu::build(a.gidx + ((int64_t)m0.bg * a.T_seg + m0.w0) * a.wg, a.wg, m0.own0 / 8, uv, &s_n,
+                                chk::kSiteCausalBwd);
+        int c = 0;
+        for (int k = threadIdx.x; k < n; k += kThreads) c += uv.list[k] < a.T_hist / 8;
+        c = __reduce_add_sync(0xFFFFFFFFu, c);
+        if (lane == 0 && c) atomicAdd(&s_hist, c);
+        const int b = m0.bg / a.Hkv, g = m0.bg % a.Hkv;
+        for (int rr = warp; rr < 128; rr += kThreads / 32) {
+            const int head = m0.head0 + rr / kRows;
+            float acc = 0.f;
+            if (head < a.G) {
+                const int64_t row = ((int64_t)(b * a.Hq + g * a.G + head)) * a.T_seg + m0.w0 + rr % kRows;
+                for (int e = 2 * lane; e < a.d; e += 64) {
+                    const float2 o = __ldg(reinterpret_cast<const float2*>(a.O + row * a.d + e));
+                    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(a.dO + row * a.d + e));
+                    acc += o.x * __uint_as_float(w << 16) + o.y * __uint_as_float(w & 0xFFFF0000u);
+                }
+            }
+            acc = warp_sum(acc);
+            if (lane == 0) Ds[rr] = acc;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const int n_rt = (n + 7) / 8, c_hist = s_hist;
+            tab[0] = make_int4(blockIdx.x, n, c_hist < n ? n_rt - c_hist / 8 + 1 : 1, 0);
+        }
+    } else {
+        // Decode the CTA's first items (warp w: items w, w + 19, ...).
         const int n_tab = n_mine < kItemTab ? n_mine : kItemTab;
         for (int k = warp; k < n_tab; k += kThreads / 32) {
             const int32_t it = __ldg(a.sched + (int64_t)k * gridDim.x + blockIdx.x);
@@ -289,45 +366,46 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         // Q / dO of item kq_ (lane 0) into buffer kq_ & 1, which held item
         // kq_-1's P / dS.
-        const int n_pairs = (a.G + 1) / 2;
         auto load_q = [&](int kq_) {
-            const int64_t itq = item_at(a, tab, kq_);
-            const int64_t u = itq / n_pairs, qb = u % a.nQB, bg = u / a.nQB;
-            const int64_t b = bg / a.Hkv, g = bg % a.Hkv;
-            const int head0 = 2 * int(itq % n_pairs);
+            Item mq;
+            decode_item<CAUSAL>(a, item_at(a, tab, kq_), mq);
+            const int64_t b = mq.bg / a.Hkv, g = mq.bg % a.Hkv;
             mbar_expect_tx(bar_q(kq_ & 1), 2 * 2 * H * 64 * 128);
-            for (int hp = 0; hp < 2; ++hp) {
-                const int head = head0 + hp;
-                const int y = head < a.G ? int((b * a.Hq + g * a.G + head) * a.T_seg + qb * 64) : a.q_rows;
+            for (int hp = 0; hp < kHeads; ++hp) {
+                const int head = mq.head0 + hp;
+                const int y = head < a.G ? int((b * a.Hq + g * a.G + head) * a.T_seg + mq.w0) : a.q_rows;
                 for (int c = 0; c < H; ++c) {
-                    const uint32_t off = c * L::kRows128 + hp * 64 * 128;
+                    const uint32_t off = c * L::kRows128 + hp * kRows * 128;
                     tma_load_2d(xbuf(kq_) + off, &tm_q, 64 * c, y, bar_q(kq_ & 1));
                     tma_load_2d(xbuf(kq_) + 2 * L::kRows128 + off, &tm_do, 64 * c, y, bar_q(kq_ & 1));
                 }
             }
         };
-        int last_k[kKStages], last_v[kVStages];              // last tile loaded per stage
-        for (int j = 0; j < kKStages; ++j) last_k[j] = -1;
+        int last_k[KST], last_v[kVStages];              // last tile loaded per stage
+        for (int j = 0; j < KST; ++j) last_k[j] = -1;
         for (int j = 0; j < kVStages; ++j) last_v[j] = -1;
         int q_issued = -1;                                  // last item whose Q / dO load was issued
         uint32_t gt = 0;
         bool ok = true;
         for (int k = 0; k < n_mine && ok; ++k) {
-            const Item m = make_item(a, tab, k, lane);
+            const Item m = make_item<CAUSAL>(a, tab, k, lane);
             const int nt = m.nt(), n_rt = m.n_rt();
             const int32_t* grow = m.grow(a);
             const int64_t kv_base = (int64_t)m.bg * a.cap;
             for (int p = 0; p < nt && ok; ++p, ++gt) {
                 const int t = nt - 1 - p;
-                const int ks = gt % kKStages, vs = gt % kVStages;
+                const int ks = gt % KST, vs = gt % kVStages;
                 // Rows of the tile: lane l < 8 holds group slot l (a routed
                 // tile) or lane 0 the own chunk's first row.
                 int y = 0;
                 if (t < n_rt) {
                     const int gi = t * 8 + lane;
-                    if (lane < 8)
-                        y = int(kv_base + (int64_t)chk::group(__ldg(grow + (gi < m.n_g ? gi : 0)),
-                                                              8 * (a.T_hist / 64 + m.qb), chk::kSiteBwdTcLoad) * 8);
+                    if (lane < 8) {
+                        int grp;
+                        if constexpr (CAUSAL) grp = uv.list[gi < m.n_g ? gi : 0];   // checked when built
+                        else grp = chk::group(__ldg(grow + (gi < m.n_g ? gi : 0)), m.own0 / 8, chk::kSiteBwdTcLoad);
+                        y = int(kv_base + (int64_t)grp * 8);
+                    }
                 } else {
                     y = int(kv_base + m.own_start(a));
                 }
@@ -354,7 +432,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         load_q(k + 1);
                         q_issued = k + 1;
                     }
-                    if (ok) ok = gt < kKStages || mbar_wait(bar_kempty(ks), ((gt / kKStages) - 1) & 1, kSiteEmpty);
+                    if (ok) ok = gt < KST || mbar_wait(bar_kempty(ks), ((gt / KST) - 1) & 1, kSiteEmpty);
                     if (ok) mbar_expect_tx(bar_kfull(ks), H * kKeys * 128);
                 }
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -377,8 +455,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // Q / dO loads before the last one were read by MMAs pfree tracked).
         __syncwarp();
         if (lane == 0 && !ok) {
-            for (int j = 0; j < kKStages; ++j)
-                if (last_k[j] >= 0) mbar_wait(bar_kfull(j), (last_k[j] / kKStages) & 1, kSiteDrain);
+            for (int j = 0; j < KST; ++j)
+                if (last_k[j] >= 0) mbar_wait(bar_kfull(j), (last_k[j] / KST) & 1, kSiteDrain);
             for (int j = 0; j < kVStages; ++j)
                 if (last_v[j] >= 0) mbar_wait(bar_vfull(j), (last_v[j] / kVStages) & 1, kSiteDrain);
             if (q_issued >= 0) mbar_wait(bar_q(q_issued & 1), (q_issued >> 1) & 1, kSiteDrain);
@@ -392,14 +470,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         bool ok = true;
         uint32_t g = 0;
         for (int k = 0; k < n_mine && ok; ++k) {
-            const int nt = make_item(a, tab, k, lane).nt();
+            const int nt = make_item<CAUSAL>(a, tab, k, lane).nt();
             for (int p = 0; p < nt && ok; ++p, ++g) {
                 bool r = true;
                 if (lane == 0) {
-                    const int ks = g % kKStages, vs = g % kVStages, bb = g & 1;
+                    const int ks = g % KST, vs = g % kVStages, bb = g & 1;
                     if (p == 0) r = mbar_wait(bar_q(k & 1), (k >> 1) & 1, kSiteQ);
                     if (r && g >= 2) r = mbar_wait(bar_sfree(bb), ((g - 2) >> 1) & 1, kSiteSfree);
-                    if (r) r = mbar_wait(bar_kfull(ks), (g / kKStages) & 1, kSiteFull);
+                    if (r) r = mbar_wait(bar_kfull(ks), (g / KST) & 1, kSiteFull);
                     if (r) r = mbar_wait(bar_vfull(vs), (g / kVStages) & 1, kSiteFull);
                     if (r) {
                         tc_fence_after();
@@ -436,10 +514,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         bool ok = true;
         uint32_t gt = 0, gs = 0;
         for (int k = 0; k < n_mine && ok; ++k) {
-            const Item mc = make_item(a, tab, k, lane);
+            const Item mc = make_item<CAUSAL>(a, tab, k, lane);
             const int nt = mc.nt(), n_seg = mc.n_seg;
             for (int p = 0; ok && p < nt; ++p, ++gt) {
-                const int ks = gt % kKStages, bb = gt & 1;
+                const int ks = gt % KST, bb = gt & 1;
                 const bool seg = p < n_seg;
                 if (lane == 0) {
                     ok = mbar_wait(bar_ps(bb), (gt >> 1) & 1, kSitePs);
@@ -502,17 +580,19 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // Thread (warp w, lane l): query row r = 32*(w%4) + l of the M-tile
         // (its tensor-memory lane) and the 16-key quarter kq = w/4 of each tile.
         const int r = (warp % 4) * 32 + lane, kq = warp / 4;
-        const int i = r & 63, hp = r >> 6;
+        const int hp = r / kRows, qi = r % kRows;          // head within the tile, query within its rows
         const uint32_t lane_off = uint32_t((warp % 4) * 32) << 16;
         // First token of the quarter's two group slots of tile t (-64: padding).
         auto group_bases = [&](const Item& m, int t, int (&gb)[2]) {
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const int gi = t * 8 + 2 * kq + q;
-                gb[q] = t == m.n_rt() ? m.own_start(a) + 16 * kq + 8 * q
-                                      : (gi < m.n_g ? chk::group(__ldg(m.grow(a) + gi), 8 * (a.T_hist / 64 + m.qb),
-                                                                 chk::kSiteBwdTcKeys) * 8
-                                                    : -64);
+                int grp = -8;
+                if (t != m.n_rt() && gi < m.n_g) {
+                    if constexpr (CAUSAL) grp = uv.list[gi];
+                    else grp = chk::group(__ldg(m.grow(a) + gi), m.own0 / 8, chk::kSiteBwdTcKeys);
+                }
+                gb[q] = t == m.n_rt() ? m.own_start(a) + 16 * kq + 8 * q : grp * 8;
             }
         };
         // dV^T / dK^T of a segment tile (d = tensor-memory lane r, keys of
@@ -536,23 +616,26 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
         };
         // Per-row constants of an item.
-        struct RowInfo { int row; bool ok; float lse2, Dr; };
+        struct RowInfo { int row, own_lim; bool ok; float lse2, Dr; };
         auto row_info = [&](const Item& m) {
             RowInfo ri;
             const int head = m.head0 + hp;
             ri.ok = head < a.G;
             const int b = m.bg / a.Hkv, g = m.bg % a.Hkv;
-            ri.row = int((b * a.Hq + g * a.G + head) * a.T_seg) + m.qb * 64 + i;
+            ri.row = int((b * a.Hq + g * a.G + head) * a.T_seg) + m.w0 + qi;
+            ri.own_lim = int(a.T_hist) + m.w0 + qi - m.own0;   // own-chunk keys 0 .. own_lim visible
             ri.lse2 = ri.ok ? __ldg(a.lse + ri.row) * kLog2e : 0.f;
-            ri.Dr = ri.ok ? __ldg(a.Drow + ri.row) : 0.f;
+            if constexpr (CAUSAL) ri.Dr = ri.ok ? Ds[r] : 0.f;
+            else ri.Dr = ri.ok ? __ldg(a.Drow + ri.row) : 0.f;
             return ri;
         };
         uint32_t gt = 0, gs = 0;
         bool ok = true;
-        Item m = make_item(a, tab, 0, lane);   // gridDim.x <= n_items
+        Item m = make_item<CAUSAL>(a, tab, 0, lane);   // gridDim.x <= n_items
         RowInfo ri = row_info(m);
         for (int k = 0; k < n_mine && ok; ++k) {
             const bool row_ok = ri.ok;
+            const int own_lim = ri.own_lim;
             const float lse2 = ri.lse2, Dr = ri.Dr;
             const uint32_t pd = xbuf(k + 1) - sbase;        // this item's P / dS buffer
             uint8_t* prow_hi = smem + pd + r * 128;
@@ -577,9 +660,20 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tmem_ld16(tmem + lane_off + kColDP + bb * kKeys + 16 * kq, pr);
                 tmem_wait_ld();
                 uint32_t ph[8], pl[8], dsw[16];             // dsw: dS hi (8), then dS lo (8)
-                // Every key of a full routed tile is valid for every row:
-                // no masks there; partial tiles and the own chunk mask keys.
-                const bool full = row_ok && !own && t * 8 + 8 <= m.n_g;
+                // Every key of a full routed tile is valid for every row (block
+                // path): no masks there; partial tiles and the own chunk mask keys.
+                const bool full = !CAUSAL && row_ok && !own && t * 8 + 8 <= m.n_g;
+                // Causal: the masks of the quarter's two group slots of the tile.
+                uint32_t mw[2] = {0u, 0u};
+                if constexpr (CAUSAL) {
+                    if (!own) {
+#pragma unroll
+                        for (int q2 = 0; q2 < 2; ++q2) {
+                            const int slot = t * 8 + 2 * kq + q2;
+                            mw[q2] = slot < m.n_g ? uv.mask[slot] : 0u;
+                        }
+                    }
+                }
                 const float2 c2 = make_float2(a.scale_log2, a.scale_log2);
                 const float2 l2 = make_float2(-lse2, -lse2), d2 = make_float2(-Dr, -Dr);
 #pragma unroll
@@ -589,8 +683,18 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                                 c2, l2);
                     float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
                     if (!full) {
-                        const bool v0 = row_ok && (own ? (j0 <= i) : (t * 8 + j0 / 8 < m.n_g));
-                        const bool v1 = row_ok && (own ? (j0 + 1 <= i) : (t * 8 + (j0 + 1) / 8 < m.n_g));
+                        bool v0, v1;
+                        if (own) {
+                            v0 = j0 <= own_lim;
+                            v1 = j0 + 1 <= own_lim;
+                        } else if constexpr (CAUSAL) {
+                            v0 = v1 = (mw[j2 / 4] >> qi) & 1u;   // keys j0, j0 + 1: one group
+                        } else {
+                            v0 = t * 8 + j0 / 8 < m.n_g;
+                            v1 = t * 8 + (j0 + 1) / 8 < m.n_g;
+                        }
+                        v0 = v0 && row_ok;
+                        v1 = v1 && row_ok;
                         pv.x = v0 ? pv.x : 0.f;
                         pv.y = v1 ? pv.y : 0.f;
                     }
@@ -655,7 +759,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             if (!ok) break;
             // The next item's index row and row constants load meanwhile.
-            const Item m_next = k + 1 < n_mine ? make_item(a, tab, k + 1, lane) : m;
+            const Item m_next = k + 1 < n_mine ? make_item<CAUSAL>(a, tab, k + 1, lane) : m;
             const RowInfo ri_next = row_info(m_next);
             if (pending) {
                 ok = mbar_wait(bar_kv, (gs - 1) & 1, kSiteKv);
@@ -677,10 +781,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(bar_dqfree);
-                uint8_t* box = smem + (xbuf(k) - sbase) + (hp * 4 + kq) * 8192 + i * 128;
+                uint8_t* box = smem + (xbuf(k) - sbase) + (hp * 4 + kq) * (kRows * 128) + qi * 128;
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    *reinterpret_cast<float4*>(box + ((j ^ (i & 7)) * 16)) =
+                    *reinterpret_cast<float4*>(box + ((j ^ (qi & 7)) * 16)) =
                         make_float4(__uint_as_float(v[4 * j]) * a.scale, __uint_as_float(v[4 * j + 1]) * a.scale,
                                     __uint_as_float(v[4 * j + 2]) * a.scale, __uint_as_float(v[4 * j + 3]) * a.scale);
                 fence_async_smem();
@@ -690,12 +794,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ok = mbar_wait(bar_dqs_full, k & 1, kSiteDqs);
                 if (ok) {
                     const int b = m.bg / a.Hkv, g = m.bg % a.Hkv;
-                    for (int h2 = 0; h2 < 2; ++h2) {
+                    for (int h2 = 0; h2 < kHeads; ++h2) {
                         const int head = m.head0 + h2;
                         if (head >= a.G) continue;           // no such head: nothing to store
-                        const int y = int((b * a.Hq + g * a.G + head) * a.T_seg) + m.qb * 64;
+                        const int y = int((b * a.Hq + g * a.G + head) * a.T_seg) + m.w0;
                         for (int c = 0; c < a.d / 32; ++c)
-                            tma_store_2d(&tm_dq, 32 * c, y, xbuf(k) + (h2 * 4 + c) * 8192);
+                            tma_store_2d(&tm_dq, 32 * c, y, xbuf(k) + (h2 * 4 + c) * (kRows * 128));
                     }
                     bulk_commit();
                 }
@@ -977,14 +1081,72 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
     a.q_rows = (int)q_rows;
     a.scale = s.scale;
     a.scale_log2 = s.scale * kLog2e;
-    const int smem = BwdSmem::alloc;
-    if ((e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+    const int smem = BwdSmem<kKStages>::alloc;
+    if ((e = cudaFuncSetAttribute(attn_bwd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
         return e;
     a.n_items = n_items;
     a.sched = sched;
-    return launch_pdl(attn_bwd_tc_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st, tq, tdo, tk8, tv8,
-                      tk64, tv64, tdq, a);
+    return launch_pdl(attn_bwd_tc_kernel<false>, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st, tq, tdo,
+                      tk8, tv8, tk64, tv64, tdq, a);
+}
+
+// Strictly causal variant: bf16, index rows of at most 64 groups (a window's
+// union of at most 2048), shared memory permitting.
+bool attn_bwd_tc_causal_supported(const Shape& s)
+{
+    const size_t smem = (size_t)BwdSmem<3>::union_off + wu::bytes(s.nG, s.wg) + 1024;
+    return attn_bwd_tc_supported(s) && s.wg <= 64 && s.T_seg % wu::kWin == 0 && smem <= 227 * 1024;
+}
+
+cudaError_t launch_attn_bwd_tc_causal(const Shape& s, const void* Q, const void* K, const void* V, const float* O,
+                                      const float* lse, const void* dO, const int32_t* gidx, float* dQ,
+                                      float* dK_seg, float* dV_seg, cudaStream_t st)
+{
+    // dK / dV accumulate with atomics: zeroed first.
+    const size_t seg_bytes = sizeof(float) * (size_t)s.B * s.Hkv * s.T_seg * s.d;
+    cudaError_t e = cudaMemsetAsync(dK_seg, 0, seg_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dV_seg, 0, seg_bytes, st);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tq, tdo, tk8, tv8, tk64, tv64, tdq;
+    const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.cap;
+    if (!make_bf16_map(&tq, Q, q_rows, s.d, wu::kWin) || !make_bf16_map(&tdo, dO, q_rows, s.d, wu::kWin) ||
+        !make_bf16_map(&tk8, K, kv_rows, s.d, 8) || !make_bf16_map(&tv8, V, kv_rows, s.d, 8) ||
+        !make_bf16_map(&tk64, K, kv_rows, s.d, 64) || !make_bf16_map(&tv64, V, kv_rows, s.d, 64) ||
+        !make_f32_map(&tdq, dQ, q_rows, s.d, wu::kWin))
+        return cudaErrorInvalidValue;
+    BwdArgs a{};
+    a.gidx = gidx;
+    a.sched = nullptr;
+    a.lse = lse;
+    a.Drow = nullptr;
+    a.dQ = dQ;
+    a.dK = dK_seg;
+    a.dV = dV_seg;
+    a.Hq = s.Hq;
+    a.Hkv = s.Hkv;
+    a.G = s.G;
+    a.wg = s.wg;
+    a.d = s.d;
+    a.T_hist = s.T_hist;
+    a.T_seg = s.T_seg;
+    a.nQB = s.nQB;
+    a.cap = s.cap;
+    a.nWin = s.T_seg / wu::kWin;
+    a.n_groups = s.nG;
+    a.O = O;
+    a.dO = static_cast<const __nv_bfloat16*>(dO);
+    a.q_rows = (int)q_rows;
+    a.scale = s.scale;
+    a.scale_log2 = s.scale * kLog2e;
+    // One window item per CTA (grid = items; the kernel's item loop runs once).
+    a.n_items = (int64_t)s.B * s.Hkv * a.nWin * ((s.G + 3) / 4);
+    const int smem = int((size_t)BwdSmem<3>::union_off + wu::bytes(s.nG, s.wg) + 1024);
+    if ((e = cudaFuncSetAttribute(attn_bwd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+        return e;
+    return launch_pdl(attn_bwd_tc_kernel<true>, dim3((unsigned)a.n_items), dim3(kThreads), (size_t)smem, st, tq, tdo,
+                      tk8, tv8, tk64, tv64, tdq, a);
 }
 
 // Check word of this translation unit's bounds checks (checked builds).

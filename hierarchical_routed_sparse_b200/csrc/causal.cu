@@ -598,6 +598,10 @@ cudaError_t launch_attn_bwd_causal(const Shape& s, const void* Q, const void* K,
                                    const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK,
                                    float* dV, cudaStream_t st)
 {
+    // bf16 on the tensor cores (the forward's windows); otherwise one warp
+    // per position.
+    if (attn_bwd_tc_causal_supported(s))
+        return launch_attn_bwd_tc_causal(s, Q, K, V, O, lse, dO, gidx, dQ, dK, dV, st);
     return dispatch<BwdOp>(s, Q, K, V, O, lse, dO, gidx, dQ, dK, dV, st);
 }
 

@@ -204,5 +204,9 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
                                const int32_t* gidx, float* dQ, float* dK_seg, float* dV_seg,
                                float* Drow, cudaStream_t st);
 int attn_bwd_tc_status(bool clear);
+bool attn_bwd_tc_causal_supported(const Shape& s);
+cudaError_t launch_attn_bwd_tc_causal(const Shape& s, const void* Q, const void* K, const void* V, const float* O,
+                                      const float* lse, const void* dO, const int32_t* gidx, float* dQ,
+                                      float* dK_seg, float* dV_seg, cudaStream_t st);
 
 }  // namespace hga

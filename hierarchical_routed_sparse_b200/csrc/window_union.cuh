@@ -52,7 +52,7 @@ __device__ __forceinline__ View view(uint8_t* buf, int64_t n_groups, int wg)
 // n_groups.  Entries outside are dropped, so no index outside the tensors
 // is ever formed (checked builds also record them).
 // Returns the number of union groups.
-__device__ int build(const int32_t* __restrict__ rows, int wg, int64_t limit, const View& v, int* s_n, int site)
+__device__ __forceinline__ int build(const int32_t* __restrict__ rows, int wg, int64_t limit, const View& v, int* s_n, int site)
 {
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
     const int nwords = int((limit + 31) / 32);
