@@ -298,7 +298,9 @@ int hga_device_status(int* status, int clear);
  * index it reads from a caller's index row before using it as an address
  * (valid: 0 <= index < the row's own chunk, in chunks or groups); an index
  * outside records a site code in a device check word and is replaced by
- * index 0 of the same (batch, kv-head), so no access leaves the tensors.
+ * index 0 of the same (batch, kv-head) (the strictly causal tensor-core
+ * kernels, which merge the index rows of 32 neighbouring positions, drop
+ * it instead), so no access leaves the tensors.
  * In that build hga_route_groups, hga_attn_fwd, hga_attn_bwd,
  * hga_attn_bwd_noalloc, hga_stage_routed, hga_attn_fwd_causal and
  * hga_attn_bwd_causal wait for their stream and return HGA_ERR_DEVICE_CHECK
