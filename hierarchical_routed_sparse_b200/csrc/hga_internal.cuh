@@ -116,22 +116,15 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 // Raise a kernel's dynamic shared memory limit to at least `bytes`, calling
-// the driver only when the limit set so far (per kernel and device) is
-// lower: a repeated launch path makes no driver call besides the launch.
+// the driver only when the limit set so far (per kernel function and device)
+// is lower: a repeated launch path makes no driver call besides the launch.
+// Kernels of one signature (template instances that differ only in
+// compile-time parameters) are told apart by their address (tma_map.cu).
+cudaError_t allow_smem_fn(const void* kernel, int bytes);
 template <typename Kern>
 cudaError_t allow_smem(Kern kernel, int bytes)
 {
-    static std::atomic<int> limit[64];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 64 && limit[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && dev < 64) {
-        int cur = limit[dev].load(std::memory_order_relaxed);
-        while (cur < bytes && !limit[dev].compare_exchange_weak(cur, bytes)) {}
-    }
-    return e;
+    return allow_smem_fn(reinterpret_cast<const void*>(kernel), bytes);
 }
 
 // ---- launchers (each returns cudaError_t of its launch) ------------------------

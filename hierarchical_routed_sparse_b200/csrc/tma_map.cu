@@ -2,7 +2,11 @@
 //
 // cuTensorMapEncodeTiled is a driver entry point; it is fetched through the
 // runtime (cudaGetDriverEntryPoint), so the library links no driver library.
+// Also the per-kernel cache of raised dynamic shared-memory limits.
 #include <cudaTypedefs.h>
+
+#include <mutex>
+#include <vector>
 
 #include "hga_internal.cuh"
 
@@ -25,6 +29,30 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 }  // namespace
 
 bool tensor_maps_available() { return encode_fn() != nullptr; }
+
+cudaError_t allow_smem_fn(const void* kernel, int bytes)
+{
+    struct Entry {
+        const void* fn;
+        int dev, bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (Entry& x : done)
+        if (x.fn == kernel && x.dev == dev) {
+            if (x.bytes >= bytes) return cudaSuccess;
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+            if (e == cudaSuccess) x.bytes = bytes;
+            return e;
+        }
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.push_back(Entry{kernel, dev, bytes});
+    return e;
+}
 
 int sm_count()
 {
