@@ -13,9 +13,20 @@
 //
 // Every row has its own key set, so there is no key tile shared by the rows
 // of a block: the kernels work per (row, kv-head) on the FMA pipes.
-//   causal_route_kernel  one warp per row: block query of one, chunk scores
-//                        (the 8 rows of a CTA share the summaries through
-//                        L1), warp top-k, group scores, warp rank selection;
+//   causal_route_win_kernel  one CTA per window of 32 neighbouring positions
+//                        of a (batch, kv-head), which share their own chunk
+//                        and so their chunk candidates: the chunk scores of
+//                        the 32 rows as a register-tiled float32 product
+//                        with the chunk summaries staged once in shared
+//                        memory, a warp top-k per row, then the group
+//                        summaries of the union of the rows' chosen chunks
+//                        read once (a chunk per warp, in registers) and
+//                        scored against every row that chose the chunk,
+//                        warp rank selection;
+//   causal_route_kernel  (shapes the window kernel does not take) one warp
+//                        per row: block query of one, chunk scores (the 8
+//                        rows of a CTA share the summaries through L1), warp
+//                        top-k, group scores, warp rank selection;
 //   causal_fwd_kernel    one warp per (row, kv-head), the G heads together,
 //                        keys in batches of 32: scores with one key per lane
 //                        (the lane reads the key's whole K row and dots it
@@ -32,11 +43,13 @@
 #include "check.cuh"
 #include "hga_internal.cuh"
 #include "router_core.cuh"
+#include "sm100.cuh"
 
 namespace hga {
 namespace {
 
 using namespace rt;
+using namespace sm100;
 
 constexpr int kWarps = 8;                   // rows (warps) per CTA
 constexpr int kThreads = 32 * kWarps;
@@ -175,6 +188,491 @@ causal_route_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, c
                                keys, 0, lane);
         __syncwarp();
         warp_select_groups(keys, ids, n, k_g, flags, grow_out, wg, lane);
+    }
+}
+
+// ---- windowed routing ------------------------------------------------------------------------
+// The 32 positions of a window lie in one chunk, so all have the same chunk
+// candidates (c < own chunk): their chunk scores are a [32 x c0] product of
+// the rows' block queries with the chunk summaries, computed in tiles of 256
+// chunks, whose summaries stream through shared memory in slices of 16 dims
+// (asynchronous copies, two buffers: slice s + 1 lands while slice s is
+// used).  Warp w covers rows 16 (w & 1) .. + 15 and chunks 64 (w >> 1) ..
+// + 63 of a tile; lane (tr, tc) = (lane >> 3, lane & 7) rows 16 (w & 1) +
+// tr + 4 i (i < 4) and chunks 64 (w >> 1) + tc + 8 j (j < 8).  Each score is one float32 chain
+// over the head dims in order.  Then the group summaries of the union of
+// the rows' chosen chunks are read once per window, a chunk per warp held in
+// registers, and scored against every row that chose the chunk.
+namespace rwin {
+constexpr int kW = 32;              // positions of a window
+constexpr int kWinThreads = 256;
+constexpr int kCT = 256;            // chunks of a score tile
+constexpr int kDS = 16;             // head dims of a staged summary slice
+constexpr int kRowsPerWarp = kW / (kWinThreads / 32);
+}  // namespace rwin
+
+struct WinLayout {
+    size_t q, c, s, crow, uni, total;
+    int sstride, gkeys, gids, gflags;   // offsets inside the S region (group stage)
+    int nwords;                         // bitmap words over the context's chunks
+};
+__host__ __device__ inline WinLayout win_layout(int64_t nC, int wc, int D)
+{
+    using namespace rwin;
+    WinLayout L;
+    const size_t qs = (size_t)D + 4;
+    L.q = 0;                                                       // block queries [kW][D + 4]
+    L.c = al16(L.q + 4 * kW * qs);                                 // two summary slices
+    const size_t cbytes = 2 * 4 * (size_t)kCT * (kDS + 4);
+    L.sstride = int((nC + 3) & ~int64_t(3));                       // chunk scores [kW][sstride]
+    const size_t ng = 8 * (size_t)wc;
+    // Group stage, in the same region: scores [kW][8 wc], then per warp the
+    // keys (8 B), ids (4 B) and flags (1 B) of 8 wc candidates.
+    constexpr int nwarps = kWinThreads / 32;
+    L.gkeys = int(al16(4 * kW * ng));
+    L.gids = int(L.gkeys + nwarps * 8 * ng);
+    L.gflags = int(L.gids + nwarps * 4 * ng);
+    const size_t sb = 4 * (size_t)kW * L.sstride, gsz = L.gflags + nwarps * al16(ng);
+    const size_t sreg = sb > gsz ? sb : gsz;
+    if (nC - 1 <= kCT) {
+        // One score tile (c0 <= 256): the scores are written after its last
+        // slice is consumed, so they (and the group stage) reuse the slices.
+        L.s = L.c;
+        L.crow = al16(L.c + (cbytes > sreg ? cbytes : sreg));
+    } else {
+        L.s = al16(L.c + cbytes);
+        L.crow = al16(L.s + sreg);
+    }
+    L.uni = al16(L.crow + 4 * (size_t)kW * wc);                    // chosen chunks [kW][wc]
+    L.nwords = int((nC + 31) / 32);                                // union: bitmap, prefix, list, masks, count
+    L.total = al16(L.uni + 8 * (size_t)L.nwords + 8 * (size_t)kW * wc + 16 + (size_t)kW * kW * wc);
+    return L;
+}
+
+// Top-k of the float scores s[0..n) (n <= 2048), "higher score, then lower
+// index", written ascending to out0 and out1, -1 up to `width`.  Lane l
+// owns candidates l + 32 m and marks its selected ones in a 64-bit mask.
+__device__ __forceinline__ void topk_scores_rounds(const float* s, int n, int k, int32_t* out0, int32_t* out1,
+                                                   int width, int lane)
+{
+    uint64_t sel = 0;
+    auto best_of = [&]() {
+        unsigned long long b = 0ull;
+        for (int m = 0, c = lane; c < n; ++m, c += 32)
+            if (!((sel >> m) & 1ull)) {
+                const unsigned long long kc = pack_key(s[c], c);
+                b = kc > b ? kc : b;
+            }
+        return b;
+    };
+    unsigned long long best = best_of();
+    for (int round = 0; round < k; ++round) {
+        const uint32_t hi = uint32_t(best >> 32), lo = uint32_t(best);
+        const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
+        const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+        if (best != 0ull && hi == mhi && lo == mlo) {   // keys are distinct: one lane wins
+            sel |= 1ull << (key_index(best) >> 5);
+            best = best_of();
+        }
+    }
+    const unsigned below = (1u << lane) - 1u;
+    int pos = 0;
+    for (int m = 0; 32 * m < n; ++m) {
+        const bool mine = (sel >> m) & 1ull;
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, mine);
+        if (mine) {
+            const int at = pos + __popc(bal & below);
+            out0[at] = lane + 32 * m;
+            out1[at] = lane + 32 * m;
+        }
+        pos += __popc(bal);
+    }
+    for (int i = pos + lane; i < width; i += 32) {
+        out0[i] = -1;
+        out1[i] = -1;
+    }
+}
+
+// Sorted (descending) list of the 8 largest keys seen by a lane.
+struct Top8 {
+    unsigned long long v[8];
+    __device__ __forceinline__ void init()
+    {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0ull;
+    }
+    __device__ __forceinline__ void push(unsigned long long x)
+    {
+        if (x <= v[7]) return;
+        v[7] = x;
+#pragma unroll
+        for (int i = 7; i > 0; --i)
+            if (v[i] > v[i - 1]) {
+                const unsigned long long t = v[i];
+                v[i] = v[i - 1];
+                v[i - 1] = t;
+            }
+    }
+    // Keep the 8 largest of this list and the list of lane ^ o (both
+    // sorted): the element-wise maximum against the partner's list reversed
+    // is a bitonic sequence holding them, sorted again by a bitonic merge.
+    __device__ __forceinline__ void merge_xor(int o)
+    {
+        unsigned long long p[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) p[i] = __shfl_xor_sync(0xFFFFFFFFu, v[i], o);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = v[i] > p[7 - i] ? v[i] : p[7 - i];
+#pragma unroll
+        for (int d = 4; d > 0; d >>= 1)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if ((i & d) == 0 && v[i + d] > v[i]) {
+                    const unsigned long long t = v[i];
+                    v[i] = v[i + d];
+                    v[i + d] = t;
+                }
+    }
+};
+
+// Top-k (k <= 8) of the float scores s[0..n) by key ("higher score, then
+// lower index"), for one row per group of 8 lanes (sub = lane & 7): each
+// lane keeps the 8 best of candidates sub, sub + 8, ..., the group merges
+// them, and lane sub writes slot sub of the row (ascending chunk indices,
+// -1 past k) to out0 and out1 (width <= 8).
+__device__ __forceinline__ void topk8_lanes(const float* s, int n, int k, int32_t* out0, int32_t* out1, int width,
+                                            int sub)
+{
+    Top8 t;
+    t.init();
+    for (int c = sub; c < n; c += 8) t.push(pack_key(s[c], c));
+    t.merge_xor(1);
+    t.merge_xor(2);
+    t.merge_xor(4);
+    int idx[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) idx[i] = i < k ? key_index(t.v[i]) : INT32_MAX;
+#pragma unroll
+    for (int a = 0; a < 8; ++a)                       // ascending (a small sort network would do too)
+#pragma unroll
+        for (int b = 0; b < 7 - a; ++b)
+            if (idx[b] > idx[b + 1]) {
+                const int x = idx[b];
+                idx[b] = idx[b + 1];
+                idx[b + 1] = x;
+            }
+    int mine = -1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        if (i == sub) mine = idx[i] == INT32_MAX ? -1 : idx[i];
+    if (sub < width) {
+        out0[sub] = mine;
+        out1[sub] = mine;
+    }
+}
+
+// Group top-k over n <= 64 candidate keys (keys[0..n), ids; one warp):
+// the k-th largest key by a bitonic sort of the 64 (lane holds elements
+// lane and lane + 32), then the candidates with a key at least that large
+// are written in candidate order, -1 up to `width`.
+__device__ __forceinline__ void select_groups64(const unsigned long long* keys, const int32_t* ids, int n, int k,
+                                               int32_t* out, int width, int lane)
+{
+    unsigned long long a = lane < n ? keys[lane] : 0ull, b = lane + 32 < n ? keys[lane + 32] : 0ull;
+#pragma unroll
+    for (int sz = 2; sz <= 64; sz <<= 1) {
+#pragma unroll
+        for (int j = sz >> 1; j > 0; j >>= 1) {
+            if (j == 32) {                                   // elements lane and lane + 32: descending
+                const unsigned long long hi = a > b ? a : b, lo = a > b ? b : a;
+                a = hi;
+                b = lo;
+                continue;
+            }
+            const bool lower = (lane & j) == 0;
+            const bool desc_a = sz == 64 || (lane & sz) == 0;
+            const bool desc_b = sz == 64 || ((lane + 32) & sz) == 0;
+            const unsigned long long pa = __shfl_xor_sync(0xFFFFFFFFu, a, j);
+            const unsigned long long pb = __shfl_xor_sync(0xFFFFFFFFu, b, j);
+            a = (lower == desc_a) ? (a > pa ? a : pa) : (a < pa ? a : pa);
+            b = (lower == desc_b) ? (b > pb ? b : pb) : (b < pb ? b : pb);
+        }
+    }
+    const int e = k - 1;                                     // descending: position k - 1
+    const unsigned long long kth = __shfl_sync(0xFFFFFFFFu, e < 32 ? a : b, e & 31);
+    const unsigned below = (1u << lane) - 1u;
+    int pos = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int j = lane + 32 * h;
+        const bool sel = j < n && keys[j] >= kth;
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, sel);
+        if (sel) out[pos + __popc(bal & below)] = ids[j];
+        pos += __popc(bal);
+    }
+    for (int i = pos + lane; i < width; i += 32) out[i] = -1;
+}
+
+// CTA x routes positions w0 .. w0 + 31 of (batch, kv-head) x / (T_seg / 32).
+template <typename TIn, int D>
+__global__ void __launch_bounds__(rwin::kWinThreads, 2)
+causal_route_win_kernel(const TIn* __restrict__ Q, const float* __restrict__ csum, const float* __restrict__ gsum,
+                        int32_t* __restrict__ cidx, int32_t* __restrict__ gidx, int Hq, int Hkv, int G,
+                        int64_t T_hist, int64_t T_seg, int64_t cap, int k_c, int wc, int k_g, int wg)
+{
+    using namespace rwin;
+    pdl_wait();
+    pdl_trigger();
+    constexpr int P = D / 32, QS = D + 4, CS = kDS + 4;
+    extern __shared__ __align__(16) uint8_t sm[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t T = T_hist + T_seg, nC = T / kChunk, nCs = cap / kChunk, nGs = cap / kGroup;
+    const WinLayout L = win_layout(nC, wc, D);
+    float* q_s = reinterpret_cast<float*>(sm + L.q);
+    float* c_s = reinterpret_cast<float*>(sm + L.c);
+    float* S = reinterpret_cast<float*>(sm + L.s);
+    int32_t* crow_s = reinterpret_cast<int32_t*>(sm + L.crow);
+    const int SS = L.sstride;
+    const int64_t nWin = T_seg / kW;
+    const int64_t bg = blockIdx.x / nWin, w0 = (blockIdx.x % nWin) * kW;
+    const int64_t b = bg / Hkv, g = bg % Hkv;
+    const int c0 = int((T_hist + w0) / kChunk);               // own chunk of every row of the window
+    // Block queries of one: the mean of each row's G q-heads' queries, a
+    // row's loads issued before its sums.
+#pragma unroll 1
+    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+        const int r = warp * kRowsPerWarp + rr;
+        float x[kMaxG][P];
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h)
+            if (h < G) Row<TIn, P>::load(Q + ((b * Hq + g * G + h) * T_seg + w0 + r) * D + lane * P, x[h]);
+        float a[P];
+#pragma unroll
+        for (int e = 0; e < P; ++e) a[e] = 0.f;
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h)
+            if (h < G)
+#pragma unroll
+                for (int e = 0; e < P; ++e) a[e] += x[h][e];
+#pragma unroll
+        for (int e = 0; e < P; ++e) q_s[r * QS + lane * P + e] = a[e] / (float)G;
+    }
+    __syncthreads();
+    // a3: chunk scores of the rows, then a top-k_c per row.
+    const bool all_c = k_c <= 0 || k_c >= c0;
+    if (!all_c) {
+        const float* cs = csum + bg * nCs * D;
+        const int rh = warp & 1, cq = warp >> 1, tr = lane >> 3, tc = lane & 7;
+        const uint32_t cbase = smem_u32(c_s);
+        constexpr int NS = D / kDS;                            // slices of a tile
+        constexpr int kCopies = kCT * (kDS / 4) / kWinThreads; // 16-byte copies per thread and slice
+        // Slice ds of chunks ct0 .. ct0 + nct into buffer `buf` (zeros past nct).
+        auto issue = [&](int ct0, int nct, int ds, int buf) {
+#pragma unroll
+            for (int k = 0; k < kCopies; ++k) {
+                const int idx = tid + k * kWinThreads;
+                const int c = idx / (kDS / 4), v = idx % (kDS / 4);
+                const bool valid = c < nct;
+                cp_async16(cbase + 4u * uint32_t(buf * kCT * CS + c * CS + 4 * v),
+                           cs + (int64_t)(valid ? ct0 + c : 0) * D + ds + 4 * v, valid);
+            }
+            cp_async_commit();
+        };
+        for (int ct0 = 0; ct0 < c0; ct0 += kCT) {
+            const int nct = min(kCT, c0 - ct0);
+            float acc[4][8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+            issue(ct0, nct, 0, 0);
+            for (int si = 0; si < NS; ++si) {
+                if (si + 1 < NS) {
+                    issue(ct0, nct, (si + 1) * kDS, (si + 1) & 1);   // its buffer's last reader synced below
+                    cp_async_wait<1>();
+                } else {
+                    cp_async_wait<0>();
+                }
+                __syncthreads();                               // slice si has landed for every thread
+                const float* cb = c_s + (si & 1) * kCT * CS;
+                const int ds = si * kDS;
+#pragma unroll
+                for (int e4 = 0; e4 < kDS / 4; ++e4) {
+                    float4 qv[4], cv[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        qv[i] = *reinterpret_cast<const float4*>(q_s + (16 * rh + tr + 4 * i) * QS + ds + 4 * e4);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        cv[j] = *reinterpret_cast<const float4*>(cb + (64 * cq + tc + 8 * j) * CS + 4 * e4);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            float t = fmaf(qv[i].x, cv[j].x, acc[i][j]);
+                            t = fmaf(qv[i].y, cv[j].y, t);
+                            t = fmaf(qv[i].z, cv[j].z, t);
+                            acc[i][j] = fmaf(qv[i].w, cv[j].w, t);
+                        }
+                }
+                __syncthreads();                               // buffer si & 1 free for slice si + 2
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int c = 64 * cq + tc + 8 * j;
+                    if (c < nct) S[(16 * rh + tr + 4 * i) * SS + ct0 + c] = acc[i][j];
+                }
+        }
+        __syncthreads();
+    }
+    if (!all_c && k_c <= 8) {
+        // Eight lanes per row: the warp's four rows at once.
+        const int r = warp * kRowsPerWarp + (lane >> 3);
+        topk8_lanes(S + r * SS, c0, k_c, crow_s + r * wc, cidx + (bg * T_seg + w0 + r) * wc, wc, lane & 7);
+    } else
+    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+        const int r = warp * kRowsPerWarp + rr;
+        int32_t* out = cidx + (bg * T_seg + w0 + r) * wc;
+        int32_t* crow = crow_s + r * wc;
+        if (all_c) {
+            for (int j = lane; j < wc; j += 32) {
+                const int32_t v = j < c0 ? j : -1;
+                crow[j] = v;
+                out[j] = v;
+            }
+        } else if (c0 <= 32 * kRegCand) {
+            unsigned long long ck[kRegCand];
+#pragma unroll
+            for (int m = 0; m < kRegCand; ++m) {
+                const int c = lane + 32 * m;
+                ck[m] = c < c0 ? pack_key(S[r * SS + c], c) : 0ull;
+            }
+            warp_topk_regs(ck, k_c, crow, out, wc, lane);
+        } else {
+            topk_scores_rounds(S + r * SS, c0, k_c, crow, out, wc, lane);
+        }
+    }
+    __syncthreads();
+    // a4: the groups of each row's chosen chunks.
+    const bool all_g = k_g <= 0 || k_g >= 8 * wc;              // every row keeps all its candidates
+    const int ng = 8 * wc;
+    float* Sg = S;                                             // [kW][8 wc] group scores (chunk scores done)
+    if (!all_g) {
+        // The union of the rows' chosen chunks (bitmap, prefix ranks, the
+        // ascending list) and per union chunk the mask of the rows that
+        // chose it.
+        uint32_t* bitmap = reinterpret_cast<uint32_t*>(sm + L.uni);
+        uint32_t* prefix = bitmap + L.nwords;
+        int32_t* ulist = reinterpret_cast<int32_t*>(prefix + L.nwords);
+        uint32_t* umask = reinterpret_cast<uint32_t*>(ulist + kW * wc);
+        int* s_u = reinterpret_cast<int*>(umask + kW * wc);
+        uint8_t* uslot = reinterpret_cast<uint8_t*>(s_u + 4);   // [union chunk][row]: the chunk's slot in the row
+        const int nwc = (c0 + 31) / 32;
+        for (int i = tid; i < nwc; i += kWinThreads) bitmap[i] = 0u;
+        for (int i = tid; i < kW * wc; i += kWinThreads) umask[i] = 0u;
+        __syncthreads();
+        for (int e = tid; e < kW * wc; e += kWinThreads) {
+            const int c = crow_s[e];
+            if (c >= 0) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int run = 0;
+            for (int base = 0; base < nwc; base += 32) {
+                const int wd = base + lane;
+                const int cnt = wd < nwc ? __popc(bitmap[wd]) : 0;
+                int incl = cnt;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                if (wd < nwc) prefix[wd] = uint32_t(run + incl - cnt);
+                run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+            }
+            if (lane == 0) *s_u = run;
+        }
+        __syncthreads();
+        for (int wd = tid; wd < nwc; wd += kWinThreads) {
+            uint32_t word = bitmap[wd];
+            int k = int(prefix[wd]);
+            while (word) {
+                ulist[k++] = wd * 32 + __ffs(word) - 1;
+                word &= word - 1;
+            }
+        }
+        for (int e = tid; e < kW * wc; e += kWinThreads) {
+            const int c = crow_s[e];
+            if (c < 0) continue;
+            const int rank = int(prefix[c >> 5]) + __popc(bitmap[c >> 5] & ((1u << (c & 31)) - 1u));
+            atomicOr(&umask[rank], 1u << (e / wc));
+            uslot[rank * kW + e / wc] = uint8_t(e % wc);
+        }
+        __syncthreads();
+        // Warp w takes union chunks w, w + 8, ...: lane (gl, sq) holds group
+        // gl's head dims 4 (sq + 4 j) .. + 3 of the chunk in registers (the
+        // next chunk's loads in flight meanwhile), and for every row that
+        // chose the chunk dots them with the row's block query; the four
+        // quarters are summed across the warp.  Each group summary is read
+        // once per window.
+        const int U = *s_u;
+        const float* gs = gsum + bg * nGs * D;
+        const int gl = lane & 7, sq = lane >> 3;
+        constexpr int J = D / 16;
+        float4 cur[J], nxt[J];
+        auto load_chunk = [&](int u, float4 (&v)[J]) {
+            const float4* grow =
+                reinterpret_cast<const float4*>(gs + ((int64_t)ulist[u] * kGroupsPerChunk + gl) * D);
+#pragma unroll
+            for (int j = 0; j < J; ++j) v[j] = __ldg(grow + sq + 4 * j);
+        };
+        if (warp < U) load_chunk(warp, cur);
+        for (int u = warp; u < U; u += kWinThreads / 32) {
+            if (u + kWinThreads / 32 < U) load_chunk(u + kWinThreads / 32, nxt);
+            uint32_t m = umask[u];
+            while (m) {                                        // the same for the whole warp
+                const int r = __ffs(m) - 1;
+                m &= m - 1;
+                const int k = uslot[u * kW + r];
+                const float* qrow = q_s + r * QS;
+                float a = 0.f;
+#pragma unroll
+                for (int j = 0; j < J; ++j) {
+                    const float4 qv = *reinterpret_cast<const float4*>(qrow + 4 * (sq + 4 * j));
+                    a = fmaf(qv.x, cur[j].x, a);
+                    a = fmaf(qv.y, cur[j].y, a);
+                    a = fmaf(qv.z, cur[j].z, a);
+                    a = fmaf(qv.w, cur[j].w, a);
+                }
+                a += __shfl_xor_sync(0xFFFFFFFFu, a, 8);
+                a += __shfl_xor_sync(0xFFFFFFFFu, a, 16);
+                if (sq == 0) Sg[r * ng + 8 * k + gl] = a;
+            }
+#pragma unroll
+            for (int j = 0; j < J; ++j) cur[j] = nxt[j];
+        }
+        __syncthreads();                                       // every row's scores are in
+    }
+    unsigned long long* keys = reinterpret_cast<unsigned long long*>(sm + L.s + L.gkeys) + (size_t)warp * ng;
+    int32_t* ids = reinterpret_cast<int32_t*>(sm + L.s + L.gids) + (size_t)warp * ng;
+    uint8_t* flags = sm + L.s + L.gflags + (size_t)warp * al16(ng);
+    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+        const int r = warp * kRowsPerWarp + rr;
+        int32_t* gout = gidx + (bg * T_seg + w0 + r) * wg;
+        const int n = prefix_count(crow_s + r * wc, wc, lane) * kGroupsPerChunk;
+        for (int j = lane; j < n; j += 32) ids[j] = crow_s[r * wc + j / 8] * kGroupsPerChunk + j % 8;
+        __syncwarp();
+        if (k_g <= 0 || k_g >= n) {
+            for (int j = lane; j < wg; j += 32) gout[j] = j < n ? ids[j] : -1;
+        } else {
+            for (int j = lane; j < n; j += 32) keys[j] = pack_key(Sg[r * ng + j], ids[j]);
+            __syncwarp();
+            if (n <= 64) select_groups64(keys, ids, n, k_g, gout, wg, lane);
+            else warp_select_groups(keys, ids, n, k_g, flags, gout, wg, lane);
+        }
+        __syncwarp();
     }
 }
 
@@ -501,10 +999,27 @@ causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
     }
 }
 
+// Shapes the window kernel takes: contexts up to 2048 chunks, k_c <= 32,
+// its shared memory within a CTA's.
+bool route_win_supported(const Shape& s)
+{
+    return s.nC <= 2048 && s.wc <= 32 && s.T_seg % rwin::kW == 0 &&
+           win_layout(s.nC, s.wc, s.d).total + 1024 <= 227 * 1024;
+}
+
 template <typename TIn, int D>
 cudaError_t launch_route(const Shape& s, const void* Q, const float* csum, const float* gsum, int32_t* cidx,
                          int32_t* gidx, cudaStream_t st)
 {
+    if (route_win_supported(s)) {
+        const size_t smem = win_layout(s.nC, s.wc, D).total;
+        auto k = causal_route_win_kernel<TIn, D>;
+        cudaError_t e = allow_smem(k, (int)smem);
+        if (e != cudaSuccess) return e;
+        const unsigned grid = (unsigned)(s.B * s.Hkv * s.T_seg / rwin::kW);
+        return launch_pdl(k, dim3(grid), dim3(rwin::kWinThreads), smem, st, static_cast<const TIn*>(Q), csum, gsum,
+                          cidx, gidx, s.Hq, s.Hkv, s.G, s.T_hist, s.T_seg, s.cap, s.k_c, s.wc, s.k_g, s.wg);
+    }
     const size_t smem = kWarps * route_warp_layout(s.nC, s.wc, D).total;
     auto k = causal_route_kernel<TIn, D>;
     cudaError_t e = allow_smem(k, (int)smem);
@@ -572,7 +1087,11 @@ template <typename TIn, int D, int GM> struct BwdOp {
 
 }  // namespace
 
-size_t route_causal_smem(const Shape& s) { return kWarps * route_warp_layout(s.nC, s.wc, s.d).total; }
+size_t route_causal_smem(const Shape& s)
+{
+    return route_win_supported(s) ? win_layout(s.nC, s.wc, s.d).total
+                                  : kWarps * route_warp_layout(s.nC, s.wc, s.d).total;
+}
 int causal_max_heads() { return kMaxG; }
 
 cudaError_t launch_route_causal(const Shape& s, const void* Q, const float* csum, const float* gsum, int32_t* cidx,
