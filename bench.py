@@ -517,6 +517,23 @@ def run_gpu(args, w) -> None:
         full_ms.append(s0.elapsed_time(s1))
     full_ms = statistics.median(full_ms[max(args.warmup, 3):])
 
+    # ---- routing + forward: the fused launch against the two launches ---------------
+    def eager_ms(fn, n):
+        ts = []
+        for _ in range(n):
+            flush.zero_()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            fn()
+            s1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(s0.elapsed_time(s1))
+        return statistics.median(ts[max(args.warmup, 3):])
+
+    n_rf = max(args.warmup, 3) + 7
+    fused_ms = eager_ms(lambda: buf.route_forward(Q, K, V, stream), n_rf)
+    separate_ms = eager_ms(lambda: (buf.route(Q, stream), buf.forward(Q, K, V, stream=stream)), n_rf)
+
     if rank == 0:
         alg = algorithmic(w)
         pk = peaks()
@@ -566,6 +583,12 @@ def run_gpu(args, w) -> None:
             ms=full_ms, algorithmic_bytes=full_bytes, gb_per_s=full_bytes / (full_ms * 1e-3) / 1e9,
             frac=full_bytes / (full_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
             note="one-shot build of all chunk / group summaries of the context, timed alone")
+        rf_bytes = stage_bytes["route"] + stage_bytes["attn_fwd"]
+        stage_roof["route_attn_fwd_fused"] = dict(
+            ms=fused_ms, separate_ms=separate_ms, algorithmic_bytes=rf_bytes,
+            gb_per_s=rf_bytes / (fused_ms * 1e-3) / 1e9, frac=rf_bytes / (fused_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            note="hga_route_attn_fwd (routing and forward in one persistent launch) against hga_route + "
+                 "hga_attn_fwd (separate_ms), each timed alone on eager launches, L2 flushed before each")
         line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype=w.dtype, data="synthetic",

@@ -26,7 +26,7 @@ CHECKED_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib
 
 EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_build_summaries_rows",
            "hga_route_chunks",
-           "hga_route_groups", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
+           "hga_route_groups", "hga_route", "hga_attn_fwd", "hga_route_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
            "hga_stage_params", "hga_stage_routed", "hga_decode", "hga_route_causal", "hga_attn_fwd_causal",
            "hga_attn_bwd_causal", "hga_device_status", "hga_device_check", "hga_checked_build",
            "hga_selftest_wait", "hga_last_error",
@@ -118,6 +118,7 @@ def load() -> ctypes.CDLL:
             "hga_route_groups": ([PP, P, P, P, P, P], ctypes.c_int),
             "hga_route": ([PP, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_attn_fwd": ([PP, P, P, P, P, P, P, P], ctypes.c_int),
+            "hga_route_attn_fwd": ([PP, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_attn_bwd": ([PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P],
                              ctypes.c_int),
             "hga_attn_bwd_noalloc": ([PP, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
@@ -241,6 +242,12 @@ def route(p: Params, Q, csum, gsum, qbar, cidx, gidx, stream=None) -> None:
 def attn_fwd(p: Params, Q, K, V, gidx, O, lse, stream=None) -> None:
     _check(load().hga_attn_fwd(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(gidx), _ptr(O),
                                _ptr(lse), _stream(stream)))
+
+
+def route_attn_fwd(p: Params, Q, K, V, csum, gsum, qbar, cidx, gidx, O, lse, stream=None) -> None:
+    """hga_route followed by hga_attn_fwd, as one persistent launch (bf16)."""
+    _check(load().hga_route_attn_fwd(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(csum), _ptr(gsum),
+                                     _ptr(qbar), _ptr(cidx), _ptr(gidx), _ptr(O), _ptr(lse), _stream(stream)))
 
 
 def attn_bwd(p: Params, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, workspace,
@@ -476,6 +483,11 @@ class Buffers:
 
     def forward(self, Q, K, V, gidx=None, stream=None):
         attn_fwd(self.p, Q, K, V, self.gidx if gidx is None else gidx, self.O, self.lse, stream)
+
+    def route_forward(self, Q, K, V, stream=None):
+        """Routing and forward in one launch (hga_route_attn_fwd)."""
+        route_attn_fwd(self.p, Q, K, V, self.csum, self.gsum, self.qbar, self.cidx, self.gidx, self.O, self.lse,
+                       stream)
 
     def backward(self, Q, K, V, dO, gidx=None, stream=None):
         attn_bwd(self.p, Q, K, V, self.O, self.lse, dO, self.gidx if gidx is None else gidx,

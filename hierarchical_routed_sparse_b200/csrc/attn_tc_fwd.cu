@@ -29,8 +29,11 @@
 // the softmax works on the current one.  With 97 KB of shared memory and 256
 // columns, two CTAs share an SM: one's prologue and epilogue overlap the
 // other's key loop.
+#include <algorithm>
+
 #include "check.cuh"
 #include "hga_internal.cuh"
+#include "router_core.cuh"
 #include "sm100.cuh"
 #include "window_union.cuh"
 
@@ -92,17 +95,21 @@ struct FwdArgs {
     float scale_log2;
 };
 
+// One M-tile of the forward: query block (or causal window) u and q-heads
+// head0 .. head0 + kHeads - 1; grow is the block's index row.  The whole CTA
+// calls it; it sets up its barriers and tensor memory, runs the tile and
+// releases both, so a CTA may run several tiles one after another.
 // CAUSAL: the strictly causal variant.  A CTA then owns wu::kWin
 // neighbouring query positions of one (batch, kv-head) and four of its
 // q-heads (row r: head r / 32, position r % 32 of the window); its key tiles
 // are the union of the positions' routed groups, built in shared memory, and
 // every row keeps only the groups its own position routed (a bit of the
 // group's mask) plus its own chunk up to itself.  Q boxes are 32 rows.
-template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(kThreads, 2)
-attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k8,
-                   const __grid_constant__ CUtensorMap tm_v8, const __grid_constant__ CUtensorMap tm_k64,
-                   const __grid_constant__ CUtensorMap tm_v64, const FwdArgs a)
+// ROUTED: the fused route + forward kernel's tiles; grow is in shared memory.
+template <int D, bool CAUSAL, bool ROUTED>
+__device__ __forceinline__ void fwd_tile(const CUtensorMap* tm_q, const CUtensorMap* tm_k8, const CUtensorMap* tm_v8,
+                                         const CUtensorMap* tm_k64, const CUtensorMap* tm_v64, const FwdArgs& a,
+                                         const int64_t u, const int head0, const int32_t* grow)
 {
     using L = FwdSmem<D>;
     constexpr int H = L::H;
@@ -125,12 +132,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __shared__ int s_abort;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    // CTAs of one query block (window) are adjacent, so they run together and
-    // share the K/V tiles through L2.
     constexpr int kHeads = CAUSAL ? 4 : 2;                  // q-heads of the M-tile
     constexpr int kRows = 128 / kHeads;                     // query rows of each head
-    const int n_y = (a.G + kHeads - 1) / kHeads;
-    const int64_t u = blockIdx.x / n_y;                     // ((b*Hkv)+g)*nQB + qb, or the window
     int64_t bg, w0, c0;                                     // first query of the tile; own chunk
     if constexpr (CAUSAL) {
         bg = u / a.nWin;
@@ -142,9 +145,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         c0 = a.T_hist / 64 + u % a.nQB;
     }
     const int64_t b = bg / a.Hkv, g = bg % a.Hkv;
-    const int head0 = kHeads * int(blockIdx.x % n_y);       // first q-head (within kv-head) of this CTA
 
-    const int32_t* grow = a.gidx + u * a.wg;                // block path's index row
     __shared__ int s_ng;
     if (threadIdx.x == 0) {
         s_ng = 0;
@@ -165,7 +166,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_init(bar_stage, kSoftmax);
         fence_mbar_init();
     }
-    if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    // Tensor memory: allocated here, or (ROUTED) once by the kernel for all its
+    // tiles -- a CTA gives up its allocation permit after its first allocation.
+    if constexpr (!ROUTED)
+        if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
     // Setup above touches no global memory; the inputs are read from here on.
     pdl_wait();
     pdl_trigger();
@@ -201,18 +205,18 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // lane j < 8 fetches group j's index and issues that group's boxes,
         // so the eight index loads overlap.
         if (lane == 0) {
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k8);
-            prefetch_tmap(&tm_v8);
-            prefetch_tmap(&tm_k64);
-            prefetch_tmap(&tm_v64);
+            prefetch_tmap(tm_q);
+            prefetch_tmap(tm_k8);
+            prefetch_tmap(tm_v8);
+            prefetch_tmap(tm_k64);
+            prefetch_tmap(tm_v64);
             mbar_expect_tx(bar_q, 2 * H * 64 * 128);
             for (int hh = 0; hh < kHeads; ++hh) {
                 const int head = head0 + hh;
                 // A missing head (G not a multiple) is read past the end: zeros.
                 const int y = head < a.G ? int((b * a.Hq + g * a.G + head) * a.T_seg + w0) : a.q_rows;
                 for (int c = 0; c < H; ++c)
-                    tma_load_2d(sbase + L::q_off + c * L::kQTile + hh * kRows * 128, &tm_q, 64 * c, y, bar_q);
+                    tma_load_2d(sbase + L::q_off + c * L::kQTile + hh * kRows * 128, tm_q, 64 * c, y, bar_q);
             }
         }
         // Lanes 0-7 load the K ring, lanes 8-15 the V ring, each at its own
@@ -220,8 +224,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (lane < 16) {
             const int ring = lane / 8, gl = lane % 8, leader = 8 * ring;
             const unsigned mask = 0xFFu << (8 * ring);
-            const CUtensorMap* m8 = ring == 0 ? &tm_k8 : &tm_v8;
-            const CUtensorMap* m64 = ring == 0 ? &tm_k64 : &tm_v64;
+            const CUtensorMap* m8 = ring == 0 ? tm_k8 : tm_v8;
+            const CUtensorMap* m64 = ring == 0 ? tm_k64 : tm_v64;
             const uint32_t base = sbase + (ring == 0 ? L::k_off : L::v_off);
             for (int t = 0; t < nt; ++t) {
                 const int s = t % kStages, r = t / kStages;
@@ -241,6 +245,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     // data whose scores the softmax masks out.
                     int grp;
                     if constexpr (CAUSAL) grp = uv.list[gi < n_g ? gi : 0];   // checked when built
+                    else if constexpr (ROUTED) grp = chk::group(grow[gi < n_g ? gi : 0], 8 * c0, chk::kSiteFwdTc);
                     else grp = chk::group(__ldg(grow + (gi < n_g ? gi : 0)), 8 * c0, chk::kSiteFwdTc);
                     const int y = int(kv_base + (int64_t)grp * 8);
                     for (int c = 0; c < H; ++c)
@@ -491,9 +496,117 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_wait(bar_q, 0, kSiteDrain);
     }
     __syncthreads();
+    if constexpr (!ROUTED) {
+        if (warp == kMmaWarp) {
+            tc_fence_after();
+            tmem_dealloc(tmem, L::kTmemCols);
+        }
+    }
+}
+
+// CTAs of one query block (window) are adjacent, so they run together and
+// share the K/V tiles through L2.
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 2)
+attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k8,
+                   const __grid_constant__ CUtensorMap tm_v8, const __grid_constant__ CUtensorMap tm_k64,
+                   const __grid_constant__ CUtensorMap tm_v64, const FwdArgs a)
+{
+    constexpr int kHeads = CAUSAL ? 4 : 2;
+    const int n_y = (a.G + kHeads - 1) / kHeads;
+    const int64_t u = blockIdx.x / n_y;                     // ((b*Hkv)+g)*nQB + qb, or the window
+    fwd_tile<D, CAUSAL, false>(&tm_q, &tm_k8, &tm_v8, &tm_k64, &tm_v64, a, u, kHeads * int(blockIdx.x % n_y),
+                               a.gidx + u * a.wg);
+}
+
+// ---- routing and forward in one persistent launch ---------------------------------------------------
+struct RouteArgs {
+    const __nv_bfloat16* Q;
+    const float* csum;
+    const float* gsum;
+    float* qbar;
+    int32_t* cidx;
+    int32_t* gidx;
+    int64_t n_blocks, nC, nCs, nGs, c_hist;
+    int k_c, wc, k_g;
+    float inv_rows;
+};
+
+// Routing scratch of the fused kernel, inside the K / V rings (free until a
+// tile's loads start): the router's row partial sums, the block query, the
+// candidate keys, ids, chosen chunks and flags.
+template <int D>
+struct RouteScratch {
+    static constexpr int RL = rt::kRouterThreads / (D / 8);   // row lanes of the block query (bf16)
+    static constexpr int part_off = 0;
+    static constexpr int qs_off = part_off + RL * D * 4;
+    static constexpr int keys_off = qs_off + D * 4;
+    __host__ __device__ static size_t bytes(int64_t nC, int wc)
+    {
+        const size_t nk = (size_t)(nC > 8 * (int64_t)wc ? nC : 8 * (int64_t)wc);
+        return keys_off + 8 * nk + 4 * 8 * (size_t)wc + 4 * (size_t)wc + 8 * (size_t)wc;
+    }
+};
+
+// CTA x takes query blocks x, x + gridDim.x, ...: for each, warps 0-7 run the
+// router's a2-a4 pieces for the block (block query, chunk and group
+// routing; qbar, cidx, gidx written as hga_route writes them) and keep its
+// group row in shared memory, then the CTA runs the forward tile of every
+// q-head pair of the block on that row.  One launch replaces the router's
+// and the forward's; the block's K / V tiles are read by its head pairs one
+// after another from L2.  (Routing the block again in every head pair's
+// tile, so that the pairs run on different CTAs at once, measured slower:
+// 61 against 52 us at 16K.)
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+route_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k8,
+                      const __grid_constant__ CUtensorMap tm_v8, const __grid_constant__ CUtensorMap tm_k64,
+                      const __grid_constant__ CUtensorMap tm_v64, const FwdArgs a, const RouteArgs r)
+{
+    using L = FwdSmem<D>;
+    using RS = RouteScratch<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* scratch = smem + L::k_off;
+    float(*part)[D] = reinterpret_cast<float(*)[D]>(scratch + RS::part_off);
+    float* qs = reinterpret_cast<float*>(scratch + RS::qs_off);
+    unsigned long long* keys = reinterpret_cast<unsigned long long*>(scratch + RS::keys_off);
+    const size_t nk = (size_t)(r.nC > 8 * (int64_t)r.wc ? r.nC : 8 * (int64_t)r.wc);
+    int32_t* ids = reinterpret_cast<int32_t*>(keys + nk);
+    int32_t* crow = ids + 8 * r.wc;
+    uint8_t* flags = reinterpret_cast<uint8_t*>(crow + r.wc);
+    int32_t* grow = reinterpret_cast<int32_t*>(smem + L::union_off);   // the block's group row
+    __shared__ int s_nvalid;
+    const int warp = threadIdx.x / 32;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::tmem_slot_off);
+    if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);   // for every tile of the CTA
+    pdl_wait();
+    pdl_trigger();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const int n_y = (a.G + 1) / 2;
+    for (int64_t u = blockIdx.x; u < r.n_blocks; u += gridDim.x) {
+        const int64_t qb = u % a.nQB, bg = u / a.nQB;
+        const int64_t b = bg / a.Hkv, g = bg % a.Hkv;
+        if (threadIdx.x < rt::kRouterThreads) {
+            const int tid = threadIdx.x;
+            rt::block_query<__nv_bfloat16, D, rt::SyncRouterThreads>(r.Q, r.qbar + u * D, qs, part, b, g, qb, a.Hq,
+                                                                      a.G, a.T_seg, r.inv_rows, tid);
+            rt::route_chunks_block<D, rt::SyncRouterThreads>(qs, r.csum + bg * r.nCs * D, int(r.c_hist + qb), r.k_c,
+                                                             r.wc, keys, r.cidx + u * r.wc, crow, tid);
+            rt::route_groups_block<D, rt::SyncRouterThreads>(qs, r.gsum + bg * r.nGs * D, crow, r.wc, r.k_g, a.wg,
+                                                             keys, ids, flags, &s_nvalid, grow, tid);
+        }
+        __syncthreads();                                    // the group row is complete
+        for (int i = threadIdx.x; i < a.wg; i += kThreads) r.gidx[u * a.wg + i] = grow[i];
+        for (int hp = 0; hp < n_y; ++hp)
+            fwd_tile<D, false, true>(&tm_q, &tm_k8, &tm_v8, &tm_k64, &tm_v64, a, u, 2 * hp, grow);
+    }
+    __syncthreads();
     if (warp == kMmaWarp) {
         tc_fence_after();
-        tmem_dealloc(tmem, L::kTmemCols);
+        tmem_dealloc(*tmem_slot, L::kTmemCols);
     }
 }
 
@@ -537,6 +650,57 @@ cudaError_t launch(const Shape& s, const void* Q, const void* K, const void* V, 
     return launch_pdl(k, dim3((unsigned)ctas), dim3(kThreads), (size_t)smem, st, tq, tk8, tv8, tk64, tv64, a);
 }
 
+template <int D>
+cudaError_t launch_route_fwd(const Shape& s, const void* Q, const void* K, const void* V, const float* csum,
+                             const float* gsum, float* qbar, int32_t* cidx, int32_t* gidx, float* O, float* lse,
+                             cudaStream_t st)
+{
+    CUtensorMap tq, tk8, tv8, tk64, tv64;
+    const uint64_t q_rows = (uint64_t)s.B * s.Hq * s.T_seg, kv_rows = (uint64_t)s.B * s.Hkv * s.cap;
+    if (!make_bf16_map(&tq, Q, q_rows, D, 64) || !make_bf16_map(&tk8, K, kv_rows, D, 8) ||
+        !make_bf16_map(&tv8, V, kv_rows, D, 8) || !make_bf16_map(&tk64, K, kv_rows, D, 64) ||
+        !make_bf16_map(&tv64, V, kv_rows, D, 64))
+        return cudaErrorInvalidValue;
+    FwdArgs a{};
+    a.gidx = gidx;
+    a.O = O;
+    a.lse = lse;
+    a.Hq = s.Hq;
+    a.Hkv = s.Hkv;
+    a.G = s.G;
+    a.wg = s.wg;
+    a.T_hist = s.T_hist;
+    a.T_seg = s.T_seg;
+    a.nQB = s.nQB;
+    a.q_rows = (int)q_rows;
+    a.kv_rows = (int)kv_rows;
+    a.cap = s.cap;
+    a.scale_log2 = s.scale * kLog2e;
+    RouteArgs r{};
+    r.Q = static_cast<const __nv_bfloat16*>(Q);
+    r.csum = csum;
+    r.gsum = gsum;
+    r.qbar = qbar;
+    r.cidx = cidx;
+    r.gidx = gidx;
+    r.n_blocks = (int64_t)s.B * s.Hkv * s.nQB;
+    r.nC = s.nC;
+    r.nCs = s.nCs;
+    r.nGs = s.nGs;
+    r.c_hist = s.T_hist / kChunk;
+    r.k_c = s.k_c;
+    r.wc = s.wc;
+    r.k_g = s.k_g;
+    r.inv_rows = 1.0f / (float)(s.G * kChunk);
+    auto k = route_attn_fwd_kernel<D>;
+    const int smem = int(FwdSmem<D>::union_off + 4 * (size_t)s.wg + 1024);
+    cudaError_t e = allow_smem(k, smem);
+    if (e != cudaSuccess) return e;
+    // Two CTAs per SM, each walking query blocks.
+    const int64_t grid = std::min<int64_t>(r.n_blocks, 2 * (int64_t)sm_count());
+    return launch_pdl(k, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, st, tq, tk8, tv8, tk64, tv64, a, r);
+}
+
 }  // namespace
 
 int attn_fwd_tc_status(bool clear)
@@ -562,6 +726,28 @@ cudaError_t launch_attn_fwd_tc(const Shape& s, const void* Q, const void* K, con
 {
     return s.d == 128 ? launch<128, false>(s, Q, K, V, gidx, O, lse, st)
                       : launch<64, false>(s, Q, K, V, gidx, O, lse, st);
+}
+
+// Routing and forward in one launch: the tensor-core forward's shapes whose
+// routing scratch fits in the K / V rings and whose group row fits beside
+// the forward's shared memory.
+bool route_attn_fwd_tc_supported(const Shape& s)
+{
+    if (!attn_fwd_tc_supported(s)) return false;
+    const size_t rings = s.d == 128 ? FwdSmem<128>::xmax_off - FwdSmem<128>::k_off
+                                    : FwdSmem<64>::xmax_off - FwdSmem<64>::k_off;
+    const size_t scratch = s.d == 128 ? RouteScratch<128>::bytes(s.nC, s.wc) : RouteScratch<64>::bytes(s.nC, s.wc);
+    const size_t smem = (size_t)(s.d == 128 ? FwdSmem<128>::union_off : FwdSmem<64>::union_off) + 4 * (size_t)s.wg +
+                        1024;
+    return scratch <= rings && smem <= 227 * 1024 / 2;
+}
+
+cudaError_t launch_route_attn_fwd_tc(const Shape& s, const void* Q, const void* K, const void* V, const float* csum,
+                                     const float* gsum, float* qbar, int32_t* cidx, int32_t* gidx, float* O,
+                                     float* lse, cudaStream_t st)
+{
+    return s.d == 128 ? launch_route_fwd<128>(s, Q, K, V, csum, gsum, qbar, cidx, gidx, O, lse, st)
+                      : launch_route_fwd<64>(s, Q, K, V, csum, gsum, qbar, cidx, gidx, O, lse, st);
 }
 
 // Strictly causal variant on the tensor cores: bf16, index rows of at most

@@ -512,6 +512,41 @@ int hga_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* 
     return finish(e, static_cast<cudaStream_t>(stream), "hga_attn_fwd");
 }
 
+int hga_route_attn_fwd(const hga_params* p, const void* Q, const void* K, const void* V, const float* csum,
+                       const float* gsum, float* qbar, int32_t* cidx, int32_t* gidx, float* O, float* lse,
+                       hga_stream_t stream)
+{
+    const NvtxRange nvtx_range("hga_route_attn_fwd");
+    hga::Shape s{};
+    if (int r = make_shape(p, &s)) return r;
+    if (s.nQB == 0) return HGA_OK;
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(csum);
+    CHECK_PTR(gsum);
+    CHECK_PTR(qbar);
+    CHECK_PTR(cidx);
+    CHECK_PTR(gidx);
+    CHECK_PTR(O);
+    CHECK_PTR(lse);
+    const auto st = static_cast<cudaStream_t>(stream);
+    if (hga::route_attn_fwd_tc_supported(s))
+        return finish(hga::launch_route_attn_fwd_tc(s, Q, K, V, csum, gsum, qbar, cidx, gidx, O, lse, st), st,
+                      "hga_route_attn_fwd");
+    // Other shapes: the router's launch, then the forward's (the same results).
+    if (hga::route_fused_smem(s) > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "routing of %lld chunks / k_c=%d exceeds the router's shared memory",
+                    (long long)s.nC, s.wc);
+    if (!hga::attn_fwd_tc_supported(s) && hga::attn_simt_smem(s, false) > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "k_g=%d too large for the attention kernel", s.wg);
+    cudaError_t e = hga::launch_route_fused(s, Q, csum, gsum, qbar, cidx, gidx, st);
+    if (e == cudaSuccess)
+        e = hga::attn_fwd_tc_supported(s) ? hga::launch_attn_fwd_tc(s, Q, K, V, gidx, O, lse, st)
+                                          : hga::launch_attn_fwd_simt(s, Q, K, V, gidx, O, lse, st);
+    return finish(e, st, "hga_route_attn_fwd");
+}
+
 int hga_attn_bwd(const hga_params* p, const void* Q, const void* K, const void* V, const float* O,
                  const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK_seg,
                  float* dV_seg, void* workspace, size_t ws_bytes, hga_stream_t stream)

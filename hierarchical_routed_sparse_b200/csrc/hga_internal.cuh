@@ -188,6 +188,10 @@ cudaError_t launch_attn_fwd_tc(const Shape& s, const void* Q, const void* K, con
 // Status word of the tensor-core kernels' bounded waits (0 = none ran out;
 // -1 = could not be read).  Synchronises with the device.
 int attn_fwd_tc_status(bool clear);
+bool route_attn_fwd_tc_supported(const Shape& s);
+cudaError_t launch_route_attn_fwd_tc(const Shape& s, const void* Q, const void* K, const void* V, const float* csum,
+                                     const float* gsum, float* qbar, int32_t* cidx, int32_t* gidx, float* O,
+                                     float* lse, cudaStream_t st);
 bool attn_fwd_tc_causal_supported(const Shape& s);
 cudaError_t launch_attn_fwd_tc_causal(const Shape& s, const void* Q, const void* K, const void* V,
                                       const int32_t* gidx, float* O, float* lse, cudaStream_t st);

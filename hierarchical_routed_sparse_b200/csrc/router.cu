@@ -25,76 +25,6 @@ namespace {
 
 using namespace rt;
 
-// 16 bytes of inputs widened to float32 (8 bf16 or 4 float).
-template <typename T> __device__ __forceinline__ void widen16(const uint4 r, float* out);
-template <> __device__ __forceinline__ void widen16<__nv_bfloat16>(const uint4 r, float* out)
-{
-    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        out[2 * i] = __uint_as_float(w[i] << 16);
-        out[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-template <> __device__ __forceinline__ void widen16<float>(const uint4 r, float* out)
-{
-    out[0] = __uint_as_float(r.x); out[1] = __uint_as_float(r.y);
-    out[2] = __uint_as_float(r.z); out[3] = __uint_as_float(r.w);
-}
-
-// Block query into qs (and qbar[u]): the mean of the block's 64 queries over
-// the G q-heads of the kv-head.  Every thread owns one 16-byte column vector
-// and issues the loads of up to 16 of its rows (kept as raw 16-byte words)
-// before widening and adding them: one memory round trip for G = 4.
-template <typename TIn, int D>
-__device__ __forceinline__ void block_query(const TIn* __restrict__ Q, float* __restrict__ qbar_row,
-                                            float* qs, float (*part)[D], int64_t b, int64_t g, int64_t qb,
-                                            int Hq, int G, int64_t T_seg, float inv_rows, int tid)
-{
-    constexpr int E = Vec16<TIn>::E;
-    constexpr int V16 = D / E;
-    constexpr int RL = kRouterThreads / V16;          // row lanes
-    const int v = tid % V16, rl = tid / V16;
-    const int rows = G * kChunk;
-    float acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    constexpr int kLoads = 16;
-    for (int r0 = rl; r0 < rows; r0 += kLoads * RL) {
-        uint4 raw[kLoads];
-#pragma unroll
-        for (int q = 0; q < kLoads; ++q) {
-            const int r = r0 + q * RL;
-            if (r < rows) {
-                const int64_t h = (int64_t)g * G + r / kChunk;
-                raw[q] = __ldg(reinterpret_cast<const uint4*>(
-                    Q + ((b * Hq + h) * T_seg + qb * kChunk + r % kChunk) * D + v * E));
-            } else {
-                raw[q] = make_uint4(0u, 0u, 0u, 0u);        // zero bits widen to 0.0f
-            }
-        }
-#pragma unroll
-        for (int q = 0; q < kLoads; ++q) {
-            float x[E];
-            widen16<TIn>(raw[q], x);
-#pragma unroll
-            for (int e = 0; e < E; ++e) acc[e] += x[e];
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < E; ++e) part[rl][v * E + e] = acc[e];
-    __syncthreads();
-    for (int col = tid; col < D; col += kRouterThreads) {
-        float a = 0.f;
-#pragma unroll 8
-        for (int r = 0; r < RL; ++r) a += part[r][col];
-        a *= inv_rows;
-        qs[col] = a;
-        qbar_row[col] = a;
-    }
-    __syncthreads();
-}
-
 // ---- a2 + a3: one CTA per (batch, kv-head, query block) ----------------------
 template <typename TIn, int D>
 __global__ void __launch_bounds__(kRouterThreads, 2)

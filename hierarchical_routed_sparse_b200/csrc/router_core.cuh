@@ -23,6 +23,20 @@ constexpr int kRouterThreads = 256;
 constexpr int kRouterWarps = kRouterThreads / 32;
 constexpr int kBatch = 16;          // candidates a warp scores at once
 
+// The barrier of the per-block routing pieces below, which run on
+// kRouterThreads threads: the CTA barrier by default; a kernel whose CTA has
+// more threads (the fused route + forward kernel) runs them on its first
+// kRouterThreads threads with a named barrier over those.
+struct SyncCta {
+    __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+struct SyncRouterThreads {
+    __device__ __forceinline__ void operator()() const
+    {
+        asm volatile("bar.sync 1, %0;" ::"n"(kRouterThreads) : "memory");
+    }
+};
+
 // Scores of candidates 0..n-1 against the block query qs (shared memory):
 // score(c) = qs . row(c), written as a selection key into keys[c].  Warp w
 // of `Warps` takes batches of 16 candidates w, w+Warps, ...; for each batch every lane
@@ -189,13 +203,85 @@ __device__ __forceinline__ void select_chunks(unsigned long long* keys, int c0, 
     if (out1) compact_selected(keys, nullptr, c0, out1, wc, lane);
 }
 
+// 16 bytes of inputs widened to float32 (8 bf16 or 4 float).
+template <typename T> __device__ __forceinline__ void widen16(const uint4 r, float* out);
+template <> __device__ __forceinline__ void widen16<__nv_bfloat16>(const uint4 r, float* out)
+{
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        out[2 * i] = __uint_as_float(w[i] << 16);
+        out[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+template <> __device__ __forceinline__ void widen16<float>(const uint4 r, float* out)
+{
+    out[0] = __uint_as_float(r.x); out[1] = __uint_as_float(r.y);
+    out[2] = __uint_as_float(r.z); out[3] = __uint_as_float(r.w);
+}
+
+// Block query into qs (and qbar[u]): the mean of the block's 64 queries over
+// the G q-heads of the kv-head.  Every thread owns one 16-byte column vector
+// and issues the loads of up to 16 of its rows (kept as raw 16-byte words)
+// before widening and adding them: one memory round trip for G = 4.
+template <typename TIn, int D, typename Sync = SyncCta>
+__device__ __forceinline__ void block_query(const TIn* __restrict__ Q, float* __restrict__ qbar_row,
+                                            float* qs, float (*part)[D], int64_t b, int64_t g, int64_t qb,
+                                            int Hq, int G, int64_t T_seg, float inv_rows, int tid)
+{
+    const Sync sync{};
+    constexpr int E = Vec16<TIn>::E;
+    constexpr int V16 = D / E;
+    constexpr int RL = kRouterThreads / V16;          // row lanes
+    const int v = tid % V16, rl = tid / V16;
+    const int rows = G * kChunk;
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    constexpr int kLoads = 16;
+    for (int r0 = rl; r0 < rows; r0 += kLoads * RL) {
+        uint4 raw[kLoads];
+#pragma unroll
+        for (int q = 0; q < kLoads; ++q) {
+            const int r = r0 + q * RL;
+            if (r < rows) {
+                const int64_t h = (int64_t)g * G + r / kChunk;
+                raw[q] = __ldg(reinterpret_cast<const uint4*>(
+                    Q + ((b * Hq + h) * T_seg + qb * kChunk + r % kChunk) * D + v * E));
+            } else {
+                raw[q] = make_uint4(0u, 0u, 0u, 0u);        // zero bits widen to 0.0f
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < kLoads; ++q) {
+            float x[E];
+            widen16<TIn>(raw[q], x);
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] += x[e];
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) part[rl][v * E + e] = acc[e];
+    sync();
+    for (int col = tid; col < D; col += kRouterThreads) {
+        float a = 0.f;
+#pragma unroll 8
+        for (int r = 0; r < RL; ++r) a += part[r][col];
+        a *= inv_rows;
+        qs[col] = a;
+        qbar_row[col] = a;
+    }
+    sync();
+}
+
 // a3: chunk routing of one block: scores of the eligible chunks c < c0, then
 // select_chunks.  Writes the row to cidx_row and (if not null) to crow_smem.
-template <int D>
+template <int D, typename Sync = SyncCta>
 __device__ __forceinline__ void route_chunks_block(const float* qs, const float* __restrict__ cs, int c0, int k_c,
                                                    int wc, unsigned long long* keys, int32_t* cidx_row,
                                                    int32_t* crow_smem, int tid)
 {
+    const Sync sync{};
     const int lane = tid & 31, warp = tid >> 5;
     if (k_c <= 0 || k_c >= c0) {                       // keep every eligible chunk
         for (int i = tid; i < wc; i += kRouterThreads) {
@@ -203,14 +289,14 @@ __device__ __forceinline__ void route_chunks_block(const float* qs, const float*
             cidx_row[i] = v;
             if (crow_smem) crow_smem[i] = v;
         }
-        __syncthreads();
+        sync();
         return;
     }
     score_candidates<D>(qs, c0, [&](int c, const float*& row) { row = cs + (int64_t)c * D; return c; }, keys,
                         warp, lane);
-    __syncthreads();
+    sync();
     select_chunks(keys, c0, k_c, wc, cidx_row, crow_smem, warp, lane);
-    __syncthreads();
+    sync();
 }
 
 // Number of valid entries of an index row (an ascending prefix); one warp.
@@ -227,9 +313,11 @@ __device__ __forceinline__ int prefix_count(const int32_t* row, int w, int lane)
 // a4 selection: of the n scored group candidates (keys, ids; block
 // synchronised) a candidate is kept when fewer than k_g candidates beat it;
 // the kept ids are written in candidate order to gidx_row.
+template <typename Sync = SyncCta>
 __device__ __forceinline__ void select_groups(unsigned long long* keys, const int32_t* ids, int n, int k_g,
                                               uint8_t* flags, int32_t* gidx_row, int wg, int tid)
 {
+    const Sync sync{};
     const int lane = tid & 31, warp = tid >> 5;
     for (int i = tid; i < n; i += kRouterThreads) {
         const unsigned long long ki = keys[i];
@@ -237,41 +325,42 @@ __device__ __forceinline__ void select_groups(unsigned long long* keys, const in
         for (int j = 0; j < n; ++j) rank += keys[j] > ki;
         flags[i] = rank < k_g;
     }
-    __syncthreads();
+    sync();
     for (int i = tid; i < n; i += kRouterThreads)
         if (flags[i]) keys[i] = 0ull;
-    __syncthreads();
+    sync();
     if (warp == 0) compact_selected(keys, ids, n, gidx_row, wg, lane);
 }
 
 // a4: group routing of one block: the 8 groups of every chunk in crow (an
 // ascending prefix of valid chunks), scored and ranked (select_groups).
-template <int D>
+template <int D, typename Sync = SyncCta>
 __device__ __forceinline__ void route_groups_block(const float* qs, const float* __restrict__ gs,
                                                    const int32_t* crow, int wc, int k_g, int wg,
                                                    unsigned long long* keys, int32_t* ids, uint8_t* flags,
                                                    int* s_count, int32_t* gidx_row, int tid,
                                                    int64_t c_limit = INT64_MAX)
 {
+    const Sync sync{};
     const int lane = tid & 31, warp = tid >> 5;
     if (warp == 0) {
         const int n = prefix_count(crow, wc, lane);
         if (lane == 0) *s_count = n;
     }
-    __syncthreads();
+    sync();
     const int n = *s_count * kGroupsPerChunk;          // candidate groups
     for (int i = tid; i < n; i += kRouterThreads)
         ids[i] = chk::chunk(crow[i / kGroupsPerChunk], c_limit, chk::kSiteRouteGroups) * kGroupsPerChunk +
                  i % kGroupsPerChunk;
-    __syncthreads();
+    sync();
     if (k_g <= 0 || k_g >= n) {                        // keep every candidate
         for (int i = tid; i < wg; i += kRouterThreads) gidx_row[i] = i < n ? ids[i] : -1;
         return;
     }
     score_candidates<D>(qs, n, [&](int c, const float*& row) { row = gs + (int64_t)ids[c] * D; return ids[c]; },
                         keys, warp, lane);
-    __syncthreads();
-    select_groups(keys, ids, n, k_g, flags, gidx_row, wg, tid);
+    sync();
+    select_groups<Sync>(keys, ids, n, k_g, flags, gidx_row, wg, tid);
 }
 
 }  // namespace rt

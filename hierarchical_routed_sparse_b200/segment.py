@@ -7,8 +7,8 @@ of earlier segments through the router, and older KV is detached -- no
 gradient flows into earlier segments.
 
 ``HGAAttention`` is the autograd function of one segment: its forward runs
-the segment's summaries, the routing and the routed attention forward of
-libhga; its backward runs the routed backward with the forward's routing
+the segment's summaries, then the routing and the routed attention forward
+in one persistent launch (hga_route_attn_fwd); its backward runs the routed backward with the forward's routing
 frozen and returns gradients for the segment's Q, K and V (history gets
 none).  ``HGASegmentLayer`` wraps it between real Q / K / V / O projections
 and keeps the KV cache and the summaries of the segments seen so far in
@@ -115,8 +115,10 @@ class HGAAttention(torch.autograd.Function):
             buf = bufs[key] = _SegmentBuffers(p, q.device)
         # The segment's summaries go next to the history's, in the cache.
         B.build_summaries_rows(p, k.detach().contiguous(), T_hist, T_hist + Ts, cache.csum, cache.gsum)
-        B.route(p, q, cache.csum, cache.gsum, buf.qbar, buf.cidx, buf.gidx)
-        B.attn_fwd(p, q, cache.K, cache.V, buf.gidx, buf.O, buf.lse)
+        # Routing and forward in one persistent launch (bf16; the same results as
+        # hga_route then hga_attn_fwd, which other shapes run).
+        B.route_attn_fwd(p, q, cache.K, cache.V, cache.csum, cache.gsum, buf.qbar, buf.cidx, buf.gidx, buf.O,
+                         buf.lse)
         O, lse, gidx = buf.O.clone(), buf.lse.clone(), buf.gidx.clone()
         ctx.p, ctx.buf = p, buf
         ctx.K, ctx.V = cache.K, cache.V          # the buffers this segment's rows live in

@@ -154,6 +154,22 @@ int hga_attn_fwd(const hga_params* p, const void* Q, const void* K,
                  const void* V, const int32_t* gidx, float* O, float* lse,
                  hga_stream_t stream);
 
+/* a2-a5 in one launch: the fused segment step's routing and forward
+ * (article section "What HGA does differently": HGA as a drop-in attention
+ * module run segment by segment).  Same arguments and results as
+ * hga_route(p, Q, csum, gsum, qbar, cidx, gidx) followed by
+ * hga_attn_fwd(p, Q, K, V, gidx, O, lse): qbar, cidx and gidx are written as
+ * hga_route writes them, O and lse as hga_attn_fwd does, bit for bit.  For
+ * bf16 inputs one persistent kernel runs both: each CTA takes query
+ * blocks, routes one (warps 0-7 run the router's steps) and runs the
+ * forward of the block's q-head pairs on the routing it keeps in shared
+ * memory.  Other shapes run the two launches.  Errors as hga_route and
+ * hga_attn_fwd. */
+int hga_route_attn_fwd(const hga_params* p, const void* Q, const void* K,
+                       const void* V, const float* csum, const float* gsum,
+                       float* qbar, int32_t* cidx, int32_t* gidx, float* O,
+                       float* lse, hga_stream_t stream);
+
 /* a6. Routed attention backward with the routing of the forward frozen
  * (same section: the router has no learned weights, so gradients reach the
  * projections as in the dense case; older KV is detached).  Given O and lse

@@ -101,6 +101,13 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert lib.hga_attn_bwd(ctypes.byref(p), P, P, P, P, P, P, P, P, P, P, P, rows_only, None) == \
         hga.HGA_ERR_INVALID_ARG
     assert str(hga.workspace_size(_p())) in lib.hga_last_error().decode()
+    # The fused routing + forward checks every pointer before any launch.
+    args = [good] * 10
+    for k, name in enumerate(("Q", "K", "V", "csum", "gsum", "qbar", "cidx", "gidx", "O", "lse")):
+        a = list(args)
+        a[k] = None
+        assert lib.hga_route_attn_fwd(ctypes.byref(p), *a, None) == hga.HGA_ERR_INVALID_ARG, name
+        assert f"{name} is NULL" in lib.hga_last_error().decode()
 
 
 def test_empty_segment_is_a_no_op(lib):
