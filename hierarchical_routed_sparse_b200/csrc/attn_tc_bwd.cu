@@ -74,7 +74,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int {
     kSiteQ = 201, kSiteFull, kSiteEmpty, kSiteSdp, kSitePs, kSiteKv, kSiteDrained, kSiteFinal, kSiteDrain,
-    kSiteQfree, kSiteDqfree, kSitePfree, kSiteDqs, kSiteSfree, kSiteFinalSdp
+    kSiteQfree, kSiteDqfree, kSitePfree, kSiteDqs, kSiteSfree, kSiteFinalSdp, kSiteDsum
 };
 
 template <int KST>                   // K stages
@@ -88,15 +88,16 @@ struct BwdSmem {
     static constexpr int k_off = x_off + 2 * kX;
     static constexpr int v_off = k_off + KST * H * kKVHalf;
     static constexpr int bar_off = v_off + kVStages * H * kKVHalf;
-    static constexpr int n_bars = 29;
+    static constexpr int n_bars = 30;
     static constexpr int tab_off = (bar_off + 8 * n_bars + 15) & ~15;   // int4 (item, n_g, n_seg) of the CTA's first items
     static constexpr int tmem_slot_off = tab_off + 16 * 64;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;
-    // Strictly causal variant: the row sums D of the CTA's 128 rows, then the
-    // window's union of routed groups (wu::bytes, sized at launch).
+    // Strictly causal variant: the four head-dim quarters' partial row sums
+    // D of the CTA's 128 rows, then the window's union of routed groups
+    // (wu::bytes, sized at launch).
     static constexpr int ds_off = bytes;
-    static constexpr int union_off = ds_off + 128 * 4;
+    static constexpr int union_off = ds_off + 4 * 128 * 4;
 };
 static_assert(BwdSmem<kKStages>::alloc <= 227 * 1024, "shared memory");
 static_assert(BwdSmem<kKStages>::tab_off % 16 == 0 && BwdSmem<kKStages>::bar_off % 8 == 0,
@@ -105,13 +106,14 @@ static_assert(BwdSmem<3>::union_off % 16 == 0, "union alignment");
 
 // mbarriers: q[2], kfull / kempty[kKStages], vfull / vempty[kVStages], sdp[2],
 // ps[2], kv, drained, pfree, qfree, dqfree, final, dqs_full, dqs_free, sfree[2],
-// final_sdp.
+// final_sdp, dsum (causal: the rows' partial sums D are in).
 constexpr int kBarQ = 0, kBarKFull = 2, kBarKEmpty = kBarKFull + kKStages, kBarVFull = kBarKEmpty + kKStages,
               kBarVEmpty = kBarVFull + kVStages, kBarSdp = kBarVEmpty + kVStages, kBarPs = kBarSdp + 2,
               kBarKv = kBarPs + 2, kBarDrained = kBarKv + 1, kBarPfree = kBarKv + 2, kBarQfree = kBarKv + 3,
               kBarDqfree = kBarKv + 4, kBarFinal = kBarKv + 5, kBarDqsFull = kBarKv + 6,
-              kBarDqsFree = kBarKv + 7, kBarSfree = kBarKv + 8, kBarFinalSdp = kBarSfree + 2;
-static_assert(kBarFinalSdp + 1 == BwdSmem<kKStages>::n_bars, "barrier count");
+              kBarDqsFree = kBarKv + 7, kBarSfree = kBarKv + 8, kBarFinalSdp = kBarSfree + 2,
+              kBarDsum = kBarFinalSdp + 1;
+static_assert(kBarDsum + 1 == BwdSmem<kKStages>::n_bars, "barrier count");
 
 // Tensor-memory columns.
 constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDV = 384, kColDK = 448;
@@ -258,6 +260,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     auto bar_ps = [&](int b) { return bar0 + 8 * (kBarPs + b); };
     auto bar_sfree = [&](int b) { return bar0 + 8 * (kBarSfree + b); };   // dQ of the buffer's tile done
     const uint32_t bar_final_sdp = bar0 + 8 * kBarFinalSdp;
+    const uint32_t bar_dsum = bar0 + 8 * kBarDsum;
     const uint32_t bar_kv = bar0 + 8 * kBarKv;
     const uint32_t bar_drained = bar0 + 8 * kBarDrained;
     const uint32_t bar_pfree = bar0 + 8 * kBarPfree;
@@ -298,43 +301,39 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_init(bar_dqs_full, kCompute);
         mbar_init(bar_dqs_free, 1);
         mbar_init(bar_final_sdp, 1);
+        mbar_init(bar_dsum, kCompute);
         fence_mbar_init();
     }
     if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
     // Setup above touches no global memory; the inputs are read from here on.
     pdl_wait();
     pdl_trigger();
-    float* Ds = reinterpret_cast<float*>(smem + L::ds_off);      // causal: row sums D
+    float* Ds = reinterpret_cast<float*>(smem + L::ds_off);      // causal: partial row sums D [4][128]
     wu::View uv{};
     if constexpr (CAUSAL) {
-        // The CTA's one item: the union of its window's routed groups, its
-        // segment tiles and the row sums D = rowsum(dO * O) of its rows.
+        // The CTA's one item: the union of its window's routed groups and its
+        // segment tiles (the rows' sums D are formed by the compute warps
+        // while the first tile's S / dP run).
         __shared__ int s_n, s_hist;
         Item m0;
         decode_item<true>(a, blockIdx.x, m0);
         uv = wu::view(smem + L::union_off, a.n_groups, a.wg);
-        if (threadIdx.x == 0) s_hist = 0;
+        if (threadIdx.x == 0) {
+            s_hist = 0;
+            // The item's rows of O (read when the rows' sums D are formed):
+            // into L2 now, one contiguous run of rows per q-head.
+            const int b0 = m0.bg / a.Hkv, g0 = m0.bg % a.Hkv;
+            for (int h = 0; h < kHeads && m0.head0 + h < a.G; ++h) {
+                const int64_t row = ((int64_t)(b0 * a.Hq + g0 * a.G + m0.head0 + h)) * a.T_seg + m0.w0;
+                bulk_prefetch_l2(a.O + row * a.d, uint32_t(kRows * a.d * 4));
+            }
+        }
         const int n = wu::build(a.gidx + ((int64_t)m0.bg * a.T_seg + m0.w0) * a.wg, a.wg, m0.own0 / 8, uv, &s_n,
                                 chk::kSiteCausalBwd);
         int c = 0;
         for (int k = threadIdx.x; k < n; k += kThreads) c += uv.list[k] < a.T_hist / 8;
         c = __reduce_add_sync(0xFFFFFFFFu, c);
         if (lane == 0 && c) atomicAdd(&s_hist, c);
-        const int b = m0.bg / a.Hkv, g = m0.bg % a.Hkv;
-        for (int rr = warp; rr < 128; rr += kThreads / 32) {
-            const int head = m0.head0 + rr / kRows;
-            float acc = 0.f;
-            if (head < a.G) {
-                const int64_t row = ((int64_t)(b * a.Hq + g * a.G + head)) * a.T_seg + m0.w0 + rr % kRows;
-                for (int e = 2 * lane; e < a.d; e += 64) {
-                    const float2 o = __ldg(reinterpret_cast<const float2*>(a.O + row * a.d + e));
-                    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(a.dO + row * a.d + e));
-                    acc += o.x * __uint_as_float(w << 16) + o.y * __uint_as_float(w & 0xFFFF0000u);
-                }
-            }
-            acc = warp_sum(acc);
-            if (lane == 0) Ds[rr] = acc;
-        }
         __syncthreads();
         if (threadIdx.x == 0) {
             const int n_rt = (n + 7) / 8, c_hist = s_hist;
@@ -625,7 +624,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ri.row = int((b * a.Hq + g * a.G + head) * a.T_seg) + m.w0 + qi;
             ri.own_lim = int(a.T_hist) + m.w0 + qi - m.own0;   // own-chunk keys 0 .. own_lim visible
             ri.lse2 = ri.ok ? __ldg(a.lse + ri.row) * kLog2e : 0.f;
-            if constexpr (CAUSAL) ri.Dr = ri.ok ? Ds[r] : 0.f;
+            if constexpr (CAUSAL) ri.Dr = 0.f;                 // formed at the item's first tile
             else ri.Dr = ri.ok ? __ldg(a.Drow + ri.row) : 0.f;
             return ri;
         };
@@ -636,7 +635,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int k = 0; k < n_mine && ok; ++k) {
             const bool row_ok = ri.ok;
             const int own_lim = ri.own_lim;
-            const float lse2 = ri.lse2, Dr = ri.Dr;
+            const float lse2 = ri.lse2;
+            float Dr = ri.Dr;
             const uint32_t pd = xbuf(k + 1) - sbase;        // this item's P / dS buffer
             uint8_t* prow_hi = smem + pd + r * 128;
             uint8_t* prow_lo = prow_hi + L::kRows128;
@@ -654,6 +654,42 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ok = mbar_wait(bar_sdp(bb), (gt >> 1) & 1, kSiteSdp);
                 if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
                 tc_fence_after();
+                if constexpr (CAUSAL) {
+                    if (p == 0) {
+                        // D = rowsum(dO * O) of row r: this thread's quarter kq of
+                        // its row of O (prefetched into L2 by the prologue) and of
+                        // the row of dO in shared memory (its load is complete:
+                        // bar_q), the four quarters summed through shared memory.
+                        ok = mbar_wait(bar_q(k & 1), (k >> 1) & 1, kSiteQ);
+                        float part = 0.f;
+                        if (row_ok && 32 * kq < a.d) {
+                            float4 o4[8];
+                            const float4* src = reinterpret_cast<const float4*>(a.O + (int64_t)ri.row * a.d + 32 * kq);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) o4[j] = __ldg(src + j);
+                            const uint8_t* drow =
+                                smem + (xbuf(k) - sbase) + 2 * L::kRows128 + (kq / 2) * L::kRows128 + r * 128;
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj) {
+                                const int phys = ((kq % 2) * 4 + jj) ^ (r & 7);   // 128-byte swizzle
+                                const uint4 w4 = *reinterpret_cast<const uint4*>(drow + phys * 16);
+                                const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+                                const float4 oa = o4[2 * jj], ob = o4[2 * jj + 1];
+                                const float of[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    part = fmaf(__uint_as_float(w[e] << 16), of[2 * e], part);
+                                    part = fmaf(__uint_as_float(w[e] & 0xFFFF0000u), of[2 * e + 1], part);
+                                }
+                            }
+                        }
+                        Ds[kq * 128 + r] = part;
+                        mbar_arrive(bar_dsum);
+                        if (ok) ok = mbar_wait(bar_dsum, 0, kSiteDsum);
+                        if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
+                        Dr = row_ok ? (Ds[r] + Ds[128 + r]) + (Ds[256 + r] + Ds[384 + r]) : 0.f;
+                    }
+                }
                 const bool own = t == n_rt;
                 uint32_t sr[16], pr[16];
                 tmem_ld16(tmem + lane_off + kColS + bb * kKeys + 16 * kq, sr);
