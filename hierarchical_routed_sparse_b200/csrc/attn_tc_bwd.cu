@@ -93,11 +93,9 @@ struct BwdSmem {
     static constexpr int tmem_slot_off = tab_off + 16 * 64;
     static constexpr int bytes = tmem_slot_off + 16;
     static constexpr int alloc = bytes + 1024;
-    // Strictly causal variant: the four head-dim quarters' partial row sums
-    // D of the CTA's 128 rows, then the window's union of routed groups
+    // Strictly causal variant: the window's union of routed groups
     // (wu::bytes, sized at launch).
-    static constexpr int ds_off = bytes;
-    static constexpr int union_off = ds_off + 4 * 128 * 4;
+    static constexpr int union_off = (bytes + 15) & ~15;
 };
 static_assert(BwdSmem<kKStages>::alloc <= 227 * 1024, "shared memory");
 static_assert(BwdSmem<kKStages>::tab_off % 16 == 0 && BwdSmem<kKStages>::bar_off % 8 == 0,
@@ -122,7 +120,7 @@ struct BwdArgs {
     const int32_t* gidx;
     const int32_t* sched;      // CTA c's k-th item at sched[k * gridDim.x + c]
     const float* lse;
-    const float* Drow;
+    const float* Drow;         // block path: the row sums D of the row-dot launch
     float* dQ;
     float* dK;
     float* dV;
@@ -130,7 +128,7 @@ struct BwdArgs {
     int64_t T_hist, T_seg, nQB, n_items;
     int64_t cap;               // K / V rows per (batch, kv-head)
     int64_t nWin, n_groups;    // strictly causal variant: windows per (b, g); groups of the context
-    const float* O;            // strictly causal variant: O and dO for the row sums
+    const float* O;            // strictly causal variant: O, for the row sums D = rowsum(dO * O)
     const __nv_bfloat16* dO;
     int q_rows;
     float scale, scale_log2;
@@ -308,26 +306,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // Setup above touches no global memory; the inputs are read from here on.
     pdl_wait();
     pdl_trigger();
-    float* Ds = reinterpret_cast<float*>(smem + L::ds_off);      // causal: partial row sums D [4][128]
     wu::View uv{};
     if constexpr (CAUSAL) {
         // The CTA's one item: the union of its window's routed groups and its
-        // segment tiles (the rows' sums D are formed by the compute warps
-        // while the first tile's S / dP run).
+        // segment tiles.
         __shared__ int s_n, s_hist;
         Item m0;
         decode_item<true>(a, blockIdx.x, m0);
         uv = wu::view(smem + L::union_off, a.n_groups, a.wg);
-        if (threadIdx.x == 0) {
-            s_hist = 0;
-            // The item's rows of O (read when the rows' sums D are formed):
-            // into L2 now, one contiguous run of rows per q-head.
-            const int b0 = m0.bg / a.Hkv, g0 = m0.bg % a.Hkv;
-            for (int h = 0; h < kHeads && m0.head0 + h < a.G; ++h) {
-                const int64_t row = ((int64_t)(b0 * a.Hq + g0 * a.G + m0.head0 + h)) * a.T_seg + m0.w0;
-                bulk_prefetch_l2(a.O + row * a.d, uint32_t(kRows * a.d * 4));
-            }
-        }
+        if (threadIdx.x == 0) s_hist = 0;
         const int n = wu::build(a.gidx + ((int64_t)m0.bg * a.T_seg + m0.w0) * a.wg, a.wg, m0.own0 / 8, uv, &s_n,
                                 chk::kSiteCausalBwd);
         int c = 0;
@@ -378,6 +365,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tma_load_2d(xbuf(kq_) + off, &tm_q, 64 * c, y, bar_q(kq_ & 1));
                     tma_load_2d(xbuf(kq_) + 2 * L::kRows128 + off, &tm_do, 64 * c, y, bar_q(kq_ & 1));
                 }
+                // Causal: the item's rows of O, read when its rows' sums D are formed.
+                if (CAUSAL && head < a.G) bulk_prefetch_l2(a.O + (int64_t)y * a.d, uint32_t(kRows * a.d * 4));
             }
         };
         int last_k[KST], last_v[kVStages];              // last tile loaded per stage
@@ -657,10 +646,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if constexpr (CAUSAL) {
                     if (p == 0) {
                         // D = rowsum(dO * O) of row r: this thread's quarter kq of
-                        // its row of O (prefetched into L2 by the prologue) and of
-                        // the row of dO in shared memory (its load is complete:
-                        // bar_q), the four quarters summed through shared memory.
+                        // its row of O (prefetched into L2 with the item's Q / dO)
+                        // and of the row of dO in shared memory (its load is
+                        // complete: bar_q).  The four quarters meet in the dQ
+                        // columns of tensor memory, free until the item's first dQ
+                        // MMA (which waits for this tile's dS) once the previous
+                        // item's dQ has been read out (dqfree).
                         ok = mbar_wait(bar_q(k & 1), (k >> 1) & 1, kSiteQ);
+                        if (ok && k > 0) ok = mbar_wait(bar_dqfree, (k - 1) & 1, kSiteDqfree);
                         float part = 0.f;
                         if (row_ok && 32 * kq < a.d) {
                             float4 o4[8];
@@ -683,11 +676,19 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 }
                             }
                         }
-                        Ds[kq * 128 + r] = part;
+                        tmem_st1(tmem + lane_off + kColDQ + kq, __float_as_uint(part));
+                        tmem_wait_st();
+                        tc_fence_before();
                         mbar_arrive(bar_dsum);
-                        if (ok) ok = mbar_wait(bar_dsum, 0, kSiteDsum);
+                        if (ok) ok = mbar_wait(bar_dsum, k & 1, kSiteDsum);
                         if (__any_sync(0xFFFFFFFFu, !ok)) { ok = false; break; }
-                        Dr = row_ok ? (Ds[r] + Ds[128 + r]) + (Ds[256 + r] + Ds[384 + r]) : 0.f;
+                        tc_fence_after();
+                        uint32_t dp[4];
+                        tmem_ld4(tmem + lane_off + kColDQ, dp);
+                        tmem_wait_ld();
+                        Dr = row_ok ? (__uint_as_float(dp[0]) + __uint_as_float(dp[1])) +
+                                          (__uint_as_float(dp[2]) + __uint_as_float(dp[3]))
+                                    : 0.f;
                     }
                 }
                 const bool own = t == n_rt;
@@ -1072,7 +1073,6 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
 {
     const int64_t rows = (int64_t)s.B * s.Hq * s.T_seg;
     const int64_t n4 = (int64_t)s.B * s.Hkv * s.T_seg * s.d / 4;   // d = 64 or 128: whole float4s
-    const int64_t rows_per_cta = 8 * kRowdotRows;
     const int64_t n_items = bwd_items(s);
     const int64_t grid = std::min<int64_t>(n_items, sm_count());
     // The scratch holds the row sums, then the schedule (Drow + rows).
@@ -1085,6 +1085,7 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
     sa.n_pairs = (s.G + 1) / 2;
     sa.wg = s.wg;
     sa.G = (int)grid;
+    const int64_t rows_per_cta = 8 * kRowdotRows;
     auto rowdot = s.d == 128 ? rowdot_kernel<128> : rowdot_kernel<64>;
     cudaError_t e = launch_pdl(rowdot, dim3((unsigned)(1 + (rows + rows_per_cta - 1) / rows_per_cta)),
                                dim3(256), 0, st, O, static_cast<const __nv_bfloat16*>(dO), Drow, rows,
@@ -1098,10 +1099,12 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
         !make_bf16_map(&tk64, K, kv_rows, s.d, 64) || !make_bf16_map(&tv64, V, kv_rows, s.d, 64) ||
         !make_f32_map(&tdq, dQ, q_rows, s.d, 64))
         return cudaErrorInvalidValue;
-    BwdArgs a;
+    BwdArgs a{};
     a.gidx = gidx;
     a.lse = lse;
     a.Drow = Drow;
+    a.O = O;
+    a.dO = static_cast<const __nv_bfloat16*>(dO);
     a.dQ = dQ;
     a.dK = dK_seg;
     a.dV = dV_seg;
@@ -1154,8 +1157,8 @@ cudaError_t launch_attn_bwd_tc_causal(const Shape& s, const void* Q, const void*
     BwdArgs a{};
     a.gidx = gidx;
     a.sched = nullptr;
-    a.lse = lse;
     a.Drow = nullptr;
+    a.lse = lse;
     a.dQ = dQ;
     a.dK = dK_seg;
     a.dV = dV_seg;
