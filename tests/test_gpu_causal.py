@@ -127,13 +127,15 @@ def test_outputs_do_not_see_later_positions(w):
     assert maxabs(a["O"][:, :, p + 1:], b["O"][:, :, p + 1:]) > 1e-2
 
 
-@pytest.mark.parametrize("T", [32768, 131072])
-def test_causal_long_context_sampled_units(T):
-    # Per-position routing over up to 511 / 2047 eligible chunks (the warp
-    # router's selection over shared memory), k_c 16, k_g 64: the whole
-    # problem on the GPU, two (batch, kv-head) units against the oracle.
+@pytest.mark.parametrize("T,k_c,k_g", [(32768, 16, 64), (131072, 16, 64), (32768, 8, 32)])
+def test_causal_long_context_sampled_units(T, k_c, k_g):
+    # Per-position routing over up to 511 / 2047 eligible chunks: at 32K the
+    # window router (k_c 16: rounds over the scores in shared memory; k_c 8:
+    # eight lanes a row past 256 candidates), at 128K the warp-per-row
+    # router.  The whole problem on the GPU, two (batch, kv-head) units
+    # against the oracle.
     from parity_util import unit_slice
-    w = W.sweep_point(T, 16, 64).with_(B=1)
+    w = W.sweep_point(T, k_c, k_g).with_(B=1)
     x = w.full()
     got = _run(w, x)
     for g in (0, w.Hkv - 1):
