@@ -793,7 +793,7 @@ causal_fwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
     const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
     const int64_t bg = row / T_seg, i = row % T_seg;
     const int64_t b = bg / Hkv, g = bg % Hkv;
-    const int64_t T = T_hist + T_seg, pos = T_hist + i, own0 = pos / kChunk * kChunk;
+    const int64_t pos = T_hist + i, own0 = pos / kChunk * kChunk;
     const int32_t* grow = gidx + row * wg;
     const int n_g = prefix_count(grow, wg, lane);
     const int n_keys = kGroup * n_g + int(pos - own0) + 1;
@@ -907,7 +907,7 @@ causal_bwd_kernel(const TIn* __restrict__ Q, const TIn* __restrict__ K, const TI
     const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
     const int64_t bg = row / T_seg, i = row % T_seg;
     const int64_t b = bg / Hkv, g = bg % Hkv;
-    const int64_t T = T_hist + T_seg, pos = T_hist + i, own0 = pos / kChunk * kChunk;
+    const int64_t pos = T_hist + i, own0 = pos / kChunk * kChunk;
     const int32_t* grow = gidx + row * wg;
     const int n_g = prefix_count(grow, wg, lane);
     const int n_keys = kGroup * n_g + int(pos - own0) + 1;
