@@ -925,7 +925,8 @@ def run_causal(args, w) -> None:
                               peak_source=pk["source"] + " (burst copy)"),
                 e2e=dict(value=w.B * w.T_seg / (e2e_ms * 1e-3), unit="tokens/s", h2d_bytes_per_step=h2d,
                          d2h_bytes_per_step=d2h),
-                gpu_launches=(1 + 1 + 1 + 1) * args.steps, clocks=clk.summary())
+                # summaries, routing + the window schedule's two kernels, forward, backward
+                gpu_launches=(1 + 3 + 1 + 1) * args.steps, clocks=clk.summary())
     print(json.dumps(line), flush=True)
 
 

@@ -27,8 +27,8 @@ CHECKED_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib
 EXPORTS = ("hga_route_widths", "hga_workspace_size", "hga_build_summaries", "hga_build_summaries_rows",
            "hga_route_chunks",
            "hga_route_groups", "hga_route", "hga_attn_fwd", "hga_route_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
-           "hga_stage_params", "hga_stage_routed", "hga_decode", "hga_route_causal", "hga_attn_fwd_causal",
-           "hga_attn_bwd_causal", "hga_device_status", "hga_device_check", "hga_checked_build",
+           "hga_stage_params", "hga_stage_routed", "hga_decode", "hga_route_causal", "hga_causal_sched_size",
+           "hga_causal_schedule", "hga_attn_fwd_causal", "hga_attn_bwd_causal", "hga_device_status", "hga_device_check", "hga_checked_build",
            "hga_selftest_wait", "hga_last_error",
            "hga_version")
 NOALLOC_MAX_ROWS = 1 << 20     # HGA_NOALLOC_MAX_ROWS
@@ -126,8 +126,10 @@ def load() -> ctypes.CDLL:
             "hga_stage_routed": ([PP, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_decode": ([PP, I64, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_route_causal": ([PP, P, P, P, P, P, P], ctypes.c_int),
-            "hga_attn_fwd_causal": ([PP, P, P, P, P, P, P, P], ctypes.c_int),
-            "hga_attn_bwd_causal": ([PP, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "hga_causal_sched_size": ([PP], ctypes.c_size_t),
+            "hga_causal_schedule": ([PP, P, P, P], ctypes.c_int),
+            "hga_attn_fwd_causal": ([PP, P, P, P, P, P, P, P, P], ctypes.c_int),
+            "hga_attn_bwd_causal": ([PP, P, P, P, P, P, P, P, P, P, P, P, P], ctypes.c_int),
             "hga_device_status": ([ctypes.POINTER(ctypes.c_int), ctypes.c_int], ctypes.c_int),
             "hga_selftest_wait": ([ctypes.c_int, ctypes.POINTER(ctypes.c_int), P], ctypes.c_int),
             "hga_device_check": ([ctypes.POINTER(ctypes.c_int), ctypes.c_int], ctypes.c_int),
@@ -315,21 +317,33 @@ def route_causal(p: Params, Q, csum, gsum, cidx, gidx, stream=None) -> None:
                                    _stream(stream)))
 
 
-def attn_fwd_causal(p: Params, Q, K, V, gidx, O, lse, stream=None) -> None:
-    _check(load().hga_attn_fwd_causal(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(gidx), _ptr(O),
-                                      _ptr(lse), _stream(stream)))
+def causal_sched_size(p: Params) -> int:
+    """Bytes of the causal window schedule (int32 [2 * n_items])."""
+    return int(load().hga_causal_sched_size(ctypes.byref(p.c())))
 
 
-def attn_bwd_causal(p: Params, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, stream=None) -> None:
+def causal_schedule(p: Params, gidx, sched, stream=None) -> None:
+    """Order the causal attention's window items heaviest first (sched[:n]),
+    their costs in sched[n:]."""
+    _check(load().hga_causal_schedule(ctypes.byref(p.c()), _ptr(gidx), _ptr(sched), _stream(stream)))
+
+
+def attn_fwd_causal(p: Params, Q, K, V, gidx, O, lse, stream=None, sched=None) -> None:
+    _check(load().hga_attn_fwd_causal(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(gidx), _ptr(sched),
+                                      _ptr(O), _ptr(lse), _stream(stream)))
+
+
+def attn_bwd_causal(p: Params, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg, stream=None, sched=None) -> None:
     _check(load().hga_attn_bwd_causal(ctypes.byref(p.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
-                                      _ptr(dO), _ptr(gidx), _ptr(dQ), _ptr(dK_seg), _ptr(dV_seg),
+                                      _ptr(dO), _ptr(gidx), _ptr(sched), _ptr(dQ), _ptr(dK_seg), _ptr(dV_seg),
                                       _stream(stream)))
 
 
 class CausalBuffers:
     """Device buffers of the strictly causal variant for one problem shape:
-    routing rows per query position; ``step`` runs summaries, routing,
-    forward and (with dO) backward."""
+    routing rows per query position and the attention's window schedule
+    (built with the routing, ordering the window items heaviest first);
+    ``step`` runs summaries, routing, forward and (with dO) backward."""
 
     def __init__(self, p: Params, device="cuda"):
         self.p = p
@@ -346,6 +360,8 @@ class CausalBuffers:
         self.dQ = torch.empty(B, Hq, Ts, d, **f32)
         self.dK = torch.empty(B, Hkv, Ts, d, **f32)
         self.dV = torch.empty(B, Hkv, Ts, d, **f32)
+        self.sched = torch.empty(max(1, causal_sched_size(p) // 4), **i32)
+        self.sched_of = None          # the index rows the schedule was built from
 
     def summaries(self, K, t_begin=None, t_end=None, stream=None):
         t_begin = self.p.T_hist if t_begin is None else t_begin
@@ -354,13 +370,26 @@ class CausalBuffers:
 
     def route(self, Q, stream=None):
         route_causal(self.p, Q, self.csum, self.gsum, self.cidx, self.gidx, stream)
+        self.schedule(self.gidx, stream)
+
+    def schedule(self, gidx, stream=None):
+        """The window schedule of index rows `gidx` (any permutation gives the
+        same results; one built from the rows the attention runs on is the
+        balanced one)."""
+        causal_schedule(self.p, gidx, self.sched, stream)
+        self.sched_of = gidx
+
+    def _sched_for(self, gidx):
+        return self.sched if self.sched_of is gidx else None
 
     def forward(self, Q, K, V, gidx=None, stream=None):
-        attn_fwd_causal(self.p, Q, K, V, self.gidx if gidx is None else gidx, self.O, self.lse, stream)
+        gidx = self.gidx if gidx is None else gidx
+        attn_fwd_causal(self.p, Q, K, V, gidx, self.O, self.lse, stream, sched=self._sched_for(gidx))
 
     def backward(self, Q, K, V, dO, gidx=None, stream=None):
-        attn_bwd_causal(self.p, Q, K, V, self.O, self.lse, dO, self.gidx if gidx is None else gidx, self.dQ,
-                        self.dK, self.dV, stream)
+        gidx = self.gidx if gidx is None else gidx
+        attn_bwd_causal(self.p, Q, K, V, self.O, self.lse, dO, gidx, self.dQ, self.dK, self.dV, stream,
+                        sched=self._sched_for(gidx))
 
     def step(self, Q, K, V, dO=None, stream=None):
         self.summaries(K, stream=stream)

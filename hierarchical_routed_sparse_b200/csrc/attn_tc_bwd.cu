@@ -118,7 +118,7 @@ constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDV = 384, kColDK =
 
 struct BwdArgs {
     const int32_t* gidx;
-    const int32_t* sched;      // CTA c's k-th item at sched[k * gridDim.x + c]
+    const int32_t* sched;      // CTA c's k-th item at sched[k * gridDim.x + c] (causal: may be null, item c)
     const float* lse;
     const float* Drow;         // block path: the row sums D of the row-dot launch
     float* dQ;
@@ -230,10 +230,11 @@ __device__ __forceinline__ Item make_item(const BwdArgs& a, const int4* tab, int
 // many as round-robin would give it.  Barrier phases run on a global
 // key-tile counter (gt), a segment-tile counter (gs) and an item counter (k)
 // that every role advances identically.
-// CAUSAL: the strictly causal variant, one window item per CTA: its key tiles
-// are the union of the window's routed groups (built in the prologue with
-// the rows' sums D), rows are masked by their position's routing, and the
-// K ring has 3 stages to make room for the union.
+// CAUSAL: the strictly causal variant, one window item per CTA (CTA c runs
+// item sched[c], the items ordered heaviest first): its key tiles are the
+// union of the window's routed groups (built in the prologue with the rows'
+// sums D), rows are masked by their position's routing, and the K ring has
+// 3 stages to make room for the union.
 template <bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -311,8 +312,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // The CTA's one item: the union of its window's routed groups and its
         // segment tiles.
         __shared__ int s_n, s_hist;
+        const int it0 = int(chk::sched_item(a.sched));   // grid = items
         Item m0;
-        decode_item<true>(a, blockIdx.x, m0);
+        decode_item<true>(a, it0, m0);
         uv = wu::view(smem + L::union_off, a.n_groups, a.wg);
         if (threadIdx.x == 0) s_hist = 0;
         const int n = wu::build(a.gidx + ((int64_t)m0.bg * a.T_seg + m0.w0) * a.wg, a.wg, m0.own0 / 8, uv, &s_n,
@@ -324,7 +326,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         __syncthreads();
         if (threadIdx.x == 0) {
             const int n_rt = (n + 7) / 8, c_hist = s_hist;
-            tab[0] = make_int4(blockIdx.x, n, c_hist < n ? n_rt - c_hist / 8 + 1 : 1, 0);
+            tab[0] = make_int4(it0, n, c_hist < n ? n_rt - c_hist / 8 + 1 : 1, 0);
         }
     } else {
         // Decode the CTA's first items (warp w: items w, w + 19, ...).
@@ -1139,8 +1141,9 @@ bool attn_bwd_tc_causal_supported(const Shape& s)
 }
 
 cudaError_t launch_attn_bwd_tc_causal(const Shape& s, const void* Q, const void* K, const void* V, const float* O,
-                                      const float* lse, const void* dO, const int32_t* gidx, float* dQ,
-                                      float* dK_seg, float* dV_seg, cudaStream_t st)
+                                      const float* lse, const void* dO, const int32_t* gidx,
+                                      const int32_t* sched, float* dQ, float* dK_seg, float* dV_seg,
+                                      cudaStream_t st)
 {
     // dK / dV accumulate with atomics: zeroed first.
     const size_t seg_bytes = sizeof(float) * (size_t)s.B * s.Hkv * s.T_seg * s.d;
@@ -1156,7 +1159,7 @@ cudaError_t launch_attn_bwd_tc_causal(const Shape& s, const void* Q, const void*
         return cudaErrorInvalidValue;
     BwdArgs a{};
     a.gidx = gidx;
-    a.sched = nullptr;
+    a.sched = sched;                 // CTA x runs item sched[x] (null: item x)
     a.Drow = nullptr;
     a.lse = lse;
     a.dQ = dQ;

@@ -93,6 +93,7 @@ struct FwdArgs {
     int kv_rows;         // B*Hkv*cap (rows of the K / V maps)
     int64_t cap;         // K / V rows per (batch, kv-head)
     float scale_log2;
+    const int32_t* sched;  // strictly causal variant: CTA x runs item sched[x] (null: item x)
 };
 
 // One M-tile of the forward: query block (or causal window) u and q-heads
@@ -504,8 +505,10 @@ __device__ __forceinline__ void fwd_tile(const CUtensorMap* tm_q, const CUtensor
     }
 }
 
-// CTAs of one query block (window) are adjacent, so they run together and
-// share the K/V tiles through L2.
+// CTAs of one query block are adjacent, so they run together and share the
+// K/V tiles through L2.  Strictly causal variant: CTA x runs window item
+// sched[x], the items ordered heaviest first (one item per CTA, and an
+// item's time grows with its union's key tiles).
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k8,
@@ -514,8 +517,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 {
     constexpr int kHeads = CAUSAL ? 4 : 2;
     const int n_y = (a.G + kHeads - 1) / kHeads;
-    const int64_t u = blockIdx.x / n_y;                     // ((b*Hkv)+g)*nQB + qb, or the window
-    fwd_tile<D, CAUSAL, false>(&tm_q, &tm_k8, &tm_v8, &tm_k64, &tm_v64, a, u, kHeads * int(blockIdx.x % n_y),
+    int64_t it = blockIdx.x;
+    if constexpr (CAUSAL) {
+        // The items' order is an input: read once the previous launch is done.
+        pdl_wait();
+        it = chk::sched_item(a.sched);
+    }
+    const int64_t u = it / n_y;                             // ((b*Hkv)+g)*nQB + qb, or the window
+    fwd_tile<D, CAUSAL, false>(&tm_q, &tm_k8, &tm_v8, &tm_k64, &tm_v64, a, u, kHeads * int(it % n_y),
                                a.gidx + u * a.wg);
 }
 
@@ -613,7 +622,7 @@ route_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 // ---- host side -------------------------------------------------------------------------------------
 template <int D, bool CAUSAL>
 cudaError_t launch(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* gidx,
-                   float* O, float* lse, cudaStream_t st)
+                   const int32_t* sched, float* O, float* lse, cudaStream_t st)
 {
     CUtensorMap tq, tk8, tv8, tk64, tv64;
     constexpr int kRows = CAUSAL ? wu::kWin : 64;           // query rows of a head in a tile
@@ -639,6 +648,7 @@ cudaError_t launch(const Shape& s, const void* Q, const void* K, const void* V, 
     a.scale_log2 = s.scale * kLog2e;
     a.nWin = s.T_seg / wu::kWin;
     a.n_groups = s.nG;
+    a.sched = CAUSAL ? sched : nullptr;
     // One tile (a head pair of a query block, or four heads of a causal
     // window) per CTA, two CTAs per SM when shared memory allows.
     auto k = attn_fwd_tc_kernel<D, CAUSAL>;
@@ -724,8 +734,8 @@ bool attn_fwd_tc_supported(const Shape& s)
 cudaError_t launch_attn_fwd_tc(const Shape& s, const void* Q, const void* K, const void* V,
                                const int32_t* gidx, float* O, float* lse, cudaStream_t st)
 {
-    return s.d == 128 ? launch<128, false>(s, Q, K, V, gidx, O, lse, st)
-                      : launch<64, false>(s, Q, K, V, gidx, O, lse, st);
+    return s.d == 128 ? launch<128, false>(s, Q, K, V, gidx, nullptr, O, lse, st)
+                      : launch<64, false>(s, Q, K, V, gidx, nullptr, O, lse, st);
 }
 
 // Routing and forward in one launch: the tensor-core forward's shapes whose
@@ -760,10 +770,11 @@ bool attn_fwd_tc_causal_supported(const Shape& s)
 }
 
 cudaError_t launch_attn_fwd_tc_causal(const Shape& s, const void* Q, const void* K, const void* V,
-                                      const int32_t* gidx, float* O, float* lse, cudaStream_t st)
+                                      const int32_t* gidx, const int32_t* sched, float* O, float* lse,
+                                      cudaStream_t st)
 {
-    return s.d == 128 ? launch<128, true>(s, Q, K, V, gidx, O, lse, st)
-                      : launch<64, true>(s, Q, K, V, gidx, O, lse, st);
+    return s.d == 128 ? launch<128, true>(s, Q, K, V, gidx, sched, O, lse, st)
+                      : launch<64, true>(s, Q, K, V, gidx, sched, O, lse, st);
 }
 
 // Check word of this translation unit's bounds checks (checked builds).

@@ -44,6 +44,7 @@
 #include "hga_internal.cuh"
 #include "router_core.cuh"
 #include "sm100.cuh"
+#include "window_union.cuh"
 
 namespace hga {
 namespace {
@@ -1085,6 +1086,160 @@ template <typename TIn, int D, int GM> struct BwdOp {
     }
 };
 
+// ---- order of the tensor-core kernels' window items -------------------------
+// The causal tensor-core kernels run one window item per CTA, and an item's
+// time grows with the key tiles of its union (and, in the backward, with its
+// segment tiles): 15 to 59 tiles at 16K context.  The hardware hands CTAs
+// to SMs in index order as slots free up, so a heavy item drawn late ends
+// well after the rest.  These two kernels order the items heaviest first
+// (longest-processing-time-first list scheduling); the kernels then map
+// CTA x to item order[x].
+namespace csched {
+constexpr int kThreads = 128;
+constexpr int kMaxCost = 1023;        // costs are clamped here (they only order the items)
+
+// Cost of the items of window u (one CTA): 2 * (union tiles + own chunk) +
+// segment tiles, counted exactly as the kernels count them: the union of the
+// window's rows over the groups before its own chunk, and of those the
+// groups that hold segment tokens.
+__global__ void __launch_bounds__(kThreads)
+causal_cost_kernel(const int32_t* __restrict__ gidx, int32_t* __restrict__ cost, int64_t T_hist, int64_t T_seg,
+                   int64_t nWin, int wg, int n_y)
+{
+    extern __shared__ uint32_t bits[];                       // bitmap of the union
+    __shared__ int s_n, s_hist;
+    const int64_t u = blockIdx.x, bg = u / nWin, w0 = (u % nWin) * wu::kWin;
+    const int64_t limit = 8 * ((T_hist + w0) / 64);          // groups before the window's own chunk
+    const int nwords = int((limit + 31) / 32);
+    const int rows = int(T_seg - w0 < wu::kWin ? T_seg - w0 : wu::kWin);
+    for (int w = threadIdx.x; w < nwords; w += kThreads) bits[w] = 0u;
+    if (threadIdx.x == 0) {
+        s_n = 0;
+        s_hist = 0;
+    }
+    pdl_wait();
+    pdl_trigger();
+    __syncthreads();
+    const int32_t* row0 = gidx + (bg * T_seg + w0) * wg;
+    auto mark = [&](int32_t j) {
+        if (j >= 0 && j < limit) atomicOr(&bits[j >> 5], 1u << (j & 31));
+    };
+    if ((wg & 3) == 0) {
+        // The window's rows are contiguous: 16-byte loads, all issued first.
+        const int n4 = rows * wg / 4;
+        const int4* r4 = reinterpret_cast<const int4*>(row0);
+        constexpr int kPer = 4;                              // loads in flight per thread
+        for (int base = threadIdx.x; base < n4; base += kPer * kThreads) {
+            int4 v[kPer];
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                const int e = base + q * kThreads;
+                v[q] = e < n4 ? __ldg(r4 + e) : make_int4(-1, -1, -1, -1);
+            }
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                mark(v[q].x);
+                mark(v[q].y);
+                mark(v[q].z);
+                mark(v[q].w);
+            }
+        }
+    } else {
+        for (int e = threadIdx.x; e < rows * wg; e += kThreads) mark(__ldg(row0 + e));
+    }
+    __syncthreads();
+    const int64_t hist_groups = T_hist / 8;                  // groups wholly in detached history
+    int n = 0, h = 0;
+    for (int w = threadIdx.x; w < nwords; w += kThreads) {
+        const uint32_t x = bits[w];
+        const int64_t lo = 32 * (int64_t)w;
+        n += __popc(x);
+        if (lo + 32 <= hist_groups) h += __popc(x);
+        else if (lo < hist_groups) h += __popc(x & ((1u << (hist_groups - lo)) - 1u));
+    }
+    n = __reduce_add_sync(0xFFFFFFFFu, n);
+    h = __reduce_add_sync(0xFFFFFFFFu, h);
+    if ((threadIdx.x & 31) == 0) {
+        atomicAdd(&s_n, n);
+        atomicAdd(&s_hist, h);
+    }
+    __syncthreads();
+    if (threadIdx.x < n_y) {
+        const int nn = s_n, ch = s_hist, n_rt = (nn + 7) / 8;
+        const int n_seg = ch < nn ? n_rt - ch / 8 + 1 : 1;
+        const int c = 2 * (n_rt + 1) + n_seg;
+        cost[u * n_y + threadIdx.x] = c < kMaxCost ? c : kMaxCost;
+    }
+}
+
+// order[0 .. n) = the items by descending cost (cost[i] = order[n + i]),
+// equal costs in index order.  One CTA of kMaxCost + 1 threads: the costs
+// into shared memory (when they fit) with a histogram, the histogram's
+// exclusive prefix from the top (thread t owns cost kMaxCost - t), then one
+// warp places the items 32 at a time.
+constexpr int kOrderThreads = kMaxCost + 1;
+__global__ void __launch_bounds__(kOrderThreads) causal_order_kernel(int32_t* __restrict__ order, int n,
+                                                                     bool keys_in_smem)
+{
+    extern __shared__ int32_t s_cost[];                      // [n] when keys_in_smem
+    __shared__ int cursor[kMaxCost + 1];
+    __shared__ int wsum[32];
+    const int32_t* cost = order + n;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    cursor[threadIdx.x] = 0;
+    pdl_wait();
+    pdl_trigger();
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kOrderThreads) {
+        int32_t c = __ldg(cost + i);
+        c = c < 0 ? 0 : (c > kMaxCost ? kMaxCost : c);     // in range as written; kept in the bins regardless
+        if (keys_in_smem) s_cost[i] = c;
+        atomicAdd(&cursor[c], 1);
+    }
+    __syncthreads();
+    {
+        const int c = kMaxCost - int(threadIdx.x);
+        const int cnt = cursor[c];
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int v = wsum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, v, o);
+                if (lane >= o) v += y;
+            }
+            wsum[lane] = v;
+        }
+        __syncthreads();
+        cursor[c] = incl - cnt + (warp ? wsum[warp - 1] : 0);   // items of higher cost
+        __syncthreads();
+    }
+    if (warp == 0) {
+        const int32_t* keys = keys_in_smem ? s_cost : cost;
+        for (int base = 0; base < n; base += 32) {
+            const int i = base + lane;
+            int key = -1;
+            if (i < n) {
+                key = keys[i];
+                key = key < 0 ? 0 : (key > kMaxCost ? kMaxCost : key);
+            }
+            const unsigned same = __match_any_sync(0xFFFFFFFFu, key);
+            if (i < n) order[cursor[key] + __popc(same & ((1u << lane) - 1u))] = i;
+            __syncwarp();
+            if (i < n && lane == 31 - __clz(same)) cursor[key] += __popc(same);
+            __syncwarp();
+        }
+    }
+}
+}  // namespace csched
+
 }  // namespace
 
 size_t route_causal_smem(const Shape& s)
@@ -1105,23 +1260,50 @@ cudaError_t launch_route_causal(const Shape& s, const void* Q, const float* csum
 }
 
 cudaError_t launch_attn_fwd_causal(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* gidx,
-                                   float* O, float* lse, cudaStream_t st)
+                                   const int32_t* sched, float* O, float* lse, cudaStream_t st)
 {
     // bf16 on the tensor cores (windows of neighbouring positions over the
     // union of their routed groups); otherwise one warp per position.
-    if (attn_fwd_tc_causal_supported(s)) return launch_attn_fwd_tc_causal(s, Q, K, V, gidx, O, lse, st);
+    if (attn_fwd_tc_causal_supported(s)) return launch_attn_fwd_tc_causal(s, Q, K, V, gidx, sched, O, lse, st);
     return dispatch<FwdOp>(s, Q, K, V, gidx, O, lse, st);
 }
 
 cudaError_t launch_attn_bwd_causal(const Shape& s, const void* Q, const void* K, const void* V, const float* O,
-                                   const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK,
-                                   float* dV, cudaStream_t st)
+                                   const float* lse, const void* dO, const int32_t* gidx, const int32_t* sched,
+                                   float* dQ, float* dK, float* dV, cudaStream_t st)
 {
     // bf16 on the tensor cores (the forward's windows); otherwise one warp
     // per position.
     if (attn_bwd_tc_causal_supported(s))
-        return launch_attn_bwd_tc_causal(s, Q, K, V, O, lse, dO, gidx, dQ, dK, dV, st);
+        return launch_attn_bwd_tc_causal(s, Q, K, V, O, lse, dO, gidx, sched, dQ, dK, dV, st);
     return dispatch<BwdOp>(s, Q, K, V, O, lse, dO, gidx, dQ, dK, dV, st);
+}
+
+int64_t causal_items(const Shape& s)
+{
+    return (int64_t)s.B * s.Hkv * ((s.T_seg + wu::kWin - 1) / wu::kWin) * ((s.G + 3) / 4);
+}
+
+size_t causal_sched_smem(const Shape& s) { return 4 * (size_t)((s.nG + 31) / 32); }
+
+cudaError_t launch_causal_schedule(const Shape& s, const int32_t* gidx, int32_t* sched, cudaStream_t st)
+{
+    const int64_t n_win = (int64_t)s.B * s.Hkv * ((s.T_seg + wu::kWin - 1) / wu::kWin);
+    const int n_y = (s.G + 3) / 4;
+    const int n = (int)causal_items(s);
+    if (n == 0) return cudaSuccess;
+    const size_t smem = causal_sched_smem(s);
+    cudaError_t e = allow_smem(csched::causal_cost_kernel, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(csched::causal_cost_kernel, dim3((unsigned)n_win), dim3(csched::kThreads), smem, st, gidx,
+                   sched + n, s.T_hist, s.T_seg, (int64_t)((s.T_seg + wu::kWin - 1) / wu::kWin), s.wg, n_y);
+    if (e != cudaSuccess) return e;
+    // The costs in shared memory when they fit (all but huge problems).
+    const size_t key_bytes = 4 * (size_t)n;
+    const bool in_smem = key_bytes <= 160 * 1024;
+    if (in_smem && (e = allow_smem(csched::causal_order_kernel, (int)key_bytes)) != cudaSuccess) return e;
+    return launch_pdl(csched::causal_order_kernel, dim3(1), dim3(csched::kOrderThreads), in_smem ? key_bytes : 0,
+                      st, sched, n, in_smem);
 }
 
 // Check word of this translation unit's bounds checks (checked builds).

@@ -32,7 +32,7 @@ constexpr bool kEnabled = false;
 // Site codes (which kernel and which read).
 enum : int {
     kSiteFwdTc = 401, kSiteBwdTcLoad, kSiteBwdTcKeys, kSiteSimtFwd, kSiteSimtBwd, kSiteCausalFwd,
-    kSiteCausalBwd, kSiteRouteGroups, kSiteStage
+    kSiteCausalBwd, kSiteRouteGroups, kSiteStage, kSiteCausalSched
 };
 
 __device__ __forceinline__ int32_t index(int32_t j, int64_t limit, int site)
@@ -53,6 +53,20 @@ __device__ __forceinline__ int32_t chunk(int32_t c, int64_t limit, int site) { r
 __device__ __forceinline__ void flag_if(bool bad, int site)
 {
     if (kEnabled && bad) atomicCAS(&g_check, 0, site);
+}
+
+// Item sched[x] of a caller's item order for CTA x of a one-item-per-CTA
+// grid.  Checked in every build (one load per CTA): an entry outside
+// [0, gridDim.x) is replaced by x, so no item index leaves the grid's range,
+// and checked builds record it.
+__device__ __forceinline__ int64_t sched_item(const int32_t* sched)
+{
+    const int64_t x = blockIdx.x;
+    if (!sched) return x;
+    const int32_t it = __ldg(sched + x);
+    const bool bad = it < 0 || (uint32_t)it >= gridDim.x;
+    flag_if(bad, kSiteCausalSched);
+    return bad ? x : it;
 }
 
 }  // namespace chk

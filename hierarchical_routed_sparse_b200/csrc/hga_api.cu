@@ -450,8 +450,33 @@ int hga_route_causal(const hga_params* p, const void* Q, const float* csum, cons
     return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route_causal");
 }
 
+size_t hga_causal_sched_size(const hga_params* p)
+{
+    hga::Shape s{};
+    if (causal_shape(p, &s)) return 0;
+    return 2 * sizeof(int32_t) * (size_t)hga::causal_items(s);
+}
+
+int hga_causal_schedule(const hga_params* p, const int32_t* gidx, int32_t* sched, hga_stream_t stream)
+{
+    const NvtxRange nvtx_range("hga_causal_schedule");
+    hga::Shape s{};
+    if (int r = causal_shape(p, &s)) return r;
+    if (hga::causal_items(s) == 0) return HGA_OK;
+    CHECK_PTR(gidx);
+    CHECK_PTR(sched);
+    if (hga::causal_items(s) > INT32_MAX / 2)
+        return fail(HGA_ERR_UNSUPPORTED, "%lld window items exceed the schedule's int32 range",
+                    (long long)hga::causal_items(s));
+    if (hga::causal_sched_smem(s) + 1024 > kMaxSmem)
+        return fail(HGA_ERR_UNSUPPORTED, "the schedule's bitmap of %lld groups exceeds shared memory",
+                    (long long)s.nG);
+    cudaError_t e = hga::launch_causal_schedule(s, gidx, sched, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_causal_schedule");
+}
+
 int hga_attn_fwd_causal(const hga_params* p, const void* Q, const void* K, const void* V, const int32_t* gidx,
-                        float* O, float* lse, hga_stream_t stream)
+                        const int32_t* sched, float* O, float* lse, hga_stream_t stream)
 {
     const NvtxRange nvtx_range("hga_attn_fwd_causal");
     hga::Shape s{};
@@ -461,15 +486,16 @@ int hga_attn_fwd_causal(const hga_params* p, const void* Q, const void* K, const
     CHECK_PTR(K);
     CHECK_PTR(V);
     CHECK_PTR(gidx);
+    if (sched) CHECK_PTR(sched);
     CHECK_PTR(O);
     CHECK_PTR(lse);
-    cudaError_t e = hga::launch_attn_fwd_causal(s, Q, K, V, gidx, O, lse, static_cast<cudaStream_t>(stream));
+    cudaError_t e = hga::launch_attn_fwd_causal(s, Q, K, V, gidx, sched, O, lse, static_cast<cudaStream_t>(stream));
     return finish(e, static_cast<cudaStream_t>(stream), "hga_attn_fwd_causal");
 }
 
 int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K, const void* V, const float* O,
-                        const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK_seg,
-                        float* dV_seg, hga_stream_t stream)
+                        const float* lse, const void* dO, const int32_t* gidx, const int32_t* sched, float* dQ,
+                        float* dK_seg, float* dV_seg, hga_stream_t stream)
 {
     const NvtxRange nvtx_range("hga_attn_bwd_causal");
     hga::Shape s{};
@@ -482,10 +508,11 @@ int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K, const
     CHECK_PTR(lse);
     CHECK_PTR(dO);
     CHECK_PTR(gidx);
+    if (sched) CHECK_PTR(sched);
     CHECK_PTR(dQ);
     CHECK_PTR(dK_seg);
     CHECK_PTR(dV_seg);
-    cudaError_t e = hga::launch_attn_bwd_causal(s, Q, K, V, O, lse, dO, gidx, dQ, dK_seg, dV_seg,
+    cudaError_t e = hga::launch_attn_bwd_causal(s, Q, K, V, O, lse, dO, gidx, sched, dQ, dK_seg, dV_seg,
                                                 static_cast<cudaStream_t>(stream));
     return finish(e, static_cast<cudaStream_t>(stream), "hga_attn_bwd_causal");
 }

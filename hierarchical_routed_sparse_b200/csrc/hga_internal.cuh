@@ -159,13 +159,21 @@ cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t st);
 // Strictly causal variant: routing per query position (causal.cu).
 cudaError_t launch_route_causal(const Shape& s, const void* Q, const float* csum, const float* gsum, int32_t* cidx,
                                 int32_t* gidx, cudaStream_t st);
+// sched: the order of the tensor-core kernels' window items (CTA x runs item
+// sched[x]), or null for index order; the warp-per-row kernels ignore it.
 cudaError_t launch_attn_fwd_causal(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* gidx,
-                                   float* O, float* lse, cudaStream_t st);
+                                   const int32_t* sched, float* O, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_causal(const Shape& s, const void* Q, const void* K, const void* V, const float* O,
-                                   const float* lse, const void* dO, const int32_t* gidx, float* dQ, float* dK,
-                                   float* dV, cudaStream_t st);
+                                   const float* lse, const void* dO, const int32_t* gidx, const int32_t* sched,
+                                   float* dQ, float* dK, float* dV, cudaStream_t st);
 size_t route_causal_smem(const Shape& s);
 int causal_max_heads();
+// Window items of the causal tensor-core kernels (B * Hkv * windows * head
+// quads), the schedule kernel's shared memory, and the schedule itself:
+// sched[0, n) the items heaviest first, sched[n, 2n) their costs.
+int64_t causal_items(const Shape& s);
+size_t causal_sched_smem(const Shape& s);
+cudaError_t launch_causal_schedule(const Shape& s, const int32_t* gidx, int32_t* sched, cudaStream_t st);
 cudaError_t launch_attn_fwd_simt(const Shape& s, const void* Q, const void* K, const void* V,
                                  const int32_t* gidx, float* O, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Shape& s, const void* Q, const void* K, const void* V,
@@ -194,7 +202,8 @@ cudaError_t launch_route_attn_fwd_tc(const Shape& s, const void* Q, const void* 
                                      float* lse, cudaStream_t st);
 bool attn_fwd_tc_causal_supported(const Shape& s);
 cudaError_t launch_attn_fwd_tc_causal(const Shape& s, const void* Q, const void* K, const void* V,
-                                      const int32_t* gidx, float* O, float* lse, cudaStream_t st);
+                                      const int32_t* gidx, const int32_t* sched, float* O, float* lse,
+                                      cudaStream_t st);
 bool attn_bwd_tc_supported(const Shape& s);
 cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, const void* V,
                                const float* O, const float* lse, const void* dO,
@@ -203,7 +212,8 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const void* Q, const void* K, con
 int attn_bwd_tc_status(bool clear);
 bool attn_bwd_tc_causal_supported(const Shape& s);
 cudaError_t launch_attn_bwd_tc_causal(const Shape& s, const void* Q, const void* K, const void* V, const float* O,
-                                      const float* lse, const void* dO, const int32_t* gidx, float* dQ,
-                                      float* dK_seg, float* dV_seg, cudaStream_t st);
+                                      const float* lse, const void* dO, const int32_t* gidx,
+                                      const int32_t* sched, float* dQ, float* dK_seg, float* dV_seg,
+                                      cudaStream_t st);
 
 }  // namespace hga

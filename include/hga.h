@@ -290,17 +290,38 @@ int hga_decode(const hga_params* p, int64_t pos, const void* q, const void* K,
  * and the other tensors are as for the block calls.  hga_attn_bwd_causal
  * zeroes dK_seg / dV_seg itself (they are accumulated with atomics, so
  * their float32 sums are not bit-reproducible run to run).  At most 8
- * q-heads per kv-head (HGA_ERR_UNSUPPORTED otherwise). */
+ * q-heads per kv-head (HGA_ERR_UNSUPPORTED otherwise).
+ *
+ * Schedule.  The bf16 attention calls run one CTA per window item (32
+ * neighbouring positions of a (batch, kv-head) and four of its q-heads),
+ * over the union of the window's routed groups; an item's time grows with
+ * that union, which the routing decides.  hga_causal_schedule orders the
+ * items by cost, heaviest first, from gidx:
+ *   sched      int32 [2 * n_items], n_items = B * Hkv * ceil(T_seg / 32)
+ *              * ceil(G / 4); hga_causal_sched_size gives its bytes (0 for
+ *              invalid parameters).  sched[0 .. n_items) is the order (a
+ *              permutation of the items), sched[n_items ..) their costs.
+ * Passing it to hga_attn_fwd_causal / hga_attn_bwd_causal changes only the
+ * order in which the items run, not their results (dQ, O and lse are the
+ * same bit for bit; dK / dV up to the order of their atomic sums); NULL runs
+ * the items in index order, and the float32 kernels ignore it.  It must be
+ * built from the gidx the attention calls are given.  Caller-owned device
+ * memory, 16-byte aligned. */
 int hga_route_causal(const hga_params* p, const void* Q, const float* csum,
                      const float* gsum, int32_t* cidx, int32_t* gidx,
                      hga_stream_t stream);
+size_t hga_causal_sched_size(const hga_params* p);
+int hga_causal_schedule(const hga_params* p, const int32_t* gidx,
+                        int32_t* sched, hga_stream_t stream);
 int hga_attn_fwd_causal(const hga_params* p, const void* Q, const void* K,
-                        const void* V, const int32_t* gidx, float* O,
-                        float* lse, hga_stream_t stream);
+                        const void* V, const int32_t* gidx,
+                        const int32_t* sched, float* O, float* lse,
+                        hga_stream_t stream);
 int hga_attn_bwd_causal(const hga_params* p, const void* Q, const void* K,
                         const void* V, const float* O, const float* lse,
-                        const void* dO, const int32_t* gidx, float* dQ,
-                        float* dK_seg, float* dV_seg, hga_stream_t stream);
+                        const void* dO, const int32_t* gidx,
+                        const int32_t* sched, float* dQ, float* dK_seg,
+                        float* dV_seg, hga_stream_t stream);
 
 /* Status word of the kernels' bounded waits: every wait of a tensor-core
  * kernel or of the decode kernel on a barrier gives up after one second, records the code of the wait

@@ -194,19 +194,36 @@ def test_causal_calls_reject_bad_arguments_on_the_host(lib):
     ok = ctypes.c_void_p(1 << 20)
     p9 = hga.Params(B=1, Hq=9, Hkv=1, d=128, T_hist=64, T_seg=64, k_c=2, k_g=4, dtype=hga.HGA_BF16).c()
     assert lib.hga_route_causal(ctypes.byref(p9), *([ok] * 5), None) == hga.HGA_ERR_UNSUPPORTED
-    assert lib.hga_attn_fwd_causal(ctypes.byref(p9), *([ok] * 6), None) == hga.HGA_ERR_UNSUPPORTED
-    assert lib.hga_attn_bwd_causal(ctypes.byref(p9), *([ok] * 10), None) == hga.HGA_ERR_UNSUPPORTED
+    assert lib.hga_attn_fwd_causal(ctypes.byref(p9), *([ok] * 7), None) == hga.HGA_ERR_UNSUPPORTED
+    assert lib.hga_attn_bwd_causal(ctypes.byref(p9), *([ok] * 11), None) == hga.HGA_ERR_UNSUPPORTED
+    assert lib.hga_causal_schedule(ctypes.byref(p9), ok, ok, None) == hga.HGA_ERR_UNSUPPORTED
+    assert lib.hga_causal_sched_size(ctypes.byref(p9)) == 0
     p = _p().c()
-    a = [ok] * 10
+    a = [ok] * 11
     a[6] = None
     assert lib.hga_attn_bwd_causal(ctypes.byref(p), *a, None) == hga.HGA_ERR_INVALID_ARG
     assert "gidx is NULL" in lib.hga_last_error().decode()
+    a = [ok] * 11
+    a[7] = ctypes.c_void_p((1 << 20) + 4)            # the schedule is optional, but aligned when given
+    assert lib.hga_attn_bwd_causal(ctypes.byref(p), *a, None) == hga.HGA_ERR_INVALID_ARG
+    assert "sched is not 16-byte aligned" in lib.hga_last_error().decode()
+    assert lib.hga_causal_schedule(ctypes.byref(p), ok, None, None) == hga.HGA_ERR_INVALID_ARG
+    assert "sched is NULL" in lib.hga_last_error().decode()
     assert lib.hga_route_causal(ctypes.byref(p), ok, ok, ctypes.c_void_p((1 << 20) + 4), ok, ok, None) == \
         hga.HGA_ERR_INVALID_ARG
     assert "gsum is not 16-byte aligned" in lib.hga_last_error().decode()
     # An empty segment is a no-op.
     p0 = _p(T_seg=0).c()
-    assert lib.hga_attn_fwd_causal(ctypes.byref(p0), *([None] * 6), None) == hga.HGA_OK
+    assert lib.hga_attn_fwd_causal(ctypes.byref(p0), *([None] * 7), None) == hga.HGA_OK
+    assert lib.hga_causal_schedule(ctypes.byref(p0), None, None, None) == hga.HGA_OK
+
+
+def test_causal_schedule_size():
+    # int32 order and costs of every window item: B * Hkv * ceil(T_seg / 32) * ceil(G / 4).
+    for kw, items in [(dict(B=2, Hq=8, Hkv=2, T_seg=256), 2 * 2 * 8 * 1),
+                      (dict(B=1, Hq=16, Hkv=2, T_seg=128), 1 * 2 * 4 * 2),
+                      (dict(B=1, Hq=2, Hkv=2, T_seg=64), 1 * 2 * 2 * 1)]:
+        assert hga.causal_sched_size(_p(**kw)) == 8 * items
 
 @pytest.mark.parametrize("compiler,suffix", [("gcc", ".c"), ("g++", ".cpp")])
 def test_plain_c_and_cpp_callers_link_and_call(lib, tmp_path, compiler, suffix):

@@ -152,3 +152,57 @@ def test_causal_long_context_sampled_units(T, k_c, k_g):
         same = (got["gidx"][:, g:g + 1] == orc["gidx"]).all(axis=-1)       # [1, 1, T_seg]
         rows = np.repeat(same, w.G, axis=1)
         assert maxabs(got["O"][:, hs][rows], orc["O"][rows]) <= TOL[w.dtype]
+
+
+def _window_costs(w, gidx):
+    """Cost of every window item as the schedule counts it, from the index
+    rows alone: 2 * (union tiles + own chunk) + segment tiles, where the union
+    is that of the window's 32 rows over the groups before its own chunk."""
+    n_y = (w.G + 3) // 4
+    cost = []
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            for w0 in range(0, w.T_seg, 32):
+                rows = gidx[b, g, w0:w0 + 32]
+                limit = 8 * ((w.T_hist + w0) // 64)
+                u = np.unique(rows[(rows >= 0) & (rows < limit)])
+                n, c_hist = len(u), int((u < w.T_hist // 8).sum())
+                n_rt = (n + 7) // 8
+                n_seg = n_rt - c_hist // 8 + 1 if c_hist < n else 1
+                cost += [min(2 * (n_rt + 1) + n_seg, 1023)] * n_y
+    return np.array(cost, dtype=np.int64)
+
+
+@pytest.mark.parametrize("w", [CASES[0], CASES[3], CASES[4], W.QWEN3_CTX16K_TRAIN], ids=lambda w: w.name)
+def test_window_schedule(w):
+    # The schedule orders the window items by cost, heaviest first, equal
+    # costs in index order (a stable sort of the costs counted from the
+    # index rows here), and changes only the order the items run in: O, lse
+    # and dQ equal the unscheduled launch's bit for bit, dK / dV (float
+    # atomics in another order) within float rounding.
+    x = w.full()
+    p = hga.Params.from_workload(w)
+    Q, K, V, dO = (to_dev(x[k], w.dtype) for k in ("Q", "K", "V", "dO"))
+    cb = hga.CausalBuffers(p)
+    cb.summaries(K, 0, w.T)
+    cb.route(Q)
+    torch.cuda.synchronize()
+    n = hga.causal_sched_size(p) // 8
+    sched = cb.sched.cpu().numpy()
+    cost = _window_costs(w, cb.gidx.cpu().numpy())
+    assert len(cost) == n
+    assert np.array_equal(sched[n:], cost)
+    assert np.array_equal(sched[:n], np.argsort(-cost, kind="stable"))
+    out = {}
+    for use in (True, False):
+        s = cb.sched if use else None
+        hga.attn_fwd_causal(p, Q, K, V, cb.gidx, cb.O, cb.lse, sched=s)
+        hga.attn_bwd_causal(p, Q, K, V, cb.O, cb.lse, dO, cb.gidx, cb.dQ, cb.dK, cb.dV, sched=s)
+        torch.cuda.synchronize()
+        assert hga.device_status() == 0
+        out[use] = {k: getattr(cb, k).cpu().numpy() for k in ("O", "lse", "dQ", "dK", "dV")}
+    for k in ("O", "lse", "dQ"):
+        assert np.array_equal(out[True][k], out[False][k]), k
+    for k in ("dK", "dV"):
+        ref = out[False][k]
+        assert maxabs(out[True][k], ref) <= 1e-5 * (1.0 + np.abs(ref).max()), k

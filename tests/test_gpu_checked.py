@@ -10,7 +10,8 @@ HGA_ERR_DEVICE_CHECK.  Checked here:
   * one planted out-of-range entry in an index row makes the forward, the
     backward, the float32 path, the strictly causal forward and the group
     router report HGA_ERR_DEVICE_CHECK without a fault, and the device is
-    usable afterwards.
+    usable afterwards; so does an out-of-range entry of a causal window
+    schedule in the causal forward and backward.
 The release build never sees a planted index.
 """
 import numpy as np
@@ -118,3 +119,28 @@ def test_planted_index_in_causal_rows_is_reported():
     cb.forward(Q, K, V)
     torch.cuda.synchronize()
     assert torch.isfinite(cb.O).all()
+
+
+def test_planted_schedule_entry_is_reported():
+    # A window schedule entry outside the grid: every build runs the CTA's
+    # own item instead (no item index leaves the grid's range); the checked
+    # build also reports it.
+    w = W_BF16
+    x = w.full()
+    p = hga.Params.from_workload(w)
+    cb = hga.CausalBuffers(p)
+    Q, K, V, dO = (to_dev(x[k], w.dtype) for k in ("Q", "K", "V", "dO"))
+    cb.summaries(K, 0, w.T)
+    cb.route(Q)
+    n = hga.causal_sched_size(p) // 8
+    for entry in (n + 5, -1):
+        sched = cb.sched.clone()
+        sched[1] = entry
+        _expect_check(lambda: hga.attn_fwd_causal(p, Q, K, V, cb.gidx, cb.O, cb.lse, sched=sched))
+        _expect_check(lambda: hga.attn_bwd_causal(p, Q, K, V, cb.O, cb.lse, dO, cb.gidx, cb.dQ, cb.dK, cb.dV,
+                                                  sched=sched))
+    cb.forward(Q, K, V)
+    cb.backward(Q, K, V, dO)
+    torch.cuda.synchronize()
+    assert hga.device_check() == 0
+    assert torch.isfinite(cb.O).all() and torch.isfinite(cb.dQ).all()
