@@ -516,6 +516,25 @@ def run_gpu(args, w) -> None:
         torch.cuda.synchronize()
         full_ms.append(s0.elapsed_time(s1))
     full_ms = statistics.median(full_ms[max(args.warmup, 3):])
+    # Context for that figure: a plain device copy moving the same bytes
+    # (half read, half written), timed the same way.  A one-shot transfer of
+    # tens of MB pays launch, ramp-up and tail, so it does not reach the
+    # copy peak measured on gigabytes.
+    full_bytes_all = (w.B * w.Hkv * w.T * w.d * (2 if w.dtype == "bf16" else 4)
+                      + w.B * w.Hkv * (w.T // 64 + w.T // 8) * w.d * 4)
+    cp_src = torch.empty(full_bytes_all // 8, dtype=torch.float32, device=dev)
+    cp_dst = torch.empty_like(cp_src)
+    copy_ms = []
+    for _ in range(max(args.warmup, 3) + 5):
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        cp_dst.copy_(cp_src)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        copy_ms.append(s0.elapsed_time(s1))
+    copy_ms = statistics.median(copy_ms[max(args.warmup, 3):])
+    del cp_src, cp_dst
 
     # ---- routing + forward: the fused launch against the two launches ---------------
     def eager_ms(fn, n):
@@ -582,7 +601,9 @@ def run_gpu(args, w) -> None:
         stage_roof["summaries_full_history"] = dict(
             ms=full_ms, algorithmic_bytes=full_bytes, gb_per_s=full_bytes / (full_ms * 1e-3) / 1e9,
             frac=full_bytes / (full_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-            note="one-shot build of all chunk / group summaries of the context, timed alone")
+            copy_same_bytes_ms=copy_ms, frac_of_copy_same_bytes=copy_ms / full_ms,
+            note="one-shot build of all chunk / group summaries of the context, timed alone; "
+                 "copy_same_bytes_ms: a device copy moving the same bytes, timed the same way")
         rf_bytes = stage_bytes["route"] + stage_bytes["attn_fwd"]
         stage_roof["route_attn_fwd_fused"] = dict(
             ms=fused_ms, separate_ms=separate_ms, algorithmic_bytes=rf_bytes,
