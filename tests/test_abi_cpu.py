@@ -218,6 +218,15 @@ def test_causal_calls_reject_bad_arguments_on_the_host(lib):
     assert lib.hga_causal_schedule(ctypes.byref(p0), None, None, None) == hga.HGA_OK
 
 
+def test_causal_schedule_refuses_contexts_past_its_bitmap(lib):
+    # The cost kernel keeps a bitmap of the context's groups in shared memory:
+    # a context of 16M tokens (2M groups) is refused on the host.
+    ok = ctypes.c_void_p(1 << 20)
+    p = _p(T_hist=16 * 1024 * 1024, T_seg=2048).c()
+    assert lib.hga_causal_schedule(ctypes.byref(p), ok, ok, None) == hga.HGA_ERR_UNSUPPORTED
+    assert "bitmap" in lib.hga_last_error().decode()
+
+
 def test_causal_schedule_size():
     # int32 order and costs of every window item: B * Hkv * ceil(T_seg / 32) * ceil(G / 4).
     for kw, items in [(dict(B=2, Hq=8, Hkv=2, T_seg=256), 2 * 2 * 8 * 1),
