@@ -113,6 +113,7 @@ def algorithmic(w) -> dict:
 KERNEL_SOURCES = {
     "attn_fwd": ["attn_tc_fwd.cu", "sm100.cuh", "hga_internal.cuh"],
     "attn_bwd": ["attn_tc_bwd.cu", "sm100.cuh", "hga_internal.cuh"],
+    "attn_bwd_causal": ["attn_tc_bwd.cu", "window_union.cuh", "sm100.cuh", "hga_internal.cuh"],
 }
 
 
@@ -941,7 +942,8 @@ def run_causal(args, w) -> None:
                             routing="per query position (a block of one); per-row key sets"),
                 stage_ms=stage_ms,
                 roofline=dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
-                              frac=achieved / pk["hbm_gbs"], traffic=None, kernel=dom,
+                              frac=achieved / pk["hbm_gbs"],
+                              traffic=recorded_traffic(dom, w) if dom in KERNEL_SOURCES else None, kernel=dom,
                               algorithmic_bytes_per_launch=alg[dom],
                               peak_source=pk["source"] + " (burst copy)"),
                 e2e=dict(value=w.B * w.T_seg / (e2e_ms * 1e-3), unit="tokens/s", h2d_bytes_per_step=h2d,
